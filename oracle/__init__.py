@@ -1,0 +1,303 @@
+"""CPU oracle for N:M semi-structured sparse linear layers (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA path shares no code with it and
+never calls it.
+
+The arithmetic lives in ``nm_oracle.c`` (plain loops, fp64 sums); this module
+compiles it with gcc on first use and marshals numpy arrays through ctypes.
+Every function states the step of the method it follows; the pages are cited
+in the C source.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nm_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+BF16, FP32 = 0, 1
+
+
+def build(force: bool = False) -> str:
+    """Compile nm_oracle.c into liboracle.so (gcc -O2 -fopenmp)."""
+    with _lock:
+        stale = (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC)
+        if force or stale:
+            tmp = _LIB + f".tmp{os.getpid()}"
+            subprocess.check_call([
+                "gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                "-Wall", "-Wextra", "-Wno-unused-parameter", _SRC, "-o", tmp,
+            ])
+            os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        sig = {
+            "or_prune": (I, [P, I, I64, I64, I, I, P]),
+            "or_mask_pack": (None, [P, I64, I64, P]),
+            "or_window_assign_batch": (None, [P, I64, I, P, P, P]),
+            "or_lifted_k": (I64, [I64, I]),
+            "or_compress": (I, [P, I, I64, I64, I, P, P, P]),
+            "or_expand_lifted": (None, [P, P, I64, I64, P]),
+            "or_decompress": (None, [P, P, I64, I64, I, P]),
+            "or_meta_hw_bytes": (I64, [I64, I64]),
+            "or_meta_hw": (None, [P, I64, I64, P]),
+            "or_lift": (I, [P, I, I64, I64, I, P]),
+            "or_to_f64": (None, [P, I, I64, P, P]),
+            "or_linear_f64": (None, [P, P, I64, I64, I64, P, I64, P]),
+            "or_colnorm_f64": (None, [P, I, I64, I64, P]),
+            "or_hybrid_dense_count": (I64, [I64, ctypes.c_double]),
+            "or_hybrid_perm": (None, [P, I64, I64, P, P]),
+            "or_gather_cols_bf16": (None, [P, I64, I64, P, P]),
+            "or_num_threads": (I, []),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(lib, name)
+            f.restype, f.argtypes = res, args
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle expects C-contiguous arrays"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dt(x: np.ndarray) -> int:
+    if x.dtype == np.uint16:
+        return BF16
+    if x.dtype == np.float32:
+        return FP32
+    raise TypeError(f"oracle inputs are bf16 bits (uint16) or float32, got {x.dtype}")
+
+
+def _as_bits(x: np.ndarray) -> np.ndarray:
+    x = np.ascontiguousarray(x)
+    return x.view(np.uint32) if x.dtype == np.float32 else x
+
+
+def num_threads() -> int:
+    return int(_load().or_num_threads())
+
+
+# ------------------------------------------------------------------ prune
+
+
+def prune(x: np.ndarray, N: int, M: int) -> np.ndarray:
+    """Keep mask (uint8 0/1, same shape as x): top-N |x| per aligned group of M
+    along the last axis, ties to the lower index."""
+    x = np.ascontiguousarray(x)
+    rows, K = x.shape
+    keep = np.zeros((rows, K), np.uint8)
+    rc = _load().or_prune(_ptr(_as_bits(x)), _dt(x), rows, K, N, M, _ptr(keep))
+    if rc != 0:
+        raise ValueError(f"or_prune rejected N={N} M={M} K={K}")
+    return keep
+
+
+def mask_pack(keep: np.ndarray) -> np.ndarray:
+    keep = np.ascontiguousarray(keep, dtype=np.uint8)
+    rows, K = keep.shape
+    out = np.zeros((rows, (K + 31) // 32), np.uint32)
+    _load().or_mask_pack(_ptr(keep), rows, K, _ptr(out))
+    return out
+
+
+# ---------------------------------------------------------------- windows
+
+
+def window_assign_batch(masks: np.ndarray, M: int):
+    """Greedy window assignment for many single-group masks (bit i = position i).
+    Returns (win[count, M], slot[count, M], status[count])."""
+    masks = np.ascontiguousarray(masks, dtype=np.uint64)
+    cnt = masks.shape[0]
+    win = np.zeros((cnt, M), np.int8)
+    slot = np.zeros((cnt, M), np.int8)
+    st = np.zeros(cnt, np.int8)
+    _load().or_window_assign_batch(_ptr(masks), cnt, M, _ptr(win), _ptr(slot), _ptr(st))
+    return win, slot, st
+
+
+def lifted_k(K: int, M: int) -> int:
+    return int(_load().or_lifted_k(K, M))
+
+
+def compress(x: np.ndarray, keep: np.ndarray, M: int):
+    """Window-compressed values (bf16 bits [rows, K'/2]) and canonical nibbles
+    ([rows, K'/4], one per byte)."""
+    x = np.ascontiguousarray(x)
+    keep = np.ascontiguousarray(keep, dtype=np.uint8)
+    rows, K = x.shape
+    Kl = lifted_k(K, M)
+    vals = np.zeros((rows, Kl // 2), np.uint16)
+    nib = np.zeros((rows, Kl // 4), np.uint8)
+    rc = _load().or_compress(_ptr(_as_bits(x)), _dt(x), rows, K, M, _ptr(keep), _ptr(vals), _ptr(nib))
+    if rc != 0:
+        raise ValueError(f"or_compress failed ({rc})")
+    return vals, nib
+
+
+def expand_lifted(vals: np.ndarray, nib: np.ndarray) -> np.ndarray:
+    rows, half = vals.shape
+    Kl = half * 2
+    out = np.zeros((rows, Kl), np.float64)
+    _load().or_expand_lifted(_ptr(np.ascontiguousarray(vals)), _ptr(np.ascontiguousarray(nib)),
+                             rows, Kl, _ptr(out))
+    return out
+
+
+def decompress(vals: np.ndarray, nib: np.ndarray, K: int, M: int) -> np.ndarray:
+    rows = vals.shape[0]
+    out = np.zeros((rows, K), np.uint16)
+    _load().or_decompress(_ptr(np.ascontiguousarray(vals)), _ptr(np.ascontiguousarray(nib)),
+                          rows, K, M, _ptr(out))
+    return out
+
+
+def meta_hw(nib: np.ndarray, Kl: int) -> np.ndarray:
+    nib = np.ascontiguousarray(nib, dtype=np.uint8)
+    rows = nib.shape[0]
+    nbytes = int(_load().or_meta_hw_bytes(rows, Kl))
+    out = np.zeros(nbytes, np.uint8)
+    _load().or_meta_hw(_ptr(nib), rows, Kl, _ptr(out))
+    return out
+
+
+def lift(src: np.ndarray, M: int) -> np.ndarray:
+    src = np.ascontiguousarray(src)
+    rows, K = src.shape
+    Kl = lifted_k(K, M)
+    out = np.zeros((rows, Kl), np.uint16)
+    rc = _load().or_lift(_ptr(_as_bits(src)), _dt(src), rows, K, M, _ptr(out))
+    if rc != 0:
+        raise ValueError("or_lift rejected the shape")
+    return out
+
+
+# ----------------------------------------------------------------- linear
+
+
+def to_f64(x: np.ndarray, keep: np.ndarray | None = None) -> np.ndarray:
+    x = np.ascontiguousarray(x)
+    out = np.zeros(x.shape, np.float64)
+    kp = _ptr(np.ascontiguousarray(keep, dtype=np.uint8)) if keep is not None else None
+    _load().or_to_f64(_ptr(_as_bits(x)), _dt(x), x.size, kp, _ptr(out))
+    return out
+
+
+def linear_f64(A: np.ndarray, B: np.ndarray, rows=None) -> np.ndarray:
+    """Y[t, o] = sum_k A[t, k] * B[o, k], k ascending, fp64.  ``rows`` selects
+    a subset of t (the result then has len(rows) rows)."""
+    A = np.ascontiguousarray(A, dtype=np.float64)
+    B = np.ascontiguousarray(B, dtype=np.float64)
+    T, K = A.shape
+    O = B.shape[0]
+    assert B.shape[1] == K
+    if rows is None:
+        Y = np.zeros((T, O), np.float64)
+        _load().or_linear_f64(_ptr(A), _ptr(B), T, O, K, None, 0, _ptr(Y))
+    else:
+        sel = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        Y = np.zeros((sel.size, O), np.float64)
+        _load().or_linear_f64(_ptr(A), _ptr(B), T, O, K, _ptr(sel), sel.size, _ptr(Y))
+    return Y
+
+
+# ----------------------------------------------------------------- hybrid
+
+
+def colnorm_f64(w: np.ndarray) -> np.ndarray:
+    w = np.ascontiguousarray(w)
+    O, K = w.shape
+    out = np.zeros(K, np.float64)
+    _load().or_colnorm_f64(_ptr(_as_bits(w)), _dt(w), O, K, _ptr(out))
+    return out
+
+
+def hybrid_dense_count(K: int, dense_frac: float) -> int:
+    return int(_load().or_hybrid_dense_count(K, float(dense_frac)))
+
+
+def hybrid_perm(colnorm: np.ndarray, D: int):
+    colnorm = np.ascontiguousarray(colnorm, dtype=np.float64)
+    K = colnorm.size
+    perm = np.zeros(K, np.int32)
+    dense = np.zeros(K, np.uint8)
+    _load().or_hybrid_perm(_ptr(colnorm), K, D, _ptr(perm), _ptr(dense))
+    return perm, dense
+
+
+def gather_cols(w: np.ndarray, perm: np.ndarray) -> np.ndarray:
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    rows, K = w.shape
+    out = np.zeros_like(w)
+    _load().or_gather_cols_bf16(_ptr(w), rows, K, _ptr(np.ascontiguousarray(perm, dtype=np.int32)),
+                                _ptr(out))
+    return out
+
+
+# ------------------------------------------------------ composite references
+
+
+def sparse_operand(x: np.ndarray, N: int, M: int):
+    """Everything the prune + compress step produces for one operand:
+    keep mask, packed bit mask, values, canonical nibbles, hardware metadata."""
+    keep = prune(x, N, M)
+    vals, nib = compress(x, keep, M)
+    Kl = lifted_k(x.shape[1], M)
+    return dict(keep=keep, mask=mask_pack(keep), vals=vals, nib=nib, meta=meta_hw(nib, Kl), K_lift=Kl)
+
+
+def act_sparse_linear(x: np.ndarray, w: np.ndarray, N: int, M: int, rows=None) -> np.ndarray:
+    """Y = prune_{N:M}(X) . W^T in fp64 (activation sparsity)."""
+    keep = prune(x, N, M)
+    return linear_f64(to_f64(x, keep), to_f64(w), rows)
+
+
+def weight_sparse_linear(x: np.ndarray, w: np.ndarray, N: int, M: int, rows=None) -> np.ndarray:
+    """Y = X . prune_{N:M}(W)^T in fp64 (weight sparsity)."""
+    keep = prune(w, N, M)
+    return linear_f64(to_f64(x), to_f64(w, keep), rows)
+
+
+def hybrid_weight(w: np.ndarray, dense_frac: float):
+    """Hybrid dense + 2:4 weight: permutation, dense block, compressed 2:4 block,
+    and the pruned weight in the original column order."""
+    O, K = w.shape
+    D = hybrid_dense_count(K, dense_frac)
+    cn = colnorm_f64(w)
+    perm, is_dense = hybrid_perm(cn, D)
+    wp = gather_cols(w, perm)
+    Ks = K - D
+    ws = np.ascontiguousarray(wp[:, :Ks])
+    wd = np.ascontiguousarray(wp[:, Ks:])
+    out = dict(D=D, Ks=Ks, colnorm=cn, perm=perm, is_dense=is_dense, W_d=wd)
+    keep_full = np.ones((O, K), np.uint8)
+    if Ks > 0:
+        keep_s = prune(ws, 2, 4)
+        vals, nib = compress(ws, keep_s, 4)
+        out.update(keep_s=keep_s, vals_s=vals, nib_s=nib, meta_s=meta_hw(nib, Ks))
+        keep_full[:, perm[:Ks]] = keep_s
+    out["keep_full"] = keep_full
+    return out
+
+
+def hybrid_linear(x: np.ndarray, w: np.ndarray, dense_frac: float, rows=None) -> np.ndarray:
+    """Y = X . Wp^T where Wp is W with the pruned entries of the 2:4 region
+    zeroed, in the original column order (fp64)."""
+    hw = hybrid_weight(w, dense_frac)
+    return linear_f64(to_f64(x), to_f64(w, hw["keep_full"]), rows)
