@@ -1,0 +1,197 @@
+/*
+ * nmsparse.h -- C ABI of the B200 (sm_100a) N:M semi-structured sparse
+ * linear-layer library.
+ *
+ * Conventions, for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    allocates no device memory; scratch space is passed in as `ws` with a
+ *    size from the matching *_workspace_size() call.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *    asynchronous on that stream and return a status code; they validate all
+ *    arguments before launching anything, and a call that returns an error
+ *    has launched nothing and written no output.
+ *  - Matrices are row-major.  "bf16" is IEEE bfloat16 (uint16 bit patterns),
+ *    "fp32" is IEEE binary32.  The reduction dimension K is the contiguous
+ *    one for every operand.
+ *  - Pointers must be 16-byte aligned and leading dimensions multiples of 8
+ *    elements (16 bytes for bf16 rows), else NM_ERR_ALIGNMENT.
+ *
+ * Terms.  An N:M pattern keeps the N entries of largest magnitude in every
+ * aligned group of M consecutive entries along K, ties going to the lower
+ * index.  For M = 2n the kept entries of a group are spread over n-1
+ * overlapping windows of width 4 and stride 2 (2 entries each), which the
+ * 2:4 sparse tensor cores execute; the dense operand is then "lifted" so that
+ * lifted column g*4(n-1) + 4w + j is source column g*2n + 2w + j.  The lifted
+ * width is K' = K * (2n-2) / n (K' = K for 2:4).
+ *   [Motivating Next-Gen Accelerators with Flexible (N:M) Activation Sparsity
+ *    via Benchmarking Lightweight Post-Training Sparsification Approaches,
+ *    technical summary sections 1 and 2.A]
+ *   [SlideSparse: Fast and Flexible (2N-2):2N Structured Sparsity, technical
+ *    summary sections 2.A (sliding windows), 2.B (activation lifting),
+ *    2.C (offline packer, online lift and 2:4 GEMM)]
+ *   [SpenseGPT: Practical One-shot Pruning Enabling Sparse and Dense GEMMs for
+ *    LLM Inference, technical summary sections 2.A (hybrid dense + 2:4 format,
+ *    input-split) and 2.B (permuting the dense indices into one block)]
+ */
+#ifndef NMSPARSE_H
+#define NMSPARSE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { NM_BF16 = 0, NM_FP32 = 1 } nm_dtype;
+
+/* Which side of Y = X . W^T carries the sparse operand.
+ * NM_ACT:    sparse = X [T x K], dense = lifted W [O x K'], Y [T x O].
+ * NM_WEIGHT: sparse = W [O x K], dense = lifted X [T x K'], Y [T x O]
+ *            (the product is formed as W . X^T and stored transposed). */
+typedef enum { NM_ACT = 0, NM_WEIGHT = 1 } nm_side;
+
+enum {
+    NM_OK = 0,
+    NM_ERR_INVALID_ARG = 1,    /* null pointer, negative size, K % M != 0, bad dtype */
+    NM_ERR_UNSUPPORTED = 2,    /* N:M or shape outside what the kernels implement */
+    NM_ERR_ALIGNMENT = 3,      /* pointer / leading dimension alignment */
+    NM_ERR_CUDA = 4,           /* a CUDA call failed; see nm_last_cuda_error() */
+    NM_ERR_DEVICE_TIMEOUT = 5, /* a kernel's bounded wait expired (nm_get_device_error) */
+    NM_ERR_WORKSPACE = 6       /* ws NULL or ws_bytes below the required size */
+};
+
+/* A window-compressed sparse operand, as written by nm_prune_compress() or
+ * slide_decompose().
+ *   vals : bf16 [rows][K_lift/2]; window j of row r holds its two entries at
+ *          vals[r][2j], vals[r][2j+1] (padding slots hold +0.0).
+ *   meta : nm_meta_bytes(rows, K, M) bytes, the sparse-MMA metadata image
+ *          (see nm_meta_bytes). */
+typedef struct {
+    const void *vals;
+    const void *meta;
+    int64_t rows;
+    int64_t K;        /* original reduction length */
+    int32_t N, M;
+    int64_t K_lift;   /* nm_lifted_k(K, M) */
+} nm_sparse_operand;
+
+/* A hybrid dense + 2:4 weight W [O x K] (device buffers owned by the caller,
+ * filled by hybrid_prepare()).
+ *   perm   : int32 [K] = [sparse columns ascending | dense columns ascending]
+ *   vals_s : bf16 [O][Ks/2], 2:4-compressed sparse block (Ks = K - K_dense,
+ *            columns in perm order)
+ *   meta_s : nm_meta_bytes(O, Ks, 4) bytes
+ *   W_d    : bf16 [O][K_dense], the dense block (columns in perm order) */
+typedef struct {
+    int32_t *perm;
+    void *vals_s;
+    void *meta_s;
+    void *W_d;
+    int64_t O, K, K_dense;
+} nm_hybrid_weight;
+
+/* ------------------------------------------------------------------ sizes */
+
+/* Lifted width K' = K*(M-2)/(M/2) for even M >= 4 (K' = K for M = 4);
+ * -1 if M is odd, below 4, or does not divide K. */
+int64_t nm_lifted_k(int64_t K, int M);
+
+/* Bytes of the metadata image of a `rows` x K operand pruned N:M.  The image
+ * is made of blocks of 128 rows x 128 lifted columns (2048 bytes, the
+ * tensor-memory image of four sparse MMAs of K = 32): block (rb, kb) starts
+ * at byte (rb * ceil(K'/128) + kb) * 2048; inside it, row m and window
+ * q (0..31, four lifted columns each) hold their 4-bit index pair at lane
+ * (m%8) + 8*((q%8)/4) + 16*(m/16), byte 4*(q/8) of that lane's 16 bytes,
+ * nibble (q%4) + 4*((m/8)%2) of that 32-bit word.  Rows and windows past the
+ * operand carry the pair (0,1).  0 on invalid arguments. */
+size_t nm_meta_bytes(int64_t rows, int64_t K, int M);
+
+/* ------------------------------------------------------------ prune steps */
+
+/* Prunes `src` [rows x K] (row stride `ld` elements, dtype NM_BF16 or
+ * NM_FP32) to N:M along K and writes its window-compressed form.
+ *   mask_out : optional (may be NULL) uint32 [rows][ceil(K/32)]; bit k%32 of
+ *              word k/32 is set iff entry k is kept.
+ *   vals_out : bf16 [rows][K'/2] (fp32 inputs are rounded to nearest even).
+ *   meta_out : nm_meta_bytes(rows, K, M) bytes.
+ * Supported: M in {4, 8, 16, 32}; N <= 2 for M = 4, else 1 <= N <= M-2.
+ * Magnitudes are compared as integers on the sign-cleared bit patterns. */
+int nm_prune_compress(const void *src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld,
+                      int N, int M, uint32_t *mask_out, void *vals_out, void *meta_out,
+                      void *stream);
+
+/* The offline weight packer of the (2N-2):2N family: the same operation as
+ * nm_prune_compress() restricted to N = M - 2 (6:8, 14:16, 30:32) or 2:4,
+ * for a weight W [rows x K] with row stride K. */
+int slide_decompose(const void *w, nm_dtype dt, int64_t rows, int64_t K, int N, int M,
+                    uint32_t *mask_out, void *vals_out, void *meta_out, void *stream);
+
+/* Lifts the dense operand: dst[r][g*4(n-1) + 4w + j] = src[r][g*2n + 2w + j]
+ * for M = 2n, src [rows x K] (row stride ld elements, bf16 or fp32),
+ * dst bf16 [rows x K'] (row stride K').  M = 4 copies (and converts fp32). */
+int nm_lift(const void *src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, int M,
+            void *dst, void *stream);
+
+/* ------------------------------------------------------------------- GEMM */
+
+/* Y = sparse . dense^T (side NM_ACT) or its transpose (NM_WEIGHT), bf16
+ * products accumulated in fp32 on the 2:4 sparse tensor cores.
+ *   S      : the compressed sparse operand (rows_s = S->rows).
+ *   D      : bf16 lifted dense operand [rows_d][S->K_lift], row stride K_lift.
+ *   Y      : NM_ACT -> [rows_s][rows_d]; NM_WEIGHT -> [rows_d][rows_s];
+ *            row-major, dtype out_dt (NM_BF16 rounds to nearest even).
+ *   ws     : scratch of nm_sparse_gemm_workspace_size() bytes (may be NULL
+ *            when that size is 0).  Its contents need no initialisation.
+ * Requires K_lift % 16 == 0. */
+size_t nm_sparse_gemm_workspace_size(const nm_sparse_operand *S, int64_t rows_d, nm_side side);
+int nm_sparse_gemm(const nm_sparse_operand *S, const void *D, int64_t rows_d, nm_side side,
+                   void *Y, nm_dtype out_dt, void *ws, size_t ws_bytes, void *stream);
+
+/* Dense comparator on the same tensor-core pipeline: Y[rows_a][rows_b] =
+ * A . B^T with A [rows_a x K], B [rows_b x K] bf16, K % 16 == 0. */
+int nm_dense_gemm(const void *A, int64_t rows_a, const void *B, int64_t rows_b, int64_t K,
+                  void *Y, nm_dtype out_dt, void *stream);
+
+/* ----------------------------------------------------------------- hybrid */
+
+/* Dense column count for a dense share f: 4 * floor(f*K/4) (0 for f <= 0,
+ * K for f >= 1). */
+int64_t hybrid_dense_count(int64_t K, double dense_frac);
+
+/* Offline: ranks the K columns of W [O x K] (bf16) by sum_r w[r][c]^2
+ * (fp64, r ascending), keeps the top hybrid_dense_count(K, dense_frac)
+ * columns dense (ties to the lower column), prunes the others 2:4 in
+ * ascending column order, and fills `out` (buffers preallocated by the caller,
+ * sizes in nm_hybrid_weight; out->O, out->K, out->K_dense must be set).
+ * ws: hybrid_prepare_workspace_size(O, K) bytes. */
+size_t hybrid_prepare_workspace_size(int64_t O, int64_t K);
+int hybrid_prepare(const void *w, int64_t O, int64_t K, double dense_frac, nm_hybrid_weight *out,
+                   void *ws, size_t ws_bytes, void *stream);
+
+/* Y [B x O] = X[:, perm_s] . W_s^T + X[:, perm_d] . W_d^T (input-split, one
+ * fp32 accumulator) for X bf16 [B x K] (row stride K).
+ * ws: hybrid_gemm_workspace_size(W, B) bytes. */
+size_t hybrid_gemm_workspace_size(const nm_hybrid_weight *W, int64_t B);
+int hybrid_gemm(const void *X, int64_t B, const nm_hybrid_weight *W, void *Y, nm_dtype out_dt,
+                void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------- diagnostics */
+
+const char *nm_status_string(int status);
+/* The cudaError_t of the last NM_ERR_CUDA returned on this thread. */
+int nm_last_cuda_error(void);
+/* Synchronises `stream`, then reads and clears the device status word that
+ * kernels set when a bounded wait expires: NM_OK or NM_ERR_DEVICE_TIMEOUT
+ * (or NM_ERR_CUDA if the synchronisation itself failed). */
+int nm_get_device_error(void *stream);
+/* Test hook for the bounded-wait path: launches one CTA that waits on an
+ * mbarrier no thread ever arrives on, giving up after timeout_us
+ * microseconds and recording NM_ERR_DEVICE_TIMEOUT.  Faults nothing. */
+int nm_debug_expire_wait(unsigned timeout_us, void *stream);
+const char *nm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NMSPARSE_H */

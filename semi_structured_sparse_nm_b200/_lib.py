@@ -1,0 +1,267 @@
+"""ctypes binding of libnmsparse.so (include/nmsparse.h).
+
+Argument marshalling only: every step of the sparse path runs in the library's
+CUDA kernels.  PyTorch provides device memory and the current stream.  If the
+shared library is missing the import fails loudly; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libnmsparse.so")
+
+NM_BF16, NM_FP32 = 0, 1
+NM_ACT, NM_WEIGHT = 0, 1
+NM_OK, NM_ERR_INVALID_ARG, NM_ERR_UNSUPPORTED, NM_ERR_ALIGNMENT = 0, 1, 2, 3
+NM_ERR_CUDA, NM_ERR_DEVICE_TIMEOUT, NM_ERR_WORKSPACE = 4, 5, 6
+
+
+class NmError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status} ({lib().nm_status_string(status).decode()})"
+                         + (f", cudaError {lib().nm_last_cuda_error()}" if status == NM_ERR_CUDA else ""))
+
+
+class SparseOperand(ctypes.Structure):
+    _fields_ = [("vals", ctypes.c_void_p), ("meta", ctypes.c_void_p), ("rows", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("N", ctypes.c_int32), ("M", ctypes.c_int32),
+                ("K_lift", ctypes.c_int64)]
+
+
+class HybridWeight(ctypes.Structure):
+    _fields_ = [("perm", ctypes.c_void_p), ("vals_s", ctypes.c_void_p), ("meta_s", ctypes.c_void_p),
+                ("W_d", ctypes.c_void_p), ("O", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("K_dense", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m semi_structured_sparse_nm_b200.build` (no CPU fallback exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I, SZ, D = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_double
+        sigs = {
+            "nm_lifted_k": (I64, [I64, I]),
+            "nm_meta_bytes": (SZ, [I64, I64, I]),
+            "nm_prune_compress": (I, [P, I, I64, I64, I64, I, I, P, P, P, P]),
+            "slide_decompose": (I, [P, I, I64, I64, I, I, P, P, P, P]),
+            "nm_lift": (I, [P, I, I64, I64, I64, I, P, P]),
+            "nm_sparse_gemm_workspace_size": (SZ, [ctypes.POINTER(SparseOperand), I64, I]),
+            "nm_sparse_gemm": (I, [ctypes.POINTER(SparseOperand), P, I64, I, P, I, P, SZ, P]),
+            "nm_dense_gemm": (I, [P, I64, P, I64, I64, P, I, P]),
+            "hybrid_dense_count": (I64, [I64, D]),
+            "hybrid_prepare_workspace_size": (SZ, [I64, I64]),
+            "hybrid_prepare": (I, [P, I64, I64, D, ctypes.POINTER(HybridWeight), P, SZ, P]),
+            "hybrid_gemm_workspace_size": (SZ, [ctypes.POINTER(HybridWeight), I64]),
+            "hybrid_gemm": (I, [P, I64, ctypes.POINTER(HybridWeight), P, I, P, SZ, P]),
+            "nm_status_string": (ctypes.c_char_p, [I]),
+            "nm_last_cuda_error": (I, []),
+            "nm_get_device_error": (I, [P]),
+            "nm_debug_expire_wait": (I, [ctypes.c_uint, P]),
+            "nm_version": (ctypes.c_char_p, []),
+        }
+        for name, (res, args) in sigs.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int):
+    if status != NM_OK:
+        raise NmError(fn, status)
+
+
+def _stream(t: torch.Tensor | None = None):
+    dev = t.device if t is not None else None
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _p(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return NM_BF16
+    if t.dtype == torch.float32:
+        return NM_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must live on a CUDA device")
+
+
+# ------------------------------------------------------------------ sizes
+
+
+def lifted_k(K: int, M: int) -> int:
+    return int(lib().nm_lifted_k(K, M))
+
+
+def meta_bytes(rows: int, K: int, M: int) -> int:
+    return int(lib().nm_meta_bytes(rows, K, M))
+
+
+def hybrid_dense_count(K: int, dense_frac: float) -> int:
+    return int(lib().hybrid_dense_count(K, dense_frac))
+
+
+# ---------------------------------------------------------------- prune
+
+
+class Compressed:
+    """A window-compressed sparse operand living on the device."""
+
+    def __init__(self, vals, meta, rows, K, N, M, mask=None):
+        self.vals, self.meta, self.mask = vals, meta, mask
+        self.rows, self.K, self.N, self.M = rows, K, N, M
+        self.K_lift = lifted_k(K, M)
+
+    def struct(self) -> SparseOperand:
+        return SparseOperand(self.vals.data_ptr(), self.meta.data_ptr(), self.rows, self.K,
+                             self.N, self.M, self.K_lift)
+
+
+def alloc_compressed(rows: int, K: int, N: int, M: int, device, with_mask=False) -> Compressed:
+    Kl = lifted_k(K, M)
+    if Kl < 0:
+        raise ValueError(f"M={M} does not divide K={K}")
+    vals = torch.empty((rows, Kl // 2), dtype=torch.bfloat16, device=device)
+    meta = torch.empty(max(meta_bytes(rows, K, M), 16), dtype=torch.uint8, device=device)
+    mask = torch.empty((rows, (K + 31) // 32), dtype=torch.int32, device=device) if with_mask else None
+    return Compressed(vals, meta, rows, K, N, M, mask)
+
+
+def prune_compress(x: torch.Tensor, N: int, M: int, out: Compressed | None = None,
+                   with_mask: bool = False) -> Compressed:
+    _need_cuda(x)
+    rows, K = x.shape
+    if out is None:
+        out = alloc_compressed(rows, K, N, M, x.device, with_mask)
+    _check("nm_prune_compress", lib().nm_prune_compress(
+        _p(x), _dt(x), rows, K, x.stride(0), N, M, _p(out.mask), _p(out.vals), _p(out.meta), _stream(x)))
+    return out
+
+
+def slide_decompose(w: torch.Tensor, N: int, M: int, with_mask: bool = False) -> Compressed:
+    _need_cuda(w)
+    rows, K = w.shape
+    out = alloc_compressed(rows, K, N, M, w.device, with_mask)
+    if w.stride(0) != K:
+        raise ValueError("slide_decompose expects a contiguous weight")
+    _check("slide_decompose", lib().slide_decompose(
+        _p(w), _dt(w), rows, K, N, M, _p(out.mask), _p(out.vals), _p(out.meta), _stream(w)))
+    return out
+
+
+def lift(src: torch.Tensor, M: int, out: torch.Tensor | None = None) -> torch.Tensor:
+    _need_cuda(src)
+    rows, K = src.shape
+    Kl = lifted_k(K, M)
+    if out is None:
+        out = torch.empty((rows, Kl), dtype=torch.bfloat16, device=src.device)
+    _check("nm_lift", lib().nm_lift(_p(src), _dt(src), rows, K, src.stride(0), M, _p(out), _stream(src)))
+    return out
+
+
+# ----------------------------------------------------------------- GEMM
+
+
+def sparse_gemm(S: Compressed, D: torch.Tensor, side: int, out_dtype=torch.bfloat16,
+                out: torch.Tensor | None = None) -> torch.Tensor:
+    """side NM_ACT: Y [S.rows, D.rows]; NM_WEIGHT: Y [D.rows, S.rows]."""
+    _need_cuda(D)
+    rows_d = D.shape[0]
+    if D.dtype != torch.bfloat16 or D.shape[1] != S.K_lift or not D.is_contiguous():
+        raise ValueError("dense operand must be contiguous bf16 [rows, K_lift]")
+    shape = (S.rows, rows_d) if side == NM_ACT else (rows_d, S.rows)
+    if out is None:
+        out = torch.empty(shape, dtype=out_dtype, device=D.device)
+    st = S.struct()
+    ws_bytes = int(lib().nm_sparse_gemm_workspace_size(ctypes.byref(st), rows_d, side))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=D.device) if ws_bytes else None
+    _check("nm_sparse_gemm", lib().nm_sparse_gemm(
+        ctypes.byref(st), _p(D), rows_d, side, _p(out), _dt(out), _p(ws), ws_bytes, _stream(D)))
+    return out
+
+
+def dense_gemm(A: torch.Tensor, B: torch.Tensor, out_dtype=torch.bfloat16, out=None) -> torch.Tensor:
+    _need_cuda(A, B)
+    if not (A.is_contiguous() and B.is_contiguous()):
+        raise ValueError("contiguous operands expected")
+    if out is None:
+        out = torch.empty((A.shape[0], B.shape[0]), dtype=out_dtype, device=A.device)
+    _check("nm_dense_gemm", lib().nm_dense_gemm(_p(A), A.shape[0], _p(B), B.shape[0], A.shape[1], _p(out),
+                                                _dt(out), _stream(A)))
+    return out
+
+
+# --------------------------------------------------------------- hybrid
+
+
+class Hybrid:
+    def __init__(self, perm, vals_s, meta_s, W_d, O, K, K_dense):
+        self.perm, self.vals_s, self.meta_s, self.W_d = perm, vals_s, meta_s, W_d
+        self.O, self.K, self.K_dense = O, K, K_dense
+
+    def struct(self) -> HybridWeight:
+        return HybridWeight(self.perm.data_ptr(), _p(self.vals_s).value or 0, _p(self.meta_s).value or 0,
+                            _p(self.W_d).value or 0, self.O, self.K, self.K_dense)
+
+
+def hybrid_prepare(w: torch.Tensor, dense_frac: float) -> Hybrid:
+    _need_cuda(w)
+    O, K = w.shape
+    D = hybrid_dense_count(K, dense_frac)
+    Ks = K - D
+    dev = w.device
+    h = Hybrid(torch.empty(K, dtype=torch.int32, device=dev),
+               torch.empty((O, Ks // 2), dtype=torch.bfloat16, device=dev) if Ks else None,
+               torch.empty(max(meta_bytes(O, Ks, 4), 16), dtype=torch.uint8, device=dev) if Ks else None,
+               torch.empty((O, D), dtype=torch.bfloat16, device=dev) if D else None, O, K, D)
+    ws_bytes = int(lib().hybrid_prepare_workspace_size(O, K))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = h.struct()
+    _check("hybrid_prepare", lib().hybrid_prepare(_p(w), O, K, dense_frac, ctypes.byref(st), _p(ws), ws_bytes,
+                                                  _stream(w)))
+    return h
+
+
+def hybrid_gemm(x: torch.Tensor, h: Hybrid, out_dtype=torch.bfloat16, out=None, ws=None) -> torch.Tensor:
+    _need_cuda(x)
+    B = x.shape[0]
+    if out is None:
+        out = torch.empty((B, h.O), dtype=out_dtype, device=x.device)
+    st = h.struct()
+    ws_bytes = int(lib().hybrid_gemm_workspace_size(ctypes.byref(st), B))
+    if ws is None:
+        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=x.device)
+    _check("hybrid_gemm", lib().hybrid_gemm(_p(x), B, ctypes.byref(st), _p(out), _dt(out), _p(ws), ws.numel(),
+                                            _stream(x)))
+    return out
+
+
+# ----------------------------------------------------------- diagnostics
+
+
+def device_error(stream=None) -> int:
+    s = stream if stream is not None else _stream()
+    return int(lib().nm_get_device_error(s))
+
+
+def debug_expire_wait(timeout_us: int):
+    _check("nm_debug_expire_wait", lib().nm_debug_expire_wait(timeout_us, _stream()))

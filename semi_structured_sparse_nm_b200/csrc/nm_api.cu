@@ -1,0 +1,448 @@
+// nm_api.cu -- the C ABI declared in include/nmsparse.h.  Host-side
+// validation, tensor-map encoding, tile/split selection and launches.  One
+// translation unit: the kernels are included from the .cuh files so that the
+// device status word is a single symbol.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "nm_device.cuh"
+#include "nm_gemm.cuh"
+#include "nm_prune.cuh"
+#include "nmsparse.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e) {
+  g_last_cuda_error = static_cast<int>(e);
+  return NM_ERR_CUDA;
+}
+
+#define NM_CUDA_TRY(expr)                        \
+  do {                                           \
+    cudaError_t _e = (expr);                     \
+    if (_e != cudaSuccess) return cuda_fail(_e); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+bool m_supported(int M) { return M == 4 || M == 8 || M == 16 || M == 32; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2D bf16 tensor [outer][inner], row pitch row_bytes, box box_inner x
+// box_outer, 128-byte swizzle, zero fill out of bounds.
+int make_tmap(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t row_bytes,
+              uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return NM_OK;
+}
+
+// ----------------------------------------------------------------- GEMM
+struct GemmPlan {
+  const void* a_s = nullptr;  // compressed sparse A [rows_a][ks_lift/2]
+  const void* a_d = nullptr;  // dense A [rows_a][kd]
+  const void* b = nullptr;    // B [rows_b][ks_lift + kd]
+  int64_t rows_a = 0, rows_b = 0, ks_lift = 0, kd = 0;
+  const uint8_t* meta = nullptr;
+  void* y = nullptr;
+  int64_t ldy = 0;
+  int out_fp32 = 0, transpose = 0;
+};
+
+template <int BN>
+int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
+  using Cfg = nm::GemmCfg<BN>;
+  CUtensorMap ta_s, ta_d, tb;
+  const int64_t kb_sparse = ceil_div(p.ks_lift, 128);
+  const int64_t kb_dense = ceil_div(p.kd, 64);
+  int rc;
+  if (kb_sparse > 0) {
+    if ((rc = make_tmap(&ta_s, p.a_s, p.ks_lift / 2, p.rows_a, p.ks_lift, 64, nm::kBM)) != NM_OK) return rc;
+  }
+  if (kb_dense > 0) {
+    if ((rc = make_tmap(&ta_d, p.a_d, p.kd, p.rows_a, p.kd * 2, 64, nm::kBM)) != NM_OK) return rc;
+  }
+  if (kb_sparse == 0) ta_s = ta_d;
+  if (kb_dense == 0) ta_d = ta_s;
+  if ((rc = make_tmap(&tb, p.b, p.ks_lift + p.kd, p.rows_b, (p.ks_lift + p.kd) * 2, 64, BN)) != NM_OK) return rc;
+
+  nm::GemmArgs args{};
+  args.rows_a = p.rows_a;
+  args.rows_b = p.rows_b;
+  args.kb_sparse = static_cast<int>(kb_sparse);
+  args.kb_dense = static_cast<int>(kb_dense);
+  args.k_dense_x0 = p.ks_lift;
+  args.meta = p.meta;
+  args.meta_kb = kb_sparse;
+  args.Y = p.y;
+  args.ldy = p.ldy;
+  args.out_fp32 = p.out_fp32;
+  args.transpose_out = p.transpose;
+  args.splits = splits;
+
+  auto kern = nm::k_nm_gemm<BN>;
+  NM_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
+
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(ceil_div(p.rows_a, nm::kBM)),
+                     static_cast<unsigned>(ceil_div(p.rows_b, BN)), static_cast<unsigned>(splits));
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  cfg.numAttrs = 0;
+  if (splits > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = static_cast<unsigned>(splits);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta_s, ta_d, tb, args));
+  NM_CUDA_TRY(cudaGetLastError());
+  return NM_OK;
+}
+
+int pick_bn(int64_t rows_b) {
+  if (rows_b <= 16) return 16;
+  if (rows_b <= 32) return 32;
+  if (rows_b <= 64) return 64;
+  return 128;
+}
+
+int num_sms() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      sms = 148;
+  }
+  return sms;
+}
+
+// Split-K only when the output tiles cannot cover the SMs; powers of two up to
+// 8 (the cluster holds the splits of one tile).
+int pick_splits(int64_t tiles, int64_t kb_total) {
+  int s = 1;
+  while (s < 8 && tiles * (s * 2) <= num_sms() && kb_total >= (s * 2) * 4) s *= 2;
+  return s;
+}
+
+int run_gemm(const GemmPlan& p, cudaStream_t st) {
+  const int bn = pick_bn(p.rows_b);
+  const int64_t tiles = ceil_div(p.rows_a, nm::kBM) * ceil_div(p.rows_b, bn);
+  const int64_t kb_total = ceil_div(p.ks_lift, 128) + ceil_div(p.kd, 64);
+  const int splits = pick_splits(tiles, kb_total);
+  switch (bn) {
+    case 16: return launch_gemm_bn<16>(p, splits, st);
+    case 32: return launch_gemm_bn<32>(p, splits, st);
+    case 64: return launch_gemm_bn<64>(p, splits, st);
+    default: return launch_gemm_bn<128>(p, splits, st);
+  }
+}
+
+// --------------------------------------------------------------- prune
+template <typename T>
+int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M, uint32_t* mask,
+                 void* vals, void* meta, cudaStream_t st) {
+  const int64_t Kl = nm_lifted_k(K, M);
+  const int64_t KB = ceil_div(Kl, 128);
+  const int64_t RB = ceil_div(rows, 128);
+  const size_t smem = static_cast<size_t>(ceil_div(KB * 32, 16) * 16 + ceil_div(K, 32) * 4);
+  if (smem > 48 * 1024) return NM_ERR_UNSUPPORTED;
+  const dim3 grid(static_cast<unsigned>(RB * 128)), block(128);
+  auto v = static_cast<uint32_t*>(vals);
+  auto e = static_cast<uint8_t*>(meta);
+  switch (M) {
+    case 4: nm::k_prune_compress<4, T><<<grid, block, smem, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB); break;
+    case 8: nm::k_prune_compress<8, T><<<grid, block, smem, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB); break;
+    case 16: nm::k_prune_compress<16, T><<<grid, block, smem, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB); break;
+    case 32: nm::k_prune_compress<32, T><<<grid, block, smem, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB); break;
+    default: return NM_ERR_UNSUPPORTED;
+  }
+  NM_CUDA_TRY(cudaGetLastError());
+  return NM_OK;
+}
+
+template <typename T>
+int launch_lift(const T* src, int64_t rows, int64_t K, int64_t ld, int M, void* dst, cudaStream_t st) {
+  const int64_t Kl = nm_lifted_k(K, M);
+  const int64_t total = rows * (K / M);
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(total, 256), int64_t(num_sms()) * 16));
+  auto d = static_cast<uint16_t*>(dst);
+  switch (M) {
+    case 4: nm::k_lift<4, T><<<static_cast<unsigned>(blocks), 256, 0, st>>>(src, rows, K, ld, d, Kl); break;
+    case 8: nm::k_lift<8, T><<<static_cast<unsigned>(blocks), 256, 0, st>>>(src, rows, K, ld, d, Kl); break;
+    case 16: nm::k_lift<16, T><<<static_cast<unsigned>(blocks), 256, 0, st>>>(src, rows, K, ld, d, Kl); break;
+    case 32: nm::k_lift<32, T><<<static_cast<unsigned>(blocks), 256, 0, st>>>(src, rows, K, ld, d, Kl); break;
+    default: return NM_ERR_UNSUPPORTED;
+  }
+  NM_CUDA_TRY(cudaGetLastError());
+  return NM_OK;
+}
+
+int check_prune_args(const void* src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, int N, int M,
+                     const void* vals, const void* meta) {
+  if (dt != NM_BF16 && dt != NM_FP32) return NM_ERR_INVALID_ARG;
+  if (rows < 0 || K <= 0 || M <= 0 || ld < K || N < 0 || N > M) return NM_ERR_INVALID_ARG;
+  if (K % M != 0) return NM_ERR_INVALID_ARG;
+  if (!m_supported(M)) return NM_ERR_UNSUPPORTED;
+  if (N > (M == 4 ? 2 : M - 2)) return NM_ERR_UNSUPPORTED;
+  if (rows == 0) return NM_OK;                 // empty operand: nothing to read or write
+  if (src == nullptr || vals == nullptr || meta == nullptr) return NM_ERR_INVALID_ARG;
+  const int64_t esz = dt == NM_BF16 ? 2 : 4;
+  if (!aligned16(src) || !aligned16(vals) || !aligned16(meta) || (ld * esz) % 16 != 0) return NM_ERR_ALIGNMENT;
+  return NM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t nm_lifted_k(int64_t K, int M) {
+  if (M < 4 || M % 2 != 0 || K <= 0 || K % M != 0) return -1;
+  return K / M * 4 * (M / 2 - 1);
+}
+
+size_t nm_meta_bytes(int64_t rows, int64_t K, int M) {
+  const int64_t Kl = nm_lifted_k(K, M);
+  if (Kl < 0 || rows < 0) return 0;
+  return static_cast<size_t>(ceil_div(rows, 128) * ceil_div(Kl, 128) * 2048);
+}
+
+int nm_prune_compress(const void* src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, int N, int M,
+                      uint32_t* mask_out, void* vals_out, void* meta_out, void* stream) {
+  int rc = check_prune_args(src, dt, rows, K, ld, N, M, vals_out, meta_out);
+  if (rc != NM_OK) return rc;
+  if (mask_out != nullptr && !aligned16(mask_out)) return NM_ERR_ALIGNMENT;
+  if (rows == 0) return NM_OK;
+  auto st = static_cast<cudaStream_t>(stream);
+  if (dt == NM_BF16)
+    return launch_prune(static_cast<const uint16_t*>(src), rows, K, ld, N, M, mask_out, vals_out, meta_out, st);
+  return launch_prune(static_cast<const uint32_t*>(src), rows, K, ld, N, M, mask_out, vals_out, meta_out, st);
+}
+
+int slide_decompose(const void* w, nm_dtype dt, int64_t rows, int64_t K, int N, int M, uint32_t* mask_out,
+                    void* vals_out, void* meta_out, void* stream) {
+  if (!(N == M - 2 || (M == 4 && N == 2))) return NM_ERR_UNSUPPORTED;
+  return nm_prune_compress(w, dt, rows, K, K, N, M, mask_out, vals_out, meta_out, stream);
+}
+
+int nm_lift(const void* src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, int M, void* dst, void* stream) {
+  if (dt != NM_BF16 && dt != NM_FP32) return NM_ERR_INVALID_ARG;
+  if (rows < 0 || K <= 0 || M <= 0 || ld < K || K % M != 0) return NM_ERR_INVALID_ARG;
+  if (!m_supported(M)) return NM_ERR_UNSUPPORTED;
+  if (rows == 0) return NM_OK;
+  if (src == nullptr || dst == nullptr) return NM_ERR_INVALID_ARG;
+  const int64_t esz = dt == NM_BF16 ? 2 : 4;
+  if (!aligned16(src) || !aligned16(dst) || (ld * esz) % 16 != 0) return NM_ERR_ALIGNMENT;
+  if (rows == 0) return NM_OK;
+  auto st = static_cast<cudaStream_t>(stream);
+  if (dt == NM_BF16) return launch_lift(static_cast<const uint16_t*>(src), rows, K, ld, M, dst, st);
+  return launch_lift(static_cast<const uint32_t*>(src), rows, K, ld, M, dst, st);
+}
+
+size_t nm_sparse_gemm_workspace_size(const nm_sparse_operand* S, int64_t rows_d, nm_side side) {
+  (void)S; (void)rows_d; (void)side;
+  return 0;   // split-K partial sums stay in the cluster's shared memory
+}
+
+int nm_sparse_gemm(const nm_sparse_operand* S, const void* D, int64_t rows_d, nm_side side, void* Y,
+                   nm_dtype out_dt, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws; (void)ws_bytes;
+  if (S == nullptr) return NM_ERR_INVALID_ARG;
+  if (side != NM_ACT && side != NM_WEIGHT) return NM_ERR_INVALID_ARG;
+  if (out_dt != NM_BF16 && out_dt != NM_FP32) return NM_ERR_INVALID_ARG;
+  if (S->rows < 0 || rows_d < 0 || S->K <= 0 || S->M <= 0 || S->K % S->M != 0) return NM_ERR_INVALID_ARG;
+  if (!m_supported(S->M)) return NM_ERR_UNSUPPORTED;
+  if (S->K_lift != nm_lifted_k(S->K, S->M)) return NM_ERR_INVALID_ARG;
+  if (S->K_lift % 16 != 0) return NM_ERR_UNSUPPORTED;
+  if (S->rows == 0 || rows_d == 0) return NM_OK;
+  if (D == nullptr || Y == nullptr || S->vals == nullptr || S->meta == nullptr) return NM_ERR_INVALID_ARG;
+  if (!aligned16(S->vals) || !aligned16(S->meta) || !aligned16(D) || !aligned16(Y)) return NM_ERR_ALIGNMENT;
+  GemmPlan p;
+  p.a_s = S->vals;
+  p.b = D;
+  p.rows_a = S->rows;
+  p.rows_b = rows_d;
+  p.ks_lift = S->K_lift;
+  p.kd = 0;
+  p.meta = static_cast<const uint8_t*>(S->meta);
+  p.y = Y;
+  p.out_fp32 = out_dt == NM_FP32;
+  p.transpose = side == NM_WEIGHT;
+  p.ldy = side == NM_ACT ? rows_d : S->rows;
+  return run_gemm(p, static_cast<cudaStream_t>(stream));
+}
+
+int nm_dense_gemm(const void* A, int64_t rows_a, const void* B, int64_t rows_b, int64_t K, void* Y,
+                  nm_dtype out_dt, void* stream) {
+  if (out_dt != NM_BF16 && out_dt != NM_FP32) return NM_ERR_INVALID_ARG;
+  if (rows_a < 0 || rows_b < 0 || K <= 0) return NM_ERR_INVALID_ARG;
+  if (K % 16 != 0) return NM_ERR_UNSUPPORTED;
+  if (rows_a == 0 || rows_b == 0) return NM_OK;
+  if (A == nullptr || B == nullptr || Y == nullptr) return NM_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(Y)) return NM_ERR_ALIGNMENT;
+  GemmPlan p;
+  p.a_d = A;
+  p.b = B;
+  p.rows_a = rows_a;
+  p.rows_b = rows_b;
+  p.ks_lift = 0;
+  p.kd = K;
+  p.y = Y;
+  p.ldy = rows_b;
+  p.out_fp32 = out_dt == NM_FP32;
+  return run_gemm(p, static_cast<cudaStream_t>(stream));
+}
+
+int64_t hybrid_dense_count(int64_t K, double dense_frac) {
+  if (K <= 0) return 0;
+  if (dense_frac <= 0.0) return 0;
+  if (dense_frac >= 1.0) return K;
+  return 4 * static_cast<int64_t>((dense_frac * static_cast<double>(K)) / 4.0);
+}
+
+size_t hybrid_prepare_workspace_size(int64_t O, int64_t K) {
+  if (O <= 0 || K <= 0) return 0;
+  const int64_t colnorm = K * 8, flags = ceil_div(K, 256) * 256, wsp = O * K * 2;
+  return static_cast<size_t>(ceil_div(colnorm, 256) * 256 + flags + wsp);
+}
+
+int hybrid_prepare(const void* w, int64_t O, int64_t K, double dense_frac, nm_hybrid_weight* out, void* ws,
+                   size_t ws_bytes, void* stream) {
+  if (w == nullptr || out == nullptr || out->perm == nullptr) return NM_ERR_INVALID_ARG;
+  if (O <= 0 || K <= 0 || K % 8 != 0) return NM_ERR_INVALID_ARG;
+  const int64_t D = hybrid_dense_count(K, dense_frac);
+  const int64_t Ks = K - D;
+  if (out->O != O || out->K != K || out->K_dense != D) return NM_ERR_INVALID_ARG;
+  if (Ks % 128 != 0) return NM_ERR_UNSUPPORTED;
+  if (Ks > 0 && (out->vals_s == nullptr || out->meta_s == nullptr)) return NM_ERR_INVALID_ARG;
+  if (D > 0 && out->W_d == nullptr) return NM_ERR_INVALID_ARG;
+  if (ws == nullptr || ws_bytes < hybrid_prepare_workspace_size(O, K)) return NM_ERR_WORKSPACE;
+  if (!aligned16(w) || !aligned16(ws) || !aligned16(out->perm) ||
+      (Ks > 0 && (!aligned16(out->vals_s) || !aligned16(out->meta_s))) || (D > 0 && !aligned16(out->W_d)))
+    return NM_ERR_ALIGNMENT;
+  auto st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  double* colnorm = reinterpret_cast<double*>(base);
+  uint8_t* is_dense = base + ceil_div(K * 8, 256) * 256;
+  uint16_t* wsp = reinterpret_cast<uint16_t*>(is_dense + ceil_div(K, 256) * 256);
+  const unsigned cb = static_cast<unsigned>(ceil_div(K, 128));
+  nm::k_colnorm_f64<<<cb, 128, 0, st>>>(static_cast<const uint16_t*>(w), O, K, colnorm);
+  nm::k_hybrid_rank<<<cb, 128, 0, st>>>(colnorm, K, D, is_dense);
+  nm::k_hybrid_perm<<<cb, 128, 0, st>>>(is_dense, K, D, out->perm);
+  const int64_t gblocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(O * K, 256), int64_t(num_sms()) * 16));
+  nm::k_gather_cols<<<static_cast<unsigned>(gblocks), 256, 0, st>>>(
+      static_cast<const uint16_t*>(w), O, K, out->perm, Ks, wsp, static_cast<uint16_t*>(out->W_d));
+  NM_CUDA_TRY(cudaGetLastError());
+  if (Ks > 0) return launch_prune(wsp, O, Ks, Ks, 2, 4, nullptr, out->vals_s, out->meta_s, st);
+  return NM_OK;
+}
+
+size_t hybrid_gemm_workspace_size(const nm_hybrid_weight* W, int64_t B) {
+  if (W == nullptr || B <= 0) return 0;
+  return static_cast<size_t>(ceil_div(B * W->K * 2, 256) * 256);
+}
+
+int hybrid_gemm(const void* X, int64_t B, const nm_hybrid_weight* W, void* Y, nm_dtype out_dt, void* ws,
+                size_t ws_bytes, void* stream) {
+  if (X == nullptr || W == nullptr || Y == nullptr || W->perm == nullptr) return NM_ERR_INVALID_ARG;
+  if (out_dt != NM_BF16 && out_dt != NM_FP32) return NM_ERR_INVALID_ARG;
+  if (B < 0 || W->O <= 0 || W->K <= 0 || W->K_dense < 0 || W->K_dense > W->K || W->K % 8 != 0)
+    return NM_ERR_INVALID_ARG;
+  const int64_t Ks = W->K - W->K_dense;
+  if (Ks % 128 != 0) return NM_ERR_UNSUPPORTED;
+  if (Ks > 0 && (W->vals_s == nullptr || W->meta_s == nullptr)) return NM_ERR_INVALID_ARG;
+  if (W->K_dense > 0 && W->W_d == nullptr) return NM_ERR_INVALID_ARG;
+  if (B == 0) return NM_OK;
+  if (ws == nullptr || ws_bytes < hybrid_gemm_workspace_size(W, B)) return NM_ERR_WORKSPACE;
+  if (!aligned16(X) || !aligned16(Y) || !aligned16(ws) || (Ks > 0 && !aligned16(W->vals_s)) ||
+      (W->K_dense > 0 && !aligned16(W->W_d)))
+    return NM_ERR_ALIGNMENT;
+  auto st = static_cast<cudaStream_t>(stream);
+  uint16_t* xp = static_cast<uint16_t*>(ws);
+  const int64_t gblocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(B * W->K, 256), int64_t(num_sms()) * 4));
+  nm::k_gather_cols<<<static_cast<unsigned>(gblocks), 256, 0, st>>>(static_cast<const uint16_t*>(X), B, W->K,
+                                                                   W->perm, W->K, xp, nullptr);
+  NM_CUDA_TRY(cudaGetLastError());
+  GemmPlan p;
+  p.a_s = W->vals_s;
+  p.a_d = W->W_d;
+  p.b = xp;
+  p.rows_a = W->O;
+  p.rows_b = B;
+  p.ks_lift = Ks;
+  p.kd = W->K_dense;
+  p.meta = static_cast<const uint8_t*>(W->meta_s);
+  p.y = Y;
+  p.ldy = W->O;
+  p.out_fp32 = out_dt == NM_FP32;
+  p.transpose = 1;
+  return run_gemm(p, st);
+}
+
+const char* nm_status_string(int s) {
+  switch (s) {
+    case NM_OK: return "ok";
+    case NM_ERR_INVALID_ARG: return "invalid argument";
+    case NM_ERR_UNSUPPORTED: return "unsupported N:M pattern or shape";
+    case NM_ERR_ALIGNMENT: return "pointer or leading dimension not 16-byte aligned";
+    case NM_ERR_CUDA: return "CUDA error";
+    case NM_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case NM_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+int nm_last_cuda_error(void) { return g_last_cuda_error; }
+
+int nm_get_device_error(void* stream) {
+  NM_CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  unsigned v = 0;
+  NM_CUDA_TRY(cudaMemcpyFromSymbol(&v, nm::g_status, sizeof(v)));
+  if (v == 0) return NM_OK;
+  const unsigned zero = 0;
+  NM_CUDA_TRY(cudaMemcpyToSymbol(nm::g_status, &zero, sizeof(zero)));
+  return static_cast<int>(v);
+}
+
+int nm_debug_expire_wait(unsigned timeout_us, void* stream) {
+  if (timeout_us == 0 || timeout_us > 10u * 1000u * 1000u) return NM_ERR_INVALID_ARG;
+  nm::k_expire_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(timeout_us) * 1000ull);
+  NM_CUDA_TRY(cudaGetLastError());
+  return NM_OK;
+}
+
+const char* nm_version(void) { return "nmsparse 0.1 (sm_100a)"; }
+
+}  // extern "C"

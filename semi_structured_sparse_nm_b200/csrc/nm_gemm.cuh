@@ -1,0 +1,286 @@
+// nm_gemm.cuh -- tcgen05 GEMM for 2:4-compressed (sparse) and dense k-blocks.
+//
+//   D[128 x BN] (TMEM, fp32) = sum over k-blocks of A_kb . B_kb^T
+//
+// A k-block is either
+//   sparse: A = 128 rows x 64 stored bf16 (128 lifted K, 2:4 compressed),
+//           B = BN rows x 128 bf16, metadata 2048 B; 4 x tcgen05.mma.sp (K=32)
+//   dense : A = 128 rows x 64 bf16, B = BN rows x 64 bf16; 4 x tcgen05.mma (K=16)
+// Sparse k-blocks come first (they cover B columns [0, K's)), then the dense
+// ones (B columns K's + 64*kd ...): this one loop serves the plain sparse
+// GEMM, the dense comparator and the hybrid input-split product.
+//
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and
+// MMA issuer, warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)..).
+// Split-K: the `splits` CTAs of one output tile form a thread-block cluster;
+// each keeps its fp32 partial tile in its own shared memory and the tile is
+// summed in rank order through distributed shared memory -- no global scratch.
+#pragma once
+#include "nm_device.cuh"
+
+namespace nm {
+
+constexpr int kBM = 128;
+constexpr int kABytes = kBM * 128;          // one 128 B-wide swizzled tile
+constexpr int kEBytes = 2048;               // metadata of one sparse k-block
+
+struct GemmArgs {
+  int64_t rows_a, rows_b;
+  int kb_sparse, kb_dense;
+  int64_t k_dense_x0;                       // B column where the dense part starts
+  const uint8_t* meta;                      // metadata image of A's sparse part
+  int64_t meta_kb;                          // metadata blocks per 128-row block
+  void* Y;
+  int64_t ldy;
+  int out_fp32;
+  int transpose_out;                        // 1: Y[b][a]; 0: Y[a][b]
+  int splits;                               // CTAs per output tile (cluster size)
+};
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kBBytes = 2 * BN * 128;
+  static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
+  static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr int kTmemNeed = BN + 4 * kStages;
+  static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
+                                 : kTmemNeed <= 256 ? 256 : 512;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(kStages >= 2, "tile too large for the shared memory ring");
+  static_assert(kBM * BN * 4 <= kStages * (kABytes + kBBytes), "split-K tile must fit the ring");
+};
+
+enum : unsigned { kWhereProducer = 1, kWhereMma = 2, kWhereEpilogue = 3 };
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void store_out(const GemmArgs& a, int64_t ra, int64_t cb, float v) {
+  if (ra >= a.rows_a || cb >= a.rows_b) return;
+  const int64_t off = a.transpose_out ? cb * a.ldy + ra : ra * a.ldy + cb;
+  if (a.out_fp32) static_cast<float*>(a.Y)[off] = v;
+  else static_cast<__nv_bfloat16*>(a.Y)[off] = __float2bfloat16_rn(v);
+}
+
+// Stores CW (16 or 32) consecutive accumulator columns of row `ra`
+// (columns cb0 .. cb0+CW-1).
+template <int CW>
+__device__ __forceinline__ void store_row_chunk(const GemmArgs& a, int64_t ra, int64_t cb0,
+                                                const uint32_t (&v)[CW]) {
+  if (ra >= a.rows_a) return;
+  if (!a.transpose_out && cb0 + CW <= a.rows_b && (a.ldy % 8) == 0) {
+    if (a.out_fp32) {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.Y) + ra * a.ldy + cb0);
+#pragma unroll
+      for (int i = 0; i < CW / 4; ++i)
+        dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                             __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+    } else {
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.Y) + ra * a.ldy + cb0);
+#pragma unroll
+      for (int i = 0; i < CW / 8; ++i) {
+        uint32_t p[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[8 * i + 2 * j]),
+                                                   __uint_as_float(v[8 * i + 2 * j + 1]));
+          p[j] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        dst[i] = make_uint4(p[0], p[1], p[2], p[3]);
+      }
+    }
+    return;
+  }
+#pragma unroll
+  for (int i = 0; i < CW; ++i) store_out(a, ra, cb0 + i, __uint_as_float(v[i]));
+}
+
+template <int BN>
+__global__ void __launch_bounds__(192, 1)
+k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUtensorMap tmA_d,
+          const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + S * kABytes;
+  uint8_t* sE = sB + S * Cfg::kBBytes;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(sE + S * kEBytes);
+  uint64_t* empty_bar = full_bar + S;
+  uint64_t* accum_bar = empty_bar + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t m_tile = blockIdx.x, n_tile = blockIdx.y;
+  const int split = static_cast<int>(blockIdx.z);
+  const int kb_total = args.kb_sparse + args.kb_dense;
+  const int kb_begin = static_cast<int>(static_cast<int64_t>(kb_total) * split / args.splits);
+  const int kb_end = static_cast<int>(static_cast<int64_t>(kb_total) * (split + 1) / args.splits);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    mbar_init(accum_bar, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA_s); prefetch_tmap(&tmA_d); prefetch_tmap(&tmB);
+  }
+  if (warp == 1) { tmem_alloc(tmem_slot, Cfg::kTmemCols); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_acc = *tmem_slot;
+  const uint32_t tmem_meta = tmem_acc + BN;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    if (elect_one()) {
+      int it = 0;
+      for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+        if (!mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag, kWhereProducer)) break;
+        uint8_t* a_dst = sA + s * kABytes;
+        uint8_t* b_dst = sB + s * Cfg::kBBytes;
+        const int32_t y_a = static_cast<int32_t>(m_tile * kBM), y_b = static_cast<int32_t>(n_tile * BN);
+        if (kb < args.kb_sparse) {
+          mbar_arrive_expect_tx(&full_bar[s], kABytes + Cfg::kBBytes + kEBytes);
+          tma_load_2d(&tmA_s, &full_bar[s], a_dst, kb * 64, y_a);
+          tma_load_2d(&tmB, &full_bar[s], b_dst, kb * 128, y_b);
+          tma_load_2d(&tmB, &full_bar[s], b_dst + BN * 128, kb * 128 + 64, y_b);
+          bulk_load(sE + s * kEBytes, args.meta + (m_tile * args.meta_kb + kb) * kEBytes, kEBytes,
+                    &full_bar[s]);
+        } else {
+          const int kd = kb - args.kb_sparse;
+          mbar_arrive_expect_tx(&full_bar[s], kABytes + BN * 128);
+          tma_load_2d(&tmA_d, &full_bar[s], a_dst, kd * 64, y_a);
+          tma_load_2d(&tmB, &full_bar[s], b_dst, static_cast<int32_t>(args.k_dense_x0) + kd * 64, y_b);
+        }
+      }
+      // Only the last S loads can still be in flight (a stage is reissued only
+      // after the MMA released it); wait for them before the CTA may exit.
+      for (int j = (it > S ? it - S : 0); j < it; ++j)
+        mbar_wait(&full_bar[j % S], static_cast<uint32_t>(j / S) & 1u, nullptr, kWhereProducer,
+                  100000000ull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    if (elect_one()) {
+      const uint32_t idesc_sp = idesc_bf16(kBM, BN, true);
+      const uint32_t idesc_dn = idesc_bf16(kBM, BN, false);
+      int it = 0;
+      bool ok = true;
+      for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+        if (!mbar_wait(&full_bar[s], ph, abort_flag, kWhereMma)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + s * kABytes);
+        const uint32_t b0 = smem_u32(sB + s * Cfg::kBBytes);
+        if (kb < args.kb_sparse) {
+          const uint32_t e_col = tmem_meta + 4u * s;
+          tc_cp_128x128b(e_col, desc_plain_128x16(smem_u32(sE + s * kEBytes)));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = desc_sw128_kmajor(a0 + 32u * kk);
+            const uint64_t bd = desc_sw128_kmajor(b0 + (kk / 2) * (BN * 128) + (kk % 2) * 64);
+            // The metadata operand is addressed in pairs of columns: the even
+            // column goes in the address, the odd/even choice in the
+            // instruction descriptor's sparse-id2 field (bits 0-1).
+            tc_mma_sp_f16(tmem_acc, ad, bd, e_col + (kk & ~1), idesc_sp | static_cast<uint32_t>(kk & 1),
+                          (it > 0 || kk > 0) ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = desc_sw128_kmajor(a0 + 32u * kk);
+            const uint64_t bd = desc_sw128_kmajor(b0 + 32u * kk);
+            tc_mma_f16(tmem_acc, ad, bd, idesc_dn, (it > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        tc_commit(&empty_bar[s]);
+      }
+      if (ok) tc_commit(accum_bar);
+    }
+  } else {
+    // -------------------------------------------------------- epilogue
+    const int q = warp % 4;
+    const bool ok = mbar_wait(accum_bar, 0u, abort_flag, kWhereEpilogue);
+    tc_fence_after();
+    if (ok) {
+      const int64_t row_local = q * 32 + lane;
+      const int64_t ra = m_tile * kBM + row_local;
+      float* red = reinterpret_cast<float*>(smem);        // split-K partial tile
+      if (args.splits > 1) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      constexpr int CW = BN < 32 ? BN : 32;              // columns per TMEM load
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += CW) {
+        uint32_t v[CW];
+        tc_ld_32x32b<CW>(tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
+        tc_wait_ld();
+        if (args.splits == 1) {
+          store_row_chunk<CW>(args, ra, n_tile * BN + c0, v);
+        } else {
+          float4* dst = reinterpret_cast<float4*>(red + row_local * BN + c0);
+#pragma unroll
+          for (int i = 0; i < CW / 4; ++i)
+            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+      }
+    }
+  }
+
+  if (args.splits > 1) {
+    // Sum the cluster's partial tiles in rank order; rank r owns rows
+    // [r*128/splits, (r+1)*128/splits) of the tile.
+    __syncwarp();
+    cluster_sync_all();
+    if (!*abort_flag) {
+      const uint32_t rank = cluster_ctarank();
+      const int rows_per = kBM / args.splits;
+      const int elems = rows_per * BN;
+      const uint32_t red_base = smem_u32(smem);
+      for (int e = threadIdx.x; e < elems; e += blockDim.x) {
+        int rl, c;
+        if (args.transpose_out) { rl = e % rows_per; c = e / rows_per; }
+        else { rl = e / BN; c = e % BN; }
+        const int row_local = static_cast<int>(rank) * rows_per + rl;
+        const uint32_t off = static_cast<uint32_t>((row_local * BN + c) * 4);
+        float acc = 0.f;
+        for (int p = 0; p < args.splits; ++p) acc += ld_dsmem_f32(mapa_shared(red_base + off, p));
+        store_out(args, m_tile * kBM + row_local, n_tile * BN + c, acc);
+      }
+    }
+    cluster_sync_all();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_acc, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace nm

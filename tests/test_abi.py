@@ -1,0 +1,89 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/nmsparse.h declares, sizes match the documented formulas, and argument
+validation rejects bad calls before anything touches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from semi_structured_sparse_nm_b200 import build as nmbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    path = nmbuild.build()
+    from semi_structured_sparse_nm_b200 import _lib
+    assert _lib.LIB_PATH == path
+    return _lib.lib()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "nmsparse.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared_functions()
+    assert len(names) >= 18, names
+    for n in ["nm_prune_compress", "slide_decompose", "nm_sparse_gemm", "hybrid_gemm", "nm_lift",
+              "hybrid_prepare", "nm_get_device_error"]:
+        assert n in names
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_sizes_match_the_oracle(L):
+    for K, M in [(4096, 4), (4096, 8), (4096, 16), (14336, 32), (96, 8), (64, 32)]:
+        assert L.nm_lifted_k(K, M) == oracle.lifted_k(K, M)
+        for rows in (1, 16, 128, 129, 2048):
+            assert L.nm_meta_bytes(rows, K, M) == oracle._load().or_meta_hw_bytes(rows, oracle.lifted_k(K, M))
+    assert L.nm_lifted_k(100, 8) == -1 and L.nm_lifted_k(12, 3) == -1
+    for K, f in [(4096, 0.25), (4096, 0.0), (4096, 1.0), (100, 0.3), (640, 0.2)]:
+        assert L.hybrid_dense_count(K, f) == oracle.hybrid_dense_count(K, f)
+
+
+def test_validation_before_launch(L):
+    from semi_structured_sparse_nm_b200 import _lib as nm
+    fake = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10001)
+    null = ctypes.c_void_p(0)
+    s = null
+    # invalid arguments
+    assert L.nm_prune_compress(null, 0, 4, 256, 256, 2, 4, null, fake, fake, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_prune_compress(fake, 0, 4, 250, 256, 2, 4, null, fake, fake, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_prune_compress(fake, 7, 4, 256, 256, 2, 4, null, fake, fake, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_prune_compress(fake, 0, 4, 256, 128, 2, 4, null, fake, fake, s) == nm.NM_ERR_INVALID_ARG
+    # unsupported patterns
+    assert L.nm_prune_compress(fake, 0, 4, 256, 256, 3, 4, null, fake, fake, s) == nm.NM_ERR_UNSUPPORTED
+    assert L.nm_prune_compress(fake, 0, 4, 240, 240, 2, 6, null, fake, fake, s) == nm.NM_ERR_UNSUPPORTED
+    assert L.nm_prune_compress(fake, 0, 4, 256, 256, 16, 16, null, fake, fake, s) == nm.NM_ERR_UNSUPPORTED
+    assert L.slide_decompose(fake, 0, 4, 256, 4, 8, null, fake, fake, s) == nm.NM_ERR_UNSUPPORTED
+    # alignment
+    assert L.nm_prune_compress(odd, 0, 4, 256, 256, 2, 4, null, fake, fake, s) == nm.NM_ERR_ALIGNMENT
+    assert L.nm_prune_compress(fake, 0, 4, 256, 260, 2, 4, null, fake, fake, s) == nm.NM_ERR_ALIGNMENT
+    # empty operands are a no-op
+    assert L.nm_prune_compress(null, 0, 0, 256, 256, 2, 4, null, null, null, s) == nm.NM_OK
+    assert L.nm_lift(null, 0, 0, 256, 256, 8, null, s) == nm.NM_OK
+    # GEMM
+    S = nm.SparseOperand(0x10000, 0x10000, 128, 256, 2, 4, 256)
+    assert L.nm_sparse_gemm(ctypes.byref(S), null, 64, 0, fake, 0, null, 0, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_sparse_gemm(ctypes.byref(S), fake, 64, 5, fake, 0, null, 0, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_sparse_gemm(ctypes.byref(S), odd, 64, 0, fake, 0, null, 0, s) == nm.NM_ERR_ALIGNMENT
+    bad = nm.SparseOperand(0x10000, 0x10000, 128, 256, 2, 4, 300)
+    assert L.nm_sparse_gemm(ctypes.byref(bad), fake, 64, 0, fake, 0, null, 0, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_dense_gemm(fake, 16, fake, 16, 40, fake, 0, s) == nm.NM_ERR_UNSUPPORTED
+    # hybrid
+    H = nm.HybridWeight(0x10000, 0x10000, 0x10000, 0x10000, 64, 512, 128)
+    assert L.hybrid_gemm(fake, 4, ctypes.byref(H), fake, 0, null, 0, s) == nm.NM_ERR_WORKSPACE
+    H2 = nm.HybridWeight(0x10000, 0x10000, 0x10000, 0x10000, 64, 512, 100)
+    assert L.hybrid_gemm(fake, 4, ctypes.byref(H2), fake, 0, fake, 1 << 20, s) == nm.NM_ERR_UNSUPPORTED
+    assert L.hybrid_prepare(fake, 64, 512, 0.25, ctypes.byref(H), null, 0, s) == nm.NM_ERR_WORKSPACE
+    assert L.nm_debug_expire_wait(0, s) == nm.NM_ERR_INVALID_ARG
+    for code in range(7):
+        assert L.nm_status_string(code)

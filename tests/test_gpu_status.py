@@ -1,0 +1,42 @@
+"""Bounded waits and error reporting on the GPU.  Nothing here faults, traps or
+hangs the device: the expired wait is a barrier nobody arrives on, with a
+1 ms limit, and the kernel returns normally after recording the status."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from semi_structured_sparse_nm_b200 import _lib as nm
+from semi_structured_sparse_nm_b200 import inputs
+from tests.gpu_util import check_close, dev, host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def test_expired_wait_is_reported_and_context_survives():
+    assert nm.device_error() == nm.NM_OK
+    nm.debug_expire_wait(1000)
+    assert nm.device_error() == nm.NM_ERR_DEVICE_TIMEOUT
+    # the status word was cleared and the context still works
+    assert nm.device_error() == nm.NM_OK
+    x = inputs.normal_bf16((32, 256), 1.0, 1)
+    w = inputs.normal_bf16((64, 256), 0.02, 2)
+    comp = nm.prune_compress(dev(x), 2, 4)
+    y = nm.sparse_gemm(comp, nm.lift(dev(w), 4), nm.NM_ACT, torch.float32)
+    torch.cuda.synchronize()
+    check_close(host_f64(y), oracle.act_sparse_linear(x, w, 2, 4))
+    assert nm.device_error() == nm.NM_OK
+
+
+def test_errors_launch_nothing():
+    x = dev(inputs.normal_bf16((8, 256), 1.0, 1))
+    comp = nm.alloc_compressed(8, 256, 2, 4, x.device)
+    before = comp.vals.clone()
+    with pytest.raises(nm.NmError) as e:
+        nm.prune_compress(x, 3, 4, out=comp)          # 3:4 is not a supported pattern
+    assert e.value.status == nm.NM_ERR_UNSUPPORTED
+    with pytest.raises(nm.NmError) as e:
+        nm.prune_compress(x[:, 4:], 2, 4)             # rows start 8 bytes off a 16-byte boundary
+    assert e.value.status == nm.NM_ERR_ALIGNMENT
+    torch.cuda.synchronize()
+    assert torch.equal(comp.vals, before)
