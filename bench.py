@@ -1,18 +1,25 @@
 """Benchmark of the N:M sparse linear layer on B200.
 
-One step = one pass of the hot path over one batch: prune + window-compress of
-X (8:16 along K) followed by the sparse GEMM against the offline-lifted weight,
-on the Llama-8B up_proj prefill shape (X [2048 x 4096] Student-t, W [14336 x
-4096] N(0, 0.02), bf16, fp32 accumulation, bf16 out).
-
-Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle on the
-host cores instead (a bounded sample of the same workload per step).
+One step = one pass of the hot path over one batch of synthetic input:
+  activation sparsity (8:16, 16:32, tiny 2:4): prune + window-compress X,
+      then the 2:4 sparse GEMM against the offline-lifted weight;
+  weight sparsity (6:8 sliding windows): lift X online, then the sparse GEMM
+      against the offline-decomposed weight;
+  hybrid dense + 2:4 weight (decode): gather X by the column permutation and
+      one input-split GEMM.
+The headline line is the Llama-8B up_proj prefill shape with 8:16 activation
+sparsity (X [2048 x 4096] Student-t, W [14336 x 4096] N(0, 0.02), bf16, fp32
+accumulation, bf16 out); the other workloads are reported under "workloads".
 
 Timing: CUDA events on the launching stream, W warm-up steps, exactly K timed
-steps between barriers + device synchronisation, max over ranks.  The weight
-(205 MB lifted) exceeds L2 and X is rotated over 8 device buffers, so no step
-reads its activations from L2.  Clocks and throttle reasons are sampled with
-NVML during the timed region.
+steps between barriers + device synchronisation, max over ranks.  Every
+workload rotates its inputs (and weights, where they would fit in L2) over
+enough device buffers that the bytes touched between two uses of a buffer
+exceed 2x L2.  Decode workloads replay the K steps from a CUDA graph.  Clocks
+and throttle reasons are polled with NVML during the timed region.
+
+`--impl reference` times the CPU oracle on the host cores instead (a bounded
+sample of the headline workload per step).
 """
 from __future__ import annotations
 
@@ -28,8 +35,12 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = "up_proj_8of16_act"
-X_ROTATE = 8
+HEADLINE = "up_proj_8of16_act"
+OTHERS = ["down_proj_16of32_act", "slide_6of8_wt_prefill", "slide_6of8_wt_decode",
+          "hybrid_decode_b1", "hybrid_decode_b8", "hybrid_decode_b32", "hybrid_decode_b128",
+          "tiny_2of4_act_fp32"]
+L2_BYTES = 126 * 1024 * 1024
+METRIC = "N:M sparse linear TFLOP/s (dense-equiv)"
 
 
 def _peaks():
@@ -63,17 +74,20 @@ class ClockSampler:
         except Exception:
             self.nv = None
 
+    def _sample(self):
+        self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+        r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        for bit, name in self.REASONS.items():
+            if r & bit:
+                self.reasons.add(name)
+
     def _run(self):
         while not self._stop.is_set():
             try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in self.REASONS.items():
-                    if r & bit:
-                        self.reasons.add(name)
+                self._sample()
             except Exception:
                 break
-            time.sleep(0.002)
+            time.sleep(0.0002)
 
     def __enter__(self):
         if self.nv is not None:
@@ -85,6 +99,10 @@ class ClockSampler:
         if self.nv is not None:
             self._stop.set()
             self.t.join()
+            try:
+                self._sample()
+            except Exception:
+                pass
 
     def summary(self):
         med = float(np.median(self.samples)) if self.samples else None
@@ -99,12 +117,15 @@ def _dist_env():
     return ws, rank, local
 
 
+# ------------------------------------------------------------ CPU baseline
+
+
 def cpu_oracle_sample(wl, x, w, budget_s: float):
-    """Times the oracle (prune + windows + fp64 GEMM) on whole rows of X until
-    about budget_s seconds have passed.  Returns (dense-equiv TFLOP/s, rows,
-    seconds, threads)."""
+    """Times the oracle (prune + windows + metadata + fp64 GEMM) on whole rows
+    of X until about budget_s seconds have passed.  Returns (dense-equiv
+    TFLOP/s, rows, seconds, threads)."""
     import oracle
-    wf = oracle.to_f64(w)                       # weight widening is setup, not timed
+    wf = oracle.to_f64(w)                       # weight widening is set-up, not timed
     rows_done, t_used = 0, 0.0
     chunk = 16
     while t_used < budget_s and rows_done < wl.T:
@@ -125,7 +146,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     from semi_structured_sparse_nm_b200 import inputs
-    wl, x, w = inputs.make_workload(WORKLOAD)
+    wl, x, w = inputs.make_workload(HEADLINE)
     times, rows = [], 0
     for i in range(args.warmup + args.steps):
         tf, r, t, thr = cpu_oracle_sample(wl, x, w, budget_s=args.ref_step_s)
@@ -136,16 +157,209 @@ def run_reference(args):
     value = 2.0 * wl.O * wl.K / per_row / 1e12
     sample = f"{rows} of {wl.T} token rows of X per step: prune+windows+metadata+fp64 GEMM against all of W"
     line = {
-        "impl": "reference", "metric": "N:M sparse linear TFLOP/s (dense-equiv)", "value": value,
+        "impl": "reference", "metric": METRIC, "value": value,
         "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": per_row * wl.T * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "T": wl.T, "K": wl.K, "O": wl.O, "N": wl.N, "M": wl.M},
+        "config": {"workload": HEADLINE, "T": wl.T, "K": wl.K, "O": wl.O, "N": wl.N, "M": wl.M},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# --------------------------------------------------------------- GPU arm
+
+
+class Workload:
+    """Device state of one workload and its step (two kernels: a prep kernel
+    -- prune, lift or gather -- and the GEMM)."""
+
+    def __init__(self, name, dev):
+        import torch
+        from semi_structured_sparse_nm_b200 import _lib as nm
+        from semi_structured_sparse_nm_b200 import inputs
+        self.nm, self.torch = nm, torch
+        self.wl, x_np, w_np = inputs.make_workload(name, seed=0)
+        self.x_np, self.w_np = x_np, w_np
+        wl = self.wl
+        self.name, self.dev = name, dev
+        to_dev = (lambda a: torch.from_numpy(a).view(torch.bfloat16).to(dev)) if wl.x_dtype == "bf16" \
+            else (lambda a: torch.from_numpy(a).to(dev))
+        X0, W = to_dev(x_np), to_dev(w_np)
+        out_dt = torch.bfloat16 if wl.out_dtype == "bf16" else torch.float32
+        self.decode = wl.side == "hybrid" or wl.T <= 128
+        if wl.side == "act":
+            self.Wl = nm.lift(W, wl.M)                                   # offline
+            self.R = max(2, min(8, int(np.ceil(2 * L2_BYTES / max(X0.numel() * X0.element_size(), 1)))))
+            self.X = [X0] + [X0.roll(r, dims=0).contiguous() for r in range(1, self.R)]
+            self.comp = [nm.alloc_compressed(wl.T, wl.K, wl.N, wl.M, dev) for _ in range(2)]
+            self.Y = torch.empty((wl.T, wl.O), dtype=out_dt, device=dev)
+            self.rows_a, self.rows_b = wl.T, wl.O
+            self.prep_name, self.gemm_name = "prune_compress", "sparse_gemm"
+        elif wl.side == "weight":
+            Wc = nm.slide_decompose(W, wl.N, wl.M)                     # offline
+            wbytes = Wc.vals.numel() * 2 + Wc.meta.numel()
+            xbytes = X0.numel() * 2
+            self.R = max(2, int(np.ceil(2 * L2_BYTES / (wbytes + xbytes))))
+            self.Wc = [Wc] + [nm.Compressed(Wc.vals.clone(), Wc.meta.clone(), wl.O, wl.K, wl.N, wl.M)
+                              for _ in range(1, self.R)]
+            self.X = [X0] + [X0.roll(r, dims=0).contiguous() for r in range(1, self.R)]
+            self.Xl = [torch.empty((wl.T, wl.K_lift), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+            self.Y = torch.empty((wl.T, wl.O), dtype=out_dt, device=dev)
+            self.rows_a, self.rows_b = wl.O, wl.T
+            self.prep_name, self.gemm_name = "lift", "sparse_gemm"
+            self.w_bytes = wbytes
+        else:
+            H = nm.hybrid_prepare(W, wl.dense_frac)                      # offline
+            wbytes = H.vals_s.numel() * 2 + H.meta_s.numel() + H.W_d.numel() * 2
+            self.R = max(2, int(np.ceil(2 * L2_BYTES / wbytes)))
+            self.H = [H] + [nm.Hybrid(H.perm.clone(), H.vals_s.clone(), H.meta_s.clone(), H.W_d.clone(),
+                                      H.O, H.K, H.K_dense) for _ in range(1, self.R)]
+            self.X = [X0.roll(r, dims=0).contiguous() if r else X0 for r in range(self.R)]
+            self.Y = torch.empty((wl.T, wl.O), dtype=out_dt, device=dev)
+            self.ws = torch.empty(max(16, wl.T * wl.K * 2), dtype=torch.uint8, device=dev)
+            self.rows_a, self.rows_b = wl.O, wl.T
+            self.prep_name, self.gemm_name = "gather", "hybrid_gemm"
+            self.w_bytes = wbytes
+        del W
+        torch.cuda.synchronize(dev)
+
+    # one step; `mark` is called between the prep kernel and the GEMM
+    def step(self, i, mark=None):
+        nm, wl = self.nm, self.wl
+        r = i % self.R
+        if wl.side == "act":
+            c = self.comp[i % 2]
+            nm.prune_compress(self.X[r], wl.N, wl.M, out=c)
+            if mark:
+                mark()
+            nm.sparse_gemm(c, self.Wl, nm.NM_ACT, self.Y.dtype, out=self.Y)
+        elif wl.side == "weight":
+            xl = self.Xl[i % 2]
+            nm.lift(self.X[r], wl.M, out=xl)
+            if mark:
+                mark()
+            nm.sparse_gemm(self.Wc[r], xl, nm.NM_WEIGHT, self.Y.dtype, out=self.Y)
+        else:
+            if mark:
+                mark()
+            nm.hybrid_gemm(self.X[r], self.H[r], self.Y.dtype, out=self.Y, ws=self.ws)
+
+    def gemm_only(self, i):
+        nm, wl = self.nm, self.wl
+        r = i % self.R
+        if wl.side == "act":
+            nm.sparse_gemm(self.comp[0], self.Wl, nm.NM_ACT, self.Y.dtype, out=self.Y)
+        elif wl.side == "weight":
+            nm.sparse_gemm(self.Wc[r], self.Xl[0], nm.NM_WEIGHT, self.Y.dtype, out=self.Y)
+        else:
+            nm.hybrid_gemm(self.X[r], self.H[r], self.Y.dtype, out=self.Y, ws=self.ws)
+
+    def algorithmic(self):
+        """(dense-equiv flops, sparse-MMA flops, bytes of the GEMM) per step."""
+        wl = self.wl
+        dense = 2.0 * wl.T * wl.O * wl.K
+        if wl.side == "hybrid":
+            D = self.H[0].K_dense
+            Ks = wl.K - D
+            mma = 2.0 * wl.T * wl.O * (Ks + D)          # sparse part counted at its 2:4 rate
+            byts = (self.w_bytes + wl.T * wl.K * 2 + wl.T * wl.O * self.Y.element_size())
+        else:
+            mma = 2.0 * wl.T * wl.O * wl.K_lift
+            sparse_bytes = self.rows_a * wl.K_lift + self.nm.meta_bytes(self.rows_a, wl.K, wl.M)
+            byts = sparse_bytes + self.rows_b * wl.K_lift * 2 + wl.T * wl.O * self.Y.element_size()
+        return dense, mma, byts
+
+
+def time_workload(wk, steps, warmup, stream, clock=None):
+    """Returns (ms per step, ms per prep kernel, ms per GEMM launch)."""
+    import torch
+    for i in range(warmup):
+        wk.step(i)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if wk.decode:
+        # replay from CUDA graphs: the host cost of building tensor maps and
+        # launching is not part of a device step
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):                      # captured on torch's side stream
+            for i in range(steps):
+                wk.step(i)
+        gg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gg):
+            for i in range(steps):
+                wk.gemm_only(i)
+        g.replay()
+        gg.replay()
+        torch.cuda.synchronize()
+        ctx = clock if clock is not None else _Null()
+        with ctx:
+            t0.record(stream)
+            g.replay()
+            t1.record(stream)
+            torch.cuda.synchronize()
+        step_ms = t0.elapsed_time(t1) / steps
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        gg.replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        gemm_ms = e0.elapsed_time(e1) / steps
+        prep_ms = max(step_ms - gemm_ms, 0.0)
+        del g, gg
+        return step_ms, prep_ms, gemm_ms
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    ctx = clock if clock is not None else _Null()
+    with ctx:
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for i in range(steps):
+            evs[i][0].record(stream)
+            wk.step(i, mark=lambda e=evs[i][1]: e.record(stream))
+            evs[i][2].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    step_ms = t0.elapsed_time(t1) / steps
+    prep_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    gemm_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    return step_ms, prep_ms, gemm_ms
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None):
+    dense, mma, byts = wk.algorithmic()
+    wl = wk.wl
+    out = {
+        "value": ws * dense / (step_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": step_ms,
+        "tokens_per_s": ws * wl.T / (step_ms * 1e-3),
+        "config": {"T": wl.T, "K": wl.K, "O": wl.O, "N": wl.N, "M": wl.M, "side": wl.side,
+                   "K_lift": wl.K_lift, "rotated_buffers": wk.R},
+        "kernels": {f"{wk.prep_name}_us": prep_ms * 1e3, f"{wk.gemm_name}_us": gemm_ms * 1e3},
+    }
+    if wk.decode:
+        achieved = byts / (gemm_ms * 1e-3) / 1e9
+        out["roofline"] = {"bound": "hbm", "kernel": wk.gemm_name, "achieved": achieved, "peak": pk["hbm"],
+                           "unit": "GB/s", "frac": achieved / pk["hbm"], "traffic": traffic,
+                           "bytes_per_launch": byts,
+                           "peak_note": f"{pk['source']} HBM copy bandwidth"}
+    else:
+        peak = 2.0 * pk["bf16"]
+        achieved = mma / (gemm_ms * 1e-3) / 1e12
+        out["roofline"] = {"bound": "tensor", "kernel": wk.gemm_name, "achieved": achieved, "peak": peak,
+                           "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                           "flops_per_launch": mma,
+                           "peak_note": f"2 x {pk['source']} bf16 burst {pk['bf16']} TFLOP/s "
+                                        f"(nominal 2:4 sparse ratio)"}
+    return out
 
 
 def run_gpu(args):
@@ -159,122 +373,95 @@ def run_gpu(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     from semi_structured_sparse_nm_b200 import _lib as nm
-    from semi_structured_sparse_nm_b200 import inputs
-
-    wl, x_np, w_np = inputs.make_workload(WORKLOAD, seed=0)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
-    X = [torch.from_numpy(x_np).view(torch.bfloat16).to(dev)]
-    for r in range(1, X_ROTATE):
-        X.append(X[0].roll(r, dims=0).contiguous())    # same distribution, distinct buffers
-    W = torch.from_numpy(w_np).view(torch.bfloat16).to(dev)
-    Wl = nm.lift(W, wl.M)                               # offline: lifted weight [O x K']
-    del W
-    comp = [nm.alloc_compressed(wl.T, wl.K, wl.N, wl.M, dev) for _ in range(2)]
-    Y = torch.empty((wl.T, wl.O), dtype=torch.bfloat16, device=dev)
-    torch.cuda.synchronize()
+    pk = _peaks()
 
-    def step(i, ev=None):
-        c = comp[i % 2]
-        if ev is not None:
-            ev[0].record(stream)
-        nm.prune_compress(X[i % X_ROTATE], wl.N, wl.M, out=c)
-        if ev is not None:
-            ev[1].record(stream)
-        nm.sparse_gemm(c, Wl, nm.NM_ACT, torch.bfloat16, out=Y)
-        if ev is not None:
-            ev[2].record(stream)
-
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
+    wk = Workload(args.workload, dev)
     if dist is not None:
         dist.barrier()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        torch.cuda.synchronize()
-        t0.record(stream)
-        for i in range(args.steps):
-            step(i, evs[i])
-        t1.record(stream)
-        torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
+    clk = ClockSampler(torch.cuda.current_device())
+    step_ms, prep_ms, gemm_ms = time_workload(wk, args.steps, args.warmup, stream, clock=clk)
     if dist is not None:
-        tt = torch.tensor([ms], device=dev)
+        tt = torch.tensor([step_ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+        step_ms = float(tt.item())
         dist.barrier()
-    prune_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
-    gemm_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
     status = nm.device_error()
+    main = summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk)
 
-    # end to end: pinned host X in, Y out, through the same calls
-    xh = torch.from_numpy(x_np).view(torch.bfloat16).pin_memory()
-    yh = torch.empty((wl.T, wl.O), dtype=torch.bfloat16).pin_memory()
-    xd = torch.empty_like(X[0])
+    # end to end through the public calls: pinned host X in, Y out
+    wl = wk.wl
+    xh = torch.from_numpy(wk.x_np).view(torch.bfloat16).pin_memory() if wl.x_dtype == "bf16" \
+        else torch.from_numpy(wk.x_np).pin_memory()
+    yh = torch.empty(tuple(wk.Y.shape), dtype=wk.Y.dtype).pin_memory()
     e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(2):
-        xd.copy_(xh, non_blocking=True)
-        nm.prune_compress(xd, wl.N, wl.M, out=comp[0])
-        nm.sparse_gemm(comp[0], Wl, nm.NM_ACT, torch.bfloat16, out=Y)
-        yh.copy_(Y, non_blocking=True)
+
+    def e2e_step(i):
+        wk.X[0].copy_(xh, non_blocking=True)
+        wk.step(0)
+        yh.copy_(wk.Y, non_blocking=True)
+
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        xd.copy_(xh, non_blocking=True)
-        nm.prune_compress(xd, wl.N, wl.M, out=comp[0])
-        nm.sparse_gemm(comp[0], Wl, nm.NM_ACT, torch.bfloat16, out=Y)
-        yh.copy_(Y, non_blocking=True)
+    for i in range(e2e_steps):
+        e2e_step(i)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    dense, _, _ = wk.algorithmic()
 
-    dense_flops = 2.0 * wl.T * wl.O * wl.K
-    sparse_flops = 2.0 * wl.T * wl.O * wl.K_lift            # MMA work of the lifted 2:4 problem
-    step_ms = ms / args.steps
-    value = ws * dense_flops / (step_ms * 1e-3) / 1e12
-    pk = _peaks()
-    sparse_peak = 2.0 * pk["bf16"]                          # 2:4 sparse = 2 x dense (nominal ratio)
-    achieved = sparse_flops / (gemm_ms * 1e-3) / 1e12
-    kl = wl.K_lift
-    prune_bytes = wl.T * wl.K * 2 + wl.T * kl + nm.meta_bytes(wl.T, wl.K, wl.M)
     line = {
-        "metric": "N:M sparse linear TFLOP/s (dense-equiv)",
-        "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "T": wl.T, "K": wl.K, "O": wl.O, "N": wl.N, "M": wl.M,
-                   "K_lift": kl, "x_dist": "student_t(4)/sqrt(2)", "w_dist": "N(0,0.02)",
-                   "l2": f"lifted W {Wl.numel() * 2 / 1e6:.0f} MB > L2; X rotated over {X_ROTATE} buffers",
-                   "parallelism": f"replicas x{ws}"},
-        "tokens_per_s": ws * wl.T / (step_ms * 1e-3),
-        "executed_tflops": ws * (sparse_flops / 2) / (step_ms * 1e-3) / 1e12,
-        "kernels": {"prune_compress_us": prune_ms * 1e3, "sparse_gemm_us": gemm_ms * 1e3,
-                    "prune_GBps": prune_bytes / (prune_ms * 1e-3) / 1e9},
-        "roofline": {"bound": "tensor", "kernel": "k_nm_gemm (tcgen05.mma.sp)", "achieved": achieved,
-                     "peak": sparse_peak, "unit": "TFLOP/s", "frac": achieved / sparse_peak,
-                     "traffic": None,
-                     "peak_note": f"2 x {pk['source']} bf16 burst {pk['bf16']} TFLOP/s (nominal 2:4 ratio)",
-                     "flops_per_launch": sparse_flops},
-        "e2e": {"value": dense_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2)},
+        "metric": METRIC, "value": main["value"], "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, **main["config"],
+                   "x_dist": wl.x_dist, "w_std": wl.w_std,
+                   "l2": f"inputs rotated over {wk.R} buffers; touched bytes between reuses > 2x L2",
+                   "parallelism": f"replicas x{ws} (no data-path collective)"},
+        "tokens_per_s": main["tokens_per_s"],
+        "kernels": main["kernels"],
+        "roofline": main["roofline"],
+        "e2e": {"value": ws * dense / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
+                "d2h_bytes_per_step": int(yh.numel() * yh.element_size())},
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
         "device_status": status,
     }
+    del wk
+    torch.cuda.empty_cache()
+
+    if not args.only_main:
+        others = {}
+        for name in OTHERS:
+            if name == args.workload:
+                continue
+            w2 = Workload(name, dev)
+            s, p, g = time_workload(w2, args.steps, args.warmup, stream)
+            others[name] = summarize(w2, s, p, g, 1, pk)
+            del w2
+            torch.cuda.empty_cache()
+        line["workloads"] = others
+        line["device_status"] = max(status, nm.device_error())
+
     if rank == 0 and not args.no_cpu_baseline:
-        tf, rows, t, thr = cpu_oracle_sample(wl, x_np, w_np, budget_s=args.cpu_budget_s)
-        line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-                                "sample": f"{rows} of {wl.T} token rows ({t:.1f} s): prune+windows+metadata"
-                                          f"+fp64 GEMM against all of W"}
+        from semi_structured_sparse_nm_b200 import inputs
+        wlh, xh_np, wh_np = inputs.make_workload(args.workload)
+        if wlh.side == "act":
+            tf, rows, t, thr = cpu_oracle_sample(wlh, xh_np, wh_np, budget_s=args.cpu_budget_s)
+            line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                                    "sample": f"{rows} of {wlh.T} token rows ({t:.1f} s): prune+windows+"
+                                              f"metadata+fp64 GEMM against all of W"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
-    return 0 if status == 0 else 1
+    return 0 if line["device_status"] == 0 else 1
 
 
 def main():
@@ -283,6 +470,8 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--only-main", action="store_true", help="skip the other workloads")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--ref-step-s", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

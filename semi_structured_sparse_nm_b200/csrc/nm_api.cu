@@ -6,11 +6,14 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <string>
 
 #include "nm_device.cuh"
 #include "nm_gemm.cuh"
+#include "nm_gemm2.cuh"
 #include "nm_prune.cuh"
 #include "nmsparse.h"
 
@@ -32,6 +35,7 @@ int cuda_fail(cudaError_t e) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 bool m_supported(int M) { return M == 4 || M == 8 || M == 16 || M == 32; }
+int num_sms();
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -130,6 +134,95 @@ int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
   return NM_OK;
 }
 
+// uint8 [rows][16] view of a metadata image, box of one 128-row block.
+int make_tmap_meta(CUtensorMap* m, const void* base, int64_t rows16) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
+  cuuint64_t dims[2] = {16, static_cast<cuuint64_t>(rows16)};
+  cuuint64_t strides[1] = {16};
+  cuuint32_t box[2] = {16, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
+  return NM_OK;
+}
+
+// Number of 2-CTA clusters of this kernel that fit on the device at once.
+template <int BN, int NACC>
+int resident_pairs() {
+  using Cfg = nm::Gemm2Cfg<BN, NACC>;
+  auto kern = nm::k_nm_gemm_2cta<BN, NACC>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) != cudaSuccess) {
+    cudaGetLastError();
+    return num_sms() / 2;
+  }
+  cudaLaunchConfig_t q{};
+  q.gridDim = dim3(2, 1, 1);
+  q.blockDim = dim3(192, 1, 1);
+  q.dynamicSmemBytes = Cfg::kSmem;
+  cudaLaunchAttribute qa[1];
+  qa[0].id = cudaLaunchAttributeClusterDimension;
+  qa[0].val.clusterDim.x = 2;
+  qa[0].val.clusterDim.y = 1;
+  qa[0].val.clusterDim.z = 1;
+  q.attrs = qa;
+  q.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &q) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = num_sms() / 2;
+  }
+  return n;
+}
+
+// Persistent 2-CTA kernel for pure-sparse products whose A side is a whole
+// number of 256-row blocks.
+template <int BN, int NACC>
+int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
+  using Cfg = nm::Gemm2Cfg<BN, NACC>;
+  CUtensorMap ta, tb, te;
+  int rc;
+  const int64_t kb = ceil_div(p.ks_lift, 128);
+  if ((rc = make_tmap(&ta, p.a_s, p.ks_lift / 2, p.rows_a, p.ks_lift, 64, 128)) != NM_OK) return rc;
+  if ((rc = make_tmap(&tb, p.b, p.ks_lift, p.rows_b, p.ks_lift * 2, 64, BN / 2)) != NM_OK) return rc;
+  if ((rc = make_tmap_meta(&te, p.meta, ceil_div(p.rows_a, 128) * kb * 128)) != NM_OK) return rc;
+  nm::Gemm2Args a{};
+  a.rows_a = p.rows_a;
+  a.rows_b = p.rows_b;
+  a.kb = static_cast<int>(kb);
+  a.meta_kb = kb;
+  a.tiles_m = static_cast<int>(ceil_div(p.rows_a, 256));
+  a.tiles_n = static_cast<int>(ceil_div(p.rows_b, BN));
+  a.Y = p.y;
+  a.ldy = p.ldy;
+  a.out_fp32 = p.out_fp32;
+  a.transpose_out = p.transpose;
+  const int tiles = a.tiles_m * a.tiles_n;
+  auto kern = nm::k_nm_gemm_2cta<BN, NACC>;
+  NM_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem));
+  cudaLaunchConfig_t cfg{};
+  // A persistent grid larger than the number of co-resident SM pairs would
+  // run its last clusters after the others: size it by the occupancy query.
+  static int resident = 0;
+  if (resident == 0) resident = resident_pairs<BN, NACC>();
+  const int clusters = std::max(1, std::min(tiles, resident));
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+  cfg.blockDim = dim3(192, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta, tb, te, a));
+  NM_CUDA_TRY(cudaGetLastError());
+  return NM_OK;
+}
 int pick_bn(int64_t rows_b) {
   if (rows_b <= 16) return 16;
   if (rows_b <= 32) return 32;
@@ -156,7 +249,50 @@ int pick_splits(int64_t tiles, int64_t kb_total) {
   return s;
 }
 
+// Rounds of the persistent 2-CTA kernel times the per-tile MMA time (BN/2
+// cycles per K = 32 slice); a single accumulator buffer adds the epilogue.
+double cost_2cta(const GemmPlan& p, int bn, int nacc, int resident) {
+  const int64_t tiles = ceil_div(p.rows_a, 256) * ceil_div(p.rows_b, bn);
+  const int64_t clusters = std::max(1, resident);
+  const double rounds = static_cast<double>(ceil_div(tiles, clusters));
+  const double mma = static_cast<double>(ceil_div(p.ks_lift, 32)) * bn / 2.0;
+  const double epi = nacc == 1 ? bn * 12.0 : 0.0;
+  return rounds * (mma + epi);
+}
+
+// Kernel choice.  NMSPARSE_GEMM pins one variant where it applies:
+// "1cta", "2cta224", "2cta256", "2cta128"; unset or "auto" picks by shape.
 int run_gemm(const GemmPlan& p, cudaStream_t st) {
+  const char* env = std::getenv("NMSPARSE_GEMM");
+  const std::string mode = env != nullptr ? env : "auto";
+  const bool eligible2 = p.kd == 0 && p.ks_lift > 0 && p.rows_a % 256 == 0;
+  if (eligible2 && mode != "1cta") {
+    if (mode == "2cta224") return launch_gemm_2cta<224, 2>(p, st);
+    if (mode == "2cta192") return launch_gemm_2cta<192, 2>(p, st);
+    if (mode == "2cta256") return launch_gemm_2cta<256, 1>(p, st);
+    if (mode == "2cta128") return launch_gemm_2cta<128, 2>(p, st);
+    if (p.rows_b >= 512 && p.ks_lift >= 512) {
+      static int res[4] = {0, 0, 0, 0};
+      if (res[0] == 0) {
+        res[0] = resident_pairs<224, 2>();
+        res[1] = resident_pairs<192, 2>();
+        res[2] = resident_pairs<256, 1>();
+        res[3] = resident_pairs<128, 2>();
+      }
+      // 128-wide tiles run near the shared-memory port limit: weight them
+      const double c[4] = {cost_2cta(p, 224, 2, res[0]), cost_2cta(p, 192, 2, res[1]),
+                           cost_2cta(p, 256, 1, res[2]), cost_2cta(p, 128, 2, res[3]) * 1.25};
+      int best = 0;
+      for (int i = 1; i < 4; ++i)
+        if (c[i] < c[best]) best = i;
+      switch (best) {
+        case 0: return launch_gemm_2cta<224, 2>(p, st);
+        case 1: return launch_gemm_2cta<192, 2>(p, st);
+        case 2: return launch_gemm_2cta<256, 1>(p, st);
+        default: return launch_gemm_2cta<128, 2>(p, st);
+      }
+    }
+  }
   const int bn = pick_bn(p.rows_b);
   const int64_t tiles = ceil_div(p.rows_a, nm::kBM) * ceil_div(p.rows_b, bn);
   const int64_t kb_total = ceil_div(p.ks_lift, 128) + ceil_div(p.kd, 64);
@@ -175,17 +311,18 @@ int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M
                  void* vals, void* meta, cudaStream_t st) {
   const int64_t Kl = nm_lifted_k(K, M);
   const int64_t KB = ceil_div(Kl, 128);
-  const int64_t RB = ceil_div(rows, 128);
-  const size_t smem = static_cast<size_t>(ceil_div(KB * 32, 16) * 16 + ceil_div(K, 32) * 4);
-  if (smem > 48 * 1024) return NM_ERR_UNSUPPORTED;
-  const dim3 grid(static_cast<unsigned>(RB * 128)), block(128);
+  const int64_t rows_pad = ceil_div(rows, 128) * 128;
+  const int64_t tasks = (rows_pad / 16) * ceil_div(K / M, 32);
+  const int64_t per_sm = M >= 32 ? 2 : 3;           // resident CTAs per SM (registers)
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(tasks, int64_t(num_sms()) * per_sm));
+  const dim3 grid(static_cast<unsigned>(blocks)), block(nm::kPruneWarps * 32);
   auto v = static_cast<uint32_t*>(vals);
   auto e = static_cast<uint8_t*>(meta);
   switch (M) {
-    case 4: nm::k_prune_compress<4, T><<<grid, block, smem, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB); break;
-    case 8: nm::k_prune_compress<8, T><<<grid, block, smem, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB); break;
-    case 16: nm::k_prune_compress<16, T><<<grid, block, smem, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB); break;
-    case 32: nm::k_prune_compress<32, T><<<grid, block, smem, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB); break;
+    case 4: nm::k_prune_compress<4, T><<<grid, block, 0, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
+    case 8: nm::k_prune_compress<8, T><<<grid, block, 0, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
+    case 16: nm::k_prune_compress<16, T><<<grid, block, 0, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
+    case 32: nm::k_prune_compress<32, T><<<grid, block, 0, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
     default: return NM_ERR_UNSUPPORTED;
   }
   NM_CUDA_TRY(cudaGetLastError());

@@ -1,0 +1,261 @@
+// nm_gemm2.cuh -- persistent 2-CTA sparse GEMM (tcgen05 cta_group::2) for
+// the large (prefill) shapes.
+//
+// A cluster of two CTAs (on two SMs) computes 256 x BN output tiles:
+//   CTA rank r holds A rows [256 tm + 128 r, +128) and B rows
+//   [BN tn + (BN/2) r, +BN/2); the leader (rank 0) issues one
+//   tcgen05.mma.sp.cta_group::2 per K = 32 slice and both CTAs receive their
+//   128 x BN half of the product in their own tensor memory.
+// Per SM this reads A 4 KB + B 8 KB (BN = 256) of shared memory per 128-cycle
+// MMA, below the shared-memory port; a one-SM 128 x 128 tile needs about
+// 1.5x the port for 2:4 operands, which is why this kernel exists.
+//
+// Pipelines (bounded waits everywhere):
+//   smem ring  : full[s] lives in the leader and counts both CTAs' TMA bytes
+//                (TMA .cta_group::2 signals the leader's barrier, no multicast);
+//                empty[s] in both CTAs is arrived by the leader's commit,
+//                multicast to the pair.
+//   accumulator: NACC buffers; tmem_full[b] in both CTAs (leader commit,
+//                multicast); tmem_empty[b] in the leader, arrived remotely by
+//                the 4 epilogue warps of both CTAs.
+// Tiles are visited A-block fastest so that concurrently running clusters
+// share the B tile (the larger, streamed operand) through L2.
+#pragma once
+#include "nm_device.cuh"
+
+namespace nm {
+
+__device__ __forceinline__ uint32_t cluster_rank_2() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t leader_addr(uint32_t local) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(r) : "r"(local));
+  return r;
+}
+// TMA 2D load into this CTA's smem, completion bytes counted on the barrier
+// at shared::cluster address `bar_cluster` (the leader's).
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* m, uint32_t bar_cluster, void* dst,
+                                                 int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];"
+      :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(bar_cluster) : "memory");
+}
+__device__ __forceinline__ void tmem_alloc2(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+               :: "r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+      :: "r"(smem_u32(bar)), "h"(static_cast<uint16_t>(3)) : "memory");
+}
+__device__ __forceinline__ void tc_cp_pair_128x128b(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" :: "r"(taddr), "l"(desc) : "memory");
+}
+__device__ __forceinline__ void tc_mma_sp_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t e_tmem,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %2, [%5], %3, p;\n\t}"
+      :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(e_tmem)
+      : "memory");
+}
+
+struct Gemm2Args {
+  int64_t rows_a, rows_b;
+  int kb;                 // sparse k-blocks (128 lifted K each)
+  int64_t meta_kb;        // metadata blocks per 128-row block
+  int tiles_m, tiles_n;
+  void* Y;
+  int64_t ldy;
+  int out_fp32;
+  int transpose_out;
+};
+
+template <int BN, int NACC>
+struct Gemm2Cfg {
+  static constexpr int kHalfN = BN / 2;
+  static constexpr int kA = 128 * 128;                 // 128 rows x 64 stored bf16
+  static constexpr int kB = 2 * kHalfN * 128;          // two 64-column halves
+  static constexpr int kE = 2048;
+  static constexpr int kStage = kA + kB + kE;
+  static constexpr int kStagesRaw = (200 * 1024) / kStage;
+  static constexpr int kStages = kStagesRaw > 6 ? 6 : kStagesRaw;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kAccStride = 256;               // accumulator b at column 256 b
+  static constexpr int kMetaCol = (NACC - 1) * kAccStride + BN;
+  static constexpr int kSmem = kStages * kStage + 1024 + 512;
+  static_assert(kMetaCol + 4 * kStages <= kTmemCols, "tensor memory budget");
+  static_assert(kHalfN % 8 == 0 && BN % 16 == 0 && BN <= 256, "MMA N");
+  static_assert(kStages >= 3, "ring too shallow");
+};
+
+template <int BN, int NACC>
+__global__ void __launch_bounds__(192, 1)
+k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               const __grid_constant__ CUtensorMap tmE, const Gemm2Args args) {
+  using Cfg = Gemm2Cfg<BN, NACC>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw2[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw2) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + S * Cfg::kA;
+  uint8_t* sE = sB + S * Cfg::kB;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(sE + S * Cfg::kE);
+  uint64_t* empty_bar = full_bar + S;
+  uint64_t* tfull_bar = empty_bar + S;
+  uint64_t* tempty_bar = tfull_bar + NACC;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + NACC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_rank_2();
+  const bool leader = rank == 0;
+  const int cluster_id = blockIdx.x / 2;
+  const int num_clusters = gridDim.x / 2;
+  const int tiles = args.tiles_m * args.tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    for (int b = 0; b < NACC; ++b) { mbar_init(&tfull_bar[b], 1); mbar_init(&tempty_bar[b], 8); }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) { prefetch_tmap(&tmA); prefetch_tmap(&tmB); prefetch_tmap(&tmE); }
+  if (warp == 1) { tmem_alloc2(tmem_slot, Cfg::kTmemCols); tmem_relinquish2(); }
+  tc_fence_before();
+  cluster_barrier();          // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t tmem_meta = tmem_base + Cfg::kMetaCol;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (elect_one()) {
+      const uint32_t stage_tx = static_cast<uint32_t>(2 * (Cfg::kA + Cfg::kB + Cfg::kE));
+      int it = 0;
+      bool ok = true;
+      for (int t = cluster_id; t < tiles && ok; t += num_clusters) {
+        const int tm = t % args.tiles_m, tn = t / args.tiles_m;
+        const int32_t ya = tm * 256 + static_cast<int32_t>(rank) * 128;
+        const int32_t yb = tn * BN + static_cast<int32_t>(rank) * Cfg::kHalfN;
+        const int32_t ye_base = static_cast<int32_t>((static_cast<int64_t>(tm) * 2 + rank) * args.meta_kb * 128);
+        for (int kb = 0; kb < args.kb; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+          if (!mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag, kWhereProducer)) { ok = false; break; }
+          const uint32_t fb = leader_addr(smem_u32(&full_bar[s]));
+          if (leader) mbar_arrive_expect_tx(&full_bar[s], stage_tx);
+          tma_load_2d_pair(&tmA, fb, sA + s * Cfg::kA, kb * 64, ya);
+          tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB, kb * 128, yb);
+          tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB + Cfg::kHalfN * 128, kb * 128 + 64, yb);
+          tma_load_2d_pair(&tmE, fb, sE + s * Cfg::kE, 0, ye_base + kb * 128);
+        }
+      }
+      // Every stage this CTA filled was released by the leader's commit
+      // (multicast to both CTAs) before the CTA may exit: wait for the last
+      // S releases so no arrival is still in flight.
+      for (int j = (it > S ? it - S : 0); j < it; ++j)
+        mbar_wait(&empty_bar[j % S], static_cast<uint32_t>(j / S) & 1u, nullptr, kWhereProducer, 200000000ull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA (leader)
+    if (leader && elect_one()) {
+      const uint32_t idesc = idesc_bf16(256, BN, true);
+      int it = 0, lt = 0;
+      bool ok = true;
+      for (int t = cluster_id; t < tiles && ok; t += num_clusters, ++lt) {
+        const int b = lt % NACC;
+        const uint32_t use = static_cast<uint32_t>(lt / NACC);
+        if (!mbar_wait(&tempty_bar[b], (use & 1u) ^ 1u, abort_flag, kWhereMma)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem_base + b * Cfg::kAccStride;
+        for (int kb = 0; kb < args.kb; ++kb, ++it) {
+          const int s = it % S;
+          const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+          if (!mbar_wait(&full_bar[s], ph, abort_flag, kWhereMma)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * Cfg::kA);
+          const uint32_t b0 = smem_u32(sB + s * Cfg::kB);
+          const uint32_t e_col = tmem_meta + 4u * s;
+          tc_cp_pair_128x128b(e_col, desc_plain_128x16(smem_u32(sE + s * Cfg::kE)));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = desc_sw128_kmajor(a0 + 32u * kk);
+            const uint64_t bd = desc_sw128_kmajor(b0 + (kk / 2) * (Cfg::kHalfN * 128) + (kk % 2) * 64);
+            tc_mma_sp_pair(acc, ad, bd, e_col + (kk & ~1), idesc | static_cast<uint32_t>(kk & 1),
+                           (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit_pair(&empty_bar[s]);
+        }
+        if (ok) tc_commit_pair(&tfull_bar[b]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp % 4;
+    const uint32_t tempty_leader[2] = {leader_addr(smem_u32(&tempty_bar[0])),
+                                       leader_addr(smem_u32(&tempty_bar[NACC > 1 ? 1 : 0]))};
+    int lt = 0;
+    GemmArgs st{};
+    st.rows_a = args.rows_a;
+    st.rows_b = args.rows_b;
+    st.Y = args.Y;
+    st.ldy = args.ldy;
+    st.out_fp32 = args.out_fp32;
+    st.transpose_out = args.transpose_out;
+    for (int t = cluster_id; t < tiles; t += num_clusters, ++lt) {
+      const int tm = t % args.tiles_m, tn = t / args.tiles_m;
+      const int b = lt % NACC;
+      const uint32_t use = static_cast<uint32_t>(lt / NACC);
+      if (!mbar_wait(&tfull_bar[b], use & 1u, abort_flag, kWhereEpilogue)) break;
+      tc_fence_after();
+      const int64_t ra = static_cast<int64_t>(tm) * 256 + rank * 128 + q * 32 + lane;
+      const uint32_t acc = tmem_base + b * Cfg::kAccStride + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        tc_ld_32x32b_x32(acc + c0, v);
+        tc_wait_ld();
+        if (c0 + 32 <= BN) {
+          store_row_chunk<32>(st, ra, static_cast<int64_t>(tn) * BN + c0, v);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c0 + i < BN) store_out(st, ra, static_cast<int64_t>(tn) * BN + c0 + i, __uint_as_float(v[i]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty_leader[b]);
+    }
+  }
+
+  tc_fence_before();
+  __syncwarp();
+  cluster_barrier();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc2(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+}  // namespace nm

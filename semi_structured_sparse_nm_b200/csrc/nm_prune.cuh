@@ -9,25 +9,30 @@ namespace nm {
 // Loads M consecutive elements (16-bit or 32-bit) of one group into registers
 // with 8- or 16-byte vector loads.  The group start is 8-byte aligned for
 // M = 4 bf16, 16-byte aligned otherwise (checked by the host).
+__device__ __forceinline__ void split_word(uint32_t w, uint16_t* out) {
+  out[0] = static_cast<uint16_t>(w & 0xFFFFu);
+  out[1] = static_cast<uint16_t>(w >> 16);
+}
+__device__ __forceinline__ void split_word(uint32_t w, uint32_t* out) { out[0] = w; }
+
 template <int M, typename T>
 __device__ __forceinline__ void load_group(const T* __restrict__ p, T (&x)[M]) {
   constexpr int BYTES = M * static_cast<int>(sizeof(T));
+  constexpr int PW = 4 / static_cast<int>(sizeof(T));          // elements per 32-bit word
   if constexpr (BYTES % 16 == 0) {
-    constexpr int V = BYTES / 16;
-    constexpr int PER = 16 / static_cast<int>(sizeof(T));
 #pragma unroll
-    for (int v = 0; v < V; ++v) {
-      uint4 u = __ldg(reinterpret_cast<const uint4*>(p) + v);
-      const T* e = reinterpret_cast<const T*>(&u);
-#pragma unroll
-      for (int i = 0; i < PER; ++i) x[v * PER + i] = e[i];
+    for (int v = 0; v < BYTES / 16; ++v) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(p) + v);
+      split_word(u.x, &x[v * 4 * PW + 0 * PW]);
+      split_word(u.y, &x[v * 4 * PW + 1 * PW]);
+      split_word(u.z, &x[v * 4 * PW + 2 * PW]);
+      split_word(u.w, &x[v * 4 * PW + 3 * PW]);
     }
   } else {
     static_assert(BYTES == 8, "group of 8 bytes expected");
-    uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
-    const T* e = reinterpret_cast<const T*>(&u);
-#pragma unroll
-    for (int i = 0; i < M; ++i) x[i] = e[i];
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    split_word(u.x, &x[0]);
+    split_word(u.y, &x[PW]);
   }
 }
 
@@ -44,105 +49,241 @@ __device__ __forceinline__ uint32_t order_key(uint16_t b, int i) {
 __device__ __forceinline__ uint64_t order_key(uint32_t b, int i) {
   return (static_cast<uint64_t>(b & 0x7FFFFFFFu) << 5) | static_cast<uint64_t>(31 - i);
 }
+template <typename K> __device__ __forceinline__ K kmax(K a, K b) { return a > b ? a : b; }
+template <typename K> __device__ __forceinline__ K kmin(K a, K b) { return a < b ? a : b; }
 
-// One CTA per row (rows past `rows`, up to the 128-row padding of the
-// metadata image, only write padding).  Each thread takes whole groups:
-//   1. keys -> ranks -> keep bits (entry i kept iff fewer than N entries beat it);
-//   2. greedy windows: window w takes the not yet placed kept entries among
-//      positions 2w..2w+3 in ascending order, at most two;
-//   3. the two values of window j go to vals[r][2j..2j+1] as one 32-bit store,
-//      its index pair (i0 | i1 << 2) to a shared nibble row;
-// then the CTA writes its row's nibbles into the metadata image, four windows
-// (one 16-bit word) at a time.
-template <int M, typename T>
-__global__ void __launch_bounds__(128)
-k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int N,
-                 uint32_t* __restrict__ mask_out, uint32_t* __restrict__ vals_out,
-                 uint8_t* __restrict__ meta_out, int64_t Kl, int64_t KB) {
-  constexpr int NW = M / 2 - 1;                 // windows per group (1 for 2:4)
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t* s_nib = smem;                                             // KB*32 nibbles
-  uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem + ((KB * 32 + 15) / 16) * 16);
+// Bitonic network, descending, on M (power of two) distinct keys in registers.
+template <int M> struct Log2 { static constexpr int value = 1 + Log2<M / 2>::value; };
+template <> struct Log2<1> { static constexpr int value = 0; };
 
-  const int64_t r = blockIdx.x;
-  const int64_t groups = K / M;
-  const int64_t nwin = Kl / 4;
-  const int64_t mask_words = (K + 31) / 32;
-  const int tid = threadIdx.x;
-
-  if (r < rows) {
-    if (mask_out != nullptr)
-      for (int64_t i = tid; i < mask_words; i += blockDim.x) s_mask[i] = 0u;
-    for (int64_t j = nwin + tid; j < KB * 32; j += blockDim.x) s_nib[j] = 0x4;
-    __syncthreads();
-    const T* row = src + r * ld;
-    for (int64_t g = tid; g < groups; g += blockDim.x) {
-      T x[M];
-      load_group<M, T>(row + g * M, x);
-      // ranks by unique keys
-      uint32_t keep = 0u;
+template <int M, typename K>
+__device__ __forceinline__ void bitonic_desc(K (&a)[M]) {
+  constexpr int L = Log2<M>::value;
+#pragma unroll
+  for (int lk = 1; lk <= L; ++lk) {
+    const int k = 1 << lk;
+#pragma unroll
+    for (int lj = lk - 1; lj >= 0; --lj) {
+      const int j = 1 << lj;
 #pragma unroll
       for (int i = 0; i < M; ++i) {
-        const auto ki = order_key(x[i], i);
-        int beaten_by = 0;
-#pragma unroll
-        for (int j = 0; j < M; ++j) beaten_by += (order_key(x[j], j) > ki) ? 1 : 0;
-        keep |= (beaten_by < N ? 1u : 0u) << i;
-      }
-      // windows
-      uint32_t placed = 0u;
-#pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        int held = 0, i0 = 0, i1 = 1;
-        uint16_t v0 = 0, v1 = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int i = 2 * w + j;
-          const bool take = ((keep >> i) & 1u) && !((placed >> i) & 1u) && held < 2;
-          if (take) {
-            const uint16_t b = to_bf16_bits(x[i]);
-            if (held == 0) { i0 = j; v0 = b; } else { i1 = j; v1 = b; }
-            placed |= 1u << i;
-            ++held;
-          }
+        const int l = i ^ j;
+        if (l > i) {
+          const K x = a[i], y = a[l];
+          if ((i & k) == 0) { a[i] = kmax(x, y); a[l] = kmin(x, y); }
+          else { a[i] = kmin(x, y); a[l] = kmax(x, y); }
         }
-        if (held == 0) {
-          i0 = 0; i1 = 1; v0 = 0; v1 = 0;
-        } else if (held == 1) {
-          const int a = i0, pad = (a == 0) ? 1 : 0;
-          if (pad < a) { i1 = a; v1 = v0; i0 = pad; v0 = 0; }
-          else { i1 = pad; v1 = 0; }
-        }
-        const int64_t jw = g * NW + w;
-        vals_out[r * (Kl / 4) + jw] = static_cast<uint32_t>(v0) | (static_cast<uint32_t>(v1) << 16);
-        s_nib[jw] = static_cast<uint8_t>(i0 | (i1 << 2));
-      }
-      if (mask_out != nullptr) {
-        const int64_t bit = g * M;
-        atomicOr(&s_mask[bit / 32], (M == 32 ? keep : (keep & ((1u << M) - 1u))) << (bit % 32));
       }
     }
-    __syncthreads();
-    if (mask_out != nullptr)
-      for (int64_t i = tid; i < mask_words; i += blockDim.x) mask_out[r * mask_words + i] = s_mask[i];
-  } else {
-    for (int64_t j = tid; j < KB * 32; j += blockDim.x) s_nib[j] = 0x4;
-    __syncthreads();
   }
+}
 
-  // metadata image: row m of row-block rb, four windows 4q..4q+3 per 16-bit word
-  const int64_t rb = r / 128;
-  const int m = static_cast<int>(r % 128);
-  for (int64_t q = tid; q < KB * 8; q += blockDim.x) {
-    const int64_t j = 4 * q;
-    const int64_t kb = j / 32;
-    const int jj = static_cast<int>(j % 32);
-    const int c = jj / 8, h = (jj % 8) / 4;
-    const uint16_t word = static_cast<uint16_t>(s_nib[j] | (s_nib[j + 1] << 4) |
-                                                (s_nib[j + 2] << 8) | (s_nib[j + 3] << 12));
-    const int lane = (m % 8) + 8 * h + 16 * (m / 16);
-    const int64_t byte = (rb * KB + kb) * 2048 + lane * 16 + c * 4 + 2 * ((m / 8) % 2);
-    *reinterpret_cast<uint16_t*>(meta_out + byte) = word;
+// Raw bytes of one group, as loaded (16-byte words, or one 8-byte word).
+template <int M, typename T>
+struct GroupRaw {
+  static constexpr int BYTES = M * static_cast<int>(sizeof(T));
+  static constexpr int NV = BYTES >= 16 ? BYTES / 16 : 1;
+  uint4 v[NV];
+};
+
+template <int M, typename T>
+__device__ __forceinline__ void load_raw(const T* __restrict__ p, GroupRaw<M, T>& g) {
+  if constexpr (GroupRaw<M, T>::BYTES >= 16) {
+#pragma unroll
+    for (int i = 0; i < GroupRaw<M, T>::NV; ++i) g.v[i] = __ldg(reinterpret_cast<const uint4*>(p) + i);
+  } else {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    g.v[0] = make_uint4(u.x, u.y, 0u, 0u);
+  }
+}
+
+template <int M, typename T>
+__device__ __forceinline__ void unpack_raw(const GroupRaw<M, T>& g, T (&x)[M]) {
+  constexpr int PW = 4 / static_cast<int>(sizeof(T));
+  constexpr int WORDS = M / PW;                                   // 32-bit words in the group
+#pragma unroll
+  for (int wi = 0; wi < WORDS; ++wi) {
+    const uint4& q = g.v[wi / 4];
+    const uint32_t w = (wi % 4 == 0) ? q.x : (wi % 4 == 1) ? q.y : (wi % 4 == 2) ? q.z : q.w;
+    split_word(w, &x[wi * PW]);
+  }
+}
+
+// The N-th largest of M distinct keys.  For N = M/2 the two halves are sorted
+// and merged: the N largest of the union are max(a_i, b_{N-1-i}).
+template <int M, typename Key>
+__device__ __forceinline__ Key nth_largest(const Key (&key)[M], int N) {
+  if constexpr (M >= 4) {
+    if (2 * N == M) {
+      constexpr int H = M / 2;
+      Key a[H], b[H];
+#pragma unroll
+      for (int i = 0; i < H; ++i) { a[i] = key[i]; b[i] = key[H + i]; }
+      bitonic_desc<H, Key>(a);
+      bitonic_desc<H, Key>(b);
+      Key thr = kmax(a[0], b[H - 1]);
+#pragma unroll
+      for (int i = 1; i < H; ++i) thr = kmin(thr, kmax(a[i], b[H - 1 - i]));
+      return thr;
+    }
+  }
+  Key srt[M];
+#pragma unroll
+  for (int i = 0; i < M; ++i) srt[i] = key[i];
+  bitonic_desc<M, Key>(srt);
+  Key thr = srt[0];
+#pragma unroll
+  for (int k = 1; k < M; ++k) thr = (N > k) ? srt[k] : thr;     // srt[N-1], kept in registers
+  return thr;
+}
+
+// Prune + window-compress one group held in registers: returns the keep bits,
+// writes the NW value words and index pairs.
+template <int M, typename T>
+__device__ __forceinline__ uint32_t compress_group(const GroupRaw<M, T>& raw, int N, uint32_t* val_out,
+                                                   uint8_t* nib_out) {
+  constexpr int NW = M / 2 - 1;
+  T x[M];
+  unpack_raw<M, T>(raw, x);
+  uint32_t P[M / 2];                          // bf16 pairs (2p, 2p+1)
+#pragma unroll
+  for (int p = 0; p < M / 2; ++p)
+    P[p] = static_cast<uint32_t>(to_bf16_bits(x[2 * p])) | (static_cast<uint32_t>(to_bf16_bits(x[2 * p + 1])) << 16);
+  using Key = decltype(order_key(x[0], 0));
+  Key key[M];
+#pragma unroll
+  for (int i = 0; i < M; ++i) key[i] = order_key(x[i], i);
+  uint32_t keep = 0u;
+  if (N > 0) {
+    const Key thr = nth_largest<M, Key>(key, N);
+#pragma unroll
+    for (int i = 0; i < M; ++i) keep |= (key[i] >= thr ? 1u : 0u) << i;
+  }
+  uint32_t placed = 0u;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const uint32_t c = (keep >> (2 * w)) & ~(placed >> (2 * w)) & 0xFu;
+    const uint32_t f = c & (0u - c);
+    const uint32_t rest = c ^ f;
+    const uint32_t sb = rest & (0u - rest);
+    placed |= (f | sb) << (2 * w);
+    int i0 = 0, i1 = 1;
+    uint32_t zmask = 0u;
+    if (sb) { i0 = __ffs(f) - 1; i1 = __ffs(sb) - 1; zmask = 0xFFFFFFFFu; }
+    else if (f) {
+      const int a = __ffs(f) - 1;
+      if (a == 0) { zmask = 0x0000FFFFu; } else { i1 = a; zmask = 0xFFFF0000u; }
+    }
+    const uint32_t sel = static_cast<uint32_t>((0x10 + 0x22 * i0) | ((0x10 + 0x22 * i1) << 8));
+    val_out[w] = __byte_perm(P[w], P[w + 1], sel) & zmask;
+    nib_out[w] = static_cast<uint8_t>(i0 | (i1 << 2));
+  }
+  return keep;
+}
+
+// One CTA task = 16 consecutive rows x 32 consecutive groups; warp w takes
+// rows 2w and 2w+1 (both loads in flight together), lane = group.  32 groups
+// hold 32*NW windows, exactly NW metadata blocks of 32 windows, and 16 rows
+// are one contiguous 256-byte run inside a block (lanes 16j..16j+15 of the
+// tensor-memory image), so the CTA writes its metadata as whole 16-byte lane
+// rows.  Per row: pruned (entry kept iff fewer than N entries beat it), split
+// over windows (window w takes the lowest two not yet placed kept entries of
+// positions 2w..2w+3; one entry is paired with the lowest other local index,
+// none gives (0, 1); padded slots hold +0.0), values written through a
+// staging row as 16-byte stores.  Rows past `rows` (up to the 128-row padding
+// of the image) and windows past K'/4 get the index pair (0, 1).
+constexpr int kPruneWarps = 8;
+
+template <int M, typename T>
+__global__ void __launch_bounds__(kPruneWarps * 32)
+k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int N,
+                 uint32_t* __restrict__ mask_out, uint32_t* __restrict__ vals_out,
+                 uint8_t* __restrict__ meta_out, int64_t Kl, int64_t KB, int64_t rows_pad) {
+  constexpr int NW = M / 2 - 1;                   // windows per group
+  constexpr int WIN = 32 * NW;                    // windows per task row = NW blocks
+  __shared__ __align__(16) uint8_t s_nib[16][WIN];
+  __shared__ __align__(16) uint32_t s_val[kPruneWarps][WIN];
+  __shared__ uint32_t s_mask[kPruneWarps][M];
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int64_t groups = K / M;
+  const int64_t cpr = (groups + 31) / 32;
+  const int64_t mask_words = (K + 31) / 32;
+  const int64_t tasks = (rows_pad / 16) * cpr;
+  const bool vec_vals = (Kl % 16) == 0;
+
+  for (int64_t task = blockIdx.x; task < tasks; task += gridDim.x) {
+    const int64_t rg = task / cpr, ch = task % cpr;
+    const int64_t g0 = ch * 32, g = g0 + lane;
+    const int ng = static_cast<int>((groups - g0) < 32 ? (groups - g0) : 32);
+    const int64_t r0 = rg * 16;
+    for (int i = threadIdx.x; i < 16 * WIN / 4; i += blockDim.x)
+      reinterpret_cast<uint32_t*>(&s_nib[0][0])[i] = 0x04040404u;
+    GroupRaw<M, T> raw[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int64_t r = r0 + 2 * warp + k;
+      if (r < rows && g < groups) load_raw<M, T>(src + r * ld + g * M, raw[k]);
+    }
+    __syncthreads();                                   // padding in place before any row writes
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int it = 2 * warp + k;
+      const int64_t r = r0 + it;
+      if (r >= rows) break;
+      if (lane < M) s_mask[warp][lane] = 0u;
+      __syncwarp();
+      if (g < groups) {
+        uint32_t vals[NW];
+        uint8_t nibs[NW];
+        const uint32_t keep = compress_group<M, T>(raw[k], N, vals, nibs);
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+          s_val[warp][lane * NW + w] = vals[w];
+          s_nib[it][lane * NW + w] = nibs[w];
+        }
+        if (mask_out != nullptr)
+          atomicOr(&s_mask[warp][(lane * M) / 32], (M == 32 ? keep : (keep & ((1u << M) - 1u))) << ((lane * M) % 32));
+      }
+      __syncwarp();
+      uint32_t* vrow = vals_out + r * (Kl / 4) + g0 * NW;
+      if (vec_vals && ng == 32) {
+        const uint4* sv = reinterpret_cast<const uint4*>(&s_val[warp][0]);
+        uint4* dv = reinterpret_cast<uint4*>(vrow);
+        for (int i = lane; i < WIN / 4; i += 32) dv[i] = sv[i];
+      } else {
+        for (int i = lane; i < ng * NW; i += 32) vrow[i] = s_val[warp][i];
+      }
+      if (mask_out != nullptr && lane < M) {
+        const int64_t wi = ch * M + lane;
+        if (wi < mask_words) mask_out[r * mask_words + wi] = s_mask[warp][lane];
+      }
+      __syncwarp();
+    }
+    __syncthreads();
+    // metadata: NW blocks x 16 lane rows of 16 bytes.  Lane row L (0..15) of
+    // block b holds rows L%8 and L%8+8 of the 16, windows 32b + 8c + 4(L/8) + 0..3
+    // in word c (low half: first row, high half: second row).
+    const int64_t rb = r0 / 128;
+    const int64_t sub = (r0 % 128) / 16;
+    for (int i = threadIdx.x; i < NW * 16; i += blockDim.x) {
+      const int b = i / 16, L = i % 16;
+      const int64_t kb = ch * NW + b;
+      if (kb >= KB) continue;
+      const int i8 = L % 8, h = L / 8;
+      uint32_t wds[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int j = 32 * b + 8 * c + 4 * h;
+        const uint32_t lo = *reinterpret_cast<const uint32_t*>(&s_nib[i8][j]);
+        const uint32_t hi = *reinterpret_cast<const uint32_t*>(&s_nib[i8 + 8][j]);
+        const uint32_t plo = (lo & 0xFu) | ((lo >> 4) & 0xF0u) | ((lo >> 8) & 0xF00u) | ((lo >> 12) & 0xF000u);
+        const uint32_t phi = (hi & 0xFu) | ((hi >> 4) & 0xF0u) | ((hi >> 8) & 0xF00u) | ((hi >> 12) & 0xF000u);
+        wds[c] = plo | (phi << 16);
+      }
+      *reinterpret_cast<uint4*>(meta_out + (rb * KB + kb) * 2048 + sub * 256 + L * 16) =
+          make_uint4(wds[0], wds[1], wds[2], wds[3]);
+    }
+    __syncthreads();                                   // s_nib is rewritten by the next task
   }
 }
 
