@@ -176,6 +176,33 @@ size_t hybrid_gemm_workspace_size(const nm_hybrid_weight *W, int64_t B);
 int hybrid_gemm(const void *X, int64_t B, const nm_hybrid_weight *W, void *Y, nm_dtype out_dt,
                 void *ws, size_t ws_bytes, void *stream);
 
+/* Capacity, in bytes, of the library's built-in scratch array used by
+ * hybrid_gemm_noalloc(): the gathered activations need B * K * 2 bytes. */
+#define NM_NOALLOC_SCRATCH_BYTES (2u * 1024u * 1024u)
+
+/* hybrid_gemm() for callers that cannot allocate device memory: no `ws`
+ * argument, nothing is allocated.  (The pages have no counterpart to this
+ * entry point; it exists for integration.)
+ *
+ * Who needs it: code whose device memory is owned and budgeted by a host
+ * engine -- a plugin inside a serving framework that plans every byte ahead of
+ * time, or a caller with no allocator of its own on the request path -- may not
+ * call cudaMalloc or take memory from an allocator it does not control.
+ *
+ * Scratch: a fixed array of NM_NOALLOC_SCRATCH_BYTES (2 MiB) compiled into
+ * the library.  Every GPU that loads the library keeps it until the process
+ * exits.  Calls with B * K * 2 > NM_NOALLOC_SCRATCH_BYTES return
+ * NM_ERR_WORKSPACE and launch nothing.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it; make that first call before any stream
+ * capture.  All calls share the one array: calls whose kernels overlap on the
+ * GPU (different streams, no ordering between them) race on it.  Nothing in
+ * the array has to start at zero -- each call writes every byte it reads.
+ * Other arguments, layouts and errors are those of hybrid_gemm(). */
+int hybrid_gemm_noalloc(const void *X, int64_t B, const nm_hybrid_weight *W, void *Y, nm_dtype out_dt,
+                        void *stream);
+
 /* ------------------------------------------------------------- diagnostics */
 
 const char *nm_status_string(int status);

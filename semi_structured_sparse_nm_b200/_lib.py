@@ -64,6 +64,7 @@ def lib():
             "hybrid_prepare": (I, [P, I64, I64, D, ctypes.POINTER(HybridWeight), P, SZ, P]),
             "hybrid_gemm_workspace_size": (SZ, [ctypes.POINTER(HybridWeight), I64]),
             "hybrid_gemm": (I, [P, I64, ctypes.POINTER(HybridWeight), P, I, P, SZ, P]),
+            "hybrid_gemm_noalloc": (I, [P, I64, ctypes.POINTER(HybridWeight), P, I, P]),
             "nm_status_string": (ctypes.c_char_p, [I]),
             "nm_last_cuda_error": (I, []),
             "nm_get_device_error": (I, [P]),
@@ -252,6 +253,22 @@ def hybrid_gemm(x: torch.Tensor, h: Hybrid, out_dtype=torch.bfloat16, out=None, 
         ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=x.device)
     _check("hybrid_gemm", lib().hybrid_gemm(_p(x), B, ctypes.byref(st), _p(out), _dt(out), _p(ws), ws.numel(),
                                             _stream(x)))
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 2 * 1024 * 1024
+
+
+def hybrid_gemm_noalloc(x: torch.Tensor, h: Hybrid, out_dtype=torch.bfloat16, out=None) -> torch.Tensor:
+    """hybrid_gemm() through the entry point that allocates nothing: its scratch
+    is the library's built-in array (B * K * 2 bytes at most 2 MiB)."""
+    _need_cuda(x)
+    B = x.shape[0]
+    if out is None:
+        out = torch.empty((B, h.O), dtype=out_dtype, device=x.device)
+    st = h.struct()
+    _check("hybrid_gemm_noalloc", lib().hybrid_gemm_noalloc(_p(x), B, ctypes.byref(st), _p(out), _dt(out),
+                                                            _stream(x)))
     return out
 
 

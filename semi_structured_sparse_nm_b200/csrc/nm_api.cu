@@ -547,6 +547,48 @@ int hybrid_gemm(const void* X, int64_t B, const nm_hybrid_weight* W, void* Y, nm
   return run_gemm(p, st);
 }
 
+}  // extern "C"
+
+// Scratch of hybrid_gemm_noalloc(): one fixed array per device, alive until
+// the process exits.  Host code may not use its name as an address; the
+// device address is looked up once per device below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NM_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (cached).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  NM_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return NM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    NM_CUDA_TRY(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return NM_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int hybrid_gemm_noalloc(const void* X, int64_t B, const nm_hybrid_weight* W, void* Y, nm_dtype out_dt,
+                        void* stream) {
+  if (W == nullptr || B < 0) return NM_ERR_INVALID_ARG;
+  if (hybrid_gemm_workspace_size(W, B) > NM_NOALLOC_SCRATCH_BYTES) return NM_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if (B > 0) {
+    const int rc = noalloc_scratch(&ws);
+    if (rc != NM_OK) return rc;
+  }
+  return hybrid_gemm(X, B, W, Y, out_dt, ws, NM_NOALLOC_SCRATCH_BYTES, stream);
+}
+
 const char* nm_status_string(int s) {
   switch (s) {
     case NM_OK: return "ok";
