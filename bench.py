@@ -36,7 +36,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 HEADLINE = "up_proj_8of16_act"
-OTHERS = ["down_proj_16of32_act", "slide_6of8_wt_prefill", "slide_6of8_wt_decode",
+OTHERS = ["up_proj_2of4_act", "down_proj_16of32_act", "slide_6of8_wt_prefill", "slide_6of8_wt_decode",
           "hybrid_decode_b1", "hybrid_decode_b8", "hybrid_decode_b32", "hybrid_decode_b128",
           "tiny_2of4_act_fp32"]
 L2_BYTES = 126 * 1024 * 1024

@@ -53,7 +53,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 2D bf16 tensor [outer][inner], row pitch row_bytes, box box_inner x
 // box_outer, 128-byte swizzle, zero fill out of bounds.
 int make_tmap(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t row_bytes,
-              uint32_t box_inner, uint32_t box_outer) {
+              uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
@@ -61,7 +62,7 @@ int make_tmap(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, in
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
   return NM_OK;
@@ -150,10 +151,10 @@ int make_tmap_meta(CUtensorMap* m, const void* base, int64_t rows16) {
 }
 
 // Number of 2-CTA clusters of this kernel that fit on the device at once.
-template <int BN, int NACC>
+template <int BN, int NACC, int MSUB>
 int resident_pairs() {
-  using Cfg = nm::Gemm2Cfg<BN, NACC>;
-  auto kern = nm::k_nm_gemm_2cta<BN, NACC>;
+  using Cfg = nm::Gemm2Cfg<BN, NACC, MSUB>;
+  auto kern = nm::k_nm_gemm_2cta<BN, NACC, MSUB>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) != cudaSuccess) {
     cudaGetLastError();
     return num_sms() / 2;
@@ -179,12 +180,18 @@ int resident_pairs() {
 
 // Persistent 2-CTA kernel for pure-sparse products whose A side is a whole
 // number of 256-row blocks.
-template <int BN, int NACC>
+template <int BN, int NACC, int MSUB>
 int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
-  using Cfg = nm::Gemm2Cfg<BN, NACC>;
-  CUtensorMap ta, tb, te;
+  using Cfg = nm::Gemm2Cfg<BN, NACC, MSUB>;
+  CUtensorMap ta, tb, te, ty;
   int rc;
   const int64_t kb = ceil_div(p.ks_lift, 128);
+  const bool tma_store = !p.out_fp32 && !p.transpose && (p.ldy % 8) == 0 &&
+                         (reinterpret_cast<uintptr_t>(p.y) & 15u) == 0;
+  if (tma_store) {
+    if ((rc = make_tmap(&ty, p.y, p.rows_b, p.rows_a, p.ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) != NM_OK)
+      return rc;
+  }
   if ((rc = make_tmap(&ta, p.a_s, p.ks_lift / 2, p.rows_a, p.ks_lift, 64, 128)) != NM_OK) return rc;
   if ((rc = make_tmap(&tb, p.b, p.ks_lift, p.rows_b, p.ks_lift * 2, 64, BN / 2)) != NM_OK) return rc;
   if ((rc = make_tmap_meta(&te, p.meta, ceil_div(p.rows_a, 128) * kb * 128)) != NM_OK) return rc;
@@ -193,20 +200,22 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   a.rows_b = p.rows_b;
   a.kb = static_cast<int>(kb);
   a.meta_kb = kb;
-  a.tiles_m = static_cast<int>(ceil_div(p.rows_a, 256));
+  a.tiles_m = static_cast<int>(ceil_div(p.rows_a, 256 * MSUB));
   a.tiles_n = static_cast<int>(ceil_div(p.rows_b, BN));
   a.Y = p.y;
   a.ldy = p.ldy;
   a.out_fp32 = p.out_fp32;
   a.transpose_out = p.transpose;
+  a.tma_store = tma_store ? 1 : 0;
+  if (!tma_store) ty = ta;                             // unused; any valid map
   const int tiles = a.tiles_m * a.tiles_n;
-  auto kern = nm::k_nm_gemm_2cta<BN, NACC>;
+  auto kern = nm::k_nm_gemm_2cta<BN, NACC, MSUB>;
   NM_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem));
   cudaLaunchConfig_t cfg{};
   // A persistent grid larger than the number of co-resident SM pairs would
   // run its last clusters after the others: size it by the occupancy query.
   static int resident = 0;
-  if (resident == 0) resident = resident_pairs<BN, NACC>();
+  if (resident == 0) resident = resident_pairs<BN, NACC, MSUB>();
   const int clusters = std::max(1, std::min(tiles, resident));
   cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
   cfg.blockDim = dim3(192, 1, 1);
@@ -219,7 +228,7 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta, tb, te, a));
+  NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta, tb, te, ty, a));
   NM_CUDA_TRY(cudaGetLastError());
   return NM_OK;
 }
@@ -249,48 +258,29 @@ int pick_splits(int64_t tiles, int64_t kb_total) {
   return s;
 }
 
-// Rounds of the persistent 2-CTA kernel times the per-tile MMA time (BN/2
-// cycles per K = 32 slice); a single accumulator buffer adds the epilogue.
-double cost_2cta(const GemmPlan& p, int bn, int nacc, int resident) {
-  const int64_t tiles = ceil_div(p.rows_a, 256) * ceil_div(p.rows_b, bn);
-  const int64_t clusters = std::max(1, resident);
-  const double rounds = static_cast<double>(ceil_div(tiles, clusters));
-  const double mma = static_cast<double>(ceil_div(p.ks_lift, 32)) * bn / 2.0;
-  const double epi = nacc == 1 ? bn * 12.0 : 0.0;
-  return rounds * (mma + epi);
-}
-
 // Kernel choice.  NMSPARSE_GEMM pins one variant where it applies:
-// "1cta", "2cta224", "2cta256", "2cta128"; unset or "auto" picks by shape.
+// "1cta", "2cta224", "2cta192", "2cta256", "2cta128", "2cta224x2", "2cta160x2";
+// unset or "auto" picks by shape.
 int run_gemm(const GemmPlan& p, cudaStream_t st) {
   const char* env = std::getenv("NMSPARSE_GEMM");
   const std::string mode = env != nullptr ? env : "auto";
   const bool eligible2 = p.kd == 0 && p.ks_lift > 0 && p.rows_a % 256 == 0;
+  const bool eligible4 = eligible2 && p.rows_a % 512 == 0;
   if (eligible2 && mode != "1cta") {
-    if (mode == "2cta224") return launch_gemm_2cta<224, 2>(p, st);
-    if (mode == "2cta192") return launch_gemm_2cta<192, 2>(p, st);
-    if (mode == "2cta256") return launch_gemm_2cta<256, 1>(p, st);
-    if (mode == "2cta128") return launch_gemm_2cta<128, 2>(p, st);
+    if (mode == "2cta224") return launch_gemm_2cta<224, 2, 1>(p, st);
+    if (mode == "2cta192") return launch_gemm_2cta<192, 2, 1>(p, st);
+    if (mode == "2cta256") return launch_gemm_2cta<256, 1, 1>(p, st);
+    if (mode == "2cta128") return launch_gemm_2cta<128, 2, 1>(p, st);
+    if (eligible4 && mode == "2cta224x2") return launch_gemm_2cta<224, 1, 2>(p, st);
+    if (eligible4 && mode == "2cta160x2") return launch_gemm_2cta<160, 1, 2>(p, st);
     if (p.rows_b >= 512 && p.ks_lift >= 512) {
-      static int res[4] = {0, 0, 0, 0};
-      if (res[0] == 0) {
-        res[0] = resident_pairs<224, 2>();
-        res[1] = resident_pairs<192, 2>();
-        res[2] = resident_pairs<256, 1>();
-        res[3] = resident_pairs<128, 2>();
-      }
-      // 128-wide tiles run near the shared-memory port limit: weight them
-      const double c[4] = {cost_2cta(p, 224, 2, res[0]), cost_2cta(p, 192, 2, res[1]),
-                           cost_2cta(p, 256, 1, res[2]), cost_2cta(p, 128, 2, res[3]) * 1.25};
-      int best = 0;
-      for (int i = 1; i < 4; ++i)
-        if (c[i] < c[best]) best = i;
-      switch (best) {
-        case 0: return launch_gemm_2cta<224, 2>(p, st);
-        case 1: return launch_gemm_2cta<192, 2>(p, st);
-        case 2: return launch_gemm_2cta<256, 1>(p, st);
-        default: return launch_gemm_2cta<128, 2>(p, st);
-      }
+      // Both 2:4 operands stream through shared memory, whose port bounds this
+      // kernel well before the tensor pipe does; measured on B200, the 224-wide
+      // tile with two accumulators (epilogue overlapped) is best except for
+      // long reductions on narrow outputs, where the 256-wide tile's fewer
+      // rounds outweigh its exposed epilogue.
+      if (p.rows_b <= 8192 && p.ks_lift >= 16384) return launch_gemm_2cta<256, 1, 1>(p, st);
+      return launch_gemm_2cta<224, 2, 1>(p, st);
     }
   }
   const int bn = pick_bn(p.rows_b);

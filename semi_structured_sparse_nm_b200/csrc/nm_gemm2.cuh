@@ -20,6 +20,12 @@
 //                the 4 epilogue warps of both CTAs.
 // Tiles are visited A-block fastest so that concurrently running clusters
 // share the B tile (the larger, streamed operand) through L2.
+//
+// MSUB = 2 makes the tile 512 x BN: each k-slice issues two M = 256 MMAs that
+// share the B stage (CTA r holds A rows 512 tm + 256 u + 128 r for u = 0, 1).
+// That cuts the shared-memory fill per MMA cycle from 64 + 8192/BN to
+// 32 + 8192/BN bytes per SM, which is what the L2 -> SM path can sustain;
+// tensor memory then holds one accumulator set (NACC = 1).
 #pragma once
 #include "nm_device.cuh"
 
@@ -79,6 +85,15 @@ __device__ __forceinline__ void tc_mma_sp_pair(uint32_t d_tmem, uint64_t adesc, 
       : "memory");
 }
 
+// TMA 2D store smem -> global (bulk-group completion), and its group waits.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+               :: "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(src)), "r"(x), "r"(y) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 struct Gemm2Args {
   int64_t rows_a, rows_b;
   int kb;                 // sparse k-blocks (128 lifted K each)
@@ -88,38 +103,44 @@ struct Gemm2Args {
   int64_t ldy;
   int out_fp32;
   int transpose_out;
+  int tma_store;          // 1: bf16 row-major Y written by TMA from a staging tile
 };
 
-template <int BN, int NACC>
+template <int BN, int NACC, int MSUB>
 struct Gemm2Cfg {
   static constexpr int kHalfN = BN / 2;
-  static constexpr int kA = 128 * 128;                 // 128 rows x 64 stored bf16
+  static constexpr int kA1 = 128 * 128;                // one subtile: 128 rows x 64 stored bf16
+  static constexpr int kA = MSUB * kA1;
   static constexpr int kB = 2 * kHalfN * 128;          // two 64-column halves
-  static constexpr int kE = 2048;
+  static constexpr int kE = MSUB * 2048;
   static constexpr int kStage = kA + kB + kE;
-  static constexpr int kStagesRaw = (200 * 1024) / kStage;
+  static constexpr int kStaging = 4 * 2 * 32 * 32 * 2;  // 4 epilogue warps x 2 buffers x 32x32 bf16
+  static constexpr int kStagesRaw = (232448 - kStaging - 2048) / kStage;
   static constexpr int kStages = kStagesRaw > 6 ? 6 : kStagesRaw;
   static constexpr int kTmemCols = 512;
-  static constexpr int kAccStride = 256;               // accumulator b at column 256 b
-  static constexpr int kMetaCol = (NACC - 1) * kAccStride + BN;
-  static constexpr int kSmem = kStages * kStage + 1024 + 512;
-  static_assert(kMetaCol + 4 * kStages <= kTmemCols, "tensor memory budget");
+  static constexpr int kAccStride = 256;               // accumulator (b, u) at column 256 (b MSUB + u)
+  static constexpr int kMetaCol = (NACC * MSUB - 1) * kAccStride + BN;
+  static constexpr int kSmem = kStages * kStage + kStaging + 1024 + 512;
+  static_assert(NACC * MSUB <= 2, "two accumulators of up to 256 columns");
+  static_assert(kMetaCol + 4 * MSUB * kStages <= kTmemCols, "tensor memory budget");
   static_assert(kHalfN % 8 == 0 && BN % 16 == 0 && BN <= 256, "MMA N");
   static_assert(kStages >= 3, "ring too shallow");
 };
 
-template <int BN, int NACC>
+template <int BN, int NACC, int MSUB>
 __global__ void __launch_bounds__(192, 1)
 k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               const __grid_constant__ CUtensorMap tmE, const Gemm2Args args) {
-  using Cfg = Gemm2Cfg<BN, NACC>;
+               const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
+               const Gemm2Args args) {
+  using Cfg = Gemm2Cfg<BN, NACC, MSUB>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw2[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw2) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + S * Cfg::kA;
   uint8_t* sE = sB + S * Cfg::kB;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(sE + S * Cfg::kE);
+  uint8_t* sY = sE + S * Cfg::kE;                    // epilogue staging (1024-aligned)
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(sY + Cfg::kStaging);
   uint64_t* empty_bar = full_bar + S;
   uint64_t* tfull_bar = empty_bar + S;
   uint64_t* tempty_bar = tfull_bar + NACC;
@@ -139,7 +160,10 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) { prefetch_tmap(&tmA); prefetch_tmap(&tmB); prefetch_tmap(&tmE); }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA); prefetch_tmap(&tmB); prefetch_tmap(&tmE);
+    if (args.tma_store) prefetch_tmap(&tmY);
+  }
   if (warp == 1) { tmem_alloc2(tmem_slot, Cfg::kTmemCols); tmem_relinquish2(); }
   tc_fence_before();
   cluster_barrier();          // barriers of both CTAs initialised, TMEM allocated
@@ -155,19 +179,22 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       bool ok = true;
       for (int t = cluster_id; t < tiles && ok; t += num_clusters) {
         const int tm = t % args.tiles_m, tn = t / args.tiles_m;
-        const int32_t ya = tm * 256 + static_cast<int32_t>(rank) * 128;
         const int32_t yb = tn * BN + static_cast<int32_t>(rank) * Cfg::kHalfN;
-        const int32_t ye_base = static_cast<int32_t>((static_cast<int64_t>(tm) * 2 + rank) * args.meta_kb * 128);
         for (int kb = 0; kb < args.kb; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
           if (!mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag, kWhereProducer)) { ok = false; break; }
           const uint32_t fb = leader_addr(smem_u32(&full_bar[s]));
           if (leader) mbar_arrive_expect_tx(&full_bar[s], stage_tx);
-          tma_load_2d_pair(&tmA, fb, sA + s * Cfg::kA, kb * 64, ya);
+#pragma unroll
+          for (int u = 0; u < MSUB; ++u) {
+            const int64_t rb = (static_cast<int64_t>(tm) * MSUB + u) * 2 + rank;       // 128-row block
+            tma_load_2d_pair(&tmA, fb, sA + s * Cfg::kA + u * Cfg::kA1, kb * 64, static_cast<int32_t>(rb * 128));
+            tma_load_2d_pair(&tmE, fb, sE + s * Cfg::kE + u * 2048, 0,
+                             static_cast<int32_t>((rb * args.meta_kb + kb) * 128));
+          }
           tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB, kb * 128, yb);
           tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB + Cfg::kHalfN * 128, kb * 128 + 64, yb);
-          tma_load_2d_pair(&tmE, fb, sE + s * Cfg::kE, 0, ye_base + kb * 128);
         }
       }
       // Every stage this CTA filled was released by the leader's commit
@@ -187,7 +214,7 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         const uint32_t use = static_cast<uint32_t>(lt / NACC);
         if (!mbar_wait(&tempty_bar[b], (use & 1u) ^ 1u, abort_flag, kWhereMma)) break;
         tc_fence_after();
-        const uint32_t acc = tmem_base + b * Cfg::kAccStride;
+        const uint32_t acc = tmem_base + b * MSUB * Cfg::kAccStride;
         for (int kb = 0; kb < args.kb; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
@@ -195,14 +222,19 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * Cfg::kA);
           const uint32_t b0 = smem_u32(sB + s * Cfg::kB);
-          const uint32_t e_col = tmem_meta + 4u * s;
-          tc_cp_pair_128x128b(e_col, desc_plain_128x16(smem_u32(sE + s * Cfg::kE)));
+          const uint32_t e_col = tmem_meta + 4u * MSUB * s;
+#pragma unroll
+          for (int u = 0; u < MSUB; ++u)
+            tc_cp_pair_128x128b(e_col + 4u * u, desc_plain_128x16(smem_u32(sE + s * Cfg::kE + u * 2048)));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = desc_sw128_kmajor(a0 + 32u * kk);
             const uint64_t bd = desc_sw128_kmajor(b0 + (kk / 2) * (Cfg::kHalfN * 128) + (kk % 2) * 64);
-            tc_mma_sp_pair(acc, ad, bd, e_col + (kk & ~1), idesc | static_cast<uint32_t>(kk & 1),
-                           (kb > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+            for (int u = 0; u < MSUB; ++u) {
+              const uint64_t ad = desc_sw128_kmajor(a0 + u * Cfg::kA1 + 32u * kk);
+              tc_mma_sp_pair(acc + u * Cfg::kAccStride, ad, bd, e_col + 4u * u + (kk & ~1),
+                             idesc | static_cast<uint32_t>(kk & 1), (kb > 0 || kk > 0) ? 1u : 0u);
+            }
           }
           tc_commit_pair(&empty_bar[s]);
         }
@@ -212,9 +244,10 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp % 4;
-    const uint32_t tempty_leader[2] = {leader_addr(smem_u32(&tempty_bar[0])),
-                                       leader_addr(smem_u32(&tempty_bar[NACC > 1 ? 1 : 0]))};
+    const uint32_t tempty_leader0 = leader_addr(smem_u32(&tempty_bar[0]));
+    const uint32_t tempty_leader1 = leader_addr(smem_u32(&tempty_bar[NACC > 1 ? 1 : 0]));
     int lt = 0;
+    uint32_t ebuf = 0;                                // staging tiles issued by this warp
     GemmArgs st{};
     st.rows_a = args.rows_a;
     st.rows_b = args.rows_b;
@@ -228,25 +261,58 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const uint32_t use = static_cast<uint32_t>(lt / NACC);
       if (!mbar_wait(&tfull_bar[b], use & 1u, abort_flag, kWhereEpilogue)) break;
       tc_fence_after();
-      const int64_t ra = static_cast<int64_t>(tm) * 256 + rank * 128 + q * 32 + lane;
-      const uint32_t acc = tmem_base + b * Cfg::kAccStride + (static_cast<uint32_t>(q * 32) << 16);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t v[32];
-        tc_ld_32x32b_x32(acc + c0, v);
-        tc_wait_ld();
-        if (c0 + 32 <= BN) {
-          store_row_chunk<32>(st, ra, static_cast<int64_t>(tn) * BN + c0, v);
-        } else {
+      for (int u = 0; u < MSUB; ++u) {
+        const int64_t row0 = (static_cast<int64_t>(tm) * MSUB + u) * 256 + rank * 128 + q * 32;
+        const int64_t ra = row0 + lane;
+        const uint32_t acc = tmem_base + (b * MSUB + u) * Cfg::kAccStride + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t v[32];
+          tc_ld_32x32b_x32(acc + c0, v);
+          tc_wait_ld();
+          if (args.tma_store) {
+            // 32 rows x 32 bf16 staging tile, 64-byte swizzle: row r's 16-byte
+            // chunk j sits at r*64 + 16*(j ^ ((r >> 1) & 3)).  Two buffers per
+            // warp; a buffer is rewritten only after its previous store read it.
+            uint8_t* buf = sY + (q * 2 + (ebuf & 1)) * 2048;
+            if (lane == 0 && ebuf >= 2) bulk_wait_read1();
+            __syncwarp();
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c0 + i < BN) store_out(st, ra, static_cast<int64_t>(tn) * BN + c0 + i, __uint_as_float(v[i]));
+            for (int j = 0; j < 4; ++j) {
+              uint32_t p[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[8 * j + 2 * k]),
+                                                         __uint_as_float(v[8 * j + 2 * k + 1]));
+                p[k] = *reinterpret_cast<uint32_t*>(&h);
+              }
+              *reinterpret_cast<uint4*>(buf + lane * 64 + 16 * (j ^ ((lane >> 1) & 3))) =
+                  make_uint4(p[0], p[1], p[2], p[3]);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, buf, static_cast<int32_t>(static_cast<int64_t>(tn) * BN + c0),
+                           static_cast<int32_t>(row0));
+              bulk_commit();
+            }
+            ++ebuf;
+          } else if (c0 + 32 <= BN) {
+            store_row_chunk<32>(st, ra, static_cast<int64_t>(tn) * BN + c0, v);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c0 + i < BN) store_out(st, ra, static_cast<int64_t>(tn) * BN + c0 + i, __uint_as_float(v[i]));
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty_leader[b]);
+      if (lane == 0) mbar_arrive_cluster(b == 0 ? tempty_leader0 : tempty_leader1);
     }
+    if (args.tma_store && lane == 0) bulk_wait_all();   // stores done before the CTA exits
+    __syncwarp();
   }
 
   tc_fence_before();

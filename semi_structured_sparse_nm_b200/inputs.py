@@ -113,6 +113,8 @@ WORKLOADS = {
     w.name: w for w in [
         Workload("tiny_2of4_act_fp32", "act", 16, 256, 128, 2, 4, "fp32", "fp32", "normal"),
         Workload("up_proj_8of16_act", "act", 2048, 4096, 14336, 8, 16, "bf16", "bf16", "student_t4"),
+        # the same shape pruned 2:4: the 2:4 prefill GEMM measurement
+        Workload("up_proj_2of4_act", "act", 2048, 4096, 14336, 2, 4, "bf16", "bf16", "student_t4"),
         Workload("slide_6of8_wt_prefill", "weight", 4096, 4096, 4096, 6, 8, "bf16", "bf16", "normal"),
         Workload("slide_6of8_wt_decode", "weight", 16, 4096, 4096, 6, 8, "bf16", "bf16", "normal"),
         Workload("down_proj_16of32_act", "act", 4096, 14336, 4096, 16, 32, "bf16", "bf16", "normal_outliers"),
