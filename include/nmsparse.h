@@ -15,6 +15,10 @@
  *    one for every operand.
  *  - Pointers must be 16-byte aligned and leading dimensions multiples of 8
  *    elements (16 bytes for bf16 rows), else NM_ERR_ALIGNMENT.
+ *  - Weight operands (the sparse operand of NM_WEIGHT products, the hybrid
+ *    weight) may be read while the kernel issued just before on the same
+ *    stream is still finishing (programmatic dependent launch); they must
+ *    not be written by that kernel.  Everything else waits for it.
  *
  * Terms.  An N:M pattern keeps the N entries of largest magnitude in every
  * aligned group of M consecutive entries along K, ties going to the lower

@@ -78,6 +78,7 @@ struct GemmPlan {
   void* y = nullptr;
   int64_t ldy = 0;
   int out_fp32 = 0, transpose = 0;
+  int a_static = 0;           // A is a weight: may be read before the preceding kernel ends
 };
 
 template <int BN>
@@ -110,6 +111,7 @@ int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
   args.out_fp32 = p.out_fp32;
   args.transpose_out = p.transpose;
   args.splits = splits;
+  args.a_static = p.a_static;
 
   auto kern = nm::k_nm_gemm<BN>;
   NM_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
@@ -120,16 +122,23 @@ int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
   cfg.blockDim = dim3(192, 1, 1);
   cfg.dynamicSmemBytes = Cfg::kSmemBytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  cfg.numAttrs = 0;
+  // Programmatic dependent launch: the kernel may start while the preceding
+  // kernel in the stream finishes; it waits for it (griddepcontrol.wait)
+  // before touching anything but the static weight operand.
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
   if (splits > 1) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = static_cast<unsigned>(splits);
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = static_cast<unsigned>(splits);
+    ++na;
   }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
   NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta_s, ta_d, tb, args));
   NM_CUDA_TRY(cudaGetLastError());
   return NM_OK;
@@ -427,6 +436,7 @@ int nm_sparse_gemm(const nm_sparse_operand* S, const void* D, int64_t rows_d, nm
   p.out_fp32 = out_dt == NM_FP32;
   p.transpose = side == NM_WEIGHT;
   p.ldy = side == NM_ACT ? rows_d : S->rows;
+  p.a_static = side == NM_WEIGHT;
   return run_gemm(p, static_cast<cudaStream_t>(stream));
 }
 
@@ -534,6 +544,7 @@ int hybrid_gemm(const void* X, int64_t B, const nm_hybrid_weight* W, void* Y, nm
   p.ldy = W->O;
   p.out_fp32 = out_dt == NM_FP32;
   p.transpose = 1;
+  p.a_static = 1;
   return run_gemm(p, st);
 }
 

@@ -35,6 +35,8 @@ struct GemmArgs {
   int out_fp32;
   int transpose_out;                        // 1: Y[b][a]; 0: Y[a][b]
   int splits;                               // CTAs per output tile (cluster size)
+  int a_static;                             // A (and its metadata) may be read before the
+                                            // preceding kernel finishes; B only after
 };
 
 template <int BN>
@@ -66,9 +68,10 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
   return v;
 }
 
@@ -155,27 +158,46 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
   if (warp == 0) {
     // ---------------------------------------------------------- producer
     if (elect_one()) {
-      int it = 0;
-      for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
-        const int s = it % S;
-        const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
-        if (!mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag, kWhereProducer)) break;
+      const int32_t y_a = static_cast<int32_t>(m_tile * kBM), y_b = static_cast<int32_t>(n_tile * BN);
+      auto load_a = [&](int kb, int s) {
         uint8_t* a_dst = sA + s * kABytes;
-        uint8_t* b_dst = sB + s * Cfg::kBBytes;
-        const int32_t y_a = static_cast<int32_t>(m_tile * kBM), y_b = static_cast<int32_t>(n_tile * BN);
         if (kb < args.kb_sparse) {
           mbar_arrive_expect_tx(&full_bar[s], kABytes + Cfg::kBBytes + kEBytes);
           tma_load_2d(&tmA_s, &full_bar[s], a_dst, kb * 64, y_a);
-          tma_load_2d(&tmB, &full_bar[s], b_dst, kb * 128, y_b);
-          tma_load_2d(&tmB, &full_bar[s], b_dst + BN * 128, kb * 128 + 64, y_b);
           bulk_load(sE + s * kEBytes, args.meta + (m_tile * args.meta_kb + kb) * kEBytes, kEBytes,
                     &full_bar[s]);
         } else {
-          const int kd = kb - args.kb_sparse;
           mbar_arrive_expect_tx(&full_bar[s], kABytes + BN * 128);
-          tma_load_2d(&tmA_d, &full_bar[s], a_dst, kd * 64, y_a);
-          tma_load_2d(&tmB, &full_bar[s], b_dst, static_cast<int32_t>(args.k_dense_x0) + kd * 64, y_b);
+          tma_load_2d(&tmA_d, &full_bar[s], a_dst, (kb - args.kb_sparse) * 64, y_a);
         }
+      };
+      auto load_b = [&](int kb, int s) {
+        uint8_t* b_dst = sB + s * Cfg::kBBytes;
+        if (kb < args.kb_sparse) {
+          tma_load_2d(&tmB, &full_bar[s], b_dst, kb * 128, y_b);
+          tma_load_2d(&tmB, &full_bar[s], b_dst + BN * 128, kb * 128 + 64, y_b);
+        } else {
+          tma_load_2d(&tmB, &full_bar[s], b_dst,
+                      static_cast<int32_t>(args.k_dense_x0) + (kb - args.kb_sparse) * 64, y_b);
+        }
+      };
+      // The static operand of the first ring's worth of stages is requested
+      // while the preceding kernel may still run; everything else waits for it.
+      int it = 0;
+      int pre = 0;
+      if (args.a_static) {
+        pre = kb_end - kb_begin < S ? kb_end - kb_begin : S;
+        for (int j = 0; j < pre; ++j) load_a(kb_begin + j, j);
+      }
+      griddep_wait();
+      for (int j = 0; j < pre; ++j) load_b(kb_begin + j, j);
+      it = pre;
+      for (int kb = kb_begin + pre; kb < kb_end; ++kb, ++it) {
+        const int s = it % S;
+        const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+        if (!mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag, kWhereProducer)) break;
+        load_a(kb, s);
+        load_b(kb, s);
       }
       // Only the last S loads can still be in flight (a stage is reissued only
       // after the MMA released it); wait for them before the CTA may exit.
@@ -226,6 +248,7 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
     // -------------------------------------------------------- epilogue
     const int q = warp % 4;
     const bool ok = mbar_wait(accum_bar, 0u, abort_flag, kWhereEpilogue);
+    griddep_wait();                                  // Y may still be in use upstream
     tc_fence_after();
     if (ok) {
       const int64_t row_local = q * 32 + lane;
@@ -257,19 +280,33 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
     __syncwarp();
     cluster_sync_all();
     if (!*abort_flag) {
+      // Four consecutive columns per thread; all partial loads are issued
+      // before the (rank-ordered, hence deterministic) sum.
       const uint32_t rank = cluster_ctarank();
       const int rows_per = kBM / args.splits;
-      const int elems = rows_per * BN;
+      const int quads = rows_per * (BN / 4);
       const uint32_t red_base = smem_u32(smem);
-      for (int e = threadIdx.x; e < elems; e += blockDim.x) {
-        int rl, c;
-        if (args.transpose_out) { rl = e % rows_per; c = e / rows_per; }
-        else { rl = e / BN; c = e % BN; }
+      griddep_wait();
+      for (int e = threadIdx.x; e < quads; e += blockDim.x) {
+        const int rl = args.transpose_out ? e % rows_per : e / (BN / 4);
+        const int c = 4 * (args.transpose_out ? e / rows_per : e % (BN / 4));
         const int row_local = static_cast<int>(rank) * rows_per + rl;
-        const uint32_t off = static_cast<uint32_t>((row_local * BN + c) * 4);
-        float acc = 0.f;
-        for (int p = 0; p < args.splits; ++p) acc += ld_dsmem_f32(mapa_shared(red_base + off, p));
-        store_out(args, m_tile * kBM + row_local, n_tile * BN + c, acc);
+        const uint32_t off = red_base + static_cast<uint32_t>((row_local * BN + c) * 4);
+        float4 part[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p)
+          if (p < args.splits) part[p] = ld_dsmem_f32x4(mapa_shared(off, static_cast<uint32_t>(p)));
+        float4 acc = part[0];
+#pragma unroll
+        for (int p = 1; p < 8; ++p)
+          if (p < args.splits) {
+            acc.x += part[p].x; acc.y += part[p].y; acc.z += part[p].z; acc.w += part[p].w;
+          }
+        const int64_t ra = m_tile * kBM + row_local, cb = n_tile * BN + c;
+        store_out(args, ra, cb, acc.x);
+        store_out(args, ra, cb + 1, acc.y);
+        store_out(args, ra, cb + 2, acc.z);
+        store_out(args, ra, cb + 3, acc.w);
       }
     }
     cluster_sync_all();

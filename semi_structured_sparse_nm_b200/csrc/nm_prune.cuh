@@ -181,6 +181,83 @@ __device__ __forceinline__ uint32_t compress_group(const GroupRaw<M, T>& raw, in
   return keep;
 }
 
+// Window table: for each 4-bit set c of still-unplaced kept positions of a
+// window (local positions 0..3), .x = byte-permute selectors (bits 0-15 pick
+// the two kept values out of the window's four, bits 16-31 then zero the
+// padded slot), .y = index pair (bits 0-3) | placed positions 2,3 (bits 4-5,
+// carried into the next window as its positions 0,1).  The window takes the
+// lowest two positions of c; one entry at a is paired with the lowest other
+// index (value +0.0), none gives (0, 1).
+__device__ __forceinline__ uint2 window_entry(uint32_t c) {
+  const uint32_t f = c & (0u - c);
+  const uint32_t rest = c ^ f;
+  const uint32_t sb = rest & (0u - rest);
+  const uint32_t taken = f | sb;
+  int i0 = 0, i1 = 1;
+  bool z0 = true, z1 = true;                      // slot holds padding
+  if (sb) { i0 = __ffs(f) - 1; i1 = __ffs(sb) - 1; z0 = z1 = false; }
+  else if (f) {
+    const int a = __ffs(f) - 1;
+    if (a == 0) { z0 = false; } else { i1 = a; z1 = false; }
+  }
+  const uint32_t sel = static_cast<uint32_t>((0x10 + 0x22 * i0) | ((0x10 + 0x22 * i1) << 8));
+  const uint32_t zsel = (z0 ? 0x54u : 0x10u) | ((z1 ? 0x76u : 0x32u) << 8);   // bytes 4..7 of 0 are zero
+  return make_uint2(sel | (zsel << 16), static_cast<uint32_t>(i0 | (i1 << 2)) | ((taken >> 2) << 4));
+}
+
+// bf16 groups held as 32-bit pair words P[p] = (x[2p], x[2p+1]): unique keys
+// are formed on the fly, kept entries are those whose key is at least the N-th
+// largest (sign of thr - 1 - key), windows come from the table.
+template <int M>
+__device__ __forceinline__ uint32_t ukey_bf16(const uint32_t (&P)[M / 2], int i) {
+  const uint32_t w = P[i >> 1];
+  const uint32_t k = (i & 1) ? ((w >> 16) & 0x7FFFu) : (w & 0x7FFFu);
+  return (k << 5) | static_cast<uint32_t>(31 - i);
+}
+
+template <int M>
+__device__ __forceinline__ uint32_t compress_group_bf16(const uint32_t (&P)[M / 2], int N, const uint2* lut,
+                                                        uint32_t* val_out, uint8_t* nib_out) {
+  constexpr int NW = M / 2 - 1;
+  uint32_t keep = 0u;
+  if (N > 0) {
+    uint32_t thr;
+    if (2 * N == M) {
+      constexpr int H = M / 2;
+      uint32_t a[H], b[H];
+#pragma unroll
+      for (int i = 0; i < H; ++i) { a[i] = ukey_bf16<M>(P, i); b[i] = ukey_bf16<M>(P, H + i); }
+      bitonic_desc<H, uint32_t>(a);
+      bitonic_desc<H, uint32_t>(b);
+      thr = kmax(a[0], b[H - 1]);
+#pragma unroll
+      for (int i = 1; i < H; ++i) thr = kmin(thr, kmax(a[i], b[H - 1 - i]));
+    } else {
+      uint32_t srt[M];
+#pragma unroll
+      for (int i = 0; i < M; ++i) srt[i] = ukey_bf16<M>(P, i);
+      bitonic_desc<M, uint32_t>(srt);
+      thr = srt[0];
+#pragma unroll
+      for (int k = 1; k < M; ++k) thr = (N > k) ? srt[k] : thr;
+    }
+    const uint32_t t1 = thr - 1u;
+#pragma unroll
+    for (int i = 0; i < M; ++i) keep |= ((t1 - ukey_bf16<M>(P, i)) >> 31) << i;
+  }
+  uint32_t carry = 0u;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) {
+    const uint32_t c = ((keep >> (2 * w)) & 0xFu) & ~carry;
+    const uint2 e = lut[c];
+    const uint32_t v = __byte_perm(P[w], P[w + 1], e.x & 0xFFFFu);
+    val_out[w] = __byte_perm(v, 0u, e.x >> 16);
+    nib_out[w] = static_cast<uint8_t>(e.y & 0xFu);
+    carry = (e.y >> 4) & 0x3u;
+  }
+  return keep;
+}
+
 // One CTA task = 16 consecutive rows x 32 consecutive groups; warp w takes
 // rows 2w and 2w+1 (both loads in flight together), lane = group.  32 groups
 // hold 32*NW windows, exactly NW metadata blocks of 32 windows, and 16 rows
@@ -204,7 +281,10 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
   __shared__ __align__(16) uint8_t s_nib[16][WIN];
   __shared__ __align__(16) uint32_t s_val[kPruneWarps][WIN];
   __shared__ uint32_t s_mask[kPruneWarps][M];
+  __shared__ uint2 s_lut[16];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  griddep_launch_dependents();
+  if (threadIdx.x < 16) s_lut[threadIdx.x] = window_entry(threadIdx.x);
   const int64_t groups = K / M;
   const int64_t cpr = (groups + 31) / 32;
   const int64_t mask_words = (K + 31) / 32;
@@ -235,7 +315,18 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
       if (g < groups) {
         uint32_t vals[NW];
         uint8_t nibs[NW];
-        const uint32_t keep = compress_group<M, T>(raw[k], N, vals, nibs);
+        uint32_t keep;
+        if constexpr (sizeof(T) == 2) {
+          uint32_t P[M / 2];
+#pragma unroll
+          for (int p = 0; p < M / 2; ++p) {
+            const uint4& q = raw[k].v[p / 4];
+            P[p] = (p % 4 == 0) ? q.x : (p % 4 == 1) ? q.y : (p % 4 == 2) ? q.z : q.w;
+          }
+          keep = compress_group_bf16<M>(P, N, s_lut, vals, nibs);
+        } else {
+          keep = compress_group<M, T>(raw[k], N, vals, nibs);
+        }
 #pragma unroll
         for (int w = 0; w < NW; ++w) {
           s_val[warp][lane * NW + w] = vals[w];
@@ -295,6 +386,7 @@ k_lift(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
   constexpr int NW = M / 2 - 1;
   const int64_t groups = K / M;
   const int64_t total = rows * groups;
+  griddep_launch_dependents();
   for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t r = t / groups, g = t % groups;
@@ -360,6 +452,7 @@ __global__ void k_gather_cols(const uint16_t* __restrict__ src, int64_t rows, in
                               const int32_t* __restrict__ perm, int64_t split,
                               uint16_t* __restrict__ dst_lo, uint16_t* __restrict__ dst_hi) {
   const int64_t total = rows * K;
+  griddep_launch_dependents();
   for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t r = t / K, i = t % K;
