@@ -133,7 +133,8 @@ int slide_decompose(const void *w, nm_dtype dt, int64_t rows, int64_t K, int N, 
 
 /* Lifts the dense operand: dst[r][g*4(n-1) + 4w + j] = src[r][g*2n + 2w + j]
  * for M = 2n, src [rows x K] (row stride ld elements, bf16 or fp32),
- * dst bf16 [rows x K'] (row stride K').  M = 4 copies (and converts fp32). */
+ * dst bf16 [rows x K'] (row stride K').  M = 4 copies (and converts fp32).
+ * K' must be a multiple of 8 (16-byte rows), else NM_ERR_ALIGNMENT. */
 int nm_lift(const void *src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, int M,
             void *dst, void *stream);
 

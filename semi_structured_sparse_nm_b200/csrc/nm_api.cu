@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <utility>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -66,6 +67,26 @@ int make_tmap(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, in
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
   return NM_OK;
+}
+
+// Launch with programmatic stream serialisation: the kernel may start while
+// the preceding kernel in the stream finishes; every kernel of this library
+// waits (griddepcontrol.wait) before it touches memory the preceding kernel
+// may own.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // ----------------------------------------------------------------- GEMM
@@ -230,13 +251,15 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   cfg.blockDim = dim3(192, 1, 1);
   cfg.dynamicSmemBytes = Cfg::kSmem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta, tb, te, ty, a));
   NM_CUDA_TRY(cudaGetLastError());
   return NM_OK;
@@ -317,13 +340,15 @@ int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M
   const dim3 grid(static_cast<unsigned>(blocks)), block(nm::kPruneWarps * 32);
   auto v = static_cast<uint32_t*>(vals);
   auto e = static_cast<uint8_t*>(meta);
+  cudaError_t err;
   switch (M) {
-    case 4: nm::k_prune_compress<4, T><<<grid, block, 0, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
-    case 8: nm::k_prune_compress<8, T><<<grid, block, 0, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
-    case 16: nm::k_prune_compress<16, T><<<grid, block, 0, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
-    case 32: nm::k_prune_compress<32, T><<<grid, block, 0, st>>>(src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
+    case 4: err = launch_pdl(nm::k_prune_compress<4, T>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
+    case 8: err = launch_pdl(nm::k_prune_compress<8, T>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
+    case 16: err = launch_pdl(nm::k_prune_compress<16, T>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
+    case 32: err = launch_pdl(nm::k_prune_compress<32, T>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
     default: return NM_ERR_UNSUPPORTED;
   }
+  NM_CUDA_TRY(err);
   NM_CUDA_TRY(cudaGetLastError());
   return NM_OK;
 }
@@ -331,16 +356,19 @@ int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M
 template <typename T>
 int launch_lift(const T* src, int64_t rows, int64_t K, int64_t ld, int M, void* dst, cudaStream_t st) {
   const int64_t Kl = nm_lifted_k(K, M);
-  const int64_t total = rows * (K / M);
-  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(total, 256), int64_t(num_sms()) * 16));
+  const int64_t total = rows * ((K / M + 1) / 2);
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(total, 256), int64_t(1) << 30));
   auto d = static_cast<uint16_t*>(dst);
+  const dim3 grid(static_cast<unsigned>(blocks)), block(256);
+  cudaError_t err;
   switch (M) {
-    case 4: nm::k_lift<4, T><<<static_cast<unsigned>(blocks), 256, 0, st>>>(src, rows, K, ld, d, Kl); break;
-    case 8: nm::k_lift<8, T><<<static_cast<unsigned>(blocks), 256, 0, st>>>(src, rows, K, ld, d, Kl); break;
-    case 16: nm::k_lift<16, T><<<static_cast<unsigned>(blocks), 256, 0, st>>>(src, rows, K, ld, d, Kl); break;
-    case 32: nm::k_lift<32, T><<<static_cast<unsigned>(blocks), 256, 0, st>>>(src, rows, K, ld, d, Kl); break;
+    case 4: err = launch_pdl(nm::k_lift<4, T>, grid, block, 0, st, src, rows, K, ld, d, Kl); break;
+    case 8: err = launch_pdl(nm::k_lift<8, T>, grid, block, 0, st, src, rows, K, ld, d, Kl); break;
+    case 16: err = launch_pdl(nm::k_lift<16, T>, grid, block, 0, st, src, rows, K, ld, d, Kl); break;
+    case 32: err = launch_pdl(nm::k_lift<32, T>, grid, block, 0, st, src, rows, K, ld, d, Kl); break;
     default: return NM_ERR_UNSUPPORTED;
   }
+  NM_CUDA_TRY(err);
   NM_CUDA_TRY(cudaGetLastError());
   return NM_OK;
 }
@@ -399,7 +427,8 @@ int nm_lift(const void* src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, i
   if (rows == 0) return NM_OK;
   if (src == nullptr || dst == nullptr) return NM_ERR_INVALID_ARG;
   const int64_t esz = dt == NM_BF16 ? 2 : 4;
-  if (!aligned16(src) || !aligned16(dst) || (ld * esz) % 16 != 0) return NM_ERR_ALIGNMENT;
+  if (!aligned16(src) || !aligned16(dst) || (ld * esz) % 16 != 0 || (nm_lifted_k(K, M) % 8) != 0)
+    return NM_ERR_ALIGNMENT;
   if (rows == 0) return NM_OK;
   auto st = static_cast<cudaStream_t>(stream);
   if (dt == NM_BF16) return launch_lift(static_cast<const uint16_t*>(src), rows, K, ld, M, dst, st);
@@ -494,13 +523,16 @@ int hybrid_prepare(const void* w, int64_t O, int64_t K, double dense_frac, nm_hy
   uint8_t* is_dense = base + ceil_div(K * 8, 256) * 256;
   uint16_t* wsp = reinterpret_cast<uint16_t*>(is_dense + ceil_div(K, 256) * 256);
   const unsigned cb = static_cast<unsigned>(ceil_div(K, 128));
-  nm::k_colnorm_f64<<<cb, 128, 0, st>>>(static_cast<const uint16_t*>(w), O, K, colnorm);
-  nm::k_hybrid_rank<<<cb, 128, 0, st>>>(colnorm, K, D, is_dense);
-  nm::k_hybrid_perm<<<cb, 128, 0, st>>>(is_dense, K, D, out->perm);
+  NM_CUDA_TRY(launch_pdl(nm::k_colnorm_f64, dim3(cb), dim3(128), 0, st, static_cast<const uint16_t*>(w), O, K,
+                         colnorm));
+  NM_CUDA_TRY(launch_pdl(nm::k_hybrid_rank, dim3(cb), dim3(128), 0, st, static_cast<const double*>(colnorm), K, D,
+                         is_dense));
+  NM_CUDA_TRY(launch_pdl(nm::k_hybrid_perm, dim3(cb), dim3(128), 0, st, static_cast<const uint8_t*>(is_dense), K,
+                         D, out->perm));
   const int64_t gblocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(O * K, 256), int64_t(num_sms()) * 16));
-  nm::k_gather_cols<<<static_cast<unsigned>(gblocks), 256, 0, st>>>(
-      static_cast<const uint16_t*>(w), O, K, out->perm, Ks, wsp, static_cast<uint16_t*>(out->W_d));
-  NM_CUDA_TRY(cudaGetLastError());
+  NM_CUDA_TRY(launch_pdl(nm::k_gather_cols, dim3(static_cast<unsigned>(gblocks)), dim3(256), 0, st,
+                         static_cast<const uint16_t*>(w), O, K, static_cast<const int32_t*>(out->perm), Ks, wsp,
+                         static_cast<uint16_t*>(out->W_d)));
   if (Ks > 0) return launch_prune(wsp, O, Ks, Ks, 2, 4, nullptr, out->vals_s, out->meta_s, st);
   return NM_OK;
 }
@@ -528,9 +560,9 @@ int hybrid_gemm(const void* X, int64_t B, const nm_hybrid_weight* W, void* Y, nm
   auto st = static_cast<cudaStream_t>(stream);
   uint16_t* xp = static_cast<uint16_t*>(ws);
   const int64_t gblocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(B * W->K, 256), int64_t(num_sms()) * 4));
-  nm::k_gather_cols<<<static_cast<unsigned>(gblocks), 256, 0, st>>>(static_cast<const uint16_t*>(X), B, W->K,
-                                                                   W->perm, W->K, xp, nullptr);
-  NM_CUDA_TRY(cudaGetLastError());
+  NM_CUDA_TRY(launch_pdl(nm::k_gather_cols, dim3(static_cast<unsigned>(gblocks)), dim3(256), 0, st,
+                         static_cast<const uint16_t*>(X), B, W->K, static_cast<const int32_t*>(W->perm), W->K, xp,
+                         static_cast<uint16_t*>(nullptr)));
   GemmPlan p;
   p.a_s = W->vals_s;
   p.a_d = W->W_d;

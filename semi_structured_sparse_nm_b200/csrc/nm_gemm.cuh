@@ -88,6 +88,20 @@ template <int CW>
 __device__ __forceinline__ void store_row_chunk(const GemmArgs& a, int64_t ra, int64_t cb0,
                                                 const uint32_t (&v)[CW]) {
   if (ra >= a.rows_a) return;
+  if (a.transpose_out && cb0 + CW <= a.rows_b) {
+    // Y[b][a]: lane = a, so each store instruction of the warp writes 32
+    // consecutive outputs of one row of Y
+    if (a.out_fp32) {
+      float* p = static_cast<float*>(a.Y) + cb0 * a.ldy + ra;
+#pragma unroll
+      for (int i = 0; i < CW; ++i) p[i * a.ldy] = __uint_as_float(v[i]);
+    } else {
+      __nv_bfloat16* p = static_cast<__nv_bfloat16*>(a.Y) + cb0 * a.ldy + ra;
+#pragma unroll
+      for (int i = 0; i < CW; ++i) p[i * a.ldy] = __float2bfloat16_rn(__uint_as_float(v[i]));
+    }
+    return;
+  }
   if (!a.transpose_out && cb0 + CW <= a.rows_b && (a.ldy % 8) == 0) {
     if (a.out_fp32) {
       float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.Y) + ra * a.ldy + cb0);
@@ -154,6 +168,7 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
   tc_fence_after();
   const uint32_t tmem_acc = *tmem_slot;
   const uint32_t tmem_meta = tmem_acc + BN;
+  griddep_launch_dependents();                       // the next kernel may begin its set-up
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer

@@ -170,6 +170,8 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t tmem_meta = tmem_base + Cfg::kMetaCol;
+  griddep_launch_dependents();
+  griddep_wait();                                    // operands and Y belong to the preceding kernel until it ends
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer

@@ -78,6 +78,38 @@ __device__ __forceinline__ void bitonic_desc(K (&a)[M]) {
   }
 }
 
+// Batcher's odd-even merge network on N (power of two) inputs, as a
+// compile-time list of comparators: N(log N)(log N - 1)/4 + N - 1 of them
+// (19 for 8, 63 for 16, 191 for 32), fewer than the bitonic network's.
+template <int N>
+struct OddEvenNet {
+  int n = 0;
+  unsigned char lo[256] = {}, hi[256] = {};
+  constexpr OddEvenNet() {
+    for (int p = 1; p < N; p <<= 1)
+      for (int k = p; k >= 1; k >>= 1)
+        for (int j = k % p; j + k < N; j += 2 * k)
+          for (int i = 0; i < k; ++i)
+            if (i + j + k < N && (i + j) / (2 * p) == (i + j + k) / (2 * p)) {
+              lo[n] = static_cast<unsigned char>(i + j);
+              hi[n] = static_cast<unsigned char>(i + j + k);
+              ++n;
+            }
+  }
+};
+
+// Sorts N keys in registers in descending order.
+template <int N, typename K>
+__device__ __forceinline__ void oddeven_desc(K (&a)[N]) {
+  constexpr OddEvenNet<N> net{};
+#pragma unroll
+  for (int c = 0; c < net.n; ++c) {
+    const K x = a[net.lo[c]], y = a[net.hi[c]];
+    a[net.lo[c]] = kmax(x, y);
+    a[net.hi[c]] = kmin(x, y);
+  }
+}
+
 // Raw bytes of one group, as loaded (16-byte words, or one 8-byte word).
 template <int M, typename T>
 struct GroupRaw {
@@ -221,29 +253,32 @@ __device__ __forceinline__ uint32_t compress_group_bf16(const uint32_t (&P)[M / 
   constexpr int NW = M / 2 - 1;
   uint32_t keep = 0u;
   if (N > 0) {
+    uint32_t key[M];
+#pragma unroll
+    for (int i = 0; i < M; ++i) key[i] = ukey_bf16<M>(P, i);
     uint32_t thr;
     if (2 * N == M) {
       constexpr int H = M / 2;
       uint32_t a[H], b[H];
 #pragma unroll
-      for (int i = 0; i < H; ++i) { a[i] = ukey_bf16<M>(P, i); b[i] = ukey_bf16<M>(P, H + i); }
-      bitonic_desc<H, uint32_t>(a);
-      bitonic_desc<H, uint32_t>(b);
+      for (int i = 0; i < H; ++i) { a[i] = key[i]; b[i] = key[H + i]; }
+      oddeven_desc<H, uint32_t>(a);
+      oddeven_desc<H, uint32_t>(b);
       thr = kmax(a[0], b[H - 1]);
 #pragma unroll
       for (int i = 1; i < H; ++i) thr = kmin(thr, kmax(a[i], b[H - 1 - i]));
     } else {
       uint32_t srt[M];
 #pragma unroll
-      for (int i = 0; i < M; ++i) srt[i] = ukey_bf16<M>(P, i);
-      bitonic_desc<M, uint32_t>(srt);
+      for (int i = 0; i < M; ++i) srt[i] = key[i];
+      oddeven_desc<M, uint32_t>(srt);
       thr = srt[0];
 #pragma unroll
       for (int k = 1; k < M; ++k) thr = (N > k) ? srt[k] : thr;
     }
     const uint32_t t1 = thr - 1u;
 #pragma unroll
-    for (int i = 0; i < M; ++i) keep |= ((t1 - ukey_bf16<M>(P, i)) >> 31) << i;
+    for (int i = 0; i < M; ++i) keep |= ((t1 - key[i]) >> 31) << i;
   }
   uint32_t carry = 0u;
 #pragma unroll
@@ -285,6 +320,7 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   griddep_launch_dependents();
   if (threadIdx.x < 16) s_lut[threadIdx.x] = window_entry(threadIdx.x);
+  griddep_wait();                                      // inputs / outputs of the preceding kernel
   const int64_t groups = K / M;
   const int64_t cpr = (groups + 31) / 32;
   const int64_t mask_words = (K + 31) / 32;
@@ -378,29 +414,47 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
   }
 }
 
-// Lift: dst[r][g*4(n-1) + 4w + j] = src[r][g*2n + 2w + j]; one thread per group.
+// Lift: dst[r][g*4(n-1) + 4w + j] = src[r][g*2n + 2w + j].  One thread per
+// pair of groups, so that the 2 * 4(n-1) lifted values (a multiple of 8) go
+// out as 16-byte stores; a row with an odd number of groups finishes its last
+// group with 8-byte stores.
+template <int M, typename T>
+__device__ __forceinline__ uint2 lift_window(const T (&x)[M], int w) {
+  uint2 v;
+  v.x = static_cast<uint32_t>(to_bf16_bits(x[2 * w])) | (static_cast<uint32_t>(to_bf16_bits(x[2 * w + 1])) << 16);
+  v.y = static_cast<uint32_t>(to_bf16_bits(x[2 * w + 2])) | (static_cast<uint32_t>(to_bf16_bits(x[2 * w + 3])) << 16);
+  return v;
+}
+
 template <int M, typename T>
 __global__ void __launch_bounds__(256)
 k_lift(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
        uint16_t* __restrict__ dst, int64_t Kl) {
   constexpr int NW = M / 2 - 1;
   const int64_t groups = K / M;
-  const int64_t total = rows * groups;
+  const int64_t pairs = (groups + 1) / 2;
+  const int64_t total = rows * pairs;
   griddep_launch_dependents();
+  griddep_wait();
   for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = t / groups, g = t % groups;
-    T x[M];
-    load_group<M, T>(src + r * ld + g * M, x);
-    uint2* out = reinterpret_cast<uint2*>(dst + r * Kl + g * 4 * NW);
+    const int64_t r = t / pairs, g = 2 * (t % pairs);
+    T x0[M];
+    load_group<M, T>(src + r * ld + g * M, x0);
+    uint16_t* out = dst + r * Kl + g * 4 * NW;
+    if (g + 1 < groups) {
+      T x1[M];
+      load_group<M, T>(src + r * ld + (g + 1) * M, x1);
+      uint2 v[2 * NW];
 #pragma unroll
-    for (int w = 0; w < NW; ++w) {
-      uint2 v;
-      v.x = static_cast<uint32_t>(to_bf16_bits(x[2 * w])) |
-            (static_cast<uint32_t>(to_bf16_bits(x[2 * w + 1])) << 16);
-      v.y = static_cast<uint32_t>(to_bf16_bits(x[2 * w + 2])) |
-            (static_cast<uint32_t>(to_bf16_bits(x[2 * w + 3])) << 16);
-      out[w] = v;
+      for (int w = 0; w < NW; ++w) { v[w] = lift_window<M, T>(x0, w); v[NW + w] = lift_window<M, T>(x1, w); }
+      uint4* o = reinterpret_cast<uint4*>(out);
+#pragma unroll
+      for (int q = 0; q < NW; ++q) o[q] = make_uint4(v[2 * q].x, v[2 * q].y, v[2 * q + 1].x, v[2 * q + 1].y);
+    } else {
+      uint2* o = reinterpret_cast<uint2*>(out);
+#pragma unroll
+      for (int w = 0; w < NW; ++w) o[w] = lift_window<M, T>(x0, w);
     }
   }
 }
@@ -411,6 +465,7 @@ k_lift(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
 // bf16 value is exact in fp64, so fused and unfused updates agree).
 __global__ void k_colnorm_f64(const uint16_t* __restrict__ w, int64_t O, int64_t K,
                               double* __restrict__ colnorm) {
+  griddep_wait();
   const int64_t c = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (c >= K) return;
   double s = 0.0;
@@ -425,6 +480,7 @@ __global__ void k_colnorm_f64(const uint16_t* __restrict__ w, int64_t O, int64_t
 // energy and lower index).
 __global__ void k_hybrid_rank(const double* __restrict__ colnorm, int64_t K, int64_t D,
                               uint8_t* __restrict__ is_dense) {
+  griddep_wait();
   const int64_t c = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (c >= K) return;
   const double e = colnorm[c];
@@ -439,6 +495,7 @@ __global__ void k_hybrid_rank(const double* __restrict__ colnorm, int64_t K, int
 // perm = [sparse columns ascending | dense columns ascending].
 __global__ void k_hybrid_perm(const uint8_t* __restrict__ is_dense, int64_t K, int64_t D,
                               int32_t* __restrict__ perm) {
+  griddep_wait();
   const int64_t c = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   if (c >= K) return;
   const uint8_t mine = is_dense[c];
@@ -453,6 +510,7 @@ __global__ void k_gather_cols(const uint16_t* __restrict__ src, int64_t rows, in
                               uint16_t* __restrict__ dst_lo, uint16_t* __restrict__ dst_hi) {
   const int64_t total = rows * K;
   griddep_launch_dependents();
+  griddep_wait();
   for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t r = t / K, i = t % K;
