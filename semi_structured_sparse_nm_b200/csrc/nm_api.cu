@@ -213,22 +213,32 @@ int resident_pairs() {
 template <int BN, int NACC, int MSUB>
 int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   using Cfg = nm::Gemm2Cfg<BN, NACC, MSUB>;
-  CUtensorMap ta, tb, te, ty;
+  CUtensorMap ta, tb, te, ty, tad;
   int rc;
   const int64_t kb = ceil_div(p.ks_lift, 128);
+  const int64_t kb_dense = ceil_div(p.kd, 64);
   const bool tma_store = !p.out_fp32 && !p.transpose && (p.ldy % 8) == 0 &&
                          (reinterpret_cast<uintptr_t>(p.y) & 15u) == 0;
   if (tma_store) {
     if ((rc = make_tmap(&ty, p.y, p.rows_b, p.rows_a, p.ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) != NM_OK)
       return rc;
   }
-  if ((rc = make_tmap(&ta, p.a_s, p.ks_lift / 2, p.rows_a, p.ks_lift, 64, 128)) != NM_OK) return rc;
-  if ((rc = make_tmap(&tb, p.b, p.ks_lift, p.rows_b, p.ks_lift * 2, 64, BN / 2)) != NM_OK) return rc;
-  if ((rc = make_tmap_meta(&te, p.meta, ceil_div(p.rows_a, 128) * kb * 128)) != NM_OK) return rc;
+  if (kb > 0) {
+    if ((rc = make_tmap(&ta, p.a_s, p.ks_lift / 2, p.rows_a, p.ks_lift, 64, 128)) != NM_OK) return rc;
+    if ((rc = make_tmap_meta(&te, p.meta, ceil_div(p.rows_a, 128) * kb * 128)) != NM_OK) return rc;
+  }
+  if (kb_dense > 0) {
+    if ((rc = make_tmap(&tad, p.a_d, p.kd, p.rows_a, p.kd * 2, 64, 128)) != NM_OK) return rc;
+  }
+  if (kb == 0) { ta = tad; te = tad; }
+  if (kb_dense == 0) tad = ta;
+  if ((rc = make_tmap(&tb, p.b, p.ks_lift + p.kd, p.rows_b, (p.ks_lift + p.kd) * 2, 64, BN / 2)) != NM_OK) return rc;
   nm::Gemm2Args a{};
   a.rows_a = p.rows_a;
   a.rows_b = p.rows_b;
   a.kb = static_cast<int>(kb);
+  a.kb_dense = static_cast<int>(kb_dense);
+  a.k_dense_x0 = p.ks_lift;
   a.meta_kb = kb;
   a.tiles_m = static_cast<int>(ceil_div(p.rows_a, 256 * MSUB));
   a.tiles_n = static_cast<int>(ceil_div(p.rows_b, BN));
@@ -260,7 +270,7 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta, tb, te, ty, a));
+  NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta, tb, te, ty, tad, a));
   NM_CUDA_TRY(cudaGetLastError());
   return NM_OK;
 }
@@ -296,7 +306,7 @@ int pick_splits(int64_t tiles, int64_t kb_total) {
 int run_gemm(const GemmPlan& p, cudaStream_t st) {
   const char* env = std::getenv("NMSPARSE_GEMM");
   const std::string mode = env != nullptr ? env : "auto";
-  const bool eligible2 = p.kd == 0 && p.ks_lift > 0 && p.rows_a % 256 == 0;
+  const bool eligible2 = (p.ks_lift + p.kd) > 0 && p.rows_a % 256 == 0 && (p.kd == 0 || p.ks_lift % 128 == 0);
   const bool eligible4 = eligible2 && p.rows_a % 512 == 0;
   if (eligible2 && mode != "1cta") {
     if (mode == "2cta224") return launch_gemm_2cta<224, 2, 1>(p, st);
@@ -305,6 +315,9 @@ int run_gemm(const GemmPlan& p, cudaStream_t st) {
     if (mode == "2cta128") return launch_gemm_2cta<128, 2, 1>(p, st);
     if (eligible4 && mode == "2cta224x2") return launch_gemm_2cta<224, 1, 2>(p, st);
     if (eligible4 && mode == "2cta160x2") return launch_gemm_2cta<160, 1, 2>(p, st);
+    // products with dense k-blocks (hybrid, dense comparator) on SM pairs
+    if (p.kd > 0 && p.rows_b >= 512) return launch_gemm_2cta<224, 2, 1>(p, st);
+    if (p.kd > 0 && p.rows_b >= 64) return launch_gemm_2cta<128, 2, 1>(p, st);
     if (p.rows_b >= 512 && p.ks_lift >= 512) {
       // Both 2:4 operands stream through shared memory, whose port bounds this
       // kernel well before the tensor pipe does; measured on B200, the 224-wide

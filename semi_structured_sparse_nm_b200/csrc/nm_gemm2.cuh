@@ -94,9 +94,21 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+__device__ __forceinline__ void tc_mma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 struct Gemm2Args {
   int64_t rows_a, rows_b;
-  int kb;                 // sparse k-blocks (128 lifted K each)
+  int kb;                 // sparse k-blocks (128 lifted K each), then kb_dense dense ones (64 K each)
+  int kb_dense;
+  int64_t k_dense_x0;     // B column where the dense part starts
   int64_t meta_kb;        // metadata blocks per 128-row block
   int tiles_m, tiles_n;
   void* Y;
@@ -131,7 +143,7 @@ template <int BN, int NACC, int MSUB>
 __global__ void __launch_bounds__(192, 1)
 k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
-               const Gemm2Args args) {
+               const __grid_constant__ CUtensorMap tmAd, const Gemm2Args args) {
   using Cfg = Gemm2Cfg<BN, NACC, MSUB>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw2[];
@@ -163,6 +175,7 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA); prefetch_tmap(&tmB); prefetch_tmap(&tmE);
     if (args.tma_store) prefetch_tmap(&tmY);
+    if (args.kb_dense > 0) prefetch_tmap(&tmAd);
   }
   if (warp == 1) { tmem_alloc2(tmem_slot, Cfg::kTmemCols); tmem_relinquish2(); }
   tc_fence_before();
@@ -177,16 +190,30 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     // ------------------------------------------------------------ producer
     if (elect_one()) {
       const uint32_t stage_tx = static_cast<uint32_t>(2 * (Cfg::kA + Cfg::kB + Cfg::kE));
+      const uint32_t dense_tx = static_cast<uint32_t>(2 * (MSUB * Cfg::kA1 + Cfg::kHalfN * 128));
+      const int kb_all = args.kb + args.kb_dense;
       int it = 0;
       bool ok = true;
       for (int t = cluster_id; t < tiles && ok; t += num_clusters) {
         const int tm = t % args.tiles_m, tn = t / args.tiles_m;
         const int32_t yb = tn * BN + static_cast<int32_t>(rank) * Cfg::kHalfN;
-        for (int kb = 0; kb < args.kb; ++kb, ++it) {
+        for (int kb = 0; kb < kb_all; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
           if (!mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag, kWhereProducer)) { ok = false; break; }
           const uint32_t fb = leader_addr(smem_u32(&full_bar[s]));
+          if (kb >= args.kb) {
+            // dense k-block: 64 K of A (per subtile) and of the B half
+            const int kd = kb - args.kb;
+            if (leader) mbar_arrive_expect_tx(&full_bar[s], dense_tx);
+#pragma unroll
+            for (int u = 0; u < MSUB; ++u) {
+              const int64_t rb = (static_cast<int64_t>(tm) * MSUB + u) * 2 + rank;
+              tma_load_2d_pair(&tmAd, fb, sA + s * Cfg::kA + u * Cfg::kA1, kd * 64, static_cast<int32_t>(rb * 128));
+            }
+            tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB, static_cast<int32_t>(args.k_dense_x0) + kd * 64, yb);
+            continue;
+          }
           if (leader) mbar_arrive_expect_tx(&full_bar[s], stage_tx);
 #pragma unroll
           for (int u = 0; u < MSUB; ++u) {
@@ -209,6 +236,8 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     // ------------------------------------------------------- MMA (leader)
     if (leader && elect_one()) {
       const uint32_t idesc = idesc_bf16(256, BN, true);
+      const uint32_t idesc_dn = idesc_bf16(256, BN, false);
+      const int kb_all = args.kb + args.kb_dense;
       int it = 0, lt = 0;
       bool ok = true;
       for (int t = cluster_id; t < tiles && ok; t += num_clusters, ++lt) {
@@ -217,13 +246,26 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (!mbar_wait(&tempty_bar[b], (use & 1u) ^ 1u, abort_flag, kWhereMma)) break;
         tc_fence_after();
         const uint32_t acc = tmem_base + b * MSUB * Cfg::kAccStride;
-        for (int kb = 0; kb < args.kb; ++kb, ++it) {
+        for (int kb = 0; kb < kb_all; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
           if (!mbar_wait(&full_bar[s], ph, abort_flag, kWhereMma)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * Cfg::kA);
           const uint32_t b0 = smem_u32(sB + s * Cfg::kB);
+          if (kb >= args.kb) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t bd = desc_sw128_kmajor(b0 + 32u * kk);
+#pragma unroll
+              for (int u = 0; u < MSUB; ++u) {
+                const uint64_t ad = desc_sw128_kmajor(a0 + u * Cfg::kA1 + 32u * kk);
+                tc_mma_pair(acc + u * Cfg::kAccStride, ad, bd, idesc_dn, (kb > 0 || kk > 0) ? 1u : 0u);
+              }
+            }
+            tc_commit_pair(&empty_bar[s]);
+            continue;
+          }
           const uint32_t e_col = tmem_meta + 4u * MSUB * s;
 #pragma unroll
           for (int u = 0; u < MSUB; ++u)

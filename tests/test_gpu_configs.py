@@ -1,0 +1,83 @@
+"""Every workload at its full size, through the same calls and launch
+configuration bench.py times, checked against the oracle: the compressed
+operand bit-exact on whole 128-row blocks, and output rows the oracle computes
+one by one within the stated tolerance."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from semi_structured_sparse_nm_b200 import _lib as nm
+from semi_structured_sparse_nm_b200 import inputs
+from tests.gpu_util import check_close, dev, host_bits, host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_block(comp, src, N, M, rb):
+    """Rows [128 rb, 128 rb + 128) of the compressed operand vs the oracle."""
+    rows = src.shape[0]
+    r0, r1 = 128 * rb, min(128 * rb + 128, rows)
+    ref = oracle.sparse_operand(np.ascontiguousarray(src[r0:r1]), N, M)
+    np.testing.assert_array_equal(host_bits(comp.vals[r0:r1]), ref["vals"], err_msg=f"values, block {rb}")
+    KB = -(-ref["K_lift"] // 128)
+    img = host_bits(comp.meta)[rb * KB * 2048:(rb + 1) * KB * 2048]
+    np.testing.assert_array_equal(img, ref["meta"], err_msg=f"metadata image, block {rb}")
+
+
+SAMPLE = np.array([0, 1, 127, 128, 1000, 1023, 2047])
+
+
+@pytest.mark.parametrize("name", ["up_proj_8of16_act", "up_proj_2of4_act", "down_proj_16of32_act"])
+def test_activation_sparse_full_size(name):
+    wl, x, w = inputs.make_workload(name)
+    comp = nm.prune_compress(dev(x), wl.N, wl.M)
+    y = nm.sparse_gemm(comp, nm.lift(dev(w), wl.M), nm.NM_ACT, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    for rb in (0, wl.T // 128 - 1):
+        _check_block(comp, x, wl.N, wl.M, rb)
+    rows = SAMPLE[SAMPLE < wl.T]
+    check_close(host_f64(y[torch.from_numpy(rows).cuda()]), oracle.act_sparse_linear(x, w, wl.N, wl.M, rows=rows),
+                name)
+
+
+@pytest.mark.parametrize("name", ["slide_6of8_wt_prefill", "slide_6of8_wt_decode"])
+def test_weight_sparse_full_size(name):
+    wl, x, w = inputs.make_workload(name)
+    comp = nm.slide_decompose(dev(w), wl.N, wl.M)
+    y = nm.sparse_gemm(comp, nm.lift(dev(x), wl.M), nm.NM_WEIGHT, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    for rb in (0, wl.O // 128 - 1):
+        _check_block(comp, w, wl.N, wl.M, rb)
+    rows = SAMPLE[SAMPLE < wl.T]
+    check_close(host_f64(y[torch.from_numpy(rows).cuda()]), oracle.weight_sparse_linear(x, w, wl.N, wl.M, rows=rows),
+                name)
+
+
+@pytest.mark.parametrize("B", [1, 8, 32, 128])
+def test_hybrid_decode_full_size(B):
+    wl, x, w = inputs.make_workload(f"hybrid_decode_b{B}")
+    h = nm.hybrid_prepare(dev(w), wl.dense_frac)
+    y = nm.hybrid_gemm(dev(x), h, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    ref = oracle.hybrid_weight(w, wl.dense_frac)
+    np.testing.assert_array_equal(h.perm.cpu().numpy(), ref["perm"])
+    np.testing.assert_array_equal(host_bits(h.W_d), ref["W_d"])
+    np.testing.assert_array_equal(host_bits(h.vals_s), ref["vals_s"])
+    np.testing.assert_array_equal(host_bits(h.meta_s)[:ref["meta_s"].size], ref["meta_s"])
+    check_close(host_f64(y), oracle.linear_f64(oracle.to_f64(x), oracle.to_f64(w, ref["keep_full"])),
+                f"hybrid b{B}")
+
+
+def test_tiny_fp32_full_size():
+    wl, x, w = inputs.make_workload("tiny_2of4_act_fp32")
+    comp = nm.prune_compress(dev(x), wl.N, wl.M, with_mask=True)
+    y = nm.sparse_gemm(comp, nm.lift(dev(w), wl.M), nm.NM_ACT, torch.float32)
+    torch.cuda.synchronize()
+    ref = oracle.sparse_operand(x, wl.N, wl.M)
+    np.testing.assert_array_equal(host_bits(comp.mask), ref["mask"])
+    np.testing.assert_array_equal(host_bits(comp.vals), ref["vals"])
+    check_close(host_f64(y), oracle.act_sparse_linear(x, w, wl.N, wl.M), "tiny")

@@ -84,3 +84,37 @@ def test_partial_last_k_block(monkeypatch):
     y = _act(x, w, 6, 8, torch.float32)
     torch.cuda.synchronize()
     np.testing.assert_array_equal(host_f64(y), oracle.act_sparse_linear(x, w, 6, 8))
+
+
+@pytest.mark.parametrize("B", [64, 128, 200])
+def test_hybrid_on_sm_pairs(B):
+    """Hybrid input-split with sparse and dense k-blocks in the 2-CTA kernel
+    (weight rows a multiple of 256, 64 or more tokens): exact on integers."""
+    rng = np.random.default_rng(B)
+    O, K = 512, 1024
+    w = _int_bf16(rng, (O, K))
+    x = _int_bf16(rng, (B, K))
+    h = nm.hybrid_prepare(dev(w), 0.25)
+    y = nm.hybrid_gemm(dev(x), h, torch.float32)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host_f64(y), oracle.hybrid_linear(x, w, 0.25))
+
+
+def test_hybrid_on_sm_pairs_random_bf16():
+    O, K, B = 1024, 2048, 128
+    w = inputs.normal_bf16((O, K), 0.02, seed=3)
+    x = inputs.normal_bf16((B, K), 1.0, seed=4)
+    h = nm.hybrid_prepare(dev(w), 0.25)
+    y = nm.hybrid_gemm(dev(x), h, torch.bfloat16)
+    torch.cuda.synchronize()
+    check_close(host_f64(y), oracle.hybrid_linear(x, w, 0.25), "hybrid pairs")
+
+
+@pytest.mark.parametrize("rows_b", [96, 700])
+def test_dense_comparator_on_sm_pairs(rows_b):
+    rng = np.random.default_rng(rows_b)
+    a = _int_bf16(rng, (512, 640))
+    b = _int_bf16(rng, (rows_b, 640))
+    y = nm.dense_gemm(dev(a), dev(b), torch.float32)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host_f64(y), oracle.linear_f64(oracle.to_f64(a), oracle.to_f64(b)))
