@@ -359,6 +359,32 @@ class _Null:
         return False
 
 
+def time_dense(wk, reps=10):
+    """In-run dense comparators for a prefill workload: the same unpruned
+    product Y = X . W^T on this library's dense tcgen05 kernel, and on cuBLAS
+    (torch.matmul) as library context.  Returns (ours_ms, cublas_ms)."""
+    import torch
+    wl = wk.wl
+    dev = wk.dev
+    X = torch.from_numpy(wk.x_np).view(torch.bfloat16).to(dev)
+    W = torch.from_numpy(wk.w_np).view(torch.bfloat16).to(dev)
+    Y = torch.empty((wl.T, wl.O), dtype=torch.bfloat16, device=dev)
+    out = []
+    for fn in (lambda: wk.nm.dense_gemm(X, W, torch.bfloat16, out=Y), lambda: torch.matmul(X, W.t(), out=Y)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        out.append(e0.elapsed_time(e1) / reps)
+    del X, W, Y
+    return out[0], out[1]
+
+
 def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None):
     dense, mma, byts = wk.algorithmic()
     wl = wk.wl
@@ -369,6 +395,13 @@ def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None):
                    "K_lift": wl.K_lift, "rotated_buffers": wk.R},
         "kernels": {f"{wk.prep_name}_us": prep_ms * 1e3, f"{wk.gemm_name}_us": gemm_ms * 1e3},
     }
+    if not wk.decode and wl.x_dtype == "bf16":
+        ours, cublas = time_dense(wk)
+        out["dense_comparator"] = {
+            "ours_us": ours * 1e3, "cublas_us": cublas * 1e3,
+            "sparse_gemm_speedup_vs_ours": ours / gemm_ms, "step_speedup_vs_ours": ours / step_ms,
+            "sparse_gemm_speedup_vs_cublas": cublas / gemm_ms,
+            "note": "same unpruned product X . W^T, bf16, fp32 accumulate; cuBLAS is context only"}
     if wk.decode:
         achieved = byts / (gemm_ms * 1e-3) / 1e9
         out["roofline"] = {"bound": "hbm", "kernel": wk.gemm_name, "achieved": achieved, "peak": pk["hbm"],
@@ -461,6 +494,7 @@ def run_gpu(args):
         "tokens_per_s": main["tokens_per_s"],
         "kernels": main["kernels"],
         "roofline": main["roofline"],
+        "dense_comparator": main.get("dense_comparator"),
         "e2e": {"value": ws * dense / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
                 "d2h_bytes_per_step": int(yh.numel() * yh.element_size())},
