@@ -347,7 +347,7 @@ int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M
   const int64_t Kl = nm_lifted_k(K, M);
   const int64_t KB = ceil_div(Kl, 128);
   const int64_t rows_pad = ceil_div(rows, 128) * 128;
-  const int64_t tasks = (rows_pad / 16) * ceil_div(K / M, 32);
+  const int64_t tasks = (rows_pad / 16) * ceil_div(K / M, 32 * nm::prune_groups_per_lane(M, sizeof(T)));
   const int64_t per_sm = M >= 32 ? 2 : 3;           // resident CTAs per SM (registers)
   const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(tasks, int64_t(num_sms()) * per_sm));
   const dim3 grid(static_cast<unsigned>(blocks)), block(nm::kPruneWarps * 32);

@@ -163,9 +163,9 @@ __device__ __forceinline__ Key nth_largest(const Key (&key)[M], int N) {
 #pragma unroll
   for (int i = 0; i < M; ++i) srt[i] = key[i];
   bitonic_desc<M, Key>(srt);
-  Key thr = srt[0];
+  Key thr = srt[0];                          // srt[N-1]: the minimum of the first N, others masked to ~0
 #pragma unroll
-  for (int k = 1; k < M; ++k) thr = (N > k) ? srt[k] : thr;     // srt[N-1], kept in registers
+  for (int k = 1; k < M; ++k) thr = kmin(thr, srt[k] | static_cast<Key>(static_cast<int64_t>(N - 1 - k) >> 63));
   return thr;
 }
 
@@ -237,6 +237,78 @@ __device__ __forceinline__ uint2 window_entry(uint32_t c) {
   return make_uint2(sel | (zsel << 16), static_cast<uint32_t>(i0 | (i1 << 2)) | ((taken >> 2) << 4));
 }
 
+// Two 16-bit lanes per 32-bit word: one instruction does two comparators.
+__device__ __forceinline__ uint32_t vmax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t vmin2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t swap16(uint32_t a) { return __byte_perm(a, 0u, 0x1032); }
+
+// Sorts the low lanes and the high lanes of H words, each descending, with
+// one odd-even merge network.
+template <int H>
+__device__ __forceinline__ void oddeven_desc_x2(uint32_t (&a)[H]) {
+  constexpr OddEvenNet<H> net{};
+#pragma unroll
+  for (int c = 0; c < net.n; ++c) {
+    const uint32_t x = a[net.lo[c]], y = a[net.hi[c]];
+    a[net.lo[c]] = vmax2(x, y);
+    a[net.hi[c]] = vmin2(x, y);
+  }
+}
+
+// Bit i (element i of the group) set iff lane value >= t, from words
+// Q[p] = (|x[2p]|, |x[2p+1]|) of 15-bit magnitudes and C = (0x8000 - t) in
+// both lanes: a lane of Q[p] + C never carries out, and its bit 15 is set iff
+// the magnitude is at least t.
+template <int H>
+__device__ __forceinline__ uint32_t lane_ge_bits(const uint32_t (&Q)[H], uint32_t C) {
+  uint32_t acc0 = 0u, acc1 = 0u;
+#pragma unroll
+  for (int p = 0; p < H; ++p) {
+    const uint32_t e = Q[p] + C;
+    const int q = p % 8;
+    const uint32_t b = (e >> (15 - 2 * q)) & (0x00010001u << (2 * q));
+    if (p < 8) acc0 |= b; else acc1 |= b;
+  }
+  uint32_t m = (acc0 & 0x5555u) | (acc0 >> 15);
+  if constexpr (H > 8) m |= ((acc1 & 0x5555u) | (acc1 >> 15)) << 16;
+  return m;
+}
+
+// Keep bits for N = M/2: the M/2 largest magnitudes, ties to the lower index.
+// The even entries (low lanes) and the odd entries (high lanes) are sorted
+// together; the M/2 largest of their union are max(a_i, b_{M/2-1-i}), whose
+// minimum is the threshold t.  Entries above t are kept; entries equal to t
+// fill the remaining places in index order.
+template <int M>
+__device__ __forceinline__ uint32_t half_keep_bf16(const uint32_t (&P)[M / 2]) {
+  constexpr int H = M / 2;
+  uint32_t Q[H], S[H];
+#pragma unroll
+  for (int p = 0; p < H; ++p) { Q[p] = P[p] & 0x7FFF7FFFu; S[p] = Q[p]; }
+  oddeven_desc_x2<H>(S);
+  uint32_t z = vmax2(S[0], swap16(S[H - 1]));
+#pragma unroll
+  for (int i = 1; i < H / 2; ++i) z = vmin2(z, vmax2(S[i], swap16(S[H - 1 - i])));
+  const uint32_t t2 = vmin2(z, swap16(z));                // t in both lanes
+  uint32_t keep = lane_ge_bits<H>(Q, 0x80008000u - t2);
+  if (__popc(keep) != H) {                                // ties at t
+    const uint32_t gt = lane_ge_bits<H>(Q, 0x80008000u - t2 - 0x00010001u);
+    uint32_t eq = keep & ~gt;
+    const int need = H - __popc(gt);
+    while (__popc(eq) > need) eq &= ~(0x80000000u >> __clz(eq));
+    keep = gt | eq;
+  }
+  return keep;
+}
+
 // bf16 groups held as 32-bit pair words P[p] = (x[2p], x[2p+1]): unique keys
 // are formed on the fly, kept entries are those whose key is at least the N-th
 // largest (sign of thr - 1 - key), windows come from the table.
@@ -252,33 +324,19 @@ __device__ __forceinline__ uint32_t compress_group_bf16(const uint32_t (&P)[M / 
                                                         uint32_t* val_out, uint8_t* nib_out) {
   constexpr int NW = M / 2 - 1;
   uint32_t keep = 0u;
-  if (N > 0) {
-    uint32_t key[M];
+  if (2 * N == M) {
+    keep = half_keep_bf16<M>(P);
+  } else if (N > 0) {
+    uint32_t srt[M];
 #pragma unroll
-    for (int i = 0; i < M; ++i) key[i] = ukey_bf16<M>(P, i);
-    uint32_t thr;
-    if (2 * N == M) {
-      constexpr int H = M / 2;
-      uint32_t a[H], b[H];
+    for (int i = 0; i < M; ++i) srt[i] = ukey_bf16<M>(P, i);
+    oddeven_desc<M, uint32_t>(srt);
+    uint32_t thr = srt[0];                      // srt[N-1]: the minimum of the first N, others masked to ~0
 #pragma unroll
-      for (int i = 0; i < H; ++i) { a[i] = key[i]; b[i] = key[H + i]; }
-      oddeven_desc<H, uint32_t>(a);
-      oddeven_desc<H, uint32_t>(b);
-      thr = kmax(a[0], b[H - 1]);
-#pragma unroll
-      for (int i = 1; i < H; ++i) thr = kmin(thr, kmax(a[i], b[H - 1 - i]));
-    } else {
-      uint32_t srt[M];
-#pragma unroll
-      for (int i = 0; i < M; ++i) srt[i] = key[i];
-      oddeven_desc<M, uint32_t>(srt);
-      thr = srt[0];
-#pragma unroll
-      for (int k = 1; k < M; ++k) thr = (N > k) ? srt[k] : thr;
-    }
+    for (int k = 1; k < M; ++k) thr = kmin(thr, srt[k] | static_cast<uint32_t>((N - 1 - k) >> 31));
     const uint32_t t1 = thr - 1u;
 #pragma unroll
-    for (int i = 0; i < M; ++i) keep |= ((t1 - key[i]) >> 31) << i;
+    for (int i = 0; i < M; ++i) keep |= ((t1 - ukey_bf16<M>(P, i)) >> 31) << i;
   }
   uint32_t carry = 0u;
 #pragma unroll
@@ -293,10 +351,38 @@ __device__ __forceinline__ uint32_t compress_group_bf16(const uint32_t (&P)[M / 
   return keep;
 }
 
-// One CTA task = 16 consecutive rows x 32 consecutive groups; warp w takes
-// rows 2w and 2w+1 (both loads in flight together), lane = group.  32 groups
-// hold 32*NW windows, exactly NW metadata blocks of 32 windows, and 16 rows
-// are one contiguous 256-byte run inside a block (lanes 16j..16j+15 of the
+// Groups per lane: a bf16 lane takes at least 16 elements (two 16-byte
+// loads), so that small groups (M = 4, 8) do not make the CTA task tiny.
+__host__ __device__ constexpr int prune_groups_per_lane(int M, int elem_bytes) { return (elem_bytes == 2 && M < 16) ? 16 / M : 1; }
+
+// Loads the G groups of one lane; a lane that runs past the end of the row
+// (only the last lane of a row whose group count is not a multiple of G)
+// loads its valid groups one by one and zeroes the rest.
+template <int M, int G, typename T>
+__device__ __forceinline__ void load_lane(const T* __restrict__ p, int64_t nvalid, GroupRaw<M * G, T>& g) {
+  if (nvalid >= G) { load_raw<M * G, T>(p, g); return; }
+  if constexpr (G > 1) {
+#pragma unroll
+    for (int i = 0; i < GroupRaw<M * G, T>::NV; ++i) g.v[i] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int j = 0; j < G; ++j) {
+      if (j < nvalid) {
+        if constexpr (M == 8) {
+          g.v[j] = __ldg(reinterpret_cast<const uint4*>(p) + j);
+        } else {
+          const uint2 u = __ldg(reinterpret_cast<const uint2*>(p) + j);
+          if (j % 2 == 0) { g.v[j / 2].x = u.x; g.v[j / 2].y = u.y; }
+          else { g.v[j / 2].z = u.x; g.v[j / 2].w = u.y; }
+        }
+      }
+    }
+  }
+}
+
+// One CTA task = 16 consecutive rows x 32 lanes of G consecutive groups; warp
+// w takes rows 2w and 2w+1 (both loads in flight together).  A task row holds
+// 32*G*NW windows, exactly G*NW metadata blocks of 32 windows, and 16 rows are
+// one contiguous 256-byte run inside a block (lanes 16j..16j+15 of the
 // tensor-memory image), so the CTA writes its metadata as whole 16-byte lane
 // rows.  Per row: pruned (entry kept iff fewer than N entries beat it), split
 // over windows (window w takes the lowest two not yet placed kept entries of
@@ -311,34 +397,37 @@ __global__ void __launch_bounds__(kPruneWarps * 32)
 k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int N,
                  uint32_t* __restrict__ mask_out, uint32_t* __restrict__ vals_out,
                  uint8_t* __restrict__ meta_out, int64_t Kl, int64_t KB, int64_t rows_pad) {
+  constexpr int G = prune_groups_per_lane(M, static_cast<int>(sizeof(T)));
   constexpr int NW = M / 2 - 1;                   // windows per group
-  constexpr int WIN = 32 * NW;                    // windows per task row = NW blocks
+  constexpr int NWL = G * NW;                     // windows per lane
+  constexpr int WIN = 32 * NWL;                   // windows per task row = NWL blocks
+  constexpr int LM = G * M;                       // elements (keep bits) per lane
   __shared__ __align__(16) uint8_t s_nib[16][WIN];
   __shared__ __align__(16) uint32_t s_val[kPruneWarps][WIN];
-  __shared__ uint32_t s_mask[kPruneWarps][M];
+  __shared__ uint32_t s_mask[kPruneWarps][LM];
   __shared__ uint2 s_lut[16];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   griddep_launch_dependents();
   if (threadIdx.x < 16) s_lut[threadIdx.x] = window_entry(threadIdx.x);
   griddep_wait();                                      // inputs / outputs of the preceding kernel
   const int64_t groups = K / M;
-  const int64_t cpr = (groups + 31) / 32;
+  const int64_t cpr = (groups + 32 * G - 1) / (32 * G);
   const int64_t mask_words = (K + 31) / 32;
   const int64_t tasks = (rows_pad / 16) * cpr;
   const bool vec_vals = (Kl % 16) == 0;
 
   for (int64_t task = blockIdx.x; task < tasks; task += gridDim.x) {
     const int64_t rg = task / cpr, ch = task % cpr;
-    const int64_t g0 = ch * 32, g = g0 + lane;
-    const int ng = static_cast<int>((groups - g0) < 32 ? (groups - g0) : 32);
+    const int64_t g0 = ch * 32 * G, gl = g0 + static_cast<int64_t>(lane) * G;
+    const int ng = static_cast<int>((groups - g0) < 32 * G ? (groups - g0) : 32 * G);
     const int64_t r0 = rg * 16;
     for (int i = threadIdx.x; i < 16 * WIN / 4; i += blockDim.x)
       reinterpret_cast<uint32_t*>(&s_nib[0][0])[i] = 0x04040404u;
-    GroupRaw<M, T> raw[2];
+    GroupRaw<LM, T> raw[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int64_t r = r0 + 2 * warp + k;
-      if (r < rows && g < groups) load_raw<M, T>(src + r * ld + g * M, raw[k]);
+      if (r < rows && gl < groups) load_lane<M, G, T>(src + r * ld + gl * M, groups - gl, raw[k]);
     }
     __syncthreads();                                   // padding in place before any row writes
 #pragma unroll
@@ -346,55 +435,68 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
       const int it = 2 * warp + k;
       const int64_t r = r0 + it;
       if (r >= rows) break;
-      if (lane < M) s_mask[warp][lane] = 0u;
+      if (lane < LM) s_mask[warp][lane] = 0u;
       __syncwarp();
-      if (g < groups) {
-        uint32_t vals[NW];
-        uint8_t nibs[NW];
-        uint32_t keep;
+      if (gl < groups) {
+        uint32_t vals[NWL];
+        uint8_t nibs[NWL];
+        uint32_t keep = 0u;
         if constexpr (sizeof(T) == 2) {
-          uint32_t P[M / 2];
+          uint32_t PL[LM / 2];
 #pragma unroll
-          for (int p = 0; p < M / 2; ++p) {
+          for (int p = 0; p < LM / 2; ++p) {
             const uint4& q = raw[k].v[p / 4];
-            P[p] = (p % 4 == 0) ? q.x : (p % 4 == 1) ? q.y : (p % 4 == 2) ? q.z : q.w;
+            PL[p] = (p % 4 == 0) ? q.x : (p % 4 == 1) ? q.y : (p % 4 == 2) ? q.z : q.w;
           }
-          keep = compress_group_bf16<M>(P, N, s_lut, vals, nibs);
+#pragma unroll
+          for (int j = 0; j < G; ++j) {
+            uint32_t P[M / 2];
+#pragma unroll
+            for (int p = 0; p < M / 2; ++p) P[p] = PL[j * (M / 2) + p];
+            uint32_t vj[NW];
+            uint8_t nj[NW];
+            const uint32_t kj = compress_group_bf16<M>(P, N, s_lut, vj, nj);
+            const bool valid = (G == 1) || (gl + j < groups);
+#pragma unroll
+            for (int w = 0; w < NW; ++w) { vals[j * NW + w] = vj[w]; nibs[j * NW + w] = valid ? nj[w] : 0x4; }
+            if (valid) keep |= (M == 32 ? kj : (kj & ((1u << M) - 1u))) << (j * M);
+          }
         } else {
           keep = compress_group<M, T>(raw[k], N, vals, nibs);
         }
 #pragma unroll
-        for (int w = 0; w < NW; ++w) {
-          s_val[warp][lane * NW + w] = vals[w];
-          s_nib[it][lane * NW + w] = nibs[w];
+        for (int w = 0; w < NWL; ++w) {
+          s_val[warp][lane * NWL + w] = vals[w];
+          s_nib[it][lane * NWL + w] = nibs[w];
         }
         if (mask_out != nullptr)
-          atomicOr(&s_mask[warp][(lane * M) / 32], (M == 32 ? keep : (keep & ((1u << M) - 1u))) << ((lane * M) % 32));
+          atomicOr(&s_mask[warp][(lane * LM) / 32],
+                   (LM == 32 ? keep : (keep & ((1u << LM) - 1u))) << ((lane * LM) % 32));
       }
       __syncwarp();
       uint32_t* vrow = vals_out + r * (Kl / 4) + g0 * NW;
-      if (vec_vals && ng == 32) {
+      if (vec_vals && ng == 32 * G) {
         const uint4* sv = reinterpret_cast<const uint4*>(&s_val[warp][0]);
         uint4* dv = reinterpret_cast<uint4*>(vrow);
         for (int i = lane; i < WIN / 4; i += 32) dv[i] = sv[i];
       } else {
         for (int i = lane; i < ng * NW; i += 32) vrow[i] = s_val[warp][i];
       }
-      if (mask_out != nullptr && lane < M) {
-        const int64_t wi = ch * M + lane;
+      if (mask_out != nullptr && lane < LM) {
+        const int64_t wi = ch * LM + lane;
         if (wi < mask_words) mask_out[r * mask_words + wi] = s_mask[warp][lane];
       }
       __syncwarp();
     }
     __syncthreads();
-    // metadata: NW blocks x 16 lane rows of 16 bytes.  Lane row L (0..15) of
+    // metadata: NWL blocks x 16 lane rows of 16 bytes.  Lane row L (0..15) of
     // block b holds rows L%8 and L%8+8 of the 16, windows 32b + 8c + 4(L/8) + 0..3
     // in word c (low half: first row, high half: second row).
     const int64_t rb = r0 / 128;
     const int64_t sub = (r0 % 128) / 16;
-    for (int i = threadIdx.x; i < NW * 16; i += blockDim.x) {
+    for (int i = threadIdx.x; i < NWL * 16; i += blockDim.x) {
       const int b = i / 16, L = i % 16;
-      const int64_t kb = ch * NW + b;
+      const int64_t kb = ch * NWL + b;
       if (kb >= KB) continue;
       const int i8 = L % 8, h = L / 8;
       uint32_t wds[4];

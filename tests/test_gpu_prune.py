@@ -21,6 +21,13 @@ CASES = [
     (5, 64, 30, 32, "ties"),
     (128, 2048, 14, 16, "normal"),
     (3, 96, 0, 8, "normal"),
+    # rows whose group count is not a multiple of the groups one lane takes
+    (19, 72, 2, 4, "ties"),
+    (130, 520, 2, 4, "student_t"),
+    (21, 40, 4, 8, "ties"),
+    (9, 40, 6, 8, "normal"),
+    (50, 1048, 4, 8, "ties"),
+    (40, 640, 16, 32, "ties"),
 ]
 
 
