@@ -348,8 +348,11 @@ int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M
   const int64_t KB = ceil_div(Kl, 128);
   const int64_t rows_pad = ceil_div(rows, 128) * 128;
   const int64_t tasks = (rows_pad / 16) * ceil_div(K / M, 32 * nm::prune_groups_per_lane(M, sizeof(T)));
-  const int64_t per_sm = M >= 32 ? 2 : 3;           // resident CTAs per SM (registers)
-  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(tasks, int64_t(num_sms()) * per_sm));
+  // one CTA per task for bf16 groups of up to 16 (the scheduler overlaps one
+  // CTA's loads with another's compute); a persistent grid otherwise
+  const bool per_task = sizeof(T) == 2 && M < 32;
+  const int64_t per_sm = nm::prune_min_blocks(M, sizeof(T));
+  const int64_t blocks = std::max<int64_t>(1, per_task ? tasks : std::min<int64_t>(tasks, int64_t(num_sms()) * per_sm));
   const dim3 grid(static_cast<unsigned>(blocks)), block(nm::kPruneWarps * 32);
   auto v = static_cast<uint32_t*>(vals);
   auto e = static_cast<uint8_t*>(meta);

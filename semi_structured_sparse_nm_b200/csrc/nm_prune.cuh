@@ -392,8 +392,15 @@ __device__ __forceinline__ void load_lane(const T* __restrict__ p, int64_t nvali
 // of the image) and windows past K'/4 get the index pair (0, 1).
 constexpr int kPruneWarps = 8;
 
+// Resident CTAs per SM the register budget is sized for: bf16 groups of up to
+// 16 run one CTA per task, four at a time per SM; M = 32 (and fp32) CTAs are
+// larger and loop over tasks.
+__host__ __device__ constexpr int prune_min_blocks(int M, int elem_bytes) {
+  return elem_bytes != 2 ? 1 : (M >= 32 ? 2 : 4);
+}
+
 template <int M, typename T>
-__global__ void __launch_bounds__(kPruneWarps * 32)
+__global__ void __launch_bounds__(kPruneWarps * 32, prune_min_blocks(M, sizeof(T)))
 k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int N,
                  uint32_t* __restrict__ mask_out, uint32_t* __restrict__ vals_out,
                  uint8_t* __restrict__ meta_out, int64_t Kl, int64_t KB, int64_t rows_pad) {
@@ -416,8 +423,14 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
   const int64_t tasks = (rows_pad / 16) * cpr;
   const bool vec_vals = (Kl % 16) == 0;
 
+  const int64_t drg = gridDim.x / cpr, dch = gridDim.x % cpr;      // grid stride as (row group, chunk)
+  int64_t rg = blockIdx.x / cpr, ch = blockIdx.x % cpr;
   for (int64_t task = blockIdx.x; task < tasks; task += gridDim.x) {
-    const int64_t rg = task / cpr, ch = task % cpr;
+    if (task != blockIdx.x) {
+      rg += drg;
+      ch += dch;
+      if (ch >= cpr) { ch -= cpr; ++rg; }
+    }
     const int64_t g0 = ch * 32 * G, gl = g0 + static_cast<int64_t>(lane) * G;
     const int ng = static_cast<int>((groups - g0) < 32 * G ? (groups - g0) : 32 * G);
     const int64_t r0 = rg * 16;
@@ -503,11 +516,10 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const int j = 32 * b + 8 * c + 4 * h;
+        // four nibble bytes n0..n3 -> bytes 0 and 2 of x | x >> 4 hold n0 | n1 << 4 and n2 | n3 << 4
         const uint32_t lo = *reinterpret_cast<const uint32_t*>(&s_nib[i8][j]);
         const uint32_t hi = *reinterpret_cast<const uint32_t*>(&s_nib[i8 + 8][j]);
-        const uint32_t plo = (lo & 0xFu) | ((lo >> 4) & 0xF0u) | ((lo >> 8) & 0xF00u) | ((lo >> 12) & 0xF000u);
-        const uint32_t phi = (hi & 0xFu) | ((hi >> 4) & 0xF0u) | ((hi >> 8) & 0xF00u) | ((hi >> 12) & 0xF000u);
-        wds[c] = plo | (phi << 16);
+        wds[c] = __byte_perm(lo | (lo >> 4), hi | (hi >> 4), 0x6420);
       }
       *reinterpret_cast<uint4*>(meta_out + (rb * KB + kb) * 2048 + sub * 256 + L * 16) =
           make_uint4(wds[0], wds[1], wds[2], wds[3]);
