@@ -12,9 +12,13 @@
 //
 // Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and
 // MMA issuer, warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)..).
-// Split-K: the `splits` CTAs of one output tile form a thread-block cluster;
-// each keeps its fp32 partial tile in its own shared memory and the tile is
-// summed in rank order through distributed shared memory -- no global scratch.
+// Split-K: the `splits` CTAs of one output tile form a thread-block cluster
+// and the tile is summed in rank order through distributed shared memory -- no
+// global scratch.  Rank r owns rows [r*128/splits, (r+1)*128/splits).  For
+// BN <= 32 every CTA pushes its partial rows into the owner's receive buffer
+// (st.async, counted on the owner's mbarrier) and the owner sums them as soon
+// as they have landed; wider tiles keep the partial in their own ring memory
+// and are summed by distributed loads between two cluster barriers.
 #pragma once
 #include "nm_device.cuh"
 
@@ -41,6 +45,8 @@ struct GemmArgs {
 
 template <int BN>
 struct GemmCfg {
+  static constexpr bool kPush = BN <= 32;                        // push split-K reduction
+  static constexpr int kRecvBytes = kPush ? kBM * BN * 4 : 0;    // [splits][128/splits][BN] fp32
   static constexpr int kBBytes = 2 * BN * 128;
   static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
   static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
@@ -48,7 +54,7 @@ struct GemmCfg {
   static constexpr int kTmemNeed = BN + 4 * kStages;
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                  : kTmemNeed <= 256 ? 256 : 512;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kRecvBytes + 1024 /*align*/ + 256 /*barriers*/;
   static_assert(kStages >= 2, "tile too large for the shared memory ring");
   static_assert(kBM * BN * 4 <= kStages * (kABytes + kBBytes), "split-K tile must fit the ring");
 };
@@ -67,6 +73,23 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
+}
+// Split cluster barrier: arrive (release) and wait (acquire), every thread once.
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t mapa_shared_bar(const uint64_t* bar, uint32_t rank) {
+  return mapa_shared(smem_u32(bar), rank);
+}
+// Asynchronous 16-byte store into a cluster peer's shared memory; its bytes
+// complete on the peer's mbarrier.
+__device__ __forceinline__ void st_async_f32x4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                               uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+               :: "r"(addr), "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar) : "memory");
 }
 __device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t addr) {
   float4 v;
@@ -140,10 +163,12 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
   uint8_t* sA = smem;
   uint8_t* sB = sA + S * kABytes;
   uint8_t* sE = sB + S * Cfg::kBBytes;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(sE + S * kEBytes);
+  float* sRecv = reinterpret_cast<float*>(sE + S * kEBytes);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(sE + S * kEBytes + Cfg::kRecvBytes);
   uint64_t* empty_bar = full_bar + S;
   uint64_t* accum_bar = empty_bar + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accum_bar + 1);
+  uint64_t* red_bar = accum_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -153,11 +178,15 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
   const int kb_begin = static_cast<int>(static_cast<int64_t>(kb_total) * split / args.splits);
   const int kb_end = static_cast<int>(static_cast<int64_t>(kb_total) * (split + 1) / args.splits);
 
+  const bool push = Cfg::kPush && args.splits > 1;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
     mbar_init(accum_bar, 1);
+    mbar_init(red_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
+    // the owner's share of every rank's partial tile: 128 rows x BN fp32 in all
+    if (push) mbar_arrive_expect_tx(red_bar, static_cast<uint32_t>(Cfg::kRecvBytes));
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA_s); prefetch_tmap(&tmA_d); prefetch_tmap(&tmB);
@@ -169,6 +198,9 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
   const uint32_t tmem_acc = *tmem_slot;
   const uint32_t tmem_meta = tmem_acc + BN;
   griddep_launch_dependents();                       // the next kernel may begin its set-up
+  // Push split-K: the cluster's receive barriers exist before any partial is
+  // pushed (epilogue warps wait on this; the other warps before they exit).
+  if (push) cluster_arrive();
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
@@ -265,18 +297,32 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
     const bool ok = mbar_wait(accum_bar, 0u, abort_flag, kWhereEpilogue);
     griddep_wait();                                  // Y may still be in use upstream
     tc_fence_after();
+    if (push) {
+      __syncwarp();
+      cluster_wait();                                // every receive barrier of the cluster is set up
+    }
     if (ok) {
       const int64_t row_local = q * 32 + lane;
       const int64_t ra = m_tile * kBM + row_local;
       float* red = reinterpret_cast<float*>(smem);        // split-K partial tile
-      if (args.splits > 1) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      if (args.splits > 1 && !push) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       constexpr int CW = BN < 32 ? BN : 32;              // columns per TMEM load
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += CW) {
         uint32_t v[CW];
         tc_ld_32x32b<CW>(tmem_acc + (static_cast<uint32_t>(q * 32) << 16) + c0, v);
         tc_wait_ld();
-        if (args.splits == 1) {
+        if (push) {
+          // this row goes to its owner's slot for this rank
+          const int rows_per = kBM / args.splits;
+          const uint32_t owner = static_cast<uint32_t>(row_local / rows_per);
+          const uint32_t slot = cluster_ctarank() * rows_per + static_cast<uint32_t>(row_local % rows_per);
+          const uint32_t dst = mapa_shared(smem_u32(sRecv + slot * BN + c0), owner);
+          const uint32_t bar = mapa_shared_bar(red_bar, owner);
+#pragma unroll
+          for (int i = 0; i < CW / 4; ++i)
+            st_async_f32x4(dst + 16u * i, v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3], bar);
+        } else if (args.splits == 1) {
           store_row_chunk<CW>(args, ra, n_tile * BN + c0, v);
         } else {
           float4* dst = reinterpret_cast<float4*>(red + row_local * BN + c0);
@@ -287,9 +333,39 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
         }
       }
     }
+    if (push) {
+      // Sum the pushed partials of this CTA's rows in rank order, once they
+      // have all landed.
+      if (mbar_wait(red_bar, 0u, nullptr, kWhereEpilogue)) {
+        const int rows_per = kBM / args.splits;
+        const uint32_t rank = cluster_ctarank();
+        const int quads = rows_per * (BN / 4);
+        const int t = threadIdx.x - 64;
+        for (int e = t; e < quads; e += 128) {
+          const int rl = args.transpose_out ? e % rows_per : e / (BN / 4);
+          const int c = 4 * (args.transpose_out ? e / rows_per : e % (BN / 4));
+          float4 acc = *reinterpret_cast<const float4*>(sRecv + rl * BN + c);
+#pragma unroll
+          for (int p = 1; p < 8; ++p)
+            if (p < args.splits) {
+              const float4 x = *reinterpret_cast<const float4*>(sRecv + (p * rows_per + rl) * BN + c);
+              acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+            }
+          const int64_t ra = m_tile * kBM + static_cast<int64_t>(rank) * rows_per + rl, cb = n_tile * BN + c;
+          store_out(args, ra, cb, acc.x);
+          store_out(args, ra, cb + 1, acc.y);
+          store_out(args, ra, cb + 2, acc.z);
+          store_out(args, ra, cb + 3, acc.w);
+        }
+      }
+    }
+  }
+  if (push && warp < 2) {
+    __syncwarp();
+    cluster_wait();                                    // matches the set-up arrival
   }
 
-  if (args.splits > 1) {
+  if (args.splits > 1 && !push) {
     // Sum the cluster's partial tiles in rank order; rank r owns rows
     // [r*128/splits, (r+1)*128/splits) of the tile.
     __syncwarp();

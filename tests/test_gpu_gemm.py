@@ -70,6 +70,8 @@ ACT_SHAPES = [
     (256, 512, 1024, 16, 32),
     (300, 40, 192, 6, 8),      # K' = 288: a partial last k-block
     (64, 24, 256, 2, 4),       # O below one column tile
+    (128, 32, 4096, 2, 4),     # one 128 x 32 tile, split-K over a cluster of 8
+    (200, 16, 1024, 8, 16),    # split-K of 2 with a ragged row tile
 ]
 
 
@@ -90,6 +92,8 @@ WEIGHT_SHAPES = [
     (8, 256, 4096, 2, 4),
     (40, 130, 512, 14, 16),
     (300, 256, 512, 6, 8),
+    (32, 256, 2048, 6, 8),     # 32-column tiles, split-K of 4
+    (16, 1024, 4096, 6, 8),    # split-K of 8
 ]
 
 
