@@ -6,35 +6,12 @@
 
 namespace nm {
 
-// Loads M consecutive elements (16-bit or 32-bit) of one group into registers
-// with 8- or 16-byte vector loads.  The group start is 8-byte aligned for
-// M = 4 bf16, 16-byte aligned otherwise (checked by the host).
+// Splits a 32-bit word into its elements (two 16-bit or one 32-bit).
 __device__ __forceinline__ void split_word(uint32_t w, uint16_t* out) {
   out[0] = static_cast<uint16_t>(w & 0xFFFFu);
   out[1] = static_cast<uint16_t>(w >> 16);
 }
 __device__ __forceinline__ void split_word(uint32_t w, uint32_t* out) { out[0] = w; }
-
-template <int M, typename T>
-__device__ __forceinline__ void load_group(const T* __restrict__ p, T (&x)[M]) {
-  constexpr int BYTES = M * static_cast<int>(sizeof(T));
-  constexpr int PW = 4 / static_cast<int>(sizeof(T));          // elements per 32-bit word
-  if constexpr (BYTES % 16 == 0) {
-#pragma unroll
-    for (int v = 0; v < BYTES / 16; ++v) {
-      const uint4 u = __ldg(reinterpret_cast<const uint4*>(p) + v);
-      split_word(u.x, &x[v * 4 * PW + 0 * PW]);
-      split_word(u.y, &x[v * 4 * PW + 1 * PW]);
-      split_word(u.z, &x[v * 4 * PW + 2 * PW]);
-      split_word(u.w, &x[v * 4 * PW + 3 * PW]);
-    }
-  } else {
-    static_assert(BYTES == 8, "group of 8 bytes expected");
-    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
-    split_word(u.x, &x[0]);
-    split_word(u.y, &x[PW]);
-  }
-}
 
 __device__ __forceinline__ uint16_t to_bf16_bits(uint16_t b) { return b; }
 __device__ __forceinline__ uint16_t to_bf16_bits(uint32_t f) {
@@ -528,48 +505,58 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
   }
 }
 
-// Lift: dst[r][g*4(n-1) + 4w + j] = src[r][g*2n + 2w + j].  One thread per
-// pair of groups, so that the 2 * 4(n-1) lifted values (a multiple of 8) go
-// out as 16-byte stores; a row with an odd number of groups finishes its last
-// group with 8-byte stores.
-template <int M, typename T>
-__device__ __forceinline__ uint2 lift_window(const T (&x)[M], int w) {
-  uint2 v;
-  v.x = static_cast<uint32_t>(to_bf16_bits(x[2 * w])) | (static_cast<uint32_t>(to_bf16_bits(x[2 * w + 1])) << 16);
-  v.y = static_cast<uint32_t>(to_bf16_bits(x[2 * w + 2])) | (static_cast<uint32_t>(to_bf16_bits(x[2 * w + 3])) << 16);
-  return v;
+// Lift: dst[r][g*4(n-1) + 4w + j] = src[r][g*2n + 2w + j].  A CTA lifts one
+// segment of kLiftElems input elements of a row: the segment is brought into
+// shared memory (as bf16) with 16-byte loads, then each thread writes whole
+// 16-byte chunks of the lifted row -- two windows of four -- so that every
+// warp store covers 512 contiguous bytes.  Rows are taken in a grid-stride
+// loop over blockIdx.y.
+constexpr int kLiftElems = 2048;
+
+__device__ __forceinline__ void to_bf16_words(const uint4& u, uint16_t* out, const uint16_t*) {
+  *reinterpret_cast<uint4*>(out) = u;
+}
+__device__ __forceinline__ void to_bf16_words(const uint4& u, uint16_t* out, const uint32_t*) {
+  const uint32_t a = to_bf16_bits(u.x), b = to_bf16_bits(u.y), c = to_bf16_bits(u.z), d = to_bf16_bits(u.w);
+  *reinterpret_cast<uint2*>(out) = make_uint2(a | (b << 16), c | (d << 16));
 }
 
 template <int M, typename T>
 __global__ void __launch_bounds__(256)
 k_lift(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
        uint16_t* __restrict__ dst, int64_t Kl) {
-  constexpr int NW = M / 2 - 1;
-  const int64_t groups = K / M;
-  const int64_t pairs = (groups + 1) / 2;
-  const int64_t total = rows * pairs;
+  constexpr int NW = M / 2 - 1;                          // windows per group
+  constexpr int PV = 16 / static_cast<int>(sizeof(T));   // elements per 16-byte load
+  __shared__ __align__(16) uint16_t s_x[kLiftElems];
+  const uint32_t* s_w = reinterpret_cast<const uint32_t*>(s_x);
+  const int64_t e0 = static_cast<int64_t>(blockIdx.x) * kLiftElems;
+  const int n_in = static_cast<int>(K - e0 < kLiftElems ? K - e0 : kLiftElems);   // a multiple of M
+  const int nwin = n_in / M * NW;
   griddep_launch_dependents();
   griddep_wait();
-  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
-       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = t / pairs, g = 2 * (t % pairs);
-    T x0[M];
-    load_group<M, T>(src + r * ld + g * M, x0);
-    uint16_t* out = dst + r * Kl + g * 4 * NW;
-    if (g + 1 < groups) {
-      T x1[M];
-      load_group<M, T>(src + r * ld + (g + 1) * M, x1);
-      uint2 v[2 * NW];
-#pragma unroll
-      for (int w = 0; w < NW; ++w) { v[w] = lift_window<M, T>(x0, w); v[NW + w] = lift_window<M, T>(x1, w); }
-      uint4* o = reinterpret_cast<uint4*>(out);
-#pragma unroll
-      for (int q = 0; q < NW; ++q) o[q] = make_uint4(v[2 * q].x, v[2 * q].y, v[2 * q + 1].x, v[2 * q + 1].y);
-    } else {
-      uint2* o = reinterpret_cast<uint2*>(out);
-#pragma unroll
-      for (int w = 0; w < NW; ++w) o[w] = lift_window<M, T>(x0, w);
+  for (int64_t r = blockIdx.y; r < rows; r += gridDim.y) {
+    const T* row = src + r * ld + e0;
+    for (int i = threadIdx.x * PV; i < n_in; i += blockDim.x * PV) {
+      if (i + PV <= n_in) {
+        to_bf16_words(__ldg(reinterpret_cast<const uint4*>(row + i)), s_x + i, row);
+      } else if constexpr (sizeof(T) == 2) {             // a bf16 row ending in half a 16-byte word
+        *reinterpret_cast<uint2*>(s_x + i) = __ldg(reinterpret_cast<const uint2*>(row + i));
+      }
     }
+    __syncthreads();
+    uint16_t* out = dst + r * Kl + e0 / M * 4 * NW;
+    for (int c = threadIdx.x; 2 * c < nwin; c += blockDim.x) {
+      const int w0 = 2 * c, w1 = 2 * c + 1;
+      const int s0 = (w0 / NW) * M + 2 * (w0 % NW);      // even element index: a 4-byte boundary
+      const uint32_t a0 = s_w[s0 / 2], a1 = s_w[s0 / 2 + 1];
+      if (w1 < nwin) {
+        const int s1 = (w1 / NW) * M + 2 * (w1 % NW);
+        reinterpret_cast<uint4*>(out)[c] = make_uint4(a0, a1, s_w[s1 / 2], s_w[s1 / 2 + 1]);
+      } else {
+        reinterpret_cast<uint2*>(out)[2 * c] = make_uint2(a0, a1);
+      }
+    }
+    __syncthreads();                                     // s_x is refilled for the next row
   }
 }
 

@@ -79,7 +79,11 @@ def test_slide_decompose(N, M):
 
 
 @pytest.mark.parametrize("rows,K,M,dt", [(33, 256, 4, "fp32"), (100, 512, 8, "bf16"), (7, 1024, 16, "bf16"),
-                                         (64, 1024, 32, "bf16")])
+                                         (64, 1024, 32, "bf16"),
+                                         # rows of several 2048-element segments with a partial last one
+                                         (5, 4624, 8, "bf16"), (3, 6144, 16, "fp32"), (9, 2112, 32, "bf16"),
+                                         # more rows than one grid dimension holds
+                                         (70000, 16, 4, "bf16")])
 def test_lift_bit_exact(rows, K, M, dt):
     if dt == "fp32":
         x = np.random.default_rng(1).standard_normal((rows, K)).astype(np.float32)
