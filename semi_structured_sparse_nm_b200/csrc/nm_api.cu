@@ -372,11 +372,12 @@ int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M
 template <typename T>
 int launch_lift(const T* src, int64_t rows, int64_t K, int64_t ld, int M, void* dst, cudaStream_t st) {
   const int64_t Kl = nm_lifted_k(K, M);
-  // one CTA per (row, segment of nm::kLiftElems input elements); rows beyond
-  // the grid's y extent are taken in a loop
+  // one CTA per (block of nm::kLiftRows rows, segment of nm::kLiftElems input
+  // elements); row blocks beyond the grid's y extent are taken in a loop
   const int64_t segs = ceil_div(K, int64_t(nm::kLiftElems));
+  const int64_t rblocks = ceil_div(rows, int64_t(nm::kLiftRows));
   auto d = static_cast<uint16_t*>(dst);
-  const dim3 grid(static_cast<unsigned>(segs), static_cast<unsigned>(std::min<int64_t>(rows, 65535))), block(256);
+  const dim3 grid(static_cast<unsigned>(segs), static_cast<unsigned>(std::min<int64_t>(rblocks, 65535))), block(256);
   cudaError_t err;
   switch (M) {
     case 4: err = launch_pdl(nm::k_lift<4, T>, grid, block, 0, st, src, rows, K, ld, d, Kl); break;

@@ -506,12 +506,13 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
 }
 
 // Lift: dst[r][g*4(n-1) + 4w + j] = src[r][g*2n + 2w + j].  A CTA lifts one
-// segment of kLiftElems input elements of a row: the segment is brought into
-// shared memory (as bf16) with 16-byte loads, then each thread writes whole
-// 16-byte chunks of the lifted row -- two windows of four -- so that every
-// warp store covers 512 contiguous bytes.  Rows are taken in a grid-stride
-// loop over blockIdx.y.
+// segment of kLiftElems input elements of kLiftRows rows: the segments are
+// brought into shared memory (as bf16) with 16-byte loads, all in flight
+// together, then each thread writes whole 16-byte chunks of the lifted rows --
+// two windows of four -- so that every warp store covers 512 contiguous
+// bytes.  Row blocks beyond the grid's y extent are taken in a loop.
 constexpr int kLiftElems = 2048;
+constexpr int kLiftRows = 4;
 
 __device__ __forceinline__ void to_bf16_words(const uint4& u, uint16_t* out, const uint16_t*) {
   *reinterpret_cast<uint4*>(out) = u;
@@ -527,36 +528,60 @@ k_lift(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
        uint16_t* __restrict__ dst, int64_t Kl) {
   constexpr int NW = M / 2 - 1;                          // windows per group
   constexpr int PV = 16 / static_cast<int>(sizeof(T));   // elements per 16-byte load
-  __shared__ __align__(16) uint16_t s_x[kLiftElems];
-  const uint32_t* s_w = reinterpret_cast<const uint32_t*>(s_x);
+  __shared__ __align__(16) uint16_t s_x[kLiftRows][kLiftElems];
   const int64_t e0 = static_cast<int64_t>(blockIdx.x) * kLiftElems;
   const int n_in = static_cast<int>(K - e0 < kLiftElems ? K - e0 : kLiftElems);   // a multiple of M
   const int nwin = n_in / M * NW;
   griddep_launch_dependents();
   griddep_wait();
-  for (int64_t r = blockIdx.y; r < rows; r += gridDim.y) {
-    const T* row = src + r * ld + e0;
-    for (int i = threadIdx.x * PV; i < n_in; i += blockDim.x * PV) {
-      if (i + PV <= n_in) {
-        to_bf16_words(__ldg(reinterpret_cast<const uint4*>(row + i)), s_x + i, row);
-      } else if constexpr (sizeof(T) == 2) {             // a bf16 row ending in half a 16-byte word
-        *reinterpret_cast<uint2*>(s_x + i) = __ldg(reinterpret_cast<const uint2*>(row + i));
+  for (int64_t r0 = static_cast<int64_t>(blockIdx.y) * kLiftRows; r0 < rows;
+       r0 += static_cast<int64_t>(gridDim.y) * kLiftRows) {
+    const int nr = static_cast<int>(rows - r0 < kLiftRows ? rows - r0 : kLiftRows);
+    if (nr == kLiftRows && n_in == kLiftElems) {
+      // whole block: every load of the kLiftRows rows issued before any store
+      constexpr int J = kLiftElems / (256 * PV);
+      uint4 u[kLiftRows][J];
+#pragma unroll
+      for (int k = 0; k < kLiftRows; ++k)
+#pragma unroll
+        for (int j = 0; j < J; ++j)
+          u[k][j] = __ldg(reinterpret_cast<const uint4*>(src + (r0 + k) * ld + e0 + (threadIdx.x + 256 * j) * PV));
+#pragma unroll
+      for (int k = 0; k < kLiftRows; ++k)
+#pragma unroll
+        for (int j = 0; j < J; ++j) to_bf16_words(u[k][j], &s_x[k][(threadIdx.x + 256 * j) * PV], src);
+    } else {
+#pragma unroll
+    for (int k = 0; k < kLiftRows; ++k) {
+      if (k < nr) {
+        const T* row = src + (r0 + k) * ld + e0;
+        for (int i = threadIdx.x * PV; i < n_in; i += blockDim.x * PV) {
+          if (i + PV <= n_in) {
+            to_bf16_words(__ldg(reinterpret_cast<const uint4*>(row + i)), &s_x[k][i], row);
+          } else if constexpr (sizeof(T) == 2) {         // a bf16 row ending in half a 16-byte word
+            *reinterpret_cast<uint2*>(&s_x[k][i]) = __ldg(reinterpret_cast<const uint2*>(row + i));
+          }
+        }
       }
+    }
     }
     __syncthreads();
-    uint16_t* out = dst + r * Kl + e0 / M * 4 * NW;
-    for (int c = threadIdx.x; 2 * c < nwin; c += blockDim.x) {
-      const int w0 = 2 * c, w1 = 2 * c + 1;
-      const int s0 = (w0 / NW) * M + 2 * (w0 % NW);      // even element index: a 4-byte boundary
-      const uint32_t a0 = s_w[s0 / 2], a1 = s_w[s0 / 2 + 1];
-      if (w1 < nwin) {
-        const int s1 = (w1 / NW) * M + 2 * (w1 % NW);
-        reinterpret_cast<uint4*>(out)[c] = make_uint4(a0, a1, s_w[s1 / 2], s_w[s1 / 2 + 1]);
-      } else {
-        reinterpret_cast<uint2*>(out)[2 * c] = make_uint2(a0, a1);
+    for (int k = 0; k < nr; ++k) {
+      const uint32_t* s_w = reinterpret_cast<const uint32_t*>(&s_x[k][0]);
+      uint16_t* out = dst + (r0 + k) * Kl + e0 / M * 4 * NW;
+      for (int c = threadIdx.x; 2 * c < nwin; c += blockDim.x) {
+        const int w0 = 2 * c, w1 = 2 * c + 1;
+        const int s0 = (w0 / NW) * M + 2 * (w0 % NW);    // even element index: a 4-byte boundary
+        const uint32_t a0 = s_w[s0 / 2], a1 = s_w[s0 / 2 + 1];
+        if (w1 < nwin) {
+          const int s1 = (w1 / NW) * M + 2 * (w1 % NW);
+          reinterpret_cast<uint4*>(out)[c] = make_uint4(a0, a1, s_w[s1 / 2], s_w[s1 / 2 + 1]);
+        } else {
+          reinterpret_cast<uint2*>(out)[2 * c] = make_uint2(a0, a1);
+        }
       }
     }
-    __syncthreads();                                     // s_x is refilled for the next row
+    __syncthreads();                                     // s_x is refilled for the next row block
   }
 }
 
