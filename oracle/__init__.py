@@ -35,7 +35,7 @@ def build(force: bool = False) -> str:
             tmp = _LIB + f".tmp{os.getpid()}"
             subprocess.check_call([
                 "gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
-                "-Wall", "-Wextra", "-Wno-unused-parameter", _SRC, "-o", tmp,
+                "-Wall", "-Wextra", "-Wno-unused-parameter", _SRC, "-o", tmp, "-lm",
             ])
             os.replace(tmp, _LIB)
     return _LIB
@@ -64,6 +64,12 @@ def _load():
             "or_hybrid_perm": (None, [P, I64, I64, P, P]),
             "or_gather_cols_bf16": (None, [P, I64, I64, P, P]),
             "or_num_threads": (I, []),
+            "or_e4m3_to_f64": (ctypes.c_double, [ctypes.c_uint8]),
+            "or_e4m3_from_f32": (ctypes.c_uint8, [ctypes.c_float]),
+            "or_quant_rows_e4m3": (None, [P, I, I64, I64, P, P]),
+            "or_quant_vals_e4m3": (None, [P, I64, I64, P, P]),
+            "or_lift_u8": (I, [P, I64, I64, I, P]),
+            "or_meta8": (None, [P, I64, I64, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -301,3 +307,86 @@ def hybrid_linear(x: np.ndarray, w: np.ndarray, dense_frac: float, rows=None) ->
     zeroed, in the original column order (fp64)."""
     hw = hybrid_weight(w, dense_frac)
     return linear_f64(to_f64(x), to_f64(w, hw["keep_full"]), rows)
+
+
+# -------------------------------------------------------------------- fp8
+
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """Values of E4M3 codes (NaN for the two NaN codes)."""
+    L = _load()
+    table = np.array([L.or_e4m3_to_f64(c) for c in range(256)], np.float64)
+    return table[np.asarray(codes, dtype=np.uint8)]
+
+
+def e4m3_from_f32(x) -> np.ndarray:
+    """E4M3 codes of fp32 values: nearest, ties to even, saturated to +-448."""
+    L = _load()
+    x = np.asarray(x, dtype=np.float32)
+    return np.array([L.or_e4m3_from_f32(float(v)) for v in x.ravel()], np.uint8).reshape(x.shape)
+
+
+def quant_rows(x: np.ndarray):
+    """Per-row E4M3 codes and fp32 scales (scale = row amax / 448)."""
+    x = np.ascontiguousarray(x)
+    rows, K = x.shape
+    codes = np.zeros((rows, K), np.uint8)
+    scale = np.zeros(rows, np.float32)
+    _load().or_quant_rows_e4m3(_ptr(_as_bits(x)), _dt(x), rows, K, _ptr(codes), _ptr(scale))
+    return codes, scale
+
+
+def quant_vals(vals: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """Codes of compressed bf16 values, row r divided by scale[r]."""
+    vals = np.ascontiguousarray(vals, dtype=np.uint16)
+    rows, nv = vals.shape
+    codes = np.zeros((rows, nv), np.uint8)
+    _load().or_quant_vals_e4m3(_ptr(vals), rows, nv, _ptr(np.ascontiguousarray(scale, dtype=np.float32)),
+                               _ptr(codes))
+    return codes
+
+
+def lift_u8(codes: np.ndarray, M: int) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    rows, K = codes.shape
+    out = np.zeros((rows, lifted_k(K, M)), np.uint8)
+    if _load().or_lift_u8(_ptr(codes), rows, K, M, _ptr(out)) != 0:
+        raise ValueError("or_lift_u8 rejected the shape")
+    return out
+
+
+def meta8(nib: np.ndarray, Kl: int) -> np.ndarray:
+    nib = np.ascontiguousarray(nib, dtype=np.uint8)
+    rows = nib.shape[0]
+    out = np.zeros(int(_load().or_meta_hw_bytes(rows, Kl)), np.uint8)
+    _load().or_meta8(_ptr(nib), rows, Kl, _ptr(out))
+    return out
+
+
+def fp8_activation(x: np.ndarray, M: int):
+    """The quantise + lift step: per-token codes lifted for windows of M, and
+    the per-token scales."""
+    codes, scale = quant_rows(x)
+    return dict(codes=codes, lifted=lift_u8(codes, M), scale=scale)
+
+
+def fp8_weight(w: np.ndarray, N: int, M: int):
+    """The offline weight packing in 8 bits: prune, windows, per-row scale of
+    the dense row, codes of the compressed values, 8-bit metadata image."""
+    keep = prune(w, N, M)
+    vals, nib = compress(w, keep, M)
+    _, scale = quant_rows(w)
+    Kl = lifted_k(w.shape[1], M)
+    return dict(keep=keep, vals=quant_vals(vals, scale), nib=nib, meta=meta8(nib, Kl), scale=scale, K_lift=Kl)
+
+
+def fp8_weight_sparse_linear(x: np.ndarray, w: np.ndarray, N: int, M: int, rows=None) -> np.ndarray:
+    """Y[t, o] = sx[t] * sw[o] * sum_k e4m3(X)[t, k] * e4m3(prune(W))[o, k] in fp64."""
+    qx, sx = quant_rows(x)
+    qw, sw = quant_rows(w)
+    keep = prune(w, N, M)
+    xd = e4m3_to_f64(qx)
+    wd = np.where(keep.astype(bool), e4m3_to_f64(qw), 0.0)
+    Y = linear_f64(xd, wd, rows)
+    sxs = sx.astype(np.float64) if rows is None else sx.astype(np.float64)[np.asarray(rows)]
+    return Y * sxs[:, None] * sw.astype(np.float64)[None, :]

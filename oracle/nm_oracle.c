@@ -33,8 +33,16 @@
  *               [SpenseGPT, technical summary §2.A (dense region + 2:4 region,
  *                input-split with accumulation) and §2.B (permutation of the
  *                intermediate indices into one contiguous dense block)]
+ *  8. fp8       8-bit (E4M3) variant: the dense operand is quantised per row
+ *               (token) and lifted, the sparse operand's kept values are
+ *               quantised per row (output channel), the sparse metadata takes
+ *               the 8-bit image, and the product is rescaled by both scales.
+ *               [SlideSparse, technical summary §2.B (lifting fused into the
+ *                per-token quantisation of INT8/FP8 inference) and §2.C
+ *                (offline packer, online quantisation-slide kernel)]
  *
- * Readings taken where the pages are silent are listed in the design doc.
+ * Where the pages are silent the plainest reading is taken and stated beside
+ * the function that takes it.
  *
  * Parity pins: every function here is pinned by tests under tests/ against
  * invariants, brute force, closed forms or exact integer arithmetic.
@@ -42,6 +50,7 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#include <math.h>
 #ifdef _OPENMP
 #include <omp.h>
 #endif
@@ -407,6 +416,107 @@ void or_gather_cols_bf16(const uint16_t *w, int64_t rows, int64_t K, const int32
                          uint16_t *wperm) {
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t i = 0; i < K; ++i) wperm[r * K + i] = w[r * K + perm[i]];
+}
+
+/* --------------------------------------------------------- fp8 (E4M3) */
+
+/* Step 8.  E4M3 as the OCP 8-bit format defines it: 1 sign bit, 4 exponent
+ * bits with bias 7, 3 mantissa bits; exponent field 0 holds the subnormals
+ * (m/8) * 2^-6; the code S.1111.111 is NaN and there is no infinity, so the
+ * largest finite magnitude is 1.75 * 2^8 = 448. */
+double or_e4m3_to_f64(uint8_t c) {
+    const int e = (c >> 3) & 0xF, m = c & 7;
+    if (e == 0xF && m == 7) return NAN;
+    const double v = e == 0 ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return (c & 0x80) ? -v : v;
+}
+
+/* The e4m3 code nearest to the fp32 value x, ties to the even code (the
+ * code's last bit is the mantissa's last bit); magnitudes of 448 and above,
+ * infinity included, saturate to 448; NaN gives 0x7F.  The positive codes
+ * 0x00..0x7E increase with their value, so the two neighbours of |x| are
+ * found by bisection.  The sign is kept, also for results that are zero. */
+uint8_t or_e4m3_from_f32(float x) {
+    if (isnan(x)) return 0x7F;
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    const double a = fabs((double)x);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    int lo = 0, hi = 0x7E;                       /* value(lo) <= a < value(hi) */
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) / 2;
+        if (or_e4m3_to_f64((uint8_t)mid) <= a) lo = mid;
+        else hi = mid;
+    }
+    const double dlo = a - or_e4m3_to_f64((uint8_t)lo), dhi = or_e4m3_to_f64((uint8_t)hi) - a;
+    const int c = dlo < dhi ? lo : (dhi < dlo ? hi : (lo % 2 == 0 ? lo : hi));
+    return (uint8_t)(sign | c);
+}
+
+static float value_f32_at(const void *src, int dt, int64_t idx) {
+    return (float)value_at(src, dt, idx);         /* exact: bf16 and fp32 are fp32 values */
+}
+
+/* Step 8a.  Per-row (per-token) quantisation.  amax = max_k |x[r][k]|,
+ * scale = amax / 448 rounded to fp32 (1 for an all-zero row), and
+ * code = e4m3(x / scale) with the quotient rounded to fp32: the quantised
+ * code is decided from the same fp32 quotient the kernel forms.  The pages
+ * say only that activations are quantised per token; a symmetric scale that
+ * maps the row maximum to the largest code is the plainest reading. */
+void or_quant_rows_e4m3(const void *src, int dt, int64_t rows, int64_t K, uint8_t *codes, float *scale) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            const float v = fabsf(value_f32_at(src, dt, r * K + k));
+            if (v > amax) amax = v;
+        }
+        const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+        scale[r] = s;
+        for (int64_t k = 0; k < K; ++k) codes[r * K + k] = or_e4m3_from_f32(value_f32_at(src, dt, r * K + k) / s);
+    }
+}
+
+/* Step 8b.  Codes of a row's compressed values (bf16 bits) with that row's
+ * scale: code = e4m3(v / scale[r]), the quotient rounded to fp32.  Padded
+ * slots (+0.0) give the code 0x00. */
+void or_quant_vals_e4m3(const uint16_t *vals, int64_t rows, int64_t nv, const float *scale, uint8_t *codes) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t i = 0; i < nv; ++i)
+            codes[r * nv + i] = or_e4m3_from_f32((float)bf16_bits_to_double(vals[r * nv + i]) / scale[r]);
+}
+
+/* Step 5 on bytes: dst[r][g*4(n-1) + 4w + j] = src[r][g*2n + 2w + j]. */
+int or_lift_u8(const uint8_t *src, int64_t rows, int64_t K, int M, uint8_t *dst) {
+    const int64_t Kl = or_lifted_k(K, M);
+    if (Kl < 0) return -1;
+    const int n = M / 2, nw = n - 1;
+    const int64_t groups = K / M;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t g = 0; g < groups; ++g)
+            for (int w = 0; w < nw; ++w)
+                for (int j = 0; j < 4; ++j)
+                    dst[r * Kl + g * 4 * nw + 4 * w + j] = src[r * K + g * M + 2 * w + j];
+    return 0;
+}
+
+/* Step 8c.  The 8-bit sparse MMA reads its metadata as one 16-byte row per
+ * operand row and 128 lifted K: in the block of rows 128 rb .. 128 rb + 127
+ * and windows 32 kb .. 32 kb + 31, row m and window j of the block land in
+ * byte m * 16 + j / 2, low nibble for even j.  Blocks are placed as in step 4
+ * (block (rb, kb) at byte (rb * KB + kb) * 2048) and padded the same way. */
+void or_meta8(const uint8_t *nib, int64_t rows, int64_t Kl, uint8_t *meta) {
+    const int64_t RB = (rows + 127) / 128, KB = (Kl + 127) / 128;
+    const int64_t nwin = Kl / 4;
+    memset(meta, 0, (size_t)(RB * KB * 2048));
+    for (int64_t rb = 0; rb < RB; ++rb)
+        for (int64_t kb = 0; kb < KB; ++kb)
+            for (int m = 0; m < 128; ++m)
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int64_t r = rb * 128 + m, j = kb * 32 + jj;
+                    uint8_t q = 0x4;
+                    if (r < rows && j < nwin) q = nib[r * nwin + j];
+                    meta[(rb * KB + kb) * 2048 + m * 16 + jj / 2] |= (uint8_t)((q & 0xF) << (4 * (jj % 2)));
+                }
 }
 
 /* ---------------------------------------------------------------- version */

@@ -1,0 +1,125 @@
+"""The oracle's 8-bit (E4M3) step pinned to what the format and the
+mathematics fix: values of codes from the format's definition, nearest-even
+rounding at every midpoint, a library conversion routine, quantisation
+invariants, and exact products when quantisation is lossless."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from semi_structured_sparse_nm_b200 import inputs
+
+# Code -> value, from the E4M3 definition: bias 7, 3 mantissa bits, subnormals
+# (m/8) 2^-6, S.1111.111 is NaN, largest finite 1.75 * 2^8.
+DECODE = [
+    (0x00, 0.0), (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9), (0x08, 2.0 ** -6), (0x38, 1.0),
+    (0x39, 1.125), (0x3F, 1.875), (0x40, 2.0), (0x77, 240.0), (0x7E, 448.0), (0xB8, -1.0), (0xFE, -448.0),
+]
+# value -> code, nearest with ties to even, saturating
+ENCODE = [
+    (0.0, 0x00), (-0.0, 0x80), (1.0, 0x38), (448.0, 0x7E), (450.0, 0x7E), (1e9, 0x7E), (math.inf, 0x7E),
+    (-1e9, 0xFE), (2.0 ** -9, 0x01), (2.0 ** -10, 0x00), (3 * 2.0 ** -10, 0x02), (5 * 2.0 ** -10, 0x02),
+    (1.0625, 0x38), (1.1875, 0x3A), (1.0625 * (1 + 2 ** -20), 0x39), (464.0, 0x7E), (0.3, 0x2A),          # 0.3 = 1.2 * 2^-2: exponent field 5, mantissa 2 (1.25)
+]
+
+
+@pytest.mark.parametrize("code,value", DECODE)
+def test_decode_values(code, value):
+    assert oracle.e4m3_to_f64([code])[0] == value
+
+
+def test_nan_codes():
+    v = oracle.e4m3_to_f64([0x7F, 0xFF])
+    assert np.isnan(v).all()
+    assert oracle.e4m3_from_f32([np.nan])[0] == 0x7F
+
+
+@pytest.mark.parametrize("value,code", ENCODE)
+def test_encode_values(value, code):
+    assert oracle.e4m3_from_f32([value])[0] == code
+
+
+def test_round_trip_every_finite_code():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    vals = oracle.e4m3_to_f64(codes).astype(np.float32)
+    assert np.array_equal(oracle.e4m3_from_f32(vals), codes)
+
+
+def test_midpoints_round_to_even():
+    codes = np.arange(0, 0x7E, dtype=np.uint8)
+    v0 = oracle.e4m3_to_f64(codes)
+    v1 = oracle.e4m3_to_f64(codes + 1)
+    mid = ((v0 + v1) / 2).astype(np.float32)                 # at most 5 significant bits: exact
+    assert np.array_equal(mid.astype(np.float64), (v0 + v1) / 2)
+    even = np.where(codes % 2 == 0, codes, codes + 1)
+    assert np.array_equal(oracle.e4m3_from_f32(mid), even)
+    up = (mid.astype(np.float64) * (1 + 2.0 ** -20)).astype(np.float32)
+    down = (mid.astype(np.float64) * (1 - 2.0 ** -20)).astype(np.float32)
+    assert np.array_equal(oracle.e4m3_from_f32(up[1:]), (codes + 1)[1:])
+    assert np.array_equal(oracle.e4m3_from_f32(down[1:]), codes[1:])
+
+
+def test_agrees_with_library_conversion_in_range():
+    rng = np.random.default_rng(3)
+    mag = np.exp(rng.uniform(np.log(2.0 ** -12), np.log(440.0), 20000))
+    x = (mag * rng.choice([-1.0, 1.0], mag.size)).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_from_f32(x), ref)
+
+
+def test_quant_rows_invariants():
+    x = inputs.student_t_bf16((40, 512), 4.0, seed=5)
+    x[7] = 0                                                   # an all-zero row
+    codes, scale = oracle.quant_rows(x)
+    xf = inputs.bf16_to_f64(x)
+    dec = oracle.e4m3_to_f64(codes)
+    assert scale[7] == 1.0 and not codes[7].any()
+    nz = np.arange(40) != 7
+    # the row maximum maps to the largest code
+    assert np.array_equal(np.abs(dec[nz]).max(axis=1), np.full(39, 448.0))
+    assert np.array_equal(scale[nz], (np.abs(xf[nz]).max(axis=1) / 448.0).astype(np.float32))
+    # within half a step of the value (3 mantissa bits; subnormal step 2^-9)
+    err = np.abs(dec * scale[:, None].astype(np.float64) - xf)
+    bound = (2.0 ** -4) * np.abs(xf) + 2.0 ** -10 * scale[:, None].astype(np.float64) * (1 + 1e-6)
+    assert (err <= bound * (1 + 1e-6)).all()
+
+
+def test_lift_u8_is_the_lift_map():
+    codes = np.random.default_rng(1).integers(0, 256, size=(9, 96), dtype=np.uint8)
+    for M in (4, 8, 16, 32):
+        ref = oracle.lift(codes.astype(np.uint16), M).astype(np.uint8)
+        assert np.array_equal(oracle.lift_u8(codes, M), ref)
+
+
+def test_meta8_holds_each_row_nibble_stream():
+    rng = np.random.default_rng(2)
+    rows, Kl = 150, 384
+    nib = rng.choice(np.array([0x4, 0x8, 0xC, 0x9, 0xD, 0xE], np.uint8), size=(rows, Kl // 4))
+    img = oracle.meta8(nib, Kl)
+    RB, KB = 2, 3
+    halves = np.stack([img & 0xF, img >> 4], axis=-1).reshape(RB, KB, 128, 32)
+    full = np.full((RB * 128, KB * 32), 0x4, np.uint8)
+    full[:rows, :Kl // 4] = nib
+    assert np.array_equal(halves.transpose(0, 2, 1, 3).reshape(RB * 128, KB * 32), full)
+    assert (oracle.meta8(np.full((3, 32), 0x4, np.uint8), 128) == 0x44).all()
+
+
+@pytest.mark.parametrize("N,M", [(6, 8), (2, 4), (14, 16)])
+def test_fp8_product_exact_when_quantisation_is_lossless(N, M):
+    """Inputs on the E4M3 grid whose row maxima are 448 (scale 1) or 112
+    (scale 1/4, a power of two): the 8-bit product equals the plain one."""
+    rng = np.random.default_rng(N + M)
+    grid = oracle.e4m3_to_f64(np.arange(0x00, 0x77, dtype=np.uint8))    # 0 .. 240
+    for top in (448.0, 112.0):
+        def make(rows, K, seed):
+            r = np.random.default_rng(seed)
+            v = r.choice(grid, size=(rows, K)) * r.choice([-1.0, 1.0], size=(rows, K)) * (top / 448.0)
+            v[:, 0] = top
+            return inputs.bf16_from_f64(v)
+        x = make(12, 64, 1)
+        w = make(40, 64, 2)
+        y8 = oracle.fp8_weight_sparse_linear(x, w, N, M)
+        y = oracle.weight_sparse_linear(x, w, N, M)
+        assert np.array_equal(y8, y)
