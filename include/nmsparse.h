@@ -158,6 +158,57 @@ int nm_sparse_gemm(const nm_sparse_operand *S, const void *D, int64_t rows_d, nm
 int nm_dense_gemm(const void *A, int64_t rows_a, const void *B, int64_t rows_b, int64_t K,
                   void *Y, nm_dtype out_dt, void *stream);
 
+/* --------------------------------------------------------- 8-bit (E4M3) */
+
+/* The 8-bit variant of the weight-sparse path: activations quantised per
+ * token and lifted in one pass, weights packed offline with per-row scales,
+ * and the sparse product run on the 8-bit sparse tensor cores (kind::f8f6f4,
+ * E4M3 x E4M3, fp32 accumulate) with both scales applied in the epilogue.
+ * [SlideSparse, technical summary §2.B (the lifting is fused into the
+ *  per-token quantisation kernel that INT8/FP8 inference already runs) and
+ *  §2.C (offline packer, online quantisation-slide kernel).]
+ *
+ * E4M3: the OCP 8-bit format with bias 7, 3 mantissa bits, largest finite
+ * 448, no infinity.  Per row: amax = max |x|, scale = amax / 448 (fp32,
+ * correctly rounded; 1 for an all-zero row), code = E4M3(x / scale) with the
+ * quotient an fp32 division, rounded to nearest even and saturated to +-448.
+ *
+ * The 8-bit metadata image has the blocks of nm_meta_bytes() (128 rows x 128
+ * lifted columns, 2048 bytes, block (rb, kb) at (rb * ceil(K'/128) + kb) *
+ * 2048); inside a block row m and window q hold their index pair at byte
+ * 16*m + q/2, low nibble for even q.  Rows and windows past the operand carry
+ * the pair (0,1). */
+
+/* Largest source row (K times the element size) nm_quant_lift_fp8() stages. */
+#define NM_FP8_MAX_ROW_BYTES (96 * 1024)
+
+/* Quantise + lift: codes_out [rows][K'] (row stride K', E4M3 codes in the
+ * lifted order of nm_lift()), scale_out [rows] fp32.  src [rows x K], row
+ * stride ld elements, NM_BF16 or NM_FP32.  K' must be a multiple of 16 and
+ * K * element size at most NM_FP8_MAX_ROW_BYTES (else NM_ERR_UNSUPPORTED);
+ * src and codes_out 16-byte aligned, scale_out 4-byte aligned. */
+int nm_quant_lift_fp8(const void *src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, int M,
+                      uint8_t *codes_out, float *scale_out, void *stream);
+
+/* Offline weight packer, 8-bit: slide_decompose() of the bf16 weight
+ * W [rows x K] (row stride K), then per row scale = amax(W[r]) / 448 and the
+ * kept values' codes E4M3(v / scale).  vals_out [rows][K'/2] codes,
+ * scale_out [rows], meta_out the 8-bit image (nm_meta_bytes(rows, K, M)
+ * bytes).  ws: slide_decompose_fp8_workspace_size() bytes of scratch (the
+ * 16-bit windows).  K' must be a multiple of 16. */
+size_t slide_decompose_fp8_workspace_size(int64_t rows, int64_t K, int M);
+int slide_decompose_fp8(const void *w, int64_t rows, int64_t K, int N, int M, uint8_t *vals_out,
+                        float *scale_out, uint8_t *meta_out, void *ws, size_t ws_bytes, void *stream);
+
+/* Y = (S . D^T) * S_scale[row of S] * D_scale[row of D], or its transpose
+ * (side NM_WEIGHT), with S the packed 8-bit sparse operand (S->vals codes,
+ * S->meta the 8-bit image) and D the lifted codes [rows_d][S->K_lift].
+ * Requires S->K_lift % 128 == 0 and S->rows % 256 == 0 (NM_ERR_UNSUPPORTED
+ * otherwise).  The S side may be read while the preceding kernel in the
+ * stream finishes, as in nm_sparse_gemm(). */
+int nm_sparse_gemm_fp8(const nm_sparse_operand *S, const float *S_scale, const void *D, const float *D_scale,
+                       int64_t rows_d, nm_side side, void *Y, nm_dtype out_dt, void *stream);
+
 /* ----------------------------------------------------------------- hybrid */
 
 /* Dense column count for a dense share f: 4 * floor(f*K/4) (0 for f <= 0,

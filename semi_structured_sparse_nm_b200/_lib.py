@@ -59,6 +59,10 @@ def lib():
             "nm_sparse_gemm_workspace_size": (SZ, [ctypes.POINTER(SparseOperand), I64, I]),
             "nm_sparse_gemm": (I, [ctypes.POINTER(SparseOperand), P, I64, I, P, I, P, SZ, P]),
             "nm_dense_gemm": (I, [P, I64, P, I64, I64, P, I, P]),
+            "nm_quant_lift_fp8": (I, [P, I, I64, I64, I64, I, P, P, P]),
+            "slide_decompose_fp8_workspace_size": (SZ, [I64, I64, I]),
+            "slide_decompose_fp8": (I, [P, I64, I64, I, I, P, P, P, P, SZ, P]),
+            "nm_sparse_gemm_fp8": (I, [ctypes.POINTER(SparseOperand), P, P, P, I64, I, P, I, P]),
             "hybrid_dense_count": (I64, [I64, D]),
             "hybrid_prepare_workspace_size": (SZ, [I64, I64]),
             "hybrid_prepare": (I, [P, I64, I64, D, ctypes.POINTER(HybridWeight), P, SZ, P]),
@@ -208,6 +212,73 @@ def dense_gemm(A: torch.Tensor, B: torch.Tensor, out_dtype=torch.bfloat16, out=N
         out = torch.empty((A.shape[0], B.shape[0]), dtype=out_dtype, device=A.device)
     _check("nm_dense_gemm", lib().nm_dense_gemm(_p(A), A.shape[0], _p(B), B.shape[0], A.shape[1], _p(out),
                                                 _dt(out), _stream(A)))
+    return out
+
+
+# ---------------------------------------------------------- 8-bit (E4M3)
+
+
+class Fp8Operand:
+    """Per-row E4M3 codes with their fp32 scales; `lifted` codes for the
+    dense side, window-compressed codes + 8-bit metadata for the sparse side."""
+
+    def __init__(self, codes, scale, rows, K, N, M, meta=None):
+        self.codes, self.scale, self.meta = codes, scale, meta
+        self.rows, self.K, self.N, self.M = rows, K, N, M
+        self.K_lift = lifted_k(K, M)
+
+    def struct(self) -> SparseOperand:
+        return SparseOperand(self.codes.data_ptr(), self.meta.data_ptr(), self.rows, self.K,
+                             self.N, self.M, self.K_lift)
+
+
+def quant_lift_fp8(x: torch.Tensor, M: int, out: Fp8Operand | None = None) -> Fp8Operand:
+    """Per-token E4M3 quantisation fused with the lift: codes [rows, K'] and
+    scales [rows]."""
+    _need_cuda(x)
+    rows, K = x.shape
+    Kl = lifted_k(K, M)
+    if out is None:
+        out = Fp8Operand(torch.empty((rows, Kl), dtype=torch.uint8, device=x.device),
+                         torch.empty(rows, dtype=torch.float32, device=x.device), rows, K, 0, M)
+    _check("nm_quant_lift_fp8", lib().nm_quant_lift_fp8(
+        _p(x), _dt(x), rows, K, x.stride(0), M, _p(out.codes), _p(out.scale), _stream(x)))
+    return out
+
+
+def slide_decompose_fp8(w: torch.Tensor, N: int, M: int) -> Fp8Operand:
+    """Offline 8-bit weight packing: window-compressed codes, per-row scales,
+    8-bit metadata image."""
+    _need_cuda(w)
+    rows, K = w.shape
+    if w.dtype != torch.bfloat16 or w.stride(0) != K:
+        raise ValueError("slide_decompose_fp8 expects a contiguous bf16 weight")
+    Kl = lifted_k(K, M)
+    codes = torch.empty((rows, Kl // 2), dtype=torch.uint8, device=w.device)
+    scale = torch.empty(rows, dtype=torch.float32, device=w.device)
+    meta = torch.empty(max(meta_bytes(rows, K, M), 16), dtype=torch.uint8, device=w.device)
+    ws_bytes = int(lib().slide_decompose_fp8_workspace_size(rows, K, M))
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=w.device)
+    _check("slide_decompose_fp8", lib().slide_decompose_fp8(
+        _p(w), rows, K, N, M, _p(codes), _p(scale), _p(meta), _p(ws), ws_bytes, _stream(w)))
+    return Fp8Operand(codes, scale, rows, K, N, M, meta)
+
+
+def sparse_gemm_fp8(S: Fp8Operand, D: Fp8Operand, side: int, out_dtype=torch.bfloat16,
+                    out: torch.Tensor | None = None) -> torch.Tensor:
+    """8-bit sparse product rescaled by both operands' row scales;
+    side NM_ACT: Y [S.rows, D.rows]; NM_WEIGHT: Y [D.rows, S.rows]."""
+    _need_cuda(D.codes)
+    rows_d = D.rows
+    if D.codes.shape[1] != S.K_lift or not D.codes.is_contiguous():
+        raise ValueError("dense operand must be contiguous codes [rows, K_lift]")
+    shape = (S.rows, rows_d) if side == NM_ACT else (rows_d, S.rows)
+    if out is None:
+        out = torch.empty(shape, dtype=out_dtype, device=D.codes.device)
+    st = S.struct()
+    _check("nm_sparse_gemm_fp8", lib().nm_sparse_gemm_fp8(
+        ctypes.byref(st), _p(S.scale), _p(D.codes), _p(D.scale), rows_d, side, _p(out), _dt(out),
+        _stream(D.codes)))
     return out
 
 

@@ -16,6 +16,7 @@
 #include "nm_gemm.cuh"
 #include "nm_gemm2.cuh"
 #include "nm_prune.cuh"
+#include "nm_fp8.cuh"
 #include "nmsparse.h"
 
 namespace {
@@ -55,14 +56,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // box_outer, 128-byte swizzle, zero fill out of bounds.
 int make_tmap(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t row_bytes,
               uint32_t box_inner, uint32_t box_outer,
-              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B,
+              CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto fn = encode_fn();
   if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  CUresult r = fn(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cuda_fail(cudaErrorInvalidValue);
@@ -100,6 +102,9 @@ struct GemmPlan {
   int64_t ldy = 0;
   int out_fp32 = 0, transpose = 0;
   int a_static = 0;           // A is a weight: may be read before the preceding kernel ends
+  int fp8 = 0;                // 8-bit (E4M3) operands, rescaled by scale_a[row] * scale_b[column]
+  const float* scale_a = nullptr;
+  const float* scale_b = nullptr;
 };
 
 template <int BN>
@@ -181,10 +186,10 @@ int make_tmap_meta(CUtensorMap* m, const void* base, int64_t rows16) {
 }
 
 // Number of 2-CTA clusters of this kernel that fit on the device at once.
-template <int BN, int NACC, int MSUB>
+template <int BN, int NACC, int MSUB, bool FP8 = false>
 int resident_pairs() {
-  using Cfg = nm::Gemm2Cfg<BN, NACC, MSUB>;
-  auto kern = nm::k_nm_gemm_2cta<BN, NACC, MSUB>;
+  using Cfg = nm::Gemm2Cfg<BN, NACC, MSUB, FP8>;
+  auto kern = nm::k_nm_gemm_2cta<BN, NACC, MSUB, FP8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) != cudaSuccess) {
     cudaGetLastError();
     return num_sms() / 2;
@@ -210,12 +215,13 @@ int resident_pairs() {
 
 // Persistent 2-CTA kernel for pure-sparse products whose A side is a whole
 // number of 256-row blocks.
-template <int BN, int NACC, int MSUB>
+template <int BN, int NACC, int MSUB, bool FP8 = false>
 int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
-  using Cfg = nm::Gemm2Cfg<BN, NACC, MSUB>;
+  using Cfg = nm::Gemm2Cfg<BN, NACC, MSUB, FP8>;
   CUtensorMap ta, tb, te, ty, tad;
   int rc;
-  const int64_t kb = ceil_div(p.ks_lift, 128);
+  // k-blocks: 128 lifted K (bf16) or 256 (8-bit, the last one possibly 128)
+  const int64_t kb = ceil_div(p.ks_lift, FP8 ? 256 : 128);
   const int64_t kb_dense = ceil_div(p.kd, 64);
   const bool tma_store = !p.out_fp32 && !p.transpose && (p.ldy % 8) == 0 &&
                          (reinterpret_cast<uintptr_t>(p.y) & 15u) == 0;
@@ -223,6 +229,15 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
     if ((rc = make_tmap(&ty, p.y, p.rows_b, p.rows_a, p.ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) != NM_OK)
       return rc;
   }
+  const int64_t meta_kb = ceil_div(p.ks_lift, 128);     // 128-K metadata blocks per 128 rows
+  if (FP8) {
+    if ((rc = make_tmap(&ta, p.a_s, p.ks_lift / 2, p.rows_a, p.ks_lift / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_DATA_TYPE_UINT8)) != NM_OK) return rc;
+    if ((rc = make_tmap_meta(&te, p.meta, ceil_div(p.rows_a, 128) * meta_kb * 128)) != NM_OK) return rc;
+    if ((rc = make_tmap(&tb, p.b, p.ks_lift, p.rows_b, p.ks_lift, 128, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_DATA_TYPE_UINT8)) != NM_OK) return rc;
+    tad = ta;
+  } else {
   if (kb > 0) {
     if ((rc = make_tmap(&ta, p.a_s, p.ks_lift / 2, p.rows_a, p.ks_lift, 64, 128)) != NM_OK) return rc;
     if ((rc = make_tmap_meta(&te, p.meta, ceil_div(p.rows_a, 128) * kb * 128)) != NM_OK) return rc;
@@ -233,13 +248,17 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   if (kb == 0) { ta = tad; te = tad; }
   if (kb_dense == 0) tad = ta;
   if ((rc = make_tmap(&tb, p.b, p.ks_lift + p.kd, p.rows_b, (p.ks_lift + p.kd) * 2, 64, BN / 2)) != NM_OK) return rc;
+  }
   nm::Gemm2Args a{};
   a.rows_a = p.rows_a;
   a.rows_b = p.rows_b;
   a.kb = static_cast<int>(kb);
   a.kb_dense = static_cast<int>(kb_dense);
   a.k_dense_x0 = p.ks_lift;
-  a.meta_kb = kb;
+  a.meta_kb = meta_kb;
+  a.scale_a = p.scale_a;
+  a.scale_b = p.scale_b;
+  a.last_half = (FP8 && p.ks_lift % 256 != 0) ? 1 : 0;
   a.tiles_m = static_cast<int>(ceil_div(p.rows_a, 256 * MSUB));
   a.tiles_n = static_cast<int>(ceil_div(p.rows_b, BN));
   a.Y = p.y;
@@ -249,13 +268,13 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   a.tma_store = tma_store ? 1 : 0;
   if (!tma_store) ty = ta;                             // unused; any valid map
   const int tiles = a.tiles_m * a.tiles_n;
-  auto kern = nm::k_nm_gemm_2cta<BN, NACC, MSUB>;
+  auto kern = nm::k_nm_gemm_2cta<BN, NACC, MSUB, FP8>;
   NM_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem));
   cudaLaunchConfig_t cfg{};
   // A persistent grid larger than the number of co-resident SM pairs would
   // run its last clusters after the others: size it by the occupancy query.
   static int resident = 0;
-  if (resident == 0) resident = resident_pairs<BN, NACC, MSUB>();
+  if (resident == 0) resident = resident_pairs<BN, NACC, MSUB, FP8>();
   const int clusters = std::max(1, std::min(tiles, resident));
   cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
   cfg.blockDim = dim3(192, 1, 1);
@@ -485,6 +504,125 @@ int nm_sparse_gemm(const nm_sparse_operand* S, const void* D, int64_t rows_d, nm
   p.ldy = side == NM_ACT ? rows_d : S->rows;
   p.a_static = side == NM_WEIGHT;
   return run_gemm(p, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------ 8-bit (E4M3)
+
+int nm_quant_lift_fp8(const void* src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, int M,
+                      uint8_t* codes_out, float* scale_out, void* stream) {
+  if (dt != NM_BF16 && dt != NM_FP32) return NM_ERR_INVALID_ARG;
+  if (rows < 0 || K <= 0 || M <= 0 || ld < K || K % M != 0) return NM_ERR_INVALID_ARG;
+  if (!m_supported(M)) return NM_ERR_UNSUPPORTED;
+  const int64_t esz = dt == NM_BF16 ? 2 : 4;
+  const int64_t Kl = nm_lifted_k(K, M);
+  if (Kl % 16 != 0 || K * esz > NM_FP8_MAX_ROW_BYTES) return NM_ERR_UNSUPPORTED;
+  if (rows == 0) return NM_OK;
+  if (src == nullptr || codes_out == nullptr || scale_out == nullptr) return NM_ERR_INVALID_ARG;
+  if (!aligned16(src) || !aligned16(codes_out) || (ld * esz) % 16 != 0 ||
+      (reinterpret_cast<uintptr_t>(scale_out) & 3u) != 0)
+    return NM_ERR_ALIGNMENT;
+  auto st = static_cast<cudaStream_t>(stream);
+  const size_t smem = static_cast<size_t>(K * esz);
+  const dim3 grid(static_cast<unsigned>(std::min<int64_t>(rows, int64_t(1) << 30))), block(256);
+  cudaError_t err;
+#define NM_QL(MM, TT)                                                                                      \
+  {                                                                                                        \
+    auto kern = nm::k_quant_lift_fp8<MM, TT>;                                                              \
+    NM_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))); \
+    err = launch_pdl(kern, grid, block, smem, st, static_cast<const TT*>(src), rows, K, ld, codes_out, scale_out, Kl); \
+  }
+  if (dt == NM_BF16) {
+    switch (M) {
+      case 4: NM_QL(4, uint16_t) break;
+      case 8: NM_QL(8, uint16_t) break;
+      case 16: NM_QL(16, uint16_t) break;
+      default: NM_QL(32, uint16_t) break;
+    }
+  } else {
+    switch (M) {
+      case 4: NM_QL(4, uint32_t) break;
+      case 8: NM_QL(8, uint32_t) break;
+      case 16: NM_QL(16, uint32_t) break;
+      default: NM_QL(32, uint32_t) break;
+    }
+  }
+#undef NM_QL
+  NM_CUDA_TRY(err);
+  NM_CUDA_TRY(cudaGetLastError());
+  return NM_OK;
+}
+
+size_t slide_decompose_fp8_workspace_size(int64_t rows, int64_t K, int M) {
+  const int64_t Kl = nm_lifted_k(K, M);
+  if (Kl < 0 || rows < 0) return 0;
+  const size_t vals = static_cast<size_t>(ceil_div(rows * (Kl / 2) * 2, int64_t(256)) * 256);
+  return vals + nm_meta_bytes(rows, K, M);
+}
+
+int slide_decompose_fp8(const void* w, int64_t rows, int64_t K, int N, int M, uint8_t* vals_out,
+                        float* scale_out, uint8_t* meta_out, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_prune_args(w, NM_BF16, rows, K, K, N, M, vals_out, meta_out);
+  if (rc != NM_OK) return rc;
+  const int64_t Kl = nm_lifted_k(K, M);
+  if (Kl % 16 != 0) return NM_ERR_UNSUPPORTED;
+  if (rows == 0) return NM_OK;
+  if (scale_out == nullptr || ws == nullptr) return NM_ERR_INVALID_ARG;
+  if (ws_bytes < slide_decompose_fp8_workspace_size(rows, K, M)) return NM_ERR_WORKSPACE;
+  if (!aligned16(ws) || (reinterpret_cast<uintptr_t>(scale_out) & 3u) != 0) return NM_ERR_ALIGNMENT;
+  auto st = static_cast<cudaStream_t>(stream);
+  auto wv = static_cast<uint8_t*>(ws);
+  uint8_t* wm = wv + (slide_decompose_fp8_workspace_size(rows, K, M) - nm_meta_bytes(rows, K, M));
+  // 16-bit windows first (the same pruning and window split), then 8-bit codes and metadata
+  if ((rc = launch_prune(static_cast<const uint16_t*>(w), rows, K, K, N, M, nullptr, wv, wm, st)) != NM_OK) return rc;
+  const unsigned rgrid = static_cast<unsigned>(std::min<int64_t>(rows, int64_t(1) << 30));
+  NM_CUDA_TRY(launch_pdl(nm::k_row_scale_fp8, dim3(rgrid), dim3(256), 0, st,
+                         static_cast<const uint16_t*>(w), rows, K, scale_out));
+  const int64_t chunks = rows * (Kl / 16);
+  const unsigned vgrid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(ceil_div(chunks, 256), int64_t(1) << 30)));
+  NM_CUDA_TRY(launch_pdl(nm::k_quant_vals_fp8, dim3(vgrid), dim3(256), 0, st,
+                         reinterpret_cast<const uint16_t*>(wv), rows, Kl / 2, static_cast<const float*>(scale_out),
+                         vals_out));
+  const int64_t blocks = ceil_div(rows, int64_t(128)) * ceil_div(Kl, int64_t(128));
+  const unsigned mgrid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(ceil_div(blocks * 128, 256), int64_t(1) << 30)));
+  NM_CUDA_TRY(launch_pdl(nm::k_meta_f16_to_8, dim3(mgrid), dim3(256), 0, st,
+                         static_cast<const uint8_t*>(wm), blocks, meta_out));
+  NM_CUDA_TRY(cudaGetLastError());
+  return NM_OK;
+}
+
+int nm_sparse_gemm_fp8(const nm_sparse_operand* S, const float* S_scale, const void* D, const float* D_scale,
+                       int64_t rows_d, nm_side side, void* Y, nm_dtype out_dt, void* stream) {
+  if (S == nullptr) return NM_ERR_INVALID_ARG;
+  if (side != NM_ACT && side != NM_WEIGHT) return NM_ERR_INVALID_ARG;
+  if (out_dt != NM_BF16 && out_dt != NM_FP32) return NM_ERR_INVALID_ARG;
+  if (S->rows < 0 || rows_d < 0 || S->K <= 0 || S->M <= 0 || S->K % S->M != 0) return NM_ERR_INVALID_ARG;
+  if (!m_supported(S->M)) return NM_ERR_UNSUPPORTED;
+  if (S->K_lift != nm_lifted_k(S->K, S->M)) return NM_ERR_INVALID_ARG;
+  if (S->K_lift % 128 != 0 || S->rows % 256 != 0) return NM_ERR_UNSUPPORTED;
+  if (S->rows == 0 || rows_d == 0) return NM_OK;
+  if (D == nullptr || Y == nullptr || S->vals == nullptr || S->meta == nullptr || S_scale == nullptr ||
+      D_scale == nullptr)
+    return NM_ERR_INVALID_ARG;
+  if (!aligned16(S->vals) || !aligned16(S->meta) || !aligned16(D) || !aligned16(Y) ||
+      (reinterpret_cast<uintptr_t>(S_scale) & 3u) != 0 || (reinterpret_cast<uintptr_t>(D_scale) & 3u) != 0)
+    return NM_ERR_ALIGNMENT;
+  GemmPlan p;
+  p.a_s = S->vals;
+  p.b = D;
+  p.rows_a = S->rows;
+  p.rows_b = rows_d;
+  p.ks_lift = S->K_lift;
+  p.kd = 0;
+  p.meta = static_cast<const uint8_t*>(S->meta);
+  p.y = Y;
+  p.out_fp32 = out_dt == NM_FP32;
+  p.transpose = side == NM_WEIGHT;
+  p.ldy = side == NM_ACT ? rows_d : S->rows;
+  p.a_static = side == NM_WEIGHT;
+  p.fp8 = 1;
+  p.scale_a = S_scale;
+  p.scale_b = D_scale;
+  return launch_gemm_2cta<224, 2, 1, true>(p, static_cast<cudaStream_t>(stream));
 }
 
 int nm_dense_gemm(const void* A, int64_t rows_a, const void* B, int64_t rows_b, int64_t K, void* Y,

@@ -252,4 +252,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool sparse) {
        | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// kind::f8f6f4 with both operands E4M3 (format code 0), fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool sparse) {
+  return (sparse ? (1u << 2) : 0u)        // sparse flag
+       | (1u << 4)                        // D format: f32
+       | (static_cast<uint32_t>(N >> 3) << 17)
+       | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 }  // namespace nm

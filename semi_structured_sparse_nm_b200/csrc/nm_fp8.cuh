@@ -1,0 +1,174 @@
+// nm_fp8.cuh -- the 8-bit (E4M3) operand preparation.
+//
+// SlideSparse runs its online path as one fused kernel that quantises each
+// token of the dense operand and writes it lifted; the weights are packed
+// offline.  Here:
+//   k_quant_lift_fp8  per row: amax, scale = amax / 448, codes of x / scale,
+//                     written in the lifted window order (one pass over X);
+//   k_row_scale_fp8   per row of W: scale = amax / 448;
+//   k_quant_vals_fp8  codes of the compressed (kept) values with their row's
+//                     scale;
+//   k_meta_f16_to_8   the 16-bit metadata image re-laid as the 8-bit one
+//                     (row-major: row m, window j of a 128 x 128-K block at
+//                     byte 16 m + j / 2, low nibble for even j).
+// Scales and quotients are IEEE fp32 (correctly rounded division); codes
+// are nearest-even with saturation to +-448 (cvt.rn.satfinite).
+#pragma once
+#include <cuda_fp8.h>
+#include "nm_device.cuh"
+
+namespace nm {
+
+__device__ __forceinline__ float elem_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+__device__ __forceinline__ float elem_f32(uint32_t f) { return __uint_as_float(f); }
+
+// Two fp32 values -> two E4M3 codes (first in the low byte).
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
+}
+
+// Block-wide maximum of a non-negative value (256 threads).
+__device__ __forceinline__ float block_max_256(float v, float* s_red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float m = s_red[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) m = fmaxf(m, s_red[i]);
+  return m;
+}
+
+__device__ __forceinline__ float fp8_scale_of(float amax) {
+  return amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+}
+
+// Per-token quantise + lift.  One CTA per row; the row is staged in dynamic
+// shared memory (K elements of T).  codes[r][g*4(n-1) + 4w + j] =
+// e4m3(x[r][g*2n + 2w + j] / scale[r]); 16-byte stores (four windows) when
+// the lifted row length is a multiple of 16 (checked by the host).
+template <int M, typename T>
+__global__ void __launch_bounds__(256)
+k_quant_lift_fp8(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
+                 uint8_t* __restrict__ codes, float* __restrict__ scale_out, int64_t Kl) {
+  constexpr int NW = M / 2 - 1;
+  constexpr int PV = 16 / static_cast<int>(sizeof(T));
+  extern __shared__ __align__(16) uint8_t qsm[];
+  T* s_x = reinterpret_cast<T*>(qsm);
+  __shared__ float s_red[8];
+  griddep_launch_dependents();
+  griddep_wait();
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const T* row = src + r * ld;
+    float amax = 0.0f;
+    for (int64_t i = static_cast<int64_t>(threadIdx.x) * PV; i < K; i += 256 * PV) {
+      if (i + PV <= K) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + i));
+        *reinterpret_cast<uint4*>(s_x + i) = u;
+        const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int j = 0; j < PV; ++j) amax = fmaxf(amax, fabsf(elem_f32(e[j])));
+      } else {                                         // a bf16 row ending in half a 16-byte word
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(row + i));
+        *reinterpret_cast<uint2*>(s_x + i) = u;
+        const T* e = reinterpret_cast<const T*>(&u);
+#pragma unroll
+        for (int j = 0; j < 8 / static_cast<int>(sizeof(T)); ++j) amax = fmaxf(amax, fabsf(elem_f32(e[j])));
+      }
+    }
+    const float sc = fp8_scale_of(block_max_256(amax, s_red));   // block_max_256 syncs: s_x is complete
+    if (threadIdx.x == 0) scale_out[r] = sc;
+    const int64_t nwin = Kl / 4;
+    uint8_t* out = codes + r * Kl;
+    for (int64_t c = threadIdx.x; 4 * c < nwin; c += 256) {
+      uint32_t wd[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int64_t W = 4 * c + q;
+        if (W < nwin) {
+          const int64_t s0 = (W / NW) * M + 2 * (W % NW);
+          const uint32_t lo = e4m3x2(__fdiv_rn(elem_f32(s_x[s0]), sc), __fdiv_rn(elem_f32(s_x[s0 + 1]), sc));
+          const uint32_t hi = e4m3x2(__fdiv_rn(elem_f32(s_x[s0 + 2]), sc), __fdiv_rn(elem_f32(s_x[s0 + 3]), sc));
+          wd[q] = lo | (hi << 16);
+        } else {
+          wd[q] = 0u;
+        }
+      }
+      if (4 * c + 4 <= nwin) {
+        reinterpret_cast<uint4*>(out)[c] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+      } else {
+        for (int q = 0; q < 4 && 4 * c + q < nwin; ++q) reinterpret_cast<uint32_t*>(out)[4 * c + q] = wd[q];
+      }
+    }
+    __syncthreads();                                   // s_x and s_red are reused by the next row
+  }
+}
+
+// scale[r] = amax(w[r][:]) / 448 for bf16 rows of length K (pitch K).
+__global__ void __launch_bounds__(256)
+k_row_scale_fp8(const uint16_t* __restrict__ w, int64_t rows, int64_t K, float* __restrict__ scale_out) {
+  __shared__ float s_red[8];
+  griddep_launch_dependents();
+  griddep_wait();
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const uint16_t* row = w + r * K;
+    float amax = 0.0f;
+    for (int64_t i = threadIdx.x; i < K; i += 256) amax = fmaxf(amax, fabsf(elem_f32(row[i])));
+    const float sc = fp8_scale_of(block_max_256(amax, s_red));
+    if (threadIdx.x == 0) scale_out[r] = sc;
+    __syncthreads();
+  }
+}
+
+// codes[r][i] = e4m3(vals[r][i] / scale[r]) for bf16 compressed values,
+// nv values per row (a multiple of 8): eight values per thread.
+__global__ void __launch_bounds__(256)
+k_quant_vals_fp8(const uint16_t* __restrict__ vals, int64_t rows, int64_t nv, const float* __restrict__ scale,
+                 uint8_t* __restrict__ codes) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int64_t per_row = nv / 8, total = rows * per_row;
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = t / per_row;
+    const float sc = scale[r];
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(vals) + t);
+    const uint16_t* e = reinterpret_cast<const uint16_t*>(&u);
+    uint32_t wd[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t lo = e4m3x2(__fdiv_rn(elem_f32(e[4 * h]), sc), __fdiv_rn(elem_f32(e[4 * h + 1]), sc));
+      const uint32_t hi = e4m3x2(__fdiv_rn(elem_f32(e[4 * h + 2]), sc), __fdiv_rn(elem_f32(e[4 * h + 3]), sc));
+      wd[h] = lo | (hi << 16);
+    }
+    reinterpret_cast<uint2*>(codes)[t] = make_uint2(wd[0], wd[1]);
+  }
+}
+
+// The 16-bit metadata image (per 128 x 128-K block: row m, window j at lane
+// (m%8) + 8((j%8)/4) + 16(m/16), word j/8, nibble (j%4) + 4((m/8)%2)) re-laid
+// as the 8-bit image (row m, window j at byte 16 m + j/2, low nibble for even
+// j).  One thread per (block, row).
+__global__ void __launch_bounds__(256)
+k_meta_f16_to_8(const uint8_t* __restrict__ in, int64_t blocks, uint8_t* __restrict__ out) {
+  griddep_launch_dependents();
+  griddep_wait();
+  const int64_t total = blocks * 128;
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t blk = t / 128;
+    const int m = static_cast<int>(t % 128);
+    const uint8_t* b = in + blk * 2048;
+    uint32_t wd[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int lane = (m % 8) + 8 * ((j % 8) / 4) + 16 * (m / 16);
+      const int nb = (j % 4) + 4 * ((m / 8) % 2);
+      const uint32_t q = (b[lane * 16 + (j / 8) * 4 + nb / 2] >> (4 * (nb % 2))) & 0xFu;
+      wd[j / 8] |= q << (4 * (j % 8));
+    }
+    reinterpret_cast<uint4*>(out + blk * 2048)[m] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+  }
+}
+
+}  // namespace nm

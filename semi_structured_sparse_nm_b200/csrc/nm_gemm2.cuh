@@ -21,6 +21,12 @@
 // Tiles are visited A-block fastest so that concurrently running clusters
 // share the B tile (the larger, streamed operand) through L2.
 //
+// FP8 = true runs the 8-bit product (tcgen05.mma.sp kind::f8f6f4, E4M3 x
+// E4M3): a k-block is then 256 lifted K -- the same bytes per stage as a
+// 128-K bf16 block -- with four K = 64 MMAs, two 16-byte-per-row metadata
+// blocks per 128 rows (tensor-memory columns +2 per MMA), and the epilogue
+// multiplies the accumulator by the row scale of A and the column scale of B.
+//
 // MSUB = 2 makes the tile 512 x BN: each k-slice issues two M = 256 MMAs that
 // share the B stage (CTA r holds A rows 512 tm + 256 u + 128 r for u = 0, 1).
 // That cuts the shared-memory fill per MMA cycle from 64 + 8192/BN to
@@ -75,6 +81,15 @@ __device__ __forceinline__ void tc_commit_pair(uint64_t* bar) {
 __device__ __forceinline__ void tc_cp_pair_128x128b(uint32_t taddr, uint64_t desc) {
   asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" :: "r"(taddr), "l"(desc) : "memory");
 }
+__device__ __forceinline__ void tc_mma_sp_pair_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                    uint32_t e_tmem, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::2.kind::f8f6f4 [%0], %1, %2, [%5], %3, p;\n\t}"
+      :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(e_tmem)
+      : "memory");
+}
 __device__ __forceinline__ void tc_mma_sp_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t e_tmem,
                                                uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -116,15 +131,19 @@ struct Gemm2Args {
   int out_fp32;
   int transpose_out;
   int tma_store;          // 1: bf16 row-major Y written by TMA from a staging tile
+  const float* scale_a;   // 8-bit product: per-row scale of A (nullptr: none)
+  const float* scale_b;   //                per-row scale of B, i.e. per output column
+  int last_half;          // 8-bit product: the last k-block holds only 128 lifted K
 };
 
-template <int BN, int NACC, int MSUB>
+template <int BN, int NACC, int MSUB, bool FP8 = false>
 struct Gemm2Cfg {
   static constexpr int kHalfN = BN / 2;
-  static constexpr int kA1 = 128 * 128;                // one subtile: 128 rows x 64 stored bf16
+  static constexpr int kA1 = 128 * 128;                // one subtile: 128 rows x 128 stored bytes
   static constexpr int kA = MSUB * kA1;
-  static constexpr int kB = 2 * kHalfN * 128;          // two 64-column halves
-  static constexpr int kE = MSUB * 2048;
+  static constexpr int kB = 2 * kHalfN * 128;          // two 128-byte-wide column halves
+  static constexpr int kEBlocks = FP8 ? 2 : 1;         // 128-K metadata blocks per k-block
+  static constexpr int kE = MSUB * 2048 * kEBlocks;
   static constexpr int kStage = kA + kB + kE;
   static constexpr int kStaging = 4 * 2 * 32 * 32 * 2;  // 4 epilogue warps x 2 buffers x 32x32 bf16
   static constexpr int kStagesRaw = (232448 - kStaging - 2048) / kStage;
@@ -132,19 +151,20 @@ struct Gemm2Cfg {
   static constexpr int kTmemCols = 512;
   static constexpr int kAccStride = 256;               // accumulator (b, u) at column 256 (b MSUB + u)
   static constexpr int kMetaCol = (NACC * MSUB - 1) * kAccStride + BN;
+  static constexpr int kMetaCols = 4 * kEBlocks * MSUB;   // metadata columns per stage
   static constexpr int kSmem = kStages * kStage + kStaging + 1024 + 512;
   static_assert(NACC * MSUB <= 2, "two accumulators of up to 256 columns");
-  static_assert(kMetaCol + 4 * MSUB * kStages <= kTmemCols, "tensor memory budget");
+  static_assert(kMetaCol + kMetaCols * kStages <= kTmemCols, "tensor memory budget");
   static_assert(kHalfN % 8 == 0 && BN % 16 == 0 && BN <= 256, "MMA N");
   static_assert(kStages >= 3, "ring too shallow");
 };
 
-template <int BN, int NACC, int MSUB>
+template <int BN, int NACC, int MSUB, bool FP8 = false>
 __global__ void __launch_bounds__(192, 1)
 k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
                const __grid_constant__ CUtensorMap tmAd, const Gemm2Args args) {
-  using Cfg = Gemm2Cfg<BN, NACC, MSUB>;
+  using Cfg = Gemm2Cfg<BN, NACC, MSUB, FP8>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw2[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw2) + 1023) & ~uintptr_t(1023));
@@ -214,6 +234,25 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB, static_cast<int32_t>(args.k_dense_x0) + kd * 64, yb);
             continue;
           }
+          if constexpr (FP8) {
+            // 256 lifted K: A 128 stored bytes, B two 128-byte halves, two
+            // metadata blocks (one when the last block holds only 128 K)
+            const int eb = (args.last_half && kb == args.kb - 1) ? 1 : 2;
+            if (leader)
+              mbar_arrive_expect_tx(&full_bar[s],
+                                    static_cast<uint32_t>(2 * (Cfg::kA + Cfg::kB / 2 * eb + MSUB * 2048 * eb)));
+#pragma unroll
+            for (int u = 0; u < MSUB; ++u) {
+              const int64_t rb = (static_cast<int64_t>(tm) * MSUB + u) * 2 + rank;
+              tma_load_2d_pair(&tmA, fb, sA + s * Cfg::kA + u * Cfg::kA1, kb * 128, static_cast<int32_t>(rb * 128));
+              for (int e = 0; e < eb; ++e)
+                tma_load_2d_pair(&tmE, fb, sE + s * Cfg::kE + (u * 2 + e) * 2048, 0,
+                                 static_cast<int32_t>((rb * args.meta_kb + 2 * kb + e) * 128));
+            }
+            tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB, kb * 256, yb);
+            if (eb == 2) tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB + Cfg::kHalfN * 128, kb * 256 + 128, yb);
+            continue;
+          }
           if (leader) mbar_arrive_expect_tx(&full_bar[s], stage_tx);
 #pragma unroll
           for (int u = 0; u < MSUB; ++u) {
@@ -266,7 +305,29 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             tc_commit_pair(&empty_bar[s]);
             continue;
           }
-          const uint32_t e_col = tmem_meta + 4u * MSUB * s;
+          const uint32_t e_col = tmem_meta + static_cast<uint32_t>(Cfg::kMetaCols) * s;
+          if constexpr (FP8) {
+            // metadata block e of subtile u -> columns e_col + 8u + 4e; MMA kk
+            // (64 lifted K) reads its two columns at e_col + 8u + 2kk
+            const int nkk = (args.last_half && kb == args.kb - 1) ? 2 : 4;
+#pragma unroll
+            for (int u = 0; u < MSUB; ++u)
+              for (int e = 0; e < nkk / 2; ++e)
+                tc_cp_pair_128x128b(e_col + 8u * u + 4u * e,
+                                    desc_plain_128x16(smem_u32(sE + s * Cfg::kE + (u * 2 + e) * 2048)));
+            const uint32_t idesc8 = idesc_e4m3(256, BN, true);
+            for (int kk = 0; kk < nkk; ++kk) {
+              const uint64_t bd = desc_sw128_kmajor(b0 + (kk / 2) * (Cfg::kHalfN * 128) + (kk % 2) * 64);
+#pragma unroll
+              for (int u = 0; u < MSUB; ++u) {
+                const uint64_t ad = desc_sw128_kmajor(a0 + u * Cfg::kA1 + 32u * kk);
+                tc_mma_sp_pair_e4m3(acc + u * Cfg::kAccStride, ad, bd, e_col + 8u * u + 2u * kk, idesc8,
+                                    (kb > 0 || kk > 0) ? 1u : 0u);
+              }
+            }
+            tc_commit_pair(&empty_bar[s]);
+            continue;
+          }
 #pragma unroll
           for (int u = 0; u < MSUB; ++u)
             tc_cp_pair_128x128b(e_col + 4u * u, desc_plain_128x16(smem_u32(sE + s * Cfg::kE + u * 2048)));
@@ -315,6 +376,16 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           uint32_t v[32];
           tc_ld_32x32b_x32(acc + c0, v);
           tc_wait_ld();
+          if constexpr (FP8) {
+            // rescale: acc * scale_a[row] * scale_b[column]
+            const float sa = ra < args.rows_a ? __ldg(args.scale_a + ra) : 0.0f;
+            const int64_t cb0 = static_cast<int64_t>(tn) * BN + c0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float sb = cb0 + i < args.rows_b ? __ldg(args.scale_b + cb0 + i) : 0.0f;
+              v[i] = __float_as_uint(__uint_as_float(v[i]) * sa * sb);
+            }
+          }
           if (args.tma_store) {
             // 32 rows x 32 bf16 staging tile, 64-byte swizzle: row r's 16-byte
             // chunk j sits at r*64 + 16*(j ^ ((r >> 1) & 3)).  Two buffers per

@@ -22,7 +22,7 @@ def host_bits(t: torch.Tensor) -> np.ndarray:
         return t.view(torch.uint16).numpy() if hasattr(torch, "uint16") else t.view(torch.int16).numpy().view(np.uint16)
     if t.dtype == torch.uint8:
         return t.numpy()
-    if t.dtype == torch.int32:
+    if t.dtype in (torch.int32, torch.float32):
         return t.numpy().view(np.uint32)
     raise TypeError(t.dtype)
 

@@ -1,0 +1,109 @@
+"""The 8-bit (E4M3) path on the GPU against the oracle: quantise + lift and
+the weight packing bit-exact (codes, scales, 8-bit metadata image), the
+rescaled sparse product within tolerance, exactly on integer grids."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from semi_structured_sparse_nm_b200 import _lib as nm
+from semi_structured_sparse_nm_b200 import inputs
+from tests.gpu_util import check_close, dev, host_bits, host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _x(rows, K, kind, seed):
+    if kind == "fp32":
+        return np.random.default_rng(seed).standard_normal((rows, K)).astype(np.float32) * 3
+    if kind == "student_t":
+        return inputs.student_t_bf16((rows, K), 4.0, seed)
+    if kind == "outliers":
+        return inputs.normal_with_outlier_channels_bf16((rows, K), 0.01, 20.0, seed)
+    if kind == "zero_rows":
+        x = inputs.normal_bf16((rows, K), 1.0, seed)
+        x[::3] = 0
+        return x
+    vals = np.array([-448.0, -2.0, -1e-3, -0.0, 0.0, 3e-6, 1.0, 2.0, 300.0])     # ties and extremes
+    return inputs.bf16_from_f64(vals[np.random.default_rng(seed).integers(0, vals.size, size=(rows, K))])
+
+
+@pytest.mark.parametrize("rows,K,M,kind", [
+    (17, 256, 8, "student_t"), (64, 1024, 8, "outliers"), (5, 512, 16, "zero_rows"), (33, 640, 4, "ties"),
+    (9, 2048, 32, "student_t"), (12, 768, 8, "fp32"), (130, 4096, 8, "student_t"),
+])
+def test_quant_lift_bit_exact(rows, K, M, kind):
+    x = _x(rows, K, kind, rows + K)
+    q = nm.quant_lift_fp8(dev(x), M)
+    torch.cuda.synchronize()
+    ref = oracle.fp8_activation(x, M)
+    np.testing.assert_array_equal(host_bits(q.scale), oracle._as_bits(ref["scale"]), err_msg="scales")
+    np.testing.assert_array_equal(q.codes.cpu().numpy(), ref["lifted"], err_msg="lifted codes")
+
+
+@pytest.mark.parametrize("rows,K,N,M", [(256, 1024, 6, 8), (130, 512, 2, 4), (40, 768, 14, 16), (9, 2048, 30, 32)])
+def test_weight_packing_bit_exact(rows, K, N, M):
+    w = inputs.normal_bf16((rows, K), 0.02, rows + 1)
+    P = nm.slide_decompose_fp8(dev(w), N, M)
+    torch.cuda.synchronize()
+    ref = oracle.fp8_weight(w, N, M)
+    np.testing.assert_array_equal(host_bits(P.scale), oracle._as_bits(ref["scale"]), err_msg="scales")
+    np.testing.assert_array_equal(P.codes.cpu().numpy(), ref["vals"], err_msg="codes")
+    np.testing.assert_array_equal(P.meta.cpu().numpy()[:ref["meta"].size], ref["meta"], err_msg="8-bit metadata")
+
+
+@pytest.mark.parametrize("T,O,K,N,M", [
+    (300, 512, 1024, 6, 8),     # 256-K blocks only
+    (40, 256, 768, 6, 8),       # K' = 1152: the last block holds 128 K
+    (16, 256, 640, 2, 4),       # 2:4, half last block, a decode-sized T
+    (129, 768, 512, 14, 16),
+])
+def test_fp8_weight_sparse_product(T, O, K, N, M):
+    x = inputs.student_t_bf16((T, K), 4.0, seed=T)
+    w = inputs.normal_bf16((O, K), 0.02, seed=O)
+    P = nm.slide_decompose_fp8(dev(w), N, M)
+    q = nm.quant_lift_fp8(dev(x), M)
+    y = nm.sparse_gemm_fp8(P, q, nm.NM_WEIGHT, torch.float32)
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    check_close(host_f64(y), oracle.fp8_weight_sparse_linear(x, w, N, M), f"fp8 {T}x{O}x{K} {N}:{M}")
+
+
+def test_fp8_product_exact_on_integer_grid():
+    """Integer values on the E4M3 grid with every row maximum at 448: both
+    scales are 1 and every product and fp32 partial sum is an exact integer."""
+    rng = np.random.default_rng(9)
+    def make(rows, K):
+        v = rng.integers(-16, 17, size=(rows, K)).astype(np.float64)
+        v[:, 0] = 448.0
+        return inputs.bf16_from_f64(v)
+    x, w = make(48, 512), make(256, 512)
+    P = nm.slide_decompose_fp8(dev(w), 6, 8)
+    q = nm.quant_lift_fp8(dev(x), 8)
+    y = nm.sparse_gemm_fp8(P, q, nm.NM_WEIGHT, torch.float32)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host_f64(y), oracle.fp8_weight_sparse_linear(x, w, 6, 8))
+
+
+def test_fp8_full_size_sampled_rows():
+    wl, x, w = inputs.make_workload("slide_6of8_wt_prefill")
+    P = nm.slide_decompose_fp8(dev(w), wl.N, wl.M)
+    q = nm.quant_lift_fp8(dev(x), wl.M)
+    y = nm.sparse_gemm_fp8(P, q, nm.NM_WEIGHT, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    rows = np.array([0, 1, 127, 128, 1000, 2047, 4095])
+    check_close(host_f64(y[torch.from_numpy(rows).cuda()]),
+                oracle.fp8_weight_sparse_linear(x, w, wl.N, wl.M, rows=rows), "fp8 full size")
+
+
+def test_fp8_unsupported_shapes_launch_nothing():
+    w = dev(inputs.normal_bf16((130, 512), 0.02, 1))
+    P = nm.slide_decompose_fp8(w, 6, 8)                       # packing works for any row count
+    q = nm.quant_lift_fp8(dev(inputs.normal_bf16((8, 512), 1.0, 2)), 8)
+    with pytest.raises(nm.NmError) as e:
+        nm.sparse_gemm_fp8(P, q, nm.NM_WEIGHT)                # the product needs whole 256-row blocks
+    assert e.value.status == nm.NM_ERR_UNSUPPORTED
+    with pytest.raises(nm.NmError) as e:
+        nm.quant_lift_fp8(dev(inputs.normal_bf16((4, 40), 1.0, 3)), 8)   # K' = 60: not a multiple of 16
+    assert e.value.status == nm.NM_ERR_UNSUPPORTED
