@@ -42,7 +42,8 @@ HEADLINE = "up_proj_8of16_act"
 TRAFFIC = {
     ("up_proj_8of16_act", "k_nm_gemm_2cta<224,2,1>"): 231897344 + 46815488,
 }
-OTHERS = ["up_proj_2of4_act", "down_proj_16of32_act", "slide_6of8_wt_prefill", "slide_6of8_wt_decode",
+OTHERS = ["up_proj_2of4_act", "down_proj_16of32_act", "slide_6of8_wt_prefill", "slide_6of8_wt_prefill_fp8",
+          "slide_6of8_wt_decode",
           "hybrid_decode_b1", "hybrid_decode_b8", "hybrid_decode_b32", "hybrid_decode_b128",
           "tiny_2of4_act_fp32"]
 L2_BYTES = 126 * 1024 * 1024
@@ -222,6 +223,21 @@ class Workload:
             self.Y = torch.empty((wl.T, wl.O), dtype=out_dt, device=dev)
             self.rows_a, self.rows_b = wl.T, wl.O
             self.prep_name, self.gemm_name = "prune_compress", "sparse_gemm"
+        elif wl.side == "weight" and wl.fp8:
+            P = nm.slide_decompose_fp8(W, wl.N, wl.M)                  # offline
+            wbytes = P.codes.numel() + P.meta.numel() + P.scale.numel() * 4
+            xbytes = X0.numel() * 2
+            self.R = max(2, int(np.ceil(2 * L2_BYTES / (wbytes + xbytes))))
+            self.P = [P] + [nm.Fp8Operand(P.codes.clone(), P.scale.clone(), wl.O, wl.K, wl.N, wl.M, P.meta.clone())
+                            for _ in range(1, self.R)]
+            self.X = [X0] + [X0.roll(r, dims=0).contiguous() for r in range(1, self.R)]
+            self.Q = [nm.Fp8Operand(torch.empty((wl.T, wl.K_lift), dtype=torch.uint8, device=dev),
+                                    torch.empty(wl.T, dtype=torch.float32, device=dev), wl.T, wl.K, 0, wl.M)
+                      for _ in range(2)]
+            self.Y = torch.empty((wl.T, wl.O), dtype=out_dt, device=dev)
+            self.rows_a, self.rows_b = wl.O, wl.T
+            self.prep_name, self.gemm_name = "quant_lift_fp8", "sparse_gemm_fp8"
+            self.w_bytes = wbytes
         elif wl.side == "weight":
             Wc = nm.slide_decompose(W, wl.N, wl.M)                     # offline
             wbytes = Wc.vals.numel() * 2 + Wc.meta.numel()
@@ -260,6 +276,12 @@ class Workload:
             if mark:
                 mark()
             nm.sparse_gemm(c, self.Wl, nm.NM_ACT, self.Y.dtype, out=self.Y)
+        elif wl.side == "weight" and wl.fp8:
+            q = self.Q[i % 2]
+            nm.quant_lift_fp8(self.X[r], wl.M, out=q)
+            if mark:
+                mark()
+            nm.sparse_gemm_fp8(self.P[r], q, nm.NM_WEIGHT, self.Y.dtype, out=self.Y)
         elif wl.side == "weight":
             xl = self.Xl[i % 2]
             nm.lift(self.X[r], wl.M, out=xl)
@@ -276,6 +298,8 @@ class Workload:
         r = i % self.R
         if wl.side == "act":
             nm.sparse_gemm(self.comp[0], self.Wl, nm.NM_ACT, self.Y.dtype, out=self.Y)
+        elif wl.side == "weight" and wl.fp8:
+            nm.sparse_gemm_fp8(self.P[r], self.Q[0], nm.NM_WEIGHT, self.Y.dtype, out=self.Y)
         elif wl.side == "weight":
             nm.sparse_gemm(self.Wc[r], self.Xl[0], nm.NM_WEIGHT, self.Y.dtype, out=self.Y)
         else:
@@ -290,6 +314,9 @@ class Workload:
             Ks = wl.K - D
             mma = 2.0 * wl.T * wl.O * (Ks + D)          # sparse part counted at its 2:4 rate
             byts = (self.w_bytes + wl.T * wl.K * 2 + wl.T * wl.O * self.Y.element_size())
+        elif wl.fp8:
+            mma = 2.0 * wl.T * wl.O * wl.K_lift
+            byts = self.w_bytes + self.rows_b * (wl.K_lift + 4) + wl.T * wl.O * self.Y.element_size()
         else:
             mma = 2.0 * wl.T * wl.O * wl.K_lift
             sparse_bytes = self.rows_a * wl.K_lift + self.nm.meta_bytes(self.rows_a, wl.K, wl.M)
@@ -393,6 +420,39 @@ def time_dense(wk, reps=10):
     return out[0], out[1]
 
 
+def time_dense_fp8(wk, reps=10):
+    """cuBLAS 8-bit dense GEMM on the same (unpruned) product as library
+    context: X and W quantised per row to E4M3, row-wise scales, bf16 out.
+    Returns ms per launch, or None where torch offers no such GEMM."""
+    import torch
+    wl = wk.wl
+    dev = wk.dev
+    try:
+        X = torch.from_numpy(wk.x_np).view(torch.bfloat16).to(dev).float()
+        W = torch.from_numpy(wk.w_np).view(torch.bfloat16).to(dev).float()
+        sx = (X.abs().amax(dim=1, keepdim=True) / 448.0).clamp_min(1e-12)
+        sw = (W.abs().amax(dim=1, keepdim=True) / 448.0).clamp_min(1e-12)
+        Xq = (X / sx).to(torch.float8_e4m3fn)
+        Wq = (W / sw).to(torch.float8_e4m3fn)
+        del X, W
+
+        def fn():
+            return torch._scaled_mm(Xq, Wq.t(), scale_a=sx, scale_b=sw.t(), out_dtype=torch.bfloat16)
+
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+    except Exception:
+        return None
+
+
 def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None):
     dense, mma, byts = wk.algorithmic()
     wl = wk.wl
@@ -406,7 +466,14 @@ def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None):
     if getattr(wk, "instrumented_step_ms", None) is not None:
         out["kernels"]["note"] = ("per-kernel times from a second pass of the same steps with an event around "
                                   "each kernel; that pass's step: %.2f us" % (wk.instrumented_step_ms * 1e3))
-    if not wk.decode and wl.x_dtype == "bf16":
+    if not wk.decode and wl.fp8:
+        c8 = time_dense_fp8(wk)
+        out["dense_comparator"] = {
+            "cublas_fp8_us": None if c8 is None else c8 * 1e3,
+            "sparse_gemm_speedup_vs_cublas_fp8": None if c8 is None else c8 / gemm_ms,
+            "note": "same unpruned product, E4M3 operands with per-row scales, bf16 out, cuBLAS "
+                    "(torch._scaled_mm); library context only"}
+    elif not wk.decode and wl.x_dtype == "bf16":
         ours, cublas = time_dense(wk)
         out["dense_comparator"] = {
             "ours_us": ours * 1e3, "cublas_us": cublas * 1e3,
@@ -419,6 +486,14 @@ def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None):
                            "unit": "GB/s", "frac": achieved / pk["hbm"], "traffic": traffic,
                            "bytes_per_launch": byts,
                            "peak_note": f"{pk['source']} HBM copy bandwidth"}
+    elif wl.fp8:
+        peak = 4.0 * pk["bf16"]
+        achieved = mma / (gemm_ms * 1e-3) / 1e12
+        out["roofline"] = {"bound": "tensor", "kernel": wk.gemm_name, "achieved": achieved, "peak": peak,
+                           "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                           "flops_per_launch": mma,
+                           "peak_note": f"4 x {pk['source']} bf16 burst {pk['bf16']} TFLOP/s (nominal 8-bit / "
+                                        f"16-bit ratio 2 x nominal 2:4 sparse ratio 2)"}
     else:
         peak = 2.0 * pk["bf16"]
         achieved = mma / (gemm_ms * 1e-3) / 1e12

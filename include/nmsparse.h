@@ -170,8 +170,9 @@ int nm_dense_gemm(const void *A, int64_t rows_a, const void *B, int64_t rows_b, 
  *
  * E4M3: the OCP 8-bit format with bias 7, 3 mantissa bits, largest finite
  * 448, no infinity.  Per row: amax = max |x|, scale = amax / 448 (fp32,
- * correctly rounded; 1 for an all-zero row), code = E4M3(x / scale) with the
- * quotient an fp32 division, rounded to nearest even and saturated to +-448.
+ * correctly rounded; 1 for an all-zero row), inv = 1 / scale (fp32, correctly
+ * rounded), code = E4M3(x * inv) with the product rounded to fp32, then to
+ * nearest even E4M3 and saturated to +-448.
  *
  * The 8-bit metadata image has the blocks of nm_meta_bytes() (128 rows x 128
  * lifted columns, 2048 bytes, block (rb, kb) at (rb * ceil(K'/128) + kb) *
@@ -192,7 +193,7 @@ int nm_quant_lift_fp8(const void *src, nm_dtype dt, int64_t rows, int64_t K, int
 
 /* Offline weight packer, 8-bit: slide_decompose() of the bf16 weight
  * W [rows x K] (row stride K), then per row scale = amax(W[r]) / 448 and the
- * kept values' codes E4M3(v / scale).  vals_out [rows][K'/2] codes,
+ * kept values' codes E4M3(v * (1 / scale)).  vals_out [rows][K'/2] codes,
  * scale_out [rows], meta_out the 8-bit image (nm_meta_bytes(rows, K, M)
  * bytes).  ws: slide_decompose_fp8_workspace_size() bytes of scratch (the
  * 16-bit windows).  K' must be a multiple of 16. */

@@ -457,11 +457,12 @@ static float value_f32_at(const void *src, int dt, int64_t idx) {
 }
 
 /* Step 8a.  Per-row (per-token) quantisation.  amax = max_k |x[r][k]|,
- * scale = amax / 448 rounded to fp32 (1 for an all-zero row), and
- * code = e4m3(x / scale) with the quotient rounded to fp32: the quantised
- * code is decided from the same fp32 quotient the kernel forms.  The pages
- * say only that activations are quantised per token; a symmetric scale that
- * maps the row maximum to the largest code is the plainest reading. */
+ * scale = amax / 448 rounded to fp32 (1 for an all-zero row), inv = 1 / scale
+ * rounded to fp32, and code = e4m3(x * inv) with the product rounded to fp32:
+ * the quantised code is decided from the same fp32 product the kernel forms.
+ * The pages say only that activations are quantised per token; a symmetric
+ * scale that maps the row maximum to the largest code, applied through its
+ * reciprocal, is the plainest reading. */
 void or_quant_rows_e4m3(const void *src, int dt, int64_t rows, int64_t K, uint8_t *codes, float *scale) {
 #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r) {
@@ -471,18 +472,21 @@ void or_quant_rows_e4m3(const void *src, int dt, int64_t rows, int64_t K, uint8_
             if (v > amax) amax = v;
         }
         const float s = amax > 0.0f ? amax / 448.0f : 1.0f;
+        const float inv = 1.0f / s;
         scale[r] = s;
-        for (int64_t k = 0; k < K; ++k) codes[r * K + k] = or_e4m3_from_f32(value_f32_at(src, dt, r * K + k) / s);
+        for (int64_t k = 0; k < K; ++k) codes[r * K + k] = or_e4m3_from_f32(value_f32_at(src, dt, r * K + k) * inv);
     }
 }
 
 /* Step 8b.  Codes of a row's compressed values (bf16 bits) with that row's
- * scale: code = e4m3(v / scale[r]), the quotient rounded to fp32.  Padded
- * slots (+0.0) give the code 0x00. */
+ * scale: code = e4m3(v * (1 / scale[r])), reciprocal and product rounded to
+ * fp32 as in step 8a.  Padded slots (+0.0) give the code 0x00. */
 void or_quant_vals_e4m3(const uint16_t *vals, int64_t rows, int64_t nv, const float *scale, uint8_t *codes) {
-    for (int64_t r = 0; r < rows; ++r)
+    for (int64_t r = 0; r < rows; ++r) {
+        const float inv = 1.0f / scale[r];
         for (int64_t i = 0; i < nv; ++i)
-            codes[r * nv + i] = or_e4m3_from_f32((float)bf16_bits_to_double(vals[r * nv + i]) / scale[r]);
+            codes[r * nv + i] = or_e4m3_from_f32((float)bf16_bits_to_double(vals[r * nv + i]) * inv);
+    }
 }
 
 /* Step 5 on bytes: dst[r][g*4(n-1) + 4w + j] = src[r][g*2n + 2w + j]. */

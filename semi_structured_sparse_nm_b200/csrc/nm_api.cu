@@ -622,7 +622,33 @@ int nm_sparse_gemm_fp8(const nm_sparse_operand* S, const float* S_scale, const v
   p.fp8 = 1;
   p.scale_a = S_scale;
   p.scale_b = D_scale;
-  return launch_gemm_2cta<224, 2, 1, true>(p, static_cast<cudaStream_t>(stream));
+  const char* env = std::getenv("NMSPARSE_GEMM");
+  const std::string mode = env != nullptr ? env : "auto";
+  auto st = static_cast<cudaStream_t>(stream);
+  int bn = 0;
+  if (mode == "2cta224") bn = 224;
+  if (mode == "2cta192") bn = 192;
+  if (mode == "2cta160") bn = 160;
+  if (mode == "2cta128") bn = 128;
+  if (bn == 0) {
+    // Tile width by waves over the SM pairs: cost = waves * (BN + 48), the
+    // 48 standing for a tile's fixed share (measured: 192 wide at 4096 rows
+    // of B, 160 at 2048, 128 at 512).
+    const int64_t pairs = std::max(1, num_sms() / 2);
+    const int64_t tiles_m = ceil_div(p.rows_a, int64_t(256));
+    int64_t best = -1;
+    for (int cand : {224, 192, 160, 128}) {
+      const int64_t waves = ceil_div(tiles_m * ceil_div(p.rows_b, int64_t(cand)), pairs);
+      const int64_t cost = waves * (cand + 48);
+      if (best < 0 || cost < best) { best = cost; bn = cand; }
+    }
+  }
+  switch (bn) {
+    case 192: return launch_gemm_2cta<192, 2, 1, true>(p, st);
+    case 160: return launch_gemm_2cta<160, 2, 1, true>(p, st);
+    case 128: return launch_gemm_2cta<128, 2, 1, true>(p, st);
+    default: return launch_gemm_2cta<224, 2, 1, true>(p, st);
+  }
 }
 
 int nm_dense_gemm(const void* A, int64_t rows_a, const void* B, int64_t rows_b, int64_t K, void* Y,

@@ -11,8 +11,10 @@
 //   k_meta_f16_to_8   the 16-bit metadata image re-laid as the 8-bit one
 //                     (row-major: row m, window j of a 128 x 128-K block at
 //                     byte 16 m + j / 2, low nibble for even j).
-// Scales and quotients are IEEE fp32 (correctly rounded division); codes
-// are nearest-even with saturation to +-448 (cvt.rn.satfinite).
+// Scales are IEEE fp32: scale = amax / 448 (correctly rounded division) and
+// its reciprocal 1 / scale (correctly rounded); a value's code is taken from
+// the fp32 product x * (1 / scale), nearest-even with saturation to +-448
+// (cvt.rn.satfinite).
 #pragma once
 #include <cuda_fp8.h>
 #include "nm_device.cuh"
@@ -45,7 +47,7 @@ __device__ __forceinline__ float fp8_scale_of(float amax) {
 
 // Per-token quantise + lift.  One CTA per row; the row is staged in dynamic
 // shared memory (K elements of T).  codes[r][g*4(n-1) + 4w + j] =
-// e4m3(x[r][g*2n + 2w + j] / scale[r]); 16-byte stores (four windows) when
+// e4m3(x[r][g*2n + 2w + j] * (1 / scale[r])); 16-byte stores (four windows) when
 // the lifted row length is a multiple of 16 (checked by the host).
 template <int M, typename T>
 __global__ void __launch_bounds__(256)
@@ -77,6 +79,7 @@ k_quant_lift_fp8(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
       }
     }
     const float sc = fp8_scale_of(block_max_256(amax, s_red));   // block_max_256 syncs: s_x is complete
+    const float inv = __frcp_rn(sc);
     if (threadIdx.x == 0) scale_out[r] = sc;
     const int64_t nwin = Kl / 4;
     uint8_t* out = codes + r * Kl;
@@ -87,8 +90,8 @@ k_quant_lift_fp8(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
         const int64_t W = 4 * c + q;
         if (W < nwin) {
           const int64_t s0 = (W / NW) * M + 2 * (W % NW);
-          const uint32_t lo = e4m3x2(__fdiv_rn(elem_f32(s_x[s0]), sc), __fdiv_rn(elem_f32(s_x[s0 + 1]), sc));
-          const uint32_t hi = e4m3x2(__fdiv_rn(elem_f32(s_x[s0 + 2]), sc), __fdiv_rn(elem_f32(s_x[s0 + 3]), sc));
+          const uint32_t lo = e4m3x2(__fmul_rn(elem_f32(s_x[s0]), inv), __fmul_rn(elem_f32(s_x[s0 + 1]), inv));
+          const uint32_t hi = e4m3x2(__fmul_rn(elem_f32(s_x[s0 + 2]), inv), __fmul_rn(elem_f32(s_x[s0 + 3]), inv));
           wd[q] = lo | (hi << 16);
         } else {
           wd[q] = 0u;
@@ -120,7 +123,7 @@ k_row_scale_fp8(const uint16_t* __restrict__ w, int64_t rows, int64_t K, float* 
   }
 }
 
-// codes[r][i] = e4m3(vals[r][i] / scale[r]) for bf16 compressed values,
+// codes[r][i] = e4m3(vals[r][i] * (1 / scale[r])) for bf16 compressed values,
 // nv values per row (a multiple of 8): eight values per thread.
 __global__ void __launch_bounds__(256)
 k_quant_vals_fp8(const uint16_t* __restrict__ vals, int64_t rows, int64_t nv, const float* __restrict__ scale,
@@ -131,14 +134,14 @@ k_quant_vals_fp8(const uint16_t* __restrict__ vals, int64_t rows, int64_t nv, co
   for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t r = t / per_row;
-    const float sc = scale[r];
+    const float inv = __frcp_rn(scale[r]);
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(vals) + t);
     const uint16_t* e = reinterpret_cast<const uint16_t*>(&u);
     uint32_t wd[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const uint32_t lo = e4m3x2(__fdiv_rn(elem_f32(e[4 * h]), sc), __fdiv_rn(elem_f32(e[4 * h + 1]), sc));
-      const uint32_t hi = e4m3x2(__fdiv_rn(elem_f32(e[4 * h + 2]), sc), __fdiv_rn(elem_f32(e[4 * h + 3]), sc));
+      const uint32_t lo = e4m3x2(__fmul_rn(elem_f32(e[4 * h]), inv), __fmul_rn(elem_f32(e[4 * h + 1]), inv));
+      const uint32_t hi = e4m3x2(__fmul_rn(elem_f32(e[4 * h + 2]), inv), __fmul_rn(elem_f32(e[4 * h + 3]), inv));
       wd[h] = lo | (hi << 16);
     }
     reinterpret_cast<uint2*>(codes)[t] = make_uint2(wd[0], wd[1]);

@@ -100,6 +100,7 @@ class Workload:
     x_dist: str     # "normal" | "student_t4" | "normal_outliers"
     w_std: float = 0.02
     dense_frac: float = 0.0
+    fp8: bool = False   # 8-bit (E4M3) operands: X quantised per token, W per output row
 
     @property
     def K_lift(self) -> int:
@@ -117,6 +118,9 @@ WORKLOADS = {
         Workload("up_proj_2of4_act", "act", 2048, 4096, 14336, 2, 4, "bf16", "bf16", "student_t4"),
         Workload("slide_6of8_wt_prefill", "weight", 4096, 4096, 4096, 6, 8, "bf16", "bf16", "normal"),
         Workload("slide_6of8_wt_decode", "weight", 16, 4096, 4096, 6, 8, "bf16", "bf16", "normal"),
+        # the same prefill product with 8-bit operands (the pages' B200 precision)
+        Workload("slide_6of8_wt_prefill_fp8", "weight", 4096, 4096, 4096, 6, 8, "bf16", "bf16", "normal",
+                 fp8=True),
         Workload("down_proj_16of32_act", "act", 4096, 14336, 4096, 16, 32, "bf16", "bf16", "normal_outliers"),
     ] + [
         Workload(f"hybrid_decode_b{b}", "hybrid", b, 4096, 14336, 2, 4, "bf16", "bf16", "normal",
