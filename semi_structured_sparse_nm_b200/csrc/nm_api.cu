@@ -171,12 +171,15 @@ int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
 }
 
 // uint8 [rows][16] view of a metadata image, box of one 128-row block.
-int make_tmap_meta(CUtensorMap* m, const void* base, int64_t rows16) {
+// The metadata image as rows of 128 bytes: one 2048-byte block (the
+// tensor-memory image of 128 operand rows) is a box of 16 such rows, fetched
+// as 16 requests of 128 bytes.
+int make_tmap_meta(CUtensorMap* m, const void* base, int64_t blocks) {
   auto fn = encode_fn();
   if (fn == nullptr) return cuda_fail(cudaErrorNotSupported);
-  cuuint64_t dims[2] = {16, static_cast<cuuint64_t>(rows16)};
-  cuuint64_t strides[1] = {16};
-  cuuint32_t box[2] = {16, 128};
+  cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(blocks * 16)};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {128, 16};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -233,14 +236,14 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   if (FP8) {
     if ((rc = make_tmap(&ta, p.a_s, p.ks_lift / 2, p.rows_a, p.ks_lift / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_DATA_TYPE_UINT8)) != NM_OK) return rc;
-    if ((rc = make_tmap_meta(&te, p.meta, ceil_div(p.rows_a, 128) * meta_kb * 128)) != NM_OK) return rc;
+    if ((rc = make_tmap_meta(&te, p.meta, ceil_div(p.rows_a, 128) * meta_kb)) != NM_OK) return rc;
     if ((rc = make_tmap(&tb, p.b, p.ks_lift, p.rows_b, p.ks_lift, 128, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_DATA_TYPE_UINT8)) != NM_OK) return rc;
     tad = ta;
   } else {
   if (kb > 0) {
     if ((rc = make_tmap(&ta, p.a_s, p.ks_lift / 2, p.rows_a, p.ks_lift, 64, 128)) != NM_OK) return rc;
-    if ((rc = make_tmap_meta(&te, p.meta, ceil_div(p.rows_a, 128) * kb * 128)) != NM_OK) return rc;
+    if ((rc = make_tmap_meta(&te, p.meta, ceil_div(p.rows_a, 128) * kb)) != NM_OK) return rc;
   }
   if (kb_dense > 0) {
     if ((rc = make_tmap(&tad, p.a_d, p.kd, p.rows_a, p.kd * 2, 64, 128)) != NM_OK) return rc;

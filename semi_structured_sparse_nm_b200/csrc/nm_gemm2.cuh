@@ -247,22 +247,22 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               tma_load_2d_pair(&tmA, fb, sA + s * Cfg::kA + u * Cfg::kA1, kb * 128, static_cast<int32_t>(rb * 128));
               for (int e = 0; e < eb; ++e)
                 tma_load_2d_pair(&tmE, fb, sE + s * Cfg::kE + (u * 2 + e) * 2048, 0,
-                                 static_cast<int32_t>((rb * args.meta_kb + 2 * kb + e) * 128));
+                                 static_cast<int32_t>((rb * args.meta_kb + 2 * kb + e) * 16));
             }
             tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB, kb * 256, yb);
             if (eb == 2) tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB + Cfg::kHalfN * 128, kb * 256 + 128, yb);
-            continue;
-          }
-          if (leader) mbar_arrive_expect_tx(&full_bar[s], stage_tx);
+          } else {
+            if (leader) mbar_arrive_expect_tx(&full_bar[s], stage_tx);
 #pragma unroll
-          for (int u = 0; u < MSUB; ++u) {
-            const int64_t rb = (static_cast<int64_t>(tm) * MSUB + u) * 2 + rank;       // 128-row block
-            tma_load_2d_pair(&tmA, fb, sA + s * Cfg::kA + u * Cfg::kA1, kb * 64, static_cast<int32_t>(rb * 128));
-            tma_load_2d_pair(&tmE, fb, sE + s * Cfg::kE + u * 2048, 0,
-                             static_cast<int32_t>((rb * args.meta_kb + kb) * 128));
+            for (int u = 0; u < MSUB; ++u) {
+              const int64_t rb = (static_cast<int64_t>(tm) * MSUB + u) * 2 + rank;     // 128-row block
+              tma_load_2d_pair(&tmA, fb, sA + s * Cfg::kA + u * Cfg::kA1, kb * 64, static_cast<int32_t>(rb * 128));
+              tma_load_2d_pair(&tmE, fb, sE + s * Cfg::kE + u * 2048, 0,
+                               static_cast<int32_t>((rb * args.meta_kb + kb) * 16));
+            }
+            tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB, kb * 128, yb);
+            tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB + Cfg::kHalfN * 128, kb * 128 + 64, yb);
           }
-          tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB, kb * 128, yb);
-          tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB + Cfg::kHalfN * 128, kb * 128 + 64, yb);
         }
       }
       // Every stage this CTA filled was released by the leader's commit
@@ -316,29 +316,31 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 tc_cp_pair_128x128b(e_col + 8u * u + 4u * e,
                                     desc_plain_128x16(smem_u32(sE + s * Cfg::kE + (u * 2 + e) * 2048)));
             const uint32_t idesc8 = idesc_e4m3(256, BN, true);
-            for (int kk = 0; kk < nkk; ++kk) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              if (kk < nkk) {
+                const uint64_t bd = desc_sw128_kmajor(b0 + (kk / 2) * (Cfg::kHalfN * 128) + (kk % 2) * 64);
+#pragma unroll
+                for (int u = 0; u < MSUB; ++u) {
+                  const uint64_t ad = desc_sw128_kmajor(a0 + u * Cfg::kA1 + 32u * kk);
+                  tc_mma_sp_pair_e4m3(acc + u * Cfg::kAccStride, ad, bd, e_col + 8u * u + 2u * kk, idesc8,
+                                      (kb > 0 || kk > 0) ? 1u : 0u);
+                }
+              }
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < MSUB; ++u)
+              tc_cp_pair_128x128b(e_col + 4u * u, desc_plain_128x16(smem_u32(sE + s * Cfg::kE + u * 2048)));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
               const uint64_t bd = desc_sw128_kmajor(b0 + (kk / 2) * (Cfg::kHalfN * 128) + (kk % 2) * 64);
 #pragma unroll
               for (int u = 0; u < MSUB; ++u) {
                 const uint64_t ad = desc_sw128_kmajor(a0 + u * Cfg::kA1 + 32u * kk);
-                tc_mma_sp_pair_e4m3(acc + u * Cfg::kAccStride, ad, bd, e_col + 8u * u + 2u * kk, idesc8,
-                                    (kb > 0 || kk > 0) ? 1u : 0u);
+                tc_mma_sp_pair(acc + u * Cfg::kAccStride, ad, bd, e_col + 4u * u + (kk & ~1),
+                               idesc | static_cast<uint32_t>(kk & 1), (kb > 0 || kk > 0) ? 1u : 0u);
               }
-            }
-            tc_commit_pair(&empty_bar[s]);
-            continue;
-          }
-#pragma unroll
-          for (int u = 0; u < MSUB; ++u)
-            tc_cp_pair_128x128b(e_col + 4u * u, desc_plain_128x16(smem_u32(sE + s * Cfg::kE + u * 2048)));
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bd = desc_sw128_kmajor(b0 + (kk / 2) * (Cfg::kHalfN * 128) + (kk % 2) * 64);
-#pragma unroll
-            for (int u = 0; u < MSUB; ++u) {
-              const uint64_t ad = desc_sw128_kmajor(a0 + u * Cfg::kA1 + 32u * kk);
-              tc_mma_sp_pair(acc + u * Cfg::kAccStride, ad, bd, e_col + 4u * u + (kk & ~1),
-                             idesc | static_cast<uint32_t>(kk & 1), (kb > 0 || kk > 0) ? 1u : 0u);
             }
           }
           tc_commit_pair(&empty_bar[s]);
