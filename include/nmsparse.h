@@ -191,6 +191,16 @@ int nm_dense_gemm(const void *A, int64_t rows_a, const void *B, int64_t rows_b, 
 int nm_quant_lift_fp8(const void *src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, int M,
                       uint8_t *codes_out, float *scale_out, void *stream);
 
+/* Prune + compress in 8 bits (the activation-sparse side): per-row scale
+ * scale_out[r] = amax(src[r]) / 448, then nm_prune_compress() of the bf16
+ * src [rows x K] (row stride ld) with the kept values written as codes
+ * E4M3(v * (1 / scale)) -- codes_out [rows][K'/2], two per window -- and the
+ * metadata as the 8-bit image (meta_out, nm_meta_bytes(rows, K, M) bytes).
+ * mask_out as in nm_prune_compress().  K' must be a multiple of 16. */
+int nm_prune_compress_fp8(const void *src, int64_t rows, int64_t K, int64_t ld, int N, int M,
+                          uint32_t *mask_out, uint8_t *codes_out, float *scale_out, uint8_t *meta_out,
+                          void *stream);
+
 /* Offline weight packer, 8-bit: slide_decompose() of the bf16 weight
  * W [rows x K] (row stride K), then per row scale = amax(W[r]) / 448 and the
  * kept values' codes E4M3(v * (1 / scale)).  vals_out [rows][K'/2] codes,

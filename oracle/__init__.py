@@ -390,3 +390,25 @@ def fp8_weight_sparse_linear(x: np.ndarray, w: np.ndarray, N: int, M: int, rows=
     Y = linear_f64(xd, wd, rows)
     sxs = sx.astype(np.float64) if rows is None else sx.astype(np.float64)[np.asarray(rows)]
     return Y * sxs[:, None] * sw.astype(np.float64)[None, :]
+
+
+def fp8_act_operand(x: np.ndarray, N: int, M: int):
+    """The 8-bit prune + compress step: keep mask, per-token scales (amax of
+    the dense row), codes of the window-compressed kept values, 8-bit image."""
+    keep = prune(x, N, M)
+    vals, nib = compress(x, keep, M)
+    _, scale = quant_rows(x)
+    Kl = lifted_k(x.shape[1], M)
+    return dict(keep=keep, mask=mask_pack(keep), vals=quant_vals(vals, scale), nib=nib, meta=meta8(nib, Kl),
+                scale=scale, K_lift=Kl)
+
+
+def fp8_act_sparse_linear(x: np.ndarray, w: np.ndarray, N: int, M: int, rows=None) -> np.ndarray:
+    """Y[t, o] = sx[t] * sw[o] * sum_k e4m3(prune(X))[t, k] * e4m3(W)[o, k] in fp64."""
+    qx, sx = quant_rows(x)
+    qw, sw = quant_rows(w)
+    keep = prune(x, N, M)
+    xd = np.where(keep.astype(bool), e4m3_to_f64(qx), 0.0)
+    Y = linear_f64(xd, e4m3_to_f64(qw), rows)
+    sxs = sx.astype(np.float64) if rows is None else sx.astype(np.float64)[np.asarray(rows)]
+    return Y * sxs[:, None] * sw.astype(np.float64)[None, :]

@@ -60,6 +60,7 @@ def lib():
             "nm_sparse_gemm": (I, [ctypes.POINTER(SparseOperand), P, I64, I, P, I, P, SZ, P]),
             "nm_dense_gemm": (I, [P, I64, P, I64, I64, P, I, P]),
             "nm_quant_lift_fp8": (I, [P, I, I64, I64, I64, I, P, P, P]),
+            "nm_prune_compress_fp8": (I, [P, I64, I64, I64, I, I, P, P, P, P, P]),
             "slide_decompose_fp8_workspace_size": (SZ, [I64, I64, I]),
             "slide_decompose_fp8": (I, [P, I64, I64, I, I, P, P, P, P, SZ, P]),
             "nm_sparse_gemm_fp8": (I, [ctypes.POINTER(SparseOperand), P, P, P, I64, I, P, I, P]),
@@ -243,6 +244,26 @@ def quant_lift_fp8(x: torch.Tensor, M: int, out: Fp8Operand | None = None) -> Fp
                          torch.empty(rows, dtype=torch.float32, device=x.device), rows, K, 0, M)
     _check("nm_quant_lift_fp8", lib().nm_quant_lift_fp8(
         _p(x), _dt(x), rows, K, x.stride(0), M, _p(out.codes), _p(out.scale), _stream(x)))
+    return out
+
+
+def prune_compress_fp8(x: torch.Tensor, N: int, M: int, out: Fp8Operand | None = None,
+                       with_mask: bool = False) -> Fp8Operand:
+    """Per-token scales, then N:M prune + window compress with the kept values
+    as E4M3 codes and the 8-bit metadata image (bf16 input)."""
+    _need_cuda(x)
+    rows, K = x.shape
+    if x.dtype != torch.bfloat16:
+        raise ValueError("prune_compress_fp8 expects bf16 input")
+    if out is None:
+        Kl = lifted_k(K, M)
+        out = Fp8Operand(torch.empty((rows, Kl // 2), dtype=torch.uint8, device=x.device),
+                         torch.empty(rows, dtype=torch.float32, device=x.device), rows, K, N, M,
+                         torch.empty(max(meta_bytes(rows, K, M), 16), dtype=torch.uint8, device=x.device))
+    mask = torch.empty((rows, (K + 31) // 32), dtype=torch.int32, device=x.device) if with_mask else None
+    out.mask = mask
+    _check("nm_prune_compress_fp8", lib().nm_prune_compress_fp8(
+        _p(x), rows, K, x.stride(0), N, M, _p(mask), _p(out.codes), _p(out.scale), _p(out.meta), _stream(x)))
     return out
 
 

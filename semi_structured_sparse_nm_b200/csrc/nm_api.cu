@@ -363,9 +363,9 @@ int run_gemm(const GemmPlan& p, cudaStream_t st) {
 }
 
 // --------------------------------------------------------------- prune
-template <typename T>
+template <typename T, bool Q8 = false>
 int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M, uint32_t* mask,
-                 void* vals, void* meta, cudaStream_t st) {
+                 void* vals, void* meta, cudaStream_t st, const float* row_scale = nullptr) {
   const int64_t Kl = nm_lifted_k(K, M);
   const int64_t KB = ceil_div(Kl, 128);
   const int64_t rows_pad = ceil_div(rows, 128) * 128;
@@ -380,10 +380,10 @@ int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M
   auto e = static_cast<uint8_t*>(meta);
   cudaError_t err;
   switch (M) {
-    case 4: err = launch_pdl(nm::k_prune_compress<4, T>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
-    case 8: err = launch_pdl(nm::k_prune_compress<8, T>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
-    case 16: err = launch_pdl(nm::k_prune_compress<16, T>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
-    case 32: err = launch_pdl(nm::k_prune_compress<32, T>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad); break;
+    case 4: err = launch_pdl(nm::k_prune_compress<4, T, Q8>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale); break;
+    case 8: err = launch_pdl(nm::k_prune_compress<8, T, Q8>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale); break;
+    case 16: err = launch_pdl(nm::k_prune_compress<16, T, Q8>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale); break;
+    case 32: err = launch_pdl(nm::k_prune_compress<32, T, Q8>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale); break;
     default: return NM_ERR_UNSUPPORTED;
   }
   NM_CUDA_TRY(err);
@@ -555,6 +555,26 @@ int nm_quant_lift_fp8(const void* src, nm_dtype dt, int64_t rows, int64_t K, int
   return NM_OK;
 }
 
+int nm_prune_compress_fp8(const void* src, int64_t rows, int64_t K, int64_t ld, int N, int M,
+                          uint32_t* mask_out, uint8_t* codes_out, float* scale_out, uint8_t* meta_out,
+                          void* stream) {
+  int rc = check_prune_args(src, NM_BF16, rows, K, ld, N, M, codes_out, meta_out);
+  if (rc != NM_OK) return rc;
+  const int64_t Kl = nm_lifted_k(K, M);
+  if (Kl % 16 != 0) return NM_ERR_UNSUPPORTED;
+  if (mask_out != nullptr && !aligned16(mask_out)) return NM_ERR_ALIGNMENT;
+  if (rows == 0) return NM_OK;
+  if (scale_out == nullptr) return NM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(scale_out) & 3u) != 0) return NM_ERR_ALIGNMENT;
+  auto st = static_cast<cudaStream_t>(stream);
+  // per-token scales first, then the prune writes the kept values' codes
+  const unsigned rgrid = static_cast<unsigned>(std::min<int64_t>(rows, int64_t(1) << 30));
+  NM_CUDA_TRY(launch_pdl(nm::k_row_scale_fp8, dim3(rgrid), dim3(256), 0, st,
+                         static_cast<const uint16_t*>(src), rows, K, ld, scale_out));
+  return launch_prune<uint16_t, true>(static_cast<const uint16_t*>(src), rows, K, ld, N, M, mask_out, codes_out,
+                                      meta_out, st, scale_out);
+}
+
 size_t slide_decompose_fp8_workspace_size(int64_t rows, int64_t K, int M) {
   const int64_t Kl = nm_lifted_k(K, M);
   if (Kl < 0 || rows < 0) return 0;
@@ -579,7 +599,7 @@ int slide_decompose_fp8(const void* w, int64_t rows, int64_t K, int N, int M, ui
   if ((rc = launch_prune(static_cast<const uint16_t*>(w), rows, K, K, N, M, nullptr, wv, wm, st)) != NM_OK) return rc;
   const unsigned rgrid = static_cast<unsigned>(std::min<int64_t>(rows, int64_t(1) << 30));
   NM_CUDA_TRY(launch_pdl(nm::k_row_scale_fp8, dim3(rgrid), dim3(256), 0, st,
-                         static_cast<const uint16_t*>(w), rows, K, scale_out));
+                         static_cast<const uint16_t*>(w), rows, K, K, scale_out));
   const int64_t chunks = rows * (Kl / 16);
   const unsigned vgrid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(ceil_div(chunks, 256), int64_t(1) << 30)));
   NM_CUDA_TRY(launch_pdl(nm::k_quant_vals_fp8, dim3(vgrid), dim3(256), 0, st,

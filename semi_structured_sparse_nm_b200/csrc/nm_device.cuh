@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 namespace nm {
 
@@ -250,6 +251,16 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool sparse) {
        | (1u << 10)                       // B format: bf16
        | (static_cast<uint32_t>(N >> 3) << 17)
        | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// bf16 bits / fp32 bits -> fp32 value.
+__device__ __forceinline__ float elem_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
+__device__ __forceinline__ float elem_f32(uint32_t f) { return __uint_as_float(f); }
+
+// Two fp32 values -> two E4M3 codes (first in the low byte), nearest even,
+// saturated to +-448.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
 }
 
 // kind::f8f6f4 with both operands E4M3 (format code 0), fp32 accumulator.

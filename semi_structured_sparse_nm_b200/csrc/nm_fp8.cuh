@@ -16,18 +16,9 @@
 // the fp32 product x * (1 / scale), nearest-even with saturation to +-448
 // (cvt.rn.satfinite).
 #pragma once
-#include <cuda_fp8.h>
 #include "nm_device.cuh"
 
 namespace nm {
-
-__device__ __forceinline__ float elem_f32(uint16_t b) { return __uint_as_float(static_cast<uint32_t>(b) << 16); }
-__device__ __forceinline__ float elem_f32(uint32_t f) { return __uint_as_float(f); }
-
-// Two fp32 values -> two E4M3 codes (first in the low byte).
-__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
-  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
-}
 
 // Block-wide maximum of a non-negative value (256 threads).
 __device__ __forceinline__ float block_max_256(float v, float* s_red) {
@@ -107,14 +98,14 @@ k_quant_lift_fp8(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
   }
 }
 
-// scale[r] = amax(w[r][:]) / 448 for bf16 rows of length K (pitch K).
+// scale[r] = amax(w[r][:]) / 448 for bf16 rows of length K (row stride ld).
 __global__ void __launch_bounds__(256)
-k_row_scale_fp8(const uint16_t* __restrict__ w, int64_t rows, int64_t K, float* __restrict__ scale_out) {
+k_row_scale_fp8(const uint16_t* __restrict__ w, int64_t rows, int64_t K, int64_t ld, float* __restrict__ scale_out) {
   __shared__ float s_red[8];
   griddep_launch_dependents();
   griddep_wait();
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
-    const uint16_t* row = w + r * K;
+    const uint16_t* row = w + r * ld;
     float amax = 0.0f;
     for (int64_t i = threadIdx.x; i < K; i += 256) amax = fmaxf(amax, fabsf(elem_f32(row[i])));
     const float sc = fp8_scale_of(block_max_256(amax, s_red));

@@ -376,11 +376,17 @@ __host__ __device__ constexpr int prune_min_blocks(int M, int elem_bytes) {
   return elem_bytes != 2 ? 1 : (M >= 32 ? 2 : 4);
 }
 
-template <int M, typename T>
+// Q8 = true (bf16 input only) writes the kept values as E4M3 codes --
+// code = e4m3(v * (1 / row_scale[r])) -- two bytes per window instead of two
+// bf16, and the metadata as the 8-bit image (row m, window j of a 128 x 128-K
+// block at byte 16 m + j/2, low nibble for even j).
+template <int M, typename T, bool Q8 = false>
 __global__ void __launch_bounds__(kPruneWarps * 32, prune_min_blocks(M, sizeof(T)))
 k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int N,
-                 uint32_t* __restrict__ mask_out, uint32_t* __restrict__ vals_out,
-                 uint8_t* __restrict__ meta_out, int64_t Kl, int64_t KB, int64_t rows_pad) {
+                 uint32_t* __restrict__ mask_out, void* __restrict__ vals_out,
+                 uint8_t* __restrict__ meta_out, int64_t Kl, int64_t KB, int64_t rows_pad,
+                 const float* __restrict__ row_scale) {
+  static_assert(!Q8 || sizeof(T) == 2, "8-bit output from bf16 input");
   constexpr int G = prune_groups_per_lane(M, static_cast<int>(sizeof(T)));
   constexpr int NW = M / 2 - 1;                   // windows per group
   constexpr int NWL = G * NW;                     // windows per lane
@@ -398,7 +404,7 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
   const int64_t cpr = (groups + 32 * G - 1) / (32 * G);
   const int64_t mask_words = (K + 31) / 32;
   const int64_t tasks = (rows_pad / 16) * cpr;
-  const bool vec_vals = (Kl % 16) == 0;
+  const bool vec_vals = Q8 ? (Kl % 32) == 0 : (Kl % 16) == 0;   // 16-byte output rows
 
   const int64_t drg = gridDim.x / cpr, dch = gridDim.x % cpr;      // grid stride as (row group, chunk)
   int64_t rg = blockIdx.x / cpr, ch = blockIdx.x % cpr;
@@ -427,6 +433,8 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
       if (r >= rows) break;
       if (lane < LM) s_mask[warp][lane] = 0u;
       __syncwarp();
+      float inv = 1.0f;
+      if constexpr (Q8) inv = __frcp_rn(row_scale[r]);
       if (gl < groups) {
         uint32_t vals[NWL];
         uint8_t nibs[NWL];
@@ -456,7 +464,13 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
         }
 #pragma unroll
         for (int w = 0; w < NWL; ++w) {
-          s_val[warp][lane * NWL + w] = vals[w];
+          if constexpr (Q8) {
+            reinterpret_cast<uint16_t*>(&s_val[warp][0])[lane * NWL + w] = static_cast<uint16_t>(
+                e4m3x2(__fmul_rn(elem_f32(static_cast<uint16_t>(vals[w] & 0xFFFFu)), inv),
+                       __fmul_rn(elem_f32(static_cast<uint16_t>(vals[w] >> 16)), inv)));
+          } else {
+            s_val[warp][lane * NWL + w] = vals[w];
+          }
           s_nib[it][lane * NWL + w] = nibs[w];
         }
         if (mask_out != nullptr)
@@ -464,13 +478,25 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
                    (LM == 32 ? keep : (keep & ((1u << LM) - 1u))) << ((lane * LM) % 32));
       }
       __syncwarp();
-      uint32_t* vrow = vals_out + r * (Kl / 4) + g0 * NW;
-      if (vec_vals && ng == 32 * G) {
-        const uint4* sv = reinterpret_cast<const uint4*>(&s_val[warp][0]);
-        uint4* dv = reinterpret_cast<uint4*>(vrow);
-        for (int i = lane; i < WIN / 4; i += 32) dv[i] = sv[i];
+      if constexpr (Q8) {
+        uint16_t* vrow = static_cast<uint16_t*>(vals_out) + r * (Kl / 4) + g0 * NW;
+        const uint16_t* sv16 = reinterpret_cast<const uint16_t*>(&s_val[warp][0]);
+        if (vec_vals && ng == 32 * G) {
+          const uint4* sv = reinterpret_cast<const uint4*>(sv16);
+          uint4* dv = reinterpret_cast<uint4*>(vrow);
+          for (int i = lane; i < WIN / 8; i += 32) dv[i] = sv[i];
+        } else {
+          for (int i = lane; i < ng * NW; i += 32) vrow[i] = sv16[i];
+        }
       } else {
-        for (int i = lane; i < ng * NW; i += 32) vrow[i] = s_val[warp][i];
+        uint32_t* vrow = static_cast<uint32_t*>(vals_out) + r * (Kl / 4) + g0 * NW;
+        if (vec_vals && ng == 32 * G) {
+          const uint4* sv = reinterpret_cast<const uint4*>(&s_val[warp][0]);
+          uint4* dv = reinterpret_cast<uint4*>(vrow);
+          for (int i = lane; i < WIN / 4; i += 32) dv[i] = sv[i];
+        } else {
+          for (int i = lane; i < ng * NW; i += 32) vrow[i] = s_val[warp][i];
+        }
       }
       if (mask_out != nullptr && lane < LM) {
         const int64_t wi = ch * LM + lane;
@@ -484,6 +510,25 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
     // in word c (low half: first row, high half: second row).
     const int64_t rb = r0 / 128;
     const int64_t sub = (r0 % 128) / 16;
+    if constexpr (Q8) {
+      // 8-bit image: row `row` of the task, windows 32b .. 32b+31 -> 16 bytes
+      for (int i = threadIdx.x; i < NWL * 16; i += blockDim.x) {
+        const int b = i / 16, row = i % 16;
+        const int64_t kb = ch * NWL + b;
+        if (kb >= KB) continue;
+        uint32_t wds[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t lo = *reinterpret_cast<const uint32_t*>(&s_nib[row][32 * b + 8 * c]);
+          const uint32_t hi = *reinterpret_cast<const uint32_t*>(&s_nib[row][32 * b + 8 * c + 4]);
+          wds[c] = __byte_perm(lo | (lo >> 4), hi | (hi >> 4), 0x6420);
+        }
+        *reinterpret_cast<uint4*>(meta_out + (rb * KB + kb) * 2048 + (sub * 16 + row) * 16) =
+            make_uint4(wds[0], wds[1], wds[2], wds[3]);
+      }
+      __syncthreads();                                 // s_nib is rewritten by the next task
+      continue;
+    }
     for (int i = threadIdx.x; i < NWL * 16; i += blockDim.x) {
       const int b = i / 16, L = i % 16;
       const int64_t kb = ch * NWL + b;

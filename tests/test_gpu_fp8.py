@@ -107,3 +107,45 @@ def test_fp8_unsupported_shapes_launch_nothing():
     with pytest.raises(nm.NmError) as e:
         nm.quant_lift_fp8(dev(inputs.normal_bf16((4, 40), 1.0, 3)), 8)   # K' = 60: not a multiple of 16
     assert e.value.status == nm.NM_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------ activation side (quantise + prune)
+
+
+@pytest.mark.parametrize("rows,K,N,M,kind", [
+    (130, 1024, 8, 16, "student_t"), (40, 640, 2, 4, "ties"), (64, 2048, 16, 32, "outliers"),
+    (33, 512, 4, 8, "zero_rows"), (256, 4096, 8, 16, "student_t"),
+])
+def test_prune_compress_fp8_bit_exact(rows, K, N, M, kind):
+    x = _x(rows, K, kind, rows + K)
+    P = nm.prune_compress_fp8(dev(x), N, M, with_mask=True)
+    torch.cuda.synchronize()
+    ref = oracle.fp8_act_operand(x, N, M)
+    np.testing.assert_array_equal(host_bits(P.scale), oracle._as_bits(ref["scale"]), err_msg="scales")
+    np.testing.assert_array_equal(host_bits(P.mask), ref["mask"], err_msg="mask")
+    np.testing.assert_array_equal(P.codes.cpu().numpy(), ref["vals"], err_msg="codes")
+    np.testing.assert_array_equal(P.meta.cpu().numpy()[:ref["meta"].size], ref["meta"], err_msg="8-bit metadata")
+
+
+@pytest.mark.parametrize("T,O,K,N,M", [(256, 384, 1024, 8, 16), (512, 136, 512, 2, 4), (256, 200, 2048, 16, 32)])
+def test_fp8_act_sparse_product(T, O, K, N, M):
+    x = inputs.student_t_bf16((T, K), 4.0, seed=T + 3)
+    w = inputs.normal_bf16((O, K), 0.02, seed=O + 3)
+    P = nm.prune_compress_fp8(dev(x), N, M)
+    Wq = nm.quant_lift_fp8(dev(w), M)                       # per output channel, lifted
+    y = nm.sparse_gemm_fp8(P, Wq, nm.NM_ACT, torch.float32)
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    check_close(host_f64(y), oracle.fp8_act_sparse_linear(x, w, N, M), f"fp8 act {T}x{O}x{K} {N}:{M}")
+
+
+def test_fp8_act_full_size_sampled_rows():
+    wl, x, w = inputs.make_workload("up_proj_8of16_act")
+    P = nm.prune_compress_fp8(dev(x), wl.N, wl.M)
+    Wq = nm.quant_lift_fp8(dev(w), wl.M)
+    y = nm.sparse_gemm_fp8(P, Wq, nm.NM_ACT, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    rows = np.array([0, 1, 127, 128, 1000, 2047])
+    check_close(host_f64(y[torch.from_numpy(rows).cuda()]),
+                oracle.fp8_act_sparse_linear(x, w, wl.N, wl.M, rows=rows), "fp8 act full size")

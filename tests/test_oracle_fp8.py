@@ -123,3 +123,32 @@ def test_fp8_product_exact_when_quantisation_is_lossless(N, M):
         y8 = oracle.fp8_weight_sparse_linear(x, w, N, M)
         y = oracle.weight_sparse_linear(x, w, N, M)
         assert np.array_equal(y8, y)
+
+
+@pytest.mark.parametrize("N,M", [(8, 16), (2, 4), (16, 32)])
+def test_fp8_act_product_exact_when_quantisation_is_lossless(N, M):
+    """The activation-sparse 8-bit product on lossless inputs equals the plain
+    activation-sparse product."""
+    grid = oracle.e4m3_to_f64(np.arange(0x00, 0x77, dtype=np.uint8))
+    for top in (448.0, 112.0):
+        def make(rows, K, seed):
+            r = np.random.default_rng(seed)
+            v = r.choice(grid, size=(rows, K)) * r.choice([-1.0, 1.0], size=(rows, K)) * (top / 448.0)
+            v[:, 0] = top
+            return inputs.bf16_from_f64(v)
+        x = make(10, 128, 3)
+        w = make(24, 128, 4)
+        assert np.array_equal(oracle.fp8_act_sparse_linear(x, w, N, M), oracle.act_sparse_linear(x, w, N, M))
+
+
+def test_fp8_act_operand_codes_are_the_kept_values():
+    """Decoded codes times the scale reproduce the kept bf16 values within
+    half an E4M3 step, in the window order of the 16-bit operand."""
+    x = inputs.student_t_bf16((20, 256), 4.0, seed=8)
+    ref16 = oracle.sparse_operand(x, 8, 16)
+    ref8 = oracle.fp8_act_operand(x, 8, 16)
+    assert np.array_equal(ref8["mask"], ref16["mask"])
+    assert np.array_equal(ref8["nib"], ref16["nib"])
+    v = inputs.bf16_to_f64(ref16["vals"])
+    d = oracle.e4m3_to_f64(ref8["vals"]) * ref8["scale"][:, None].astype(np.float64)
+    assert (np.abs(d - v) <= 2.0 ** -4 * np.abs(v) + 2.0 ** -10 * ref8["scale"][:, None] * 1.000001).all()
