@@ -42,7 +42,7 @@ HEADLINE = "up_proj_8of16_act"
 TRAFFIC = {
     ("up_proj_8of16_act", "k_nm_gemm_2cta<224,2,1>"): 232299264 + 48795136,
 }
-OTHERS = ["up_proj_2of4_act", "down_proj_16of32_act", "slide_6of8_wt_prefill", "slide_6of8_wt_prefill_fp8",
+OTHERS = ["up_proj_2of4_act", "up_proj_8of16_act_fp8", "down_proj_16of32_act", "slide_6of8_wt_prefill", "slide_6of8_wt_prefill_fp8",
           "slide_6of8_wt_decode",
           "hybrid_decode_b1", "hybrid_decode_b8", "hybrid_decode_b32", "hybrid_decode_b128",
           "tiny_2of4_act_fp32"]
@@ -215,7 +215,20 @@ class Workload:
         X0, W = to_dev(x_np), to_dev(w_np)
         out_dt = torch.bfloat16 if wl.out_dtype == "bf16" else torch.float32
         self.decode = wl.side == "hybrid" or wl.T <= 128
-        if wl.side == "act":
+        if wl.side == "act" and wl.fp8:
+            self.Wq = nm.quant_lift_fp8(W, wl.M)                         # offline: per-channel codes, lifted
+            self.R = max(2, min(8, int(np.ceil(2 * L2_BYTES / max(X0.numel() * X0.element_size(), 1)))))
+            self.X = [X0] + [X0.roll(r, dims=0).contiguous() for r in range(1, self.R)]
+            Kl = wl.K_lift
+            self.comp = [nm.Fp8Operand(torch.empty((wl.T, Kl // 2), dtype=torch.uint8, device=dev),
+                                       torch.empty(wl.T, dtype=torch.float32, device=dev), wl.T, wl.K, wl.N, wl.M,
+                                       torch.empty(max(nm.meta_bytes(wl.T, wl.K, wl.M), 16), dtype=torch.uint8,
+                                                   device=dev)) for _ in range(2)]
+            self.Y = torch.empty((wl.T, wl.O), dtype=out_dt, device=dev)
+            self.rows_a, self.rows_b = wl.T, wl.O
+            self.prep_name, self.gemm_name = "prune_compress_fp8", "sparse_gemm_fp8"
+            self.launches_per_step = 3                               # row scales, prune, GEMM
+        elif wl.side == "act":
             self.Wl = nm.lift(W, wl.M)                                   # offline
             self.R = max(2, min(8, int(np.ceil(2 * L2_BYTES / max(X0.numel() * X0.element_size(), 1)))))
             self.X = [X0] + [X0.roll(r, dims=0).contiguous() for r in range(1, self.R)]
@@ -263,6 +276,7 @@ class Workload:
             self.rows_a, self.rows_b = wl.O, wl.T
             self.prep_name, self.gemm_name = "gather", "hybrid_gemm"
             self.w_bytes = wbytes
+        self.launches_per_step = getattr(self, "launches_per_step", 2)
         del W
         torch.cuda.synchronize(dev)
 
@@ -270,7 +284,13 @@ class Workload:
     def step(self, i, mark=None):
         nm, wl = self.nm, self.wl
         r = i % self.R
-        if wl.side == "act":
+        if wl.side == "act" and wl.fp8:
+            c = self.comp[i % 2]
+            nm.prune_compress_fp8(self.X[r], wl.N, wl.M, out=c)
+            if mark:
+                mark()
+            nm.sparse_gemm_fp8(c, self.Wq, nm.NM_ACT, self.Y.dtype, out=self.Y)
+        elif wl.side == "act":
             c = self.comp[i % 2]
             nm.prune_compress(self.X[r], wl.N, wl.M, out=c)
             if mark:
@@ -296,7 +316,9 @@ class Workload:
     def gemm_only(self, i):
         nm, wl = self.nm, self.wl
         r = i % self.R
-        if wl.side == "act":
+        if wl.side == "act" and wl.fp8:
+            nm.sparse_gemm_fp8(self.comp[0], self.Wq, nm.NM_ACT, self.Y.dtype, out=self.Y)
+        elif wl.side == "act":
             nm.sparse_gemm(self.comp[0], self.Wl, nm.NM_ACT, self.Y.dtype, out=self.Y)
         elif wl.side == "weight" and wl.fp8:
             nm.sparse_gemm_fp8(self.P[r], self.Q[0], nm.NM_WEIGHT, self.Y.dtype, out=self.Y)
@@ -314,6 +336,10 @@ class Workload:
             Ks = wl.K - D
             mma = 2.0 * wl.T * wl.O * (Ks + D)          # sparse part counted at its 2:4 rate
             byts = (self.w_bytes + wl.T * wl.K * 2 + wl.T * wl.O * self.Y.element_size())
+        elif wl.fp8 and wl.side == "act":
+            mma = 2.0 * wl.T * wl.O * wl.K_lift
+            byts = (self.rows_a * (wl.K_lift // 2 + 4) + self.nm.meta_bytes(self.rows_a, wl.K, wl.M)
+                    + self.rows_b * (wl.K_lift + 4) + wl.T * wl.O * self.Y.element_size())
         elif wl.fp8:
             mma = 2.0 * wl.T * wl.O * wl.K_lift
             byts = self.w_bytes + self.rows_b * (wl.K_lift + 4) + wl.T * wl.O * self.Y.element_size()
@@ -584,7 +610,7 @@ def run_gpu(args):
         "e2e": {"value": ws * dense / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
                 "d2h_bytes_per_step": int(yh.numel() * yh.element_size())},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": wk.launches_per_step * args.steps,
         "clocks": clk.summary(),
         "device_status": status,
     }

@@ -116,6 +116,8 @@ WORKLOADS = {
         Workload("up_proj_8of16_act", "act", 2048, 4096, 14336, 8, 16, "bf16", "bf16", "student_t4"),
         # the same shape pruned 2:4: the 2:4 prefill GEMM measurement
         Workload("up_proj_2of4_act", "act", 2048, 4096, 14336, 2, 4, "bf16", "bf16", "student_t4"),
+        # the same 8:16 product with 8-bit operands (X per token, W per output channel)
+        Workload("up_proj_8of16_act_fp8", "act", 2048, 4096, 14336, 8, 16, "bf16", "bf16", "student_t4", fp8=True),
         Workload("slide_6of8_wt_prefill", "weight", 4096, 4096, 4096, 6, 8, "bf16", "bf16", "normal"),
         Workload("slide_6of8_wt_decode", "weight", 16, 4096, 4096, 6, 8, "bf16", "bf16", "normal"),
         # the same prefill product with 8-bit operands (the pages' B200 precision)
