@@ -180,14 +180,11 @@ int nm_dense_gemm(const void *A, int64_t rows_a, const void *B, int64_t rows_b, 
  * 16*m + q/2, low nibble for even q.  Rows and windows past the operand carry
  * the pair (0,1). */
 
-/* Largest source row (K times the element size) nm_quant_lift_fp8() stages. */
-#define NM_FP8_MAX_ROW_BYTES (96 * 1024)
-
 /* Quantise + lift: codes_out [rows][K'] (row stride K', E4M3 codes in the
  * lifted order of nm_lift()), scale_out [rows] fp32.  src [rows x K], row
- * stride ld elements, NM_BF16 or NM_FP32.  K' must be a multiple of 16 and
- * K * element size at most NM_FP8_MAX_ROW_BYTES (else NM_ERR_UNSUPPORTED);
- * src and codes_out 16-byte aligned, scale_out 4-byte aligned. */
+ * stride ld elements, NM_BF16 or NM_FP32.  K' must be a multiple of 16
+ * (else NM_ERR_UNSUPPORTED); src and codes_out 16-byte aligned, scale_out
+ * 4-byte aligned. */
 int nm_quant_lift_fp8(const void *src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, int M,
                       uint8_t *codes_out, float *scale_out, void *stream);
 

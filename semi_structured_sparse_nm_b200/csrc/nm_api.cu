@@ -518,22 +518,18 @@ int nm_quant_lift_fp8(const void* src, nm_dtype dt, int64_t rows, int64_t K, int
   if (!m_supported(M)) return NM_ERR_UNSUPPORTED;
   const int64_t esz = dt == NM_BF16 ? 2 : 4;
   const int64_t Kl = nm_lifted_k(K, M);
-  if (Kl % 16 != 0 || K * esz > NM_FP8_MAX_ROW_BYTES) return NM_ERR_UNSUPPORTED;
+  if (Kl % 16 != 0) return NM_ERR_UNSUPPORTED;
   if (rows == 0) return NM_OK;
   if (src == nullptr || codes_out == nullptr || scale_out == nullptr) return NM_ERR_INVALID_ARG;
   if (!aligned16(src) || !aligned16(codes_out) || (ld * esz) % 16 != 0 ||
       (reinterpret_cast<uintptr_t>(scale_out) & 3u) != 0)
     return NM_ERR_ALIGNMENT;
   auto st = static_cast<cudaStream_t>(stream);
-  const size_t smem = static_cast<size_t>(K * esz);
   const dim3 grid(static_cast<unsigned>(std::min<int64_t>(rows, int64_t(1) << 30))), block(256);
   cudaError_t err;
 #define NM_QL(MM, TT)                                                                                      \
-  {                                                                                                        \
-    auto kern = nm::k_quant_lift_fp8<MM, TT>;                                                              \
-    NM_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))); \
-    err = launch_pdl(kern, grid, block, smem, st, static_cast<const TT*>(src), rows, K, ld, codes_out, scale_out, Kl); \
-  }
+  err = launch_pdl(nm::k_quant_lift_fp8<MM, TT>, grid, block, 0, st, static_cast<const TT*>(src), rows, K, ld, \
+                   codes_out, scale_out, Kl);
   if (dt == NM_BF16) {
     switch (M) {
       case 4: NM_QL(4, uint16_t) break;

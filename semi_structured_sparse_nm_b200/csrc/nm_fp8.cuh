@@ -36,65 +36,85 @@ __device__ __forceinline__ float fp8_scale_of(float amax) {
   return amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
 }
 
-// Per-token quantise + lift.  One CTA per row; the row is staged in dynamic
-// shared memory (K elements of T).  codes[r][g*4(n-1) + 4w + j] =
-// e4m3(x[r][g*2n + 2w + j] * (1 / scale[r])); 16-byte stores (four windows) when
-// the lifted row length is a multiple of 16 (checked by the host).
+// Per-token quantise + lift.  One CTA per row.  Pass 1 reduces |x| over the
+// row to its maximum (16-byte loads, block reduction); pass 2 takes one group
+// of M elements per thread (read again, now from L1), converts each element
+// once -- code = e4m3(x * (1 / scale)) -- and forms the group's n-1 windows
+// codes[r][g*4(n-1) + 4w + j] = code[g*2n + 2w + j] by byte permutes of the
+// packed codes, one 4-byte store per window.
+template <int M, typename T>
+__device__ __forceinline__ void load_group_words(const T* __restrict__ p, uint32_t (&wd)[M * sizeof(T) / 4]) {
+  constexpr int BYTES = M * static_cast<int>(sizeof(T));
+  if constexpr (BYTES >= 16) {
+#pragma unroll
+    for (int v = 0; v < BYTES / 16; ++v) {
+      const uint4 u = __ldg(reinterpret_cast<const uint4*>(p) + v);
+      wd[4 * v] = u.x; wd[4 * v + 1] = u.y; wd[4 * v + 2] = u.z; wd[4 * v + 3] = u.w;
+    }
+  } else {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+    wd[0] = u.x; wd[1] = u.y;
+  }
+}
+
 template <int M, typename T>
 __global__ void __launch_bounds__(256)
 k_quant_lift_fp8(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
                  uint8_t* __restrict__ codes, float* __restrict__ scale_out, int64_t Kl) {
   constexpr int NW = M / 2 - 1;
   constexpr int PV = 16 / static_cast<int>(sizeof(T));
-  extern __shared__ __align__(16) uint8_t qsm[];
-  T* s_x = reinterpret_cast<T*>(qsm);
+  constexpr int WORDS = M * static_cast<int>(sizeof(T)) / 4;     // 32-bit words of one group
   __shared__ float s_red[8];
   griddep_launch_dependents();
   griddep_wait();
+  const int64_t groups = K / M;
   for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
     const T* row = src + r * ld;
     float amax = 0.0f;
     for (int64_t i = static_cast<int64_t>(threadIdx.x) * PV; i < K; i += 256 * PV) {
       if (i + PV <= K) {
         const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + i));
-        *reinterpret_cast<uint4*>(s_x + i) = u;
         const T* e = reinterpret_cast<const T*>(&u);
 #pragma unroll
         for (int j = 0; j < PV; ++j) amax = fmaxf(amax, fabsf(elem_f32(e[j])));
-      } else {                                         // a bf16 row ending in half a 16-byte word
+      } else if constexpr (sizeof(T) == 2) {           // a bf16 row ending in half a 16-byte word
         const uint2 u = __ldg(reinterpret_cast<const uint2*>(row + i));
-        *reinterpret_cast<uint2*>(s_x + i) = u;
         const T* e = reinterpret_cast<const T*>(&u);
 #pragma unroll
-        for (int j = 0; j < 8 / static_cast<int>(sizeof(T)); ++j) amax = fmaxf(amax, fabsf(elem_f32(e[j])));
+        for (int j = 0; j < 4; ++j) amax = fmaxf(amax, fabsf(elem_f32(e[j])));
       }
     }
-    const float sc = fp8_scale_of(block_max_256(amax, s_red));   // block_max_256 syncs: s_x is complete
+    const float sc = fp8_scale_of(block_max_256(amax, s_red));
     const float inv = __frcp_rn(sc);
     if (threadIdx.x == 0) scale_out[r] = sc;
-    const int64_t nwin = Kl / 4;
-    uint8_t* out = codes + r * Kl;
-    for (int64_t c = threadIdx.x; 4 * c < nwin; c += 256) {
-      uint32_t wd[4];
+    uint32_t* out = reinterpret_cast<uint32_t*>(codes + r * Kl);
+    for (int64_t g = threadIdx.x; g < groups; g += 256) {
+      uint32_t wd[WORDS];
+      load_group_words<M, T>(row + g * M, wd);
+      uint32_t q[M / 4];                               // codes of the group, four per word
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int64_t W = 4 * c + q;
-        if (W < nwin) {
-          const int64_t s0 = (W / NW) * M + 2 * (W % NW);
-          const uint32_t lo = e4m3x2(__fmul_rn(elem_f32(s_x[s0]), inv), __fmul_rn(elem_f32(s_x[s0 + 1]), inv));
-          const uint32_t hi = e4m3x2(__fmul_rn(elem_f32(s_x[s0 + 2]), inv), __fmul_rn(elem_f32(s_x[s0 + 3]), inv));
-          wd[q] = lo | (hi << 16);
-        } else {
-          wd[q] = 0u;
+      for (int c = 0; c < M / 4; ++c) {
+        float f[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int e = 4 * c + j;
+          if constexpr (sizeof(T) == 2) {
+            const uint32_t w = wd[e / 2];
+            f[j] = __uint_as_float((e % 2 == 0) ? (w << 16) : (w & 0xFFFF0000u));
+          } else {
+            f[j] = __uint_as_float(wd[e]);
+          }
         }
+        q[c] = e4m3x2(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv)) |
+               (e4m3x2(__fmul_rn(f[2], inv), __fmul_rn(f[3], inv)) << 16);
       }
-      if (4 * c + 4 <= nwin) {
-        reinterpret_cast<uint4*>(out)[c] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-      } else {
-        for (int q = 0; q < 4 && 4 * c + q < nwin; ++q) reinterpret_cast<uint32_t*>(out)[4 * c + q] = wd[q];
-      }
+      // window w = codes 2w .. 2w+3: word w/2 when w is even, else the upper
+      // half of word (w-1)/2 and the lower half of the next one
+#pragma unroll
+      for (int w = 0; w < NW; ++w)
+        out[g * NW + w] = (w % 2 == 0) ? q[w / 2] : __byte_perm(q[w / 2], q[w / 2 + 1], 0x5432);
     }
-    __syncthreads();                                   // s_x and s_red are reused by the next row
+    __syncthreads();                                   // s_red is reused by the next row
   }
 }
 

@@ -526,9 +526,7 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
         *reinterpret_cast<uint4*>(meta_out + (rb * KB + kb) * 2048 + (sub * 16 + row) * 16) =
             make_uint4(wds[0], wds[1], wds[2], wds[3]);
       }
-      __syncthreads();                                 // s_nib is rewritten by the next task
-      continue;
-    }
+    } else {
     for (int i = threadIdx.x; i < NWL * 16; i += blockDim.x) {
       const int b = i / 16, L = i % 16;
       const int64_t kb = ch * NWL + b;
@@ -545,6 +543,7 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
       }
       *reinterpret_cast<uint4*>(meta_out + (rb * KB + kb) * 2048 + sub * 256 + L * 16) =
           make_uint4(wds[0], wds[1], wds[2], wds[3]);
+    }
     }
     __syncthreads();                                   // s_nib is rewritten by the next task
   }
