@@ -226,10 +226,15 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   // k-blocks: 128 lifted K (bf16) or 256 (8-bit, the last one possibly 128)
   const int64_t kb = ceil_div(p.ks_lift, FP8 ? 256 : 128);
   const int64_t kb_dense = ceil_div(p.kd, 64);
-  const bool tma_store = !p.out_fp32 && !p.transpose && (p.ldy % 8) == 0 &&
-                         (reinterpret_cast<uintptr_t>(p.y) & 15u) == 0;
-  if (tma_store) {
+  // bf16 outputs leave through TMA stores of 32 x 32 staging tiles: Y[a][b]
+  // row-major (64-byte swizzled tile), or Y[b][a] for the transposed product
+  const bool y_ok = !p.out_fp32 && (p.ldy % 8) == 0 && (reinterpret_cast<uintptr_t>(p.y) & 15u) == 0;
+  const int tma_store = !y_ok ? 0 : (p.transpose ? 2 : 1);
+  if (tma_store == 1) {
     if ((rc = make_tmap(&ty, p.y, p.rows_b, p.rows_a, p.ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) != NM_OK)
+      return rc;
+  } else if (tma_store == 2) {
+    if ((rc = make_tmap(&ty, p.y, p.rows_a, p.rows_b, p.ldy * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE)) != NM_OK)
       return rc;
   }
   const int64_t meta_kb = ceil_div(p.ks_lift, 128);     // 128-K metadata blocks per 128 rows
@@ -268,7 +273,7 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   a.ldy = p.ldy;
   a.out_fp32 = p.out_fp32;
   a.transpose_out = p.transpose;
-  a.tma_store = tma_store ? 1 : 0;
+  a.tma_store = tma_store;
   if (!tma_store) ty = ta;                             // unused; any valid map
   const int tiles = a.tiles_m * a.tiles_n;
   auto kern = nm::k_nm_gemm_2cta<BN, NACC, MSUB, FP8>;

@@ -130,7 +130,8 @@ struct Gemm2Args {
   int64_t ldy;
   int out_fp32;
   int transpose_out;
-  int tma_store;          // 1: bf16 row-major Y written by TMA from a staging tile
+  int tma_store;          // 1: bf16 row-major Y written by TMA from a staging tile;
+                          // 2: the same for Y stored transposed (Y[b][a])
   const float* scale_a;   // 8-bit product: per-row scale of A (nullptr: none)
   const float* scale_b;   //                per-row scale of B, i.e. per output column
   int last_half;          // 8-bit product: the last k-block holds only 128 lifted K
@@ -388,7 +389,24 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               v[i] = __float_as_uint(__uint_as_float(v[i]) * sa * sb);
             }
           }
-          if (args.tma_store) {
+          if (args.tma_store == 2) {
+            // transposed: the staging tile is [32 columns of this tile][32 rows],
+            // so that each of its rows is 64 contiguous bytes of one row of Y
+            uint8_t* buf = sY + (q * 2 + (ebuf & 1)) * 2048;
+            if (lane == 0 && ebuf >= 2) bulk_wait_read1();
+            __syncwarp();
+            __nv_bfloat16* t = reinterpret_cast<__nv_bfloat16*>(buf);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) t[i * 32 + lane] = __float2bfloat16_rn(__uint_as_float(v[i]));
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmY, buf, static_cast<int32_t>(row0),
+                           static_cast<int32_t>(static_cast<int64_t>(tn) * BN + c0));
+              bulk_commit();
+            }
+            ++ebuf;
+          } else if (args.tma_store) {
             // 32 rows x 32 bf16 staging tile, 64-byte swizzle: row r's 16-byte
             // chunk j sits at r*64 + 16*(j ^ ((r >> 1) & 3)).  Two buffers per
             // warp; a buffer is rewritten only after its previous store read it.
