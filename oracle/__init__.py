@@ -60,6 +60,8 @@ def _load():
             "or_to_f64": (None, [P, I, I64, P, P]),
             "or_linear_f64": (None, [P, P, I64, I64, I64, P, I64, P]),
             "or_colnorm_f64": (None, [P, I, I64, I64, P]),
+            "or_rownorm_f64": (None, [P, I, I64, I64, P]),
+            "or_silu_f64": (None, [P, I64, P]),
             "or_hybrid_dense_count": (I64, [I64, ctypes.c_double]),
             "or_hybrid_perm": (None, [P, I64, I64, P, P]),
             "or_gather_cols_bf16": (None, [P, I64, I64, P, P]),
@@ -412,3 +414,80 @@ def fp8_act_sparse_linear(x: np.ndarray, w: np.ndarray, N: int, M: int, rows=Non
     Y = linear_f64(xd, e4m3_to_f64(qw), rows)
     sxs = sx.astype(np.float64) if rows is None else sx.astype(np.float64)[np.asarray(rows)]
     return Y * sxs[:, None] * sw.astype(np.float64)[None, :]
+
+
+# ------------------------------------------------------- GLU MLP (hybrid)
+
+
+def rownorm_f64(w: np.ndarray) -> np.ndarray:
+    w = np.ascontiguousarray(w)
+    O, K = w.shape
+    out = np.zeros(O, np.float64)
+    _load().or_rownorm_f64(_ptr(_as_bits(w)), _dt(w), O, K, _ptr(out))
+    return out
+
+
+def silu_f64(z: np.ndarray) -> np.ndarray:
+    z = np.ascontiguousarray(z, dtype=np.float64)
+    out = np.zeros_like(z)
+    _load().or_silu_f64(_ptr(z), z.size, _ptr(out))
+    return out
+
+
+def spense_dense_count(I: int, dense_frac: float) -> int:
+    """Dense intermediate indices: whole blocks of 256, 256 * floor(f * I / 256)."""
+    if dense_frac <= 0.0:
+        return 0
+    if dense_frac >= 1.0:
+        return I
+    return 256 * int((dense_frac * I) / 256.0)
+
+
+def spense_mlp_weights(w_up: np.ndarray, w_gate: np.ndarray, w_down: np.ndarray, dense_frac: float):
+    """The GLU-MLP packing: score = rownorm(up) + rownorm(gate) + colnorm(down)
+    (fp64, summed in that order), the top D intermediate indices dense (ties to
+    the lower index), perm = [sparse asc | dense asc]; keep masks of the
+    pruned weights in the original index order."""
+    I, d = w_up.shape
+    D = spense_dense_count(I, dense_frac)
+    score = (rownorm_f64(w_up) + rownorm_f64(w_gate)) + colnorm_f64(w_down)
+    perm, is_dense = hybrid_perm(score, D)
+    Is = I - D
+    keep_up = np.ones((I, d), np.uint8)
+    keep_gate = np.ones((I, d), np.uint8)
+    keep_down = np.ones(w_down.shape, np.uint8)
+    out = dict(D=D, Is=Is, score=score, perm=perm, is_dense=is_dense)
+    if Is > 0:
+        sp = perm[:Is]
+        up_s = np.ascontiguousarray(w_up[sp])
+        gate_s = np.ascontiguousarray(w_gate[sp])
+        ku, kg = prune(up_s, 2, 4), prune(gate_s, 2, 4)
+        keep_up[sp] = ku
+        keep_gate[sp] = kg
+        ug = np.ascontiguousarray(np.concatenate([up_s, gate_s]))
+        vals, nib = compress(ug, np.concatenate([ku, kg]), 4)
+        out.update(ug_vals=vals, ug_meta=meta_hw(nib, d))
+        dp = gather_cols(w_down, perm)
+        ds = np.ascontiguousarray(dp[:, :Is])
+        kd = prune(ds, 2, 4)
+        keep_down[:, sp] = kd
+        vals_d, nib_d = compress(ds, kd, 4)
+        out.update(down_vals=vals_d, down_meta=meta_hw(nib_d, Is))
+    if D > 0:
+        dn = perm[Is:]
+        out["ug_dense"] = np.ascontiguousarray(np.concatenate([w_up[dn], w_gate[dn]]))
+        out["down_dense"] = np.ascontiguousarray(gather_cols(w_down, perm)[:, Is:])
+    out.update(keep_up=keep_up, keep_gate=keep_gate, keep_down=keep_down)
+    return out
+
+
+def spense_mlp(x: np.ndarray, w_up: np.ndarray, w_gate: np.ndarray, w_down: np.ndarray, dense_frac: float,
+               rows=None) -> np.ndarray:
+    """y = (silu(x . Gp^T) * (x . Up^T)) . Dp^T in fp64, with Up, Gp, Dp the
+    pruned weights in the original index order."""
+    p = spense_mlp_weights(w_up, w_gate, w_down, dense_frac)
+    xd = to_f64(x)
+    u = linear_f64(xd, to_f64(w_up, p["keep_up"]), rows)
+    g = linear_f64(xd, to_f64(w_gate, p["keep_gate"]), rows)
+    h = silu_f64(g) * u
+    return linear_f64(h, to_f64(w_down, p["keep_down"]))

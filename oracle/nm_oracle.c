@@ -33,6 +33,17 @@
  *               [SpenseGPT, technical summary §2.A (dense region + 2:4 region,
  *                input-split with accumulation) and §2.B (permutation of the
  *                intermediate indices into one contiguous dense block)]
+ *  7'. glu mlp  the GLU mapping of the hybrid format: one set of intermediate
+ *               indices stays dense in all three projections, chosen by
+ *               the summed fp64 energies of the up and gate rows and the down
+ *               column; the indices are permuted into [sparse | dense]; up
+ *               and gate are split by output (their sparse rows pruned 2:4
+ *               along the model dimension), down by input (its sparse
+ *               columns pruned 2:4 in the permuted order); h = silu(gate) * up.
+ *               [SpenseGPT, technical summary §2.A (output-split for W_up
+ *                and W_gate, input-split for W_down in GLU MLPs) and §2.B
+ *                (intermediate indices can be permuted without changing the
+ *                result; the dense ones are moved into one contiguous block)]
  *  8. fp8       8-bit (E4M3) variant: the dense operand is quantised per row
  *               (token) and lifted, the sparse operand's kept values are
  *               quantised per row (output channel), the sparse metadata takes
@@ -383,6 +394,23 @@ void or_colnorm_f64(const void *w, int dt, int64_t O, int64_t K, double *colnorm
             double v = value_at(w, dt, r * K + c);
             colnorm[c] += v * v;
         }
+}
+
+/* Step 7'a.  rownorm[r] = sum_{k ascending} w[r][k]^2 in fp64. */
+void or_rownorm_f64(const void *w, int dt, int64_t O, int64_t K, double *rownorm) {
+    for (int64_t r = 0; r < O; ++r) {
+        double s = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            const double v = value_at(w, dt, r * K + k);
+            s += v * v;
+        }
+        rownorm[r] = s;
+    }
+}
+
+/* Step 7'b.  silu(z) = z / (1 + e^-z), elementwise in fp64. */
+void or_silu_f64(const double *z, int64_t n, double *out) {
+    for (int64_t i = 0; i < n; ++i) out[i] = z[i] / (1.0 + exp(-z[i]));
 }
 
 /* Number of dense columns for a dense share f of K: 4 * floor(f * K / 4), so
