@@ -95,6 +95,28 @@ typedef struct {
     int64_t O, K, K_dense;
 } nm_hybrid_weight;
 
+/* A GLU MLP y = (silu(x . W_gate^T) * (x . W_up^T)) . W_down^T in the
+ * hybrid format (device buffers owned by the caller, filled by
+ * spense_mlp_prepare()).  W_up, W_gate are [I x d], W_down is [d x I]; D of
+ * the I intermediate indices stay dense (Is = I - D are 2:4).
+ *   perm      : int32 [I] = [sparse indices ascending | dense ascending]
+ *   ug_vals   : bf16 [2 Is][d/2], rows [up_s; gate_s] 2:4-compressed along d
+ *   ug_meta   : nm_meta_bytes(2 Is, d, 4) bytes
+ *   ug_dense  : bf16 [2 D][d], rows [up_d; gate_d]
+ *   down_vals : bf16 [d][Is/2], W_down's sparse input columns (permuted order)
+ *   down_meta : nm_meta_bytes(d, Is, 4) bytes
+ *   down_dense: bf16 [d][D], W_down's dense input columns (permuted order) */
+typedef struct {
+    int32_t *perm;
+    void *ug_vals;
+    void *ug_meta;
+    void *ug_dense;
+    void *down_vals;
+    void *down_meta;
+    void *down_dense;
+    int64_t d, I, D;
+} nm_spense_mlp;
+
 /* ------------------------------------------------------------------ sizes */
 
 /* Lifted width K' = K*(M-2)/(M/2) for even M >= 4 (K' = K for M = 4);
@@ -234,11 +256,36 @@ int hybrid_prepare(const void *w, int64_t O, int64_t K, double dense_frac, nm_hy
                    void *ws, size_t ws_bytes, void *stream);
 
 /* Y [B x O] = X[:, perm_s] . W_s^T + X[:, perm_d] . W_d^T (input-split, one
- * fp32 accumulator) for X bf16 [B x K] (row stride K).
- * ws: hybrid_gemm_workspace_size(W, B) bytes. */
+ * fp32 accumulator) for X bf16 [B x K] (row stride K).  With W->perm NULL,
+ * X is taken as already permuted ([sparse columns | dense columns]) and no
+ * gather runs.  ws: hybrid_gemm_workspace_size(W, B) bytes. */
 size_t hybrid_gemm_workspace_size(const nm_hybrid_weight *W, int64_t B);
 int hybrid_gemm(const void *X, int64_t B, const nm_hybrid_weight *W, void *Y, nm_dtype out_dt,
                 void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------- hybrid GLU MLP */
+
+/* The GLU mapping of the hybrid format.
+ * [SpenseGPT, technical summary §2.A (output-split for W_up and W_gate,
+ *  input-split for W_down) and §2.B (the intermediate indices can be
+ *  permuted without changing the result; the dense ones are moved into one
+ *  contiguous block).]
+ * Dense count: D = 256 * floor(f * I / 256) (0 for f <= 0, I for f >= 1).
+ * Selection: score[i] = (sum_k up[i][k]^2 + sum_k gate[i][k]^2) +
+ * sum_o down[o][i]^2 in fp64 (each sum in ascending order); index i is dense
+ * iff fewer than D indices beat it (higher score, or equal and lower index).
+ * Requires d % 128 == 0 and I % 256 == 0. */
+int64_t spense_dense_count(int64_t I, double dense_frac);
+size_t spense_mlp_prepare_workspace_size(int64_t d, int64_t I);
+int spense_mlp_prepare(const void *w_up, const void *w_gate, const void *w_down, double dense_frac,
+                       nm_spense_mlp *out, void *ws, size_t ws_bytes, void *stream);
+
+/* y [B x d] = the MLP of x [B x d] (bf16, row stride d): one output-split
+ * GEMM for up and gate, silu(gate) * up in fp32, one input-split GEMM for
+ * down; bf16 intermediates.  ws: spense_mlp_workspace_size(W, B) bytes. */
+size_t spense_mlp_workspace_size(const nm_spense_mlp *W, int64_t B);
+int spense_mlp(const void *X, int64_t B, const nm_spense_mlp *W, void *Y, void *ws, size_t ws_bytes,
+               void *stream);
 
 /* Capacity, in bytes, of the library's built-in scratch array used by
  * hybrid_gemm_noalloc(): the gathered activations need B * K * 2 bytes. */

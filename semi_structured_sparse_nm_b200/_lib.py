@@ -33,6 +33,12 @@ class SparseOperand(ctypes.Structure):
                 ("K_lift", ctypes.c_int64)]
 
 
+class SpenseMlpStruct(ctypes.Structure):
+    _fields_ = [("perm", ctypes.c_void_p), ("ug_vals", ctypes.c_void_p), ("ug_meta", ctypes.c_void_p),
+                ("ug_dense", ctypes.c_void_p), ("down_vals", ctypes.c_void_p), ("down_meta", ctypes.c_void_p),
+                ("down_dense", ctypes.c_void_p), ("d", ctypes.c_int64), ("I", ctypes.c_int64), ("D", ctypes.c_int64)]
+
+
 class HybridWeight(ctypes.Structure):
     _fields_ = [("perm", ctypes.c_void_p), ("vals_s", ctypes.c_void_p), ("meta_s", ctypes.c_void_p),
                 ("W_d", ctypes.c_void_p), ("O", ctypes.c_int64), ("K", ctypes.c_int64),
@@ -70,6 +76,11 @@ def lib():
             "hybrid_gemm_workspace_size": (SZ, [ctypes.POINTER(HybridWeight), I64]),
             "hybrid_gemm": (I, [P, I64, ctypes.POINTER(HybridWeight), P, I, P, SZ, P]),
             "hybrid_gemm_noalloc": (I, [P, I64, ctypes.POINTER(HybridWeight), P, I, P]),
+            "spense_dense_count": (I64, [I64, D]),
+            "spense_mlp_prepare_workspace_size": (SZ, [I64, I64]),
+            "spense_mlp_prepare": (I, [P, P, P, D, ctypes.POINTER(SpenseMlpStruct), P, SZ, P]),
+            "spense_mlp_workspace_size": (SZ, [ctypes.POINTER(SpenseMlpStruct), I64]),
+            "spense_mlp": (I, [P, I64, ctypes.POINTER(SpenseMlpStruct), P, P, SZ, P]),
             "nm_status_string": (ctypes.c_char_p, [I]),
             "nm_last_cuda_error": (I, []),
             "nm_get_device_error": (I, [P]),
@@ -374,3 +385,67 @@ def device_error(stream=None) -> int:
 
 def debug_expire_wait(timeout_us: int):
     _check("nm_debug_expire_wait", lib().nm_debug_expire_wait(timeout_us, _stream()))
+
+
+# ------------------------------------------------------- hybrid GLU MLP
+
+
+class SpenseMlp:
+    """A GLU MLP in the hybrid format (device buffers)."""
+
+    def __init__(self, perm, ug_vals, ug_meta, ug_dense, down_vals, down_meta, down_dense, d, I, D):
+        self.perm, self.ug_vals, self.ug_meta, self.ug_dense = perm, ug_vals, ug_meta, ug_dense
+        self.down_vals, self.down_meta, self.down_dense = down_vals, down_meta, down_dense
+        self.d, self.I, self.D = d, I, D
+
+    def struct(self) -> SpenseMlpStruct:
+        return SpenseMlpStruct(_p(self.perm), _p(self.ug_vals), _p(self.ug_meta), _p(self.ug_dense),
+                               _p(self.down_vals), _p(self.down_meta), _p(self.down_dense), self.d, self.I, self.D)
+
+
+def spense_dense_count(I: int, dense_frac: float) -> int:
+    return int(lib().spense_dense_count(I, dense_frac))
+
+
+def spense_mlp_prepare(w_up: torch.Tensor, w_gate: torch.Tensor, w_down: torch.Tensor,
+                       dense_frac: float) -> SpenseMlp:
+    """Offline: dense intermediate set, permutation, packed up/gate (output
+    split) and down (input split)."""
+    _need_cuda(w_up, w_gate, w_down)
+    I, d = w_up.shape
+    if w_gate.shape != (I, d) or w_down.shape != (d, I):
+        raise ValueError("expected W_up, W_gate [I, d] and W_down [d, I]")
+    for t in (w_up, w_gate, w_down):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("contiguous bf16 weights expected")
+    D = spense_dense_count(I, dense_frac)
+    Is = I - D
+    dev = w_up.device
+    e = lambda *shape, dt=torch.bfloat16: torch.empty(shape, dtype=dt, device=dev)
+    W = SpenseMlp(e(I, dt=torch.int32),
+                  e(2 * Is, d // 2) if Is else None, e(max(meta_bytes(2 * Is, d, 4), 16), dt=torch.uint8) if Is else None,
+                  e(2 * D, d) if D else None,
+                  e(d, Is // 2) if Is else None, e(max(meta_bytes(d, Is, 4), 16), dt=torch.uint8) if Is else None,
+                  e(d, D) if D else None, d, I, D)
+    ws_bytes = int(lib().spense_mlp_prepare_workspace_size(d, I))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = W.struct()
+    _check("spense_mlp_prepare", lib().spense_mlp_prepare(_p(w_up), _p(w_gate), _p(w_down), dense_frac,
+                                                          ctypes.byref(st), _p(ws), ws_bytes, _stream(w_up)))
+    return W
+
+
+def spense_mlp(x: torch.Tensor, W: SpenseMlp, out: torch.Tensor | None = None, ws=None) -> torch.Tensor:
+    """y = (silu(x . W_gate^T) * (x . W_up^T)) . W_down^T through the packed weights."""
+    _need_cuda(x)
+    B = x.shape[0]
+    if x.dtype != torch.bfloat16 or x.shape[1] != W.d or not x.is_contiguous():
+        raise ValueError("x must be contiguous bf16 [B, d]")
+    if out is None:
+        out = torch.empty((B, W.d), dtype=torch.bfloat16, device=x.device)
+    st = W.struct()
+    ws_bytes = int(lib().spense_mlp_workspace_size(ctypes.byref(st), B))
+    if ws is None:
+        ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=x.device)
+    _check("spense_mlp", lib().spense_mlp(_p(x), B, ctypes.byref(st), _p(out), _p(ws), ws_bytes, _stream(x)))
+    return out

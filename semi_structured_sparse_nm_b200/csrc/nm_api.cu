@@ -17,6 +17,7 @@
 #include "nm_gemm2.cuh"
 #include "nm_prune.cuh"
 #include "nm_fp8.cuh"
+#include "nm_mlp.cuh"
 #include "nmsparse.h"
 
 namespace {
@@ -102,6 +103,7 @@ struct GemmPlan {
   int64_t ldy = 0;
   int out_fp32 = 0, transpose = 0;
   int a_static = 0;           // A is a weight: may be read before the preceding kernel ends
+  int64_t out_split_rows = -1;  // output-split: A rows [0, this) sparse (a_s), the rest dense (a_d)
   int fp8 = 0;                // 8-bit (E4M3) operands, rescaled by scale_a[row] * scale_b[column]
   const float* scale_a = nullptr;
   const float* scale_b = nullptr;
@@ -114,15 +116,21 @@ int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
   const int64_t kb_sparse = ceil_div(p.ks_lift, 128);
   const int64_t kb_dense = ceil_div(p.kd, 64);
   int rc;
-  if (kb_sparse > 0) {
-    if ((rc = make_tmap(&ta_s, p.a_s, p.ks_lift / 2, p.rows_a, p.ks_lift, 64, nm::kBM)) != NM_OK) return rc;
+  // output-split: the sparse and the dense A are separate matrices over the
+  // same B columns [0, K)
+  const bool osplit = p.out_split_rows >= 0;
+  const int64_t rows_s = osplit ? p.out_split_rows : p.rows_a;
+  const int64_t rows_d = osplit ? p.rows_a - p.out_split_rows : p.rows_a;
+  const int64_t b_cols = osplit ? p.ks_lift : p.ks_lift + p.kd;
+  if (kb_sparse > 0 && rows_s > 0) {
+    if ((rc = make_tmap(&ta_s, p.a_s, p.ks_lift / 2, rows_s, p.ks_lift, 64, nm::kBM)) != NM_OK) return rc;
   }
-  if (kb_dense > 0) {
-    if ((rc = make_tmap(&ta_d, p.a_d, p.kd, p.rows_a, p.kd * 2, 64, nm::kBM)) != NM_OK) return rc;
+  if (kb_dense > 0 && rows_d > 0) {
+    if ((rc = make_tmap(&ta_d, p.a_d, p.kd, rows_d, p.kd * 2, 64, nm::kBM)) != NM_OK) return rc;
   }
-  if (kb_sparse == 0) ta_s = ta_d;
-  if (kb_dense == 0) ta_d = ta_s;
-  if ((rc = make_tmap(&tb, p.b, p.ks_lift + p.kd, p.rows_b, (p.ks_lift + p.kd) * 2, 64, BN)) != NM_OK) return rc;
+  if (kb_sparse == 0 || rows_s == 0) ta_s = ta_d;
+  if (kb_dense == 0 || rows_d == 0) ta_d = ta_s;
+  if ((rc = make_tmap(&tb, p.b, b_cols, p.rows_b, b_cols * 2, 64, BN)) != NM_OK) return rc;
 
   nm::GemmArgs args{};
   args.rows_a = p.rows_a;
@@ -138,6 +146,8 @@ int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
   args.transpose_out = p.transpose;
   args.splits = splits;
   args.a_static = p.a_static;
+  args.out_split_tiles = osplit ? static_cast<int>(p.out_split_rows / nm::kBM) : -1;
+  if (osplit) args.k_dense_x0 = 0;
 
   auto kern = nm::k_nm_gemm<BN>;
   NM_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
@@ -333,7 +343,8 @@ int pick_splits(int64_t tiles, int64_t kb_total) {
 int run_gemm(const GemmPlan& p, cudaStream_t st) {
   const char* env = std::getenv("NMSPARSE_GEMM");
   const std::string mode = env != nullptr ? env : "auto";
-  const bool eligible2 = (p.ks_lift + p.kd) > 0 && p.rows_a % 256 == 0 && (p.kd == 0 || p.ks_lift % 128 == 0);
+  const bool eligible2 = p.out_split_rows < 0 && (p.ks_lift + p.kd) > 0 && p.rows_a % 256 == 0 &&
+                         (p.kd == 0 || p.ks_lift % 128 == 0);
   const bool eligible4 = eligible2 && p.rows_a % 512 == 0;
   if (eligible2 && mode != "1cta") {
     if (mode == "2cta224") return launch_gemm_2cta<224, 2, 1>(p, st);
@@ -750,7 +761,7 @@ size_t hybrid_gemm_workspace_size(const nm_hybrid_weight* W, int64_t B) {
 
 int hybrid_gemm(const void* X, int64_t B, const nm_hybrid_weight* W, void* Y, nm_dtype out_dt, void* ws,
                 size_t ws_bytes, void* stream) {
-  if (X == nullptr || W == nullptr || Y == nullptr || W->perm == nullptr) return NM_ERR_INVALID_ARG;
+  if (X == nullptr || W == nullptr || Y == nullptr) return NM_ERR_INVALID_ARG;
   if (out_dt != NM_BF16 && out_dt != NM_FP32) return NM_ERR_INVALID_ARG;
   if (B < 0 || W->O <= 0 || W->K <= 0 || W->K_dense < 0 || W->K_dense > W->K || W->K % 8 != 0)
     return NM_ERR_INVALID_ARG;
@@ -759,16 +770,21 @@ int hybrid_gemm(const void* X, int64_t B, const nm_hybrid_weight* W, void* Y, nm
   if (Ks > 0 && (W->vals_s == nullptr || W->meta_s == nullptr)) return NM_ERR_INVALID_ARG;
   if (W->K_dense > 0 && W->W_d == nullptr) return NM_ERR_INVALID_ARG;
   if (B == 0) return NM_OK;
-  if (ws == nullptr || ws_bytes < hybrid_gemm_workspace_size(W, B)) return NM_ERR_WORKSPACE;
-  if (!aligned16(X) || !aligned16(Y) || !aligned16(ws) || (Ks > 0 && !aligned16(W->vals_s)) ||
+  const bool gather = W->perm != nullptr;
+  if (gather && (ws == nullptr || ws_bytes < hybrid_gemm_workspace_size(W, B))) return NM_ERR_WORKSPACE;
+  if (!aligned16(X) || !aligned16(Y) || (gather && !aligned16(ws)) || (Ks > 0 && !aligned16(W->vals_s)) ||
       (W->K_dense > 0 && !aligned16(W->W_d)))
     return NM_ERR_ALIGNMENT;
   auto st = static_cast<cudaStream_t>(stream);
-  uint16_t* xp = static_cast<uint16_t*>(ws);
-  const int64_t gblocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(B * W->K, 256), int64_t(num_sms()) * 4));
-  NM_CUDA_TRY(launch_pdl(nm::k_gather_cols, dim3(static_cast<unsigned>(gblocks)), dim3(256), 0, st,
-                         static_cast<const uint16_t*>(X), B, W->K, static_cast<const int32_t*>(W->perm), W->K, xp,
-                         static_cast<uint16_t*>(nullptr)));
+  const uint16_t* xp = static_cast<const uint16_t*>(X);
+  if (gather) {
+    uint16_t* g = static_cast<uint16_t*>(ws);
+    const int64_t gblocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(B * W->K, 256), int64_t(num_sms()) * 4));
+    NM_CUDA_TRY(launch_pdl(nm::k_gather_cols, dim3(static_cast<unsigned>(gblocks)), dim3(256), 0, st,
+                           static_cast<const uint16_t*>(X), B, W->K, static_cast<const int32_t*>(W->perm), W->K, g,
+                           static_cast<uint16_t*>(nullptr)));
+    xp = g;
+  }
   GemmPlan p;
   p.a_s = W->vals_s;
   p.a_d = W->W_d;
@@ -784,6 +800,133 @@ int hybrid_gemm(const void* X, int64_t B, const nm_hybrid_weight* W, void* Y, nm
   p.transpose = 1;
   p.a_static = 1;
   return run_gemm(p, st);
+}
+
+// --------------------------------------------------------- hybrid GLU MLP
+
+int64_t spense_dense_count(int64_t I, double dense_frac) {
+  if (I <= 0 || dense_frac <= 0.0) return 0;
+  if (dense_frac >= 1.0) return I;
+  return 256 * static_cast<int64_t>((dense_frac * static_cast<double>(I)) / 256.0);
+}
+
+size_t spense_mlp_prepare_workspace_size(int64_t d, int64_t I) {
+  if (d <= 0 || I <= 0) return 0;
+  const int64_t vec = ceil_div(I * 8, int64_t(256)) * 256;                 // one fp64 vector of I
+  const int64_t flags = ceil_div(I, int64_t(256)) * 256;
+  const int64_t ug = ceil_div(2 * I * d * 2, int64_t(256)) * 256;          // gathered sparse up/gate rows
+  const int64_t dn = ceil_div(d * I * 2, int64_t(256)) * 256;              // gathered sparse down columns
+  return static_cast<size_t>(4 * vec + flags + ug + dn);
+}
+
+int spense_mlp_prepare(const void* w_up, const void* w_gate, const void* w_down, double dense_frac,
+                       nm_spense_mlp* out, void* ws, size_t ws_bytes, void* stream) {
+  if (w_up == nullptr || w_gate == nullptr || w_down == nullptr || out == nullptr || out->perm == nullptr)
+    return NM_ERR_INVALID_ARG;
+  const int64_t d = out->d, I = out->I, D = spense_dense_count(I, dense_frac), Is = I - D;
+  if (d <= 0 || I <= 0 || out->D != D) return NM_ERR_INVALID_ARG;
+  if (d % 128 != 0 || I % 256 != 0) return NM_ERR_UNSUPPORTED;
+  if (Is > 0 && (out->ug_vals == nullptr || out->ug_meta == nullptr || out->down_vals == nullptr ||
+                 out->down_meta == nullptr))
+    return NM_ERR_INVALID_ARG;
+  if (D > 0 && (out->ug_dense == nullptr || out->down_dense == nullptr)) return NM_ERR_INVALID_ARG;
+  if (ws == nullptr || ws_bytes < spense_mlp_prepare_workspace_size(d, I)) return NM_ERR_WORKSPACE;
+  if (!aligned16(w_up) || !aligned16(w_gate) || !aligned16(w_down) || !aligned16(ws) || !aligned16(out->perm) ||
+      (Is > 0 && (!aligned16(out->ug_vals) || !aligned16(out->ug_meta) || !aligned16(out->down_vals) ||
+                  !aligned16(out->down_meta))) ||
+      (D > 0 && (!aligned16(out->ug_dense) || !aligned16(out->down_dense))))
+    return NM_ERR_ALIGNMENT;
+  auto st = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const int64_t vec = ceil_div(I * 8, int64_t(256)) * 256;
+  double* rn_up = reinterpret_cast<double*>(base);
+  double* rn_gate = reinterpret_cast<double*>(base + vec);
+  double* cn_down = reinterpret_cast<double*>(base + 2 * vec);
+  double* score = reinterpret_cast<double*>(base + 3 * vec);
+  uint8_t* is_dense = base + 4 * vec;
+  uint16_t* ug_sp = reinterpret_cast<uint16_t*>(is_dense + ceil_div(I, int64_t(256)) * 256);
+  uint16_t* dn_sp = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(ug_sp) +
+                                                ceil_div(2 * I * d * 2, int64_t(256)) * 256);
+  const auto* up = static_cast<const uint16_t*>(w_up);
+  const auto* gate = static_cast<const uint16_t*>(w_gate);
+  const auto* down = static_cast<const uint16_t*>(w_down);
+  const unsigned ib = static_cast<unsigned>(ceil_div(I, int64_t(128)));
+  NM_CUDA_TRY(launch_pdl(nm::k_rownorm_f64, dim3(ib), dim3(128), 0, st, up, I, d, rn_up));
+  NM_CUDA_TRY(launch_pdl(nm::k_rownorm_f64, dim3(ib), dim3(128), 0, st, gate, I, d, rn_gate));
+  NM_CUDA_TRY(launch_pdl(nm::k_colnorm_f64, dim3(ib), dim3(128), 0, st, down, d, I, cn_down));
+  NM_CUDA_TRY(launch_pdl(nm::k_add3_f64, dim3(ib), dim3(128), 0, st, static_cast<const double*>(rn_up),
+                         static_cast<const double*>(rn_gate), static_cast<const double*>(cn_down), I, score));
+  NM_CUDA_TRY(launch_pdl(nm::k_hybrid_rank, dim3(ib), dim3(128), 0, st, static_cast<const double*>(score), I, D,
+                         is_dense));
+  NM_CUDA_TRY(launch_pdl(nm::k_hybrid_perm, dim3(ib), dim3(128), 0, st, static_cast<const uint8_t*>(is_dense), I,
+                         D, out->perm));
+  const unsigned gb = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(ceil_div(2 * I * (d / 8), int64_t(256)),
+                                                                                   int64_t(num_sms()) * 16)));
+  NM_CUDA_TRY(launch_pdl(nm::k_gather_rows_ug, dim3(gb), dim3(256), 0, st, up, gate, d,
+                         static_cast<const int32_t*>(out->perm), I, Is, ug_sp,
+                         static_cast<uint16_t*>(out->ug_dense)));
+  const unsigned cb = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(ceil_div(d * I, int64_t(256)),
+                                                                                   int64_t(num_sms()) * 16)));
+  NM_CUDA_TRY(launch_pdl(nm::k_gather_cols, dim3(cb), dim3(256), 0, st, down, d, I,
+                         static_cast<const int32_t*>(out->perm), Is, dn_sp, static_cast<uint16_t*>(out->down_dense)));
+  int rc;
+  if (Is > 0) {
+    if ((rc = launch_prune(static_cast<const uint16_t*>(ug_sp), 2 * Is, d, d, 2, 4, nullptr, out->ug_vals,
+                           out->ug_meta, st)) != NM_OK)
+      return rc;
+    if ((rc = launch_prune(static_cast<const uint16_t*>(dn_sp), d, Is, Is, 2, 4, nullptr, out->down_vals,
+                           out->down_meta, st)) != NM_OK)
+      return rc;
+  }
+  return NM_OK;
+}
+
+size_t spense_mlp_workspace_size(const nm_spense_mlp* W, int64_t B) {
+  if (W == nullptr || B <= 0 || W->I <= 0) return 0;
+  return static_cast<size_t>(ceil_div(B * 2 * W->I * 2, int64_t(256)) * 256 + ceil_div(B * W->I * 2, int64_t(256)) * 256);
+}
+
+int spense_mlp(const void* X, int64_t B, const nm_spense_mlp* W, void* Y, void* ws, size_t ws_bytes, void* stream) {
+  if (X == nullptr || W == nullptr || Y == nullptr) return NM_ERR_INVALID_ARG;
+  const int64_t d = W->d, I = W->I, D = W->D, Is = I - D;
+  if (B < 0 || d <= 0 || I <= 0 || D < 0 || D > I) return NM_ERR_INVALID_ARG;
+  if (d % 128 != 0 || I % 256 != 0 || D % 256 != 0) return NM_ERR_UNSUPPORTED;
+  if (B == 0) return NM_OK;
+  if (ws == nullptr || ws_bytes < spense_mlp_workspace_size(W, B)) return NM_ERR_WORKSPACE;
+  if (!aligned16(X) || !aligned16(Y) || !aligned16(ws)) return NM_ERR_ALIGNMENT;
+  auto st = static_cast<cudaStream_t>(stream);
+  uint16_t* y_ug = static_cast<uint16_t*>(ws);
+  uint16_t* h = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + ceil_div(B * 2 * I * 2, int64_t(256)) * 256);
+  // up and gate: one output-split product, columns [up_s | gate_s | up_d | gate_d]
+  GemmPlan p;
+  p.a_s = W->ug_vals;
+  p.a_d = W->ug_dense;
+  p.meta = static_cast<const uint8_t*>(W->ug_meta);
+  p.b = X;
+  p.rows_a = 2 * I;
+  p.rows_b = B;
+  p.ks_lift = d;
+  p.kd = d;
+  p.out_split_rows = 2 * Is;
+  p.y = y_ug;
+  p.ldy = 2 * I;
+  p.transpose = 1;
+  p.a_static = 1;
+  int rc;
+  if ((rc = run_gemm(p, st)) != NM_OK) return rc;
+  const unsigned sb = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(ceil_div(B * (I / 8), int64_t(256)),
+                                                                                   int64_t(num_sms()) * 8)));
+  NM_CUDA_TRY(launch_pdl(nm::k_silu_mul, dim3(sb), dim3(256), 0, st, static_cast<const uint16_t*>(y_ug), B, I, Is, h));
+  // down: input-split on h, which is already in the permuted order
+  nm_hybrid_weight dw{};
+  dw.perm = nullptr;
+  dw.vals_s = W->down_vals;
+  dw.meta_s = W->down_meta;
+  dw.W_d = W->down_dense;
+  dw.O = d;
+  dw.K = I;
+  dw.K_dense = D;
+  return hybrid_gemm(h, B, &dw, Y, NM_BF16, nullptr, 0, stream);
 }
 
 }  // extern "C"

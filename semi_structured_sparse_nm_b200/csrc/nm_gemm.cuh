@@ -8,7 +8,11 @@
 //   dense : A = 128 rows x 64 bf16, B = BN rows x 64 bf16; 4 x tcgen05.mma (K=16)
 // Sparse k-blocks come first (they cover B columns [0, K's)), then the dense
 // ones (B columns K's + 64*kd ...): this one loop serves the plain sparse
-// GEMM, the dense comparator and the hybrid input-split product.
+// GEMM, the dense comparator and the hybrid input-split product.  In an
+// output-split product (out_split_tiles >= 0) A's first out_split_tiles
+// row tiles are sparse and run the sparse k-blocks only, the rest are dense
+// (rows of the dense A matrix from 0) and run the dense k-blocks only, both
+// over B columns [0, K); dense tiles are scheduled first (they are longer).
 //
 // Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and
 // MMA issuer, warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4)..).
@@ -41,6 +45,8 @@ struct GemmArgs {
   int splits;                               // CTAs per output tile (cluster size)
   int a_static;                             // A (and its metadata) may be read before the
                                             // preceding kernel finishes; B only after
+  int out_split_tiles;                      // -1, or the number of sparse row tiles of an
+                                            // output-split product
 };
 
 template <int BN>
@@ -172,11 +178,19 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t m_tile = blockIdx.x, n_tile = blockIdx.y;
+  const int64_t tiles_m = gridDim.x;
+  const int tsp = args.out_split_tiles;
+  // output-split: dense tiles (the longer ones) take the first blocks
+  const int64_t m_tile = tsp < 0 ? blockIdx.x
+                                 : (blockIdx.x < tiles_m - tsp ? tsp + blockIdx.x : blockIdx.x - (tiles_m - tsp));
+  const int64_t n_tile = blockIdx.y;
+  const bool dense_tile = tsp >= 0 && m_tile >= tsp;
   const int split = static_cast<int>(blockIdx.z);
-  const int kb_total = args.kb_sparse + args.kb_dense;
-  const int kb_begin = static_cast<int>(static_cast<int64_t>(kb_total) * split / args.splits);
-  const int kb_end = static_cast<int>(static_cast<int64_t>(kb_total) * (split + 1) / args.splits);
+  const int kb_lo = dense_tile ? args.kb_sparse : 0;
+  const int kb_hi = tsp < 0 ? args.kb_sparse + args.kb_dense : (dense_tile ? args.kb_sparse + args.kb_dense : args.kb_sparse);
+  const int kb_total = kb_hi - kb_lo;
+  const int kb_begin = kb_lo + static_cast<int>(static_cast<int64_t>(kb_total) * split / args.splits);
+  const int kb_end = kb_lo + static_cast<int>(static_cast<int64_t>(kb_total) * (split + 1) / args.splits);
 
   const bool push = Cfg::kPush && args.splits > 1;
   if (threadIdx.x == 0) {
@@ -205,7 +219,8 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
   if (warp == 0) {
     // ---------------------------------------------------------- producer
     if (elect_one()) {
-      const int32_t y_a = static_cast<int32_t>(m_tile * kBM), y_b = static_cast<int32_t>(n_tile * BN);
+      const int32_t y_a = static_cast<int32_t>((dense_tile ? m_tile - tsp : m_tile) * kBM);
+      const int32_t y_b = static_cast<int32_t>(n_tile * BN);
       auto load_a = [&](int kb, int s) {
         uint8_t* a_dst = sA + s * kABytes;
         if (kb < args.kb_sparse) {
