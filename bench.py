@@ -6,7 +6,9 @@ One step = one pass of the hot path over one batch of synthetic input:
   weight sparsity (6:8 sliding windows): lift X online, then the sparse GEMM
       against the offline-decomposed weight;
   hybrid dense + 2:4 weight (decode): gather X by the column permutation and
-      one input-split GEMM.
+      one input-split GEMM;
+  hybrid GLU MLP (decode): one output-split GEMM for up and gate, the SiLU
+      gate, one input-split GEMM for down.
 The headline line is the Llama-8B up_proj prefill shape with 8:16 activation
 sparsity (X [2048 x 4096] Student-t, W [14336 x 4096] N(0, 0.02), bf16, fp32
 accumulation, bf16 out); the other workloads are reported under "workloads".
@@ -45,6 +47,7 @@ TRAFFIC = {
 OTHERS = ["up_proj_2of4_act", "up_proj_8of16_act_fp8", "down_proj_16of32_act", "slide_6of8_wt_prefill", "slide_6of8_wt_prefill_fp8",
           "slide_6of8_wt_decode",
           "hybrid_decode_b1", "hybrid_decode_b8", "hybrid_decode_b32", "hybrid_decode_b128",
+          "spense_mlp_decode_b1", "spense_mlp_decode_b8", "spense_mlp_decode_b32", "spense_mlp_decode_b128",
           "tiny_2of4_act_fp32"]
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "N:M sparse linear TFLOP/s (dense-equiv)"
@@ -264,6 +267,22 @@ class Workload:
             self.rows_a, self.rows_b = wl.O, wl.T
             self.prep_name, self.gemm_name = "lift", "sparse_gemm"
             self.w_bytes = wbytes
+        elif wl.side == "mlp":
+            _, g_np, d_np = inputs.make_mlp_weights(wl, seed=0)
+            S = nm.spense_mlp_prepare(W, to_dev(g_np), to_dev(d_np), wl.dense_frac)   # offline
+            self.g_np, self.d_np = g_np, d_np
+            parts = [S.ug_vals, S.ug_meta, S.ug_dense, S.down_vals, S.down_meta, S.down_dense]
+            wbytes = sum(t.numel() * t.element_size() for t in parts if t is not None)
+            self.R = max(2, int(np.ceil(2 * L2_BYTES / wbytes)))
+            cl = lambda t: None if t is None else t.clone()
+            self.S = [S] + [nm.SpenseMlp(S.perm, *[cl(t) for t in parts], S.d, S.I, S.D) for _ in range(1, self.R)]
+            self.X = [X0.roll(r, dims=0).contiguous() if r else X0 for r in range(self.R)]
+            self.Y = torch.empty((wl.T, wl.K), dtype=out_dt, device=dev)
+            self.ws = torch.empty(max(16, nm.spense_mlp_workspace_size(S, wl.T)), dtype=torch.uint8, device=dev)
+            self.rows_a, self.rows_b = 2 * wl.O, wl.T
+            self.prep_name, self.gemm_name = "none", "spense_mlp"
+            self.w_bytes = wbytes
+            self.launches_per_step = 3                               # up/gate GEMM, SiLU gate, down GEMM
         else:
             H = nm.hybrid_prepare(W, wl.dense_frac)                      # offline
             wbytes = H.vals_s.numel() * 2 + H.meta_s.numel() + H.W_d.numel() * 2
@@ -308,6 +327,10 @@ class Workload:
             if mark:
                 mark()
             nm.sparse_gemm(self.Wc[r], xl, nm.NM_WEIGHT, self.Y.dtype, out=self.Y)
+        elif wl.side == "mlp":
+            if mark:
+                mark()
+            nm.spense_mlp(self.X[r], self.S[r], out=self.Y, ws=self.ws)
         else:
             if mark:
                 mark()
@@ -324,6 +347,8 @@ class Workload:
             nm.sparse_gemm_fp8(self.P[r], self.Q[0], nm.NM_WEIGHT, self.Y.dtype, out=self.Y)
         elif wl.side == "weight":
             nm.sparse_gemm(self.Wc[r], self.Xl[0], nm.NM_WEIGHT, self.Y.dtype, out=self.Y)
+        elif wl.side == "mlp":
+            nm.spense_mlp(self.X[r], self.S[r], out=self.Y, ws=self.ws)
         else:
             nm.hybrid_gemm(self.X[r], self.H[r], self.Y.dtype, out=self.Y, ws=self.ws)
 
@@ -331,7 +356,13 @@ class Workload:
         """(dense-equiv flops, sparse-MMA flops, bytes of the GEMM) per step."""
         wl = self.wl
         dense = 2.0 * wl.T * wl.O * wl.K
-        if wl.side == "hybrid":
+        if wl.side == "mlp":
+            # three projections; bytes: packed weights, x in, y out, the
+            # up/gate product written and read, h written and read
+            dense = 3.0 * dense
+            mma = dense
+            byts = (self.w_bytes + 2 * wl.T * wl.K * 2 + 2 * wl.T * 2 * wl.O * 2 + 2 * wl.T * wl.O * 2)
+        elif wl.side == "hybrid":
             D = self.H[0].K_dense
             Ks = wl.K - D
             mma = 2.0 * wl.T * wl.O * (Ks + D)          # sparse part counted at its 2:4 rate
@@ -479,6 +510,44 @@ def time_dense_fp8(wk, reps=10):
         return None
 
 
+def time_dense_mlp(wk, reps=20):
+    """The same GLU MLP unpruned, on cuBLAS (torch.matmul) and torch's SiLU,
+    replayed from a CUDA graph: library context for the decode MLP.  The
+    three dense weights (3 x O x K bf16) exceed 2x L2 by themselves.  Returns
+    ms per MLP."""
+    import torch
+    dev = wk.dev
+    bf = lambda a: torch.from_numpy(a).view(torch.bfloat16).to(dev)
+    Wu, Wg, Wd = bf(wk.w_np), bf(wk.g_np), bf(wk.d_np)
+    x = wk.X[0]
+
+    def fn():
+        u = torch.matmul(x, Wu.t())
+        g = torch.matmul(x, Wg.t())
+        return torch.matmul(torch.nn.functional.silu(g) * u, Wd.t())
+
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            fn()
+    torch.cuda.current_stream(dev).wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    del g, Wu, Wg, Wd
+    return e0.elapsed_time(e1) / reps
+
+
 def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None):
     dense, mma, byts = wk.algorithmic()
     wl = wk.wl
@@ -489,6 +558,15 @@ def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None):
                    "K_lift": wl.K_lift, "rotated_buffers": wk.R},
         "kernels": {f"{wk.prep_name}_us": prep_ms * 1e3, f"{wk.gemm_name}_us": gemm_ms * 1e3},
     }
+    if wl.side == "mlp":
+        out["config"].update(d=wl.K, I=wl.O, dense_frac=wl.dense_frac, D=wk.S[0].D)
+        out["kernels"] = {"spense_mlp_us": step_ms * 1e3,
+                          "note": "one MLP = three launches (up/gate output-split GEMM, SiLU gate, "
+                                  "down input-split GEMM) replayed from a CUDA graph"}
+        cb = time_dense_mlp(wk)
+        out["dense_comparator"] = {"cublas_mlp_us": cb * 1e3, "speedup_vs_cublas": cb / step_ms,
+                                   "note": "the same MLP unpruned: three cuBLAS GEMMs and torch's SiLU and "
+                                           "product, bf16, from a CUDA graph; library context only"}
     if getattr(wk, "instrumented_step_ms", None) is not None:
         out["kernels"]["note"] = ("per-kernel times from a second pass of the same steps with an event around "
                                   "each kernel; that pass's step: %.2f us" % (wk.instrumented_step_ms * 1e3))
@@ -508,7 +586,8 @@ def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None):
             "note": "same unpruned product X . W^T, bf16, fp32 accumulate; cuBLAS is context only"}
     if wk.decode:
         achieved = byts / (gemm_ms * 1e-3) / 1e9
-        out["roofline"] = {"bound": "hbm", "kernel": wk.gemm_name, "achieved": achieved, "peak": pk["hbm"],
+        out["roofline"] = {"bound": "hbm", "kernel": wk.gemm_name if wl.side != "mlp" else
+                           "spense_mlp (its three launches together)", "achieved": achieved, "peak": pk["hbm"],
                            "unit": "GB/s", "frac": achieved / pk["hbm"], "traffic": traffic,
                            "bytes_per_launch": byts,
                            "peak_note": f"{pk['source']} HBM copy bandwidth"}

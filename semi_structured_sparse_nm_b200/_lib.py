@@ -435,6 +435,11 @@ def spense_mlp_prepare(w_up: torch.Tensor, w_gate: torch.Tensor, w_down: torch.T
     return W
 
 
+def spense_mlp_workspace_size(W: SpenseMlp, B: int) -> int:
+    """Bytes of scratch spense_mlp() needs for a batch of B tokens."""
+    return int(lib().spense_mlp_workspace_size(ctypes.byref(W.struct()), B))
+
+
 def spense_mlp(x: torch.Tensor, W: SpenseMlp, out: torch.Tensor | None = None, ws=None) -> torch.Tensor:
     """y = (silu(x . W_gate^T) * (x . W_up^T)) . W_down^T through the packed weights."""
     _need_cuda(x)
@@ -444,7 +449,7 @@ def spense_mlp(x: torch.Tensor, W: SpenseMlp, out: torch.Tensor | None = None, w
     if out is None:
         out = torch.empty((B, W.d), dtype=torch.bfloat16, device=x.device)
     st = W.struct()
-    ws_bytes = int(lib().spense_mlp_workspace_size(ctypes.byref(st), B))
+    ws_bytes = spense_mlp_workspace_size(W, B)
     if ws is None:
         ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=x.device)
     _check("spense_mlp", lib().spense_mlp(_p(x), B, ctypes.byref(st), _p(out), _p(ws), ws_bytes, _stream(x)))

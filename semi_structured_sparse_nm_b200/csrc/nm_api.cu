@@ -256,16 +256,23 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
                         CU_TENSOR_MAP_DATA_TYPE_UINT8)) != NM_OK) return rc;
     tad = ta;
   } else {
-  if (kb > 0) {
-    if ((rc = make_tmap(&ta, p.a_s, p.ks_lift / 2, p.rows_a, p.ks_lift, 64, 128)) != NM_OK) return rc;
-    if ((rc = make_tmap_meta(&te, p.meta, ceil_div(p.rows_a, 128) * kb)) != NM_OK) return rc;
+  // output-split: the 2:4 rows and the dense rows are separate matrices over
+  // the same B columns [0, K)
+  const bool osplit = p.out_split_rows >= 0;
+  const int64_t rows_s = osplit ? p.out_split_rows : p.rows_a;
+  const int64_t rows_d = osplit ? p.rows_a - p.out_split_rows : p.rows_a;
+  const int64_t b_cols = osplit ? p.ks_lift : p.ks_lift + p.kd;
+  const bool has_s = kb > 0 && rows_s > 0, has_d = kb_dense > 0 && rows_d > 0;
+  if (has_s) {
+    if ((rc = make_tmap(&ta, p.a_s, p.ks_lift / 2, rows_s, p.ks_lift, 64, 128)) != NM_OK) return rc;
+    if ((rc = make_tmap_meta(&te, p.meta, ceil_div(rows_s, 128) * kb)) != NM_OK) return rc;
   }
-  if (kb_dense > 0) {
-    if ((rc = make_tmap(&tad, p.a_d, p.kd, p.rows_a, p.kd * 2, 64, 128)) != NM_OK) return rc;
+  if (has_d) {
+    if ((rc = make_tmap(&tad, p.a_d, p.kd, rows_d, p.kd * 2, 64, 128)) != NM_OK) return rc;
   }
-  if (kb == 0) { ta = tad; te = tad; }
-  if (kb_dense == 0) tad = ta;
-  if ((rc = make_tmap(&tb, p.b, p.ks_lift + p.kd, p.rows_b, (p.ks_lift + p.kd) * 2, 64, BN / 2)) != NM_OK) return rc;
+  if (!has_s) { ta = tad; te = tad; }
+  if (!has_d) tad = ta;
+  if ((rc = make_tmap(&tb, p.b, b_cols, p.rows_b, b_cols * 2, 64, BN / 2)) != NM_OK) return rc;
   }
   nm::Gemm2Args a{};
   a.rows_a = p.rows_a;
@@ -277,6 +284,8 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   a.scale_a = p.scale_a;
   a.scale_b = p.scale_b;
   a.last_half = (FP8 && p.ks_lift % 256 != 0) ? 1 : 0;
+  a.out_split_tiles = p.out_split_rows >= 0 ? static_cast<int>(p.out_split_rows / (256 * MSUB)) : -1;
+  if (p.out_split_rows >= 0) a.k_dense_x0 = 0;
   a.tiles_m = static_cast<int>(ceil_div(p.rows_a, 256 * MSUB));
   a.tiles_n = static_cast<int>(ceil_div(p.rows_b, BN));
   a.Y = p.y;
@@ -343,9 +352,13 @@ int pick_splits(int64_t tiles, int64_t kb_total) {
 int run_gemm(const GemmPlan& p, cudaStream_t st) {
   const char* env = std::getenv("NMSPARSE_GEMM");
   const std::string mode = env != nullptr ? env : "auto";
-  const bool eligible2 = p.out_split_rows < 0 && (p.ks_lift + p.kd) > 0 && p.rows_a % 256 == 0 &&
-                         (p.kd == 0 || p.ks_lift % 128 == 0);
-  const bool eligible4 = eligible2 && p.rows_a % 512 == 0;
+  // an output-split product needs whole 256-row tiles on both sides of the split
+  const bool osplit = p.out_split_rows >= 0;
+  const bool eligible2 = (!osplit || p.out_split_rows % 256 == 0) && (p.ks_lift + p.kd) > 0 &&
+                         p.rows_a % 256 == 0 && (p.kd == 0 || p.ks_lift % 128 == 0);
+  const bool eligible4 = eligible2 && !osplit && p.rows_a % 512 == 0;
+  // SM pairs the 2-CTA kernel would occupy with 128-wide tiles
+  const int64_t pairs128 = (p.rows_a / 256) * ceil_div(p.rows_b, int64_t(128));
   if (eligible2 && mode != "1cta") {
     if (mode == "2cta224") return launch_gemm_2cta<224, 2, 1>(p, st);
     if (mode == "2cta192") return launch_gemm_2cta<192, 2, 1>(p, st);
@@ -353,9 +366,11 @@ int run_gemm(const GemmPlan& p, cudaStream_t st) {
     if (mode == "2cta128") return launch_gemm_2cta<128, 2, 1>(p, st);
     if (eligible4 && mode == "2cta224x2") return launch_gemm_2cta<224, 1, 2>(p, st);
     if (eligible4 && mode == "2cta160x2") return launch_gemm_2cta<160, 1, 2>(p, st);
-    // products with dense k-blocks (hybrid, dense comparator) on SM pairs
+    // products with dense k-blocks (hybrid, output-split, dense comparator)
+    // on SM pairs; a narrow product with too few tiles to occupy half of the
+    // SMs runs on single CTAs with split-K instead
     if (p.kd > 0 && p.rows_b >= 512) return launch_gemm_2cta<224, 2, 1>(p, st);
-    if (p.kd > 0 && p.rows_b >= 64) return launch_gemm_2cta<128, 2, 1>(p, st);
+    if (p.kd > 0 && p.rows_b >= 64 && 4 * pairs128 >= num_sms()) return launch_gemm_2cta<128, 2, 1>(p, st);
     if (p.rows_b >= 512 && p.ks_lift >= 512) {
       // Both 2:4 operands stream through shared memory, whose port bounds this
       // kernel well before the tensor pipe does; measured on B200, the 224-wide

@@ -135,7 +135,25 @@ struct Gemm2Args {
   const float* scale_a;   // 8-bit product: per-row scale of A (nullptr: none)
   const float* scale_b;   //                per-row scale of B, i.e. per output column
   int last_half;          // 8-bit product: the last k-block holds only 128 lifted K
+  int out_split_tiles;    // output-split (-1: none): output m-tiles below it are 2:4 rows
+                          // (sparse k-blocks only), the rest dense rows (dense k-blocks
+                          // only, A rows counted from the dense matrix's first row, B from
+                          // column 0)
 };
+
+// One m-tile's place: the output tile index, the tile index inside its A
+// matrix, and its k-blocks [kb_lo, kb_hi).  Output-split products schedule
+// their dense tiles (twice the bytes of a 2:4 tile) first.
+struct Tile2 {
+  int out, a, kb_lo, kb_hi;
+};
+__device__ __forceinline__ Tile2 tile2_of(const Gemm2Args& g, int tm) {
+  const int tsp = g.out_split_tiles;
+  if (tsp < 0) return {tm, tm, 0, g.kb + g.kb_dense};
+  const int nd = g.tiles_m - tsp;
+  if (tm < nd) return {tsp + tm, tm, g.kb, g.kb + g.kb_dense};
+  return {tm - nd, tm - nd, 0, g.kb};
+}
 
 template <int BN, int NACC, int MSUB, bool FP8 = false>
 struct Gemm2Cfg {
@@ -212,13 +230,13 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (elect_one()) {
       const uint32_t stage_tx = static_cast<uint32_t>(2 * (Cfg::kA + Cfg::kB + Cfg::kE));
       const uint32_t dense_tx = static_cast<uint32_t>(2 * (MSUB * Cfg::kA1 + Cfg::kHalfN * 128));
-      const int kb_all = args.kb + args.kb_dense;
       int it = 0;
       bool ok = true;
       for (int t = cluster_id; t < tiles && ok; t += num_clusters) {
-        const int tm = t % args.tiles_m, tn = t / args.tiles_m;
+        const Tile2 tl = tile2_of(args, t % args.tiles_m);
+        const int tm = tl.a, tn = t / args.tiles_m;
         const int32_t yb = tn * BN + static_cast<int32_t>(rank) * Cfg::kHalfN;
-        for (int kb = 0; kb < kb_all; ++kb, ++it) {
+        for (int kb = tl.kb_lo; kb < tl.kb_hi; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
           if (!mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag, kWhereProducer)) { ok = false; break; }
@@ -277,18 +295,19 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     if (leader && elect_one()) {
       const uint32_t idesc = idesc_bf16(256, BN, true);
       const uint32_t idesc_dn = idesc_bf16(256, BN, false);
-      const int kb_all = args.kb + args.kb_dense;
       int it = 0, lt = 0;
       bool ok = true;
       for (int t = cluster_id; t < tiles && ok; t += num_clusters, ++lt) {
+        const Tile2 tl = tile2_of(args, t % args.tiles_m);
         const int b = lt % NACC;
         const uint32_t use = static_cast<uint32_t>(lt / NACC);
         if (!mbar_wait(&tempty_bar[b], (use & 1u) ^ 1u, abort_flag, kWhereMma)) break;
         tc_fence_after();
         const uint32_t acc = tmem_base + b * MSUB * Cfg::kAccStride;
-        for (int kb = 0; kb < kb_all; ++kb, ++it) {
+        for (int kb = tl.kb_lo; kb < tl.kb_hi; ++kb, ++it) {
           const int s = it % S;
           const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+          const uint32_t accum0 = kb > tl.kb_lo ? 1u : 0u;     // the tile's first k-block overwrites
           if (!mbar_wait(&full_bar[s], ph, abort_flag, kWhereMma)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * Cfg::kA);
@@ -300,7 +319,7 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 #pragma unroll
               for (int u = 0; u < MSUB; ++u) {
                 const uint64_t ad = desc_sw128_kmajor(a0 + u * Cfg::kA1 + 32u * kk);
-                tc_mma_pair(acc + u * Cfg::kAccStride, ad, bd, idesc_dn, (kb > 0 || kk > 0) ? 1u : 0u);
+                tc_mma_pair(acc + u * Cfg::kAccStride, ad, bd, idesc_dn, (accum0 | static_cast<uint32_t>(kk > 0)));
               }
             }
             tc_commit_pair(&empty_bar[s]);
@@ -325,7 +344,7 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
                 for (int u = 0; u < MSUB; ++u) {
                   const uint64_t ad = desc_sw128_kmajor(a0 + u * Cfg::kA1 + 32u * kk);
                   tc_mma_sp_pair_e4m3(acc + u * Cfg::kAccStride, ad, bd, e_col + 8u * u + 2u * kk, idesc8,
-                                      (kb > 0 || kk > 0) ? 1u : 0u);
+                                      (accum0 | static_cast<uint32_t>(kk > 0)));
                 }
               }
             }
@@ -340,7 +359,7 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               for (int u = 0; u < MSUB; ++u) {
                 const uint64_t ad = desc_sw128_kmajor(a0 + u * Cfg::kA1 + 32u * kk);
                 tc_mma_sp_pair(acc + u * Cfg::kAccStride, ad, bd, e_col + 4u * u + (kk & ~1),
-                               idesc | static_cast<uint32_t>(kk & 1), (kb > 0 || kk > 0) ? 1u : 0u);
+                               idesc | static_cast<uint32_t>(kk & 1), (accum0 | static_cast<uint32_t>(kk > 0)));
               }
             }
           }
@@ -364,7 +383,7 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     st.out_fp32 = args.out_fp32;
     st.transpose_out = args.transpose_out;
     for (int t = cluster_id; t < tiles; t += num_clusters, ++lt) {
-      const int tm = t % args.tiles_m, tn = t / args.tiles_m;
+      const int tm = tile2_of(args, t % args.tiles_m).out, tn = t / args.tiles_m;
       const int b = lt % NACC;
       const uint32_t use = static_cast<uint32_t>(lt / NACC);
       if (!mbar_wait(&tfull_bar[b], use & 1u, abort_flag, kWhereEpilogue)) break;

@@ -9,7 +9,8 @@ Recipe (all workloads):
   * fp64 draws from numpy's PCG64 generator, then one round-to-nearest-even to
     fp32 and, for bf16 tensors, one more round-to-nearest-even from fp32 to bf16;
   * X uses stream ``seed``, W uses ``seed + 1``, the outlier-channel choice uses
-    ``seed + 2`` (seed 0 by default);
+    ``seed + 2`` (seed 0 by default); the GLU-MLP workloads take W_up from
+    ``seed + 1``, W_gate from ``seed + 3`` and W_down from ``seed + 4``;
   * N(0, s) means standard deviation s;
   * Student-t(nu=4) is divided by sqrt(2) so that its variance is 1;
   * "0.1% of channels scaled x20" picks round(0.001*K) K-columns by a seeded
@@ -28,7 +29,7 @@ import numpy as np
 
 __all__ = [
     "bf16_from_f64", "bf16_to_f64", "bf16_to_f32", "f32_bits",
-    "normal_bf16", "student_t_bf16", "Workload", "WORKLOADS", "make_workload",
+    "normal_bf16", "student_t_bf16", "Workload", "WORKLOADS", "make_workload", "make_mlp_weights",
 ]
 
 
@@ -87,6 +88,10 @@ class Workload:
     side: "act"    -> X is pruned N:M along K at run time (activation sparsity)
           "weight" -> W is pruned N:M along K offline (weight sparsity)
           "hybrid" -> W keeps a dense share of K columns, the rest is 2:4
+          "mlp"    -> a GLU MLP (W_up, W_gate [O x K], W_down [K x O]) whose
+                      dense share of intermediate indices stays dense in all
+                      three projections, the rest 2:4 (K = model width,
+                      O = intermediate width)
     """
     name: str
     side: str
@@ -104,7 +109,7 @@ class Workload:
 
     @property
     def K_lift(self) -> int:
-        if self.side == "hybrid":
+        if self.side in ("hybrid", "mlp"):
             return self.K
         n = self.M // 2
         return self.K * (2 * n - 2) // n
@@ -127,6 +132,9 @@ WORKLOADS = {
     ] + [
         Workload(f"hybrid_decode_b{b}", "hybrid", b, 4096, 14336, 2, 4, "bf16", "bf16", "normal",
                  dense_frac=0.25) for b in (1, 8, 32, 128)
+    ] + [
+        Workload(f"spense_mlp_decode_b{b}", "mlp", b, 4096, 14336, 2, 4, "bf16", "bf16", "normal",
+                 dense_frac=0.25) for b in (1, 8, 32, 128)
     ]
 }
 
@@ -148,6 +156,12 @@ def make_w(w: Workload, seed: int = 0) -> np.ndarray:
     if w.x_dtype == "fp32":
         return (_rng(seed + 1).standard_normal((w.O, w.K)) * w.w_std).astype(np.float32)
     return normal_bf16((w.O, w.K), w.w_std, seed + 1)
+
+
+def make_mlp_weights(w: Workload, seed: int = 0):
+    """(W_up [O x K], W_gate [O x K], W_down [K x O]) of a GLU-MLP workload."""
+    return (normal_bf16((w.O, w.K), w.w_std, seed + 1), normal_bf16((w.O, w.K), w.w_std, seed + 3),
+            normal_bf16((w.K, w.O), w.w_std, seed + 4))
 
 
 def make_workload(name: str, seed: int = 0, T: int | None = None):

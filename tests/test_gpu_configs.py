@@ -81,3 +81,24 @@ def test_tiny_fp32_full_size():
     np.testing.assert_array_equal(host_bits(comp.mask), ref["mask"])
     np.testing.assert_array_equal(host_bits(comp.vals), ref["vals"])
     check_close(host_f64(y), oracle.act_sparse_linear(x, w, wl.N, wl.M), "tiny")
+
+
+@pytest.mark.parametrize("B", [1, 128])
+def test_spense_mlp_decode_full_size(B):
+    """The GLU-MLP decode workloads (d = 4096, I = 14336, a quarter of the
+    intermediate indices dense) through the calls bench.py times: the packed
+    weights bit-exact, every output row within tolerance."""
+    wl, x, wu = inputs.make_workload(f"spense_mlp_decode_b{B}")
+    _, wg, wd = inputs.make_mlp_weights(wl)
+    W = nm.spense_mlp_prepare(dev(wu), dev(wg), dev(wd), wl.dense_frac)
+    ws = torch.empty(max(16, nm.spense_mlp_workspace_size(W, wl.T)), dtype=torch.uint8, device="cuda")
+    y = nm.spense_mlp(dev(x), W, ws=ws)
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    ref = oracle.spense_mlp_weights(wu, wg, wd, wl.dense_frac)
+    np.testing.assert_array_equal(W.perm.cpu().numpy(), ref["perm"])
+    np.testing.assert_array_equal(host_bits(W.ug_vals), ref["ug_vals"])
+    np.testing.assert_array_equal(host_bits(W.ug_dense), ref["ug_dense"])
+    np.testing.assert_array_equal(host_bits(W.down_vals), ref["down_vals"])
+    np.testing.assert_array_equal(host_bits(W.down_dense), ref["down_dense"])
+    check_close(host_f64(y), oracle.spense_mlp(x, wu, wg, wd, wl.dense_frac), f"spense mlp b{B}")

@@ -61,3 +61,20 @@ def test_mlp_full_size_decode():
     torch.cuda.synchronize()
     assert nm.device_error() == nm.NM_OK and W.D == 3584
     check_close(host_f64(y), oracle.spense_mlp(x, wu, wg, wd, 0.25), "mlp full size")
+
+
+@pytest.mark.parametrize("variant", ["1cta", "2cta128", "2cta224"])
+@pytest.mark.parametrize("B,I,d,frac", [(40, 1024, 256, 0.25), (130, 1024, 384, 0.5), (72, 768, 256, 0.0),
+                                        (96, 512, 256, 1.0)])
+def test_mlp_every_gemm_variant(monkeypatch, variant, B, I, d, frac):
+    """The output-split up/gate product and the input-split down product on
+    each GEMM kernel: single CTAs (128-row tiles, split-K) and SM pairs
+    (256-row tiles; dense tiles scheduled first)."""
+    monkeypatch.setenv("NMSPARSE_GEMM", variant)
+    wu, wg, wd = _weights(I, d, 5 * I + d + B)
+    x = inputs.normal_bf16((B, d), 1.0, B + 1)
+    W = nm.spense_mlp_prepare(dev(wu), dev(wg), dev(wd), frac)
+    y = nm.spense_mlp(dev(x), W)
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    check_close(host_f64(y), oracle.spense_mlp(x, wu, wg, wd, frac), f"mlp {variant} B={B} I={I} d={d} f={frac}")
