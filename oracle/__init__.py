@@ -72,6 +72,10 @@ def _load():
             "or_quant_vals_e4m3": (None, [P, I64, I64, P, P]),
             "or_lift_u8": (I, [P, I64, I64, I, P]),
             "or_meta8": (None, [P, I64, I64, P]),
+            "or_row_mean": (None, [P, I, I64, I64, P, P]),
+            "or_shift_bf16": (None, [P, I, I64, I64, P, P]),
+            "or_var_scale": (None, [P, P, I64, I64, P]),
+            "or_rowsum_f64": (None, [P, I, I64, I64, P]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -491,3 +495,77 @@ def spense_mlp(x: np.ndarray, w_up: np.ndarray, w_gate: np.ndarray, w_down: np.n
     g = linear_f64(xd, to_f64(w_gate, p["keep_gate"]), rows)
     h = silu_f64(g) * u
     return linear_f64(h, to_f64(w_down, p["keep_down"]))
+
+
+# ------------------------------------------------- shift and variance (step 9)
+
+
+def row_mean(x: np.ndarray):
+    """Step 9a: the per-token mean in fp64 and rounded to fp32."""
+    x = np.ascontiguousarray(x)
+    rows, K = x.shape
+    mu64 = np.empty(rows, np.float64)
+    mu32 = np.empty(rows, np.float32)
+    _load().or_row_mean(_ptr(_as_bits(x)), _dt(x), rows, K, _ptr(mu64), _ptr(mu32))
+    return mu64, mu32
+
+
+def shift_bf16(x: np.ndarray, mu32: np.ndarray) -> np.ndarray:
+    """Step 9b: bf16(fl32(x - mu32)) per token (bf16 bits)."""
+    x = np.ascontiguousarray(x)
+    rows, K = x.shape
+    mu32 = np.ascontiguousarray(mu32, np.float32)
+    out = np.empty((rows, K), np.uint16)
+    _load().or_shift_bf16(_ptr(_as_bits(x)), _dt(x), rows, K, _ptr(mu32), _ptr(out))
+    return out
+
+
+def var_scale(v: np.ndarray, keep: np.ndarray) -> np.ndarray:
+    """Step 9c: alpha = sqrt(var(v) / var(v * keep)) per token (1 if the
+    pruned token has no variance)."""
+    v = np.ascontiguousarray(v, np.uint16)
+    keep = np.ascontiguousarray(keep, np.uint8)
+    rows, K = v.shape
+    out = np.empty(rows, np.float64)
+    _load().or_var_scale(_ptr(v), _ptr(keep), rows, K, _ptr(out))
+    return out
+
+
+def rowsum_f64(w: np.ndarray) -> np.ndarray:
+    """Step 9d: s[o] = sum_k w[o][k] in fp64."""
+    w = np.ascontiguousarray(w)
+    O, K = w.shape
+    out = np.empty(O, np.float64)
+    _load().or_rowsum_f64(_ptr(_as_bits(w)), _dt(w), O, K, _ptr(out))
+    return out
+
+
+def act_transform(x: np.ndarray, N: int, M: int, shift: bool, var: bool):
+    """The activation operand with the optional corrections of step 9: the
+    shift (mu64, mu32; zero without D-PTS), the token the prune runs on
+    (xs), its keep mask and compressed form, and the VAR factor (alpha in
+    fp64 and rounded to fp32; one without VAR)."""
+    rows = x.shape[0]
+    if shift:
+        mu64, mu32 = row_mean(x)
+        xs = shift_bf16(x, mu32)
+    else:
+        mu64, mu32 = np.zeros(rows, np.float64), np.zeros(rows, np.float32)
+        xs = np.ascontiguousarray(x)
+    # the compressed form exists for windowable patterns (at most 2n-2 of 2n kept)
+    op = sparse_operand(xs, N, M) if N <= (2 if M == 4 else M - 2) else dict(keep=prune(xs, N, M))
+    alpha = var_scale(xs, op["keep"]) if var else np.ones(rows, np.float64)
+    return dict(op, mu64=mu64, mu32=mu32, xs=xs, alpha=alpha, alpha32=alpha.astype(np.float32))
+
+
+def act_sparse_linear_xf(x: np.ndarray, w: np.ndarray, N: int, M: int, shift: bool, var: bool,
+                         rows=None) -> np.ndarray:
+    """Y[t][o] = alpha[t] * (prune(xs[t]) . W[o]) + mu32[t] * s[o] in fp64:
+    the shifted token pruned and rescaled, the shift added back through the
+    weight's row sums."""
+    t = act_transform(x, N, M, shift, var)
+    y = linear_f64(to_f64(t["xs"], t["keep"]), to_f64(w), rows)
+    sel = slice(None) if rows is None else np.asarray(rows)
+    a = t["alpha"][sel][:, None]
+    mu = t["mu32"].astype(np.float64)[sel][:, None]
+    return a * y + mu * rowsum_f64(w)[None, :]

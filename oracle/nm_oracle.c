@@ -51,6 +51,15 @@
  *               [SlideSparse, technical summary §2.B (lifting fused into the
  *                per-token quantisation of INT8/FP8 inference) and §2.C
  *                (offline packer, online quantisation-slide kernel)]
+ *  9. shift/var two per-token corrections around the activation prune: the
+ *               token is centred on its mean before pruning and the mean is
+ *               added back through the weight's row sums (D-PTS, dynamic
+ *               shift); the survivors are rescaled so that the pruned token
+ *               keeps the variance of the token it came from (VAR).
+ *               [Flexible (N:M) Activation Sparsity, technical summary §2.B
+ *                (error mitigation: D-PTS, a dynamic per-token shift that
+ *                centres the activations on zero; VAR, a per-token variance
+ *                correction after pruning)]
  *
  * Where the pages are silent the plainest reading is taken and stated beside
  * the function that takes it.
@@ -549,6 +558,69 @@ void or_meta8(const uint8_t *nib, int64_t rows, int64_t Kl, uint8_t *meta) {
                     if (r < rows && j < nwin) q = nib[r * nwin + j];
                     meta[(rb * KB + kb) * 2048 + m * 16 + jj / 2] |= (uint8_t)((q & 0xF) << (4 * (jj % 2)));
                 }
+}
+
+/* ------------------------------------------------- shift and variance */
+
+/* Step 9a (D-PTS).  The page names a dynamic per-token shift that centres the
+ * activations on zero and gives no formula; the plainest reading is the
+ * token's mean: mu[r] = (sum_{k ascending} x[r][k]) / K in fp64, and the
+ * shift the kernels apply is that mean rounded to fp32.  For bf16 inputs whose
+ * magnitudes span fewer than 53 - 8 - log2(K) binades every partial sum is
+ * exact, so the mean does not depend on the order of summation. */
+void or_row_mean(const void *src, int dt, int64_t rows, int64_t K, double *mu64, float *mu32) {
+    for (int64_t r = 0; r < rows; ++r) {
+        double s = 0.0;
+        for (int64_t k = 0; k < K; ++k) s += value_at(src, dt, r * K + k);
+        mu64[r] = s / (double)K;
+        mu32[r] = (float)mu64[r];
+    }
+}
+
+/* Step 9b.  The shifted token, stored in the compute format:
+ * xs[r][k] = bf16(fl32(x[r][k] - mu32[r])), the difference rounded to fp32,
+ * then to bf16 (nearest-even both times).  The prune of step 1 runs on xs. */
+void or_shift_bf16(const void *src, int dt, int64_t rows, int64_t K, const float *mu32, uint16_t *xs) {
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            const float d = value_f32_at(src, dt, r * K + k) - mu32[r];
+            uint32_t u;
+            memcpy(&u, &d, 4);
+            xs[r * K + k] = f32_bits_to_bf16_rne(u);
+        }
+}
+
+/* Step 9c (VAR).  The page names a per-token variance correction after
+ * pruning and gives no formula; the plainest reading that keeps the pattern
+ * sparse is one factor per token on the survivors:
+ * alpha[r] = sqrt(var(v[r]) / var(v[r] * keep[r])), where v is the token the
+ * prune ran on, var(u) = (1/K) sum u^2 - ((1/K) sum u)^2 over all K entries
+ * (pruned ones as zeros), sums in fp64, k ascending; alpha = 1 when the
+ * pruned token has no variance. */
+void or_var_scale(const uint16_t *v, const uint8_t *keep, int64_t rows, int64_t K, double *alpha) {
+    for (int64_t r = 0; r < rows; ++r) {
+        double s = 0.0, q = 0.0, sp = 0.0, qp = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            const double x = bf16_bits_to_double(v[r * K + k]);
+            s += x;
+            q += x * x;
+            if (keep[r * K + k]) { sp += x; qp += x * x; }
+        }
+        const double mi = s / (double)K, mp = sp / (double)K;
+        const double var_in = q / (double)K - mi * mi;
+        const double var_p = qp / (double)K - mp * mp;
+        alpha[r] = var_p > 0.0 ? sqrt(var_in / var_p) : 1.0;
+    }
+}
+
+/* Step 9d.  Row sums of the weight, s[o] = sum_{k ascending} w[o][k] in fp64:
+ * the shift mu enters the product as mu * s[o]. */
+void or_rowsum_f64(const void *w, int dt, int64_t O, int64_t K, double *s) {
+    for (int64_t o = 0; o < O; ++o) {
+        double a = 0.0;
+        for (int64_t k = 0; k < K; ++k) a += value_at(w, dt, o * K + k);
+        s[o] = a;
+    }
 }
 
 /* ---------------------------------------------------------------- version */
