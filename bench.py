@@ -2,7 +2,8 @@
 
 One step = one pass of the hot path over one batch of synthetic input:
   activation sparsity (8:16, 16:32, tiny 2:4): prune + window-compress X,
-      then the 2:4 sparse GEMM against the offline-lifted weight;
+      then the 2:4 sparse GEMM against the offline-lifted weight (optionally
+      with the per-token shift and variance corrections around the prune);
   weight sparsity (6:8 sliding windows): lift X online, then the sparse GEMM
       against the offline-decomposed weight;
   hybrid dense + 2:4 weight (decode): gather X by the column permutation and
@@ -44,7 +45,7 @@ HEADLINE = "up_proj_8of16_act"
 TRAFFIC = {
     ("up_proj_8of16_act", "k_nm_gemm_2cta<224,2,1>"): 232299264 + 48795136,
 }
-OTHERS = ["up_proj_2of4_act", "up_proj_8of16_act_fp8", "down_proj_16of32_act", "slide_6of8_wt_prefill", "slide_6of8_wt_prefill_fp8",
+OTHERS = ["up_proj_2of4_act", "up_proj_8of16_act_fp8", "up_proj_8of16_act_xf", "down_proj_16of32_act", "slide_6of8_wt_prefill", "slide_6of8_wt_prefill_fp8",
           "slide_6of8_wt_decode",
           "hybrid_decode_b1", "hybrid_decode_b8", "hybrid_decode_b32", "hybrid_decode_b128",
           "spense_mlp_decode_b1", "spense_mlp_decode_b8", "spense_mlp_decode_b32", "spense_mlp_decode_b128",
@@ -231,6 +232,17 @@ class Workload:
             self.rows_a, self.rows_b = wl.T, wl.O
             self.prep_name, self.gemm_name = "prune_compress_fp8", "sparse_gemm_fp8"
             self.launches_per_step = 3                               # row scales, prune, GEMM
+        elif wl.side == "act" and wl.xf:
+            self.Wl = nm.lift(W, wl.M)                                   # offline
+            self.wsum = nm.row_sums(W)                                   # offline
+            self.R = max(2, min(8, int(np.ceil(2 * L2_BYTES / max(X0.numel() * X0.element_size(), 1)))))
+            self.X = [X0] + [X0.roll(r, dims=0).contiguous() for r in range(1, self.R)]
+            self.comp = [nm.alloc_xf(wl.T, wl.K, wl.N, wl.M, wl.xf, dev) for _ in range(2)]
+            self.Y = torch.empty((wl.T, wl.O), dtype=out_dt, device=dev)
+            self.rows_a, self.rows_b = wl.T, wl.O
+            self.prep_name, self.gemm_name = "prune_compress_xf", "sparse_gemm_xf"
+            # token means (with the shift), prune, factors, GEMM
+            self.launches_per_step = 4 if wl.xf & nm.NM_XF_SHIFT else 3
         elif wl.side == "act":
             self.Wl = nm.lift(W, wl.M)                                   # offline
             self.R = max(2, min(8, int(np.ceil(2 * L2_BYTES / max(X0.numel() * X0.element_size(), 1)))))
@@ -309,6 +321,12 @@ class Workload:
             if mark:
                 mark()
             nm.sparse_gemm_fp8(c, self.Wq, nm.NM_ACT, self.Y.dtype, out=self.Y)
+        elif wl.side == "act" and wl.xf:
+            c = self.comp[i % 2]
+            nm.prune_compress_xf(self.X[r], wl.N, wl.M, wl.xf, out=c)
+            if mark:
+                mark()
+            nm.sparse_gemm_xf(c, self.Wl, self.wsum, self.Y.dtype, out=self.Y)
         elif wl.side == "act":
             c = self.comp[i % 2]
             nm.prune_compress(self.X[r], wl.N, wl.M, out=c)
@@ -341,6 +359,8 @@ class Workload:
         r = i % self.R
         if wl.side == "act" and wl.fp8:
             nm.sparse_gemm_fp8(self.comp[0], self.Wq, nm.NM_ACT, self.Y.dtype, out=self.Y)
+        elif wl.side == "act" and wl.xf:
+            nm.sparse_gemm_xf(self.comp[0], self.Wl, self.wsum, self.Y.dtype, out=self.Y)
         elif wl.side == "act":
             nm.sparse_gemm(self.comp[0], self.Wl, nm.NM_ACT, self.Y.dtype, out=self.Y)
         elif wl.side == "weight" and wl.fp8:
@@ -558,6 +578,8 @@ def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None):
                    "K_lift": wl.K_lift, "rotated_buffers": wk.R},
         "kernels": {f"{wk.prep_name}_us": prep_ms * 1e3, f"{wk.gemm_name}_us": gemm_ms * 1e3},
     }
+    if wl.xf:
+        out["config"]["corrections"] = {1: "shift (D-PTS)", 2: "variance (VAR)", 3: "shift (D-PTS) + variance (VAR)"}[wl.xf]
     if wl.side == "mlp":
         out["config"].update(d=wl.K, I=wl.O, dense_frac=wl.dense_frac, D=wk.S[0].D)
         out["kernels"] = {"spense_mlp_us": step_ms * 1e3,

@@ -287,6 +287,54 @@ size_t spense_mlp_workspace_size(const nm_spense_mlp *W, int64_t B);
 int spense_mlp(const void *X, int64_t B, const nm_spense_mlp *W, void *Y, void *ws, size_t ws_bytes,
                void *stream);
 
+/* ------------------------------------------ per-token activation corrections */
+
+/* Two corrections around the activation prune that need no calibration data.
+ * [Motivating Next-Gen Accelerators with Flexible (N:M) Activation Sparsity,
+ *  technical summary §2.B: D-PTS, a dynamic per-token shift that centres the
+ *  activations on zero, and VAR, a per-token variance correction after
+ *  pruning.  The page gives no formulas; these are the plainest readings.]
+ *
+ * NM_XF_SHIFT (D-PTS): mu[t] = fl32((sum_k x[t][k]) / K), the sum in fp64;
+ *   the prune runs on xs[t][k] = bf16(fl32(x[t][k] - mu[t])) (nearest-even
+ *   both times), and the product adds the shift back as mu[t] * s[o], with
+ *   s[o] = fl32(sum_k W[o][k]) from nm_row_sums().
+ * NM_XF_VAR: the kept entries of token t are rescaled by
+ *   alpha[t] = sqrt(var(xs[t]) / var(kept xs[t])), var(u) = mean(u^2) -
+ *   mean(u)^2 over all K entries (pruned ones as zeros), sums in fp64;
+ *   alpha = 1 when the kept token has no variance.
+ * The result is Y[t][o] = alpha[t] * (prune(xs[t]) . W[o]) + mu[t] * s[o],
+ * with alpha = 1 without VAR and mu = 0 without the shift. */
+#define NM_XF_SHIFT 1u
+#define NM_XF_VAR 2u
+
+/* nm_prune_compress() of the bf16 activation src [rows x K] (row stride ld)
+ * with the corrections in `flags`: the compressed operand is that of xs (the
+ * shifted token, or src itself without NM_XF_SHIFT), row_shift_out [rows]
+ * receives mu (0 without the shift) and row_scale_out [rows] alpha (1 without
+ * VAR), both fp32.  ws: nm_prune_compress_xf_workspace_size() bytes of scratch
+ * when NM_XF_VAR is set (the per-chunk partial sums), else unused.  The
+ * scales are 4-byte aligned; everything else as in nm_prune_compress(). */
+size_t nm_prune_compress_xf_workspace_size(int64_t rows, int64_t K, int M);
+int nm_prune_compress_xf(const void *src, int64_t rows, int64_t K, int64_t ld, int N, int M,
+                         unsigned flags, uint32_t *mask_out, void *vals_out, void *meta_out,
+                         float *row_scale_out, float *row_shift_out, void *ws, size_t ws_bytes,
+                         void *stream);
+
+/* Offline: sums_out[r] = fl32(sum_k w[r][k]) of a bf16 matrix [rows x K]
+ * (row stride ld), the sum in fp64. */
+int nm_row_sums(const void *w, int64_t rows, int64_t K, int64_t ld, float *sums_out, void *stream);
+
+/* The activation-sparse product with the corrections applied in the GEMM
+ * epilogue: Y[t][o] = (X_c[t] . W'[o]) * row_scale[t] + row_shift[t] *
+ * w_row_sums[o], accumulated in fp32, stored as out_dt.  X is the operand
+ * written by nm_prune_compress_xf(), W_lift the lifted weight [rows_w][K']
+ * and w_row_sums [rows_w] the unlifted weight's row sums.  Other arguments
+ * as in nm_sparse_gemm() with side NM_ACT. */
+int nm_sparse_gemm_xf(const nm_sparse_operand *X, const void *W_lift, int64_t rows_w,
+                      const float *row_scale, const float *row_shift, const float *w_row_sums,
+                      void *Y, nm_dtype out_dt, void *stream);
+
 /* Capacity, in bytes, of the library's built-in scratch array used by
  * hybrid_gemm_noalloc(): the gathered activations need B * K * 2 bytes. */
 #define NM_NOALLOC_SCRATCH_BYTES (2u * 1024u * 1024u)

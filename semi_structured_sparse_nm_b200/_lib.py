@@ -81,6 +81,10 @@ def lib():
             "spense_mlp_prepare": (I, [P, P, P, D, ctypes.POINTER(SpenseMlpStruct), P, SZ, P]),
             "spense_mlp_workspace_size": (SZ, [ctypes.POINTER(SpenseMlpStruct), I64]),
             "spense_mlp": (I, [P, I64, ctypes.POINTER(SpenseMlpStruct), P, P, SZ, P]),
+            "nm_prune_compress_xf_workspace_size": (SZ, [I64, I64, I]),
+            "nm_prune_compress_xf": (I, [P, I64, I64, I64, I, I, ctypes.c_uint, P, P, P, P, P, P, SZ, P]),
+            "nm_row_sums": (I, [P, I64, I64, I64, P, P]),
+            "nm_sparse_gemm_xf": (I, [ctypes.POINTER(SparseOperand), P, I64, P, P, P, P, I, P]),
             "nm_status_string": (ctypes.c_char_p, [I]),
             "nm_last_cuda_error": (I, []),
             "nm_get_device_error": (I, [P]),
@@ -224,6 +228,73 @@ def dense_gemm(A: torch.Tensor, B: torch.Tensor, out_dtype=torch.bfloat16, out=N
         out = torch.empty((A.shape[0], B.shape[0]), dtype=out_dtype, device=A.device)
     _check("nm_dense_gemm", lib().nm_dense_gemm(_p(A), A.shape[0], _p(B), B.shape[0], A.shape[1], _p(out),
                                                 _dt(out), _stream(A)))
+    return out
+
+
+# ------------------------------------------ per-token activation corrections
+
+NM_XF_SHIFT, NM_XF_VAR = 1, 2
+
+
+class XfOperand:
+    """An activation operand pruned with the per-token corrections: the
+    compressed shifted token plus its VAR factor and shift (fp32 per row)."""
+
+    def __init__(self, comp: Compressed, row_scale: torch.Tensor, row_shift: torch.Tensor, flags: int,
+                 ws: torch.Tensor | None):
+        self.comp, self.row_scale, self.row_shift, self.flags, self.ws = comp, row_scale, row_shift, flags, ws
+
+
+def alloc_xf(rows: int, K: int, N: int, M: int, flags: int, device, with_mask=False) -> XfOperand:
+    comp = alloc_compressed(rows, K, N, M, device, with_mask)
+    ws_bytes = int(lib().nm_prune_compress_xf_workspace_size(rows, K, M)) if flags & NM_XF_VAR else 0
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device) if ws_bytes else None
+    f = lambda: torch.empty(rows, dtype=torch.float32, device=device)
+    return XfOperand(comp, f(), f(), flags, ws)
+
+
+def prune_compress_xf(x: torch.Tensor, N: int, M: int, flags: int, out: XfOperand | None = None,
+                      with_mask: bool = False) -> XfOperand:
+    """Prune + compress of the bf16 activation with NM_XF_SHIFT (D-PTS) and/or
+    NM_XF_VAR applied."""
+    _need_cuda(x)
+    rows, K = x.shape
+    if out is None:
+        out = alloc_xf(rows, K, N, M, flags, x.device, with_mask)
+    c = out.comp
+    ws_bytes = out.ws.numel() if out.ws is not None else 0
+    _check("nm_prune_compress_xf", lib().nm_prune_compress_xf(
+        _p(x), rows, K, x.stride(0), N, M, flags, _p(c.mask), _p(c.vals), _p(c.meta), _p(out.row_scale),
+        _p(out.row_shift), _p(out.ws), ws_bytes, _stream(x)))
+    return out
+
+
+def row_sums(w: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """fp32 row sums of a bf16 matrix (fp64 accumulation)."""
+    _need_cuda(w)
+    rows, K = w.shape
+    if out is None:
+        out = torch.empty(rows, dtype=torch.float32, device=w.device)
+    _check("nm_row_sums", lib().nm_row_sums(_p(w), rows, K, w.stride(0), _p(out), _stream(w)))
+    return out
+
+
+def sparse_gemm_xf(X: XfOperand, W_lift: torch.Tensor, w_row_sums: torch.Tensor, out_dtype=torch.bfloat16,
+                   out: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = (X_c . W'^T) * row_scale + row_shift * w_row_sums (activation side)."""
+    _need_cuda(W_lift, w_row_sums)
+    S = X.comp
+    rows_w = W_lift.shape[0]
+    if W_lift.dtype != torch.bfloat16 or W_lift.shape[1] != S.K_lift or not W_lift.is_contiguous():
+        raise ValueError("lifted weight must be contiguous bf16 [rows, K_lift]")
+    if w_row_sums.dtype != torch.float32 or w_row_sums.numel() != rows_w:
+        raise ValueError("w_row_sums must be fp32 [rows of W]")
+    if out is None:
+        out = torch.empty((S.rows, rows_w), dtype=out_dtype, device=W_lift.device)
+    st = S.struct()
+    _check("nm_sparse_gemm_xf", lib().nm_sparse_gemm_xf(
+        ctypes.byref(st), _p(W_lift), rows_w, _p(X.row_scale), _p(X.row_shift), _p(w_row_sums), _p(out),
+        _dt(out), _stream(W_lift)))
     return out
 
 

@@ -18,6 +18,7 @@
 #include "nm_prune.cuh"
 #include "nm_fp8.cuh"
 #include "nm_mlp.cuh"
+#include "nm_xf.cuh"
 #include "nmsparse.h"
 
 namespace {
@@ -104,6 +105,9 @@ struct GemmPlan {
   int out_fp32 = 0, transpose = 0;
   int a_static = 0;           // A is a weight: may be read before the preceding kernel ends
   int64_t out_split_rows = -1;  // output-split: A rows [0, this) sparse (a_s), the rest dense (a_d)
+  const float* row_scale = nullptr;   // bf16 affine epilogue: y = acc * row_scale[a] + row_shift[a] * col_sum[b]
+  const float* row_shift = nullptr;
+  const float* col_sum = nullptr;
   int fp8 = 0;                // 8-bit (E4M3) operands, rescaled by scale_a[row] * scale_b[column]
   const float* scale_a = nullptr;
   const float* scale_b = nullptr;
@@ -147,6 +151,9 @@ int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
   args.splits = splits;
   args.a_static = p.a_static;
   args.out_split_tiles = osplit ? static_cast<int>(p.out_split_rows / nm::kBM) : -1;
+  args.row_scale = p.row_scale;
+  args.row_shift = p.row_shift;
+  args.col_sum = p.col_sum;
   if (osplit) args.k_dense_x0 = 0;
 
   auto kern = nm::k_nm_gemm<BN>;
@@ -281,8 +288,10 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   a.kb_dense = static_cast<int>(kb_dense);
   a.k_dense_x0 = p.ks_lift;
   a.meta_kb = meta_kb;
-  a.scale_a = p.scale_a;
+  a.scale_a = FP8 ? p.scale_a : p.row_scale;
   a.scale_b = p.scale_b;
+  a.shift_a = p.row_shift;
+  a.sum_b = p.col_sum;
   a.last_half = (FP8 && p.ks_lift % 256 != 0) ? 1 : 0;
   a.out_split_tiles = p.out_split_rows >= 0 ? static_cast<int>(p.out_split_rows / (256 * MSUB)) : -1;
   if (p.out_split_rows >= 0) a.k_dense_x0 = 0;
@@ -394,9 +403,10 @@ int run_gemm(const GemmPlan& p, cudaStream_t st) {
 }
 
 // --------------------------------------------------------------- prune
-template <typename T, bool Q8 = false>
+template <typename T, bool Q8 = false, bool XF = false>
 int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M, uint32_t* mask,
-                 void* vals, void* meta, cudaStream_t st, const float* row_scale = nullptr) {
+                 void* vals, void* meta, cudaStream_t st, const float* row_scale = nullptr,
+                 const float* row_shift = nullptr, double* stats = nullptr) {
   const int64_t Kl = nm_lifted_k(K, M);
   const int64_t KB = ceil_div(Kl, 128);
   const int64_t rows_pad = ceil_div(rows, 128) * 128;
@@ -411,10 +421,10 @@ int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M
   auto e = static_cast<uint8_t*>(meta);
   cudaError_t err;
   switch (M) {
-    case 4: err = launch_pdl(nm::k_prune_compress<4, T, Q8>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale); break;
-    case 8: err = launch_pdl(nm::k_prune_compress<8, T, Q8>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale); break;
-    case 16: err = launch_pdl(nm::k_prune_compress<16, T, Q8>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale); break;
-    case 32: err = launch_pdl(nm::k_prune_compress<32, T, Q8>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale); break;
+    case 4: err = launch_pdl(nm::k_prune_compress<4, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale, row_shift, stats); break;
+    case 8: err = launch_pdl(nm::k_prune_compress<8, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale, row_shift, stats); break;
+    case 16: err = launch_pdl(nm::k_prune_compress<16, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale, row_shift, stats); break;
+    case 32: err = launch_pdl(nm::k_prune_compress<32, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale, row_shift, stats); break;
     default: return NM_ERR_UNSUPPORTED;
   }
   NM_CUDA_TRY(err);
@@ -511,9 +521,15 @@ size_t nm_sparse_gemm_workspace_size(const nm_sparse_operand* S, int64_t rows_d,
   return 0;   // split-K partial sums stay in the cluster's shared memory
 }
 
-int nm_sparse_gemm(const nm_sparse_operand* S, const void* D, int64_t rows_d, nm_side side, void* Y,
-                   nm_dtype out_dt, void* ws, size_t ws_bytes, void* stream) {
-  (void)ws; (void)ws_bytes;
+}  // extern "C"
+
+namespace {
+
+// Validates a sparse x lifted-dense product and fills its plan; NM_OK with
+// *empty set when there is nothing to compute.
+int sparse_plan(const nm_sparse_operand* S, const void* D, int64_t rows_d, nm_side side, void* Y,
+                nm_dtype out_dt, GemmPlan* plan, bool* empty) {
+  *empty = false;
   if (S == nullptr) return NM_ERR_INVALID_ARG;
   if (side != NM_ACT && side != NM_WEIGHT) return NM_ERR_INVALID_ARG;
   if (out_dt != NM_BF16 && out_dt != NM_FP32) return NM_ERR_INVALID_ARG;
@@ -521,10 +537,10 @@ int nm_sparse_gemm(const nm_sparse_operand* S, const void* D, int64_t rows_d, nm
   if (!m_supported(S->M)) return NM_ERR_UNSUPPORTED;
   if (S->K_lift != nm_lifted_k(S->K, S->M)) return NM_ERR_INVALID_ARG;
   if (S->K_lift % 16 != 0) return NM_ERR_UNSUPPORTED;
-  if (S->rows == 0 || rows_d == 0) return NM_OK;
+  if (S->rows == 0 || rows_d == 0) { *empty = true; return NM_OK; }
   if (D == nullptr || Y == nullptr || S->vals == nullptr || S->meta == nullptr) return NM_ERR_INVALID_ARG;
   if (!aligned16(S->vals) || !aligned16(S->meta) || !aligned16(D) || !aligned16(Y)) return NM_ERR_ALIGNMENT;
-  GemmPlan p;
+  GemmPlan& p = *plan;
   p.a_s = S->vals;
   p.b = D;
   p.rows_a = S->rows;
@@ -537,8 +553,90 @@ int nm_sparse_gemm(const nm_sparse_operand* S, const void* D, int64_t rows_d, nm
   p.transpose = side == NM_WEIGHT;
   p.ldy = side == NM_ACT ? rows_d : S->rows;
   p.a_static = side == NM_WEIGHT;
+  return NM_OK;
+}
+
+int64_t prune_chunks(int64_t K, int M) { return ceil_div(K / M, 32 * nm::prune_groups_per_lane(M, 2)); }
+
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int nm_sparse_gemm(const nm_sparse_operand* S, const void* D, int64_t rows_d, nm_side side, void* Y,
+                   nm_dtype out_dt, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws; (void)ws_bytes;
+  GemmPlan p;
+  bool empty = false;
+  const int rc = sparse_plan(S, D, rows_d, side, Y, out_dt, &p, &empty);
+  if (rc != NM_OK || empty) return rc;
   return run_gemm(p, static_cast<cudaStream_t>(stream));
 }
+
+// ------------------------------------------------ per-token corrections
+
+size_t nm_prune_compress_xf_workspace_size(int64_t rows, int64_t K, int M) {
+  if (rows <= 0 || K <= 0 || !m_supported(M) || K % M != 0) return 0;
+  return static_cast<size_t>(rows * prune_chunks(K, M) * 4 * static_cast<int64_t>(sizeof(double)));
+}
+
+int nm_prune_compress_xf(const void* src, int64_t rows, int64_t K, int64_t ld, int N, int M, unsigned flags,
+                         uint32_t* mask_out, void* vals_out, void* meta_out, float* row_scale_out,
+                         float* row_shift_out, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_prune_args(src, NM_BF16, rows, K, ld, N, M, vals_out, meta_out);
+  if (rc != NM_OK) return rc;
+  if ((flags & ~(NM_XF_SHIFT | NM_XF_VAR)) != 0u) return NM_ERR_INVALID_ARG;
+  if (rows == 0) return NM_OK;
+  if (row_scale_out == nullptr || row_shift_out == nullptr) return NM_ERR_INVALID_ARG;
+  if ((mask_out != nullptr && !aligned16(mask_out)) || !aligned4(row_scale_out) || !aligned4(row_shift_out))
+    return NM_ERR_ALIGNMENT;
+  const bool shift = (flags & NM_XF_SHIFT) != 0u, var = (flags & NM_XF_VAR) != 0u;
+  if (var) {
+    if (ws == nullptr || ws_bytes < nm_prune_compress_xf_workspace_size(rows, K, M)) return NM_ERR_WORKSPACE;
+    if (!aligned16(ws)) return NM_ERR_ALIGNMENT;
+  }
+  auto st = static_cast<cudaStream_t>(stream);
+  const auto* x = static_cast<const uint16_t*>(src);
+  if (shift) {
+    const dim3 grid(static_cast<unsigned>(std::min<int64_t>(rows, int64_t(num_sms()) * 8))), block(256);
+    NM_CUDA_TRY(launch_pdl(nm::k_row_sum_bf16<true>, grid, block, 0, st, x, rows, K, ld, row_shift_out));
+  }
+  double* stats = var ? static_cast<double*>(ws) : nullptr;
+  if ((rc = launch_prune<uint16_t, false, true>(x, rows, K, ld, N, M, mask_out, vals_out, meta_out, st, nullptr,
+                                                shift ? row_shift_out : nullptr, stats)) != NM_OK)
+    return rc;
+  const dim3 fgrid(static_cast<unsigned>(ceil_div(rows, int64_t(256)))), fblock(256);
+  NM_CUDA_TRY(launch_pdl(nm::k_xf_finalize, fgrid, fblock, 0, st, static_cast<const double*>(stats), rows,
+                         prune_chunks(K, M), K, var ? 1 : 0, shift ? 0 : 1, row_scale_out, row_shift_out));
+  return NM_OK;
+}
+
+int nm_row_sums(const void* w, int64_t rows, int64_t K, int64_t ld, float* sums_out, void* stream) {
+  if (rows < 0 || K <= 0 || ld < K) return NM_ERR_INVALID_ARG;
+  if (rows == 0) return NM_OK;
+  if (w == nullptr || sums_out == nullptr) return NM_ERR_INVALID_ARG;
+  if (!aligned16(w) || (ld * 2) % 16 != 0 || !aligned4(sums_out)) return NM_ERR_ALIGNMENT;
+  const dim3 grid(static_cast<unsigned>(std::min<int64_t>(rows, int64_t(num_sms()) * 8))), block(256);
+  NM_CUDA_TRY(launch_pdl(nm::k_row_sum_bf16<false>, grid, block, 0, static_cast<cudaStream_t>(stream),
+                         static_cast<const uint16_t*>(w), rows, K, ld, sums_out));
+  return NM_OK;
+}
+
+int nm_sparse_gemm_xf(const nm_sparse_operand* X, const void* W_lift, int64_t rows_w, const float* row_scale,
+                      const float* row_shift, const float* w_row_sums, void* Y, nm_dtype out_dt, void* stream) {
+  GemmPlan p;
+  bool empty = false;
+  const int rc = sparse_plan(X, W_lift, rows_w, NM_ACT, Y, out_dt, &p, &empty);
+  if (rc != NM_OK || empty) return rc;
+  if (row_scale == nullptr || row_shift == nullptr || w_row_sums == nullptr) return NM_ERR_INVALID_ARG;
+  if (!aligned4(row_scale) || !aligned4(row_shift) || !aligned4(w_row_sums)) return NM_ERR_ALIGNMENT;
+  p.row_scale = row_scale;
+  p.row_shift = row_shift;
+  p.col_sum = w_row_sums;
+  return run_gemm(p, static_cast<cudaStream_t>(stream));
+}
+
 
 // ------------------------------------------------------------ 8-bit (E4M3)
 

@@ -47,6 +47,11 @@ struct GemmArgs {
                                             // preceding kernel finishes; B only after
   int out_split_tiles;                      // -1, or the number of sparse row tiles of an
                                             // output-split product
+  // affine epilogue of the per-token activation corrections (all three or
+  // none): y = acc * row_scale[a] + row_shift[a] * col_sum[b]
+  const float* row_scale;
+  const float* row_shift;
+  const float* col_sum;
 };
 
 template <int BN>
@@ -104,19 +109,36 @@ __device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t addr) {
   return v;
 }
 
-__device__ __forceinline__ void store_out(const GemmArgs& a, int64_t ra, int64_t cb, float v) {
+__device__ __forceinline__ void store_out_raw(const GemmArgs& a, int64_t ra, int64_t cb, float v) {
   if (ra >= a.rows_a || cb >= a.rows_b) return;
   const int64_t off = a.transpose_out ? cb * a.ldy + ra : ra * a.ldy + cb;
   if (a.out_fp32) static_cast<float*>(a.Y)[off] = v;
   else static_cast<__nv_bfloat16*>(a.Y)[off] = __float2bfloat16_rn(v);
 }
 
+__device__ __forceinline__ void store_out(const GemmArgs& a, int64_t ra, int64_t cb, float v) {
+  if (ra >= a.rows_a || cb >= a.rows_b) return;
+  if (a.row_scale != nullptr) v = __fmaf_rn(a.row_shift[ra], a.col_sum[cb], v * a.row_scale[ra]);
+  store_out_raw(a, ra, cb, v);
+}
+
 // Stores CW (16 or 32) consecutive accumulator columns of row `ra`
 // (columns cb0 .. cb0+CW-1).
 template <int CW>
 __device__ __forceinline__ void store_row_chunk(const GemmArgs& a, int64_t ra, int64_t cb0,
-                                                const uint32_t (&v)[CW]) {
+                                                const uint32_t (&v_in)[CW]) {
   if (ra >= a.rows_a) return;
+  uint32_t v[CW];
+#pragma unroll
+  for (int i = 0; i < CW; ++i) v[i] = v_in[i];
+  if (a.row_scale != nullptr) {
+    const float sc = a.row_scale[ra], mu = a.row_shift[ra];
+#pragma unroll
+    for (int i = 0; i < CW; ++i) {
+      const float cs = cb0 + i < a.rows_b ? a.col_sum[cb0 + i] : 0.0f;
+      v[i] = __float_as_uint(__fmaf_rn(mu, cs, __uint_as_float(v[i]) * sc));
+    }
+  }
   if (a.transpose_out && cb0 + CW <= a.rows_b) {
     // Y[b][a]: lane = a, so each store instruction of the warp writes 32
     // consecutive outputs of one row of Y
@@ -155,7 +177,7 @@ __device__ __forceinline__ void store_row_chunk(const GemmArgs& a, int64_t ra, i
     return;
   }
 #pragma unroll
-  for (int i = 0; i < CW; ++i) store_out(a, ra, cb0 + i, __uint_as_float(v[i]));
+  for (int i = 0; i < CW; ++i) store_out_raw(a, ra, cb0 + i, __uint_as_float(v[i]));
 }
 
 template <int BN>

@@ -132,8 +132,11 @@ struct Gemm2Args {
   int transpose_out;
   int tma_store;          // 1: bf16 row-major Y written by TMA from a staging tile;
                           // 2: the same for Y stored transposed (Y[b][a])
-  const float* scale_a;   // 8-bit product: per-row scale of A (nullptr: none)
-  const float* scale_b;   //                per-row scale of B, i.e. per output column
+  const float* scale_a;   // 8-bit product: per-row scale of A (nullptr: none); bf16 product:
+                          // the row scale of the affine epilogue (nullptr: none)
+  const float* scale_b;   // 8-bit product: per-row scale of B, i.e. per output column
+  const float* shift_a;   // bf16 affine epilogue: y = acc * scale_a[a] + shift_a[a] * sum_b[b]
+  const float* sum_b;
   int last_half;          // 8-bit product: the last k-block holds only 128 lifted K
   int out_split_tiles;    // output-split (-1: none): output m-tiles below it are 2:4 rows
                           // (sparse k-blocks only), the rest dense rows (dense k-blocks
@@ -406,6 +409,16 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             for (int i = 0; i < 32; ++i) {
               const float sb = cb0 + i < args.rows_b ? __ldg(args.scale_b + cb0 + i) : 0.0f;
               v[i] = __float_as_uint(__uint_as_float(v[i]) * sa * sb);
+            }
+          } else if (args.scale_a != nullptr) {
+            // the per-token corrections of the activation operand
+            const float sa = ra < args.rows_a ? __ldg(args.scale_a + ra) : 0.0f;
+            const float mu = ra < args.rows_a ? __ldg(args.shift_a + ra) : 0.0f;
+            const int64_t cb0 = static_cast<int64_t>(tn) * BN + c0;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float cs = cb0 + i < args.rows_b ? __ldg(args.sum_b + cb0 + i) : 0.0f;
+              v[i] = __float_as_uint(__fmaf_rn(mu, cs, __uint_as_float(v[i]) * sa));
             }
           }
           if (args.tma_store == 2) {

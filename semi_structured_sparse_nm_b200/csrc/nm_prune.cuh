@@ -380,13 +380,22 @@ __host__ __device__ constexpr int prune_min_blocks(int M, int elem_bytes) {
 // code = e4m3(v * (1 / row_scale[r])) -- two bytes per window instead of two
 // bf16, and the metadata as the 8-bit image (row m, window j of a 128 x 128-K
 // block at byte 16 m + j/2, low nibble for even j).
-template <int M, typename T, bool Q8 = false>
-__global__ void __launch_bounds__(kPruneWarps * 32, prune_min_blocks(M, sizeof(T)))
+//
+// XF = true (bf16 input only) is the transform mode of the per-token
+// corrections: with row_shift, every element is first replaced by
+// bf16(fl32(x - row_shift[r])) and the prune runs on that (D-PTS); with
+// stats, each (row, chunk of 32 G groups) leaves four fp64 partial sums
+// {sum xs, sum xs^2, sum kept, sum kept^2} at stats[(r * chunks + chunk) * 4]
+// for the VAR factor.
+template <int M, typename T, bool Q8 = false, bool XF = false>
+__global__ void __launch_bounds__(kPruneWarps * 32, prune_min_blocks(M, sizeof(T)) - ((XF && M < 32) ? 1 : 0))
 k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int N,
                  uint32_t* __restrict__ mask_out, void* __restrict__ vals_out,
                  uint8_t* __restrict__ meta_out, int64_t Kl, int64_t KB, int64_t rows_pad,
-                 const float* __restrict__ row_scale) {
+                 const float* __restrict__ row_scale, const float* __restrict__ row_shift,
+                 double* __restrict__ stats) {
   static_assert(!Q8 || sizeof(T) == 2, "8-bit output from bf16 input");
+  static_assert(!XF || (sizeof(T) == 2 && !Q8), "transform mode: bf16 input, bf16 output");
   constexpr int G = prune_groups_per_lane(M, static_cast<int>(sizeof(T)));
   constexpr int NW = M / 2 - 1;                   // windows per group
   constexpr int NWL = G * NW;                     // windows per lane
@@ -435,6 +444,7 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
       __syncwarp();
       float inv = 1.0f;
       if constexpr (Q8) inv = __frcp_rn(row_scale[r]);
+      double st[4] = {0.0, 0.0, 0.0, 0.0};             // transform mode: partial sums of this lane
       if (gl < groups) {
         uint32_t vals[NWL];
         uint8_t nibs[NWL];
@@ -445,6 +455,27 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
           for (int p = 0; p < LM / 2; ++p) {
             const uint4& q = raw[k].v[p / 4];
             PL[p] = (p % 4 == 0) ? q.x : (p % 4 == 1) ? q.y : (p % 4 == 2) ? q.z : q.w;
+          }
+          if constexpr (XF) {
+            if (row_shift != nullptr) {
+              const float mu = row_shift[r];
+#pragma unroll
+              for (int p = 0; p < LM / 2; ++p) {
+                const __nv_bfloat162 h = __floats2bfloat162_rn(__fsub_rn(__uint_as_float(PL[p] << 16), mu),
+                                                               __fsub_rn(__uint_as_float(PL[p] & 0xFFFF0000u), mu));
+                PL[p] = *reinterpret_cast<const uint32_t*>(&h);
+              }
+            }
+            if (stats != nullptr) {
+#pragma unroll
+              for (int p = 0; p < LM / 2; ++p) {
+                if ((G == 1) || (gl + (2 * p) / M < groups)) {
+                  const double a = __uint_as_float(PL[p] << 16), b = __uint_as_float(PL[p] & 0xFFFF0000u);
+                  st[0] += a + b;
+                  st[1] += a * a + b * b;
+                }
+              }
+            }
           }
 #pragma unroll
           for (int j = 0; j < G; ++j) {
@@ -461,6 +492,20 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
           }
         } else {
           keep = compress_group<M, T>(raw[k], N, vals, nibs);
+        }
+        if constexpr (XF) {
+          if (stats != nullptr) {
+            // kept values: both slots of every window of the valid groups
+            // (padded slots hold +0.0)
+#pragma unroll
+            for (int w = 0; w < NWL; ++w) {
+              if ((G == 1) || (gl + w / NW < groups)) {
+                const double a = __uint_as_float(vals[w] << 16), b = __uint_as_float(vals[w] & 0xFFFF0000u);
+                st[2] += a + b;
+                st[3] += a * a + b * b;
+              }
+            }
+          }
         }
 #pragma unroll
         for (int w = 0; w < NWL; ++w) {
@@ -501,6 +546,19 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
       if (mask_out != nullptr && lane < LM) {
         const int64_t wi = ch * LM + lane;
         if (wi < mask_words) mask_out[r * mask_words + wi] = s_mask[warp][lane];
+      }
+      if constexpr (XF) {
+        if (stats != nullptr) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) st[i] += __shfl_xor_sync(0xFFFFFFFFu, st[i], o);
+          if (lane == 0) {
+            double2* dst = reinterpret_cast<double2*>(stats + (r * cpr + ch) * 4);
+            dst[0] = make_double2(st[0], st[1]);
+            dst[1] = make_double2(st[2], st[3]);
+          }
+        }
       }
       __syncwarp();
     }

@@ -106,6 +106,7 @@ class Workload:
     w_std: float = 0.02
     dense_frac: float = 0.0
     fp8: bool = False   # 8-bit (E4M3) operands: X quantised per token, W per output row
+    xf: int = 0         # per-token corrections of the activation prune: 1 shift (D-PTS), 2 VAR, 3 both
 
     @property
     def K_lift(self) -> int:
@@ -123,6 +124,8 @@ WORKLOADS = {
         Workload("up_proj_2of4_act", "act", 2048, 4096, 14336, 2, 4, "bf16", "bf16", "student_t4"),
         # the same 8:16 product with 8-bit operands (X per token, W per output channel)
         Workload("up_proj_8of16_act_fp8", "act", 2048, 4096, 14336, 8, 16, "bf16", "bf16", "student_t4", fp8=True),
+        # the same 8:16 product with the D-PTS shift and the VAR rescale around the prune
+        Workload("up_proj_8of16_act_xf", "act", 2048, 4096, 14336, 8, 16, "bf16", "bf16", "student_t4", xf=3),
         Workload("slide_6of8_wt_prefill", "weight", 4096, 4096, 4096, 6, 8, "bf16", "bf16", "normal"),
         Workload("slide_6of8_wt_decode", "weight", 16, 4096, 4096, 6, 8, "bf16", "bf16", "normal"),
         # the same prefill product with 8-bit operands (the pages' B200 precision)

@@ -87,3 +87,42 @@ def test_validation_before_launch(L):
     assert L.nm_debug_expire_wait(0, s) == nm.NM_ERR_INVALID_ARG
     for code in range(7):
         assert L.nm_status_string(code)
+
+
+def test_correction_calls_validate_before_launch(L):
+    from semi_structured_sparse_nm_b200 import _lib as nm
+    fake = ctypes.c_void_p(0x10000)
+    odd4 = ctypes.c_void_p(0x10002)
+    null = ctypes.c_void_p(0)
+    s = null
+    both = nm.NM_XF_SHIFT | nm.NM_XF_VAR
+    # workspace: one fp64 quadruple per (row, chunk of 32 G groups)
+    assert L.nm_prune_compress_xf_workspace_size(16, 4096, 16) == 16 * (256 // 32) * 32
+    assert L.nm_prune_compress_xf_workspace_size(16, 4096, 4) == 16 * (1024 // 128) * 32
+    assert L.nm_prune_compress_xf_workspace_size(0, 4096, 16) == 0
+    # bad flags, missing scale outputs, missing workspace with VAR, misaligned scales
+    assert L.nm_prune_compress_xf(fake, 16, 256, 256, 2, 4, 4, null, fake, fake, fake, fake, fake, 4096, s) \
+        == nm.NM_ERR_INVALID_ARG
+    assert L.nm_prune_compress_xf(fake, 16, 256, 256, 2, 4, both, null, fake, fake, null, fake, fake, 4096, s) \
+        == nm.NM_ERR_INVALID_ARG
+    assert L.nm_prune_compress_xf(fake, 16, 256, 256, 2, 4, both, null, fake, fake, fake, fake, null, 0, s) \
+        == nm.NM_ERR_WORKSPACE
+    assert L.nm_prune_compress_xf(fake, 16, 256, 256, 2, 4, both, null, fake, fake, fake, fake, fake, 16, s) \
+        == nm.NM_ERR_WORKSPACE
+    assert L.nm_prune_compress_xf(fake, 16, 256, 256, 2, 4, nm.NM_XF_SHIFT, null, fake, fake, odd4, fake,
+                                  null, 0, s) == nm.NM_ERR_ALIGNMENT
+    assert L.nm_prune_compress_xf(fake, 16, 256, 256, 3, 4, both, null, fake, fake, fake, fake, fake, 4096, s) \
+        == nm.NM_ERR_UNSUPPORTED
+    assert L.nm_prune_compress_xf(null, 0, 256, 256, 2, 4, both, null, null, null, null, null, null, 0, s) \
+        == nm.NM_OK
+    # row sums
+    assert L.nm_row_sums(null, 4, 256, 256, fake, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_row_sums(fake, 4, 256, 252, fake, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_row_sums(fake, 4, 252, 260, fake, s) == nm.NM_ERR_ALIGNMENT
+    assert L.nm_row_sums(fake, 4, 256, 256, odd4, s) == nm.NM_ERR_ALIGNMENT
+    assert L.nm_row_sums(null, 0, 256, 256, null, s) == nm.NM_OK
+    # the corrected GEMM
+    S = nm.SparseOperand(0x10000, 0x10000, 128, 256, 2, 4, 256)
+    assert L.nm_sparse_gemm_xf(ctypes.byref(S), fake, 64, null, fake, fake, fake, 0, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_sparse_gemm_xf(ctypes.byref(S), fake, 64, fake, fake, odd4, fake, 0, s) == nm.NM_ERR_ALIGNMENT
+    assert L.nm_sparse_gemm_xf(ctypes.byref(S), fake, 0, null, null, null, fake, 0, s) == nm.NM_OK
