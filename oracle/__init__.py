@@ -74,7 +74,7 @@ def _load():
             "or_meta8": (None, [P, I64, I64, P]),
             "or_row_mean": (None, [P, I, I64, I64, P, P]),
             "or_shift_bf16": (None, [P, I, I64, I64, P, P]),
-            "or_var_scale": (None, [P, P, I64, I64, P]),
+            "or_var_scale": (None, [P, I, P, P, I64, I64, P]),
             "or_rowsum_f64": (None, [P, I, I64, I64, P]),
         }
         for name, (res, args) in sig.items():
@@ -520,14 +520,16 @@ def shift_bf16(x: np.ndarray, mu32: np.ndarray) -> np.ndarray:
     return out
 
 
-def var_scale(v: np.ndarray, keep: np.ndarray) -> np.ndarray:
-    """Step 9c: alpha = sqrt(var(v) / var(v * keep)) per token (1 if the
-    pruned token has no variance)."""
+def var_scale(x: np.ndarray, v: np.ndarray, keep: np.ndarray) -> np.ndarray:
+    """Step 9c: alpha = sqrt(var(x) / var(v * keep)) per token, x the token as
+    it came in, v the token the prune ran on (1 if the pruned token has no
+    variance)."""
+    x = np.ascontiguousarray(x)
     v = np.ascontiguousarray(v, np.uint16)
     keep = np.ascontiguousarray(keep, np.uint8)
     rows, K = v.shape
     out = np.empty(rows, np.float64)
-    _load().or_var_scale(_ptr(v), _ptr(keep), rows, K, _ptr(out))
+    _load().or_var_scale(_ptr(_as_bits(x)), _dt(x), _ptr(v), _ptr(keep), rows, K, _ptr(out))
     return out
 
 
@@ -554,7 +556,7 @@ def act_transform(x: np.ndarray, N: int, M: int, shift: bool, var: bool):
         xs = np.ascontiguousarray(x)
     # the compressed form exists for windowable patterns (at most 2n-2 of 2n kept)
     op = sparse_operand(xs, N, M) if N <= (2 if M == 4 else M - 2) else dict(keep=prune(xs, N, M))
-    alpha = var_scale(xs, op["keep"]) if var else np.ones(rows, np.float64)
+    alpha = var_scale(x, xs, op["keep"]) if var else np.ones(rows, np.float64)
     return dict(op, mu64=mu64, mu32=mu32, xs=xs, alpha=alpha, alpha32=alpha.astype(np.float32))
 
 

@@ -592,19 +592,27 @@ void or_shift_bf16(const void *src, int dt, int64_t rows, int64_t K, const float
 
 /* Step 9c (VAR).  The page names a per-token variance correction after
  * pruning and gives no formula; the plainest reading that keeps the pattern
- * sparse is one factor per token on the survivors:
- * alpha[r] = sqrt(var(v[r]) / var(v[r] * keep[r])), where v is the token the
- * prune ran on, var(u) = (1/K) sum u^2 - ((1/K) sum u)^2 over all K entries
- * (pruned ones as zeros), sums in fp64, k ascending; alpha = 1 when the
- * pruned token has no variance. */
-void or_var_scale(const uint16_t *v, const uint8_t *keep, int64_t rows, int64_t K, double *alpha) {
+ * sparse is one factor per token on the survivors, chosen so that the pruned
+ * token gets back the variance of the dense token:
+ * alpha[r] = sqrt(var(x[r]) / var(v[r] * keep[r])), where x is the token as
+ * it came in, v the token the prune ran on (x itself, or the shifted token of
+ * step 9b -- the variance does not change under a shift),
+ * var(u) = (1/K) sum u^2 - ((1/K) sum u)^2 over all K entries (pruned ones as
+ * zeros), sums in fp64, k ascending; alpha = 1 when the pruned token has no
+ * variance. */
+void or_var_scale(const void *x_in, int dt, const uint16_t *v, const uint8_t *keep, int64_t rows, int64_t K,
+                  double *alpha) {
     for (int64_t r = 0; r < rows; ++r) {
         double s = 0.0, q = 0.0, sp = 0.0, qp = 0.0;
         for (int64_t k = 0; k < K; ++k) {
-            const double x = bf16_bits_to_double(v[r * K + k]);
+            const double x = value_at(x_in, dt, r * K + k);
             s += x;
             q += x * x;
-            if (keep[r * K + k]) { sp += x; qp += x * x; }
+            if (keep[r * K + k]) {
+                const double y = bf16_bits_to_double(v[r * K + k]);
+                sp += y;
+                qp += y * y;
+            }
         }
         const double mi = s / (double)K, mp = sp / (double)K;
         const double var_in = q / (double)K - mi * mi;

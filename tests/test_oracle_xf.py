@@ -111,15 +111,27 @@ def test_worked_example():
 def test_var_factor_matches_library_variance(N, M):
     x = inputs.student_t_bf16((32, 512), 4.0, 10)
     keep = oracle.prune(x, N, M)
-    alpha = oracle.var_scale(x, keep)
+    alpha = oracle.var_scale(x, x, keep)
     xf = inputs.bf16_to_f64(x)
     ref = np.sqrt(np.var(xf, axis=1) / np.var(xf * keep, axis=1))
     np.testing.assert_allclose(alpha, ref, rtol=1e-12)
     # the rescaled survivors have the variance of the token they came from
     np.testing.assert_allclose(np.var(alpha[:, None] * xf * keep, axis=1), np.var(xf, axis=1), rtol=1e-12)
     # nothing pruned: factor 1; a token whose survivors are all zero: factor 1
-    np.testing.assert_array_equal(oracle.var_scale(x, np.ones_like(keep)), np.ones(32))
-    np.testing.assert_array_equal(oracle.var_scale(x, np.zeros_like(keep)), np.ones(32))
+    np.testing.assert_array_equal(oracle.var_scale(x, x, np.ones_like(keep)), np.ones(32))
+    np.testing.assert_array_equal(oracle.var_scale(x, x, np.zeros_like(keep)), np.ones(32))
+
+
+def test_var_with_the_shift_restores_the_dense_token_variance():
+    """With the shift, the kept entries are those of the shifted token and
+    the target variance is the incoming token's."""
+    x = inputs.bf16_from_f64(inputs.bf16_to_f64(inputs.student_t_bf16((16, 512), 4.0, 16)) + 2.0)
+    t = oracle.act_transform(x, 8, 16, True, True)
+    xf, xs = inputs.bf16_to_f64(x), inputs.bf16_to_f64(t["xs"])
+    ref = np.sqrt(np.var(xf, axis=1) / np.var(xs * t["keep"], axis=1))
+    np.testing.assert_allclose(t["alpha"], ref, rtol=1e-12)
+    # the shifted token has the same variance up to its bf16 rounding
+    np.testing.assert_allclose(np.var(xs, axis=1), np.var(xf, axis=1), rtol=1e-2)
 
 
 def test_shift_error_is_the_bf16_rounding_of_the_shifted_token():
