@@ -576,9 +576,13 @@ int nm_sparse_gemm(const nm_sparse_operand* S, const void* D, int64_t rows_d, nm
 
 // ------------------------------------------------ per-token corrections
 
+// VAR scratch: the token moments (rows x 2 fp64, padded to 256 bytes), then
+// the kept sums of every (row, chunk) (rows x chunks x 2 fp64).
+int64_t xf_moments_bytes(int64_t rows) { return ceil_div(rows * 16, int64_t(256)) * 256; }
+
 size_t nm_prune_compress_xf_workspace_size(int64_t rows, int64_t K, int M) {
   if (rows <= 0 || K <= 0 || !m_supported(M) || K % M != 0) return 0;
-  return static_cast<size_t>(rows * prune_chunks(K, M) * 4 * static_cast<int64_t>(sizeof(double)));
+  return static_cast<size_t>(xf_moments_bytes(rows) + rows * prune_chunks(K, M) * 16);
 }
 
 int nm_prune_compress_xf(const void* src, int64_t rows, int64_t K, int64_t ld, int N, int M, unsigned flags,
@@ -598,17 +602,19 @@ int nm_prune_compress_xf(const void* src, int64_t rows, int64_t K, int64_t ld, i
   }
   auto st = static_cast<cudaStream_t>(stream);
   const auto* x = static_cast<const uint16_t*>(src);
-  if (shift) {
-    const dim3 grid(static_cast<unsigned>(std::min<int64_t>(rows, int64_t(num_sms()) * 8))), block(256);
-    NM_CUDA_TRY(launch_pdl(nm::k_row_sum_bf16<true>, grid, block, 0, st, x, rows, K, ld, row_shift_out));
-  }
-  double* stats = var ? static_cast<double*>(ws) : nullptr;
+  double* moments = var ? static_cast<double*>(ws) : nullptr;
+  double* kept = var ? reinterpret_cast<double*>(static_cast<uint8_t*>(ws) + xf_moments_bytes(rows)) : nullptr;
+  const dim3 wgrid(static_cast<unsigned>(std::min<int64_t>(ceil_div(rows, int64_t(8)), int64_t(1) << 30))),
+      block(256);
+  if (shift || var)   // token mean and / or moments, one warp per row
+    NM_CUDA_TRY(launch_pdl(nm::k_row_prep_bf16, wgrid, block, 0, st, x, rows, K, ld, shift ? 1 : 0, row_shift_out,
+                           moments));
   if ((rc = launch_prune<uint16_t, false, true>(x, rows, K, ld, N, M, mask_out, vals_out, meta_out, st, nullptr,
-                                                shift ? row_shift_out : nullptr, stats)) != NM_OK)
+                                                shift ? row_shift_out : nullptr, kept)) != NM_OK)
     return rc;
-  const dim3 fgrid(static_cast<unsigned>(ceil_div(rows, int64_t(256)))), fblock(256);
-  NM_CUDA_TRY(launch_pdl(nm::k_xf_finalize, fgrid, fblock, 0, st, static_cast<const double*>(stats), rows,
-                         prune_chunks(K, M), K, var ? 1 : 0, shift ? 0 : 1, row_scale_out, row_shift_out));
+  NM_CUDA_TRY(launch_pdl(nm::k_xf_finalize, wgrid, block, 0, st, static_cast<const double*>(moments),
+                         static_cast<const double*>(kept), rows, prune_chunks(K, M), K, shift ? 0 : 1, row_scale_out,
+                         row_shift_out));
   return NM_OK;
 }
 
@@ -617,8 +623,8 @@ int nm_row_sums(const void* w, int64_t rows, int64_t K, int64_t ld, float* sums_
   if (rows == 0) return NM_OK;
   if (w == nullptr || sums_out == nullptr) return NM_ERR_INVALID_ARG;
   if (!aligned16(w) || (ld * 2) % 16 != 0 || !aligned4(sums_out)) return NM_ERR_ALIGNMENT;
-  const dim3 grid(static_cast<unsigned>(std::min<int64_t>(rows, int64_t(num_sms()) * 8))), block(256);
-  NM_CUDA_TRY(launch_pdl(nm::k_row_sum_bf16<false>, grid, block, 0, static_cast<cudaStream_t>(stream),
+  const dim3 grid(static_cast<unsigned>(std::min<int64_t>(ceil_div(rows, int64_t(8)), int64_t(1) << 30))), block(256);
+  NM_CUDA_TRY(launch_pdl(nm::k_row_sum_bf16, grid, block, 0, static_cast<cudaStream_t>(stream),
                          static_cast<const uint16_t*>(w), rows, K, ld, sums_out));
   return NM_OK;
 }

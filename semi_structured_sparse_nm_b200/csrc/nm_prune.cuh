@@ -384,11 +384,11 @@ __host__ __device__ constexpr int prune_min_blocks(int M, int elem_bytes) {
 // XF = true (bf16 input only) is the transform mode of the per-token
 // corrections: with row_shift, every element is first replaced by
 // bf16(fl32(x - row_shift[r])) and the prune runs on that (D-PTS); with
-// stats, each (row, chunk of 32 G groups) leaves four fp64 partial sums
-// {sum xs, sum xs^2, sum kept, sum kept^2} at stats[(r * chunks + chunk) * 4]
-// for the VAR factor.
+// stats, each (row, chunk of 32 G groups) leaves the fp64 sum and sum of
+// squares of its kept entries at stats[(r * chunks + chunk) * 2] for the VAR
+// factor.
 template <int M, typename T, bool Q8 = false, bool XF = false>
-__global__ void __launch_bounds__(kPruneWarps * 32, prune_min_blocks(M, sizeof(T)) - ((XF && M < 32) ? 1 : 0))
+__global__ void __launch_bounds__(kPruneWarps * 32, prune_min_blocks(M, sizeof(T)))
 k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int N,
                  uint32_t* __restrict__ mask_out, void* __restrict__ vals_out,
                  uint8_t* __restrict__ meta_out, int64_t Kl, int64_t KB, int64_t rows_pad,
@@ -444,7 +444,7 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
       __syncwarp();
       float inv = 1.0f;
       if constexpr (Q8) inv = __frcp_rn(row_scale[r]);
-      double st[4] = {0.0, 0.0, 0.0, 0.0};             // transform mode: partial sums of this lane
+      double st[2] = {0.0, 0.0};                       // transform mode: kept sums of this lane
       if (gl < groups) {
         uint32_t vals[NWL];
         uint8_t nibs[NWL];
@@ -464,16 +464,6 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
                 const __nv_bfloat162 h = __floats2bfloat162_rn(__fsub_rn(__uint_as_float(PL[p] << 16), mu),
                                                                __fsub_rn(__uint_as_float(PL[p] & 0xFFFF0000u), mu));
                 PL[p] = *reinterpret_cast<const uint32_t*>(&h);
-              }
-            }
-            if (stats != nullptr) {
-#pragma unroll
-              for (int p = 0; p < LM / 2; ++p) {
-                if ((G == 1) || (gl + (2 * p) / M < groups)) {
-                  const double a = __uint_as_float(PL[p] << 16), b = __uint_as_float(PL[p] & 0xFFFF0000u);
-                  st[0] += a + b;
-                  st[1] += a * a + b * b;
-                }
               }
             }
           }
@@ -501,8 +491,8 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
             for (int w = 0; w < NWL; ++w) {
               if ((G == 1) || (gl + w / NW < groups)) {
                 const double a = __uint_as_float(vals[w] << 16), b = __uint_as_float(vals[w] & 0xFFFF0000u);
-                st[2] += a + b;
-                st[3] += a * a + b * b;
+                st[0] += a + b;
+                st[1] += a * a + b * b;
               }
             }
           }
@@ -550,14 +540,10 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
       if constexpr (XF) {
         if (stats != nullptr) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
+          for (int i = 0; i < 2; ++i)
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) st[i] += __shfl_xor_sync(0xFFFFFFFFu, st[i], o);
-          if (lane == 0) {
-            double2* dst = reinterpret_cast<double2*>(stats + (r * cpr + ch) * 4);
-            dst[0] = make_double2(st[0], st[1]);
-            dst[1] = make_double2(st[2], st[3]);
-          }
+          if (lane == 0) reinterpret_cast<double2*>(stats)[r * cpr + ch] = make_double2(st[0], st[1]);
         }
       }
       __syncwarp();

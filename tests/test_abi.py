@@ -96,9 +96,10 @@ def test_correction_calls_validate_before_launch(L):
     null = ctypes.c_void_p(0)
     s = null
     both = nm.NM_XF_SHIFT | nm.NM_XF_VAR
-    # workspace: one fp64 quadruple per (row, chunk of 32 G groups)
-    assert L.nm_prune_compress_xf_workspace_size(16, 4096, 16) == 16 * (256 // 32) * 32
-    assert L.nm_prune_compress_xf_workspace_size(16, 4096, 4) == 16 * (1024 // 128) * 32
+    # workspace: the token moments (two fp64 per row, padded to 256 bytes) and
+    # two fp64 per (row, chunk of 32 G groups)
+    assert L.nm_prune_compress_xf_workspace_size(16, 4096, 16) == 256 + 16 * (256 // 32) * 16
+    assert L.nm_prune_compress_xf_workspace_size(100, 4096, 4) == 1792 + 100 * (1024 // 128) * 16
     assert L.nm_prune_compress_xf_workspace_size(0, 4096, 16) == 0
     # bad flags, missing scale outputs, missing workspace with VAR, misaligned scales
     assert L.nm_prune_compress_xf(fake, 16, 256, 256, 2, 4, 4, null, fake, fake, fake, fake, fake, 4096, s) \
