@@ -144,6 +144,17 @@ struct Gemm2Args {
                           // column 0)
 };
 
+// The tile a cluster takes in its round j of the persistent loop: round j
+// covers tiles [j P, j P + P) for P clusters.  Output-split products, whose
+// tiles differ in length (dense tiles first, then 2:4 ones), run the odd
+// rounds in reverse cluster order, so that the clusters that took the longest
+// tiles in one round take the shortest in the next (the sequence increases,
+// so the first index past the end closes the loop).
+__device__ __forceinline__ int tile2_at(int round, int cluster, int clusters, int out_split_tiles) {
+  const bool rev = out_split_tiles >= 0 && (round & 1);
+  return round * clusters + (rev ? clusters - 1 - cluster : cluster);
+}
+
 // One m-tile's place: the output tile index, the tile index inside its A
 // matrix, and its k-blocks [kb_lo, kb_hi).  Output-split products schedule
 // their dense tiles (twice the bytes of a 2:4 tile) first.
@@ -235,7 +246,7 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const uint32_t dense_tx = static_cast<uint32_t>(2 * (MSUB * Cfg::kA1 + Cfg::kHalfN * 128));
       int it = 0;
       bool ok = true;
-      for (int t = cluster_id; t < tiles && ok; t += num_clusters) {
+      for (int j = 0, t = cluster_id; t < tiles && ok; t = tile2_at(++j, cluster_id, num_clusters, args.out_split_tiles)) {
         const Tile2 tl = tile2_of(args, t % args.tiles_m);
         const int tm = tl.a, tn = t / args.tiles_m;
         const int32_t yb = tn * BN + static_cast<int32_t>(rank) * Cfg::kHalfN;
@@ -300,7 +311,8 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const uint32_t idesc_dn = idesc_bf16(256, BN, false);
       int it = 0, lt = 0;
       bool ok = true;
-      for (int t = cluster_id; t < tiles && ok; t += num_clusters, ++lt) {
+      for (int j = 0, t = cluster_id; t < tiles && ok;
+           t = tile2_at(++j, cluster_id, num_clusters, args.out_split_tiles), ++lt) {
         const Tile2 tl = tile2_of(args, t % args.tiles_m);
         const int b = lt % NACC;
         const uint32_t use = static_cast<uint32_t>(lt / NACC);
@@ -385,7 +397,7 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     st.ldy = args.ldy;
     st.out_fp32 = args.out_fp32;
     st.transpose_out = args.transpose_out;
-    for (int t = cluster_id; t < tiles; t += num_clusters, ++lt) {
+    for (int j = 0, t = cluster_id; t < tiles; t = tile2_at(++j, cluster_id, num_clusters, args.out_split_tiles), ++lt) {
       const int tm = tile2_of(args, t % args.tiles_m).out, tn = t / args.tiles_m;
       const int b = lt % NACC;
       const uint32_t use = static_cast<uint32_t>(lt / NACC);
