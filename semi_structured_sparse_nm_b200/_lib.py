@@ -85,6 +85,8 @@ def lib():
             "nm_prune_compress_xf": (I, [P, I64, I64, I64, I, I, ctypes.c_uint, P, P, P, P, P, P, SZ, P]),
             "nm_row_sums": (I, [P, I64, I64, I64, P, P]),
             "nm_sparse_gemm_xf": (I, [ctypes.POINTER(SparseOperand), P, I64, P, P, P, P, I, P]),
+            "nm_act_sparse_linear_host_workspace_size": (SZ, [I64, I64, I, I, I64, I64]),
+            "nm_act_sparse_linear_host": (I, [P, I64, I64, I, I, P, I64, P, I64, P, SZ, P]),
             "nm_status_string": (ctypes.c_char_p, [I]),
             "nm_last_cuda_error": (I, []),
             "nm_get_device_error": (I, [P]),
@@ -296,6 +298,37 @@ def sparse_gemm_xf(X: XfOperand, W_lift: torch.Tensor, w_row_sums: torch.Tensor,
         ctypes.byref(st), _p(W_lift), rows_w, _p(X.row_scale), _p(X.row_shift), _p(w_row_sums), _p(out),
         _dt(out), _stream(W_lift)))
     return out
+
+
+# ------------------------------------------------- host-buffer pipeline
+
+
+def act_sparse_linear_host_workspace(T: int, K: int, N: int, M: int, O: int, device, chunk_rows: int = 0):
+    n = int(lib().nm_act_sparse_linear_host_workspace_size(T, K, N, M, O, chunk_rows))
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def act_sparse_linear_host(x_host: torch.Tensor, W_lift: torch.Tensor, N: int, M: int, y_host: torch.Tensor,
+                           ws: torch.Tensor | None = None, chunk_rows: int = 0) -> torch.Tensor:
+    """y_host = prune_{N:M}(x_host) . W^T with x_host, y_host bf16 tensors in
+    (page-locked) host memory and the lifted weight on the device; chunked
+    copies in and out overlap the math.  Asynchronous on the current stream."""
+    _need_cuda(W_lift)
+    if x_host.is_cuda or y_host.is_cuda:
+        raise ValueError("x_host and y_host live in host memory")
+    for t in (x_host, y_host):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("contiguous bf16 host tensors expected")
+    T, K = x_host.shape
+    O = W_lift.shape[0]
+    if tuple(y_host.shape) != (T, O):
+        raise ValueError("y_host must be [T, O]")
+    if ws is None:
+        ws = act_sparse_linear_host_workspace(T, K, N, M, O, W_lift.device, chunk_rows)
+    _check("nm_act_sparse_linear_host", lib().nm_act_sparse_linear_host(
+        ctypes.c_void_p(x_host.data_ptr()), T, K, N, M, _p(W_lift), O, ctypes.c_void_p(y_host.data_ptr()),
+        chunk_rows, _p(ws), ws.numel(), _stream(W_lift)))
+    return y_host
 
 
 # ---------------------------------------------------------- 8-bit (E4M3)

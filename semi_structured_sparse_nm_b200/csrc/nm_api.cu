@@ -1090,6 +1090,130 @@ int hybrid_gemm_noalloc(const void* X, int64_t B, const nm_hybrid_weight* W, voi
   return hybrid_gemm(X, B, W, Y, out_dt, ws, NM_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+// ------------------------------------------------ host-buffer pipeline
+
+}  // extern "C"
+
+namespace {
+// Two auxiliary streams (copies in, copies out) and the events that chain
+// the two buffer slots of the chunked host-buffer pipeline, one set per
+// device, created on first use and kept until the process exits.
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t start = nullptr;
+  cudaEvent_t in[2] = {}, done[2] = {}, out[2] = {};
+};
+std::mutex g_pipe_mu;
+HostPipe g_pipe[kMaxDevices];
+
+int host_pipe(HostPipe** out) {
+  int dev = 0;
+  NM_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return NM_ERR_UNSUPPORTED;
+  HostPipe& p = g_pipe[dev];
+  if (!p.ready) {
+    NM_CUDA_TRY(cudaStreamCreateWithFlags(&p.s_in, cudaStreamNonBlocking));
+    NM_CUDA_TRY(cudaStreamCreateWithFlags(&p.s_out, cudaStreamNonBlocking));
+    NM_CUDA_TRY(cudaEventCreateWithFlags(&p.start, cudaEventDisableTiming));
+    for (int b = 0; b < 2; ++b) {
+      NM_CUDA_TRY(cudaEventCreateWithFlags(&p.in[b], cudaEventDisableTiming));
+      NM_CUDA_TRY(cudaEventCreateWithFlags(&p.done[b], cudaEventDisableTiming));
+      NM_CUDA_TRY(cudaEventCreateWithFlags(&p.out[b], cudaEventDisableTiming));
+    }
+    p.ready = true;
+  }
+  *out = &p;
+  return NM_OK;
+}
+
+constexpr int64_t kHostChunkRows = 256;
+
+int64_t round256(int64_t b) { return ceil_div(b, int64_t(256)) * 256; }
+
+// Bytes of one buffer slot: X chunk, compressed values, metadata, Y chunk.
+int64_t host_slot_bytes(int64_t Tc, int64_t K, int M, int64_t O) {
+  const int64_t Kl = nm_lifted_k(K, M);
+  return round256(Tc * K * 2) + round256(Tc * (Kl / 2) * 2) +
+         round256(static_cast<int64_t>(nm_meta_bytes(Tc, K, M))) + round256(Tc * O * 2);
+}
+}  // namespace
+
+extern "C" {
+
+size_t nm_act_sparse_linear_host_workspace_size(int64_t T, int64_t K, int N, int M, int64_t O, int64_t chunk_rows) {
+  (void)N;
+  if (T <= 0 || K <= 0 || O <= 0 || nm_lifted_k(K, M) < 0) return 0;
+  const int64_t Tc = std::min(T, chunk_rows > 0 ? chunk_rows : kHostChunkRows);
+  return static_cast<size_t>(2 * host_slot_bytes(Tc, K, M, O));
+}
+
+int nm_act_sparse_linear_host(const void* x_host, int64_t T, int64_t K, int N, int M, const void* w_lift, int64_t O,
+                              void* y_host, int64_t chunk_rows, void* ws, size_t ws_bytes, void* stream) {
+  if (T < 0 || K <= 0 || O <= 0 || chunk_rows < 0) return NM_ERR_INVALID_ARG;
+  if (chunk_rows % 128 != 0) return NM_ERR_INVALID_ARG;
+  const int64_t Tc = std::min(T, chunk_rows > 0 ? chunk_rows : kHostChunkRows);
+  // the pattern and shapes are validated before anything is enqueued (the
+  // placeholder address stands for the chunk buffers, which are never read here)
+  void* const placeholder = reinterpret_cast<void*>(uintptr_t(256));
+  int rc = check_prune_args(placeholder, NM_BF16, 1, K, K, N, M, placeholder, placeholder);
+  if (rc != NM_OK) return rc;
+  const int64_t Kl = nm_lifted_k(K, M);
+  if (Kl % 16 != 0) return NM_ERR_UNSUPPORTED;
+  if (T == 0) return NM_OK;
+  if (x_host == nullptr || y_host == nullptr || w_lift == nullptr || ws == nullptr) return NM_ERR_INVALID_ARG;
+  if (!aligned16(w_lift) || !aligned16(ws)) return NM_ERR_ALIGNMENT;
+  if (ws_bytes < nm_act_sparse_linear_host_workspace_size(T, K, N, M, O, chunk_rows)) return NM_ERR_WORKSPACE;
+
+  const int64_t slot = host_slot_bytes(Tc, K, M, O);
+  uint8_t* base[2] = {static_cast<uint8_t*>(ws), static_cast<uint8_t*>(ws) + slot};
+  auto st = static_cast<cudaStream_t>(stream);
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe* p = nullptr;
+  if ((rc = host_pipe(&p)) != NM_OK) return rc;
+  // copies in start after the work already on `stream`
+  NM_CUDA_TRY(cudaEventRecord(p->start, st));
+  NM_CUDA_TRY(cudaStreamWaitEvent(p->s_in, p->start, 0));
+  const int64_t chunks = ceil_div(T, Tc);
+  for (int64_t c = 0; c < chunks; ++c) {
+    const int b = static_cast<int>(c % 2);
+    const int64_t r0 = c * Tc, rows = std::min(Tc, T - r0);
+    uint8_t* xd = base[b];
+    uint8_t* vals = xd + round256(Tc * K * 2);
+    uint8_t* meta = vals + round256(Tc * (Kl / 2) * 2);
+    uint8_t* yd = meta + round256(static_cast<int64_t>(nm_meta_bytes(Tc, K, M)));
+    // copy in: slot b's X is free once the prune of chunk c - 2 has read it
+    NM_CUDA_TRY(cudaStreamWaitEvent(p->s_in, p->done[b], 0));
+    NM_CUDA_TRY(cudaMemcpyAsync(xd, static_cast<const uint8_t*>(x_host) + r0 * K * 2, static_cast<size_t>(rows * K * 2),
+                                cudaMemcpyHostToDevice, p->s_in));
+    NM_CUDA_TRY(cudaEventRecord(p->in[b], p->s_in));
+    // prune + GEMM on the caller's stream; slot b's Y is free once the copy
+    // out of chunk c - 2 has read it
+    NM_CUDA_TRY(cudaStreamWaitEvent(st, p->in[b], 0));
+    NM_CUDA_TRY(cudaStreamWaitEvent(st, p->out[b], 0));
+    if ((rc = nm_prune_compress(xd, NM_BF16, rows, K, K, N, M, nullptr, vals, meta, stream)) != NM_OK) return rc;
+    nm_sparse_operand S{};
+    S.vals = vals;
+    S.meta = meta;
+    S.rows = rows;
+    S.K = K;
+    S.N = N;
+    S.M = M;
+    S.K_lift = Kl;
+    if ((rc = nm_sparse_gemm(&S, w_lift, O, NM_ACT, yd, NM_BF16, nullptr, 0, stream)) != NM_OK) return rc;
+    NM_CUDA_TRY(cudaEventRecord(p->done[b], st));
+    // copy out
+    NM_CUDA_TRY(cudaStreamWaitEvent(p->s_out, p->done[b], 0));
+    NM_CUDA_TRY(cudaMemcpyAsync(static_cast<uint8_t*>(y_host) + r0 * O * 2, yd, static_cast<size_t>(rows * O * 2),
+                                cudaMemcpyDeviceToHost, p->s_out));
+    NM_CUDA_TRY(cudaEventRecord(p->out[b], p->s_out));
+  }
+  // `stream` reaches this point once every chunk has been copied out
+  NM_CUDA_TRY(cudaStreamWaitEvent(st, p->out[0], 0));
+  NM_CUDA_TRY(cudaStreamWaitEvent(st, p->out[1], 0));
+  return NM_OK;
+}
+
 const char* nm_status_string(int s) {
   switch (s) {
     case NM_OK: return "ok";

@@ -127,3 +127,29 @@ def test_correction_calls_validate_before_launch(L):
     assert L.nm_sparse_gemm_xf(ctypes.byref(S), fake, 64, null, fake, fake, fake, 0, s) == nm.NM_ERR_INVALID_ARG
     assert L.nm_sparse_gemm_xf(ctypes.byref(S), fake, 64, fake, fake, odd4, fake, 0, s) == nm.NM_ERR_ALIGNMENT
     assert L.nm_sparse_gemm_xf(ctypes.byref(S), fake, 0, null, null, null, fake, 0, s) == nm.NM_OK
+
+
+def test_host_pipeline_validates_before_launch(L):
+    from semi_structured_sparse_nm_b200 import _lib as nm
+    fake = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10001)
+    null = ctypes.c_void_p(0)
+    s = null
+    ws = L.nm_act_sparse_linear_host_workspace_size(600, 1024, 8, 16, 768, 256)
+    Kl = 1024 * 7 // 4                                                 # K' = 1.75 K for 8:16
+    slot = (256 * 1024 * 2) + (256 * Kl) + L.nm_meta_bytes(256, 1024, 16) + (256 * 768 * 2)
+    assert ws == 2 * slot
+    assert L.nm_act_sparse_linear_host_workspace_size(100, 1024, 8, 16, 768, 0) == \
+        2 * ((100 * 2048 + 255) // 256 * 256 + (100 * Kl + 255) // 256 * 256 + L.nm_meta_bytes(100, 1024, 16)
+             + (100 * 1536 + 255) // 256 * 256)
+    assert L.nm_act_sparse_linear_host(fake, 600, 1024, 8, 16, fake, 768, fake, 100, fake, ws, s) \
+        == nm.NM_ERR_INVALID_ARG                                           # chunk not a multiple of 128
+    assert L.nm_act_sparse_linear_host(fake, 600, 1024, 15, 16, fake, 768, fake, 0, fake, ws, s) \
+        == nm.NM_ERR_UNSUPPORTED
+    assert L.nm_act_sparse_linear_host(null, 600, 1024, 8, 16, fake, 768, fake, 0, fake, ws, s) \
+        == nm.NM_ERR_INVALID_ARG
+    assert L.nm_act_sparse_linear_host(fake, 600, 1024, 8, 16, odd, 768, fake, 0, fake, ws, s) \
+        == nm.NM_ERR_ALIGNMENT
+    assert L.nm_act_sparse_linear_host(fake, 600, 1024, 8, 16, fake, 768, fake, 0, fake, ws - 1, s) \
+        == nm.NM_ERR_WORKSPACE
+    assert L.nm_act_sparse_linear_host(null, 0, 1024, 8, 16, null, 768, null, 0, null, 0, s) == nm.NM_OK
