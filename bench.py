@@ -568,7 +568,16 @@ def time_dense_mlp(wk, reps=20):
     return e0.elapsed_time(e1) / reps
 
 
-def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None):
+def mma_probe():
+    """The library's tensor-core rate probe (MMAs from shared memory on every
+    SM pair, no loads): the rate the GEMMs' MMA instructions can reach at
+    this moment's clocks, in TFLOP/s dense-equivalent."""
+    from semi_structured_sparse_nm_b200 import _lib as nm
+    return {"bf16_dense": nm.mma_rate_probe(0), "bf16_sparse": nm.mma_rate_probe(1),
+            "e4m3_sparse": nm.mma_rate_probe(2)}
+
+
+def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None, probe=None):
     dense, mma, byts = wk.algorithmic()
     wl = wk.wl
     out = {
@@ -621,6 +630,9 @@ def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None):
                            "flops_per_launch": mma,
                            "peak_note": f"4 x {pk['source']} bf16 burst {pk['bf16']} TFLOP/s (nominal 8-bit / "
                                         f"16-bit ratio 2 x nominal 2:4 sparse ratio 2)"}
+        if probe:
+            out["roofline"]["probe_tflops"] = probe["e4m3_sparse"]
+            out["roofline"]["frac_of_probe"] = achieved / probe["e4m3_sparse"]
     else:
         peak = 2.0 * pk["bf16"]
         achieved = mma / (gemm_ms * 1e-3) / 1e12
@@ -630,6 +642,9 @@ def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None):
                            "flops_per_launch": mma,
                            "peak_note": f"2 x {pk['source']} bf16 burst {pk['bf16']} TFLOP/s "
                                         f"(nominal 2:4 sparse ratio)"}
+        if probe:
+            out["roofline"]["probe_tflops"] = probe["bf16_sparse"]
+            out["roofline"]["frac_of_probe"] = achieved / probe["bf16_sparse"]
     return out
 
 
@@ -669,8 +684,9 @@ def run_gpu(args):
         step_ms = max_over_ranks(step_ms, dist, dev)
         dist.barrier()
     status = nm.device_error()
+    probe = mma_probe()
     main = summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk,
-                     traffic=TRAFFIC.get((args.workload, "k_nm_gemm_2cta<224,2,1>")))
+                     traffic=TRAFFIC.get((args.workload, "k_nm_gemm_2cta<224,2,1>")), probe=probe)
 
     # end to end through the public calls: pinned host X in, Y out
     wl = wk.wl
@@ -715,6 +731,9 @@ def run_gpu(args):
         "tokens_per_s": main["tokens_per_s"],
         "kernels": main["kernels"],
         "roofline": main["roofline"],
+        "mma_probe": {**probe, "unit": "TFLOP/s",
+                      "note": "nm_mma_rate_probe: 256 x 256 MMAs from shared memory on every SM pair, no loads; "
+                              "best of 5 launches of about 1 ms, dense-equivalent flops"},
         "dense_comparator": main.get("dense_comparator"),
         "e2e": {"value": ws * dense / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
@@ -735,7 +754,7 @@ def run_gpu(args):
                 continue
             w2 = Workload(name, dev)
             s, p, g = time_workload(w2, args.steps, args.warmup, stream)
-            others[name] = summarize(w2, s, p, g, 1, pk)
+            others[name] = summarize(w2, s, p, g, 1, pk, probe=probe)
             del w2
             torch.cuda.empty_cache()
         line["workloads"] = others

@@ -400,6 +400,15 @@ int nm_get_device_error(void *stream);
  * mbarrier no thread ever arrives on, giving up after timeout_us
  * microseconds and recording NM_ERR_DEVICE_TIMEOUT.  Faults nothing. */
 int nm_debug_expire_wait(unsigned timeout_us, void *stream);
+/* Tensor-core rate probe (diagnostic; grounds the roofline denominators):
+ * every SM pair issues 4 * iters MMAs of 256 x 256 x K (cta_group::2) from
+ * operands held in shared memory -- no loads, no epilogue -- so that
+ * *flops_out / (the launch's duration) is the tensor pipe's own rate.
+ * mode 0: bf16 dense (K = 16); 1: bf16 2:4 sparse (K = 32 logical);
+ * 2: E4M3 2:4 sparse (K = 64 logical).  *flops_out counts 2 * M * N * K per
+ * MMA (dense-equivalent), set on return; the caller times the launch (for
+ * example with events around the call on `stream`). */
+int nm_mma_rate_probe(int mode, int iters, double *flops_out, void *stream);
 const char *nm_version(void);
 
 #ifdef __cplusplus

@@ -87,6 +87,7 @@ def lib():
             "nm_sparse_gemm_xf": (I, [ctypes.POINTER(SparseOperand), P, I64, P, P, P, P, I, P]),
             "nm_act_sparse_linear_host_workspace_size": (SZ, [I64, I64, I, I, I64, I64]),
             "nm_act_sparse_linear_host": (I, [P, I64, I64, I, I, P, I64, P, I64, P, SZ, P]),
+            "nm_mma_rate_probe": (I, [I, I, ctypes.POINTER(ctypes.c_double), P]),
             "nm_status_string": (ctypes.c_char_p, [I]),
             "nm_last_cuda_error": (I, []),
             "nm_get_device_error": (I, [P]),
@@ -485,6 +486,24 @@ def hybrid_gemm_noalloc(x: torch.Tensor, h: Hybrid, out_dtype=torch.bfloat16, ou
 def device_error(stream=None) -> int:
     s = stream if stream is not None else _stream()
     return int(lib().nm_get_device_error(s))
+
+
+def mma_rate_probe(mode: int, iters: int = 4000, reps: int = 5) -> float:
+    """Tensor-core rate in TFLOP/s (dense-equivalent) of back-to-back MMAs from
+    shared memory on every SM pair: mode 0 bf16 dense, 1 bf16 2:4 sparse,
+    2 E4M3 2:4 sparse.  Best of `reps` timed launches after one warm-up."""
+    st = _stream()
+    flops = ctypes.c_double(0.0)
+    _check("nm_mma_rate_probe", lib().nm_mma_rate_probe(mode, iters, ctypes.byref(flops), st))
+    best = float("inf")
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        _check("nm_mma_rate_probe", lib().nm_mma_rate_probe(mode, iters, ctypes.byref(flops), st))
+        e1.record()
+        e1.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    return flops.value / (best * 1e-3) / 1e12
 
 
 def debug_expire_wait(timeout_us: int):

@@ -19,6 +19,7 @@
 #include "nm_fp8.cuh"
 #include "nm_mlp.cuh"
 #include "nm_xf.cuh"
+#include "nm_peak.cuh"
 #include "nmsparse.h"
 
 namespace {
@@ -1244,6 +1245,44 @@ int nm_debug_expire_wait(unsigned timeout_us, void* stream) {
   nm::k_expire_wait<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<unsigned long long>(timeout_us) * 1000ull);
   NM_CUDA_TRY(cudaGetLastError());
+  return NM_OK;
+}
+
+int nm_mma_rate_probe(int mode, int iters, double* flops_out, void* stream) {
+  if (mode < 0 || mode > 2 || iters <= 0 || iters > 1000000 || flops_out == nullptr) return NM_ERR_INVALID_ARG;
+  const int clusters = std::max(1, num_sms() / 2);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = nm::kProbeSmemLaunch;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static_assert(nm::kProbeSmem <= nm::kProbeSmemLaunch, "probe shared memory");
+  cudaError_t e;
+  switch (mode) {
+    case 0:
+      NM_CUDA_TRY(cudaFuncSetAttribute(nm::k_mma_probe<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, nm::kProbeSmemLaunch));
+      e = cudaLaunchKernelEx(&cfg, nm::k_mma_probe<0>, iters);
+      break;
+    case 1:
+      NM_CUDA_TRY(cudaFuncSetAttribute(nm::k_mma_probe<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, nm::kProbeSmemLaunch));
+      e = cudaLaunchKernelEx(&cfg, nm::k_mma_probe<1>, iters);
+      break;
+    default:
+      NM_CUDA_TRY(cudaFuncSetAttribute(nm::k_mma_probe<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, nm::kProbeSmemLaunch));
+      e = cudaLaunchKernelEx(&cfg, nm::k_mma_probe<2>, iters);
+      break;
+  }
+  NM_CUDA_TRY(e);
+  NM_CUDA_TRY(cudaGetLastError());
+  const double k = mode == 0 ? 16.0 : (mode == 1 ? 32.0 : 64.0);   // logical K per MMA
+  *flops_out = static_cast<double>(clusters) * iters * 4.0 * 2.0 * 256.0 * nm::kProbeN * k;
   return NM_OK;
 }
 

@@ -1,6 +1,7 @@
-"""Bounded waits and error reporting on the GPU.  Nothing here faults, traps or
-hangs the device: the expired wait is a barrier nobody arrives on, with a
-1 ms limit, and the kernel returns normally after recording the status."""
+"""Bounded waits, error reporting and the tensor-core rate probe on the GPU.
+Nothing here faults, traps or hangs the device: the expired wait is a barrier
+nobody arrives on, with a 1 ms limit, and the kernel returns normally after
+recording the status."""
 import numpy as np
 import pytest
 import torch
@@ -41,3 +42,15 @@ def test_errors_launch_nothing():
     assert e.value.status == nm.NM_ERR_ALIGNMENT
     torch.cuda.synchronize()
     assert torch.equal(comp.vals.view(torch.int16), before.view(torch.int16))
+
+
+def test_mma_rate_probe():
+    """The tensor-core probe runs on every SM pair and reports sane rates: the
+    2:4 modes execute twice the logical K per MMA, the 8-bit one four times."""
+    dense = nm.mma_rate_probe(0, iters=2000, reps=3)
+    sp16 = nm.mma_rate_probe(1, iters=2000, reps=3)
+    sp8 = nm.mma_rate_probe(2, iters=2000, reps=3)
+    assert nm.device_error() == nm.NM_OK
+    assert 500.0 < dense < 2600.0, dense
+    assert 1.5 * dense < sp16 < 2.2 * dense, (dense, sp16)
+    assert 1.5 * sp16 < sp8 < 2.2 * sp16, (sp16, sp8)
