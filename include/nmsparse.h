@@ -16,9 +16,14 @@
  *  - Pointers must be 16-byte aligned and leading dimensions multiples of 8
  *    elements (16 bytes for bf16 rows), else NM_ERR_ALIGNMENT.
  *  - Weight operands (the sparse operand of NM_WEIGHT products, the hybrid
- *    weight) may be read while the kernel issued just before on the same
- *    stream is still finishing (programmatic dependent launch); they must
- *    not be written by that kernel.  Everything else waits for it.
+ *    and GLU-MLP weights) may be read before a kernel waits for the work
+ *    queued ahead of it.  Every kernel of this library lets the next one
+ *    start early (programmatic dependent launch), so a run of library calls
+ *    can be in flight together: a weight must not be written by a library
+ *    call that may still be running.  Prepare weights ahead, and separate
+ *    the preparation from their use by a stream synchronisation, an event
+ *    wait or a copy (as offline preparation is).  Everything else waits for
+ *    the preceding work.
  *
  * Terms.  An N:M pattern keeps the N entries of largest magnitude in every
  * aligned group of M consecutive entries along K, ties going to the lower
