@@ -52,6 +52,7 @@ OTHERS = ["up_proj_2of4_act", "up_proj_8of16_act_fp8", "up_proj_8of16_act_xf", "
           "tiny_2of4_act_fp32"]
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "N:M sparse linear TFLOP/s (dense-equiv)"
+REF_TOTAL_S = 150.0
 
 
 def _peaks():
@@ -149,12 +150,14 @@ def whole_job_rate(per_rank_work: float, world_size: int, ms_max: float) -> floa
 # ------------------------------------------------------------ CPU baseline
 
 
-def cpu_oracle_sample(wl, x, w, budget_s: float):
+def cpu_oracle_sample(wl, x, w, budget_s: float, wf=None):
     """Times the oracle (prune + windows + metadata + fp64 GEMM) on whole rows
     of X until about budget_s seconds have passed.  Returns (dense-equiv
-    TFLOP/s, rows, seconds, threads)."""
+    TFLOP/s, rows, seconds, threads).  wf: W widened to fp64 (set-up, not
+    timed), computed here when not given."""
     import oracle
-    wf = oracle.to_f64(w)                       # weight widening is set-up, not timed
+    if wf is None:
+        wf = oracle.to_f64(w)
     rows_done, t_used = 0, 0.0
     chunk = 16
     while t_used < budget_s and rows_done < wl.T:
@@ -174,11 +177,16 @@ def run_reference(args):
     ws, rank, _ = _dist_env()
     if rank != 0:
         return 0
+    import oracle
     from semi_structured_sparse_nm_b200 import inputs
     wl, x, w = inputs.make_workload(HEADLINE)
+    wf = oracle.to_f64(w)
+    # each step is a bounded sample of the workload: the whole run stays
+    # within about REF_TOTAL_S seconds of oracle time
+    step_s = min(args.ref_step_s, max(0.25, REF_TOTAL_S / (args.warmup + args.steps)))
     times, rows = [], 0
     for i in range(args.warmup + args.steps):
-        tf, r, t, thr = cpu_oracle_sample(wl, x, w, budget_s=args.ref_step_s)
+        tf, r, t, thr = cpu_oracle_sample(wl, x, w, budget_s=step_s, wf=wf)
         if i >= args.warmup:
             times.append(t / r)
             rows = r
