@@ -159,6 +159,7 @@ def cpu_oracle_sample(wl, x, w, budget_s: float, wf=None):
     if wf is None:
         wf = oracle.to_f64(w)
     rows_done, t_used = 0, 0.0
+    t_prune = 0.0
     chunk = 16
     while t_used < budget_s and rows_done < wl.T:
         xs = np.ascontiguousarray(x[rows_done:rows_done + chunk])
@@ -166,10 +167,14 @@ def cpu_oracle_sample(wl, x, w, budget_s: float, wf=None):
         keep = oracle.prune(xs, wl.N, wl.M)
         vals, nib = oracle.compress(xs, keep, wl.M)
         oracle.meta_hw(nib, oracle.lifted_k(wl.K, wl.M))
+        t1 = time.perf_counter()
         oracle.linear_f64(oracle.to_f64(xs, keep), wf)
-        t_used += time.perf_counter() - t0
+        t2 = time.perf_counter()
+        t_prune += t1 - t0
+        t_used += t2 - t0
         rows_done += xs.shape[0]
     flops = 2.0 * rows_done * wl.O * wl.K
+    cpu_oracle_sample.last_split = {"prune_windows_meta_s": t_prune, "fp64_gemm_s": t_used - t_prune}
     return flops / t_used / 1e12, rows_done, t_used, oracle.num_threads()
 
 
@@ -775,7 +780,8 @@ def run_gpu(args):
             tf, rows, t, thr = cpu_oracle_sample(wlh, xh_np, wh_np, budget_s=args.cpu_budget_s)
             line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                                     "sample": f"{rows} of {wlh.T} token rows ({t:.1f} s): prune+windows+"
-                                              f"metadata+fp64 GEMM against all of W"}
+                                              f"metadata+fp64 GEMM against all of W",
+                                    "split_s": getattr(cpu_oracle_sample, "last_split", None)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
