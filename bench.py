@@ -46,7 +46,7 @@ TRAFFIC = {
     ("up_proj_8of16_act", "k_nm_gemm_2cta<224,2,1>"): 232774656 + 46312192,
 }
 OTHERS = ["up_proj_2of4_act", "up_proj_8of16_act_fp8", "up_proj_8of16_act_xf", "down_proj_16of32_act", "slide_6of8_wt_prefill", "slide_6of8_wt_prefill_fp8",
-          "slide_6of8_wt_decode",
+          "slide_6of8_wt_decode", "slide_6of8_wt_decode_fp8",
           "hybrid_decode_b1", "hybrid_decode_b8", "hybrid_decode_b32", "hybrid_decode_b128",
           "spense_mlp_decode_b1", "spense_mlp_decode_b8", "spense_mlp_decode_b32", "spense_mlp_decode_b128",
           "tiny_2of4_act_fp32"]

@@ -238,9 +238,12 @@ int slide_decompose_fp8(const void *w, int64_t rows, int64_t K, int N, int M, ui
 /* Y = (S . D^T) * S_scale[row of S] * D_scale[row of D], or its transpose
  * (side NM_WEIGHT), with S the packed 8-bit sparse operand (S->vals codes,
  * S->meta the 8-bit image) and D the lifted codes [rows_d][S->K_lift].
- * Requires S->K_lift % 128 == 0 and S->rows % 256 == 0 (NM_ERR_UNSUPPORTED
- * otherwise).  The S side may be read while the preceding kernel in the
- * stream finishes, as in nm_sparse_gemm(). */
+ * Requires S->K_lift % 128 == 0, and S->rows % 256 == 0 unless rows_d <= 64
+ * (NM_ERR_UNSUPPORTED otherwise): decode-shaped products -- a few rows of D,
+ * the tokens of a weight-sparse product -- run on single CTAs, 128 rows of S
+ * per tile with split-K over the reduction, and take any row count; larger
+ * ones run on SM pairs.  For NM_WEIGHT, S is a weight operand (see the
+ * conventions at the top). */
 int nm_sparse_gemm_fp8(const nm_sparse_operand *S, const float *S_scale, const void *D, const float *D_scale,
                        int64_t rows_d, nm_side side, void *Y, nm_dtype out_dt, void *stream);
 

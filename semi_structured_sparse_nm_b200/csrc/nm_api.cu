@@ -114,13 +114,22 @@ struct GemmPlan {
   const float* scale_b = nullptr;
 };
 
-template <int BN>
+template <int BN, bool FP8 = false>
 int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
-  using Cfg = nm::GemmCfg<BN>;
+  using Cfg = nm::GemmCfg<BN, FP8>;
   CUtensorMap ta_s, ta_d, tb;
-  const int64_t kb_sparse = ceil_div(p.ks_lift, 128);
+  const int64_t kb_sparse = ceil_div(p.ks_lift, FP8 ? 256 : 128);
   const int64_t kb_dense = ceil_div(p.kd, 64);
   int rc;
+  if (FP8) {
+    // 8-bit codes: A stored [rows_a][K'/2] bytes, B lifted [rows_b][K'] bytes,
+    // boxes of 128 bytes; sparse k-blocks only
+    if ((rc = make_tmap(&ta_s, p.a_s, p.ks_lift / 2, p.rows_a, p.ks_lift / 2, 128, nm::kBM,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_DATA_TYPE_UINT8)) != NM_OK) return rc;
+    if ((rc = make_tmap(&tb, p.b, p.ks_lift, p.rows_b, p.ks_lift, 128, BN, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_DATA_TYPE_UINT8)) != NM_OK) return rc;
+    ta_d = ta_s;
+  } else {
   // output-split: the sparse and the dense A are separate matrices over the
   // same B columns [0, K)
   const bool osplit = p.out_split_rows >= 0;
@@ -136,6 +145,7 @@ int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
   if (kb_sparse == 0 || rows_s == 0) ta_s = ta_d;
   if (kb_dense == 0 || rows_d == 0) ta_d = ta_s;
   if ((rc = make_tmap(&tb, p.b, b_cols, p.rows_b, b_cols * 2, 64, BN)) != NM_OK) return rc;
+  }
 
   nm::GemmArgs args{};
   args.rows_a = p.rows_a;
@@ -144,20 +154,22 @@ int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
   args.kb_dense = static_cast<int>(kb_dense);
   args.k_dense_x0 = p.ks_lift;
   args.meta = p.meta;
-  args.meta_kb = kb_sparse;
+  args.meta_kb = FP8 ? ceil_div(p.ks_lift, 128) : kb_sparse;
   args.Y = p.y;
   args.ldy = p.ldy;
   args.out_fp32 = p.out_fp32;
   args.transpose_out = p.transpose;
   args.splits = splits;
   args.a_static = p.a_static;
-  args.out_split_tiles = osplit ? static_cast<int>(p.out_split_rows / nm::kBM) : -1;
-  args.row_scale = p.row_scale;
+  args.out_split_tiles = p.out_split_rows >= 0 ? static_cast<int>(p.out_split_rows / nm::kBM) : -1;
+  args.row_scale = FP8 ? p.scale_a : p.row_scale;
+  args.col_scale = FP8 ? p.scale_b : nullptr;
   args.row_shift = p.row_shift;
   args.col_sum = p.col_sum;
-  if (osplit) args.k_dense_x0 = 0;
+  args.fp8_last_half = (FP8 && p.ks_lift % 256 != 0) ? 1 : 0;
+  if (p.out_split_rows >= 0) args.k_dense_x0 = 0;
 
-  auto kern = nm::k_nm_gemm<BN>;
+  auto kern = nm::k_nm_gemm<BN, FP8>;
   NM_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
 
   cudaLaunchConfig_t cfg{};
@@ -753,7 +765,14 @@ int nm_sparse_gemm_fp8(const nm_sparse_operand* S, const float* S_scale, const v
   if (S->rows < 0 || rows_d < 0 || S->K <= 0 || S->M <= 0 || S->K % S->M != 0) return NM_ERR_INVALID_ARG;
   if (!m_supported(S->M)) return NM_ERR_UNSUPPORTED;
   if (S->K_lift != nm_lifted_k(S->K, S->M)) return NM_ERR_INVALID_ARG;
-  if (S->K_lift % 128 != 0 || S->rows % 256 != 0) return NM_ERR_UNSUPPORTED;
+  if (S->K_lift % 128 != 0) return NM_ERR_UNSUPPORTED;
+  const char* env = std::getenv("NMSPARSE_GEMM");
+  const std::string mode = env != nullptr ? env : "auto";
+  // decode-shaped products (a few rows of B) and NMSPARSE_GEMM=1cta take the
+  // single-CTA kernel (any row count); the SM-pair kernel needs whole
+  // 256-row blocks of the sparse operand
+  const bool single = mode == "1cta" || (mode == "auto" && rows_d <= 64);
+  if (!single && S->rows % 256 != 0) return NM_ERR_UNSUPPORTED;
   if (S->rows == 0 || rows_d == 0) return NM_OK;
   if (D == nullptr || Y == nullptr || S->vals == nullptr || S->meta == nullptr || S_scale == nullptr ||
       D_scale == nullptr)
@@ -777,9 +796,21 @@ int nm_sparse_gemm_fp8(const nm_sparse_operand* S, const float* S_scale, const v
   p.fp8 = 1;
   p.scale_a = S_scale;
   p.scale_b = D_scale;
-  const char* env = std::getenv("NMSPARSE_GEMM");
-  const std::string mode = env != nullptr ? env : "auto";
   auto st = static_cast<cudaStream_t>(stream);
+  // Decode-shaped products (a few rows of B: tokens of a weight-sparse
+  // product) run on single CTAs, 128 rows of A per tile, with cluster split-K
+  // over the reduction.
+  if (single) {
+    const int bn1 = pick_bn(p.rows_b);
+    const int64_t tiles1 = ceil_div(p.rows_a, int64_t(nm::kBM)) * ceil_div(p.rows_b, int64_t(bn1));
+    const int splits = pick_splits(tiles1, ceil_div(p.ks_lift, int64_t(256)));
+    switch (bn1) {
+      case 16: return launch_gemm_bn<16, true>(p, splits, st);
+      case 32: return launch_gemm_bn<32, true>(p, splits, st);
+      case 64: return launch_gemm_bn<64, true>(p, splits, st);
+      default: return launch_gemm_bn<128, true>(p, splits, st);
+    }
+  }
   int bn = 0;
   if (mode == "2cta224") bn = 224;
   if (mode == "2cta192") bn = 192;

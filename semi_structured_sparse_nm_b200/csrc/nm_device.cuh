@@ -172,6 +172,17 @@ __device__ __forceinline__ void tc_mma_sp_f16(uint32_t d_tmem, uint64_t adesc, u
       :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(e_tmem)
       : "memory");
 }
+// The same for 8-bit operands: kind::f8f6f4 (E4M3 x E4M3 through the
+// instruction descriptor), K = 64 per instruction.
+__device__ __forceinline__ void tc_mma_sp_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t e_tmem, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::f8f6f4 [%0], %1, %2, [%5], %3, p;\n\t}"
+      :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(e_tmem)
+      : "memory");
+}
 // D(tmem) (+)= A(smem) * B(smem)^T, dense.
 __device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                            uint32_t idesc, uint32_t accumulate) {

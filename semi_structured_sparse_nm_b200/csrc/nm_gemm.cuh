@@ -47,22 +47,30 @@ struct GemmArgs {
                                             // preceding kernel finishes; B only after
   int out_split_tiles;                      // -1, or the number of sparse row tiles of an
                                             // output-split product
-  // affine epilogue of the per-token activation corrections (all three or
-  // none): y = acc * row_scale[a] + row_shift[a] * col_sum[b]
+  // epilogue scaling: y = (acc * row_scale[a]) * col_scale[b] + row_shift[a] *
+  // col_sum[b], each factor or term left out when its pointer is null (the
+  // per-token corrections: row_scale, row_shift, col_sum; the 8-bit product:
+  // row_scale, col_scale)
   const float* row_scale;
   const float* row_shift;
   const float* col_sum;
+  const float* col_scale;
+  int fp8_last_half;                        // 8-bit product: the last k-block holds only 128 lifted K
 };
 
-template <int BN>
+// FP8: a sparse k-block is 256 lifted K of E4M3 codes (A 128 stored bytes
+// per row, B two 128-byte halves, two metadata blocks into 8 TMEM columns).
+template <int BN, bool FP8 = false>
 struct GemmCfg {
   static constexpr bool kPush = BN <= 32;                        // push split-K reduction
   static constexpr int kRecvBytes = kPush ? kBM * BN * 4 : 0;    // [splits][128/splits][BN] fp32
   static constexpr int kBBytes = 2 * BN * 128;
-  static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
+  static constexpr int kEStage = FP8 ? 2 * kEBytes : kEBytes;    // metadata bytes per stage
+  static constexpr int kMetaCols = FP8 ? 8 : 4;                  // TMEM columns of metadata per stage
+  static constexpr int kStageBytes = kABytes + kBBytes + kEStage;
   static constexpr int kStagesRaw = (200 * 1024) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr int kTmemNeed = BN + 4 * kStages;
+  static constexpr int kTmemNeed = BN + kMetaCols * kStages;
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                  : kTmemNeed <= 256 ? 256 : 512;
   static constexpr int kSmemBytes = kStages * kStageBytes + kRecvBytes + 1024 /*align*/ + 256 /*barriers*/;
@@ -116,10 +124,16 @@ __device__ __forceinline__ void store_out_raw(const GemmArgs& a, int64_t ra, int
   else static_cast<__nv_bfloat16*>(a.Y)[off] = __float2bfloat16_rn(v);
 }
 
+__device__ __forceinline__ float scale_out(const GemmArgs& a, int64_t ra, int64_t cb, float v) {
+  if (a.row_scale != nullptr) v = v * a.row_scale[ra];
+  if (a.col_scale != nullptr) v = v * a.col_scale[cb];
+  if (a.row_shift != nullptr) v = __fmaf_rn(a.row_shift[ra], a.col_sum[cb], v);
+  return v;
+}
+
 __device__ __forceinline__ void store_out(const GemmArgs& a, int64_t ra, int64_t cb, float v) {
   if (ra >= a.rows_a || cb >= a.rows_b) return;
-  if (a.row_scale != nullptr) v = __fmaf_rn(a.row_shift[ra], a.col_sum[cb], v * a.row_scale[ra]);
-  store_out_raw(a, ra, cb, v);
+  store_out_raw(a, ra, cb, scale_out(a, ra, cb, v));
 }
 
 // Stores CW (16 or 32) consecutive accumulator columns of row `ra`
@@ -131,13 +145,10 @@ __device__ __forceinline__ void store_row_chunk(const GemmArgs& a, int64_t ra, i
   uint32_t v[CW];
 #pragma unroll
   for (int i = 0; i < CW; ++i) v[i] = v_in[i];
-  if (a.row_scale != nullptr) {
-    const float sc = a.row_scale[ra], mu = a.row_shift[ra];
+  if (a.row_scale != nullptr || a.col_scale != nullptr || a.row_shift != nullptr) {
 #pragma unroll
-    for (int i = 0; i < CW; ++i) {
-      const float cs = cb0 + i < a.rows_b ? a.col_sum[cb0 + i] : 0.0f;
-      v[i] = __float_as_uint(__fmaf_rn(mu, cs, __uint_as_float(v[i]) * sc));
-    }
+    for (int i = 0; i < CW; ++i)
+      if (cb0 + i < a.rows_b) v[i] = __float_as_uint(scale_out(a, ra, cb0 + i, __uint_as_float(v[i])));
   }
   if (a.transpose_out && cb0 + CW <= a.rows_b) {
     // Y[b][a]: lane = a, so each store instruction of the warp writes 32
@@ -180,19 +191,19 @@ __device__ __forceinline__ void store_row_chunk(const GemmArgs& a, int64_t ra, i
   for (int i = 0; i < CW; ++i) store_out_raw(a, ra, cb0 + i, __uint_as_float(v[i]));
 }
 
-template <int BN>
+template <int BN, bool FP8 = false>
 __global__ void __launch_bounds__(192, 1)
 k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUtensorMap tmA_d,
           const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<BN, FP8>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + S * kABytes;
   uint8_t* sE = sB + S * Cfg::kBBytes;
-  float* sRecv = reinterpret_cast<float*>(sE + S * kEBytes);
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(sE + S * kEBytes + Cfg::kRecvBytes);
+  float* sRecv = reinterpret_cast<float*>(sE + S * Cfg::kEStage);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(sE + S * Cfg::kEStage + Cfg::kRecvBytes);
   uint64_t* empty_bar = full_bar + S;
   uint64_t* accum_bar = empty_bar + S;
   uint64_t* red_bar = accum_bar + 1;
@@ -243,12 +254,22 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
     if (elect_one()) {
       const int32_t y_a = static_cast<int32_t>((dense_tile ? m_tile - tsp : m_tile) * kBM);
       const int32_t y_b = static_cast<int32_t>(n_tile * BN);
+      // 8-bit: metadata blocks (and B halves) in this k-block, 1 for a last
+      // block of 128 lifted K
+      auto halves = [&](int kb) { return (FP8 && args.fp8_last_half && kb == args.kb_sparse - 1) ? 1 : 2; };
       auto load_a = [&](int kb, int s) {
         uint8_t* a_dst = sA + s * kABytes;
-        if (kb < args.kb_sparse) {
+        if constexpr (FP8) {
+          const int eb = halves(kb);
+          mbar_arrive_expect_tx(&full_bar[s], kABytes + BN * 128 * eb + kEBytes * eb);
+          tma_load_2d(&tmA_s, &full_bar[s], a_dst, kb * 128, y_a);
+          for (int e = 0; e < eb; ++e)
+            bulk_load(sE + s * Cfg::kEStage + e * kEBytes, args.meta + (m_tile * args.meta_kb + 2 * kb + e) * kEBytes,
+                      kEBytes, &full_bar[s]);
+        } else if (kb < args.kb_sparse) {
           mbar_arrive_expect_tx(&full_bar[s], kABytes + Cfg::kBBytes + kEBytes);
           tma_load_2d(&tmA_s, &full_bar[s], a_dst, kb * 64, y_a);
-          bulk_load(sE + s * kEBytes, args.meta + (m_tile * args.meta_kb + kb) * kEBytes, kEBytes,
+          bulk_load(sE + s * Cfg::kEStage, args.meta + (m_tile * args.meta_kb + kb) * kEBytes, kEBytes,
                     &full_bar[s]);
         } else {
           mbar_arrive_expect_tx(&full_bar[s], kABytes + BN * 128);
@@ -257,7 +278,10 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
       };
       auto load_b = [&](int kb, int s) {
         uint8_t* b_dst = sB + s * Cfg::kBBytes;
-        if (kb < args.kb_sparse) {
+        if constexpr (FP8) {
+          tma_load_2d(&tmB, &full_bar[s], b_dst, kb * 256, y_b);
+          if (halves(kb) == 2) tma_load_2d(&tmB, &full_bar[s], b_dst + BN * 128, kb * 256 + 128, y_b);
+        } else if (kb < args.kb_sparse) {
           tma_load_2d(&tmB, &full_bar[s], b_dst, kb * 128, y_b);
           tma_load_2d(&tmB, &full_bar[s], b_dst + BN * 128, kb * 128 + 64, y_b);
         } else {
@@ -303,9 +327,25 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
         tc_fence_after();
         const uint32_t a0 = smem_u32(sA + s * kABytes);
         const uint32_t b0 = smem_u32(sB + s * Cfg::kBBytes);
-        if (kb < args.kb_sparse) {
+        if constexpr (FP8) {
+          // two metadata blocks -> columns e_col, e_col + 4; MMA kk (64
+          // lifted K) reads the column pair at e_col + 2 kk
+          const uint32_t e_col = tmem_meta + static_cast<uint32_t>(Cfg::kMetaCols) * s;
+          const int nkk = (args.fp8_last_half && kb == args.kb_sparse - 1) ? 2 : 4;
+          for (int e = 0; e < nkk / 2; ++e)
+            tc_cp_128x128b(e_col + 4u * e, desc_plain_128x16(smem_u32(sE + s * Cfg::kEStage + e * kEBytes)));
+          const uint32_t idesc8 = idesc_e4m3(kBM, BN, true);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            if (kk < nkk) {
+              const uint64_t ad = desc_sw128_kmajor(a0 + 32u * kk);
+              const uint64_t bd = desc_sw128_kmajor(b0 + (kk / 2) * (BN * 128) + (kk % 2) * 64);
+              tc_mma_sp_e4m3(tmem_acc, ad, bd, e_col + 2u * kk, idesc8, (it > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
+        } else if (kb < args.kb_sparse) {
           const uint32_t e_col = tmem_meta + 4u * s;
-          tc_cp_128x128b(e_col, desc_plain_128x16(smem_u32(sE + s * kEBytes)));
+          tc_cp_128x128b(e_col, desc_plain_128x16(smem_u32(sE + s * Cfg::kEStage)));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t ad = desc_sw128_kmajor(a0 + 32u * kk);

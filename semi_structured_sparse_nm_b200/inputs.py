@@ -128,6 +128,7 @@ WORKLOADS = {
         Workload("up_proj_8of16_act_xf", "act", 2048, 4096, 14336, 8, 16, "bf16", "bf16", "student_t4", xf=3),
         Workload("slide_6of8_wt_prefill", "weight", 4096, 4096, 4096, 6, 8, "bf16", "bf16", "normal"),
         Workload("slide_6of8_wt_decode", "weight", 16, 4096, 4096, 6, 8, "bf16", "bf16", "normal"),
+        Workload("slide_6of8_wt_decode_fp8", "weight", 16, 4096, 4096, 6, 8, "bf16", "bf16", "normal", fp8=True),
         # the same prefill product with 8-bit operands (the pages' B200 precision)
         Workload("slide_6of8_wt_prefill_fp8", "weight", 4096, 4096, 4096, 6, 8, "bf16", "bf16", "normal",
                  fp8=True),

@@ -98,12 +98,17 @@ def test_fp8_full_size_sampled_rows():
 
 
 def test_fp8_unsupported_shapes_launch_nothing():
-    w = dev(inputs.normal_bf16((130, 512), 0.02, 1))
-    P = nm.slide_decompose_fp8(w, 6, 8)                       # packing works for any row count
-    q = nm.quant_lift_fp8(dev(inputs.normal_bf16((8, 512), 1.0, 2)), 8)
+    w_np = inputs.normal_bf16((130, 512), 0.02, 1)
+    P = nm.slide_decompose_fp8(dev(w_np), 6, 8)              # packing works for any row count
+    q = nm.quant_lift_fp8(dev(inputs.normal_bf16((100, 512), 1.0, 2)), 8)
     with pytest.raises(nm.NmError) as e:
-        nm.sparse_gemm_fp8(P, q, nm.NM_WEIGHT)                # the product needs whole 256-row blocks
+        nm.sparse_gemm_fp8(P, q, nm.NM_WEIGHT)                # 100 tokens: SM pairs, whole 256-row blocks
     assert e.value.status == nm.NM_ERR_UNSUPPORTED
+    # a decode shape (8 tokens) runs on single CTAs, which take the 130 rows
+    x8 = inputs.normal_bf16((8, 512), 1.0, 2)
+    y = nm.sparse_gemm_fp8(P, nm.quant_lift_fp8(dev(x8), 8), nm.NM_WEIGHT, torch.float32)
+    torch.cuda.synchronize()
+    check_close(host_f64(y), oracle.fp8_weight_sparse_linear(x8, w_np, 6, 8), "fp8 130 rows, 8 tokens")
     with pytest.raises(nm.NmError) as e:
         nm.quant_lift_fp8(dev(inputs.normal_bf16((4, 40), 1.0, 3)), 8)   # K' = 60: not a multiple of 16
     assert e.value.status == nm.NM_ERR_UNSUPPORTED
@@ -149,3 +154,63 @@ def test_fp8_act_full_size_sampled_rows():
     rows = np.array([0, 1, 127, 128, 1000, 2047])
     check_close(host_f64(y[torch.from_numpy(rows).cuda()]),
                 oracle.fp8_act_sparse_linear(x, w, wl.N, wl.M, rows=rows), "fp8 act full size")
+
+
+# ------------------------------------------------ decode shapes (single-CTA kernel)
+
+
+@pytest.mark.parametrize("variant", ["auto", "1cta"])
+@pytest.mark.parametrize("T,O,K,N,M", [
+    (1, 256, 1024, 6, 8),       # one token
+    (16, 512, 768, 6, 8),       # K' = 1152: the last block holds 128 K
+    (33, 384, 2048, 14, 16),
+    (64, 256, 640, 2, 4),       # 2:4, half last block
+    (200, 256, 1024, 30, 32),   # wider than a decode tile: 1cta only when forced
+])
+def test_fp8_weight_sparse_single_cta(monkeypatch, variant, T, O, K, N, M):
+    monkeypatch.setenv("NMSPARSE_GEMM", variant)
+    x = inputs.student_t_bf16((T, K), 4.0, seed=T + 11)
+    w = inputs.normal_bf16((O, K), 0.02, seed=O + 11)
+    P = nm.slide_decompose_fp8(dev(w), N, M)
+    q = nm.quant_lift_fp8(dev(x), M)
+    for out_dt in (torch.float32, torch.bfloat16):
+        y = nm.sparse_gemm_fp8(P, q, nm.NM_WEIGHT, out_dt)
+        torch.cuda.synchronize()
+        assert nm.device_error() == nm.NM_OK
+        check_close(host_f64(y), oracle.fp8_weight_sparse_linear(x, w, N, M), f"fp8 1cta {T}x{O}x{K} {N}:{M}")
+
+
+def test_fp8_act_sparse_single_cta(monkeypatch):
+    monkeypatch.setenv("NMSPARSE_GEMM", "1cta")
+    T, O, K, N, M = 256, 200, 1024, 8, 16
+    x = inputs.student_t_bf16((T, K), 4.0, seed=5)
+    w = inputs.normal_bf16((O, K), 0.02, seed=6)
+    P = nm.prune_compress_fp8(dev(x), N, M)
+    y = nm.sparse_gemm_fp8(P, nm.quant_lift_fp8(dev(w), M), nm.NM_ACT, torch.float32)
+    torch.cuda.synchronize()
+    check_close(host_f64(y), oracle.fp8_act_sparse_linear(x, w, N, M), "fp8 act 1cta")
+
+
+def test_fp8_single_cta_exact_on_integer_grid():
+    rng = np.random.default_rng(19)
+
+    def make(rows, K):
+        v = rng.integers(-16, 17, size=(rows, K)).astype(np.float64)
+        v[:, 0] = 448.0
+        return inputs.bf16_from_f64(v)
+    x, w = make(16, 1536), make(512, 1536)
+    P = nm.slide_decompose_fp8(dev(w), 6, 8)
+    y = nm.sparse_gemm_fp8(P, nm.quant_lift_fp8(dev(x), 8), nm.NM_WEIGHT, torch.float32)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(host_f64(y), oracle.fp8_weight_sparse_linear(x, w, 6, 8))
+
+
+def test_fp8_decode_full_size():
+    """The 6:8 weight-sparse decode workload (T = 16, K = O = 4096) in 8 bits,
+    every output against the oracle."""
+    wl, x, w = inputs.make_workload("slide_6of8_wt_decode")
+    P = nm.slide_decompose_fp8(dev(w), wl.N, wl.M)
+    y = nm.sparse_gemm_fp8(P, nm.quant_lift_fp8(dev(x), wl.M), nm.NM_WEIGHT, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    check_close(host_f64(y), oracle.fp8_weight_sparse_linear(x, w, wl.N, wl.M), "fp8 decode full size")
