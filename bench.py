@@ -43,7 +43,7 @@ HEADLINE = "up_proj_8of16_act"
 # dominant kernel, from one ncu capture of the kernel as it stands (see
 # profiles/); drop an entry whenever that kernel changes.
 TRAFFIC = {
-    ("up_proj_8of16_act", "k_nm_gemm_2cta<224,2,1>"): 232774656 + 46312192,
+    ("up_proj_8of16_act", "k_nm_gemm_2cta<224,2,1>"): 233678592 + 46385664,
 }
 OTHERS = ["up_proj_2of4_act", "up_proj_8of16_act_fp8", "up_proj_8of16_act_xf", "down_proj_16of32_act", "slide_6of8_wt_prefill", "slide_6of8_wt_prefill_fp8",
           "slide_6of8_wt_decode", "slide_6of8_wt_decode_fp8",
@@ -584,10 +584,16 @@ def time_dense_mlp(wk, reps=20):
 def mma_probe():
     """The library's tensor-core rate probe (MMAs from shared memory on every
     SM pair, no loads): the rate the GEMMs' MMA instructions can reach at
-    this moment's clocks, in TFLOP/s dense-equivalent."""
+    this moment's clocks, in TFLOP/s dense-equivalent, with the SM clock seen
+    while it ran (a pure tensor loop can hit the power cap)."""
+    import torch
     from semi_structured_sparse_nm_b200 import _lib as nm
-    return {"bf16_dense": nm.mma_rate_probe(0), "bf16_sparse": nm.mma_rate_probe(1),
-            "e4m3_sparse": nm.mma_rate_probe(2)}
+    clk = ClockSampler(torch.cuda.current_device())
+    with clk:
+        out = {"bf16_dense": nm.mma_rate_probe(0), "bf16_sparse": nm.mma_rate_probe(1),
+               "e4m3_sparse": nm.mma_rate_probe(2)}
+    out["clocks"] = clk.summary()
+    return out
 
 
 def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None, probe=None):

@@ -376,15 +376,16 @@ int hybrid_gemm_noalloc(const void *X, int64_t B, const nm_hybrid_weight *W, voi
  * y_host[T][O] = prune_{N:M}(x_host) . W^T, x_host bf16 [T][K] and y_host bf16
  * [T][O] in HOST memory (row-major, row strides K and O), w_lift the
  * device-resident lifted weight [O][K'] (nm_lift()).  The rows go through in
- * chunks of chunk_rows (a multiple of 128; 0 = 256): each chunk is copied in
- * on one auxiliary stream, pruned and multiplied on `stream`, and copied out
- * on another auxiliary stream, two chunks in flight, so that the copies of
- * one chunk overlap the math of its neighbours.  The auxiliary streams and
- * their events are created on the first call on a device and kept; calls are
- * serialised on the host.  Host buffers should be page-locked
+ * chunks of chunk_rows (a multiple of 128; 0 = 256): each chunk is copied in,
+ * pruned and multiplied on `stream` and copied out on an auxiliary stream,
+ * two chunks in flight, so that the copies out (the larger transfer) overlap
+ * the copies in and the math of the following chunks.  The auxiliary stream
+ * and its events are created on the first call on a device and kept; calls
+ * are serialised on the host.  Host buffers should be page-locked
  * (cudaHostAlloc / cudaHostRegister), else the copies are not asynchronous.
  * Returns once everything is enqueued; y_host is complete when `stream`
- * reaches the point of the call.  Not for stream capture.
+ * reaches the point of the call, and both host buffers must stay allocated
+ * until then.  Not for stream capture.
  * ws: nm_act_sparse_linear_host_workspace_size() bytes of device scratch (two
  * slots of: the chunk of X, its compressed values and metadata, the chunk of
  * Y), 16-byte aligned.  Results equal those of nm_prune_compress() +

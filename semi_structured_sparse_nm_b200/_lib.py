@@ -313,7 +313,8 @@ def act_sparse_linear_host(x_host: torch.Tensor, W_lift: torch.Tensor, N: int, M
                            ws: torch.Tensor | None = None, chunk_rows: int = 0) -> torch.Tensor:
     """y_host = prune_{N:M}(x_host) . W^T with x_host, y_host bf16 tensors in
     (page-locked) host memory and the lifted weight on the device; chunked
-    copies in and out overlap the math.  Asynchronous on the current stream."""
+    copies in and out overlap the math.  Asynchronous on the current stream:
+    keep x_host and y_host alive until the stream has passed the call."""
     _need_cuda(W_lift)
     if x_host.is_cuda or y_host.is_cuda:
         raise ValueError("x_host and y_host live in host memory")

@@ -1127,14 +1127,13 @@ int hybrid_gemm_noalloc(const void* X, int64_t B, const nm_hybrid_weight* W, voi
 }  // extern "C"
 
 namespace {
-// Two auxiliary streams (copies in, copies out) and the events that chain
-// the two buffer slots of the chunked host-buffer pipeline, one set per
-// device, created on first use and kept until the process exits.
+// The auxiliary stream of the chunked host-buffer pipeline (copies out) and
+// the events that chain its two buffer slots, one set per device, created on
+// first use and kept until the process exits.
 struct HostPipe {
   bool ready = false;
-  cudaStream_t s_in = nullptr, s_out = nullptr;
-  cudaEvent_t start = nullptr;
-  cudaEvent_t in[2] = {}, done[2] = {}, out[2] = {};
+  cudaStream_t s_out = nullptr;
+  cudaEvent_t done[2] = {}, out[2] = {};
 };
 std::mutex g_pipe_mu;
 HostPipe g_pipe[kMaxDevices];
@@ -1145,11 +1144,8 @@ int host_pipe(HostPipe** out) {
   if (dev < 0 || dev >= kMaxDevices) return NM_ERR_UNSUPPORTED;
   HostPipe& p = g_pipe[dev];
   if (!p.ready) {
-    NM_CUDA_TRY(cudaStreamCreateWithFlags(&p.s_in, cudaStreamNonBlocking));
     NM_CUDA_TRY(cudaStreamCreateWithFlags(&p.s_out, cudaStreamNonBlocking));
-    NM_CUDA_TRY(cudaEventCreateWithFlags(&p.start, cudaEventDisableTiming));
     for (int b = 0; b < 2; ++b) {
-      NM_CUDA_TRY(cudaEventCreateWithFlags(&p.in[b], cudaEventDisableTiming));
       NM_CUDA_TRY(cudaEventCreateWithFlags(&p.done[b], cudaEventDisableTiming));
       NM_CUDA_TRY(cudaEventCreateWithFlags(&p.out[b], cudaEventDisableTiming));
     }
@@ -1203,9 +1199,6 @@ int nm_act_sparse_linear_host(const void* x_host, int64_t T, int64_t K, int N, i
   std::lock_guard<std::mutex> lock(g_pipe_mu);
   HostPipe* p = nullptr;
   if ((rc = host_pipe(&p)) != NM_OK) return rc;
-  // copies in start after the work already on `stream`
-  NM_CUDA_TRY(cudaEventRecord(p->start, st));
-  NM_CUDA_TRY(cudaStreamWaitEvent(p->s_in, p->start, 0));
   const int64_t chunks = ceil_div(T, Tc);
   for (int64_t c = 0; c < chunks; ++c) {
     const int b = static_cast<int>(c % 2);
@@ -1214,15 +1207,13 @@ int nm_act_sparse_linear_host(const void* x_host, int64_t T, int64_t K, int N, i
     uint8_t* vals = xd + round256(Tc * K * 2);
     uint8_t* meta = vals + round256(Tc * (Kl / 2) * 2);
     uint8_t* yd = meta + round256(static_cast<int64_t>(nm_meta_bytes(Tc, K, M)));
-    // copy in: slot b's X is free once the prune of chunk c - 2 has read it
-    NM_CUDA_TRY(cudaStreamWaitEvent(p->s_in, p->done[b], 0));
-    NM_CUDA_TRY(cudaMemcpyAsync(xd, static_cast<const uint8_t*>(x_host) + r0 * K * 2, static_cast<size_t>(rows * K * 2),
-                                cudaMemcpyHostToDevice, p->s_in));
-    NM_CUDA_TRY(cudaEventRecord(p->in[b], p->s_in));
-    // prune + GEMM on the caller's stream; slot b's Y is free once the copy
-    // out of chunk c - 2 has read it
-    NM_CUDA_TRY(cudaStreamWaitEvent(st, p->in[b], 0));
+    // Copy in, prune and GEMM in order on the caller's stream (the copy sits
+    // between the kernels of consecutive chunks, so each chunk's kernels
+    // start only after its copy has landed).  Slot b's Y is free once the
+    // copy out of chunk c - 2 has read it.
     NM_CUDA_TRY(cudaStreamWaitEvent(st, p->out[b], 0));
+    NM_CUDA_TRY(cudaMemcpyAsync(xd, static_cast<const uint8_t*>(x_host) + r0 * K * 2, static_cast<size_t>(rows * K * 2),
+                                cudaMemcpyHostToDevice, st));
     if ((rc = nm_prune_compress(xd, NM_BF16, rows, K, K, N, M, nullptr, vals, meta, stream)) != NM_OK) return rc;
     nm_sparse_operand S{};
     S.vals = vals;

@@ -45,7 +45,8 @@ def test_host_pipeline_exact_on_integers():
     x = inputs.bf16_from_f64(rng.integers(-8, 9, size=(T, K)).astype(np.float64))
     w = inputs.bf16_from_f64(rng.integers(-3, 4, size=(O, K)).astype(np.float64))
     yh = torch.empty((T, O), dtype=torch.bfloat16).pin_memory()
-    nm.act_sparse_linear_host(_host(x), nm.lift(dev(w), 8), 4, 8, yh)
+    xh = _host(x)
+    nm.act_sparse_linear_host(xh, nm.lift(dev(w), 8), 4, 8, yh)
     torch.cuda.synchronize()
     ref = oracle.act_sparse_linear(x, w, 4, 8)
     np.testing.assert_array_equal(inputs.bf16_to_f64(host_bits(yh)), inputs.bf16_to_f64(inputs.bf16_from_f64(ref)))
@@ -62,8 +63,9 @@ def test_host_pipeline_back_to_back_calls_reuse_buffers():
     ws = nm.act_sparse_linear_host_workspace(T, K, 8, 16, O, Wl.device)
     y1 = torch.empty((T, O), dtype=torch.bfloat16).pin_memory()
     y2 = torch.empty((T, O), dtype=torch.bfloat16).pin_memory()
-    nm.act_sparse_linear_host(_host(x1), Wl, 8, 16, y1, ws=ws)
-    nm.act_sparse_linear_host(_host(x2), Wl, 8, 16, y2, ws=ws)
+    h1, h2 = _host(x1), _host(x2)          # host inputs stay alive until the copies have run
+    nm.act_sparse_linear_host(h1, Wl, 8, 16, y1, ws=ws)
+    nm.act_sparse_linear_host(h2, Wl, 8, 16, y2, ws=ws)
     torch.cuda.synchronize()
     check_close(inputs.bf16_to_f64(host_bits(y1)), oracle.act_sparse_linear(x1, w, 8, 16), "first call")
     check_close(inputs.bf16_to_f64(host_bits(y2)), oracle.act_sparse_linear(x2, w, 8, 16), "second call")
