@@ -178,6 +178,19 @@ def cpu_oracle_sample(wl, x, w, budget_s: float, wf=None):
     return flops / t_used / 1e12, rows_done, t_used, oracle.num_threads()
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), for the CPU baseline."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def run_reference(args):
     ws, rank, _ = _dist_env()
     if rank != 0:
@@ -204,7 +217,8 @@ def run_reference(args):
         "ms_per_step": per_row * wl.T * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": HEADLINE, "T": wl.T, "K": wl.K, "O": wl.O, "N": wl.N, "M": wl.M},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle", "sample": sample,
+                         "cpu": cpu_model(), "nproc": os.cpu_count()},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -787,7 +801,8 @@ def run_gpu(args):
             line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                                     "sample": f"{rows} of {wlh.T} token rows ({t:.1f} s): prune+windows+"
                                               f"metadata+fp64 GEMM against all of W",
-                                    "split_s": getattr(cpu_oracle_sample, "last_split", None)}
+                                    "split_s": getattr(cpu_oracle_sample, "last_split", None),
+                                    "cpu": cpu_model(), "nproc": os.cpu_count()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
