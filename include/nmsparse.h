@@ -405,6 +405,12 @@ int nm_last_cuda_error(void);
  * kernels set when a bounded wait expires: NM_OK or NM_ERR_DEVICE_TIMEOUT
  * (or NM_ERR_CUDA if the synchronisation itself failed). */
 int nm_get_device_error(void *stream);
+/* Test hook for the launch-error path: the next kernel launch made by a call
+ * of this library on the calling thread fails with cudaError_t `cuda_error`
+ * (0 clears the hook) instead of launching, so that the call returns
+ * NM_ERR_CUDA and nm_last_cuda_error() reports the code.  Nothing reaches
+ * the GPU. */
+int nm_debug_fail_next_launch(int cuda_error);
 /* Test hook for the bounded-wait path: launches one CTA that waits on an
  * mbarrier no thread ever arrives on, giving up after timeout_us
  * microseconds and recording NM_ERR_DEVICE_TIMEOUT.  Faults nothing. */

@@ -92,6 +92,7 @@ def lib():
             "nm_last_cuda_error": (I, []),
             "nm_get_device_error": (I, [P]),
             "nm_debug_expire_wait": (I, [ctypes.c_uint, P]),
+            "nm_debug_fail_next_launch": (I, [I]),
             "nm_version": (ctypes.c_char_p, []),
         }
         for name, (res, args) in sigs.items():
@@ -505,6 +506,14 @@ def mma_rate_probe(mode: int, iters: int = 4000, reps: int = 5) -> float:
         e1.synchronize()
         best = min(best, e0.elapsed_time(e1))
     return flops.value / (best * 1e-3) / 1e12
+
+
+def debug_fail_next_launch(cuda_error: int):
+    _check("nm_debug_fail_next_launch", lib().nm_debug_fail_next_launch(cuda_error))
+
+
+def last_cuda_error() -> int:
+    return int(lib().nm_last_cuda_error())
 
 
 def debug_expire_wait(timeout_us: int):

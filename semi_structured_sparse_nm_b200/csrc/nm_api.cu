@@ -25,6 +25,15 @@
 namespace {
 
 thread_local int g_last_cuda_error = 0;
+// Test hook (nm_debug_fail_next_launch): the next kernel launch on this
+// thread returns this error instead of launching (0: none).
+thread_local int g_fail_next_launch = 0;
+
+cudaError_t injected_launch_error() {
+  const int c = g_fail_next_launch;
+  g_fail_next_launch = 0;
+  return static_cast<cudaError_t>(c);
+}
 
 int cuda_fail(cudaError_t e) {
   g_last_cuda_error = static_cast<int>(e);
@@ -91,6 +100,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (g_fail_next_launch != 0) return injected_launch_error();
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
@@ -195,6 +205,7 @@ int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
+  if (g_fail_next_launch != 0) NM_CUDA_TRY(injected_launch_error());
   NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta_s, ta_d, tb, args));
   NM_CUDA_TRY(cudaGetLastError());
   return NM_OK;
@@ -338,6 +349,7 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
+  if (g_fail_next_launch != 0) NM_CUDA_TRY(injected_launch_error());
   NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta, tb, te, ty, tad, a));
   NM_CUDA_TRY(cudaGetLastError());
   return NM_OK;
@@ -1260,6 +1272,12 @@ int nm_get_device_error(void* stream) {
   const unsigned zero = 0;
   NM_CUDA_TRY(cudaMemcpyToSymbol(nm::g_status, &zero, sizeof(zero)));
   return static_cast<int>(v);
+}
+
+int nm_debug_fail_next_launch(int cuda_error) {
+  if (cuda_error < 0) return NM_ERR_INVALID_ARG;
+  g_fail_next_launch = cuda_error;
+  return NM_OK;
 }
 
 int nm_debug_expire_wait(unsigned timeout_us, void* stream) {

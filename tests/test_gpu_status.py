@@ -54,3 +54,34 @@ def test_mma_rate_probe():
     assert 500.0 < dense < 2600.0, dense
     assert 1.5 * dense < sp16 < 2.2 * dense, (dense, sp16)
     assert 1.5 * sp16 < sp8 < 2.2 * sp16, (sp16, sp8)
+
+
+def test_injected_launch_error_launches_nothing():
+    """A launch that fails (injected on the host) makes the call return
+    NM_ERR_CUDA with the error code; nothing runs, the outputs keep their
+    contents, and the next call works."""
+    x = inputs.normal_bf16((48, 512), 1.0, 3)
+    w = inputs.normal_bf16((96, 512), 0.02, 4)
+    comp = nm.alloc_compressed(48, 512, 8, 16, "cuda")
+    comp.vals.fill_(7.0)
+    before = comp.vals.clone()
+    nm.debug_fail_next_launch(701)
+    with pytest.raises(nm.NmError) as e:
+        nm.prune_compress(dev(x), 8, 16, out=comp)
+    assert e.value.status == nm.NM_ERR_CUDA and nm.last_cuda_error() == 701
+    torch.cuda.synchronize()
+    assert torch.equal(comp.vals, before)
+    # the GEMM path (its own launcher) and a call made of several launches
+    Wl = nm.lift(dev(w), 16)
+    nm.prune_compress(dev(x), 8, 16, out=comp)
+    Y = torch.full((48, 96), 3.0, dtype=torch.float32, device="cuda")
+    nm.debug_fail_next_launch(719)
+    with pytest.raises(nm.NmError) as e:
+        nm.sparse_gemm(comp, Wl, nm.NM_ACT, torch.float32, out=Y)
+    assert e.value.status == nm.NM_ERR_CUDA and nm.last_cuda_error() == 719
+    torch.cuda.synchronize()
+    assert bool((Y == 3.0).all())
+    nm.sparse_gemm(comp, Wl, nm.NM_ACT, torch.float32, out=Y)
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    check_close(host_f64(Y), oracle.act_sparse_linear(x, w, 8, 16))
