@@ -180,6 +180,30 @@ size_t nm_sparse_gemm_workspace_size(const nm_sparse_operand *S, int64_t rows_d,
 int nm_sparse_gemm(const nm_sparse_operand *S, const void *D, int64_t rows_d, nm_side side,
                    void *Y, nm_dtype out_dt, void *ws, size_t ws_bytes, void *stream);
 
+/* The online half of the sliding-window method in one call: the activation
+ * lift and the weight-sparse product, Y[rows_x][W->rows] = lift(X) . W_c^T
+ * with lift() as in nm_lift().
+ * [SlideSparse, technical summary §2.B (activation lifting: X is expanded
+ *  to K' so that the windowed weight runs on 2:4 hardware) and §2.C (the
+ *  online lift followed by the 2:4 GEMM).]
+ *   W     : the packed weight (slide_decompose() or nm_prune_compress() of W).
+ *   X     : raw bf16 activations [rows_x][W->K], row stride ldx elements
+ *           (a multiple of 8), 16-byte aligned; NOT lifted.
+ *   Y     : [rows_x][W->rows] row-major, dtype out_dt.
+ *   ws    : slide_gemm_workspace_size() bytes, 16-byte aligned, or NULL when
+ *           that size is 0.
+ * Decode shapes (rows_x <= 32, when the CTA's lifted panel fits its shared
+ * memory -- every K up to several thousand) run as ONE kernel: each CTA
+ * loads the raw columns of X its k-range needs and writes their lift into
+ * shared memory itself, so the lifted X never goes through global memory and
+ * no workspace is used (size 0).  Other shapes lift into ws first and run
+ * nm_sparse_gemm().  Results equal nm_lift() followed by nm_sparse_gemm()
+ * bit for bit.  X may be written by the preceding kernel in the stream; W
+ * follows the weight rule of nm_sparse_gemm(). */
+size_t slide_gemm_workspace_size(const nm_sparse_operand *W, int64_t rows_x);
+int slide_gemm(const nm_sparse_operand *W, const void *X, int64_t rows_x, int64_t ldx, void *Y,
+               nm_dtype out_dt, void *ws, size_t ws_bytes, void *stream);
+
 /* Dense comparator on the same tensor-core pipeline: Y[rows_a][rows_b] =
  * A . B^T with A [rows_a x K], B [rows_b x K] bf16, K % 16 == 0. */
 int nm_dense_gemm(const void *A, int64_t rows_a, const void *B, int64_t rows_b, int64_t K,
@@ -403,7 +427,9 @@ const char *nm_status_string(int status);
 int nm_last_cuda_error(void);
 /* Synchronises `stream`, then reads and clears the device status word that
  * kernels set when a bounded wait expires: NM_OK or NM_ERR_DEVICE_TIMEOUT
- * (or NM_ERR_CUDA if the synchronisation itself failed). */
+ * (or NM_ERR_CUDA if the synchronisation itself failed; NM_ERR_UNSUPPORTED
+ * if a kernel found its launch shape beyond its shared-memory plan, which
+ * the host-side checks rule out). */
 int nm_get_device_error(void *stream);
 /* Test hook for the launch-error path: the next kernel launch made by a call
  * of this library on the calling thread fails with cudaError_t `cuda_error`

@@ -64,6 +64,8 @@ def lib():
             "nm_lift": (I, [P, I, I64, I64, I64, I, P, P]),
             "nm_sparse_gemm_workspace_size": (SZ, [ctypes.POINTER(SparseOperand), I64, I]),
             "nm_sparse_gemm": (I, [ctypes.POINTER(SparseOperand), P, I64, I, P, I, P, SZ, P]),
+            "slide_gemm_workspace_size": (SZ, [ctypes.POINTER(SparseOperand), I64]),
+            "slide_gemm": (I, [ctypes.POINTER(SparseOperand), P, I64, I64, P, I, P, SZ, P]),
             "nm_dense_gemm": (I, [P, I64, P, I64, I64, P, I, P]),
             "nm_quant_lift_fp8": (I, [P, I, I64, I64, I64, I, P, P, P]),
             "nm_prune_compress_fp8": (I, [P, I64, I64, I64, I, I, P, P, P, P, P]),
@@ -221,6 +223,29 @@ def sparse_gemm(S: Compressed, D: torch.Tensor, side: int, out_dtype=torch.bfloa
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=D.device) if ws_bytes else None
     _check("nm_sparse_gemm", lib().nm_sparse_gemm(
         ctypes.byref(st), _p(D), rows_d, side, _p(out), _dt(out), _p(ws), ws_bytes, _stream(D)))
+    return out
+
+
+def slide_gemm_workspace_size(W: Compressed, rows_x: int) -> int:
+    st = W.struct()
+    return int(lib().slide_gemm_workspace_size(ctypes.byref(st), rows_x))
+
+
+def slide_gemm(W: Compressed, X: torch.Tensor, out_dtype=torch.bfloat16, out: torch.Tensor | None = None,
+               ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Y [X.rows, W.rows] = lift(X) . W_c^T from the raw (unlifted) bf16 X."""
+    _need_cuda(X)
+    rows_x = X.shape[0]
+    if X.dtype != torch.bfloat16 or X.shape[1] != W.K or X.stride(1) != 1:
+        raise ValueError("X must be bf16 [rows, K] with unit column stride")
+    if out is None:
+        out = torch.empty((rows_x, W.rows), dtype=out_dtype, device=X.device)
+    st = W.struct()
+    ws_bytes = int(lib().slide_gemm_workspace_size(ctypes.byref(st), rows_x))
+    if ws_bytes and (ws is None or ws.numel() < ws_bytes):
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=X.device)
+    _check("slide_gemm", lib().slide_gemm(ctypes.byref(st), _p(X), rows_x, X.stride(0), _p(out), _dt(out),
+                                          _p(ws if ws_bytes else None), ws_bytes, _stream(X)))
     return out
 
 

@@ -122,7 +122,49 @@ struct GemmPlan {
   int fp8 = 0;                // 8-bit (E4M3) operands, rescaled by scale_a[row] * scale_b[column]
   const float* scale_a = nullptr;
   const float* scale_b = nullptr;
+  const void* lift_x = nullptr;  // in-GEMM lift: B = lift(lift_x), raw bf16 [rows_b][lift_k], row stride lift_ldx
+  int64_t lift_ldx = 0, lift_k = 0;
+  int lift_m = 0;
 };
+
+// Ring depths of the in-GEMM lift kernel (compile-time instantiations), in
+// order of preference: 6 stages of A (about half the k-range of the 6:8
+// decode product, whose ring no longer has to hold B), else 4.
+constexpr int kLiftRings[2] = {6, 4};
+
+// Shared-memory plan of the in-GEMM lift for one launch shape: the largest
+// raw-X box count and k-block count over the splits, and the layout
+// [ring of A + metadata | receive buffer | barriers | raw X boxes | panel].
+struct LiftSmem {
+  int boxes = 0, kb = 0, ring = 0, raw_off = 0, panel_off = 0, bytes = 0;
+};
+constexpr int kMaxDynSmem = 232448;   // 227 KB per CTA on sm_100
+
+template <int BN>
+bool plan_lift_smem(int64_t kb_total, int splits, int64_t K, int M, LiftSmem* out) {
+  using Cfg = nm::GemmCfg<BN, false>;
+  const int L = 2 * (M - 2);                        // lifted columns per group: 4 (M/2 - 1)
+  const int64_t k_lift = (K / M) * L;
+  LiftSmem ls;
+  for (int sp = 0; sp < splits; ++sp) {
+    const int64_t b0 = kb_total * sp / splits, b1 = kb_total * (sp + 1) / splits;
+    ls.kb = std::max<int>(ls.kb, static_cast<int>(b1 - b0));
+    const int64_t j_lo = b0 * 128, j_hi = std::min<int64_t>(b1 * 128, k_lift);
+    const int64_t c_base = ((j_lo / L) * M) & ~int64_t(7);
+    const int64_t c_end = j_hi > j_lo ? ((j_hi - 1) / L + 1) * M : c_base;
+    ls.boxes = std::max<int>(ls.boxes, static_cast<int>(ceil_div(c_end - c_base, int64_t(256))));
+  }
+  const int raw_bytes = ls.boxes * BN * 512, panel_bytes = ls.kb * Cfg::kBBytes;
+  for (int r : kLiftRings) {
+    const int fixed = r * (nm::kABytes + Cfg::kEStage) + Cfg::kRecvBytes + 256;
+    ls.raw_off = static_cast<int>(ceil_div(int64_t(fixed), int64_t(1024)) * 1024);
+    ls.panel_off = static_cast<int>(ceil_div(int64_t(ls.raw_off + raw_bytes), int64_t(1024)) * 1024);
+    ls.bytes = 1024 + ls.panel_off + panel_bytes;
+    ls.ring = r;
+    if (ls.bytes <= kMaxDynSmem) { *out = ls; return true; }
+  }
+  return false;
+}
 
 template <int BN, bool FP8 = false>
 int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
@@ -154,7 +196,13 @@ int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
   }
   if (kb_sparse == 0 || rows_s == 0) ta_s = ta_d;
   if (kb_dense == 0 || rows_d == 0) ta_d = ta_s;
-  if ((rc = make_tmap(&tb, p.b, b_cols, p.rows_b, b_cols * 2, 64, BN)) != NM_OK) return rc;
+  if (p.lift_x != nullptr) {
+    // in-GEMM lift: tmB maps the raw activation, boxes of 256 columns x BN rows
+    if ((rc = make_tmap(&tb, p.lift_x, p.lift_k, p.rows_b, p.lift_ldx * 2, 256, BN,
+                        CU_TENSOR_MAP_SWIZZLE_NONE)) != NM_OK) return rc;
+  } else if ((rc = make_tmap(&tb, p.b, b_cols, p.rows_b, b_cols * 2, 64, BN)) != NM_OK) {
+    return rc;
+  }
   }
 
   nm::GemmArgs args{};
@@ -177,16 +225,35 @@ int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
   args.row_shift = p.row_shift;
   args.col_sum = p.col_sum;
   args.fp8_last_half = (FP8 && p.ks_lift % 256 != 0) ? 1 : 0;
+  int smem = Cfg::kSmemBytes;
   if (p.out_split_rows >= 0) args.k_dense_x0 = 0;
-
-  auto kern = nm::k_nm_gemm<BN, FP8>;
-  NM_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes));
+  // in-GEMM lift: its own instantiation (ring of 6 or 4 stages of A) and
+  // parameter type
+  nm::LiftArgs largs{};
+  int lift_ring = 0;
+  if (p.lift_x != nullptr) {
+    if constexpr (FP8 || BN > 32) {
+      return NM_ERR_UNSUPPORTED;
+    } else {
+      LiftSmem ls;
+      if (!plan_lift_smem<BN>(kb_sparse, splits, p.lift_k, p.lift_m, &ls)) return NM_ERR_UNSUPPORTED;
+      static_cast<nm::GemmArgs&>(largs) = args;
+      largs.lift_m = p.lift_m;
+      largs.lift_k = p.lift_k;
+      largs.lift_boxes = ls.boxes;
+      largs.lift_kb = ls.kb;
+      largs.lift_raw_off = ls.raw_off;
+      largs.lift_panel_off = ls.panel_off;
+      lift_ring = ls.ring;
+      smem = ls.bytes;
+    }
+  }
 
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(ceil_div(p.rows_a, nm::kBM)),
                      static_cast<unsigned>(ceil_div(p.rows_b, BN)), static_cast<unsigned>(splits));
   cfg.blockDim = dim3(192, 1, 1);
-  cfg.dynamicSmemBytes = Cfg::kSmemBytes;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   // Programmatic dependent launch: the kernel may start while the preceding
   // kernel in the stream finishes; it waits for it (griddepcontrol.wait)
@@ -205,10 +272,18 @@ int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  if (g_fail_next_launch != 0) NM_CUDA_TRY(injected_launch_error());
-  NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta_s, ta_d, tb, args));
-  NM_CUDA_TRY(cudaGetLastError());
-  return NM_OK;
+  auto launch = [&](auto kern, const auto& a) -> int {
+    NM_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    if (g_fail_next_launch != 0) NM_CUDA_TRY(injected_launch_error());
+    NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta_s, ta_d, tb, a));
+    NM_CUDA_TRY(cudaGetLastError());
+    return NM_OK;
+  };
+  if constexpr (!FP8 && BN <= 32) {
+    if (lift_ring == 6) return launch(nm::k_nm_gemm<BN, false, 6>, largs);
+    if (lift_ring == 4) return launch(nm::k_nm_gemm<BN, false, 4>, largs);
+  }
+  return launch(nm::k_nm_gemm<BN, FP8>, args);
 }
 
 // uint8 [rows][16] view of a metadata image, box of one 128-row block.
@@ -585,6 +660,24 @@ int64_t prune_chunks(int64_t K, int M) { return ceil_div(K / M, 32 * nm::prune_g
 
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
+// In-GEMM lift (slide_gemm): the single-CTA kernel's tile width and split
+// for rows_x activation rows, and whether the lifted panel fits its shared
+// memory.
+template <int BN>
+bool slide_fused_fits(const nm_sparse_operand* W, int splits) {
+  const int64_t kb_total = ceil_div(W->K_lift, int64_t(128));
+  LiftSmem ls;
+  return plan_lift_smem<BN>(kb_total, splits, W->K, W->M, &ls);
+}
+
+bool slide_fused_plan(const nm_sparse_operand* W, int64_t rows_x, int* bn, int* splits) {
+  if (rows_x > 32 || W->K_lift >= (int64_t(1) << 24)) return false;   // the kernel's 32-bit window math
+  *bn = pick_bn(rows_x);
+  *splits = pick_splits(ceil_div(W->rows, int64_t(nm::kBM)), ceil_div(W->K_lift, int64_t(128)));
+  return *bn == 16 ? slide_fused_fits<16>(W, *splits) : slide_fused_fits<32>(W, *splits);
+}
+
+
 }  // namespace
 
 extern "C" {
@@ -597,6 +690,41 @@ int nm_sparse_gemm(const nm_sparse_operand* S, const void* D, int64_t rows_d, nm
   const int rc = sparse_plan(S, D, rows_d, side, Y, out_dt, &p, &empty);
   if (rc != NM_OK || empty) return rc;
   return run_gemm(p, static_cast<cudaStream_t>(stream));
+}
+
+size_t slide_gemm_workspace_size(const nm_sparse_operand* W, int64_t rows_x) {
+  if (W == nullptr || rows_x <= 0 || W->rows <= 0 || W->K <= 0 || W->M <= 0 || !m_supported(W->M) ||
+      W->K % W->M != 0 || W->K_lift != nm_lifted_k(W->K, W->M))
+    return 0;
+  int bn = 0, splits = 0;
+  if (slide_fused_plan(W, rows_x, &bn, &splits)) return 0;
+  return static_cast<size_t>(ceil_div(rows_x * W->K_lift * 2, int64_t(16)) * 16);
+}
+
+int slide_gemm(const nm_sparse_operand* W, const void* X, int64_t rows_x, int64_t ldx, void* Y, nm_dtype out_dt,
+               void* ws, size_t ws_bytes, void* stream) {
+  if (W == nullptr || rows_x < 0 || ldx < W->K) return NM_ERR_INVALID_ARG;
+  GemmPlan p;
+  bool empty = false;
+  int rc = sparse_plan(W, X, rows_x, NM_WEIGHT, Y, out_dt, &p, &empty);
+  if (rc != NM_OK || empty) return rc;
+  if ((ldx * 2) % 16 != 0) return NM_ERR_ALIGNMENT;
+  auto st = static_cast<cudaStream_t>(stream);
+  int bn = 0, splits = 0;
+  if (slide_fused_plan(W, rows_x, &bn, &splits)) {
+    p.b = nullptr;
+    p.lift_x = X;
+    p.lift_ldx = ldx;
+    p.lift_k = W->K;
+    p.lift_m = W->M;
+    return bn == 16 ? launch_gemm_bn<16>(p, splits, st) : launch_gemm_bn<32>(p, splits, st);
+  }
+  // lift into the workspace, then the plain product
+  if (ws == nullptr || ws_bytes < slide_gemm_workspace_size(W, rows_x)) return NM_ERR_WORKSPACE;
+  if (!aligned16(ws)) return NM_ERR_ALIGNMENT;
+  if ((rc = nm_lift(X, NM_BF16, rows_x, W->K, ldx, W->M, ws, stream)) != NM_OK) return rc;
+  p.b = ws;
+  return run_gemm(p, st);
 }
 
 // ------------------------------------------------ per-token corrections

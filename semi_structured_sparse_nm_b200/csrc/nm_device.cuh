@@ -17,6 +17,7 @@ namespace nm {
 __device__ unsigned int g_status;
 __device__ unsigned int g_status_where;
 
+constexpr unsigned kStatusUnsupported = 2u;     // == NM_ERR_UNSUPPORTED: a launch shape past the kernel's budget
 constexpr unsigned kStatusTimeout = 5u;         // == NM_ERR_DEVICE_TIMEOUT
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s per wait
 

@@ -24,6 +24,8 @@
 // as they have landed; wider tiles keep the partial in their own ring memory
 // and are summed by distributed loads between two cluster barriers.
 #pragma once
+#include <type_traits>
+
 #include "nm_device.cuh"
 
 namespace nm {
@@ -56,6 +58,19 @@ struct GemmArgs {
   const float* col_sum;
   const float* col_scale;
   int fp8_last_half;                        // 8-bit product: the last k-block holds only 128 lifted K
+};
+
+// In-GEMM lift (weight-side products, bf16, BN <= 32): B is the lift of a
+// raw activation X [rows_b][lift_k] (tensor map tmB, boxes of 256 columns x
+// BN rows, no swizzle), formed once per CTA in shared memory.  A separate
+// parameter type, so that the other instantiations keep theirs unchanged.
+struct LiftArgs : GemmArgs {
+  int lift_m;                               // group size M of the (2n-2):2n pattern
+  int64_t lift_k;                           // raw K
+  int lift_boxes;                           // raw-X boxes a CTA may load (shared-memory budget)
+  int lift_kb;                              // k-blocks a CTA may hold in its lifted panel
+  int lift_raw_off, lift_panel_off;         // byte offsets of the raw boxes and the panel from the
+                                            // (1024-aligned) shared-memory base
 };
 
 // FP8: a sparse k-block is 256 lifted K of E4M3 codes (A 128 stored bytes
@@ -191,17 +206,118 @@ __device__ __forceinline__ void store_row_chunk(const GemmArgs& a, int64_t ra, i
   for (int i = 0; i < CW; ++i) store_out_raw(a, ra, cb0 + i, __uint_as_float(v[i]));
 }
 
-template <int BN, bool FP8 = false>
+// In-GEMM lift, run by the four epilogue warps (128 threads) of one CTA
+// before its epilogue.  The CTA's k-blocks [kb_begin, kb_end) cover lifted
+// columns [128 kb_begin, 128 kb_end); lifted column j of a (2n-2):2n pattern
+// (M = 2n, n-1 windows of width 4 at stride 2 per group) is raw column
+// g M + 2w + (j % 4) with g = j / (4(n-1)), w = (j % (4(n-1))) / 4.  The raw
+// columns [c_base, (g_hi + 1) M) come in by TMA (boxes of 256 columns x BN
+// rows, zero-filled past the matrix), then every 16-byte chunk of the panel
+// -- two windows of one row -- is assembled from shared memory and stored in
+// the 128-byte-swizzled K-major image the MMA descriptors expect (k-block i,
+// half h, row r, chunk c at i*2*BN*128 + h*BN*128 + r*128 + 16*(c ^ (r % 8))).
+// Lifted columns past K' are zero, as a TMA load of the lifted matrix would
+// leave them.  The async proxy is fenced before the arrival on panel_bar.
+template <int BN>
+__device__ __forceinline__ void lift_panel(const LiftArgs& args, const CUtensorMap& tmX, int kb_begin, int kb_end,
+                                           uint8_t* sXr, uint8_t* sP, uint64_t* xraw_bar, uint64_t* panel_bar,
+                                           volatile int* abort_flag) {
+  const int t = static_cast<int>(threadIdx.x) - 64;              // 0 .. 127
+  // 32-bit index arithmetic throughout: K and K' are below 2^24 (host check)
+  const int M = args.lift_m;
+  const int nw = M / 2 - 1;                                       // windows per group
+  const uint32_t L = 4u * static_cast<uint32_t>(nw);              // lifted columns per group
+  const uint32_t k_lift = (static_cast<uint32_t>(args.lift_k) / static_cast<uint32_t>(M)) * L;
+  const uint32_t j_lo = static_cast<uint32_t>(kb_begin) * 128u;
+  const uint32_t j_hi = min(static_cast<uint32_t>(kb_end) * 128u, k_lift);
+  const uint32_t c_base = ((j_lo / L) * static_cast<uint32_t>(M)) & ~7u;   // 16-byte aligned TMA x coordinate
+  const uint32_t c_end = (j_hi > j_lo) ? ((j_hi - 1u) / L + 1u) * static_cast<uint32_t>(M) : c_base;
+  const int nbox = static_cast<int>((c_end - c_base + 255u) / 256u);
+  bool ok = nbox <= args.lift_boxes && (kb_end - kb_begin) <= args.lift_kb;
+  if (!ok) {
+    if (t == 0) record_status(kStatusUnsupported, kWhereEpilogue);
+  } else {
+    if (t == 0) {
+      griddep_wait();                                             // X may come from the preceding kernel
+      mbar_arrive_expect_tx(xraw_bar, static_cast<uint32_t>(nbox * BN * 512));
+      for (int b = 0; b < nbox; ++b)
+        tma_load_2d(&tmX, xraw_bar, sXr + b * (BN * 512), static_cast<int32_t>(c_base + 256u * b), 0);
+    }
+    ok = mbar_wait(xraw_bar, 0u, abort_flag, kWhereEpilogue);
+    // copies still in flight land before the CTA may exit
+    if (!ok && t == 0) mbar_wait(xraw_bar, 0u, nullptr, kWhereEpilogue, 100000000ull);
+  }
+  if (ok) {
+    // Window-major: a thread takes windows t, t+128, ... of the CTA's range;
+    // the index arithmetic is done once per window (g = q / nw as a
+    // multiply-high by ceil(2^32 / nw), exact for q < 2^22 and nw <= 15), then
+    // the window is copied down all BN rows: two 4-byte loads and one 8-byte
+    // store per row at compile-time row offsets, all independent.  A warp's
+    // 32 windows are one k-block: its stores fill two 128-byte panel rows.
+    const uint32_t magic = nw > 1 ? 0xFFFFFFFFu / static_cast<uint32_t>(nw) + 1u : 0u;
+    // the raw base address passes through a volatile asm placed after the
+    // wait on xraw_bar, so the (non-volatile, freely scheduled) loads below
+    // cannot be hoisted above it
+    uint32_t raw_s;
+    asm volatile("mov.b32 %0, %1;" : "=r"(raw_s) : "r"(smem_u32(sXr)) : "memory");
+    const uint32_t pan_s = smem_u32(sP);
+    const uint32_t q_lo = j_lo / 4u, nwin = (j_hi - j_lo) / 4u;
+    for (uint32_t qi = static_cast<uint32_t>(t); qi < nwin; qi += 128u) {
+      const uint32_t q = q_lo + qi;
+      const uint32_t g = nw > 1 ? __umulhi(q, magic) : q;
+      const uint32_t w = q - g * static_cast<uint32_t>(nw);
+      const uint32_t col = g * static_cast<uint32_t>(M) + 2u * w - c_base;   // 4 columns, never across a box edge
+      const uint32_t src = raw_s + (col / 256u) * (BN * 512) + (col % 256u) * 2u;
+      const uint32_t p = 4u * qi;
+      const uint32_t c = (p % 64u) / 8u;
+      const uint32_t dst = pan_s + (p / 128u) * (2 * BN * 128) + ((p % 128u) / 64u) * (BN * 128) + 8u * ((p % 8u) / 4u);
+      uint32_t a[BN], b[BN];
+#pragma unroll
+      for (int r = 0; r < BN; ++r) {
+        asm("ld.shared.b32 %0, [%1];" : "=r"(a[r]) : "r"(src + r * 512));
+        asm("ld.shared.b32 %0, [%1];" : "=r"(b[r]) : "r"(src + r * 512 + 4));
+      }
+#pragma unroll
+      for (int r = 0; r < BN; ++r)
+        asm volatile("st.shared.v2.b32 [%0], {%1, %2};"
+                     :: "r"(dst + r * 128 + 16u * (c ^ static_cast<uint32_t>(r % 8))), "r"(a[r]), "r"(b[r]) : "memory");
+    }
+    // lifted columns [j_hi, 128 kb_end) past K' are zero, as a TMA load of
+    // the lifted matrix would leave them
+    const uint32_t p_end = static_cast<uint32_t>(kb_end - kb_begin) * 128u;
+    for (uint32_t e = static_cast<uint32_t>(t); e < (p_end - (j_hi - j_lo)) / 4u * BN; e += 128u) {
+      const uint32_t r = e % BN, p = (j_hi - j_lo) + 4u * (e / BN);
+      const uint32_t c = (p % 64u) / 8u;
+      const uint32_t dst = pan_s + (p / 128u) * (2 * BN * 128) + ((p % 128u) / 64u) * (BN * 128) + r * 128 +
+                           16u * (c ^ (r % 8u)) + 8u * ((p % 8u) / 4u);
+      asm volatile("st.shared.v2.b32 [%0], {%1, %2};" :: "r"(dst), "r"(0u), "r"(0u) : "memory");
+    }
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");    // generic writes -> tensor-core reads
+  // Arrive even on failure: the MMA issuer then sees the abort flag or a
+  // zero panel, never waits forever.
+  if (!ok) *abort_flag = 1;
+  mbar_arrive(panel_bar);
+}
+
+// LIFT_RING > 0 is the in-GEMM lift instantiation (bf16, BN <= 32): B comes
+// from the lifted panel and the ring holds LIFT_RING stages of A and
+// metadata; otherwise the ring holds Cfg::kStages full stages.
+template <int BN, bool FP8 = false, int LIFT_RING = 0>
 __global__ void __launch_bounds__(192, 1)
 k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUtensorMap tmA_d,
-          const __grid_constant__ CUtensorMap tmB, const GemmArgs args) {
+          const __grid_constant__ CUtensorMap tmB,
+          const std::conditional_t<(LIFT_RING > 0), LiftArgs, GemmArgs> args) {
   using Cfg = GemmCfg<BN, FP8>;
-  constexpr int S = Cfg::kStages;
+  constexpr bool lift = LIFT_RING > 0;
+  static_assert(!lift || (!FP8 && BN <= 32), "in-GEMM lift: bf16, at most 32 activation rows");
+  constexpr int S = lift ? LIFT_RING : Cfg::kStages;
+  constexpr int b_stage = lift ? 0 : Cfg::kBBytes;   // in-GEMM lift: B lives in the panel, not the ring
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + S * kABytes;
-  uint8_t* sE = sB + S * Cfg::kBBytes;
+  uint8_t* sE = sB + S * b_stage;
   float* sRecv = reinterpret_cast<float*>(sE + S * Cfg::kEStage);
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(sE + S * Cfg::kEStage + Cfg::kRecvBytes);
   uint64_t* empty_bar = full_bar + S;
@@ -209,6 +325,10 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
   uint64_t* red_bar = accum_bar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(red_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* xraw_bar = red_bar + 2;                  // in-GEMM lift: raw X landed
+  uint64_t* panel_bar = red_bar + 3;                 // in-GEMM lift: lifted panel written
+  uint8_t* sP = nullptr;                             // in-GEMM lift: the lifted panel
+  if constexpr (lift) sP = smem + args.lift_panel_off;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t tiles_m = gridDim.x;
@@ -230,6 +350,10 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
     for (int s = 0; s < S; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
     mbar_init(accum_bar, 1);
     mbar_init(red_bar, 1);
+    if constexpr (lift) {
+      mbar_init(xraw_bar, 1);
+      mbar_init(panel_bar, 128);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     // the owner's share of every rank's partial tile: 128 rows x BN fp32 in all
@@ -267,7 +391,7 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
             bulk_load(sE + s * Cfg::kEStage + e * kEBytes, args.meta + (m_tile * args.meta_kb + 2 * kb + e) * kEBytes,
                       kEBytes, &full_bar[s]);
         } else if (kb < args.kb_sparse) {
-          mbar_arrive_expect_tx(&full_bar[s], kABytes + Cfg::kBBytes + kEBytes);
+          mbar_arrive_expect_tx(&full_bar[s], kABytes + b_stage + kEBytes);
           tma_load_2d(&tmA_s, &full_bar[s], a_dst, kb * 64, y_a);
           bulk_load(sE + s * Cfg::kEStage, args.meta + (m_tile * args.meta_kb + kb) * kEBytes, kEBytes,
                     &full_bar[s]);
@@ -277,6 +401,7 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
         }
       };
       auto load_b = [&](int kb, int s) {
+        if constexpr (lift) return;                      // B is formed in the panel
         uint8_t* b_dst = sB + s * Cfg::kBBytes;
         if constexpr (FP8) {
           tma_load_2d(&tmB, &full_bar[s], b_dst, kb * 256, y_b);
@@ -320,13 +445,15 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
       const uint32_t idesc_dn = idesc_bf16(kBM, BN, false);
       int it = 0;
       bool ok = true;
-      for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+      if constexpr (lift) ok = mbar_wait(panel_bar, 0u, abort_flag, kWhereMma);
+      const int kb_stop = ok ? kb_end : kb_begin;
+      for (int kb = kb_begin; kb < kb_stop; ++kb, ++it) {
         const int s = it % S;
         const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
         if (!mbar_wait(&full_bar[s], ph, abort_flag, kWhereMma)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a0 = smem_u32(sA + s * kABytes);
-        const uint32_t b0 = smem_u32(sB + s * Cfg::kBBytes);
+        const uint32_t b0 = lift ? smem_u32(sP + (kb - kb_begin) * Cfg::kBBytes) : smem_u32(sB + s * Cfg::kBBytes);
         if constexpr (FP8) {
           // two metadata blocks -> columns e_col, e_col + 4; MMA kk (64
           // lifted K) reads the column pair at e_col + 2 kk
@@ -371,6 +498,9 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
   } else {
     // -------------------------------------------------------- epilogue
     const int q = warp % 4;
+    if constexpr (lift) {
+      lift_panel<BN>(args, tmB, kb_begin, kb_end, smem + args.lift_raw_off, sP, xraw_bar, panel_bar, abort_flag);
+    }
     const bool ok = mbar_wait(accum_bar, 0u, abort_flag, kWhereEpilogue);
     griddep_wait();                                  // Y may still be in use upstream
     tc_fence_after();

@@ -153,3 +153,34 @@ def test_host_pipeline_validates_before_launch(L):
     assert L.nm_act_sparse_linear_host(fake, 600, 1024, 8, 16, fake, 768, fake, 0, fake, ws - 1, s) \
         == nm.NM_ERR_WORKSPACE
     assert L.nm_act_sparse_linear_host(null, 0, 1024, 8, 16, null, 768, null, 0, null, 0, s) == nm.NM_OK
+
+
+def test_slide_gemm_sizes_and_validation(L):
+    """slide_gemm runs fused (no workspace) on decode shapes whose lifted panel
+    fits a CTA's shared memory, else it needs rows x K' bf16 of workspace for
+    the separate lift; arguments are checked before any launch."""
+    from semi_structured_sparse_nm_b200 import _lib as nm
+    fake = ctypes.c_void_p(0x10000)
+    odd = ctypes.c_void_p(0x10008)
+    null = ctypes.c_void_p(0)
+    s = null
+    W68 = nm.SparseOperand(0x10000, 0x10000, 4096, 4096, 6, 8, 6144)       # the 6:8 decode weight
+    for rows_x in (1, 16):
+        assert L.slide_gemm_workspace_size(ctypes.byref(W68), rows_x) == 0
+    # 17..32 rows double the panel and the raw boxes: no room left for 4 ring stages
+    for rows_x in (17, 32, 33):
+        assert L.slide_gemm_workspace_size(ctypes.byref(W68), rows_x) == rows_x * 6144 * 2
+    W68s = nm.SparseOperand(0x10000, 0x10000, 4096, 1024, 6, 8, 1536)    # shorter K: 32 rows fit
+    assert L.slide_gemm_workspace_size(ctypes.byref(W68s), 32) == 0
+    # a long reduction on one row tile: 96 k-blocks per CTA cannot be held as a panel
+    Wlong = nm.SparseOperand(0x10000, 0x10000, 128, 65536, 6, 8, 98304)
+    assert L.slide_gemm_workspace_size(ctypes.byref(Wlong), 8) == 8 * 98304 * 2
+    W24 = nm.SparseOperand(0x10000, 0x10000, 256, 512, 2, 4, 512)
+    assert L.slide_gemm_workspace_size(ctypes.byref(W24), 16) == 0
+    assert L.slide_gemm(ctypes.byref(W68), fake, 16, 4000, fake, 0, null, 0, s) == nm.NM_ERR_INVALID_ARG
+    assert L.slide_gemm(ctypes.byref(W68), null, 16, 4096, fake, 0, null, 0, s) == nm.NM_ERR_INVALID_ARG
+    assert L.slide_gemm(ctypes.byref(W68), odd, 16, 4096, fake, 0, null, 0, s) == nm.NM_ERR_ALIGNMENT
+    assert L.slide_gemm(ctypes.byref(W68), fake, 16, 4100, fake, 0, null, 0, s) == nm.NM_ERR_ALIGNMENT
+    assert L.slide_gemm(ctypes.byref(W68), fake, 16, 4096, fake, 7, null, 0, s) == nm.NM_ERR_INVALID_ARG
+    assert L.slide_gemm(ctypes.byref(W68), fake, 40, 4096, fake, 0, null, 0, s) == nm.NM_ERR_WORKSPACE
+    assert L.slide_gemm(ctypes.byref(W68), null, 0, 4096, null, 0, null, 0, s) == nm.NM_OK
