@@ -212,12 +212,13 @@ __device__ __forceinline__ void store_row_chunk(const GemmArgs& a, int64_t ra, i
 // (M = 2n, n-1 windows of width 4 at stride 2 per group) is raw column
 // g M + 2w + (j % 4) with g = j / (4(n-1)), w = (j % (4(n-1))) / 4.  The raw
 // columns [c_base, (g_hi + 1) M) come in by TMA (boxes of 256 columns x BN
-// rows, zero-filled past the matrix), then every 16-byte chunk of the panel
-// -- two windows of one row -- is assembled from shared memory and stored in
-// the 128-byte-swizzled K-major image the MMA descriptors expect (k-block i,
-// half h, row r, chunk c at i*2*BN*128 + h*BN*128 + r*128 + 16*(c ^ (r % 8))).
-// Lifted columns past K' are zero, as a TMA load of the lifted matrix would
-// leave them.  The async proxy is fenced before the arrival on panel_bar.
+// rows, zero-filled past the matrix); then every window (4 lifted columns, 8
+// bytes per row) is copied from shared memory into the 128-byte-swizzled
+// K-major image the MMA descriptors expect (k-block i, half h, row r, 16-byte
+// chunk c at i*2*BN*128 + h*BN*128 + r*128 + 16*(c ^ (r % 8)); a window is
+// either half of a chunk).  Lifted columns past K' are zero, as a TMA load of
+// the lifted matrix would leave them.  The async proxy is fenced before the
+// arrival on panel_bar.
 template <int BN>
 __device__ __forceinline__ void lift_panel(const LiftArgs& args, const CUtensorMap& tmX, int kb_begin, int kb_end,
                                            uint8_t* sXr, uint8_t* sP, uint64_t* xraw_bar, uint64_t* panel_bar,
@@ -229,7 +230,7 @@ __device__ __forceinline__ void lift_panel(const LiftArgs& args, const CUtensorM
   const uint32_t L = 4u * static_cast<uint32_t>(nw);              // lifted columns per group
   const uint32_t k_lift = (static_cast<uint32_t>(args.lift_k) / static_cast<uint32_t>(M)) * L;
   const uint32_t j_lo = static_cast<uint32_t>(kb_begin) * 128u;
-  const uint32_t j_hi = min(static_cast<uint32_t>(kb_end) * 128u, k_lift);
+  const uint32_t j_hi = max(min(static_cast<uint32_t>(kb_end) * 128u, k_lift), j_lo);   // empty range: no windows
   const uint32_t c_base = ((j_lo / L) * static_cast<uint32_t>(M)) & ~7u;   // 16-byte aligned TMA x coordinate
   const uint32_t c_end = (j_hi > j_lo) ? ((j_hi - 1u) / L + 1u) * static_cast<uint32_t>(M) : c_base;
   const int nbox = static_cast<int>((c_end - c_base + 255u) / 256u);
