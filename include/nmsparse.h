@@ -192,12 +192,13 @@ int nm_sparse_gemm(const nm_sparse_operand *S, const void *D, int64_t rows_d, nm
  *   Y     : [rows_x][W->rows] row-major, dtype out_dt.
  *   ws    : slide_gemm_workspace_size() bytes, 16-byte aligned, or NULL when
  *           that size is 0.
- * Decode shapes (rows_x <= 32, when the CTA's lifted panel fits its shared
- * memory -- every K up to several thousand) run as ONE kernel: each CTA
- * loads the raw columns of X its k-range needs and writes their lift into
- * shared memory itself, so the lifted X never goes through global memory and
- * no workspace is used (size 0).  Other shapes lift into ws first and run
- * nm_sparse_gemm().  Results equal nm_lift() followed by nm_sparse_gemm()
+ * Decode shapes run as ONE kernel -- rows_x <= 32 and the lifted panel of a
+ * CTA's k-range fits its shared memory (16 rows at K = 4096 for 6:8 do; 32
+ * rows need K of about 2048 or less): each CTA loads the raw columns of X
+ * its k-range needs and writes their lift into shared memory itself, so the
+ * lifted X never goes through global memory and no workspace is used.
+ * slide_gemm_workspace_size() returns 0 exactly for these shapes.  Other
+ * shapes lift into ws first and run nm_sparse_gemm().  Results equal nm_lift() followed by nm_sparse_gemm()
  * bit for bit.  X may be written by the preceding kernel in the stream; W
  * follows the weight rule of nm_sparse_gemm(). */
 size_t slide_gemm_workspace_size(const nm_sparse_operand *W, int64_t rows_x);
