@@ -1182,9 +1182,18 @@ int spense_mlp(const void* X, int64_t B, const nm_spense_mlp* W, void* Y, void* 
   const int64_t d = W->d, I = W->I, D = W->D, Is = I - D;
   if (B < 0 || d <= 0 || I <= 0 || D < 0 || D > I) return NM_ERR_INVALID_ARG;
   if (d % 128 != 0 || I % 256 != 0 || D % 256 != 0) return NM_ERR_UNSUPPORTED;
+  // every packed weight the three launches read, checked before the first
+  if (Is > 0 && (W->ug_vals == nullptr || W->ug_meta == nullptr || W->down_vals == nullptr ||
+                 W->down_meta == nullptr))
+    return NM_ERR_INVALID_ARG;
+  if (D > 0 && (W->ug_dense == nullptr || W->down_dense == nullptr)) return NM_ERR_INVALID_ARG;
   if (B == 0) return NM_OK;
   if (ws == nullptr || ws_bytes < spense_mlp_workspace_size(W, B)) return NM_ERR_WORKSPACE;
-  if (!aligned16(X) || !aligned16(Y) || !aligned16(ws)) return NM_ERR_ALIGNMENT;
+  if (!aligned16(X) || !aligned16(Y) || !aligned16(ws) ||
+      (Is > 0 && (!aligned16(W->ug_vals) || !aligned16(W->ug_meta) || !aligned16(W->down_vals) ||
+                  !aligned16(W->down_meta))) ||
+      (D > 0 && (!aligned16(W->ug_dense) || !aligned16(W->down_dense))))
+    return NM_ERR_ALIGNMENT;
   auto st = static_cast<cudaStream_t>(stream);
   uint16_t* y_ug = static_cast<uint16_t*>(ws);
   uint16_t* h = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + ceil_div(B * 2 * I * 2, int64_t(256)) * 256);

@@ -184,3 +184,120 @@ def test_slide_gemm_sizes_and_validation(L):
     assert L.slide_gemm(ctypes.byref(W68), fake, 16, 4096, fake, 7, null, 0, s) == nm.NM_ERR_INVALID_ARG
     assert L.slide_gemm(ctypes.byref(W68), fake, 40, 4096, fake, 0, null, 0, s) == nm.NM_ERR_WORKSPACE
     assert L.slide_gemm(ctypes.byref(W68), null, 0, 4096, null, 0, null, 0, s) == nm.NM_OK
+
+
+def _ceil256(n):
+    return (n + 255) // 256 * 256
+
+
+def test_fp8_calls_size_and_validate_before_launch(L):
+    """The 8-bit (E4M3) entry points: documented workspace size, and every
+    bad call rejected before anything reaches the device."""
+    from semi_structured_sparse_nm_b200 import _lib as nm
+    fake = ctypes.c_void_p(0x10000)
+    odd4 = ctypes.c_void_p(0x10002)
+    null = ctypes.c_void_p(0)
+    s = null
+    # scratch of the 8-bit packer: the 16-bit windows, then the 16-bit metadata image
+    for rows, K, M in [(4096, 4096, 8), (100, 1024, 16), (256, 512, 4)]:
+        Kl = L.nm_lifted_k(K, M)
+        assert L.slide_decompose_fp8_workspace_size(rows, K, M) == \
+            _ceil256(rows * (Kl // 2) * 2) + L.nm_meta_bytes(rows, K, M)
+    assert L.slide_decompose_fp8_workspace_size(16, 100, 8) == 0
+    # quantise + lift
+    assert L.nm_quant_lift_fp8(fake, 7, 16, 4096, 4096, 8, fake, fake, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_quant_lift_fp8(fake, nm.NM_BF16, 16, 4100, 4100, 8, fake, fake, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_quant_lift_fp8(fake, nm.NM_BF16, 16, 4092, 4096, 6, fake, fake, s) == nm.NM_ERR_UNSUPPORTED
+    assert L.nm_quant_lift_fp8(fake, nm.NM_BF16, 16, 8, 8, 8, fake, fake, s) == nm.NM_ERR_UNSUPPORTED  # K' = 12
+    assert L.nm_quant_lift_fp8(null, nm.NM_BF16, 16, 4096, 4096, 8, fake, fake, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_quant_lift_fp8(fake, nm.NM_BF16, 16, 4096, 4096, 8, fake, odd4, s) == nm.NM_ERR_ALIGNMENT
+    assert L.nm_quant_lift_fp8(fake, nm.NM_BF16, 16, 4096, 4100, 8, fake, fake, s) == nm.NM_ERR_ALIGNMENT
+    assert L.nm_quant_lift_fp8(null, nm.NM_BF16, 0, 4096, 4096, 8, null, null, s) == nm.NM_OK
+    # quantise + prune (activation side)
+    assert L.nm_prune_compress_fp8(fake, 16, 4096, 4096, 3, 4, null, fake, fake, fake, s) == nm.NM_ERR_UNSUPPORTED
+    assert L.nm_prune_compress_fp8(fake, 16, 4096, 4096, 8, 16, null, fake, null, fake, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_prune_compress_fp8(fake, 16, 4096, 4096, 8, 16, null, fake, odd4, fake, s) == nm.NM_ERR_ALIGNMENT
+    assert L.nm_prune_compress_fp8(null, 0, 4096, 4096, 8, 16, null, null, null, null, s) == nm.NM_OK
+    # offline 8-bit packer
+    ws = L.slide_decompose_fp8_workspace_size(256, 4096, 8)
+    assert L.slide_decompose_fp8(fake, 256, 4096, 6, 8, fake, fake, fake, null, ws, s) == nm.NM_ERR_INVALID_ARG
+    assert L.slide_decompose_fp8(fake, 256, 4096, 6, 8, fake, fake, fake, fake, ws - 1, s) == nm.NM_ERR_WORKSPACE
+    assert L.slide_decompose_fp8(fake, 256, 4096, 6, 8, fake, odd4, fake, fake, ws, s) == nm.NM_ERR_ALIGNMENT
+    # 8-bit product
+    S = nm.SparseOperand(0x10000, 0x10000, 4096, 4096, 6, 8, 6144)
+    P = ctypes.byref(S)
+    assert L.nm_sparse_gemm_fp8(P, fake, fake, fake, 16, 5, fake, 0, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_sparse_gemm_fp8(P, fake, fake, fake, 16, 0, fake, 7, s) == nm.NM_ERR_INVALID_ARG
+    S2 = nm.SparseOperand(0x10000, 0x10000, 4096, 1040, 2, 4, 1040)       # K' % 128 != 0
+    assert L.nm_sparse_gemm_fp8(ctypes.byref(S2), fake, fake, fake, 16, 0, fake, 0, s) == nm.NM_ERR_UNSUPPORTED
+    S3 = nm.SparseOperand(0x10000, 0x10000, 300, 4096, 6, 8, 6144)        # SM pairs need 256-row blocks
+    assert L.nm_sparse_gemm_fp8(ctypes.byref(S3), fake, fake, fake, 512, 0, fake, 0, s) == nm.NM_ERR_UNSUPPORTED
+    assert L.nm_sparse_gemm_fp8(P, null, fake, fake, 16, 1, fake, 0, s) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_sparse_gemm_fp8(P, odd4, fake, fake, 16, 1, fake, 0, s) == nm.NM_ERR_ALIGNMENT
+    assert L.nm_sparse_gemm_fp8(P, null, null, null, 0, 1, null, 0, s) == nm.NM_OK
+
+
+def test_hybrid_and_mlp_sizes_and_validation(L):
+    """Workspace sizes of the hybrid and GLU-MLP calls match their documented
+    layouts, the MLP's dense count matches the oracle's, and incomplete or
+    misaligned weights are rejected before the first launch."""
+    from semi_structured_sparse_nm_b200 import _lib as nm
+    fake = ctypes.c_void_p(0x10000)
+    null = ctypes.c_void_p(0)
+    s = null
+    for O, K in [(14336, 4096), (640, 4096), (128, 512)]:
+        assert L.hybrid_prepare_workspace_size(O, K) == _ceil256(K * 8) + _ceil256(K) + O * K * 2
+        H = nm.HybridWeight(0x10000, 0x10000, 0x10000, 0x10000, O, K, L.hybrid_dense_count(K, 0.25))
+        for B in (1, 8, 128):
+            assert L.hybrid_gemm_workspace_size(ctypes.byref(H), B) == _ceil256(B * K * 2)
+    assert L.hybrid_prepare_workspace_size(0, 4096) == 0
+    for I, f in [(14336, 0.25), (14336, 0.0), (14336, 1.0), (1024, 0.3), (512, 0.2)]:
+        assert L.spense_dense_count(I, f) == oracle.spense_dense_count(I, f)
+    for d, I in [(4096, 14336), (256, 512)]:
+        assert L.spense_mlp_prepare_workspace_size(d, I) == \
+            4 * _ceil256(I * 8) + _ceil256(I) + _ceil256(2 * I * d * 2) + _ceil256(d * I * 2)
+    # a complete weight: the Llama-8B shape with a quarter of the intermediate indices dense
+    d, I = 4096, 14336
+    D = L.spense_dense_count(I, 0.25)
+    full = [0x10000] * 7
+    Wm = nm.SpenseMlpStruct(*full, d, I, D)
+    for B in (1, 32):
+        assert L.spense_mlp_workspace_size(ctypes.byref(Wm), B) == _ceil256(B * 2 * I * 2) + _ceil256(B * I * 2)
+    ws = L.spense_mlp_workspace_size(ctypes.byref(Wm), 8)
+    assert L.spense_mlp(fake, 8, ctypes.byref(Wm), fake, null, 0, s) == nm.NM_ERR_WORKSPACE
+    assert L.spense_mlp(fake, 0, ctypes.byref(Wm), fake, null, 0, s) == nm.NM_OK
+    bad_d = nm.SpenseMlpStruct(*full, d, I, 1000)                            # D not whole 256-blocks
+    assert L.spense_mlp(fake, 8, ctypes.byref(bad_d), fake, fake, ws, s) == nm.NM_ERR_UNSUPPORTED
+    # missing or misaligned packed weights: perm, ug_vals, ug_meta, ug_dense, down_vals, down_meta, down_dense
+    for i in range(1, 7):
+        parts = list(full)
+        parts[i] = 0
+        assert L.spense_mlp(fake, 8, ctypes.byref(nm.SpenseMlpStruct(*parts, d, I, D)), fake, fake, ws, s) \
+            == nm.NM_ERR_INVALID_ARG, i
+        parts[i] = 0x10008
+        assert L.spense_mlp(fake, 8, ctypes.byref(nm.SpenseMlpStruct(*parts, d, I, D)), fake, fake, ws, s) \
+            == nm.NM_ERR_ALIGNMENT, i
+    # all-sparse and all-dense weights need only their own parts
+    sparse_only = nm.SpenseMlpStruct(0x10000, 0x10000, 0x10000, 0, 0x10000, 0x10000, 0, d, I, 0)
+    assert L.spense_mlp(fake, 0, ctypes.byref(sparse_only), fake, null, 0, s) == nm.NM_OK
+    dense_only = nm.SpenseMlpStruct(0x10000, 0, 0, 0x10000, 0, 0, 0x10000, d, I, I)
+    assert L.spense_mlp(fake, 0, ctypes.byref(dense_only), fake, null, 0, s) == nm.NM_OK
+    # preparation
+    pws = L.spense_mlp_prepare_workspace_size(d, I)
+    assert L.spense_mlp_prepare(fake, fake, fake, 0.25, ctypes.byref(nm.SpenseMlpStruct(*full, d, I, D + 256)),
+                                fake, pws, s) == nm.NM_ERR_INVALID_ARG             # D disagrees with the share
+    assert L.spense_mlp_prepare(fake, fake, fake, 0.25, ctypes.byref(Wm), fake, pws - 1, s) == nm.NM_ERR_WORKSPACE
+    odd_d = nm.SpenseMlpStruct(*full, 4000, I, D)
+    assert L.spense_mlp_prepare(fake, fake, fake, 0.25, ctypes.byref(odd_d), fake, pws, s) == nm.NM_ERR_UNSUPPORTED
+
+
+def test_misc_entry_points(L):
+    from semi_structured_sparse_nm_b200 import _lib as nm
+    assert b"sm_100a" in L.nm_version()
+    S = nm.SparseOperand(0x10000, 0x10000, 4096, 4096, 8, 16, 7168)
+    assert L.nm_sparse_gemm_workspace_size(ctypes.byref(S), 2048, 0) == 0   # split-K stays in the cluster
+    out = ctypes.c_double(0.0)
+    null = ctypes.c_void_p(0)
+    assert L.nm_mma_rate_probe(3, 10, ctypes.byref(out), null) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_mma_rate_probe(0, 0, ctypes.byref(out), null) == nm.NM_ERR_INVALID_ARG
+    assert L.nm_mma_rate_probe(0, 10, None, null) == nm.NM_ERR_INVALID_ARG
