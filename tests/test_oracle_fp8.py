@@ -152,3 +152,31 @@ def test_fp8_act_operand_codes_are_the_kept_values():
     v = inputs.bf16_to_f64(ref16["vals"])
     d = oracle.e4m3_to_f64(ref8["vals"]) * ref8["scale"][:, None].astype(np.float64)
     assert (np.abs(d - v) <= 2.0 ** -4 * np.abs(v) + 2.0 ** -10 * ref8["scale"][:, None] * 1.000001).all()
+
+
+def test_quant_vals_are_the_row_codes_of_the_kept_entries():
+    """The 8-bit weight packing quantises the window-compressed values with
+    each row's dense-row scale: scattered back to their positions, those codes
+    must be the per-row codes of quant_rows at every kept entry (a wrong row's
+    scale or a misplaced window fails)."""
+    w = inputs.normal_bf16((40, 256), 0.02, seed=12)
+    for N, M in [(6, 8), (2, 4), (14, 16)]:
+        keep = oracle.prune(w, N, M)
+        vals, nib = oracle.compress(w, keep, M)
+        row_codes, scale = oracle.quant_rows(w)
+        qv = oracle.quant_vals(vals, scale)
+        placed = oracle.decompress(qv.astype(np.uint16), nib, w.shape[1], M)
+        assert np.array_equal(placed, np.where(keep, row_codes, 0).astype(np.uint16)), (N, M)
+        packed = oracle.fp8_weight(w, N, M)
+        assert np.array_equal(packed["vals"], qv) and np.array_equal(packed["scale"], scale)
+
+
+def test_fp8_activation_lift_is_the_lift_map():
+    """The quantise + lift step's byte lift equals the bf16 lift applied to the
+    same codes (two independent implementations of the lift map)."""
+    x = inputs.student_t_bf16((24, 512), 4.0, seed=13)
+    for M in (4, 8, 16, 32):
+        a = oracle.fp8_activation(x, M)
+        assert np.array_equal(a["lifted"], oracle.lift(a["codes"].astype(np.uint16), M).astype(np.uint8)), M
+        codes, scale = oracle.quant_rows(x)
+        assert np.array_equal(a["codes"], codes) and np.array_equal(a["scale"], scale)

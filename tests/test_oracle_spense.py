@@ -86,3 +86,26 @@ def test_permuted_packing_reproduces_the_original_order(frac):
     down = np.concatenate([f(oracle.decompress(p["down_vals"], kd_s, Is, 4)), f(p["down_dense"])], axis=1)
     y_perm = h @ down.T
     assert np.allclose(y_perm, oracle.spense_mlp(x, wu, wg, wd, frac), rtol=1e-10, atol=1e-14)
+
+
+def test_rownorm_exact_on_integers_and_the_transpose_of_colnorm():
+    rng = np.random.default_rng(21)
+    wi = rng.integers(-9, 10, size=(48, 200))
+    w = inputs.bf16_from_f64(wi.astype(np.float64))
+    exact = np.array([sum(int(v) * int(v) for v in row) for row in wi], dtype=np.float64)
+    assert np.array_equal(oracle.rownorm_f64(w), exact)
+    g = inputs.normal_bf16((64, 96), 0.02, seed=22)
+    assert np.array_equal(oracle.rownorm_f64(g), oracle.colnorm_f64(np.ascontiguousarray(g.T)))
+
+
+@pytest.mark.parametrize("I", [256, 1024, 14336])
+def test_dense_count_invariants(I):
+    """Whole blocks of 256 intermediate indices, never above the share f * I
+    and within one block of it; nothing at f <= 0, everything at f >= 1."""
+    for f in (0.05, 0.25, 0.3, 0.5, 0.99):
+        D = oracle.spense_dense_count(I, f)
+        assert D % 256 == 0 and D <= f * I < D + 256, (I, f, D)
+    assert oracle.spense_dense_count(I, 0.0) == 0 and oracle.spense_dense_count(I, -1.0) == 0
+    assert oracle.spense_dense_count(I, 1.0) == I and oracle.spense_dense_count(I, 2.0) == I
+    if I == 14336:
+        assert oracle.spense_dense_count(I, 0.25) == 3584          # the Llama-8B MLP workload
