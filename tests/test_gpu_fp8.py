@@ -85,16 +85,27 @@ def test_fp8_product_exact_on_integer_grid():
     np.testing.assert_array_equal(host_f64(y), oracle.fp8_weight_sparse_linear(x, w, 6, 8))
 
 
-def test_fp8_full_size_sampled_rows():
+def test_fp8_full_size():
+    """The 6:8 weight-sparse prefill workload in 8 bits: the packed weight and
+    the quantised, lifted activations bit-exact, every output row within
+    tolerance."""
     wl, x, w = inputs.make_workload("slide_6of8_wt_prefill")
     P = nm.slide_decompose_fp8(dev(w), wl.N, wl.M)
     q = nm.quant_lift_fp8(dev(x), wl.M)
     y = nm.sparse_gemm_fp8(P, q, nm.NM_WEIGHT, torch.bfloat16)
     torch.cuda.synchronize()
     assert nm.device_error() == nm.NM_OK
-    rows = np.array([0, 1, 127, 128, 1000, 2047, 4095])
-    check_close(host_f64(y[torch.from_numpy(rows).cuda()]),
-                oracle.fp8_weight_sparse_linear(x, w, wl.N, wl.M, rows=rows), "fp8 full size")
+    wref = oracle.fp8_weight(w, wl.N, wl.M)
+    np.testing.assert_array_equal(P.codes.cpu().numpy(), wref["vals"], err_msg="weight codes")
+    np.testing.assert_array_equal(host_bits(P.scale), oracle._as_bits(wref["scale"]), err_msg="weight scales")
+    np.testing.assert_array_equal(P.meta.cpu().numpy()[:wref["meta"].size], wref["meta"], err_msg="8-bit metadata")
+    xref = oracle.fp8_activation(x, wl.M)
+    np.testing.assert_array_equal(q.codes.cpu().numpy(), xref["lifted"], err_msg="lifted activation codes")
+    np.testing.assert_array_equal(host_bits(q.scale), oracle._as_bits(xref["scale"]), err_msg="activation scales")
+    y = host_f64(y)
+    y_ref = oracle.fp8_weight_sparse_linear(x, w, wl.N, wl.M)
+    for r0 in range(0, wl.T, 512):
+        check_close(y[r0:r0 + 512], y_ref[r0:r0 + 512], f"fp8 full size, rows {r0}..")
 
 
 def test_fp8_unsupported_shapes_launch_nothing():
@@ -144,16 +155,23 @@ def test_fp8_act_sparse_product(T, O, K, N, M):
     check_close(host_f64(y), oracle.fp8_act_sparse_linear(x, w, N, M), f"fp8 act {T}x{O}x{K} {N}:{M}")
 
 
-def test_fp8_act_full_size_sampled_rows():
+def test_fp8_act_full_size():
+    """The 8:16 up_proj workload in 8 bits: the quantised, pruned activation
+    operand bit-exact, every output row within tolerance."""
     wl, x, w = inputs.make_workload("up_proj_8of16_act")
     P = nm.prune_compress_fp8(dev(x), wl.N, wl.M)
     Wq = nm.quant_lift_fp8(dev(w), wl.M)
     y = nm.sparse_gemm_fp8(P, Wq, nm.NM_ACT, torch.bfloat16)
     torch.cuda.synchronize()
     assert nm.device_error() == nm.NM_OK
-    rows = np.array([0, 1, 127, 128, 1000, 2047])
-    check_close(host_f64(y[torch.from_numpy(rows).cuda()]),
-                oracle.fp8_act_sparse_linear(x, w, wl.N, wl.M, rows=rows), "fp8 act full size")
+    ref = oracle.fp8_act_operand(x, wl.N, wl.M)
+    np.testing.assert_array_equal(host_bits(P.scale), oracle._as_bits(ref["scale"]), err_msg="scales")
+    np.testing.assert_array_equal(P.codes.cpu().numpy(), ref["vals"], err_msg="codes")
+    np.testing.assert_array_equal(P.meta.cpu().numpy()[:ref["meta"].size], ref["meta"], err_msg="8-bit metadata")
+    y = host_f64(y)
+    y_ref = oracle.fp8_act_sparse_linear(x, w, wl.N, wl.M)
+    for r0 in range(0, wl.T, 512):
+        check_close(y[r0:r0 + 512], y_ref[r0:r0 + 512], f"fp8 act full size, rows {r0}..")
 
 
 # ------------------------------------------------ decode shapes (single-CTA kernel)

@@ -52,15 +52,14 @@ def test_one_hot(variant, monkeypatch):
 
 @pytest.mark.parametrize("variant", VARIANTS + ["auto"])
 def test_many_tiles_per_cluster(variant, monkeypatch):
-    """2048 x 4096 output: more tiles than SM pairs, sampled rows checked."""
+    """2048 x 4096 output: more tiles than SM pairs, every row checked."""
     monkeypatch.setenv("NMSPARSE_GEMM", variant)
     T, O, K = 2048, 4096, 512
     x = inputs.student_t_bf16((T, K), 4.0, seed=5)
     w = inputs.normal_bf16((O, K), 0.02, seed=6)
     y = _act(x, w, 2, 4, torch.bfloat16)
     torch.cuda.synchronize()
-    rows = np.r_[0:3, 255:258, 1000:1003, T - 3:T]
-    check_close(host_f64(y)[rows], oracle.act_sparse_linear(x, w, 2, 4, rows=rows), variant)
+    check_close(host_f64(y), oracle.act_sparse_linear(x, w, 2, 4), variant)
 
 
 @pytest.mark.parametrize("variant", VARIANTS)

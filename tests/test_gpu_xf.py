@@ -110,8 +110,8 @@ def test_empty_and_unshifted_calls():
 def test_full_size_up_proj():
     """The 8:16 up_proj workload (T = 2048, K = 4096, O = 14336) with both
     corrections, in the launch configuration bench.py times: first and last
-    128-row blocks of the operand bit-exact, every shift and VAR factor,
-    sampled output rows within tolerance."""
+    the whole operand bit-exact, every shift and VAR factor, every output
+    row within tolerance."""
     wl, x, w = inputs.make_workload("up_proj_8of16_act")
     flags = SHIFT | VAR
     W = dev(w)
@@ -126,10 +126,13 @@ def test_full_size_up_proj():
     vals = host_bits(X.comp.vals)
     meta = host_bits(X.comp.meta)
     KB = -(-Kl // 128)
-    for rb in (0, wl.T // 128 - 1):
-        np.testing.assert_array_equal(vals[128 * rb:128 * rb + 128], ref["vals"][128 * rb:128 * rb + 128])
+    for rb in range(wl.T // 128):
+        np.testing.assert_array_equal(vals[128 * rb:128 * rb + 128], ref["vals"][128 * rb:128 * rb + 128],
+                                      err_msg=f"values, row block {rb}")
         np.testing.assert_array_equal(meta[rb * KB * 2048:(rb + 1) * KB * 2048],
-                                      ref["meta"][rb * KB * 2048:(rb + 1) * KB * 2048])
-    rows = np.array([0, 1, 127, 128, 1000, 2047])
-    check_close(host_f64(y[torch.from_numpy(rows).cuda()]),
-                oracle.act_sparse_linear_xf(x, w, wl.N, wl.M, True, True, rows=rows), "up_proj xf")
+                                      ref["meta"][rb * KB * 2048:(rb + 1) * KB * 2048],
+                                      err_msg=f"metadata, row block {rb}")
+    y = host_f64(y)
+    y_ref = oracle.act_sparse_linear_xf(x, w, wl.N, wl.M, True, True)
+    for r0 in range(0, wl.T, 512):
+        check_close(y[r0:r0 + 512], y_ref[r0:r0 + 512], f"up_proj xf, rows {r0}..")

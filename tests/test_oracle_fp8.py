@@ -93,17 +93,65 @@ def test_lift_u8_is_the_lift_map():
         assert np.array_equal(oracle.lift_u8(codes, M), ref)
 
 
-def test_meta8_holds_each_row_nibble_stream():
+def _decode_meta8_tensor_view(meta, rows, Kl):
+    """Independent reading of the 8-bit sparse-MMA metadata image, as the
+    tensor core sees it (PTX ISA, tcgen05.cp and the sparse metadata of
+    tcgen05.mma.sp with kind::f8f6f4).  A copy of shape 128x128b moves one
+    2048-byte block into tensor memory as 128 lanes of four 32-bit columns:
+    lane m receives the m-th 16 bytes, column c the c-th little-endian word of
+    them.  An 8-bit sparse MMA covers 64 lifted K and reads a 64-bit metadata
+    word per row from a pair of columns, the lower column holding the low 32
+    bits; the 4-bit field i of that word belongs to the i-th group of four K.
+    The two MMAs of a 128-K block use column pairs (0, 1) and (2, 3).
+    Returns the nibble of every (row, window) over the padded extent."""
+    RB, KB = -(-rows // 128), -(-Kl // 128)
+    words = np.ascontiguousarray(meta[:RB * KB * 2048]).view("<u4").reshape(RB, KB, 128, 4)
+    out = np.zeros((RB * 128, KB * 32), np.uint8)
+    for mma in range(2):
+        w64 = words[..., 2 * mma].astype(np.uint64) | (words[..., 2 * mma + 1].astype(np.uint64) << np.uint64(32))
+        for i in range(16):
+            field = ((w64 >> np.uint64(4 * i)) & np.uint64(0xF)).astype(np.uint8)      # [RB, KB, 128]
+            for kb in range(KB):
+                out[:, kb * 32 + 16 * mma + i] = field[:, kb, :].reshape(RB * 128)
+    return out
+
+
+def test_meta8_decodes_to_nibbles():
     rng = np.random.default_rng(2)
     rows, Kl = 150, 384
     nib = rng.choice(np.array([0x4, 0x8, 0xC, 0x9, 0xD, 0xE], np.uint8), size=(rows, Kl // 4))
     img = oracle.meta8(nib, Kl)
-    RB, KB = 2, 3
-    halves = np.stack([img & 0xF, img >> 4], axis=-1).reshape(RB, KB, 128, 32)
-    full = np.full((RB * 128, KB * 32), 0x4, np.uint8)
-    full[:rows, :Kl // 4] = nib
-    assert np.array_equal(halves.transpose(0, 2, 1, 3).reshape(RB * 128, KB * 32), full)
+    assert img.size == 2 * 3 * 2048
+    dec = _decode_meta8_tensor_view(img, rows, Kl)
+    np.testing.assert_array_equal(dec[:rows, :Kl // 4], nib)
+    # padding rows and windows carry the valid index pair (0, 1)
+    assert (dec[rows:, :] == 0x4).all() and (dec[:, Kl // 4:] == 0x4).all()
     assert (oracle.meta8(np.full((3, 32), 0x4, np.uint8), 128) == 0x44).all()
+
+
+@pytest.mark.parametrize("rows,K,N,M", [(130, 512, 6, 8), (64, 640, 2, 4), (40, 1024, 14, 16), (9, 2048, 30, 32)])
+def test_meta8_tensor_view_reproduces_the_pruned_product(rows, K, N, M):
+    """Emulates the 8-bit sparse MMA from the packed weight alone: each
+    window's two codes, placed at the lifted positions the tensor-view decode
+    of the metadata gives, times integer activations lifted by the lift map,
+    summed exactly; this equals the product of the pruned weight's codes with
+    the unlifted activations."""
+    w = inputs.normal_bf16((rows, K), 0.02, seed=rows + K)
+    P = oracle.fp8_weight(w, N, M)
+    Kl = P["K_lift"]
+    dec = _decode_meta8_tensor_view(P["meta"], rows, Kl)[:rows, :Kl // 4].astype(np.int64)
+    codes = oracle.e4m3_to_f64(P["vals"])                        # [rows, Kl / 2] kept values, window order
+    dense_lifted = np.zeros((rows, Kl))
+    r = np.arange(rows)[:, None]
+    j = np.arange(Kl // 4)[None, :]
+    np.add.at(dense_lifted, (r, 4 * j + (dec & 3)), codes[:, 0::2])
+    np.add.at(dense_lifted, (r, 4 * j + ((dec >> 2) & 3)), codes[:, 1::2])
+    xi = np.random.default_rng(5).integers(-3, 4, size=(7, K)).astype(np.float64)
+    xl = inputs.bf16_to_f64(oracle.lift(inputs.bf16_from_f64(xi), M))
+    got = dense_lifted @ xl.T
+    q, _ = oracle.quant_rows(w)
+    kept = oracle.e4m3_to_f64(q) * P["keep"]
+    np.testing.assert_array_equal(got, kept @ xi.T)
 
 
 @pytest.mark.parametrize("N,M", [(6, 8), (2, 4), (14, 16)])

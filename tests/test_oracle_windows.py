@@ -70,6 +70,65 @@ def test_greedy_fits_random_32():
     _check_assignment(masks, M, win, slot, st)
 
 
+def _check_assignment_fast(masks, M, win, slot, st):
+    """The invariants of _check_assignment in whole-array form, for large
+    batches of 32-position groups: every kept position is placed once, in a
+    window that covers it; along the kept positions the (window, slot) order
+    strictly increases, so no window holds more than two entries and no slot
+    is used twice; a slot 1 always follows its window's slot 0."""
+    assert M == 32
+    bits = np.unpackbits(masks.astype("<u4").view(np.uint8).reshape(-1, 4), axis=1, bitorder="little").view(bool)
+    assert (st == 0).all()
+    assert ((win >= 0) == bits).all()
+    half = (np.arange(M) // 2).astype(np.int8)[None, :]
+    d = half - win                                  # 0 or 1 for a kept position (window w covers 2w .. 2w+3)
+    assert (((d == 0) | (d == 1)) & (win <= M // 2 - 2) | ~bits).all()
+    o = np.where(bits, 2 * win + slot, np.int8(-1))
+    prev = np.empty_like(o)
+    prev[:, 0] = -1
+    np.maximum.accumulate(o[:, :-1], axis=1, out=prev[:, 1:])
+    assert ((o > prev) | ~bits).all()
+    assert ((slot == 0) | (prev == o - 1) | ~bits).all()
+
+
+def test_greedy_fits_every_pair_count_vector_32():
+    """n-1 windows suffice for every pattern of at most 2n-2 kept entries, for
+    2n = 32.  The greedy fills window w from pairs w and w+1, so whether a
+    pattern fits depends on how many entries of each pair are kept (0, 1 or
+    2); all 3^16 such pair-count vectors are enumerated, each as one mask (a
+    pair keeping one entry keeps its lower or its upper position, chosen by a
+    multiplicative hash), as every pairing of the 3^8 vectors of the lower
+    eight pairs with the 3^8 of the upper eight.  The 17 vectors with 31 or
+    32 kept entries must fail."""
+    M, H = 32, 8                                  # two halves of 8 pairs: 3^8 vectors each
+    v = np.arange(3 ** H, dtype=np.int64)
+    cnt = (v[:, None] // (3 ** np.arange(H, dtype=np.int64))[None, :]) % 3
+    h = (v.astype(np.uint64) * np.uint64(0x9E3779B1)) >> np.uint64(7)
+    upper = ((h[:, None] >> np.arange(H, dtype=np.uint64)) & np.uint64(1)).astype(bool)
+    lo = (cnt == 2) | ((cnt == 1) & ~upper)
+    hi = (cnt == 2) | ((cnt == 1) & upper)
+    sh = (2 * np.arange(H)).astype(np.uint64)
+    half = ((lo.astype(np.uint64) << sh) | (hi.astype(np.uint64) << (sh + np.uint64(1)))).sum(axis=1, dtype=np.uint64)
+    half_pop = cnt.sum(axis=1)
+    # the upper half's choice of position is decorrelated from the lower's
+    half_hi = np.roll(half, 1234)
+    pop_hi = np.roll(half_pop, 1234)
+    failing = 0
+    step = 256
+    for b0 in range(0, v.size, step):
+        masks = (half[None, :] | (half_hi[b0:b0 + step, None] << np.uint64(16))).ravel()
+        pop = (half_pop[None, :] + pop_hi[b0:b0 + step, None]).ravel()
+        win, slot, st = oracle.window_assign_batch(masks, M)
+        fits = pop <= M - 2
+        if fits.all():
+            _check_assignment_fast(masks, M, win, slot, st)
+        else:
+            _check_assignment_fast(masks[fits], M, win[fits], slot[fits], st[fits])
+            assert (st[~fits] != 0).all()
+            failing += int((~fits).sum())
+    assert failing == 17
+
+
 @pytest.mark.parametrize("n", [2, 3, 4, 8, 16])
 def test_fewer_windows_cannot_hold_the_pattern(n):
     """n-2 windows of two entries hold 2n-4 < 2n-2 entries: the page's
