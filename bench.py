@@ -10,9 +10,12 @@ One step = one pass of the hot path over one batch of synthetic input:
       one input-split GEMM;
   hybrid GLU MLP (decode): one output-split GEMM for up and gate, the SiLU
       gate, one input-split GEMM for down.
-The headline line is the Llama-8B up_proj prefill shape with 8:16 activation
-sparsity (X [2048 x 4096] Student-t, W [14336 x 4096] N(0, 0.02), bf16, fp32
-accumulation, bf16 out); the other workloads are reported under "workloads".
+The headline line is the largest single-GPU workload: the Llama-8B down_proj
+prefill shape with 16:32 activation sparsity (X [4096 x 14336] N(0, 1) with
+0.1% of the channels scaled x20, W [4096 x 14336] N(0, 0.02), bf16, fp32
+accumulation, bf16 out).  Every other workload is reported, compactly, under
+"workloads" in the same line (fields named by "workloads_fields"); --detail
+PATH also writes every workload's full record to PATH.
 
 Timing: CUDA events on the launching stream, W warm-up steps, exactly K timed
 steps between barriers + device synchronisation, max over ranks.  Every
@@ -38,14 +41,15 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-HEADLINE = "up_proj_8of16_act"
+HEADLINE = "down_proj_16of32_act"
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the
 # dominant kernel, from one ncu capture of the kernel as it stands (see
 # profiles/); drop an entry whenever that kernel changes.
 TRAFFIC = {
     ("up_proj_8of16_act", "k_nm_gemm_2cta<224,2,1>"): 233678592 + 46385664,
 }
-OTHERS = ["up_proj_2of4_act", "up_proj_8of16_act_fp8", "up_proj_8of16_act_xf", "down_proj_16of32_act", "slide_6of8_wt_prefill", "slide_6of8_wt_prefill_fp8",
+OTHERS = ["up_proj_8of16_act", "up_proj_2of4_act", "up_proj_8of16_act_fp8", "up_proj_8of16_act_xf",
+          "slide_6of8_wt_prefill", "slide_6of8_wt_prefill_fp8",
           "slide_6of8_wt_decode", "slide_6of8_wt_decode_fp8",
           "hybrid_decode_b1", "hybrid_decode_b8", "hybrid_decode_b32", "hybrid_decode_b128",
           "spense_mlp_decode_b1", "spense_mlp_decode_b8", "spense_mlp_decode_b32", "spense_mlp_decode_b128",
@@ -53,6 +57,26 @@ OTHERS = ["up_proj_2of4_act", "up_proj_8of16_act_fp8", "up_proj_8of16_act_xf", "
 L2_BYTES = 126 * 1024 * 1024
 METRIC = "N:M sparse linear TFLOP/s (dense-equiv)"
 REF_TOTAL_S = 150.0
+
+
+def workload_config(wl, ws: int = 1) -> dict:
+    """The workload's `config` dict; both arms print the same one."""
+    c = {"workload": wl.name, "T": wl.T, "K": wl.K, "O": wl.O, "N": wl.N, "M": wl.M, "side": wl.side,
+         "K_lift": wl.K_lift, "x_dist": wl.x_dist, "w_std": wl.w_std,
+         "l2": "rotated buffers, >2x L2 touched between reuses",
+         "parallelism": f"replicas x{ws} (no data-path collective)"}
+    if wl.fp8:
+        c["precision"] = "e4m3 operands"
+    if wl.xf:
+        c["corrections"] = {1: "D-PTS", 2: "VAR", 3: "D-PTS+VAR"}[wl.xf]
+    return c
+
+
+def sig(v, n: int = 4):
+    """v rounded to n significant digits (None stays None)."""
+    if v is None:
+        return None
+    return float(f"{v:.{n}g}")
 
 
 def _peaks():
@@ -199,27 +223,28 @@ def run_reference(args):
     from semi_structured_sparse_nm_b200 import inputs
     wl, x, w = inputs.make_workload(HEADLINE)
     wf = oracle.to_f64(w)
-    # each step is a bounded sample of the workload: the whole run stays
-    # within about REF_TOTAL_S seconds of oracle time
+    # each step is a bounded sample of the workload (whole token rows): the
+    # whole run stays within about REF_TOTAL_S seconds of oracle time, and a
+    # step's time is the time of the work it did
     step_s = min(args.ref_step_s, max(0.25, REF_TOTAL_S / (args.warmup + args.steps)))
-    times, rows = [], 0
+    secs, rows_list = [], []
     for i in range(args.warmup + args.steps):
         tf, r, t, thr = cpu_oracle_sample(wl, x, w, budget_s=step_s, wf=wf)
         if i >= args.warmup:
-            times.append(t / r)
-            rows = r
-    per_row = float(np.mean(times))
-    value = 2.0 * wl.O * wl.K / per_row / 1e12
-    sample = f"{rows} of {wl.T} token rows of X per step: prune+windows+metadata+fp64 GEMM against all of W"
+            secs.append(t)
+            rows_list.append(r)
+    t_step = float(np.mean(secs))
+    value = 2.0 * wl.O * wl.K * float(np.sum(rows_list)) / float(np.sum(secs)) / 1e12
+    sample = (f"{int(np.mean(rows_list))} of {wl.T} token rows per step: prune+windows+metadata+fp64 GEMM "
+              f"against all of W")
     line = {
-        "impl": "reference", "metric": METRIC, "value": value,
-        "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": per_row * wl.T * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": HEADLINE, "T": wl.T, "K": wl.K, "O": wl.O, "N": wl.N, "M": wl.M},
-        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": thr, "kind": "oracle", "sample": sample,
+        "impl": "reference", "metric": METRIC, "value": sig(value), "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sig(t_step * 1e3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(wl, ws),
+        "cpu_baseline": {"value": sig(value), "unit": "TFLOP/s", "cores": thr, "kind": "oracle", "sample": sample,
                          "cpu": cpu_model(), "nproc": os.cpu_count()},
-        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "e2e": {"value": sig(value), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -478,6 +503,7 @@ def time_workload(wk, steps, warmup, stream, clock=None):
         torch.cuda.synchronize()
         gemm_ms = e0.elapsed_time(e1) / steps
         prep_ms = max(step_ms - gemm_ms, 0.0)
+        wk.kernel_name = wk.nm.last_gemm_kernel()
         del g, gg
         return step_ms, prep_ms, gemm_ms
     # the step as a user runs it: K steps back to back, events only around them
@@ -491,6 +517,7 @@ def time_workload(wk, steps, warmup, stream, clock=None):
         t1.record(stream)
         torch.cuda.synchronize()
     step_ms = t0.elapsed_time(t1) / steps
+    wk.kernel_name = wk.nm.last_gemm_kernel()
     # the same K steps again with an event around each kernel: per-kernel times
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     torch.cuda.synchronize()
@@ -648,9 +675,11 @@ def mma_probe():
     return out
 
 
-def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None, probe=None):
+def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, probe=None):
     dense, mma, byts = wk.algorithmic()
     wl = wk.wl
+    kname = getattr(wk, "kernel_name", "") or wk.gemm_name
+    traffic = TRAFFIC.get((wl.name, kname))
     out = {
         "value": whole_job_rate(dense, ws, step_ms) / 1e12, "unit": "TFLOP/s", "ms_per_step": step_ms,
         "tokens_per_s": whole_job_rate(wl.T, ws, step_ms),
@@ -692,7 +721,7 @@ def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None, probe=None):
                                   "GEMM (slide_gemm), replayed from a CUDA graph")
     if wk.decode:
         achieved = byts / (gemm_ms * 1e-3) / 1e9
-        out["roofline"] = {"bound": "hbm", "kernel": wk.gemm_name if wl.side != "mlp" else
+        out["roofline"] = {"bound": "hbm", "kernel": kname if wl.side != "mlp" else
                            "spense_mlp (its three launches together)", "achieved": achieved, "peak": pk["hbm"],
                            "unit": "GB/s", "frac": achieved / pk["hbm"], "traffic": traffic,
                            "bytes_per_launch": byts,
@@ -700,7 +729,7 @@ def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None, probe=None):
     elif wl.fp8:
         peak = 4.0 * pk["bf16"]
         achieved = mma / (gemm_ms * 1e-3) / 1e12
-        out["roofline"] = {"bound": "tensor", "kernel": wk.gemm_name, "achieved": achieved, "peak": peak,
+        out["roofline"] = {"bound": "tensor", "kernel": kname, "achieved": achieved, "peak": peak,
                            "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                            "flops_per_launch": mma,
                            "peak_note": f"4 x {pk['source']} bf16 burst {pk['bf16']} TFLOP/s (nominal 8-bit / "
@@ -711,7 +740,7 @@ def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None, probe=None):
     else:
         peak = 2.0 * pk["bf16"]
         achieved = mma / (gemm_ms * 1e-3) / 1e12
-        out["roofline"] = {"bound": "tensor", "kernel": "k_nm_gemm_2cta<224,2,1>" if traffic else wk.gemm_name,
+        out["roofline"] = {"bound": "tensor", "kernel": kname,
                            "achieved": achieved, "peak": peak,
                            "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
                            "flops_per_launch": mma,
@@ -720,7 +749,21 @@ def summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, traffic=None, probe=None):
         if probe:
             out["roofline"]["probe_tflops"] = probe["bf16_sparse"]
             out["roofline"]["frac_of_probe"] = achieved / probe["bf16_sparse"]
+    # the compact row printed in the bench line (fields: ROW_FIELDS)
+    extra = out["kernels"].get("slide_gemm_step_us")
+    out["row"] = [sig(out["value"]), sig(step_ms * 1e3), sig(prep_ms * 1e3, 3), sig(gemm_ms * 1e3),
+                  sig(out["roofline"]["frac"], 3), out["roofline"]["bound"][0],
+                  None if traffic is None else sig(traffic / byts, 3)]
+    if extra is not None:
+        out["row"].append(sig(extra, 3))
     return out
+
+
+# TFLOP/s dense-equivalent; step, prep-kernel and GEMM microseconds; the
+# GEMM's roofline fraction and bound (t: tensor, h: HBM); its DRAM traffic
+# over its algorithmic bytes (from an ncu capture, null if none); the 6:8
+# decode step as one slide_gemm launch
+ROW_FIELDS = ["TFLOP/s", "step_us", "prep_us", "gemm_us", "frac", "bound", "traffic/alg", "slide_gemm_us"]
 
 
 def run_gpu(args):
@@ -764,8 +807,8 @@ def run_gpu(args):
         dist.barrier()
     status = nm.device_error()
     probe = mma_probe()
-    main = summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk,
-                     traffic=TRAFFIC.get((args.workload, "k_nm_gemm_2cta<224,2,1>")), probe=probe)
+    main = summarize(wk, step_ms, prep_ms, gemm_ms, ws, pk, probe=probe)
+    detail = {args.workload: {k: v for k, v in main.items() if k != "row"}}
 
     # end to end through the public calls: pinned host X in, Y out
     wl = wk.wl
@@ -799,58 +842,69 @@ def run_gpu(args):
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     dense, _, _ = wk.algorithmic()
 
+    rf = main["roofline"]
+    roofline = {"bound": rf["bound"], "kernel": rf["kernel"], "achieved": sig(rf["achieved"]), "peak": rf["peak"],
+                "unit": rf["unit"], "frac": sig(rf["frac"], 3), "traffic": rf["traffic"],
+                "peak_src": ("2x" if wl.side == "act" and not wl.fp8 else "") + f" {pk['source']} bf16 burst"}
+    if "flops_per_launch" in rf:
+        roofline["flops_per_launch"] = rf["flops_per_launch"]
+    if "bytes_per_launch" in rf:
+        roofline["bytes_per_launch"] = rf["bytes_per_launch"]
+    if "probe_tflops" in rf:
+        roofline["frac_of_probe"] = sig(rf["frac_of_probe"], 3)
+    dc = main.get("dense_comparator") or {}
     line = {
-        "metric": METRIC, "value": main["value"], "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "metric": METRIC, "value": sig(main["value"]), "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sig(step_ms), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": args.workload, **main["config"],
-                   "x_dist": wl.x_dist, "w_std": wl.w_std,
-                   "l2": f"inputs rotated over {wk.R} buffers; touched bytes between reuses > 2x L2",
-                   "parallelism": f"replicas x{ws} (no data-path collective)"},
-        "tokens_per_s": main["tokens_per_s"],
-        "kernels": main["kernels"],
-        "roofline": main["roofline"],
-        "mma_probe": {**probe, "unit": "TFLOP/s",
-                      "note": "nm_mma_rate_probe: 256 x 256 MMAs from shared memory on every SM pair, no loads; "
-                              "best of 5 launches of about 1 ms, dense-equivalent flops"},
-        "dense_comparator": main.get("dense_comparator"),
-        "e2e": {"value": ws * dense / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "config": workload_config(wl, ws),
+        "tokens_per_s": sig(main["tokens_per_s"]),
+        "kernels_us": {k[:-3]: sig(v) for k, v in main["kernels"].items() if k.endswith("_us")},
+        "roofline": roofline,
+        "e2e": {"value": sig(ws * dense / (e2e_ms * 1e-3) / 1e12), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
                 "d2h_bytes_per_step": int(yh.numel() * yh.element_size()),
-                "path": ("nm_act_sparse_linear_host (pinned host X and Y, chunked copies overlapping the math)"
-                         if pipelined else "pinned host X copied in, the step, Y copied out")},
+                "path": "nm_act_sparse_linear_host" if pipelined else "copy in, step, copy out"},
         "gpu_launches": wk.launches_per_step * args.steps,
         "clocks": clk.summary(),
         "device_status": status,
     }
+    if dc.get("ours_us") is not None:
+        line["dense_us"] = {"ours": sig(dc["ours_us"]), "cublas": sig(dc["cublas_us"])}
+    line["probe_tflops"] = {k: sig(v) for k, v in probe.items() if k != "clocks"}
     del wk
     torch.cuda.empty_cache()
 
     if not args.only_main:
-        others = {}
+        rows = {}
         for name in OTHERS:
             if name == args.workload:
                 continue
             w2 = Workload(name, dev)
-            s, p, g = time_workload(w2, args.steps, args.warmup, stream)
-            others[name] = summarize(w2, s, p, g, 1, pk, probe=probe)
+            s_, p_, g_ = time_workload(w2, args.steps, args.warmup, stream)
+            full = summarize(w2, s_, p_, g_, 1, pk, probe=probe)
+            rows[name] = full.pop("row")
+            detail[name] = full
             del w2
             torch.cuda.empty_cache()
-        line["workloads"] = others
+        line["workloads_fields"] = ROW_FIELDS
+        line["workloads"] = rows
         line["device_status"] = max(status, nm.device_error())
 
     if rank == 0 and not args.no_cpu_baseline:
         from semi_structured_sparse_nm_b200 import inputs
         wlh, xh_np, wh_np = inputs.make_workload(args.workload)
         if wlh.side == "act":
-            tf, rows, t, thr = cpu_oracle_sample(wlh, xh_np, wh_np, budget_s=args.cpu_budget_s)
-            line["cpu_baseline"] = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
-                                    "sample": f"{rows} of {wlh.T} token rows ({t:.1f} s): prune+windows+"
-                                              f"metadata+fp64 GEMM against all of W",
-                                    "split_s": getattr(cpu_oracle_sample, "last_split", None),
-                                    "cpu": cpu_model(), "nproc": os.cpu_count()}
+            tf, rows_done, t, thr = cpu_oracle_sample(wlh, xh_np, wh_np, budget_s=args.cpu_budget_s)
+            line["cpu_baseline"] = {"value": sig(tf), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+                                    "sample": f"{rows_done} of {wlh.T} token rows (prune, windows, metadata, fp64 GEMM), {t:.1f} s",
+                                    "cpu": cpu_model()}
+            detail["cpu_baseline_split_s"] = getattr(cpu_oracle_sample, "last_split", None)
     if rank == 0:
-        print(json.dumps(line), flush=True)
+        if args.detail:
+            with open(args.detail, "w") as f:
+                json.dump(detail, f, indent=1)
+        print(json.dumps(line, separators=(",", ":")), flush=True)
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
@@ -868,6 +922,7 @@ def main():
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     ap.add_argument("--ref-step-s", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--detail", default="", help="write every workload's full record (JSON) to this path")
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="run this many plain steps of --workload and exit (for ncu captures)")
     args = ap.parse_args()

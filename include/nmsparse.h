@@ -142,6 +142,10 @@ size_t nm_meta_bytes(int64_t rows, int64_t K, int M);
 
 /* Prunes `src` [rows x K] (row stride `ld` elements, dtype NM_BF16 or
  * NM_FP32) to N:M along K and writes its window-compressed form.
+ * [Flexible (N:M) Activation Sparsity, technical summary §1 (N:M blocks:
+ *  keep N of every M consecutive entries, chosen anew for every input) and
+ *  §2.A (ACT: the absolute magnitude decides); SlideSparse, §2.A (the kept
+ *  entries of a group of 2n spread over n-1 windows of width 4, stride 2).]
  *   mask_out : optional (may be NULL) uint32 [rows][ceil(K/32)]; bit k%32 of
  *              word k/32 is set iff entry k is kept.
  *   vals_out : bf16 [rows][K'/2] (fp32 inputs are rounded to nearest even).
@@ -154,11 +158,17 @@ int nm_prune_compress(const void *src, nm_dtype dt, int64_t rows, int64_t K, int
 
 /* The offline weight packer of the (2N-2):2N family: the same operation as
  * nm_prune_compress() restricted to N = M - 2 (6:8, 14:16, 30:32) or 2:4,
- * for a weight W [rows x K] with row stride K. */
+ * for a weight W [rows x K] with row stride K.
+ * [SlideSparse, technical summary §2.A (sliding-window decomposition: n-1
+ *  windows are necessary and sufficient for 2n-2 of 2n) and §2.C (the
+ *  offline packer).] */
 int slide_decompose(const void *w, nm_dtype dt, int64_t rows, int64_t K, int N, int M,
                     uint32_t *mask_out, void *vals_out, void *meta_out, void *stream);
 
-/* Lifts the dense operand: dst[r][g*4(n-1) + 4w + j] = src[r][g*2n + 2w + j]
+/* [SlideSparse, technical summary §2.B (activation lifting: the dense
+ *  operand is widened to K' = K (2n-2)/n so that every window meets its
+ *  own copy of the columns it covers).]
+ * Lifts the dense operand: dst[r][g*4(n-1) + 4w + j] = src[r][g*2n + 2w + j]
  * for M = 2n, src [rows x K] (row stride ld elements, bf16 or fp32),
  * dst bf16 [rows x K'] (row stride K').  M = 4 copies (and converts fp32).
  * K' must be a multiple of 8 (16-byte rows), else NM_ERR_ALIGNMENT. */
@@ -169,6 +179,8 @@ int nm_lift(const void *src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, i
 
 /* Y = sparse . dense^T (side NM_ACT) or its transpose (NM_WEIGHT), bf16
  * products accumulated in fp32 on the 2:4 sparse tensor cores.
+ * [SlideSparse, technical summary §2.C (the windowed operand against the
+ *  lifted one on 2:4 hardware; ideal speedup n/(n-1) over dense, §4).]
  *   S      : the compressed sparse operand (rows_s = S->rows).
  *   D      : bf16 lifted dense operand [rows_d][S->K_lift], row stride K_lift.
  *   Y      : NM_ACT -> [rows_s][rows_d]; NM_WEIGHT -> [rows_d][rows_s];
@@ -278,7 +290,11 @@ int nm_sparse_gemm_fp8(const nm_sparse_operand *S, const float *S_scale, const v
  * K for f >= 1). */
 int64_t hybrid_dense_count(int64_t K, double dense_frac);
 
-/* Offline: ranks the K columns of W [O x K] (bf16) by sum_r w[r][c]^2
+/* [SpenseGPT, technical summary §2.A (a dense region of K next to a 2:4
+ *  region) and §2.B (the dense indices permuted into one contiguous block;
+ *  the pages rank them by a calibration loss, replaced here by the weight's
+ *  column energy).]
+ * Offline: ranks the K columns of W [O x K] (bf16) by sum_r w[r][c]^2
  * (fp64, r ascending), keeps the top hybrid_dense_count(K, dense_frac)
  * columns dense (ties to the lower column), prunes the others 2:4 in
  * ascending column order, and fills `out` (buffers preallocated by the caller,
@@ -288,7 +304,9 @@ size_t hybrid_prepare_workspace_size(int64_t O, int64_t K);
 int hybrid_prepare(const void *w, int64_t O, int64_t K, double dense_frac, nm_hybrid_weight *out,
                    void *ws, size_t ws_bytes, void *stream);
 
-/* Y [B x O] = X[:, perm_s] . W_s^T + X[:, perm_d] . W_d^T (input-split, one
+/* [SpenseGPT, technical summary §2.A (input-split: the sparse and the
+ *  dense part of K accumulate into the same output).]
+ * Y [B x O] = X[:, perm_s] . W_s^T + X[:, perm_d] . W_d^T (input-split, one
  * fp32 accumulator) for X bf16 [B x K] (row stride K).  With W->perm NULL,
  * X is taken as already permuted ([sparse columns | dense columns]) and no
  * gather runs.  ws: hybrid_gemm_workspace_size(W, B) bytes. */
@@ -383,12 +401,18 @@ int nm_sparse_gemm_xf(const nm_sparse_operand *X, const void *W_lift, int64_t ro
  *
  * Scratch: a fixed array of NM_NOALLOC_SCRATCH_BYTES (2 MiB) compiled into
  * the library.  Every GPU that loads the library keeps it until the process
- * exits.  Calls with B * K * 2 > NM_NOALLOC_SCRATCH_BYTES return
- * NM_ERR_WORKSPACE and launch nothing.
+ * exits.  Only a weight with a column permutation (W->perm not NULL) uses
+ * it, for the gathered activations (B * K * 2 bytes); such calls with
+ * B * K * 2 > NM_NOALLOC_SCRATCH_BYTES return NM_ERR_WORKSPACE and launch
+ * nothing.  A malformed W (O or K not positive, K_dense outside [0, K])
+ * returns NM_ERR_INVALID_ARG first.
  *
  * The first call on each device looks up the array's device address (with
  * that device current) and caches it; make that first call before any stream
- * capture.  All calls share the one array: calls whose kernels overlap on the
+ * capture.  The cached address does not survive cudaDeviceReset() (or any
+ * other teardown of the device's primary context): after one, do not call
+ * this entry point again in the same process.  All calls share the one
+ * array: calls whose kernels overlap on the
  * GPU (different streams, no ordering between them) race on it.  Nothing in
  * the array has to start at zero -- each call writes every byte it reads.
  * Other arguments, layouts and errors are those of hybrid_gemm(). */
@@ -417,6 +441,11 @@ int hybrid_gemm_noalloc(const void *X, int64_t B, const nm_hybrid_weight *W, voi
  * nm_sparse_gemm() on each chunk. */
 size_t nm_act_sparse_linear_host_workspace_size(int64_t T, int64_t K, int N, int M, int64_t O,
                                                 int64_t chunk_rows);
+/* Error after queuing: argument errors are found before anything is queued
+ * (nothing runs, nothing is written).  A launch or copy that fails after
+ * earlier chunks were queued returns its error with those chunks still
+ * queued: their rows of y_host are written, the rest are not, and `stream`
+ * is made to wait for the copies already queued, as on success. */
 int nm_act_sparse_linear_host(const void *x_host, int64_t T, int64_t K, int N, int M, const void *w_lift,
                               int64_t O, void *y_host, int64_t chunk_rows, void *ws, size_t ws_bytes,
                               void *stream);
@@ -426,6 +455,13 @@ int nm_act_sparse_linear_host(const void *x_host, int64_t T, int64_t K, int N, i
 const char *nm_status_string(int status);
 /* The cudaError_t of the last NM_ERR_CUDA returned on this thread. */
 int nm_last_cuda_error(void);
+/* Name of the GEMM kernel instantiation that the most recent GEMM launch of
+ * this library on the calling thread used, for example
+ * "k_nm_gemm_2cta<256,1,1>" (tile width, accumulator buffers, 256-row
+ * subtiles; ",fp8" for 8-bit operands) or "k_nm_gemm<32>" (single-CTA
+ * kernel, tile width); "" before the first.  The string is owned by the
+ * library and stays valid until the next GEMM launch on this thread. */
+const char *nm_last_gemm_kernel(void);
 /* Synchronises `stream`, then reads and clears the device status word that
  * kernels set when a bounded wait expires: NM_OK or NM_ERR_DEVICE_TIMEOUT
  * (or NM_ERR_CUDA if the synchronisation itself failed; NM_ERR_UNSUPPORTED

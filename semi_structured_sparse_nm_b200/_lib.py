@@ -92,6 +92,7 @@ def lib():
             "nm_mma_rate_probe": (I, [I, I, ctypes.POINTER(ctypes.c_double), P]),
             "nm_status_string": (ctypes.c_char_p, [I]),
             "nm_last_cuda_error": (I, []),
+            "nm_last_gemm_kernel": (ctypes.c_char_p, []),
             "nm_get_device_error": (I, [P]),
             "nm_debug_expire_wait": (I, [ctypes.c_uint, P]),
             "nm_debug_fail_next_launch": (I, [I]),
@@ -539,6 +540,11 @@ def debug_fail_next_launch(cuda_error: int):
 
 def last_cuda_error() -> int:
     return int(lib().nm_last_cuda_error())
+
+
+def last_gemm_kernel() -> str:
+    """The GEMM kernel instantiation the latest GEMM call on this thread launched."""
+    return lib().nm_last_gemm_kernel().decode()
 
 
 def debug_expire_wait(timeout_us: int):

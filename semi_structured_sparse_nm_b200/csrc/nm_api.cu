@@ -28,6 +28,9 @@ thread_local int g_last_cuda_error = 0;
 // Test hook (nm_debug_fail_next_launch): the next kernel launch on this
 // thread returns this error instead of launching (0: none).
 thread_local int g_fail_next_launch = 0;
+// Name of the GEMM kernel instantiation most recently launched on this
+// thread (nm_last_gemm_kernel).
+thread_local char g_last_gemm[64] = "";
 
 cudaError_t injected_launch_error() {
   const int c = g_fail_next_launch;
@@ -272,6 +275,10 @@ int launch_gemm_bn(const GemmPlan& p, int splits, cudaStream_t st) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
+  if (lift_ring > 0)
+    std::snprintf(g_last_gemm, sizeof(g_last_gemm), "k_nm_gemm<%d,lift%d>", BN, lift_ring);
+  else
+    std::snprintf(g_last_gemm, sizeof(g_last_gemm), "k_nm_gemm<%d%s>", BN, FP8 ? ",fp8" : "");
   auto launch = [&](auto kern, const auto& a) -> int {
     NM_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     if (g_fail_next_launch != 0) NM_CUDA_TRY(injected_launch_error());
@@ -424,6 +431,7 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
+  std::snprintf(g_last_gemm, sizeof(g_last_gemm), "k_nm_gemm_2cta<%d,%d,%d%s>", BN, NACC, MSUB, FP8 ? ",fp8" : "");
   if (g_fail_next_launch != 0) NM_CUDA_TRY(injected_launch_error());
   NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta, tb, te, ty, tad, a));
   NM_CUDA_TRY(cudaGetLastError());
@@ -1261,14 +1269,17 @@ extern "C" {
 
 int hybrid_gemm_noalloc(const void* X, int64_t B, const nm_hybrid_weight* W, void* Y, nm_dtype out_dt,
                         void* stream) {
-  if (W == nullptr || B < 0) return NM_ERR_INVALID_ARG;
-  if (hybrid_gemm_workspace_size(W, B) > NM_NOALLOC_SCRATCH_BYTES) return NM_ERR_WORKSPACE;
+  if (X == nullptr || W == nullptr || Y == nullptr || B < 0) return NM_ERR_INVALID_ARG;
+  if (W->O <= 0 || W->K <= 0 || W->K_dense < 0 || W->K_dense > W->K) return NM_ERR_INVALID_ARG;
+  // Only the gather (W->perm set) uses scratch: B x K bf16 values, B * K * 2
+  // bytes, compared without forming the product (no overflow).
   void* ws = nullptr;
-  if (B > 0) {
+  if (W->perm != nullptr && B > 0) {
+    if (B > static_cast<int64_t>(NM_NOALLOC_SCRATCH_BYTES / 2) / W->K) return NM_ERR_WORKSPACE;
     const int rc = noalloc_scratch(&ws);
     if (rc != NM_OK) return rc;
   }
-  return hybrid_gemm(X, B, W, Y, out_dt, ws, NM_NOALLOC_SCRATCH_BYTES, stream);
+  return hybrid_gemm(X, B, W, Y, out_dt, ws, ws != nullptr ? NM_NOALLOC_SCRATCH_BYTES : 0, stream);
 }
 
 // ------------------------------------------------ host-buffer pipeline
@@ -1349,7 +1360,7 @@ int nm_act_sparse_linear_host(const void* x_host, int64_t T, int64_t K, int N, i
   HostPipe* p = nullptr;
   if ((rc = host_pipe(&p)) != NM_OK) return rc;
   const int64_t chunks = ceil_div(T, Tc);
-  for (int64_t c = 0; c < chunks; ++c) {
+  auto enqueue_chunk = [&](int64_t c) -> int {
     const int b = static_cast<int>(c % 2);
     const int64_t r0 = c * Tc, rows = std::min(Tc, T - r0);
     uint8_t* xd = base[b];
@@ -1363,7 +1374,8 @@ int nm_act_sparse_linear_host(const void* x_host, int64_t T, int64_t K, int N, i
     NM_CUDA_TRY(cudaStreamWaitEvent(st, p->out[b], 0));
     NM_CUDA_TRY(cudaMemcpyAsync(xd, static_cast<const uint8_t*>(x_host) + r0 * K * 2, static_cast<size_t>(rows * K * 2),
                                 cudaMemcpyHostToDevice, st));
-    if ((rc = nm_prune_compress(xd, NM_BF16, rows, K, K, N, M, nullptr, vals, meta, stream)) != NM_OK) return rc;
+    int r = nm_prune_compress(xd, NM_BF16, rows, K, K, N, M, nullptr, vals, meta, stream);
+    if (r != NM_OK) return r;
     nm_sparse_operand S{};
     S.vals = vals;
     S.meta = meta;
@@ -1372,17 +1384,24 @@ int nm_act_sparse_linear_host(const void* x_host, int64_t T, int64_t K, int N, i
     S.N = N;
     S.M = M;
     S.K_lift = Kl;
-    if ((rc = nm_sparse_gemm(&S, w_lift, O, NM_ACT, yd, NM_BF16, nullptr, 0, stream)) != NM_OK) return rc;
+    if ((r = nm_sparse_gemm(&S, w_lift, O, NM_ACT, yd, NM_BF16, nullptr, 0, stream)) != NM_OK) return r;
     NM_CUDA_TRY(cudaEventRecord(p->done[b], st));
     // copy out
     NM_CUDA_TRY(cudaStreamWaitEvent(p->s_out, p->done[b], 0));
     NM_CUDA_TRY(cudaMemcpyAsync(static_cast<uint8_t*>(y_host) + r0 * O * 2, yd, static_cast<size_t>(rows * O * 2),
                                 cudaMemcpyDeviceToHost, p->s_out));
     NM_CUDA_TRY(cudaEventRecord(p->out[b], p->s_out));
-  }
-  // `stream` reaches this point once every chunk has been copied out
-  NM_CUDA_TRY(cudaStreamWaitEvent(st, p->out[0], 0));
-  NM_CUDA_TRY(cudaStreamWaitEvent(st, p->out[1], 0));
+    return NM_OK;
+  };
+  for (int64_t c = 0; c < chunks && rc == NM_OK; ++c) rc = enqueue_chunk(c);
+  // `stream` reaches this point once every queued chunk has been copied out;
+  // the join is made on the error path too, so that no copy into y_host is
+  // still in flight when work queued after this call on `stream` runs
+  const cudaError_t j0 = cudaStreamWaitEvent(st, p->out[0], 0);
+  const cudaError_t j1 = cudaStreamWaitEvent(st, p->out[1], 0);
+  if (rc != NM_OK) return rc;
+  NM_CUDA_TRY(j0);
+  NM_CUDA_TRY(j1);
   return NM_OK;
 }
 
@@ -1400,6 +1419,8 @@ const char* nm_status_string(int s) {
 }
 
 int nm_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* nm_last_gemm_kernel(void) { return g_last_gemm; }
 
 int nm_get_device_error(void* stream) {
   NM_CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
