@@ -464,7 +464,8 @@ int pick_splits(int64_t tiles, int64_t kb_total) {
 }
 
 // Kernel choice.  NMSPARSE_GEMM pins one variant where it applies:
-// "1cta", "2cta224", "2cta192", "2cta256", "2cta128", "2cta224x2", "2cta160x2";
+// "1cta", "2cta224", "2cta192", "2cta256", "2cta128", "2cta224x2", "2cta192x2",
+// "2cta160x2", "2cta128x2";
 // unset or "auto" picks by shape.
 int run_gemm(const GemmPlan& p, cudaStream_t st) {
   const char* env = std::getenv("NMSPARSE_GEMM");
@@ -482,7 +483,9 @@ int run_gemm(const GemmPlan& p, cudaStream_t st) {
     if (mode == "2cta256") return launch_gemm_2cta<256, 1, 1>(p, st);
     if (mode == "2cta128") return launch_gemm_2cta<128, 2, 1>(p, st);
     if (eligible4 && mode == "2cta224x2") return launch_gemm_2cta<224, 1, 2>(p, st);
+    if (eligible4 && mode == "2cta192x2") return launch_gemm_2cta<192, 1, 2>(p, st);
     if (eligible4 && mode == "2cta160x2") return launch_gemm_2cta<160, 1, 2>(p, st);
+    if (eligible4 && mode == "2cta128x2") return launch_gemm_2cta<128, 1, 2>(p, st);
     // products with dense k-blocks (hybrid, output-split, dense comparator)
     // on SM pairs; a narrow product with too few tiles to occupy half of the
     // SMs runs on single CTAs with split-K instead
@@ -518,21 +521,22 @@ int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M
   const int64_t Kl = nm_lifted_k(K, M);
   const int64_t KB = ceil_div(Kl, 128);
   const int64_t rows_pad = ceil_div(rows, 128) * 128;
-  const int64_t tasks = (rows_pad / 16) * ceil_div(K / M, 32 * nm::prune_groups_per_lane(M, sizeof(T)));
-  // one CTA per task for bf16 groups of up to 16 (the scheduler overlaps one
-  // CTA's loads with another's compute); a persistent grid otherwise
-  const bool per_task = sizeof(T) == 2 && M < 32;
+  const int64_t cpr = ceil_div(K / M, 32 * nm::prune_groups_per_lane(M, sizeof(T)));
+  const int64_t tasks = (rows_pad / 16) * cpr;
+  if (tasks >= (int64_t(1) << 31)) return NM_ERR_UNSUPPORTED;
+  // persistent grid: the resident CTAs of every SM take the tasks in turn
   const int64_t per_sm = nm::prune_min_blocks(M, sizeof(T));
-  const int64_t blocks = std::max<int64_t>(1, per_task ? tasks : std::min<int64_t>(tasks, int64_t(num_sms()) * per_sm));
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(tasks, int64_t(num_sms()) * per_sm));
   const dim3 grid(static_cast<unsigned>(blocks)), block(nm::kPruneWarps * 32);
+  nm::PruneGrid pg{static_cast<uint32_t>(cpr), static_cast<uint32_t>(tasks)};
   auto v = static_cast<uint32_t*>(vals);
   auto e = static_cast<uint8_t*>(meta);
   cudaError_t err;
   switch (M) {
-    case 4: err = launch_pdl(nm::k_prune_compress<4, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale, row_shift, stats); break;
-    case 8: err = launch_pdl(nm::k_prune_compress<8, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale, row_shift, stats); break;
-    case 16: err = launch_pdl(nm::k_prune_compress<16, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale, row_shift, stats); break;
-    case 32: err = launch_pdl(nm::k_prune_compress<32, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, rows_pad, row_scale, row_shift, stats); break;
+    case 4: err = launch_pdl(nm::k_prune_compress<4, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, pg, row_scale, row_shift, stats); break;
+    case 8: err = launch_pdl(nm::k_prune_compress<8, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, pg, row_scale, row_shift, stats); break;
+    case 16: err = launch_pdl(nm::k_prune_compress<16, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, pg, row_scale, row_shift, stats); break;
+    case 32: err = launch_pdl(nm::k_prune_compress<32, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, pg, row_scale, row_shift, stats); break;
     default: return NM_ERR_UNSUPPORTED;
   }
   NM_CUDA_TRY(err);
@@ -958,6 +962,12 @@ int nm_sparse_gemm_fp8(const nm_sparse_operand* S, const float* S_scale, const v
       case 64: return launch_gemm_bn<64, true>(p, splits, st);
       default: return launch_gemm_bn<128, true>(p, splits, st);
     }
+  }
+  if (p.rows_a % 512 == 0) {
+    // 512-row tiles (two 256-row MMAs per k-slice share the B stage)
+    if (mode == "2cta192x2") return launch_gemm_2cta<192, 1, 2, true>(p, st);
+    if (mode == "2cta160x2") return launch_gemm_2cta<160, 1, 2, true>(p, st);
+    if (mode == "2cta128x2") return launch_gemm_2cta<128, 1, 2, true>(p, st);
   }
   int bn = 0;
   if (mode == "2cta224") bn = 224;

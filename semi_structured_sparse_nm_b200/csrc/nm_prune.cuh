@@ -356,8 +356,8 @@ __device__ __forceinline__ void load_lane(const T* __restrict__ p, int64_t nvali
   }
 }
 
-// One CTA task = 16 consecutive rows x 32 lanes of G consecutive groups; warp
-// w takes rows 2w and 2w+1 (both loads in flight together).  A task row holds
+// One CTA task = 16 consecutive rows x 32 lanes of G consecutive groups (a
+// "chunk" of the row group); warp w takes rows 2w and 2w+1.  A task row holds
 // 32*G*NW windows, exactly G*NW metadata blocks of 32 windows, and 16 rows are
 // one contiguous 256-byte run inside a block (lanes 16j..16j+15 of the
 // tensor-memory image), so the CTA writes its metadata as whole 16-byte lane
@@ -367,14 +367,26 @@ __device__ __forceinline__ void load_lane(const T* __restrict__ p, int64_t nvali
 // none gives (0, 1); padded slots hold +0.0), values written through a
 // staging row as 16-byte stores.  Rows past `rows` (up to the 128-row padding
 // of the image) and windows past K'/4 get the index pair (0, 1).
+//
+// The grid is persistent: CTA b takes tasks b, b + gridDim.x, ... (row-group
+// major), stepped without divisions.  Each warp keeps the two rows it works
+// on in registers and requests the next task's row k as soon as it has
+// consumed row k of the current one, so one row's loads are in flight while
+// the other is processed and while the CTA writes the metadata.
 constexpr int kPruneWarps = 8;
 
 // Resident CTAs per SM the register budget is sized for: bf16 groups of up to
-// 16 run one CTA per task, four at a time per SM; M = 32 (and fp32) CTAs are
-// larger and loop over tasks.
+// 16 run four CTAs per SM; M = 32 (and fp32) CTAs are larger.
 __host__ __device__ constexpr int prune_min_blocks(int M, int elem_bytes) {
   return elem_bytes != 2 ? 1 : (M >= 32 ? 2 : 4);
 }
+
+// Task geometry: chunks per row group, ceil(groups / (32 G)), and the task
+// count, (rows rounded up to 128) / 16 * cpr.
+struct PruneGrid {
+  uint32_t cpr;
+  uint32_t tasks;
+};
 
 // Q8 = true (bf16 input only) writes the kept values as E4M3 codes --
 // code = e4m3(v * (1 / row_scale[r])) -- two bytes per window instead of two
@@ -391,7 +403,7 @@ template <int M, typename T, bool Q8 = false, bool XF = false>
 __global__ void __launch_bounds__(kPruneWarps * 32, prune_min_blocks(M, sizeof(T)))
 k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int N,
                  uint32_t* __restrict__ mask_out, void* __restrict__ vals_out,
-                 uint8_t* __restrict__ meta_out, int64_t Kl, int64_t KB, int64_t rows_pad,
+                 uint8_t* __restrict__ meta_out, int64_t Kl, int64_t KB, PruneGrid pg,
                  const float* __restrict__ row_scale, const float* __restrict__ row_shift,
                  double* __restrict__ stats) {
   static_assert(!Q8 || sizeof(T) == 2, "8-bit output from bf16 input");
@@ -410,155 +422,169 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
   if (threadIdx.x < 16) s_lut[threadIdx.x] = window_entry(threadIdx.x);
   griddep_wait();                                      // inputs / outputs of the preceding kernel
   const int64_t groups = K / M;
-  const int64_t cpr = (groups + 32 * G - 1) / (32 * G);
   const int64_t mask_words = (K + 31) / 32;
-  const int64_t tasks = (rows_pad / 16) * cpr;
   const bool vec_vals = Q8 ? (Kl % 32) == 0 : (Kl % 16) == 0;   // 16-byte output rows
+  const uint32_t cpr = pg.cpr;
+  const uint32_t drg = gridDim.x / cpr, dch = gridDim.x - drg * cpr;   // grid stride as (row group, chunk)
+  uint32_t task = blockIdx.x;
+  uint32_t rg = task / cpr, ch = task - rg * cpr;
 
-  const int64_t drg = gridDim.x / cpr, dch = gridDim.x % cpr;      // grid stride as (row group, chunk)
-  int64_t rg = blockIdx.x / cpr, ch = blockIdx.x % cpr;
-  for (int64_t task = blockIdx.x; task < tasks; task += gridDim.x) {
-    if (task != blockIdx.x) {
-      rg += drg;
-      ch += dch;
-      if (ch >= cpr) { ch -= cpr; ++rg; }
-    }
-    const int64_t g0 = ch * 32 * G, gl = g0 + static_cast<int64_t>(lane) * G;
+  // row k of this warp in task (rg_, ch_) -> raw[k] (nothing for rows or
+  // lanes past the operand)
+  GroupRaw<LM, T> raw[2];
+  auto load_row = [&](uint32_t rg_, uint32_t ch_, int k) {
+    const int64_t r = static_cast<int64_t>(rg_) * 16 + 2 * warp + k;
+    const int64_t gl = static_cast<int64_t>(ch_) * (32 * G) + lane * G;
+    if (r < rows && gl < groups) load_lane<M, G, T>(src + r * ld + gl * M, groups - gl, raw[k]);
+  };
+  if (task < pg.tasks) {
+    load_row(rg, ch, 0);
+    load_row(rg, ch, 1);
+  }
+  __syncthreads();                                     // s_lut
+  while (task < pg.tasks) {
+    const uint32_t next = task + gridDim.x;
+    uint32_t rg_n = rg + drg, ch_n = ch + dch;
+    if (ch_n >= cpr) { ch_n -= cpr; ++rg_n; }
+    const bool has_next = next < pg.tasks;
+    const int64_t g0 = static_cast<int64_t>(ch) * (32 * G), gl = g0 + static_cast<int64_t>(lane) * G;
     const int ng = static_cast<int>((groups - g0) < 32 * G ? (groups - g0) : 32 * G);
-    const int64_t r0 = rg * 16;
-    for (int i = threadIdx.x; i < 16 * WIN / 4; i += blockDim.x)
-      reinterpret_cast<uint32_t*>(&s_nib[0][0])[i] = 0x04040404u;
-    GroupRaw<LM, T> raw[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int64_t r = r0 + 2 * warp + k;
-      if (r < rows && gl < groups) load_lane<M, G, T>(src + r * ld + gl * M, groups - gl, raw[k]);
+    const int64_t r0 = static_cast<int64_t>(rg) * 16;
+    if (r0 + 16 > rows || ng != 32 * G) {
+      // a partial task: padding rows and windows carry the index pair (0, 1)
+      for (int i = threadIdx.x; i < 16 * WIN / 4; i += blockDim.x)
+        reinterpret_cast<uint32_t*>(&s_nib[0][0])[i] = 0x04040404u;
+      __syncthreads();                                 // padding in place before any row writes
     }
-    __syncthreads();                                   // padding in place before any row writes
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
       const int it = 2 * warp + k;
       const int64_t r = r0 + it;
-      if (r >= rows) break;
-      if (lane < LM) s_mask[warp][lane] = 0u;
-      __syncwarp();
-      float inv = 1.0f;
-      if constexpr (Q8) inv = __frcp_rn(row_scale[r]);
-      double st[2] = {0.0, 0.0};                       // transform mode: kept sums of this lane
-      if (gl < groups) {
-        uint32_t vals[NWL];
-        uint8_t nibs[NWL];
-        uint32_t keep = 0u;
-        if constexpr (sizeof(T) == 2) {
-          uint32_t PL[LM / 2];
+      if (r < rows) {
+        if (lane < LM) s_mask[warp][lane] = 0u;
+        __syncwarp();
+        float inv = 1.0f;
+        if constexpr (Q8) inv = __frcp_rn(row_scale[r]);
+        double st[2] = {0.0, 0.0};                     // transform mode: kept sums of this lane
+        if (gl < groups) {
+          uint32_t vals[NWL];
+          uint8_t nibs[NWL];
+          uint32_t keep = 0u;
+          if constexpr (sizeof(T) == 2) {
+            uint32_t PL[LM / 2];
 #pragma unroll
-          for (int p = 0; p < LM / 2; ++p) {
-            const uint4& q = raw[k].v[p / 4];
-            PL[p] = (p % 4 == 0) ? q.x : (p % 4 == 1) ? q.y : (p % 4 == 2) ? q.z : q.w;
+            for (int p = 0; p < LM / 2; ++p) {
+              const uint4& q = raw[k].v[p / 4];
+              PL[p] = (p % 4 == 0) ? q.x : (p % 4 == 1) ? q.y : (p % 4 == 2) ? q.z : q.w;
+            }
+            if constexpr (XF) {
+              if (row_shift != nullptr) {
+                const float mu = row_shift[r];
+#pragma unroll
+                for (int p = 0; p < LM / 2; ++p) {
+                  const __nv_bfloat162 h = __floats2bfloat162_rn(__fsub_rn(__uint_as_float(PL[p] << 16), mu),
+                                                                 __fsub_rn(__uint_as_float(PL[p] & 0xFFFF0000u), mu));
+                  PL[p] = *reinterpret_cast<const uint32_t*>(&h);
+                }
+              }
+            }
+#pragma unroll
+            for (int j = 0; j < G; ++j) {
+              uint32_t P[M / 2];
+#pragma unroll
+              for (int p = 0; p < M / 2; ++p) P[p] = PL[j * (M / 2) + p];
+              uint32_t vj[NW];
+              uint8_t nj[NW];
+              const uint32_t kj = compress_group_bf16<M>(P, N, s_lut, vj, nj);
+              const bool valid = (G == 1) || (gl + j < groups);
+#pragma unroll
+              for (int w = 0; w < NW; ++w) { vals[j * NW + w] = vj[w]; nibs[j * NW + w] = valid ? nj[w] : 0x4; }
+              if (valid) keep |= (M == 32 ? kj : (kj & ((1u << M) - 1u))) << (j * M);
+            }
+          } else {
+            keep = compress_group<M, T>(raw[k], N, vals, nibs);
           }
           if constexpr (XF) {
-            if (row_shift != nullptr) {
-              const float mu = row_shift[r];
+            if (stats != nullptr) {
+              // kept values: both slots of every window of the valid groups
+              // (padded slots hold +0.0)
 #pragma unroll
-              for (int p = 0; p < LM / 2; ++p) {
-                const __nv_bfloat162 h = __floats2bfloat162_rn(__fsub_rn(__uint_as_float(PL[p] << 16), mu),
-                                                               __fsub_rn(__uint_as_float(PL[p] & 0xFFFF0000u), mu));
-                PL[p] = *reinterpret_cast<const uint32_t*>(&h);
+              for (int w = 0; w < NWL; ++w) {
+                if ((G == 1) || (gl + w / NW < groups)) {
+                  const double a = __uint_as_float(vals[w] << 16), b = __uint_as_float(vals[w] & 0xFFFF0000u);
+                  st[0] += a + b;
+                  st[1] += a * a + b * b;
+                }
               }
             }
           }
 #pragma unroll
-          for (int j = 0; j < G; ++j) {
-            uint32_t P[M / 2];
-#pragma unroll
-            for (int p = 0; p < M / 2; ++p) P[p] = PL[j * (M / 2) + p];
-            uint32_t vj[NW];
-            uint8_t nj[NW];
-            const uint32_t kj = compress_group_bf16<M>(P, N, s_lut, vj, nj);
-            const bool valid = (G == 1) || (gl + j < groups);
-#pragma unroll
-            for (int w = 0; w < NW; ++w) { vals[j * NW + w] = vj[w]; nibs[j * NW + w] = valid ? nj[w] : 0x4; }
-            if (valid) keep |= (M == 32 ? kj : (kj & ((1u << M) - 1u))) << (j * M);
+          for (int w = 0; w < NWL; ++w) {
+            if constexpr (Q8) {
+              reinterpret_cast<uint16_t*>(&s_val[warp][0])[lane * NWL + w] = static_cast<uint16_t>(
+                  e4m3x2(__fmul_rn(elem_f32(static_cast<uint16_t>(vals[w] & 0xFFFFu)), inv),
+                         __fmul_rn(elem_f32(static_cast<uint16_t>(vals[w] >> 16)), inv)));
+            } else {
+              s_val[warp][lane * NWL + w] = vals[w];
+            }
+            s_nib[it][lane * NWL + w] = nibs[w];
+          }
+          if (mask_out != nullptr)
+            atomicOr(&s_mask[warp][(lane * LM) / 32],
+                     (LM == 32 ? keep : (keep & ((1u << LM) - 1u))) << ((lane * LM) % 32));
+        }
+        // raw[k] is consumed: request this warp's row k of the next task
+        if (has_next) load_row(rg_n, ch_n, k);
+        __syncwarp();
+        if constexpr (Q8) {
+          uint16_t* vrow = static_cast<uint16_t*>(vals_out) + r * (Kl / 4) + g0 * NW;
+          const uint16_t* sv16 = reinterpret_cast<const uint16_t*>(&s_val[warp][0]);
+          if (vec_vals && ng == 32 * G) {
+            const uint4* sv = reinterpret_cast<const uint4*>(sv16);
+            uint4* dv = reinterpret_cast<uint4*>(vrow);
+            for (int i = lane; i < WIN / 8; i += 32) dv[i] = sv[i];
+          } else {
+            for (int i = lane; i < ng * NW; i += 32) vrow[i] = sv16[i];
           }
         } else {
-          keep = compress_group<M, T>(raw[k], N, vals, nibs);
+          uint32_t* vrow = static_cast<uint32_t*>(vals_out) + r * (Kl / 4) + g0 * NW;
+          if (vec_vals && ng == 32 * G) {
+            const uint4* sv = reinterpret_cast<const uint4*>(&s_val[warp][0]);
+            uint4* dv = reinterpret_cast<uint4*>(vrow);
+            for (int i = lane; i < WIN / 4; i += 32) dv[i] = sv[i];
+          } else {
+            for (int i = lane; i < ng * NW; i += 32) vrow[i] = s_val[warp][i];
+          }
+        }
+        if (mask_out != nullptr && lane < LM) {
+          const int64_t wi = static_cast<int64_t>(ch) * LM + lane;
+          if (wi < mask_words) mask_out[r * mask_words + wi] = s_mask[warp][lane];
         }
         if constexpr (XF) {
           if (stats != nullptr) {
-            // kept values: both slots of every window of the valid groups
-            // (padded slots hold +0.0)
 #pragma unroll
-            for (int w = 0; w < NWL; ++w) {
-              if ((G == 1) || (gl + w / NW < groups)) {
-                const double a = __uint_as_float(vals[w] << 16), b = __uint_as_float(vals[w] & 0xFFFF0000u);
-                st[0] += a + b;
-                st[1] += a * a + b * b;
-              }
-            }
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) st[i] += __shfl_xor_sync(0xFFFFFFFFu, st[i], o);
+            if (lane == 0) reinterpret_cast<double2*>(stats)[r * cpr + ch] = make_double2(st[0], st[1]);
           }
         }
-#pragma unroll
-        for (int w = 0; w < NWL; ++w) {
-          if constexpr (Q8) {
-            reinterpret_cast<uint16_t*>(&s_val[warp][0])[lane * NWL + w] = static_cast<uint16_t>(
-                e4m3x2(__fmul_rn(elem_f32(static_cast<uint16_t>(vals[w] & 0xFFFFu)), inv),
-                       __fmul_rn(elem_f32(static_cast<uint16_t>(vals[w] >> 16)), inv)));
-          } else {
-            s_val[warp][lane * NWL + w] = vals[w];
-          }
-          s_nib[it][lane * NWL + w] = nibs[w];
-        }
-        if (mask_out != nullptr)
-          atomicOr(&s_mask[warp][(lane * LM) / 32],
-                   (LM == 32 ? keep : (keep & ((1u << LM) - 1u))) << ((lane * LM) % 32));
+        __syncwarp();
+      } else if (has_next) {
+        load_row(rg_n, ch_n, k);
       }
-      __syncwarp();
-      if constexpr (Q8) {
-        uint16_t* vrow = static_cast<uint16_t*>(vals_out) + r * (Kl / 4) + g0 * NW;
-        const uint16_t* sv16 = reinterpret_cast<const uint16_t*>(&s_val[warp][0]);
-        if (vec_vals && ng == 32 * G) {
-          const uint4* sv = reinterpret_cast<const uint4*>(sv16);
-          uint4* dv = reinterpret_cast<uint4*>(vrow);
-          for (int i = lane; i < WIN / 8; i += 32) dv[i] = sv[i];
-        } else {
-          for (int i = lane; i < ng * NW; i += 32) vrow[i] = sv16[i];
-        }
-      } else {
-        uint32_t* vrow = static_cast<uint32_t*>(vals_out) + r * (Kl / 4) + g0 * NW;
-        if (vec_vals && ng == 32 * G) {
-          const uint4* sv = reinterpret_cast<const uint4*>(&s_val[warp][0]);
-          uint4* dv = reinterpret_cast<uint4*>(vrow);
-          for (int i = lane; i < WIN / 4; i += 32) dv[i] = sv[i];
-        } else {
-          for (int i = lane; i < ng * NW; i += 32) vrow[i] = s_val[warp][i];
-        }
-      }
-      if (mask_out != nullptr && lane < LM) {
-        const int64_t wi = ch * LM + lane;
-        if (wi < mask_words) mask_out[r * mask_words + wi] = s_mask[warp][lane];
-      }
-      if constexpr (XF) {
-        if (stats != nullptr) {
-#pragma unroll
-          for (int i = 0; i < 2; ++i)
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) st[i] += __shfl_xor_sync(0xFFFFFFFFu, st[i], o);
-          if (lane == 0) reinterpret_cast<double2*>(stats)[r * cpr + ch] = make_double2(st[0], st[1]);
-        }
-      }
-      __syncwarp();
     }
     __syncthreads();
     // metadata: NWL blocks x 16 lane rows of 16 bytes.  Lane row L (0..15) of
     // block b holds rows L%8 and L%8+8 of the 16, windows 32b + 8c + 4(L/8) + 0..3
     // in word c (low half: first row, high half: second row).
-    const int64_t rb = r0 / 128;
-    const int64_t sub = (r0 % 128) / 16;
+    const int64_t rb = rg / 8;
+    const int sub = static_cast<int>(rg % 8);
     if constexpr (Q8) {
       // 8-bit image: row `row` of the task, windows 32b .. 32b+31 -> 16 bytes
       for (int i = threadIdx.x; i < NWL * 16; i += blockDim.x) {
         const int b = i / 16, row = i % 16;
-        const int64_t kb = ch * NWL + b;
+        const int64_t kb = static_cast<int64_t>(ch) * NWL + b;
         if (kb >= KB) continue;
         uint32_t wds[4];
 #pragma unroll
@@ -571,25 +597,28 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
             make_uint4(wds[0], wds[1], wds[2], wds[3]);
       }
     } else {
-    for (int i = threadIdx.x; i < NWL * 16; i += blockDim.x) {
-      const int b = i / 16, L = i % 16;
-      const int64_t kb = ch * NWL + b;
-      if (kb >= KB) continue;
-      const int i8 = L % 8, h = L / 8;
-      uint32_t wds[4];
+      for (int i = threadIdx.x; i < NWL * 16; i += blockDim.x) {
+        const int b = i / 16, L = i % 16;
+        const int64_t kb = static_cast<int64_t>(ch) * NWL + b;
+        if (kb >= KB) continue;
+        const int i8 = L % 8, h = L / 8;
+        uint32_t wds[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const int j = 32 * b + 8 * c + 4 * h;
-        // four nibble bytes n0..n3 -> bytes 0 and 2 of x | x >> 4 hold n0 | n1 << 4 and n2 | n3 << 4
-        const uint32_t lo = *reinterpret_cast<const uint32_t*>(&s_nib[i8][j]);
-        const uint32_t hi = *reinterpret_cast<const uint32_t*>(&s_nib[i8 + 8][j]);
-        wds[c] = __byte_perm(lo | (lo >> 4), hi | (hi >> 4), 0x6420);
+        for (int c = 0; c < 4; ++c) {
+          const int j = 32 * b + 8 * c + 4 * h;
+          // four nibble bytes n0..n3 -> bytes 0 and 2 of x | x >> 4 hold n0 | n1 << 4 and n2 | n3 << 4
+          const uint32_t lo = *reinterpret_cast<const uint32_t*>(&s_nib[i8][j]);
+          const uint32_t hi = *reinterpret_cast<const uint32_t*>(&s_nib[i8 + 8][j]);
+          wds[c] = __byte_perm(lo | (lo >> 4), hi | (hi >> 4), 0x6420);
+        }
+        *reinterpret_cast<uint4*>(meta_out + (rb * KB + kb) * 2048 + sub * 256 + L * 16) =
+            make_uint4(wds[0], wds[1], wds[2], wds[3]);
       }
-      *reinterpret_cast<uint4*>(meta_out + (rb * KB + kb) * 2048 + sub * 256 + L * 16) =
-          make_uint4(wds[0], wds[1], wds[2], wds[3]);
-    }
     }
     __syncthreads();                                   // s_nib is rewritten by the next task
+    task = next;
+    rg = rg_n;
+    ch = ch_n;
   }
 }
 

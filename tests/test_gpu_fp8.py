@@ -85,6 +85,26 @@ def test_fp8_product_exact_on_integer_grid():
     np.testing.assert_array_equal(host_f64(y), oracle.fp8_weight_sparse_linear(x, w, 6, 8))
 
 
+@pytest.mark.parametrize("variant", ["2cta224", "2cta160", "2cta192x2", "2cta160x2", "2cta128x2"])
+def test_fp8_tile_variants_exact_on_integer_grid(monkeypatch, variant):
+    """Every 8-bit tile variant of the SM-pair kernel, 512-row tiles included,
+    on E4M3-grid integers with row maxima 448 (both scales 1): exact, with a
+    partial last column tile and more tiles than one round of SM pairs."""
+    monkeypatch.setenv("NMSPARSE_GEMM", variant)
+    rng = np.random.default_rng(17)
+
+    def make(rows, K):
+        v = rng.integers(-16, 17, size=(rows, K)).astype(np.float64)
+        v[:, 0] = 448.0
+        return inputs.bf16_from_f64(v)
+    x, w = make(1000, 768), make(1024, 768)
+    P = nm.slide_decompose_fp8(dev(w), 6, 8)
+    y = nm.sparse_gemm_fp8(P, nm.quant_lift_fp8(dev(x), 8), nm.NM_WEIGHT, torch.float32)
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    np.testing.assert_array_equal(host_f64(y), oracle.fp8_weight_sparse_linear(x, w, 6, 8))
+
+
 def test_fp8_full_size():
     """The 6:8 weight-sparse prefill workload in 8 bits: the packed weight and
     the quantised, lifted activations bit-exact, every output row within

@@ -13,7 +13,7 @@ from tests.gpu_util import check_close, dev, host_f64
 
 pytestmark = pytest.mark.gpu
 
-VARIANTS = ["2cta224", "2cta192", "2cta256", "2cta128", "2cta224x2", "2cta160x2"]
+VARIANTS = ["2cta224", "2cta192", "2cta256", "2cta128", "2cta224x2", "2cta192x2", "2cta160x2", "2cta128x2"]
 
 
 def _int_bf16(rng, shape, lo=-4, hi=5):
