@@ -185,8 +185,15 @@ int nm_lift(const void *src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, i
  *   D      : bf16 lifted dense operand [rows_d][S->K_lift], row stride K_lift.
  *   Y      : NM_ACT -> [rows_s][rows_d]; NM_WEIGHT -> [rows_d][rows_s];
  *            row-major, dtype out_dt (NM_BF16 rounds to nearest even).
- *   ws     : scratch of nm_sparse_gemm_workspace_size() bytes (may be NULL
- *            when that size is 0).  Its contents need no initialisation.
+ *   ws     : optional scratch of nm_sparse_gemm_workspace_size() bytes,
+ *            16-byte aligned (NULL, or fewer bytes: none).  Products on SM
+ *            pairs whose tiles leave a last persistent round in which fewer
+ *            than half the pairs would work split that round's tiles along K
+ *            across the idle pairs, the parts' fp32 partial tiles going to ws
+ *            and a second launch adding them in part order (stream-K tail);
+ *            without ws that round runs whole.  The result is deterministic
+ *            either way; the two schedules round the fp32 sums in different
+ *            orders.  Its contents need no initialisation.
  * Requires K_lift % 16 == 0. */
 size_t nm_sparse_gemm_workspace_size(const nm_sparse_operand *S, int64_t rows_d, nm_side side);
 int nm_sparse_gemm(const nm_sparse_operand *S, const void *D, int64_t rows_d, nm_side side,
@@ -209,10 +216,17 @@ int nm_sparse_gemm(const nm_sparse_operand *S, const void *D, int64_t rows_d, nm
  * rows need K of about 2048 or less): each CTA loads the raw columns of X
  * its k-range needs and writes their lift into shared memory itself, so the
  * lifted X never goes through global memory and no workspace is used.
- * slide_gemm_workspace_size() returns 0 exactly for these shapes.  Other
- * shapes lift into ws first and run nm_sparse_gemm().  Results equal nm_lift() followed by nm_sparse_gemm()
- * bit for bit.  X may be written by the preceding kernel in the stream; W
- * follows the weight rule of nm_sparse_gemm(). */
+ * Prefill shapes also run as ONE kernel -- W->rows a multiple of 256 and
+ * rows_x >= 64: the SM-pair product, whose lift warps write every lifted B
+ * stage into shared memory straight from X (global memory, no staging copy)
+ * in place of the TMA load of a lifted copy.  slide_gemm_workspace_size()
+ * returns 0 exactly for these two families of shapes.  Other shapes lift
+ * into ws first and run nm_sparse_gemm().  Results equal nm_lift() followed
+ * by nm_sparse_gemm() bit for bit (on the prefill path, with the tile width
+ * that nm_sparse_gemm() picks for the same product: 128 below 512 rows of X,
+ * else 224, or 256 when K' >= 16384 and rows_x <= 8192).  X may be written by
+ * the preceding kernel in the stream; W follows the weight rule of
+ * nm_sparse_gemm(); the prefill path needs ldx even. */
 size_t slide_gemm_workspace_size(const nm_sparse_operand *W, int64_t rows_x);
 int slide_gemm(const nm_sparse_operand *W, const void *X, int64_t rows_x, int64_t ldx, void *Y,
                nm_dtype out_dt, void *ws, size_t ws_bytes, void *stream);
@@ -425,11 +439,14 @@ int hybrid_gemm_noalloc(const void *X, int64_t B, const nm_hybrid_weight *W, voi
  * y_host[T][O] = prune_{N:M}(x_host) . W^T, x_host bf16 [T][K] and y_host bf16
  * [T][O] in HOST memory (row-major, row strides K and O), w_lift the
  * device-resident lifted weight [O][K'] (nm_lift()).  The rows go through in
- * chunks of chunk_rows (a multiple of 128; 0 = 256): each chunk is copied in,
- * pruned and multiplied on `stream` and copied out on an auxiliary stream,
- * two chunks in flight, so that the copies out (the larger transfer) overlap
- * the copies in and the math of the following chunks.  The auxiliary stream
- * and its events are created on the first call on a device and kept; calls
+ * chunks of chunk_rows (a multiple of 128; 0 = 256): each chunk is copied in
+ * on one auxiliary stream, pruned and multiplied on `stream`, and copied out
+ * on another, with two buffer slots, so that the copy in of the next chunk
+ * and the copy out of the previous one overlap the math of the current one
+ * (PCIe carries both directions at once).  The prune of a chunk is launched
+ * without programmatic serialisation, so it starts only after its copy in.
+ * The auxiliary streams and their events are created on the first call on a
+ * device and kept; calls
  * are serialised on the host.  Host buffers should be page-locked
  * (cudaHostAlloc / cudaHostRegister), else the copies are not asynchronous.
  * Returns once everything is enqueued; y_host is complete when `stream`
@@ -458,8 +475,9 @@ int nm_last_cuda_error(void);
 /* Name of the GEMM kernel instantiation that the most recent GEMM launch of
  * this library on the calling thread used, for example
  * "k_nm_gemm_2cta<256,1,1>" (tile width, accumulator buffers, 256-row
- * subtiles; ",fp8" for 8-bit operands) or "k_nm_gemm<32>" (single-CTA
- * kernel, tile width); "" before the first.  The string is owned by the
+ * subtiles; ",fp8" for 8-bit operands, ",lift" for the in-GEMM lift,
+ * "+splitS" when the last round's tiles were split into S parts along K) or
+ * "k_nm_gemm<32>" (single-CTA kernel, tile width); "" before the first.  The string is owned by the
  * library and stays valid until the next GEMM launch on this thread. */
 const char *nm_last_gemm_kernel(void);
 /* Synchronises `stream`, then reads and clears the device status word that

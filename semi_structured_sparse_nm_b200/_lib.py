@@ -209,8 +209,13 @@ def lift(src: torch.Tensor, M: int, out: torch.Tensor | None = None) -> torch.Te
 # ----------------------------------------------------------------- GEMM
 
 
+def sparse_gemm_workspace_size(S: Compressed, rows_d: int, side: int) -> int:
+    st = S.struct()
+    return int(lib().nm_sparse_gemm_workspace_size(ctypes.byref(st), rows_d, side))
+
+
 def sparse_gemm(S: Compressed, D: torch.Tensor, side: int, out_dtype=torch.bfloat16,
-                out: torch.Tensor | None = None) -> torch.Tensor:
+                out: torch.Tensor | None = None, ws: torch.Tensor | None = None) -> torch.Tensor:
     """side NM_ACT: Y [S.rows, D.rows]; NM_WEIGHT: Y [D.rows, S.rows]."""
     _need_cuda(D)
     rows_d = D.shape[0]
@@ -221,9 +226,11 @@ def sparse_gemm(S: Compressed, D: torch.Tensor, side: int, out_dtype=torch.bfloa
         out = torch.empty(shape, dtype=out_dtype, device=D.device)
     st = S.struct()
     ws_bytes = int(lib().nm_sparse_gemm_workspace_size(ctypes.byref(st), rows_d, side))
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=D.device) if ws_bytes else None
+    if ws_bytes and (ws is None or ws.numel() < ws_bytes):
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=D.device)
     _check("nm_sparse_gemm", lib().nm_sparse_gemm(
-        ctypes.byref(st), _p(D), rows_d, side, _p(out), _dt(out), _p(ws), ws_bytes, _stream(D)))
+        ctypes.byref(st), _p(D), rows_d, side, _p(out), _dt(out), _p(ws if ws_bytes else None), ws_bytes,
+        _stream(D)))
     return out
 
 

@@ -107,6 +107,23 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// The same launch without programmatic serialisation: the kernel starts only
+// after everything queued before it on the stream (kernels, copies, event
+// waits) has completed.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_plain(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                         Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  if (g_fail_next_launch != 0) return injected_launch_error();
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // ----------------------------------------------------------------- GEMM
 struct GemmPlan {
   const void* a_s = nullptr;  // compressed sparse A [rows_a][ks_lift/2]
@@ -128,7 +145,13 @@ struct GemmPlan {
   const void* lift_x = nullptr;  // in-GEMM lift: B = lift(lift_x), raw bf16 [rows_b][lift_k], row stride lift_ldx
   int64_t lift_ldx = 0, lift_k = 0;
   int lift_m = 0;
+  void* ws = nullptr;            // optional scratch: the split last round's partial tiles (stream-K tail)
+  size_t ws_bytes = 0;
 };
+
+// Scratch bound of the split last round on SM pairs: at most one 256 x 256
+// fp32 partial tile per SM pair.
+size_t sk_workspace_bound() { return static_cast<size_t>(std::max(1, num_sms() / 2)) * 256 * 256 * 4; }
 
 // Ring depths of the in-GEMM lift kernel (compile-time instantiations), in
 // order of preference: 6 stages of A (about half the k-range of the 6:8
@@ -312,17 +335,17 @@ int make_tmap_meta(CUtensorMap* m, const void* base, int64_t blocks) {
 }
 
 // Number of 2-CTA clusters of this kernel that fit on the device at once.
-template <int BN, int NACC, int MSUB, bool FP8 = false>
+template <int BN, int NACC, int MSUB, bool FP8 = false, bool LIFT = false>
 int resident_pairs() {
   using Cfg = nm::Gemm2Cfg<BN, NACC, MSUB, FP8>;
-  auto kern = nm::k_nm_gemm_2cta<BN, NACC, MSUB, FP8>;
+  auto kern = nm::k_nm_gemm_2cta<BN, NACC, MSUB, FP8, LIFT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem) != cudaSuccess) {
     cudaGetLastError();
     return num_sms() / 2;
   }
   cudaLaunchConfig_t q{};
   q.gridDim = dim3(2, 1, 1);
-  q.blockDim = dim3(192, 1, 1);
+  q.blockDim = dim3(LIFT ? nm::kLiftThreads2 : 192, 1, 1);
   q.dynamicSmemBytes = Cfg::kSmem;
   cudaLaunchAttribute qa[1];
   qa[0].id = cudaLaunchAttributeClusterDimension;
@@ -341,9 +364,10 @@ int resident_pairs() {
 
 // Persistent 2-CTA kernel for pure-sparse products whose A side is a whole
 // number of 256-row blocks.
-template <int BN, int NACC, int MSUB, bool FP8 = false>
+template <int BN, int NACC, int MSUB, bool FP8 = false, bool LIFT = false>
 int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   using Cfg = nm::Gemm2Cfg<BN, NACC, MSUB, FP8>;
+  if (LIFT != (p.lift_x != nullptr)) return NM_ERR_UNSUPPORTED;
   CUtensorMap ta, tb, te, ty, tad;
   int rc;
   // k-blocks: 128 lifted K (bf16) or 256 (8-bit, the last one possibly 128)
@@ -385,7 +409,11 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   }
   if (!has_s) { ta = tad; te = tad; }
   if (!has_d) tad = ta;
-  if ((rc = make_tmap(&tb, p.b, b_cols, p.rows_b, b_cols * 2, 64, BN / 2)) != NM_OK) return rc;
+  if (LIFT) {
+    tb = ta;                                         // B is written by the lift warps; any valid map
+  } else if ((rc = make_tmap(&tb, p.b, b_cols, p.rows_b, b_cols * 2, 64, BN / 2)) != NM_OK) {
+    return rc;
+  }
   }
   nm::Gemm2Args a{};
   a.rows_a = p.rows_a;
@@ -410,16 +438,39 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   a.tma_store = tma_store;
   if (!tma_store) ty = ta;                             // unused; any valid map
   const int tiles = a.tiles_m * a.tiles_n;
-  auto kern = nm::k_nm_gemm_2cta<BN, NACC, MSUB, FP8>;
+  auto kern = nm::k_nm_gemm_2cta<BN, NACC, MSUB, FP8, LIFT>;
   NM_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem));
   cudaLaunchConfig_t cfg{};
   // A persistent grid larger than the number of co-resident SM pairs would
   // run its last clusters after the others: size it by the occupancy query.
   static int resident = 0;
-  if (resident == 0) resident = resident_pairs<BN, NACC, MSUB, FP8>();
+  if (resident == 0) resident = resident_pairs<BN, NACC, MSUB, FP8, LIFT>();
   const int clusters = std::max(1, std::min(tiles, resident));
+  // Split last round (stream-K tail): when the tiles leave a last persistent
+  // round in which fewer than half the SM pairs would work, and the caller
+  // gave scratch, each of that round's L tiles is split along K into
+  // clusters / L parts (at least two k-blocks each) run by otherwise idle
+  // pairs; k_sk_fixup adds the parts in order.  Plain bf16/fp32 outputs of
+  // pure 2:4 products only (no dense k-blocks, output split or epilogue
+  // scaling).
+  a.sk_full = tiles;
+  a.sk_parts = 0;
+  a.sk_ws = nullptr;
+  if (p.ws != nullptr && aligned16(p.ws) && MSUB == 1 && !FP8 && p.out_split_rows < 0 && p.kd == 0 &&
+      p.row_scale == nullptr && p.row_shift == nullptr) {
+    const int R = tiles / clusters, L = tiles - R * clusters;
+    if (R >= 1 && L > 0) {
+      const int parts = std::min(clusters / L, static_cast<int>(kb / 2));
+      const size_t need = static_cast<size_t>(L) * parts * 256 * BN * 4;
+      if (parts >= 2 && p.ws_bytes >= need) {
+        a.sk_full = R * clusters;
+        a.sk_parts = parts;
+        a.sk_ws = static_cast<float*>(p.ws);
+      }
+    }
+  }
   cfg.gridDim = dim3(static_cast<unsigned>(2 * clusters), 1, 1);
-  cfg.blockDim = dim3(192, 1, 1);
+  cfg.blockDim = dim3(LIFT ? nm::kLiftThreads2 : 192, 1, 1);
   cfg.dynamicSmemBytes = Cfg::kSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
@@ -431,10 +482,32 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  std::snprintf(g_last_gemm, sizeof(g_last_gemm), "k_nm_gemm_2cta<%d,%d,%d%s>", BN, NACC, MSUB, FP8 ? ",fp8" : "");
+  std::snprintf(g_last_gemm, sizeof(g_last_gemm), "k_nm_gemm_2cta<%d,%d,%d%s>", BN, NACC, MSUB,
+                FP8 ? ",fp8" : (LIFT ? ",lift" : ""));
   if (g_fail_next_launch != 0) NM_CUDA_TRY(injected_launch_error());
-  NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta, tb, te, ty, tad, a));
+  if constexpr (LIFT) {
+    nm::Gemm2LiftArgs la{};
+    static_cast<nm::Gemm2Args&>(la) = a;
+    la.lift_x = static_cast<const uint16_t*>(p.lift_x);
+    la.lift_ldx = p.lift_ldx;
+    la.lift_k = p.lift_k;
+    la.lift_m = p.lift_m;
+    NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta, tb, te, ty, tad, la));
+  } else {
+    NM_CUDA_TRY(cudaLaunchKernelEx(&cfg, kern, ta, tb, te, ty, tad, a));
+  }
   NM_CUDA_TRY(cudaGetLastError());
+  if (a.sk_parts > 1) {
+    const size_t n = std::strlen(g_last_gemm);
+    std::snprintf(g_last_gemm + n, sizeof(g_last_gemm) - n, "+split%d", a.sk_parts);
+    const int tail = tiles - a.sk_full;
+    const int64_t total = static_cast<int64_t>(tail) * 64 * BN;     // 4-output quads
+    const int64_t blocks = std::min<int64_t>(ceil_div(total, int64_t(256)), int64_t(num_sms()) * 8);
+    NM_CUDA_TRY(launch_pdl(nm::k_sk_fixup, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
+                           static_cast<const float*>(a.sk_ws), a.sk_full, a.sk_parts, tail, a.tiles_m, BN,
+                           p.rows_a, p.rows_b, p.y, p.ldy, p.out_fp32, p.transpose));
+    NM_CUDA_TRY(cudaGetLastError());
+  }
   return NM_OK;
 }
 int pick_bn(int64_t rows_b) {
@@ -514,10 +587,12 @@ int run_gemm(const GemmPlan& p, cudaStream_t st) {
 }
 
 // --------------------------------------------------------------- prune
+// early = false launches without programmatic serialisation (the prune then
+// waits for copies and event waits queued before it, not only for kernels).
 template <typename T, bool Q8 = false, bool XF = false>
 int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M, uint32_t* mask,
                  void* vals, void* meta, cudaStream_t st, const float* row_scale = nullptr,
-                 const float* row_shift = nullptr, double* stats = nullptr) {
+                 const float* row_shift = nullptr, double* stats = nullptr, bool early = true) {
   const int64_t Kl = nm_lifted_k(K, M);
   const int64_t KB = ceil_div(Kl, 128);
   const int64_t rows_pad = ceil_div(rows, 128) * 128;
@@ -531,12 +606,18 @@ int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M
   nm::PruneGrid pg{static_cast<uint32_t>(cpr), static_cast<uint32_t>(tasks)};
   auto v = static_cast<uint32_t*>(vals);
   auto e = static_cast<uint8_t*>(meta);
+  auto go = [&](auto kern) {
+    return early ? launch_pdl(kern, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, pg, row_scale,
+                              row_shift, stats)
+                 : launch_plain(kern, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, pg, row_scale,
+                                row_shift, stats);
+  };
   cudaError_t err;
   switch (M) {
-    case 4: err = launch_pdl(nm::k_prune_compress<4, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, pg, row_scale, row_shift, stats); break;
-    case 8: err = launch_pdl(nm::k_prune_compress<8, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, pg, row_scale, row_shift, stats); break;
-    case 16: err = launch_pdl(nm::k_prune_compress<16, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, pg, row_scale, row_shift, stats); break;
-    case 32: err = launch_pdl(nm::k_prune_compress<32, T, Q8, XF>, grid, block, 0, st, src, rows, K, ld, N, mask, v, e, Kl, KB, pg, row_scale, row_shift, stats); break;
+    case 4: err = go(nm::k_prune_compress<4, T, Q8, XF>); break;
+    case 8: err = go(nm::k_prune_compress<8, T, Q8, XF>); break;
+    case 16: err = go(nm::k_prune_compress<16, T, Q8, XF>); break;
+    case 32: err = go(nm::k_prune_compress<32, T, Q8, XF>); break;
     default: return NM_ERR_UNSUPPORTED;
   }
   NM_CUDA_TRY(err);
@@ -629,8 +710,13 @@ int nm_lift(const void* src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, i
 }
 
 size_t nm_sparse_gemm_workspace_size(const nm_sparse_operand* S, int64_t rows_d, nm_side side) {
-  (void)S; (void)rows_d; (void)side;
-  return 0;   // split-K partial sums stay in the cluster's shared memory
+  (void)side;
+  // products on SM pairs (whole 256-row tiles of the sparse operand, at
+  // least 512 rows of the dense one) may split their last round; the split-K
+  // of the single-CTA kernel keeps its partial sums in the cluster's shared
+  // memory
+  if (S == nullptr || S->rows <= 0 || S->rows % 256 != 0 || rows_d < 512) return 0;
+  return sk_workspace_bound();
 }
 
 }  // extern "C"
@@ -682,6 +768,16 @@ bool slide_fused_fits(const nm_sparse_operand* W, int splits) {
   return plan_lift_smem<BN>(kb_total, splits, W->K, W->M, &ls);
 }
 
+// In-GEMM lift on SM pairs (prefill shapes): the weight in whole 256-row
+// tiles, at least 64 activation rows, and the 32-bit window arithmetic of the
+// lift warps.  Returns the tile width (0: not this path).
+int slide_pair_bn(const nm_sparse_operand* W, int64_t rows_x) {
+  if (W->rows % 256 != 0 || rows_x < 64 || W->K_lift / 4 >= (int64_t(1) << 31)) return 0;
+  if (rows_x < 512) return 128;
+  if (rows_x <= 8192 && W->K_lift >= 16384) return 256;
+  return 224;
+}
+
 bool slide_fused_plan(const nm_sparse_operand* W, int64_t rows_x, int* bn, int* splits) {
   if (rows_x > 32 || W->K_lift >= (int64_t(1) << 24)) return false;   // the kernel's 32-bit window math
   *bn = pick_bn(rows_x);
@@ -696,11 +792,12 @@ extern "C" {
 
 int nm_sparse_gemm(const nm_sparse_operand* S, const void* D, int64_t rows_d, nm_side side, void* Y,
                    nm_dtype out_dt, void* ws, size_t ws_bytes, void* stream) {
-  (void)ws; (void)ws_bytes;
   GemmPlan p;
   bool empty = false;
   const int rc = sparse_plan(S, D, rows_d, side, Y, out_dt, &p, &empty);
   if (rc != NM_OK || empty) return rc;
+  p.ws = ws;
+  p.ws_bytes = ws != nullptr ? ws_bytes : 0;
   return run_gemm(p, static_cast<cudaStream_t>(stream));
 }
 
@@ -710,6 +807,8 @@ size_t slide_gemm_workspace_size(const nm_sparse_operand* W, int64_t rows_x) {
     return 0;
   int bn = 0, splits = 0;
   if (slide_fused_plan(W, rows_x, &bn, &splits)) return 0;
+  // SM pairs: optional scratch for a split last round (the lift needs none)
+  if (slide_pair_bn(W, rows_x) != 0) return rows_x >= 512 ? sk_workspace_bound() : 0;
   return static_cast<size_t>(ceil_div(rows_x * W->K_lift * 2, int64_t(16)) * 16);
 }
 
@@ -730,6 +829,20 @@ int slide_gemm(const nm_sparse_operand* W, const void* X, int64_t rows_x, int64_
     p.lift_k = W->K;
     p.lift_m = W->M;
     return bn == 16 ? launch_gemm_bn<16>(p, splits, st) : launch_gemm_bn<32>(p, splits, st);
+  }
+  if ((bn = slide_pair_bn(W, rows_x)) != 0) {
+    // prefill shapes: the lift warps of the SM-pair kernel write B from X
+    if (ldx % 2 != 0) return NM_ERR_ALIGNMENT;
+    p.ws = ws;
+    p.ws_bytes = ws != nullptr ? ws_bytes : 0;
+    p.b = nullptr;
+    p.lift_x = X;
+    p.lift_ldx = ldx;
+    p.lift_k = W->K;
+    p.lift_m = W->M;
+    if (bn == 128) return launch_gemm_2cta<128, 2, 1, false, true>(p, st);
+    if (bn == 256) return launch_gemm_2cta<256, 1, 1, false, true>(p, st);
+    return launch_gemm_2cta<224, 2, 1, false, true>(p, st);
   }
   // lift into the workspace, then the plain product
   if (ws == nullptr || ws_bytes < slide_gemm_workspace_size(W, rows_x)) return NM_ERR_WORKSPACE;
@@ -825,11 +938,25 @@ int nm_quant_lift_fp8(const void* src, nm_dtype dt, int64_t rows, int64_t K, int
       (reinterpret_cast<uintptr_t>(scale_out) & 3u) != 0)
     return NM_ERR_ALIGNMENT;
   auto st = static_cast<cudaStream_t>(stream);
-  const dim3 grid(static_cast<unsigned>(std::min<int64_t>(rows, int64_t(1) << 30))), block(256);
+  // one warp per row; CTAs of up to eight warps, fewer when there are few
+  // rows (so that they spread over the SMs); a grid of at most eight CTAs per
+  // SM loops over the rows
+  const int wpb = static_cast<int>(std::min<int64_t>(nm::kQuantWarps, std::max<int64_t>(1, rows / num_sms())));
+  const int64_t ctas = std::min<int64_t>(ceil_div(rows, int64_t(wpb)), int64_t(num_sms()) * 8);
+  const dim3 grid(static_cast<unsigned>(ctas)), block(wpb * 32);
+  const int64_t gpl = ceil_div(K / M, int64_t(32));             // groups per lane
   cudaError_t err;
-#define NM_QL(MM, TT)                                                                                      \
-  err = launch_pdl(nm::k_quant_lift_fp8<MM, TT>, grid, block, 0, st, static_cast<const TT*>(src), rows, K, ld, \
-                   codes_out, scale_out, Kl);
+  // the lane's groups stay in registers when there are at most GR of them
+#define NM_QL(MM, TT)                                                                                       \
+  {                                                                                                         \
+    constexpr int GR = nm::quant_groups_in_regs(MM, sizeof(TT));                                            \
+    if (gpl <= GR)                                                                                          \
+      err = launch_pdl(nm::k_quant_lift_fp8<MM, TT, GR>, grid, block, 0, st, static_cast<const TT*>(src), rows, \
+                       K, ld, codes_out, scale_out, Kl);                                                    \
+    else                                                                                                    \
+      err = launch_pdl(nm::k_quant_lift_fp8<MM, TT, 0>, grid, block, 0, st, static_cast<const TT*>(src), rows, \
+                       K, ld, codes_out, scale_out, Kl);                                                    \
+  }
   if (dt == NM_BF16) {
     switch (M) {
       case 4: NM_QL(4, uint16_t) break;
@@ -1302,8 +1429,9 @@ namespace {
 // first use and kept until the process exits.
 struct HostPipe {
   bool ready = false;
-  cudaStream_t s_out = nullptr;
-  cudaEvent_t done[2] = {}, out[2] = {};
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  // per buffer slot: X copied in, X consumed by the prune, GEMM done, Y copied out
+  cudaEvent_t in[2] = {}, x_free[2] = {}, done[2] = {}, out[2] = {};
 };
 std::mutex g_pipe_mu;
 HostPipe g_pipe[kMaxDevices];
@@ -1314,8 +1442,11 @@ int host_pipe(HostPipe** out) {
   if (dev < 0 || dev >= kMaxDevices) return NM_ERR_UNSUPPORTED;
   HostPipe& p = g_pipe[dev];
   if (!p.ready) {
+    NM_CUDA_TRY(cudaStreamCreateWithFlags(&p.s_in, cudaStreamNonBlocking));
     NM_CUDA_TRY(cudaStreamCreateWithFlags(&p.s_out, cudaStreamNonBlocking));
     for (int b = 0; b < 2; ++b) {
+      NM_CUDA_TRY(cudaEventCreateWithFlags(&p.in[b], cudaEventDisableTiming));
+      NM_CUDA_TRY(cudaEventCreateWithFlags(&p.x_free[b], cudaEventDisableTiming));
       NM_CUDA_TRY(cudaEventCreateWithFlags(&p.done[b], cudaEventDisableTiming));
       NM_CUDA_TRY(cudaEventCreateWithFlags(&p.out[b], cudaEventDisableTiming));
     }
@@ -1370,6 +1501,15 @@ int nm_act_sparse_linear_host(const void* x_host, int64_t T, int64_t K, int N, i
   HostPipe* p = nullptr;
   if ((rc = host_pipe(&p)) != NM_OK) return rc;
   const int64_t chunks = ceil_div(T, Tc);
+  // The caller's stream orders the call: both copy streams start after the
+  // work queued on it so far.
+  NM_CUDA_TRY(cudaEventRecord(p->done[0], st));
+  NM_CUDA_TRY(cudaStreamWaitEvent(p->s_in, p->done[0], 0));
+  NM_CUDA_TRY(cudaStreamWaitEvent(p->s_out, p->done[0], 0));
+  NM_CUDA_TRY(cudaEventRecord(p->x_free[0], st));
+  NM_CUDA_TRY(cudaEventRecord(p->x_free[1], st));
+  NM_CUDA_TRY(cudaEventRecord(p->out[0], st));
+  NM_CUDA_TRY(cudaEventRecord(p->out[1], st));
   auto enqueue_chunk = [&](int64_t c) -> int {
     const int b = static_cast<int>(c % 2);
     const int64_t r0 = c * Tc, rows = std::min(Tc, T - r0);
@@ -1377,15 +1517,22 @@ int nm_act_sparse_linear_host(const void* x_host, int64_t T, int64_t K, int N, i
     uint8_t* vals = xd + round256(Tc * K * 2);
     uint8_t* meta = vals + round256(Tc * (Kl / 2) * 2);
     uint8_t* yd = meta + round256(static_cast<int64_t>(nm_meta_bytes(Tc, K, M)));
-    // Copy in, prune and GEMM in order on the caller's stream (the copy sits
-    // between the kernels of consecutive chunks, so each chunk's kernels
-    // start only after its copy has landed).  Slot b's Y is free once the
-    // copy out of chunk c - 2 has read it.
-    NM_CUDA_TRY(cudaStreamWaitEvent(st, p->out[b], 0));
+    // copy in on its own stream, once the prune of chunk c - 2 has read slot
+    // b's X: it overlaps the prune and GEMM of chunk c - 1
+    NM_CUDA_TRY(cudaStreamWaitEvent(p->s_in, p->x_free[b], 0));
     NM_CUDA_TRY(cudaMemcpyAsync(xd, static_cast<const uint8_t*>(x_host) + r0 * K * 2, static_cast<size_t>(rows * K * 2),
-                                cudaMemcpyHostToDevice, st));
-    int r = nm_prune_compress(xd, NM_BF16, rows, K, K, N, M, nullptr, vals, meta, stream);
+                                cudaMemcpyHostToDevice, p->s_in));
+    NM_CUDA_TRY(cudaEventRecord(p->in[b], p->s_in));
+    // prune and GEMM on the caller's stream, once X has landed and the copy
+    // out of chunk c - 2 has read slot b's Y; the prune is launched without
+    // programmatic serialisation, so it waits for the event, not only for the
+    // preceding kernel
+    NM_CUDA_TRY(cudaStreamWaitEvent(st, p->in[b], 0));
+    NM_CUDA_TRY(cudaStreamWaitEvent(st, p->out[b], 0));
+    int r = launch_prune(reinterpret_cast<const uint16_t*>(xd), rows, K, K, N, M, nullptr, vals, meta, st, nullptr,
+                         nullptr, nullptr, /*early=*/false);
     if (r != NM_OK) return r;
+    NM_CUDA_TRY(cudaEventRecord(p->x_free[b], st));
     nm_sparse_operand S{};
     S.vals = vals;
     S.meta = meta;
@@ -1404,14 +1551,19 @@ int nm_act_sparse_linear_host(const void* x_host, int64_t T, int64_t K, int N, i
     return NM_OK;
   };
   for (int64_t c = 0; c < chunks && rc == NM_OK; ++c) rc = enqueue_chunk(c);
-  // `stream` reaches this point once every queued chunk has been copied out;
-  // the join is made on the error path too, so that no copy into y_host is
-  // still in flight when work queued after this call on `stream` runs
+  // `stream` reaches this point once every queued chunk has been copied out
+  // (and, through them, every copy in); the join is made on the error path
+  // too, so that no copy into y_host is still in flight when work queued
+  // after this call on `stream` runs
   const cudaError_t j0 = cudaStreamWaitEvent(st, p->out[0], 0);
   const cudaError_t j1 = cudaStreamWaitEvent(st, p->out[1], 0);
+  const cudaError_t j2 = cudaStreamWaitEvent(st, p->in[0], 0);
+  const cudaError_t j3 = cudaStreamWaitEvent(st, p->in[1], 0);
   if (rc != NM_OK) return rc;
   NM_CUDA_TRY(j0);
   NM_CUDA_TRY(j1);
+  NM_CUDA_TRY(j2);
+  NM_CUDA_TRY(j3);
   return NM_OK;
 }
 

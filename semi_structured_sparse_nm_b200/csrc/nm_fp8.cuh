@@ -36,12 +36,14 @@ __device__ __forceinline__ float fp8_scale_of(float amax) {
   return amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
 }
 
-// Per-token quantise + lift.  One CTA per row.  Pass 1 reduces |x| over the
-// row to its maximum (16-byte loads, block reduction); pass 2 takes one group
-// of M elements per thread (read again, now from L1), converts each element
-// once -- code = e4m3(x * (1 / scale)) -- and forms the group's n-1 windows
-// codes[r][g*4(n-1) + 4w + j] = code[g*2n + 2w + j] by byte permutes of the
-// packed codes, one 4-byte store per window.
+// Per-token quantise + lift.  One warp per row, eight rows per CTA.  Lane l
+// takes a contiguous run of groups (a multiple of four), so that its lifted
+// codes are one contiguous run of whole 16-byte words.  Pass 1 reduces |x|
+// over the lane's groups (16-byte loads) and the warp's lanes to the row
+// maximum; pass 2 reads the groups again (from L1) four at a time, converts
+// each element once -- code = e4m3(x * (1 / scale)) -- and forms each
+// group's n-1 windows codes[r][g*4(n-1) + 4w + j] = code[g*2n + 2w + j] by
+// byte permutes of the packed codes, stored as 16-byte words.
 template <int M, typename T>
 __device__ __forceinline__ void load_group_words(const T* __restrict__ p, uint32_t (&wd)[M * sizeof(T) / 4]) {
   constexpr int BYTES = M * static_cast<int>(sizeof(T));
@@ -57,66 +59,111 @@ __device__ __forceinline__ void load_group_words(const T* __restrict__ p, uint32
   }
 }
 
+// element e of a group held as 32-bit words, as fp32
+template <typename T, int WORDS>
+__device__ __forceinline__ float group_elem(const uint32_t (&wd)[WORDS], int e) {
+  if constexpr (sizeof(T) == 2) {
+    const uint32_t w = wd[e / 2];
+    return __uint_as_float((e % 2 == 0) ? (w << 16) : (w & 0xFFFF0000u));
+  } else {
+    return __uint_as_float(wd[e]);
+  }
+}
+
+// The group's codes (four per word) and its NW window words.
 template <int M, typename T>
-__global__ void __launch_bounds__(256)
+__device__ __forceinline__ void quant_group_windows(const uint32_t (&wd)[M * sizeof(T) / 4], float inv,
+                                                    uint32_t* win) {
+  constexpr int NW = M / 2 - 1;
+  constexpr int WORDS = M * static_cast<int>(sizeof(T)) / 4;
+  uint32_t q[M / 4];
+#pragma unroll
+  for (int c = 0; c < M / 4; ++c) {
+    const float f0 = group_elem<T, WORDS>(wd, 4 * c), f1 = group_elem<T, WORDS>(wd, 4 * c + 1);
+    const float f2 = group_elem<T, WORDS>(wd, 4 * c + 2), f3 = group_elem<T, WORDS>(wd, 4 * c + 3);
+    q[c] = e4m3x2(__fmul_rn(f0, inv), __fmul_rn(f1, inv)) | (e4m3x2(__fmul_rn(f2, inv), __fmul_rn(f3, inv)) << 16);
+  }
+  // window w = codes 2w .. 2w+3: word w/2 when w is even, else the upper
+  // half of word (w-1)/2 and the lower half of the next one
+#pragma unroll
+  for (int w = 0; w < NW; ++w) win[w] = (w % 2 == 0) ? q[w / 2] : __byte_perm(q[w / 2], q[w / 2 + 1], 0x5432);
+}
+
+constexpr int kQuantWarps = 8;
+
+// One warp per row; the grid's CTAs hold up to kQuantWarps warps (fewer for
+// short batches, so that a few rows still spread over as many SMs).  Lane l
+// takes groups l, l + 32, l + 64, ... so that each load instruction of the
+// warp reads 32 consecutive groups.  With G > 0 the lane's groups (at most G)
+// stay in registers between the maximum and the conversion; G = 0 reads them
+// twice (the second time from L1).
+template <int M, typename T, int G>
+__global__ void __launch_bounds__(kQuantWarps * 32)
 k_quant_lift_fp8(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
                  uint8_t* __restrict__ codes, float* __restrict__ scale_out, int64_t Kl) {
   constexpr int NW = M / 2 - 1;
-  constexpr int PV = 16 / static_cast<int>(sizeof(T));
   constexpr int WORDS = M * static_cast<int>(sizeof(T)) / 4;     // 32-bit words of one group
-  __shared__ float s_red[8];
   griddep_launch_dependents();
   griddep_wait();
+  const int wpb = blockDim.x / 32;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t groups = K / M;
-  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+  for (int64_t r = static_cast<int64_t>(blockIdx.x) * wpb + warp; r < rows; r += static_cast<int64_t>(gridDim.x) * wpb) {
     const T* row = src + r * ld;
-    float amax = 0.0f;
-    for (int64_t i = static_cast<int64_t>(threadIdx.x) * PV; i < K; i += 256 * PV) {
-      if (i + PV <= K) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(row + i));
-        const T* e = reinterpret_cast<const T*>(&u);
-#pragma unroll
-        for (int j = 0; j < PV; ++j) amax = fmaxf(amax, fabsf(elem_f32(e[j])));
-      } else if constexpr (sizeof(T) == 2) {           // a bf16 row ending in half a 16-byte word
-        const uint2 u = __ldg(reinterpret_cast<const uint2*>(row + i));
-        const T* e = reinterpret_cast<const T*>(&u);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) amax = fmaxf(amax, fabsf(elem_f32(e[j])));
-      }
-    }
-    const float sc = fp8_scale_of(block_max_256(amax, s_red));
-    const float inv = __frcp_rn(sc);
-    if (threadIdx.x == 0) scale_out[r] = sc;
     uint32_t* out = reinterpret_cast<uint32_t*>(codes + r * Kl);
-    for (int64_t g = threadIdx.x; g < groups; g += 256) {
-      uint32_t wd[WORDS];
-      load_group_words<M, T>(row + g * M, wd);
-      uint32_t q[M / 4];                               // codes of the group, four per word
+    float amax = 0.0f;
+    if constexpr (G > 0) {
+      uint32_t wd[G][WORDS];
 #pragma unroll
-      for (int c = 0; c < M / 4; ++c) {
-        float f[4];
+      for (int k = 0; k < G; ++k) {
+        const int64_t g = lane + 32 * k;
+        if (g < groups) {
+          load_group_words<M, T>(row + g * M, wd[k]);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int e = 4 * c + j;
-          if constexpr (sizeof(T) == 2) {
-            const uint32_t w = wd[e / 2];
-            f[j] = __uint_as_float((e % 2 == 0) ? (w << 16) : (w & 0xFFFF0000u));
-          } else {
-            f[j] = __uint_as_float(wd[e]);
-          }
+          for (int e = 0; e < M; ++e) amax = fmaxf(amax, fabsf(group_elem<T, WORDS>(wd[k], e)));
         }
-        q[c] = e4m3x2(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv)) |
-               (e4m3x2(__fmul_rn(f[2], inv), __fmul_rn(f[3], inv)) << 16);
       }
-      // window w = codes 2w .. 2w+3: word w/2 when w is even, else the upper
-      // half of word (w-1)/2 and the lower half of the next one
 #pragma unroll
-      for (int w = 0; w < NW; ++w)
-        out[g * NW + w] = (w % 2 == 0) ? q[w / 2] : __byte_perm(q[w / 2], q[w / 2 + 1], 0x5432);
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      const float sc = fp8_scale_of(amax);
+      const float inv = __frcp_rn(sc);
+      if (lane == 0) scale_out[r] = sc;
+#pragma unroll
+      for (int k = 0; k < G; ++k) {
+        const int64_t g = lane + 32 * k;
+        if (g < groups) {
+          uint32_t win[NW];
+          quant_group_windows<M, T>(wd[k], inv, win);
+#pragma unroll
+          for (int w = 0; w < NW; ++w) out[g * NW + w] = win[w];
+        }
+      }
+    } else {
+      for (int64_t g = lane; g < groups; g += 32) {
+        uint32_t wd[WORDS];
+        load_group_words<M, T>(row + g * M, wd);
+#pragma unroll
+        for (int e = 0; e < M; ++e) amax = fmaxf(amax, fabsf(group_elem<T, WORDS>(wd, e)));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      const float sc = fp8_scale_of(amax);
+      const float inv = __frcp_rn(sc);
+      if (lane == 0) scale_out[r] = sc;
+      for (int64_t g = lane; g < groups; g += 32) {
+        uint32_t wd[WORDS], win[NW];
+        load_group_words<M, T>(row + g * M, wd);
+        quant_group_windows<M, T>(wd, inv, win);
+#pragma unroll
+        for (int w = 0; w < NW; ++w) out[g * NW + w] = win[w];
+      }
     }
-    __syncthreads();                                   // s_red is reused by the next row
   }
 }
+
+// Groups per lane held in registers (at most 256 bytes of a row per lane),
+// or 0 for the two-pass form.
+__host__ __device__ constexpr int quant_groups_in_regs(int M, int elem_bytes) { return 256 / (M * elem_bytes); }
 
 // scale[r] = amax(w[r][:]) / 448 for bf16 rows of length K (row stride ld).
 __global__ void __launch_bounds__(256)

@@ -27,12 +27,32 @@
 // blocks per 128 rows (tensor-memory columns +2 per MMA), and the epilogue
 // multiplies the accumulator by the row scale of A and the column scale of B.
 //
+// LIFT = true is the in-GEMM lift of the weight-side (2n-2):2n product: B,
+// the lifted activations, is not read from a lifted copy in global memory.
+// Eight more warps ("lift warps", 256 threads per CTA) fill each stage's B
+// half themselves, from the raw activations X [rows_b][K] (row stride
+// lift_ldx), in the layout the TMA would have left: lifted column j of a
+// k-block is raw column g M + 2w + (j % 4) with (g, w) the group and window of
+// lifted window j / 4, rows and columns past the operand zero.  A lane takes
+// one window (8 bytes) of a 128-lifted-column row, so that one instruction of
+// a warp reads about 170 consecutive bytes of X; the copies are asynchronous
+// global -> shared copies (cp.async, one of 8 bytes or two of 4 by the
+// source's alignment, zero-filled past the operand) written straight into
+// the swizzled stage, so no register holds the data and several stages are
+// in flight at once.  Each lift thread then arrives on its CTA's lift
+// barrier when its copies have landed; one more warp per CTA (the forwarder)
+// waits on it, fences the async proxy and arrives on the leader's full
+// barrier (two arrivals per stage besides the producer's).  The summation
+// order is that of the TMA-fed product, so results are equal bit for bit.
+//
 // MSUB = 2 makes the tile 512 x BN: each k-slice issues two M = 256 MMAs that
 // share the B stage (CTA r holds A rows 512 tm + 256 u + 128 r for u = 0, 1).
 // That cuts the shared-memory fill per MMA cycle from 64 + 8192/BN to
 // 32 + 8192/BN bytes per SM, which is what the L2 -> SM path can sustain;
 // tensor memory then holds one accumulator set (NACC = 1).
 #pragma once
+#include <type_traits>
+
 #include "nm_device.cuh"
 
 namespace nm {
@@ -142,7 +162,42 @@ struct Gemm2Args {
                           // (sparse k-blocks only), the rest dense rows (dense k-blocks
                           // only, A rows counted from the dense matrix's first row, B from
                           // column 0)
+  // Split last round (stream-K tail; sk_parts < 2: none).  Tiles [0, sk_full)
+  // run whole in persistent rounds (sk_full is a multiple of the cluster
+  // count); in the round after them, cluster u takes k-part u % sk_parts of
+  // tile sk_full + u / sk_parts and leaves its fp32 accumulator in sk_ws
+  // (unit ((tile - sk_full) * sk_parts + part), [256 rows][BN], no epilogue
+  // scaling); k_sk_fixup sums the parts and writes those tiles of Y.
+  int sk_full;
+  int sk_parts;
+  float* sk_ws;
 };
+
+// In-GEMM lift parameters (LIFT = true only; the other instantiations keep
+// the plain parameter type).
+struct Gemm2LiftArgs : Gemm2Args {
+  const uint16_t* lift_x;   // raw activations [rows_b][lift_k], bf16
+  int64_t lift_ldx;         // row stride of lift_x, elements
+  int64_t lift_k;           // raw K
+  int lift_m;               // group size M of the (2n-2):2n pattern
+};
+constexpr int kLiftWarps2 = 8;
+constexpr int kLiftThreads2 = 192 + 32 * kLiftWarps2 + 32;   // + the forwarder warp
+enum : unsigned { kWhereLift2 = 4 };
+
+// Asynchronous global -> shared copies of 4 or 8 bytes (zero-filled when
+// `valid` is false: no byte is read), and the arrival on an mbarrier once the
+// calling thread's earlier copies have landed (counted in the barrier's
+// arrival count).
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" :: "r"(dst), "l"(src), "r"(valid ? 4 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_8(uint32_t dst, const void* src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" :: "r"(dst), "l"(src), "r"(valid ? 8 : 0) : "memory");
+}
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" :: "r"(smem_u32(bar)) : "memory");
+}
 
 // The tile a cluster takes in its round j of the persistent loop: round j
 // covers tiles [j P, j P + P) for P clusters.  Output-split products, whose
@@ -169,6 +224,34 @@ __device__ __forceinline__ Tile2 tile2_of(const Gemm2Args& g, int tm) {
   return {tm - nd, tm - nd, 0, g.kb};
 }
 
+// The j-th piece of work of a cluster: an output tile (t < 0: no more work),
+// its k-block range, and its stream-K part (-1: the whole tile).
+struct Work2 {
+  int t, part;
+  Tile2 tl;
+};
+__device__ __forceinline__ Work2 work2_at(const Gemm2Args& g, int j, int cluster, int clusters) {
+  const int tiles = g.tiles_m * g.tiles_n;
+  Work2 w{-1, -1, {0, 0, 0, 0}};
+  if (g.sk_parts > 1 && j >= g.sk_full / clusters) {
+    if (j > g.sk_full / clusters) return w;
+    const int t = g.sk_full + cluster / g.sk_parts;
+    if (t >= tiles) return w;
+    w.t = t;
+    w.part = cluster % g.sk_parts;
+    w.tl = tile2_of(g, t % g.tiles_m);
+    const int lo = w.tl.kb_lo, n = w.tl.kb_hi - w.tl.kb_lo;
+    w.tl.kb_lo = lo + n * w.part / g.sk_parts;
+    w.tl.kb_hi = lo + n * (w.part + 1) / g.sk_parts;
+    return w;
+  }
+  const int t = tile2_at(j, cluster, clusters, g.out_split_tiles);
+  if (t >= tiles) return w;
+  w.t = t;
+  w.tl = tile2_of(g, t % g.tiles_m);
+  return w;
+}
+
 template <int BN, int NACC, int MSUB, bool FP8 = false>
 struct Gemm2Cfg {
   static constexpr int kHalfN = BN / 2;
@@ -192,11 +275,51 @@ struct Gemm2Cfg {
   static_assert(kStages >= 3, "ring too shallow");
 };
 
-template <int BN, int NACC, int MSUB, bool FP8 = false>
-__global__ void __launch_bounds__(192, 1)
+// Issues the copies of one stage's B half for the in-GEMM lift (lift warps,
+// 256 threads): rows [y0, y0 + BN/2) of the lifted activations, lifted
+// columns [128 kb, 128 kb + 128), into the two 128-byte-swizzled column
+// halves at sB_stage.  Lane l copies window 32 kb + l of rows w, w + 8, ...
+// (w the lift warp).
+template <int BN>
+__device__ __forceinline__ void lift_stage_b(const Gemm2LiftArgs& args, int kb, int64_t y0, uint8_t* sB_stage) {
+  constexpr int HN = BN / 2;
+  const int t = static_cast<int>(threadIdx.x) - 192;     // 0 .. 255
+  const int lw = t / 32, lane = t % 32;
+  // 32-bit index arithmetic: K' / 4 < 2^31 (host check)
+  const uint32_t M = static_cast<uint32_t>(args.lift_m);
+  const uint32_t nw = M / 2 - 1;
+  const uint32_t nwin = static_cast<uint32_t>(args.lift_k / args.lift_m) * nw;   // lifted windows per row
+  const uint32_t q = static_cast<uint32_t>(kb) * 32u + static_cast<uint32_t>(lane);
+  const uint32_t g = q / nw, w = q - g * nw;
+  const bool q_ok = q < nwin;
+  const int64_t e0 = q_ok ? static_cast<int64_t>(g) * M + 2 * w : 0;    // raw element of the window
+  const bool wide = (e0 % 4) == 0;                        // the window's 8 source bytes are 8-byte aligned
+  // destination: chunk lane / 2 of the 128-column row (half lane / 16), its
+  // lower or upper 8 bytes
+  const int c = lane / 2, h = c / 8, c8 = c % 8;
+  const uint32_t sb = smem_u32(sB_stage) + h * (HN * 128) + 8 * (lane % 2);
+  const uint16_t* x = args.lift_x;
+  for (int rr = lw; rr < HN; rr += kLiftWarps2) {
+    const int64_t row = y0 + rr;
+    const bool ok = q_ok && row < args.rows_b;
+    const uint16_t* src = x + (ok ? row * args.lift_ldx + e0 : 0);
+    const uint32_t dst = sb + rr * 128 + 16 * (c8 ^ (rr % 8));
+    if (wide) {
+      cp_async_8(dst, src, ok);
+    } else {
+      cp_async_4(dst, src, ok);
+      cp_async_4(dst + 4, src + 2, ok);
+    }
+  }
+}
+
+template <int BN, int NACC, int MSUB, bool FP8 = false, bool LIFT = false>
+__global__ void __launch_bounds__(LIFT ? kLiftThreads2 : 192, 1)
 k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
-               const __grid_constant__ CUtensorMap tmAd, const Gemm2Args args) {
+               const __grid_constant__ CUtensorMap tmAd,
+               const std::conditional_t<LIFT, Gemm2LiftArgs, Gemm2Args> args) {
+  static_assert(!LIFT || (!FP8 && MSUB == 1), "in-GEMM lift: bf16, 256-row tiles");
   using Cfg = Gemm2Cfg<BN, NACC, MSUB, FP8>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw2[];
@@ -209,7 +332,8 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   uint64_t* empty_bar = full_bar + S;
   uint64_t* tfull_bar = empty_bar + S;
   uint64_t* tempty_bar = tfull_bar + NACC;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty_bar + NACC);
+  uint64_t* lift_bar = tempty_bar + NACC;            // in-GEMM lift: the stage's copies have landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lift_bar + (LIFT ? S : 0));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -220,7 +344,12 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   const int tiles = args.tiles_m * args.tiles_n;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) { mbar_init(&full_bar[s], 1); mbar_init(&empty_bar[s], 1); }
+    // full: the producer's expect_tx arrival, plus (in-GEMM lift) the
+    // forwarder's of both CTAs; lift: one arrival per lift thread, made when
+    // its copies of the stage have landed
+    for (int s = 0; s < S; ++s) { mbar_init(&full_bar[s], LIFT ? 3 : 1); mbar_init(&empty_bar[s], 1); }
+    if (LIFT)
+      for (int s = 0; s < S; ++s) mbar_init(&lift_bar[s], 32 * kLiftWarps2);
     for (int b = 0; b < NACC; ++b) { mbar_init(&tfull_bar[b], 1); mbar_init(&tempty_bar[b], 8); }
     *abort_flag = 0;
     fence_mbar_init();
@@ -246,9 +375,11 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const uint32_t dense_tx = static_cast<uint32_t>(2 * (MSUB * Cfg::kA1 + Cfg::kHalfN * 128));
       int it = 0;
       bool ok = true;
-      for (int j = 0, t = cluster_id; t < tiles && ok; t = tile2_at(++j, cluster_id, num_clusters, args.out_split_tiles)) {
-        const Tile2 tl = tile2_of(args, t % args.tiles_m);
-        const int tm = tl.a, tn = t / args.tiles_m;
+      for (int j = 0; ok; ++j) {
+        const Work2 wk = work2_at(args, j, cluster_id, num_clusters);
+        if (wk.t < 0) break;
+        const Tile2 tl = wk.tl;
+        const int tm = tl.a, tn = wk.t / args.tiles_m;
         const int32_t yb = tn * BN + static_cast<int32_t>(rank) * Cfg::kHalfN;
         for (int kb = tl.kb_lo; kb < tl.kb_hi; ++kb, ++it) {
           const int s = it % S;
@@ -285,7 +416,8 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
             tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB, kb * 256, yb);
             if (eb == 2) tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB + Cfg::kHalfN * 128, kb * 256 + 128, yb);
           } else {
-            if (leader) mbar_arrive_expect_tx(&full_bar[s], stage_tx);
+            // in-GEMM lift: B comes from the lift warps, the TMA brings A and metadata
+            if (leader) mbar_arrive_expect_tx(&full_bar[s], LIFT ? stage_tx - 2 * Cfg::kB : stage_tx);
 #pragma unroll
             for (int u = 0; u < MSUB; ++u) {
               const int64_t rb = (static_cast<int64_t>(tm) * MSUB + u) * 2 + rank;     // 128-row block
@@ -293,8 +425,10 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
               tma_load_2d_pair(&tmE, fb, sE + s * Cfg::kE + u * 2048, 0,
                                static_cast<int32_t>((rb * args.meta_kb + kb) * 16));
             }
-            tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB, kb * 128, yb);
-            tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB + Cfg::kHalfN * 128, kb * 128 + 64, yb);
+            if constexpr (!LIFT) {
+              tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB, kb * 128, yb);
+              tma_load_2d_pair(&tmB, fb, sB + s * Cfg::kB + Cfg::kHalfN * 128, kb * 128 + 64, yb);
+            }
           }
         }
       }
@@ -311,9 +445,10 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const uint32_t idesc_dn = idesc_bf16(256, BN, false);
       int it = 0, lt = 0;
       bool ok = true;
-      for (int j = 0, t = cluster_id; t < tiles && ok;
-           t = tile2_at(++j, cluster_id, num_clusters, args.out_split_tiles), ++lt) {
-        const Tile2 tl = tile2_of(args, t % args.tiles_m);
+      for (int j = 0; ok; ++j, ++lt) {
+        const Work2 wk = work2_at(args, j, cluster_id, num_clusters);
+        if (wk.t < 0) break;
+        const Tile2 tl = wk.tl;
         const int b = lt % NACC;
         const uint32_t use = static_cast<uint32_t>(lt / NACC);
         if (!mbar_wait(&tempty_bar[b], (use & 1u) ^ 1u, abort_flag, kWhereMma)) break;
@@ -323,7 +458,7 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           const int s = it % S;
           const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
           const uint32_t accum0 = kb > tl.kb_lo ? 1u : 0u;     // the tile's first k-block overwrites
-          if (!mbar_wait(&full_bar[s], ph, abort_flag, kWhereMma)) { ok = false; break; }
+          if (!mbar_wait<LIFT>(&full_bar[s], ph, abort_flag, kWhereMma)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * Cfg::kA);
           const uint32_t b0 = smem_u32(sB + s * Cfg::kB);
@@ -383,6 +518,38 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
         if (ok) tc_commit_pair(&tfull_bar[b]);
       }
     }
+  } else if (LIFT && warp >= 6) {
+    // ------------------------------------- lift warps and their forwarder
+    if constexpr (LIFT) {
+      const bool forwarder = warp == 6 + kLiftWarps2;
+      if (!forwarder || lane == 0) {
+        int it = 0;
+        bool ok = true;
+        for (int j = 0; ok; ++j) {
+          const Work2 wk = work2_at(args, j, cluster_id, num_clusters);
+          if (wk.t < 0) break;
+          const int tn = wk.t / args.tiles_m;
+          const int64_t y0 = static_cast<int64_t>(tn) * BN + static_cast<int64_t>(rank) * Cfg::kHalfN;
+          for (int kb = wk.tl.kb_lo; kb < wk.tl.kb_hi; ++kb, ++it) {
+            const int s = it % S;
+            const uint32_t ph = static_cast<uint32_t>(it / S) & 1u;
+            if (forwarder) {
+              // the lift threads' copies of this stage have landed: publish
+              // them to the tensor cores of the pair
+              if (!mbar_wait(&lift_bar[s], ph, abort_flag, kWhereLift2)) { ok = false; break; }
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+              mbar_arrive_cluster(leader_addr(smem_u32(&full_bar[s])));
+            } else {
+              if (!mbar_wait(&empty_bar[s], ph ^ 1u, abort_flag, kWhereLift2)) { ok = false; break; }
+              lift_stage_b<BN>(args, kb, y0, sB + s * Cfg::kB);
+              cp_async_arrive_noinc(&lift_bar[s]);
+            }
+          }
+        }
+        // copies still in flight land before the CTA may exit
+        if (!forwarder) asm volatile("cp.async.wait_all;" ::: "memory");
+      }
+    }
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp % 4;
@@ -397,8 +564,10 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     st.ldy = args.ldy;
     st.out_fp32 = args.out_fp32;
     st.transpose_out = args.transpose_out;
-    for (int j = 0, t = cluster_id; t < tiles; t = tile2_at(++j, cluster_id, num_clusters, args.out_split_tiles), ++lt) {
-      const int tm = tile2_of(args, t % args.tiles_m).out, tn = t / args.tiles_m;
+    for (int j = 0;; ++j, ++lt) {
+      const Work2 wk = work2_at(args, j, cluster_id, num_clusters);
+      if (wk.t < 0) break;
+      const int tm = wk.tl.out, tn = wk.t / args.tiles_m;
       const int b = lt % NACC;
       const uint32_t use = static_cast<uint32_t>(lt / NACC);
       if (!mbar_wait(&tfull_bar[b], use & 1u, abort_flag, kWhereEpilogue)) break;
@@ -413,6 +582,17 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           uint32_t v[32];
           tc_ld_32x32b_x32(acc + c0, v);
           tc_wait_ld();
+          if (wk.part >= 0) {
+            // stream-K part: the raw fp32 accumulator goes to its workspace unit
+            float4* dst = reinterpret_cast<float4*>(
+                args.sk_ws + (static_cast<size_t>(wk.t - args.sk_full) * args.sk_parts + wk.part) * (256 * BN) +
+                static_cast<size_t>(rank * 128 + q * 32 + lane) * BN + c0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            continue;
+          }
           if constexpr (FP8) {
             // rescale: acc * scale_a[row] * scale_b[column]
             const float sa = ra < args.rows_a ? __ldg(args.scale_a + ra) : 0.0f;
@@ -500,6 +680,48 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc2(tmem_base, Cfg::kTmemCols);
+  }
+}
+
+// Stream-K fixup: every split tile of Y is the sum, in part order, of its
+// parts' fp32 partial tiles (workspace units, [256 rows][BN]), converted as
+// the GEMM epilogue converts (fp32 or bf16 nearest-even; Y[a][b] or, with
+// transpose, Y[b][a]).  A thread takes four consecutive columns of one row
+// (one 16-byte load per part); consecutive threads take consecutive columns
+// (Y[a][b]) or consecutive rows (Y[b][a]), so that the stores coalesce.
+__global__ void __launch_bounds__(256)
+k_sk_fixup(const float* __restrict__ ws, int sk_full, int sk_parts, int tail_tiles, int tiles_m, int BN,
+           int64_t rows_a, int64_t rows_b, void* __restrict__ Y, int64_t ldy, int out_fp32, int transpose) {
+  griddep_launch_dependents();
+  griddep_wait();                                      // the partial tiles of the preceding GEMM
+  const int64_t unit = 256 * static_cast<int64_t>(BN);
+  const int64_t quads = unit / 4;
+  const int64_t total = static_cast<int64_t>(tail_tiles) * quads;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int tl = static_cast<int>(idx / quads);
+    const int e = static_cast<int>(idx - tl * quads);
+    const int t = sk_full + tl;
+    const int64_t a0 = static_cast<int64_t>(t % tiles_m) * 256, b0 = static_cast<int64_t>(t / tiles_m) * BN;
+    const int ra = transpose ? e % 256 : e / (BN / 4);
+    const int cb = 4 * (transpose ? e / 256 : e % (BN / 4));
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int p = 0; p < sk_parts; ++p) {
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(
+          ws + (static_cast<int64_t>(tl) * sk_parts + p) * unit + static_cast<int64_t>(ra) * BN + cb));
+      acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+    }
+    const float v[4] = {acc.x, acc.y, acc.z, acc.w};
+    const int64_t a = a0 + ra;
+    if (a >= rows_a) continue;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t b = b0 + cb + i;
+      if (b >= rows_b) continue;
+      const int64_t off = transpose ? b * ldy + a : a * ldy + b;
+      if (out_fp32) static_cast<float*>(Y)[off] = v[i];
+      else static_cast<__nv_bfloat16*>(Y)[off] = __float2bfloat16_rn(v[i]);
+    }
   }
 }
 

@@ -177,6 +177,16 @@ def test_slide_gemm_sizes_and_validation(L):
     assert L.slide_gemm_workspace_size(ctypes.byref(Wlong), 8) == 8 * 98304 * 2
     W24 = nm.SparseOperand(0x10000, 0x10000, 256, 512, 2, 4, 512)
     assert L.slide_gemm_workspace_size(ctypes.byref(W24), 16) == 0
+    # prefill shapes on SM pairs (whole 256-row weight tiles, >= 64 rows of X):
+    # the lift warps write B from X; from 512 rows on, optional scratch for a
+    # split last round (the sparse product's own bound)
+    for rows_x in (64, 511):
+        assert L.slide_gemm_workspace_size(ctypes.byref(W68), rows_x) == 0
+    for rows_x in (512, 4096):
+        assert L.slide_gemm_workspace_size(ctypes.byref(W68), rows_x) == \
+            L.nm_sparse_gemm_workspace_size(ctypes.byref(W68), rows_x, 1)
+    W200 = nm.SparseOperand(0x10000, 0x10000, 200, 4096, 6, 8, 6144)     # not whole 256-row tiles
+    assert L.slide_gemm_workspace_size(ctypes.byref(W200), 4096) == 4096 * 6144 * 2
     assert L.slide_gemm(ctypes.byref(W68), fake, 16, 4000, fake, 0, null, 0, s) == nm.NM_ERR_INVALID_ARG
     assert L.slide_gemm(ctypes.byref(W68), null, 16, 4096, fake, 0, null, 0, s) == nm.NM_ERR_INVALID_ARG
     assert L.slide_gemm(ctypes.byref(W68), odd, 16, 4096, fake, 0, null, 0, s) == nm.NM_ERR_ALIGNMENT
@@ -295,7 +305,14 @@ def test_misc_entry_points(L):
     from semi_structured_sparse_nm_b200 import _lib as nm
     assert b"sm_100a" in L.nm_version()
     S = nm.SparseOperand(0x10000, 0x10000, 4096, 4096, 8, 16, 7168)
-    assert L.nm_sparse_gemm_workspace_size(ctypes.byref(S), 2048, 0) == 0   # split-K stays in the cluster
+    # SM-pair products: optional scratch for a split last round, at most one
+    # 256 x 256 fp32 tile per SM pair; single-CTA products need none (their
+    # split-K stays in the cluster)
+    bound = L.nm_sparse_gemm_workspace_size(ctypes.byref(S), 2048, 0)
+    assert bound > 0 and bound % (256 * 256 * 4) == 0
+    assert L.nm_sparse_gemm_workspace_size(ctypes.byref(S), 16, 0) == 0
+    S200 = nm.SparseOperand(0x10000, 0x10000, 200, 4096, 8, 16, 7168)
+    assert L.nm_sparse_gemm_workspace_size(ctypes.byref(S200), 2048, 0) == 0
     out = ctypes.c_double(0.0)
     null = ctypes.c_void_p(0)
     assert L.nm_mma_rate_probe(3, 10, ctypes.byref(out), null) == nm.NM_ERR_INVALID_ARG

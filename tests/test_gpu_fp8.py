@@ -31,6 +31,10 @@ def _x(rows, K, kind, seed):
 @pytest.mark.parametrize("rows,K,M,kind", [
     (17, 256, 8, "student_t"), (64, 1024, 8, "outliers"), (5, 512, 16, "zero_rows"), (33, 640, 4, "ties"),
     (9, 2048, 32, "student_t"), (12, 768, 8, "fp32"), (130, 4096, 8, "student_t"),
+    # group counts that leave lanes partly or wholly idle, and more rows than
+    # one pass of the grid (one warp per row, at most eight CTAs per SM)
+    (11, 800, 8, "student_t"), (6, 2112, 16, "ties"), (5, 1152, 32, "outliers"), (70, 528, 4, "student_t"),
+    (10000, 256, 8, "student_t"), (3, 14336, 16, "fp32"),
 ])
 def test_quant_lift_bit_exact(rows, K, M, kind):
     x = _x(rows, K, kind, rows + K)

@@ -69,3 +69,25 @@ def test_host_pipeline_back_to_back_calls_reuse_buffers():
     torch.cuda.synchronize()
     check_close(inputs.bf16_to_f64(host_bits(y1)), oracle.act_sparse_linear(x1, w, 8, 16), "first call")
     check_close(inputs.bf16_to_f64(host_bits(y2)), oracle.act_sparse_linear(x2, w, 8, 16), "second call")
+
+
+def test_host_pipeline_many_chunks():
+    """Sixteen chunks through the two slots: every copy in must land before
+    its prune, and no slot may be overwritten while a copy still reads it."""
+    T, K, O, N, M = 2048, 4096, 1024, 8, 16
+    x = inputs.student_t_bf16((T, K), 4.0, 31)
+    w = inputs.normal_bf16((O, K), 0.02, 32)
+    Wl = nm.lift(dev(w), M)
+    xh = _host(x)
+    yh = torch.empty((T, O), dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        yh.zero_()
+        nm.act_sparse_linear_host(xh, Wl, N, M, yh, chunk_rows=128)
+        torch.cuda.synchronize()
+        assert nm.device_error() == nm.NM_OK
+        ref = []
+        for r0 in range(0, T, 128):                  # the same kernels, chunk by chunk
+            c = nm.prune_compress(dev(x[r0:r0 + 128]), N, M)
+            ref.append(host_bits(nm.sparse_gemm(c, Wl, nm.NM_ACT, torch.bfloat16)))
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(host_bits(yh), np.concatenate(ref))

@@ -113,3 +113,70 @@ def test_consecutive_calls_with_new_activations():
     torch.cuda.synchronize()
     for i in range(4):
         check_close(host_f64(outs[i]), oracle.weight_sparse_linear(xs[i], w, 6, 8), f"call {i}")
+
+
+# ----------------------------------------------- prefill shapes (SM pairs)
+# slide_gemm with at least 64 activation rows and the weight in whole 256-row
+# tiles runs the SM-pair kernel whose lift warps write the lifted B stages
+# from X; the two-call reference runs the same tile variant.
+# (T, K, O, N, M, variant of the reference)
+PAIR_SHAPES = [
+    (4096, 4096, 4096, 6, 8, "auto"),      # the 6:8 prefill workload
+    (600, 1024, 512, 6, 8, "auto"),        # ragged last column tile
+    (1000, 2048, 768, 14, 16, "auto"),
+    (512, 4096, 256, 30, 32, "auto"),
+    (520, 1024, 512, 2, 4, "auto"),        # 2:4: the lift is the identity
+    (200, 1024, 512, 6, 8, "2cta128"),     # 128-wide tiles below 512 rows
+    (64, 960, 256, 6, 8, "2cta128"),       # K' = 1440: a partial last k-block
+    (2048, 16384, 256, 6, 8, "auto"),      # K' >= 16384: the 256-wide tile
+]
+
+
+@pytest.mark.parametrize("T,K,O,N,M,variant", PAIR_SHAPES)
+def test_prefill_equals_the_two_call_path(monkeypatch, T, K, O, N, M, variant):
+    x = inputs.normal_bf16((T, K), 1.0, seed=T + 7 * K)
+    w = inputs.normal_bf16((O, K), 0.02, seed=O + 11)
+    Wc = nm.slide_decompose(dev(w), N, M)
+    xd = dev(x)
+    assert nm.slide_gemm_workspace_size(Wc, T) == (0 if T < 512 else nm.sparse_gemm_workspace_size(Wc, T, nm.NM_WEIGHT))
+    for out_dtype in (torch.bfloat16, torch.float32):
+        y = nm.slide_gemm(Wc, xd, out_dtype)
+        assert ",lift>" in nm.last_gemm_kernel(), nm.last_gemm_kernel()
+        monkeypatch.setenv("NMSPARSE_GEMM", variant)
+        ref = two_call(Wc, xd, out_dtype)
+        monkeypatch.delenv("NMSPARSE_GEMM")
+        torch.cuda.synchronize()
+        assert np.array_equal(host_bits(y), host_bits(ref)), f"{T}x{K}x{O} {N}:{M} {out_dtype}"
+    assert nm.device_error() == nm.NM_OK
+    y = host_f64(y)
+    y_ref = oracle.weight_sparse_linear(x, w, N, M)
+    for r0 in range(0, T, 512):
+        check_close(y[r0:r0 + 512], y_ref[r0:r0 + 512], f"slide prefill {T}x{K}x{O} {N}:{M}, rows {r0}..")
+
+
+def test_prefill_integer_inputs_exact():
+    rng = np.random.default_rng(13)
+    T, K, O = 700, 1024, 768
+    x = inputs.bf16_from_f64(rng.integers(-8, 9, size=(T, K)).astype(np.float64))
+    w = inputs.bf16_from_f64(rng.integers(-8, 9, size=(O, K)).astype(np.float64))
+    for N, M in ((6, 8), (14, 16)):
+        Wc = nm.slide_decompose(dev(w), N, M)
+        y = nm.slide_gemm(Wc, dev(x), torch.float32)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(host_f64(y), oracle.weight_sparse_linear(x, w, N, M))
+
+
+def test_prefill_strided_activation_rows():
+    """X as a column slice of a wider tensor (row stride K + 64) on the
+    SM-pair path."""
+    T, K, O = 640, 2048, 512
+    big = inputs.normal_bf16((T, K + 64), 1.0, seed=15)
+    w = inputs.normal_bf16((O, K), 0.02, seed=16)
+    Wc = nm.slide_decompose(dev(w), 6, 8)
+    xd = dev(big)[:, 32:32 + K]
+    y = nm.slide_gemm(Wc, xd, torch.float32)
+    ref = two_call(Wc, xd.contiguous(), torch.float32)
+    torch.cuda.synchronize()
+    assert np.array_equal(host_bits(y), host_bits(ref))
+    check_close(host_f64(y), oracle.weight_sparse_linear(np.ascontiguousarray(big[:, 32:32 + K]), w, 6, 8),
+                "strided prefill")

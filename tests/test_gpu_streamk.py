@@ -1,0 +1,73 @@
+"""The split last round of the SM-pair GEMM (stream-K tail): with the
+workspace nm_sparse_gemm_workspace_size() reports, a last persistent round
+that would leave most SM pairs idle is split along K across them and a second
+kernel adds the parts.  Exact on integer inputs (any summation order is exact
+there), equal to the unsplit schedule on them, within tolerance of the oracle
+on random data, deterministic from call to call."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from semi_structured_sparse_nm_b200 import _lib as nm
+from semi_structured_sparse_nm_b200 import inputs
+from tests.gpu_util import check_close, dev, host_bits, host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _int_bf16(rng, shape, lo=-4, hi=5):
+    return inputs.bf16_from_f64(rng.integers(lo, hi, size=shape).astype(np.float64))
+
+
+# (rows of the sparse operand, rows of the dense one, K, N, M, side): tile
+# counts a little above one round of 74 SM pairs, so that a short last round
+# is split; the weight side stores Y transposed
+SHAPES = [
+    (2560, 1792, 2048, 2, 4, "act"),        # 10 x 8 tiles of 256 x 224
+    (2560, 1800, 1024, 8, 16, "act"),       # a partial last column tile
+    (4096, 4096, 1024, 6, 8, "weight"),     # the 6:8 prefill tile count (16 x 19)
+]
+
+
+@pytest.mark.parametrize("ra,rb,K,N,M,side", SHAPES)
+def test_split_round_exact_on_integers(ra, rb, K, N, M, side):
+    rng = np.random.default_rng(ra + rb + K)
+    a = _int_bf16(rng, (ra, K))
+    b = _int_bf16(rng, (rb, K), -3, 4)
+    S = nm.prune_compress(dev(a), N, M)
+    D = nm.lift(dev(b), M)
+    sd = nm.NM_ACT if side == "act" else nm.NM_WEIGHT
+    y = nm.sparse_gemm(S, D, sd, torch.float32)
+    kname = nm.last_gemm_kernel()
+    assert "+split" in kname, kname
+    y_plain = torch.empty_like(y)
+    st = S.struct()
+    import ctypes
+    nm._check("nm_sparse_gemm", nm.lib().nm_sparse_gemm(ctypes.byref(st), nm._p(D), rb, sd, nm._p(y_plain),
+                                                          nm.NM_FP32, None, 0, nm._stream(D)))
+    assert "+split" not in nm.last_gemm_kernel()
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    ref = oracle.act_sparse_linear(a, b, N, M) if side == "act" else oracle.act_sparse_linear(a, b, N, M).T
+    np.testing.assert_array_equal(host_f64(y), ref)
+    np.testing.assert_array_equal(host_f64(y_plain), ref)
+
+
+@pytest.mark.parametrize("ra,rb,K,N,M,side", SHAPES)
+def test_split_round_random_within_tolerance_and_deterministic(ra, rb, K, N, M, side):
+    a = inputs.student_t_bf16((ra, K), 4.0, seed=ra)
+    b = inputs.normal_bf16((rb, K), 0.02, seed=rb)
+    S = nm.prune_compress(dev(a), N, M)
+    D = nm.lift(dev(b), M)
+    sd = nm.NM_ACT if side == "act" else nm.NM_WEIGHT
+    y1 = nm.sparse_gemm(S, D, sd, torch.bfloat16)
+    y2 = nm.sparse_gemm(S, D, sd, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    ref = oracle.act_sparse_linear(a, b, N, M)
+    y = host_f64(y1)
+    if side == "weight":
+        y = y.T
+    for r0 in range(0, ra, 512):
+        check_close(y[r0:r0 + 512], ref[r0:r0 + 512], f"split round {ra}x{rb}x{K}, rows {r0}..")
