@@ -449,10 +449,12 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   // Split last round (stream-K tail): when the tiles leave a last persistent
   // round in which fewer than half the SM pairs would work, and the caller
   // gave scratch, each of that round's L tiles is split along K into
-  // clusters / L parts (at least two k-blocks each) run by otherwise idle
-  // pairs; k_sk_fixup adds the parts in order.  Plain bf16/fp32 outputs of
-  // pure 2:4 products only (no dense k-blocks, output split or epilogue
-  // scaling).
+  // clusters / L parts, run by otherwise idle pairs; k_sk_fixup adds the
+  // parts in order.  A part keeps at least 16 k-blocks: the partial tiles
+  // cost a write and a read of 256 x BN fp32 each, which a shorter part does
+  // not pay back (measured on B200: 6:8 prefill, 48 k-blocks in 9 parts,
+  // 10 us of fixup for 3 us saved).  Plain bf16/fp32 outputs of pure 2:4
+  // products only (no dense k-blocks, output split or epilogue scaling).
   a.sk_full = tiles;
   a.sk_parts = 0;
   a.sk_ws = nullptr;
@@ -460,7 +462,7 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
       p.row_scale == nullptr && p.row_shift == nullptr) {
     const int R = tiles / clusters, L = tiles - R * clusters;
     if (R >= 1 && L > 0) {
-      const int parts = std::min(clusters / L, static_cast<int>(kb / 2));
+      const int parts = std::min(clusters / L, static_cast<int>(kb / 16));
       const size_t need = static_cast<size_t>(L) * parts * 256 * BN * 4;
       if (parts >= 2 && p.ws_bytes >= need) {
         a.sk_full = R * clusters;

@@ -705,11 +705,18 @@ k_sk_fixup(const float* __restrict__ ws, int sk_full, int sk_parts, int tail_til
     const int64_t a0 = static_cast<int64_t>(t % tiles_m) * 256, b0 = static_cast<int64_t>(t / tiles_m) * BN;
     const int ra = transpose ? e % 256 : e / (BN / 4);
     const int cb = 4 * (transpose ? e / 256 : e % (BN / 4));
+    // all of a group of up to eight parts' loads in flight before the adds
+    // (still added in part order)
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int p = 0; p < sk_parts; ++p) {
-      const float4 x = __ldcg(reinterpret_cast<const float4*>(
-          ws + (static_cast<int64_t>(tl) * sk_parts + p) * unit + static_cast<int64_t>(ra) * BN + cb));
-      acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+    const float* u0 = ws + static_cast<int64_t>(tl) * sk_parts * unit + static_cast<int64_t>(ra) * BN + cb;
+    for (int p0 = 0; p0 < sk_parts; p0 += 8) {
+      float4 x[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (p0 + i < sk_parts) x[i] = __ldcg(reinterpret_cast<const float4*>(u0 + (p0 + i) * unit));
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (p0 + i < sk_parts) { acc.x += x[i].x; acc.y += x[i].y; acc.z += x[i].z; acc.w += x[i].w; }
     }
     const float v[4] = {acc.x, acc.y, acc.z, acc.w};
     const int64_t a = a0 + ra;

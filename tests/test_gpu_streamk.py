@@ -23,10 +23,11 @@ def _int_bf16(rng, shape, lo=-4, hi=5):
 # (rows of the sparse operand, rows of the dense one, K, N, M, side): tile
 # counts a little above one round of 74 SM pairs, so that a short last round
 # is split; the weight side stores Y transposed
+# (each part keeps at least 16 k-blocks of 128 lifted K)
 SHAPES = [
-    (2560, 1792, 2048, 2, 4, "act"),        # 10 x 8 tiles of 256 x 224
-    (2560, 1800, 1024, 8, 16, "act"),       # a partial last column tile
-    (4096, 4096, 1024, 6, 8, "weight"),     # the 6:8 prefill tile count (16 x 19)
+    (2560, 1792, 4096, 2, 4, "act"),        # 10 x 8 tiles of 256 x 224, 2 parts
+    (2560, 1800, 4096, 8, 16, "act"),       # a partial last column tile, 3 parts
+    (4096, 4096, 4096, 6, 8, "weight"),     # the 6:8 prefill workload's tiles (16 x 19), 3 parts
 ]
 
 
