@@ -107,6 +107,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// The same wait for a whole warp: lane 0 polls (the other lanes sit at the
+// warp barrier instead of polling the mbarrier too), then every lane
+// acquires the completed phase itself with one more test -- which succeeds:
+// the barrier cannot complete a further phase before this warp has done its
+// part.  All 32 lanes must call it.
+template <bool CLUSTER = false>
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                               unsigned where,
+                                               unsigned long long limit_ns = kWaitLimitNs) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait<CLUSTER>(bar, parity, abort, where, limit_ns);
+  ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+  if (ok) ok = mbar_wait<CLUSTER>(bar, parity, abort, where, limit_ns);
+  return ok;
+}
+
 // ------------------------------------------- programmatic dependent launch
 // A kernel launched with programmatic stream serialisation may start before
 // the preceding kernel in the stream has finished; griddep_wait() blocks

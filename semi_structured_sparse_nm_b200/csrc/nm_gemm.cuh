@@ -502,7 +502,7 @@ k_nm_gemm(const __grid_constant__ CUtensorMap tmA_s, const __grid_constant__ CUt
     if constexpr (lift) {
       lift_panel<BN>(args, tmB, kb_begin, kb_end, smem + args.lift_raw_off, sP, xraw_bar, panel_bar, abort_flag);
     }
-    const bool ok = mbar_wait(accum_bar, 0u, abort_flag, kWhereEpilogue);
+    const bool ok = mbar_wait_warp(accum_bar, 0u, abort_flag, kWhereEpilogue);
     griddep_wait();                                  // Y may still be in use upstream
     tc_fence_after();
     if (push) {

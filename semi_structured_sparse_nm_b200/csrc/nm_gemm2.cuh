@@ -570,7 +570,7 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const int tm = wk.tl.out, tn = wk.t / args.tiles_m;
       const int b = lt % NACC;
       const uint32_t use = static_cast<uint32_t>(lt / NACC);
-      if (!mbar_wait(&tfull_bar[b], use & 1u, abort_flag, kWhereEpilogue)) break;
+      if (!mbar_wait_warp(&tfull_bar[b], use & 1u, abort_flag, kWhereEpilogue)) break;
       tc_fence_after();
 #pragma unroll 1
       for (int u = 0; u < MSUB; ++u) {
