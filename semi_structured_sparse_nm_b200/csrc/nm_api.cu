@@ -461,7 +461,10 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   if (p.ws != nullptr && aligned16(p.ws) && MSUB == 1 && !FP8 && p.out_split_rows < 0 && p.kd == 0 &&
       p.row_scale == nullptr && p.row_shift == nullptr) {
     const int R = tiles / clusters, L = tiles - R * clusters;
-    if (R >= 1 && L > 0) {
+    // a last round made only of the last, partial column of tiles is short
+    // already (its tiles carry fewer rows of B): no split
+    const bool tail_partial = (p.rows_b % BN) != 0 && (tiles - L) / a.tiles_m == a.tiles_n - 1;
+    if (R >= 1 && L > 0 && !tail_partial) {
       const int parts = std::min(clusters / L, static_cast<int>(kb / 16));
       const size_t need = static_cast<size_t>(L) * parts * 256 * BN * 4;
       if (parts >= 2 && p.ws_bytes >= need) {

@@ -27,8 +27,20 @@ def _int_bf16(rng, shape, lo=-4, hi=5):
 SHAPES = [
     (2560, 1792, 4096, 2, 4, "act"),        # 10 x 8 tiles of 256 x 224, 2 parts
     (2560, 1800, 4096, 8, 16, "act"),       # a partial last column tile, 3 parts
-    (4096, 4096, 4096, 6, 8, "weight"),     # the 6:8 prefill workload's tiles (16 x 19), 3 parts
+    (4096, 4480, 4096, 6, 8, "weight"),     # 16 x 20 tiles of 256 x 224 (whole columns), 3 parts
 ]
+
+
+def test_no_split_when_the_last_round_is_the_partial_last_column():
+    """The 6:8 prefill workload's tiles (16 x 19 of 256 x 224, 4096 rows of X):
+    the eight tiles of the last round are the last column, which holds 64 of
+    224 rows, so the round is short already and runs whole."""
+    w = inputs.normal_bf16((4096, 4096), 0.02, seed=1)
+    x = inputs.normal_bf16((4096, 4096), 1.0, seed=2)
+    Wc = nm.slide_decompose(dev(w), 6, 8)
+    nm.sparse_gemm(Wc, nm.lift(dev(x), 8), nm.NM_WEIGHT, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert nm.last_gemm_kernel() == "k_nm_gemm_2cta<224,2,1>", nm.last_gemm_kernel()
 
 
 @pytest.mark.parametrize("ra,rb,K,N,M,side", SHAPES)
