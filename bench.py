@@ -515,6 +515,13 @@ class Workload:
         return dense, mma, byts
 
 
+def _count_fixup(wk):
+    """A GEMM whose last round was split launches the fixup kernel too."""
+    if "+split" in (wk.kernel_name or "") and not getattr(wk, "fixup_counted", False):
+        wk.launches_per_step += 1
+        wk.fixup_counted = True
+
+
 def time_workload(wk, steps, warmup, stream, clock=None):
     """Returns (ms per step, ms per prep kernel, ms per GEMM launch)."""
     import torch
@@ -551,6 +558,7 @@ def time_workload(wk, steps, warmup, stream, clock=None):
         gemm_ms = e0.elapsed_time(e1) / steps
         prep_ms = max(step_ms - gemm_ms, 0.0)
         wk.kernel_name = wk.nm.last_gemm_kernel()
+        _count_fixup(wk)
         del g, gg
         return step_ms, prep_ms, gemm_ms
     # the step as a user runs it: K steps back to back, events only around them
@@ -565,6 +573,7 @@ def time_workload(wk, steps, warmup, stream, clock=None):
         torch.cuda.synchronize()
     step_ms = t0.elapsed_time(t1) / steps
     wk.kernel_name = wk.nm.last_gemm_kernel()
+    _count_fixup(wk)
     # the same K steps again with an event around each kernel: per-kernel times
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
     torch.cuda.synchronize()

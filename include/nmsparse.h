@@ -439,7 +439,9 @@ int hybrid_gemm_noalloc(const void *X, int64_t B, const nm_hybrid_weight *W, voi
  * y_host[T][O] = prune_{N:M}(x_host) . W^T, x_host bf16 [T][K] and y_host bf16
  * [T][O] in HOST memory (row-major, row strides K and O), w_lift the
  * device-resident lifted weight [O][K'] (nm_lift()).  The rows go through in
- * chunks of chunk_rows (a multiple of 128; 0 = 256): each chunk is copied in
+ * chunks of chunk_rows (a multiple of 128; 0 = 256 rows, or a multiple of 256
+ * large enough that a chunk's product occupies at least half the SM pairs:
+ * 512 for O = 4096 on 148 SMs): each chunk is copied in
  * on one auxiliary stream, pruned and multiplied on `stream`, and copied out
  * on another, with two buffer slots, so that the copy in of the next chunk
  * and the copy out of the previous one overlap the math of the current one

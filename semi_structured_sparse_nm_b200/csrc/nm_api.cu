@@ -1461,7 +1461,17 @@ int host_pipe(HostPipe** out) {
   return NM_OK;
 }
 
-constexpr int64_t kHostChunkRows = 256;
+// Default chunk of the host-buffer pipeline: 256 rows, or more when the
+// chunk's product would otherwise leave more than half the SM pairs idle
+// (256-row tiles x 224-wide columns), so that the math of a chunk stays well
+// below the time of its copy in.
+int64_t host_chunk_rows(int64_t T, int64_t O, int64_t chunk_rows) {
+  if (chunk_rows > 0) return std::min(T, chunk_rows);
+  const int64_t pairs = std::max(1, num_sms() / 2);
+  const int64_t col_tiles = ceil_div(O, int64_t(224));
+  const int64_t m_tiles = std::max<int64_t>(1, ceil_div(pairs, 2 * col_tiles));
+  return std::min(T, 256 * m_tiles);
+}
 
 int64_t round256(int64_t b) { return ceil_div(b, int64_t(256)) * 256; }
 
@@ -1478,7 +1488,7 @@ extern "C" {
 size_t nm_act_sparse_linear_host_workspace_size(int64_t T, int64_t K, int N, int M, int64_t O, int64_t chunk_rows) {
   (void)N;
   if (T <= 0 || K <= 0 || O <= 0 || nm_lifted_k(K, M) < 0) return 0;
-  const int64_t Tc = std::min(T, chunk_rows > 0 ? chunk_rows : kHostChunkRows);
+  const int64_t Tc = host_chunk_rows(T, O, chunk_rows);
   return static_cast<size_t>(2 * host_slot_bytes(Tc, K, M, O));
 }
 
@@ -1486,7 +1496,7 @@ int nm_act_sparse_linear_host(const void* x_host, int64_t T, int64_t K, int N, i
                               void* y_host, int64_t chunk_rows, void* ws, size_t ws_bytes, void* stream) {
   if (T < 0 || K <= 0 || O <= 0 || chunk_rows < 0) return NM_ERR_INVALID_ARG;
   if (chunk_rows % 128 != 0) return NM_ERR_INVALID_ARG;
-  const int64_t Tc = std::min(T, chunk_rows > 0 ? chunk_rows : kHostChunkRows);
+  const int64_t Tc = host_chunk_rows(T, O, chunk_rows);
   // the pattern and shapes are validated before anything is enqueued (the
   // placeholder address stands for the chunk buffers, which are never read here)
   void* const placeholder = reinterpret_cast<void*>(uintptr_t(256));

@@ -28,8 +28,11 @@ def test_host_pipeline_matches_device_calls(chunk, T, K, O, N, M):
     nm.act_sparse_linear_host(xh, Wl, N, M, yh, chunk_rows=chunk)
     torch.cuda.synchronize()
     assert nm.device_error() == nm.NM_OK
-    # the same kernels, called chunk by chunk on device buffers
-    Tc = chunk or 256
+    # the same kernels, called chunk by chunk on device buffers; the default
+    # chunk is 256 rows, or more when a chunk's product would leave more than
+    # half the SM pairs idle
+    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    Tc = chunk or min(T, 256 * max(1, -(-pairs // (2 * -(-O // 224)))))
     ref = []
     for r0 in range(0, T, Tc):
         c = nm.prune_compress(dev(x[r0:r0 + Tc]), N, M)

@@ -129,6 +129,7 @@ PAIR_SHAPES = [
     (200, 1024, 512, 6, 8, "2cta128"),     # 128-wide tiles below 512 rows
     (64, 960, 256, 6, 8, "2cta128"),       # K' = 1440: a partial last k-block
     (2048, 16384, 256, 6, 8, "auto"),      # K' >= 16384: the 256-wide tile
+    (1792, 4096, 2560, 6, 8, "auto"),      # 10 x 8 tiles: the last round split in 3 (lift warps and parts)
 ]
 
 
@@ -142,6 +143,8 @@ def test_prefill_equals_the_two_call_path(monkeypatch, T, K, O, N, M, variant):
     for out_dtype in (torch.bfloat16, torch.float32):
         y = nm.slide_gemm(Wc, xd, out_dtype)
         assert ",lift>" in nm.last_gemm_kernel(), nm.last_gemm_kernel()
+        if (T, O) == (1792, 2560):
+            assert nm.last_gemm_kernel().endswith("+split3"), nm.last_gemm_kernel()
         monkeypatch.setenv("NMSPARSE_GEMM", variant)
         ref = two_call(Wc, xd, out_dtype)
         monkeypatch.delenv("NMSPARSE_GEMM")
