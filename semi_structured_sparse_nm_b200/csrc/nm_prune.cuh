@@ -190,14 +190,17 @@ __device__ __forceinline__ uint32_t compress_group(const GroupRaw<M, T>& raw, in
   return keep;
 }
 
-// Window table: for each 4-bit set c of still-unplaced kept positions of a
-// window (local positions 0..3), .x = byte-permute selectors (bits 0-15 pick
-// the two kept values out of the window's four, bits 16-31 then zero the
-// padded slot), .y = index pair (bits 0-3) | placed positions 2,3 (bits 4-5,
-// carried into the next window as its positions 0,1).  The window takes the
-// lowest two positions of c; one entry at a is paired with the lowest other
-// index (value +0.0), none gives (0, 1).
-__device__ __forceinline__ uint2 window_entry(uint32_t c) {
+// Window tables, indexed by the 4-bit set c of still-unplaced kept positions
+// of a window (local positions 0..3).  The window takes the lowest two
+// positions of c; one entry at a is paired with the lowest other index (its
+// slot holds +0.0), none gives (0, 1) with both slots +0.0.
+//   wt[c]      = {byte-permute selector picking the two values out of the
+//                 window's four (bits 0-15), AND mask zeroing padded slots}
+//   wt[16 + c] = {allowed mask of the next window, scaled by 8 (bits 3-6:
+//                 its positions 0,1 unless this window placed them as its
+//                 positions 2,3; positions 2,3 always), index pair i0 | i1 << 2}
+// A table row is 8 bytes, so that c * 8 is the row's byte offset.
+__device__ __forceinline__ void window_rows(uint32_t c, uint2* row_val, uint2* row_next) {
   const uint32_t f = c & (0u - c);
   const uint32_t rest = c ^ f;
   const uint32_t sb = rest & (0u - rest);
@@ -210,8 +213,10 @@ __device__ __forceinline__ uint2 window_entry(uint32_t c) {
     if (a == 0) { z0 = false; } else { i1 = a; z1 = false; }
   }
   const uint32_t sel = static_cast<uint32_t>((0x10 + 0x22 * i0) | ((0x10 + 0x22 * i1) << 8));
-  const uint32_t zsel = (z0 ? 0x54u : 0x10u) | ((z1 ? 0x76u : 0x32u) << 8);   // bytes 4..7 of 0 are zero
-  return make_uint2(sel | (zsel << 16), static_cast<uint32_t>(i0 | (i1 << 2)) | ((taken >> 2) << 4));
+  const uint32_t zmask = (z0 ? 0u : 0x0000FFFFu) | (z1 ? 0u : 0xFFFF0000u);
+  const uint32_t allowed = ((~(taken >> 2)) & 0x3u) | 0xCu;
+  *row_val = make_uint2(sel, zmask);
+  *row_next = make_uint2(allowed << 3, static_cast<uint32_t>(i0 | (i1 << 2)));
 }
 
 // Two 16-bit lanes per 32-bit word: one instruction does two comparators.
@@ -297,7 +302,7 @@ __device__ __forceinline__ uint32_t ukey_bf16(const uint32_t (&P)[M / 2], int i)
 }
 
 template <int M>
-__device__ __forceinline__ uint32_t compress_group_bf16(const uint32_t (&P)[M / 2], int N, const uint2* lut,
+__device__ __forceinline__ uint32_t compress_group_bf16(const uint32_t (&P)[M / 2], int N, const uint2* wt,
                                                         uint32_t* val_out, uint8_t* nib_out) {
   constexpr int NW = M / 2 - 1;
   uint32_t keep = 0u;
@@ -315,15 +320,20 @@ __device__ __forceinline__ uint32_t compress_group_bf16(const uint32_t (&P)[M / 
 #pragma unroll
     for (int i = 0; i < M; ++i) keep |= ((t1 - ukey_bf16<M>(P, i)) >> 31) << i;
   }
-  uint32_t carry = 0u;
+  // Windows left to right: the row offset of window w is its four keep bits,
+  // scaled by 8, masked by what window w - 1 allows (the chain is one AND and
+  // one table read per window).
+  const char* tv = reinterpret_cast<const char*>(wt);
+  uint32_t allowed8 = 0x78u;
 #pragma unroll
   for (int w = 0; w < NW; ++w) {
-    const uint32_t c = ((keep >> (2 * w)) & 0xFu) & ~carry;
-    const uint2 e = lut[c];
-    const uint32_t v = __byte_perm(P[w], P[w + 1], e.x & 0xFFFFu);
-    val_out[w] = __byte_perm(v, 0u, e.x >> 16);
-    nib_out[w] = static_cast<uint8_t>(e.y & 0xFu);
-    carry = (e.y >> 4) & 0x3u;
+    const uint32_t k8 = (w == 0) ? (keep << 3) : (w == 1) ? (keep << 1) : (keep >> (2 * w - 3));
+    const uint32_t off = k8 & allowed8 & 0x78u;
+    const uint2 ev = *reinterpret_cast<const uint2*>(tv + off);
+    const uint2 en = *reinterpret_cast<const uint2*>(tv + 128 + off);
+    val_out[w] = __byte_perm(P[w], P[w + 1], ev.x) & ev.y;
+    nib_out[w] = static_cast<uint8_t>(en.y);
+    allowed8 = en.x;
   }
   return keep;
 }
@@ -365,8 +375,10 @@ __device__ __forceinline__ void load_lane(const T* __restrict__ p, int64_t nvali
 // over windows (window w takes the lowest two not yet placed kept entries of
 // positions 2w..2w+3; one entry is paired with the lowest other local index,
 // none gives (0, 1); padded slots hold +0.0), values written through a
-// staging row as 16-byte stores.  Rows past `rows` (up to the 128-row padding
-// of the image) and windows past K'/4 get the index pair (0, 1).
+// shared-memory staging row that leaves as one bulk copy (two staging rows
+// per warp, so a copy reads while the other row is formed).  Rows past `rows`
+// (up to the 128-row padding of the image) and windows past K'/4 get the
+// index pair (0, 1).
 //
 // The grid is persistent: CTA b takes tasks b, b + gridDim.x, ... (row-group
 // major), stepped without divisions.  Each warp keeps the two rows it works
@@ -376,9 +388,10 @@ __device__ __forceinline__ void load_lane(const T* __restrict__ p, int64_t nvali
 constexpr int kPruneWarps = 8;
 
 // Resident CTAs per SM the register budget is sized for: bf16 groups of up to
-// 16 run four CTAs per SM; M = 32 (and fp32) CTAs are larger.
+// 16 run four CTAs per SM, M = 32 three (80 registers; measured faster than
+// two CTAs of 123 registers, and than four with spills); fp32 CTAs are larger.
 __host__ __device__ constexpr int prune_min_blocks(int M, int elem_bytes) {
-  return elem_bytes != 2 ? 1 : (M >= 32 ? 2 : 4);
+  return elem_bytes != 2 ? 1 : (M >= 32 ? 3 : 4);
 }
 
 // Task geometry: chunks per row group, ceil(groups / (32 G)), and the task
@@ -413,13 +426,16 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
   constexpr int NWL = G * NW;                     // windows per lane
   constexpr int WIN = 32 * NWL;                   // windows per task row = NWL blocks
   constexpr int LM = G * M;                       // elements (keep bits) per lane
+  // staged rows of 768 bytes and more leave as bulk copies; shorter ones (2:4)
+  // were measured faster as 16-byte stores by the lanes
+  constexpr bool kBulkRow = WIN * (Q8 ? 2 : 4) >= 768;
   __shared__ __align__(16) uint8_t s_nib[16][WIN];
-  __shared__ __align__(16) uint32_t s_val[kPruneWarps][WIN];
+  __shared__ __align__(16) uint32_t s_val[kPruneWarps][kBulkRow ? 2 : 1][WIN];   // row k of the warp, staged
   __shared__ uint32_t s_mask[kPruneWarps][LM];
-  __shared__ uint2 s_lut[16];
+  __shared__ __align__(16) uint2 s_wt[32];
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   griddep_launch_dependents();
-  if (threadIdx.x < 16) s_lut[threadIdx.x] = window_entry(threadIdx.x);
+  if (threadIdx.x < 16) window_rows(threadIdx.x, &s_wt[threadIdx.x], &s_wt[16 + threadIdx.x]);
   griddep_wait();                                      // inputs / outputs of the preceding kernel
   const int64_t groups = K / M;
   const int64_t mask_words = (K + 31) / 32;
@@ -441,7 +457,7 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
     load_row(rg, ch, 0);
     load_row(rg, ch, 1);
   }
-  __syncthreads();                                     // s_lut
+  __syncthreads();                                     // s_wt
   while (task < pg.tasks) {
     const uint32_t next = task + gridDim.x;
     uint32_t rg_n = rg + drg, ch_n = ch + dch;
@@ -461,6 +477,10 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
       const int it = 2 * warp + k;
       const int64_t r = r0 + it;
       if (r < rows) {
+        // the bulk store that last read this staging row (one task ago) is done reading
+        if constexpr (kBulkRow) {
+          if (lane == 0) bulk_wait_read1();
+        }
         if (lane < LM) s_mask[warp][lane] = 0u;
         __syncwarp();
         float inv = 1.0f;
@@ -495,7 +515,7 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
               for (int p = 0; p < M / 2; ++p) P[p] = PL[j * (M / 2) + p];
               uint32_t vj[NW];
               uint8_t nj[NW];
-              const uint32_t kj = compress_group_bf16<M>(P, N, s_lut, vj, nj);
+              const uint32_t kj = compress_group_bf16<M>(P, N, s_wt, vj, nj);
               const bool valid = (G == 1) || (gl + j < groups);
 #pragma unroll
               for (int w = 0; w < NW; ++w) { vals[j * NW + w] = vj[w]; nibs[j * NW + w] = valid ? nj[w] : 0x4; }
@@ -521,11 +541,11 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
 #pragma unroll
           for (int w = 0; w < NWL; ++w) {
             if constexpr (Q8) {
-              reinterpret_cast<uint16_t*>(&s_val[warp][0])[lane * NWL + w] = static_cast<uint16_t>(
+              reinterpret_cast<uint16_t*>(&s_val[warp][kBulkRow ? k : 0][0])[lane * NWL + w] = static_cast<uint16_t>(
                   e4m3x2(__fmul_rn(elem_f32(static_cast<uint16_t>(vals[w] & 0xFFFFu)), inv),
                          __fmul_rn(elem_f32(static_cast<uint16_t>(vals[w] >> 16)), inv)));
             } else {
-              s_val[warp][lane * NWL + w] = vals[w];
+              s_val[warp][kBulkRow ? k : 0][lane * NWL + w] = vals[w];
             }
             s_nib[it][lane * NWL + w] = nibs[w];
           }
@@ -535,11 +555,18 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
         }
         // raw[k] is consumed: request this warp's row k of the next task
         if (has_next) load_row(rg_n, ch_n, k);
+        // A whole task row (16-byte aligned start and size) leaves as one
+        // bulk copy issued by lane 0 (or as 16-byte stores when short); a
+        // partial one is copied element by element.
+        const bool bulk = kBulkRow && vec_vals && ng == 32 * G;
+        if (bulk) fence_proxy_async_smem();            // this lane's staging stores -> the copy engine
         __syncwarp();
         if constexpr (Q8) {
           uint16_t* vrow = static_cast<uint16_t*>(vals_out) + r * (Kl / 4) + g0 * NW;
-          const uint16_t* sv16 = reinterpret_cast<const uint16_t*>(&s_val[warp][0]);
-          if (vec_vals && ng == 32 * G) {
+          const uint16_t* sv16 = reinterpret_cast<const uint16_t*>(&s_val[warp][kBulkRow ? k : 0][0]);
+          if (bulk) {
+            if (lane == 0) bulk_store(vrow, sv16, WIN * 2);
+          } else if (vec_vals && ng == 32 * G) {
             const uint4* sv = reinterpret_cast<const uint4*>(sv16);
             uint4* dv = reinterpret_cast<uint4*>(vrow);
             for (int i = lane; i < WIN / 8; i += 32) dv[i] = sv[i];
@@ -548,12 +575,14 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
           }
         } else {
           uint32_t* vrow = static_cast<uint32_t*>(vals_out) + r * (Kl / 4) + g0 * NW;
-          if (vec_vals && ng == 32 * G) {
-            const uint4* sv = reinterpret_cast<const uint4*>(&s_val[warp][0]);
+          if (bulk) {
+            if (lane == 0) bulk_store(vrow, &s_val[warp][kBulkRow ? k : 0][0], WIN * 4);
+          } else if (vec_vals && ng == 32 * G) {
+            const uint4* sv = reinterpret_cast<const uint4*>(&s_val[warp][kBulkRow ? k : 0][0]);
             uint4* dv = reinterpret_cast<uint4*>(vrow);
             for (int i = lane; i < WIN / 4; i += 32) dv[i] = sv[i];
           } else {
-            for (int i = lane; i < ng * NW; i += 32) vrow[i] = s_val[warp][i];
+            for (int i = lane; i < ng * NW; i += 32) vrow[i] = s_val[warp][kBulkRow ? k : 0][i];
           }
         }
         if (mask_out != nullptr && lane < LM) {
@@ -572,6 +601,11 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
         __syncwarp();
       } else if (has_next) {
         load_row(rg_n, ch_n, k);
+      }
+      // one bulk group per (task, row k), empty or not, so that a wait for
+      // all but the newest group always covers this staging row's last copy
+      if constexpr (kBulkRow) {
+        if (lane == 0) bulk_commit();
       }
     }
     __syncthreads();
@@ -619,6 +653,9 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
     task = next;
     rg = rg_n;
     ch = ch_n;
+  }
+  if constexpr (kBulkRow) {
+    if (lane == 0) bulk_wait_all();                    // the staging rows stay until the copies are done
   }
 }
 
