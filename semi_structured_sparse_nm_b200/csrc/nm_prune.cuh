@@ -429,7 +429,10 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
   // staged rows of 768 bytes and more leave as bulk copies; shorter ones (2:4)
   // were measured faster as 16-byte stores by the lanes
   constexpr bool kBulkRow = WIN * (Q8 ? 2 : 4) >= 768;
-  __shared__ __align__(16) uint8_t s_nib[16][WIN];
+  // index pairs of the task's 16 rows; two buffers (alternate tasks), so one
+  // barrier per task separates a task's rows from its metadata pass, and the
+  // next barrier separates that pass from the rewrite two tasks later
+  __shared__ __align__(16) uint8_t s_nib_buf[2][16][WIN];
   __shared__ __align__(16) uint32_t s_val[kPruneWarps][kBulkRow ? 2 : 1][WIN];   // row k of the warp, staged
   __shared__ uint32_t s_mask[kPruneWarps][LM];
   __shared__ __align__(16) uint2 s_wt[32];
@@ -458,7 +461,9 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
     load_row(rg, ch, 1);
   }
   __syncthreads();                                     // s_wt
+  uint32_t tb = 0;                                     // s_nib buffer of this task
   while (task < pg.tasks) {
+    uint8_t (*s_nib)[WIN] = s_nib_buf[tb];
     const uint32_t next = task + gridDim.x;
     uint32_t rg_n = rg + drg, ch_n = ch + dch;
     if (ch_n >= cpr) { ch_n -= cpr; ++rg_n; }
@@ -649,8 +654,8 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
             make_uint4(wds[0], wds[1], wds[2], wds[3]);
       }
     }
-    __syncthreads();                                   // s_nib is rewritten by the next task
     task = next;
+    tb ^= 1u;
     rg = rg_n;
     ch = ch_n;
   }
