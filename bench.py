@@ -898,6 +898,18 @@ def run_gpu(args):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    # the host link's own rate for context: a plain pinned copy of the same X
+    # into device memory (the end-to-end step cannot beat its copy in)
+    xd_probe = torch.empty(tuple(xh.shape), dtype=xh.dtype, device=dev)
+    xd_probe.copy_(xh, non_blocking=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(3):
+        xd_probe.copy_(xh, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    h2d_gbs = xh.numel() * xh.element_size() * 3 / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    del xd_probe
     dense, _, _ = wk.algorithmic()
 
     rf = main["roofline"]
@@ -922,7 +934,8 @@ def run_gpu(args):
         "e2e": {"value": sig(ws * dense / (e2e_ms * 1e-3) / 1e12), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": int(xh.numel() * xh.element_size()),
                 "d2h_bytes_per_step": int(yh.numel() * yh.element_size()),
-                "path": "nm_act_sparse_linear_host" if pipelined else "copy in, step, copy out"},
+                "path": "nm_act_sparse_linear_host" if pipelined else "copy in, step, copy out",
+                "h2d_copy_GBps": sig(h2d_gbs)},
         "gpu_launches": wk.launches_per_step * args.steps,
         "clocks": clk.summary(),
         "device_status": status,

@@ -58,6 +58,21 @@ def test_prune_compress_bit_exact(rows, K, N, M, dist):
     _check_operand(x, N, M, comp)
 
 
+@pytest.mark.parametrize("rows,K,N,M,dist", [
+    # several tasks per CTA (persistent grid), a ragged last row group, and a
+    # last chunk of each row group that holds 2 of 32 groups, so that whole
+    # and partial task rows (bulk-copied and element-copied values) alternate
+    # in one CTA's sequence of tasks
+    (4100, 14400, 16, 32, "outliers"),
+    (2051, 4128, 8, 16, "student_t"),
+    (1030, 2112, 3, 8, "ties"),
+])
+def test_prune_many_tasks_ragged(rows, K, N, M, dist):
+    x = _make(rows, K, dist, seed=rows + K)
+    comp = nm.prune_compress(dev(x), N, M, with_mask=True)
+    _check_operand(x, N, M, comp)
+
+
 def test_prune_fp32_input():
     x = np.random.default_rng(0).standard_normal((16, 256)).astype(np.float32)
     comp = nm.prune_compress(dev(x), 2, 4, with_mask=True)
