@@ -54,3 +54,26 @@ def test_reference_arm_only_on_rank_zero(monkeypatch, capsys):
         steps, warmup, gpus, ref_step_s = 1, 3, 2, 0.01
     assert bench.run_reference(A()) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_line_on_rank_zero(monkeypatch, capsys):
+    """The reference arm (the CPU oracle on a bounded sample) prints one JSON
+    line with the ours-arm's metric, unit and workload config, and its own
+    cpu_baseline and e2e objects."""
+    import json
+    from semi_structured_sparse_nm_b200 import inputs
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+
+    class A:
+        steps, warmup, gpus, ref_step_s = 1, 0, 1, 0.01
+    assert bench.run_reference(A()) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["metric"] == bench.METRIC and line["unit"] == "TFLOP/s" and line["higher_is_better"]
+    assert line["config"] == bench.workload_config(inputs.WORKLOADS[bench.HEADLINE], 1)
+    assert line["config"]["workload"] == bench.HEADLINE
+    assert line["value"] > 0 and line["ms_per_step"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                           "d2h_bytes_per_step": 0}
