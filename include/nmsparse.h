@@ -441,7 +441,9 @@ int hybrid_gemm_noalloc(const void *X, int64_t B, const nm_hybrid_weight *W, voi
  * device-resident lifted weight [O][K'] (nm_lift()).  The rows go through in
  * chunks of chunk_rows (a multiple of 128; 0 = 256 rows, or a multiple of 256
  * large enough that a chunk's product occupies at least half the SM pairs:
- * 512 for O = 4096 on 148 SMs): each chunk is copied in
+ * 512 for O = 4096 on 148 SMs; with this default a last chunk of F >= 256
+ * rows goes as F - 128 and 128 rows, which shortens the work left after the
+ * final copy in): each chunk is copied in
  * on one auxiliary stream, pruned and multiplied on `stream`, and copied out
  * on another, with two buffer slots, so that the copy in of the next chunk
  * and the copy out of the previous one overlap the math of the current one

@@ -1473,6 +1473,31 @@ int64_t host_chunk_rows(int64_t T, int64_t O, int64_t chunk_rows) {
   return std::min(T, 256 * m_tiles);
 }
 
+// Chunk c of the host-buffer pipeline: rows [r0, r0 + rows).  Chunks of Tc
+// rows, the last one what is left; with the default chunk size a last chunk
+// of 256 rows or more is split into (F - 128, 128), so that the work after the
+// final copy in (the last chunk's prune, product and copy out) is short.
+struct HostChunks {
+  int64_t T, Tc, n;                               // rows, chunk rows, chunks
+  bool split_tail;
+};
+HostChunks host_chunks(int64_t T, int64_t Tc, bool default_chunk) {
+  const int64_t n = ceil_div(T, Tc);
+  const int64_t last = T - (n - 1) * Tc;
+  const bool split = default_chunk && last >= 256;
+  return {T, Tc, split ? n + 1 : n, split};
+}
+void host_chunk_at(const HostChunks& h, int64_t c, int64_t* r0, int64_t* rows) {
+  if (h.split_tail && c >= h.n - 2) {
+    const int64_t last0 = (h.n - 2) * h.Tc;        // start of the chunk that was split
+    if (c == h.n - 2) { *r0 = last0; *rows = h.T - last0 - 128; }
+    else { *r0 = h.T - 128; *rows = 128; }
+    return;
+  }
+  *r0 = c * h.Tc;
+  *rows = std::min(h.Tc, h.T - *r0);
+}
+
 int64_t round256(int64_t b) { return ceil_div(b, int64_t(256)) * 256; }
 
 // Bytes of one buffer slot: X chunk, compressed values, metadata, Y chunk.
@@ -1515,7 +1540,8 @@ int nm_act_sparse_linear_host(const void* x_host, int64_t T, int64_t K, int N, i
   std::lock_guard<std::mutex> lock(g_pipe_mu);
   HostPipe* p = nullptr;
   if ((rc = host_pipe(&p)) != NM_OK) return rc;
-  const int64_t chunks = ceil_div(T, Tc);
+  const HostChunks plan = host_chunks(T, Tc, chunk_rows == 0);
+  const int64_t chunks = plan.n;
   // The caller's stream orders the call: both copy streams start after the
   // work queued on it so far.
   NM_CUDA_TRY(cudaEventRecord(p->done[0], st));
@@ -1527,7 +1553,8 @@ int nm_act_sparse_linear_host(const void* x_host, int64_t T, int64_t K, int N, i
   NM_CUDA_TRY(cudaEventRecord(p->out[1], st));
   auto enqueue_chunk = [&](int64_t c) -> int {
     const int b = static_cast<int>(c % 2);
-    const int64_t r0 = c * Tc, rows = std::min(Tc, T - r0);
+    int64_t r0 = 0, rows = 0;
+    host_chunk_at(plan, c, &r0, &rows);
     uint8_t* xd = base[b];
     uint8_t* vals = xd + round256(Tc * K * 2);
     uint8_t* meta = vals + round256(Tc * (Kl / 2) * 2);

@@ -17,8 +17,22 @@ def _host(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a)).view(torch.bfloat16).pin_memory()
 
 
+def _chunks(T, O, chunk):
+    """The pipeline's chunks as (first row, rows).  The default chunk is 256
+    rows, or more when a chunk's product would leave more than half the SM
+    pairs idle, and its last chunk of F >= 256 rows goes as F - 128 and 128."""
+    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
+    Tc = chunk or min(T, 256 * max(1, -(-pairs // (2 * -(-O // 224)))))
+    out = [(r0, min(Tc, T - r0)) for r0 in range(0, T, Tc)]
+    r0, last = out[-1]
+    if chunk == 0 and last >= 256:
+        out[-1:] = [(r0, last - 128), (T - 128, 128)]
+    return out
+
+
 @pytest.mark.parametrize("chunk", [0, 128, 384])
-@pytest.mark.parametrize("T,K,O,N,M", [(600, 1024, 768, 8, 16), (256, 512, 1024, 2, 4), (130, 2048, 512, 16, 32)])
+@pytest.mark.parametrize("T,K,O,N,M", [(600, 1024, 768, 8, 16), (256, 512, 1024, 2, 4), (130, 2048, 512, 16, 32),
+                                       (1000, 1024, 4096, 8, 16)])
 def test_host_pipeline_matches_device_calls(chunk, T, K, O, N, M):
     x = inputs.student_t_bf16((T, K), 4.0, T + K)
     w = inputs.normal_bf16((O, K), 0.02, O)
@@ -28,14 +42,10 @@ def test_host_pipeline_matches_device_calls(chunk, T, K, O, N, M):
     nm.act_sparse_linear_host(xh, Wl, N, M, yh, chunk_rows=chunk)
     torch.cuda.synchronize()
     assert nm.device_error() == nm.NM_OK
-    # the same kernels, called chunk by chunk on device buffers; the default
-    # chunk is 256 rows, or more when a chunk's product would leave more than
-    # half the SM pairs idle
-    pairs = torch.cuda.get_device_properties(0).multi_processor_count // 2
-    Tc = chunk or min(T, 256 * max(1, -(-pairs // (2 * -(-O // 224)))))
+    # the same kernels, called chunk by chunk on device buffers
     ref = []
-    for r0 in range(0, T, Tc):
-        c = nm.prune_compress(dev(x[r0:r0 + Tc]), N, M)
+    for r0, rows in _chunks(T, O, chunk):
+        c = nm.prune_compress(dev(x[r0:r0 + rows]), N, M)
         ref.append(host_bits(nm.sparse_gemm(c, Wl, nm.NM_ACT, torch.bfloat16)))
     torch.cuda.synchronize()
     np.testing.assert_array_equal(host_bits(yh), np.concatenate(ref))
