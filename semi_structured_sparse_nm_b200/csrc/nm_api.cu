@@ -453,20 +453,24 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
   // parts in order.  A part keeps at least 16 k-blocks: the partial tiles
   // cost a write and a read of 256 x BN fp32 each, which a shorter part does
   // not pay back (measured on B200: 6:8 prefill, 48 k-blocks in 9 parts,
-  // 10 us of fixup for 3 us saved).  Plain bf16/fp32 outputs of pure 2:4
-  // products only (no dense k-blocks, output split or epilogue scaling).
+  // 10 us of fixup for 3 us saved), and the parts' units must fit the
+  // scratch.  Plain bf16/fp32 outputs of pure 2:4 products only (no dense
+  // k-blocks, output split or epilogue scaling); 256- and 512-row tiles.
   a.sk_full = tiles;
   a.sk_parts = 0;
   a.sk_ws = nullptr;
-  if (p.ws != nullptr && aligned16(p.ws) && MSUB == 1 && !FP8 && p.out_split_rows < 0 && p.kd == 0 &&
+  if (p.ws != nullptr && aligned16(p.ws) && !FP8 && p.out_split_rows < 0 && p.kd == 0 &&
       p.row_scale == nullptr && p.row_shift == nullptr) {
     const int R = tiles / clusters, L = tiles - R * clusters;
     // a last round made only of the last, partial column of tiles is short
     // already (its tiles carry fewer rows of B): no split
     const bool tail_partial = (p.rows_b % BN) != 0 && (tiles - L) / a.tiles_m == a.tiles_n - 1;
     if (R >= 1 && L > 0 && !tail_partial) {
-      const int parts = std::min(clusters / L, static_cast<int>(kb / 16));
-      const size_t need = static_cast<size_t>(L) * parts * 256 * BN * 4;
+      // parts also limited by the scratch: L x parts units of 256 MSUB x BN fp32
+      const size_t unit_bytes = static_cast<size_t>(256) * MSUB * BN * 4;
+      const int64_t fit = static_cast<int64_t>(p.ws_bytes / (unit_bytes * static_cast<size_t>(L)));
+      const int parts = static_cast<int>(std::min<int64_t>(std::min<int64_t>(clusters / L, kb / 16), fit));
+      const size_t need = static_cast<size_t>(L) * parts * unit_bytes;
       if (parts >= 2 && p.ws_bytes >= need) {
         a.sk_full = R * clusters;
         a.sk_parts = parts;
@@ -506,11 +510,11 @@ int launch_gemm_2cta(const GemmPlan& p, cudaStream_t st) {
     const size_t n = std::strlen(g_last_gemm);
     std::snprintf(g_last_gemm + n, sizeof(g_last_gemm) - n, "+split%d", a.sk_parts);
     const int tail = tiles - a.sk_full;
-    const int64_t total = static_cast<int64_t>(tail) * 64 * BN;     // 4-output quads
+    const int64_t total = static_cast<int64_t>(tail) * 64 * MSUB * BN;     // 4-output quads
     const int64_t blocks = std::min<int64_t>(ceil_div(total, int64_t(256)), int64_t(num_sms()) * 8);
     NM_CUDA_TRY(launch_pdl(nm::k_sk_fixup, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
-                           static_cast<const float*>(a.sk_ws), a.sk_full, a.sk_parts, tail, a.tiles_m, BN,
-                           p.rows_a, p.rows_b, p.y, p.ldy, p.out_fp32, p.transpose));
+                           static_cast<const float*>(a.sk_ws), a.sk_full, a.sk_parts, tail, a.tiles_m, 256 * MSUB,
+                           BN, p.rows_a, p.rows_b, p.y, p.ldy, p.out_fp32, p.transpose));
     NM_CUDA_TRY(cudaGetLastError());
   }
   return NM_OK;

@@ -164,7 +164,7 @@ struct Gemm2Args {
   // run whole in persistent rounds (sk_full is a multiple of the cluster
   // count); in the round after them, cluster u takes k-part u % sk_parts of
   // tile sk_full + u / sk_parts and leaves its fp32 accumulator in sk_ws
-  // (unit ((tile - sk_full) * sk_parts + part), [256 rows][BN], no epilogue
+  // (unit ((tile - sk_full) * sk_parts + part), [256 MSUB rows][BN], no epilogue
   // scaling); k_sk_fixup sums the parts and writes those tiles of Y.
   int sk_full;
   int sk_parts;
@@ -583,8 +583,9 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           if (wk.part >= 0) {
             // stream-K part: the raw fp32 accumulator goes to its workspace unit
             float4* dst = reinterpret_cast<float4*>(
-                args.sk_ws + (static_cast<size_t>(wk.t - args.sk_full) * args.sk_parts + wk.part) * (256 * BN) +
-                static_cast<size_t>(rank * 128 + q * 32 + lane) * BN + c0);
+                args.sk_ws +
+                (static_cast<size_t>(wk.t - args.sk_full) * args.sk_parts + wk.part) * (256 * MSUB * BN) +
+                static_cast<size_t>(u * 256 + rank * 128 + q * 32 + lane) * BN + c0);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
@@ -682,17 +683,17 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
 }
 
 // Stream-K fixup: every split tile of Y is the sum, in part order, of its
-// parts' fp32 partial tiles (workspace units, [256 rows][BN]), converted as
+// parts' fp32 partial tiles (workspace units, [tile_rows][BN]), converted as
 // the GEMM epilogue converts (fp32 or bf16 nearest-even; Y[a][b] or, with
 // transpose, Y[b][a]).  A thread takes four consecutive columns of one row
 // (one 16-byte load per part); consecutive threads take consecutive columns
 // (Y[a][b]) or consecutive rows (Y[b][a]), so that the stores coalesce.
 __global__ void __launch_bounds__(256)
-k_sk_fixup(const float* __restrict__ ws, int sk_full, int sk_parts, int tail_tiles, int tiles_m, int BN,
-           int64_t rows_a, int64_t rows_b, void* __restrict__ Y, int64_t ldy, int out_fp32, int transpose) {
+k_sk_fixup(const float* __restrict__ ws, int sk_full, int sk_parts, int tail_tiles, int tiles_m, int tile_rows,
+           int BN, int64_t rows_a, int64_t rows_b, void* __restrict__ Y, int64_t ldy, int out_fp32, int transpose) {
   griddep_launch_dependents();
   griddep_wait();                                      // the partial tiles of the preceding GEMM
-  const int64_t unit = 256 * static_cast<int64_t>(BN);
+  const int64_t unit = static_cast<int64_t>(tile_rows) * BN;
   const int64_t quads = unit / 4;
   const int64_t total = static_cast<int64_t>(tail_tiles) * quads;
   for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
@@ -700,9 +701,9 @@ k_sk_fixup(const float* __restrict__ ws, int sk_full, int sk_parts, int tail_til
     const int tl = static_cast<int>(idx / quads);
     const int e = static_cast<int>(idx - tl * quads);
     const int t = sk_full + tl;
-    const int64_t a0 = static_cast<int64_t>(t % tiles_m) * 256, b0 = static_cast<int64_t>(t / tiles_m) * BN;
-    const int ra = transpose ? e % 256 : e / (BN / 4);
-    const int cb = 4 * (transpose ? e / 256 : e % (BN / 4));
+    const int64_t a0 = static_cast<int64_t>(t % tiles_m) * tile_rows, b0 = static_cast<int64_t>(t / tiles_m) * BN;
+    const int ra = transpose ? e % tile_rows : e / (BN / 4);
+    const int cb = 4 * (transpose ? e / tile_rows : e % (BN / 4));
     // all of a group of up to eight parts' loads in flight before the adds
     // (still added in part order)
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);

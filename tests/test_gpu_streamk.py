@@ -84,3 +84,41 @@ def test_split_round_random_within_tolerance_and_deterministic(ra, rb, K, N, M, 
         y = y.T
     for r0 in range(0, ra, 512):
         check_close(y[r0:r0 + 512], ref[r0:r0 + 512], f"split round {ra}x{rb}x{K}, rows {r0}..")
+
+
+# 512-row tiles (two M = 256 MMAs per B stage), pinned by NMSPARSE_GEMM:
+# (sparse rows, dense rows, K, N, M, side, variant), one round of 74 pairs
+# and a few tiles more
+SHAPES_512 = [
+    (4096, 2240, 4096, 2, 4, "act", "2cta224x2"),      # 8 x 10 tiles of 512 x 224, 2 parts
+    (4096, 1280, 4096, 6, 8, "weight", "2cta128x2"),   # 8 x 10 tiles of 512 x 128, 3 parts
+]
+
+
+@pytest.mark.parametrize("ra,rb,K,N,M,side,variant", SHAPES_512)
+def test_split_round_on_512_row_tiles(monkeypatch, ra, rb, K, N, M, side, variant):
+    monkeypatch.setenv("NMSPARSE_GEMM", variant)
+    rng = np.random.default_rng(ra + rb + K + 1)
+    a = _int_bf16(rng, (ra, K))
+    b = _int_bf16(rng, (rb, K), -3, 4)
+    S = nm.prune_compress(dev(a), N, M)
+    D = nm.lift(dev(b), M)
+    sd = nm.NM_ACT if side == "act" else nm.NM_WEIGHT
+    y = nm.sparse_gemm(S, D, sd, torch.float32)
+    kname = nm.last_gemm_kernel()
+    assert ",1,2>" in kname and "+split" in kname, kname
+    # random data: within tolerance of the oracle and deterministic
+    ar = inputs.student_t_bf16((ra, K), 4.0, seed=ra + 7)
+    br = inputs.normal_bf16((rb, K), 0.02, seed=rb + 7)
+    Sr = nm.prune_compress(dev(ar), N, M)
+    Dr = nm.lift(dev(br), M)
+    y1 = nm.sparse_gemm(Sr, Dr, sd, torch.bfloat16)
+    y2 = nm.sparse_gemm(Sr, Dr, sd, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    ref = oracle.act_sparse_linear(a, b, N, M)
+    np.testing.assert_array_equal(host_f64(y), ref if side == "act" else ref.T)
+    assert torch.equal(y1, y2)
+    ref_r = oracle.act_sparse_linear(ar, br, N, M)
+    check_close(host_f64(y1), ref_r if side == "act" else ref_r.T, f"512-row tiles {variant}")
+
