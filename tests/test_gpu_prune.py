@@ -66,6 +66,8 @@ def test_prune_compress_bit_exact(rows, K, N, M, dist):
     (4100, 14400, 16, 32, "outliers"),
     (2051, 4128, 8, 16, "student_t"),
     (1030, 2112, 3, 8, "ties"),
+    # about eleven whole tasks per CTA, each row one bulk-copied chunk
+    (100003, 512, 4, 8, "student_t"),
 ])
 def test_prune_many_tasks_ragged(rows, K, N, M, dist):
     x = _make(rows, K, dist, seed=rows + K)

@@ -109,3 +109,30 @@ def test_fp8_weight_side(i):
     torch.cuda.synchronize()
     assert nm.device_error() == nm.NM_OK
     check_close(host_f64(y), oracle.fp8_weight_sparse_linear(x, w, N, M), f"fp8 {T}x{K}x{O} {N}:{M}")
+
+
+@pytest.mark.parametrize("T,K,O,N,M,side", [
+    (40, 131072, 300, 8, 16, "act"),       # 114688 lifted K: 896 k-blocks, split-K on single CTAs
+    (256, 65536, 512, 16, 32, "act"),      # 122880 lifted K on SM pairs
+    (16, 98304, 256, 6, 8, "weight"),      # 147456 lifted K, decode shape
+])
+def test_long_reductions(T, K, O, N, M, side):
+    """Reductions far beyond the workloads' (up to 147456 lifted K): the
+    operand stays bit-exact and the product within tolerance, so no index
+    or k-block count overflows on the way."""
+    x = inputs.student_t_bf16((T, K), 4.0, T + K)
+    w = inputs.normal_bf16((O, K), 0.02, O + K)
+    if side == "act":
+        comp = nm.prune_compress(dev(x), N, M, with_mask=True)
+        y = nm.sparse_gemm(comp, nm.lift(dev(w), M), nm.NM_ACT, torch.float32)
+        ref_op, y_ref = oracle.sparse_operand(x, N, M), oracle.act_sparse_linear(x, w, N, M)
+    else:
+        comp = nm.slide_decompose(dev(w), N, M, with_mask=True)
+        y = nm.sparse_gemm(comp, nm.lift(dev(x), M), nm.NM_WEIGHT, torch.float32)
+        ref_op, y_ref = oracle.sparse_operand(w, N, M), oracle.weight_sparse_linear(x, w, N, M)
+    torch.cuda.synchronize()
+    assert nm.device_error() == nm.NM_OK
+    np.testing.assert_array_equal(host_bits(comp.mask), ref_op["mask"], err_msg="mask")
+    np.testing.assert_array_equal(host_bits(comp.vals), ref_op["vals"], err_msg="values")
+    np.testing.assert_array_equal(host_bits(comp.meta)[:ref_op["meta"].size], ref_op["meta"], err_msg="metadata")
+    check_close(host_f64(y), y_ref, f"K={K} {N}:{M} {side}")
