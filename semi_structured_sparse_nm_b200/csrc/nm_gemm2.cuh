@@ -570,6 +570,66 @@ k_nm_gemm_2cta(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
       const uint32_t use = static_cast<uint32_t>(lt / NACC);
       if (!mbar_wait_warp(&tfull_bar[b], use & 1u, abort_flag, kWhereEpilogue)) break;
       tc_fence_after();
+      if constexpr (NACC == 1 && MSUB == 1 && !FP8 && !LIFT) {
+        // One accumulator: the next tile's MMAs wait for it.  A plain bf16
+        // tile is read out whole into registers (BN / 2 bf16 pairs per
+        // thread) and the accumulator released before the stores, so the
+        // stores overlap the next tile's MMAs.
+        if (wk.part < 0 && args.tma_store != 0 && args.scale_a == nullptr) {
+          const int64_t row0 = static_cast<int64_t>(tm) * 256 + rank * 128 + q * 32;
+          const uint32_t acc = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+          uint32_t pk[BN / 2];
+#pragma unroll
+          for (int c0 = 0; c0 < BN; c0 += 32) {
+            uint32_t v[32];
+            tc_ld_32x32b_x32(acc + c0, v);
+            tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+              pk[c0 / 2 + i] = *reinterpret_cast<uint32_t*>(&h);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty_leader0);
+#pragma unroll
+          for (int c0 = 0; c0 < BN; c0 += 32) {
+            uint8_t* buf = sY + (q * 2 + (ebuf & 1)) * 2048;
+            if (lane == 0 && ebuf >= 2) bulk_wait_read1();
+            __syncwarp();
+            if (args.tma_store == 2) {
+              // transposed: [32 columns of this tile][32 rows] staging tile
+              uint16_t* t = reinterpret_cast<uint16_t*>(buf);
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                t[(2 * i) * 32 + lane] = static_cast<uint16_t>(pk[c0 / 2 + i] & 0xFFFFu);
+                t[(2 * i + 1) * 32 + lane] = static_cast<uint16_t>(pk[c0 / 2 + i] >> 16);
+              }
+            } else {
+              // 32 rows x 32 bf16, 64-byte swizzle (as below)
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                *reinterpret_cast<uint4*>(buf + lane * 64 + 16 * (j ^ ((lane >> 1) & 3))) =
+                    make_uint4(pk[c0 / 2 + 4 * j], pk[c0 / 2 + 4 * j + 1], pk[c0 / 2 + 4 * j + 2],
+                               pk[c0 / 2 + 4 * j + 3]);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+              if (args.tma_store == 2)
+                tma_store_2d(&tmY, buf, static_cast<int32_t>(row0),
+                             static_cast<int32_t>(static_cast<int64_t>(tn) * BN + c0));
+              else
+                tma_store_2d(&tmY, buf, static_cast<int32_t>(static_cast<int64_t>(tn) * BN + c0),
+                             static_cast<int32_t>(row0));
+              bulk_commit();
+            }
+            ++ebuf;
+          }
+          continue;
+        }
+      }
 #pragma unroll 1
       for (int u = 0; u < MSUB; ++u) {
         const int64_t row0 = (static_cast<int64_t>(tm) * MSUB + u) * 256 + rank * 128 + q * 32;
