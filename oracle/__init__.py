@@ -274,6 +274,42 @@ def sparse_operand(x: np.ndarray, N: int, M: int):
     return dict(keep=keep, mask=mask_pack(keep), vals=vals, nib=nib, meta=meta_hw(nib, Kl), K_lift=Kl)
 
 
+def split_window_order(K: int, M: int) -> np.ndarray:
+    """The split window order of a row of K = G M elements (M = 2n, n even):
+    window w of group g covers positions g M + 2w .. g M + 2w + 3 (SlideSparse
+    page, technical summary §2.A), so the even windows 0, 2, ..., n - 2 of a
+    group tile it exactly and the odd ones overlap them.  The split order
+    lists every group's even windows, group by group, then every group's odd
+    windows: entry j is the natural (group-major) index of the window placed
+    j-th.  Lifting in this order gives [X | the odd windows of X]."""
+    assert M % 4 == 0 and K % M == 0
+    NW, NE = M // 2 - 1, M // 4
+    G = K // M
+    even = [g * NW + 2 * e for g in range(G) for e in range(NE)]
+    odd = [g * NW + 2 * o + 1 for g in range(G) for o in range(NE - 1)]
+    return np.array(even + odd, dtype=np.int64)
+
+
+def lift_split(x: np.ndarray, M: int) -> np.ndarray:
+    """The lifted operand with its windows in the split order (bf16 bits)."""
+    rows, K = x.shape
+    nat = lift(x, M)
+    perm = split_window_order(K, M)
+    return np.ascontiguousarray(nat.reshape(rows, -1, 4)[:, perm, :].reshape(rows, -1))
+
+
+def sparse_operand_split(x: np.ndarray, N: int, M: int):
+    """sparse_operand() with the windows in the split order: values and
+    index pairs moved window by window, the metadata image built from them."""
+    ref = sparse_operand(x, N, M)
+    rows, K = x.shape
+    perm = split_window_order(K, M)
+    vals = np.ascontiguousarray(ref["vals"].reshape(rows, -1, 2)[:, perm, :].reshape(rows, -1))
+    nib = np.ascontiguousarray(ref["nib"][:, perm])
+    return dict(keep=ref["keep"], mask=ref["mask"], vals=vals, nib=nib, meta=meta_hw(nib, ref["K_lift"]),
+                K_lift=ref["K_lift"])
+
+
 def act_sparse_linear(x: np.ndarray, w: np.ndarray, N: int, M: int, rows=None) -> np.ndarray:
     """Y = prune_{N:M}(X) . W^T in fp64 (activation sparsity)."""
     keep = prune(x, N, M)
