@@ -175,6 +175,35 @@ int slide_decompose(const void *w, nm_dtype dt, int64_t rows, int64_t K, int N, 
 int nm_lift(const void *src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, int M,
             void *dst, void *stream);
 
+/* The split window order (a layout of this library, for the (2N-2):2N
+ * weight side).  Window w of group g covers elements g*2n + 2w .. + 3, so
+ * a group's even windows 0, 2, ..., n-2 tile it and its odd windows overlap
+ * them [SlideSparse, technical summary §2.A].  In the split order each row's
+ * windows are every group's even windows, group by group, then every group's
+ * odd windows; the lifted activations in that order are [X | the odd windows
+ * of X], so the GEMM reads the raw activations for two thirds (6:8) of its
+ * reduction and only the odd windows are materialised [§2.B-§2.C place the
+ * lift inside the online kernel; this keeps X where it is instead].
+ *
+ * slide_decompose_split(): slide_decompose() with the windows of every row
+ * in the split order: bf16 W [rows x K] (row stride K), N = M - 2 with
+ * M = 8, 16 or 32, K a multiple of 128 (so that the even windows end on a
+ * 128-K metadata block); else NM_ERR_UNSUPPORTED.  Outputs as
+ * nm_prune_compress() (values [rows][K'/2], metadata image, optional mask);
+ * the operand is multiplied by nm_sparse_gemm() (NM_WEIGHT) against lifted
+ * activations in the same order, which nm_lift_odd() makes in place. */
+int slide_decompose_split(const void *w, int64_t rows, int64_t K, int N, int M, uint32_t *mask_out,
+                          void *vals_out, void *meta_out, void *stream);
+
+/* nm_lift_odd(): x bf16 [rows x ld] holds X [rows x K] in its first K
+ * columns; columns [K, K') receive the odd windows of X in the split order
+ * (group g's odd window o = X[r][g*M + 4o + 2 .. + 5] at column
+ * K + g*4(M/4 - 1) + 4o).  M = 8, 16 or 32 and K a multiple of 128 (else
+ * NM_ERR_UNSUPPORTED); ld >= K' (else NM_ERR_INVALID_ARG); x 16-byte aligned
+ * with 16-byte rows (else NM_ERR_ALIGNMENT).  With ld = K' the buffer is the
+ * dense operand of nm_sparse_gemm() for a slide_decompose_split() weight. */
+int nm_lift_odd(void *x, int64_t rows, int64_t K, int64_t ld, int M, void *stream);
+
 /* ------------------------------------------------------------------- GEMM */
 
 /* Y = sparse . dense^T (side NM_ACT) or its transpose (NM_WEIGHT), bf16

@@ -62,6 +62,8 @@ def lib():
             "nm_prune_compress": (I, [P, I, I64, I64, I64, I, I, P, P, P, P]),
             "slide_decompose": (I, [P, I, I64, I64, I, I, P, P, P, P]),
             "nm_lift": (I, [P, I, I64, I64, I64, I, P, P]),
+            "slide_decompose_split": (I, [P, I64, I64, I, I, P, P, P, P]),
+            "nm_lift_odd": (I, [P, I64, I64, I64, I, P]),
             "nm_sparse_gemm_workspace_size": (SZ, [ctypes.POINTER(SparseOperand), I64, I]),
             "nm_sparse_gemm": (I, [ctypes.POINTER(SparseOperand), P, I64, I, P, I, P, SZ, P]),
             "slide_gemm_workspace_size": (SZ, [ctypes.POINTER(SparseOperand), I64]),
@@ -194,6 +196,31 @@ def slide_decompose(w: torch.Tensor, N: int, M: int, with_mask: bool = False) ->
     _check("slide_decompose", lib().slide_decompose(
         _p(w), _dt(w), rows, K, N, M, _p(out.mask), _p(out.vals), _p(out.meta), _stream(w)))
     return out
+
+
+def slide_decompose_split(w: torch.Tensor, N: int, M: int, with_mask: bool = False) -> Compressed:
+    """slide_decompose() with every row's windows in the split order (each
+    group's even windows, then its odd ones); multiply it by lifted
+    activations in the same order (lift_odd())."""
+    _need_cuda(w)
+    rows, K = w.shape
+    if w.stride(0) != K or w.dtype != torch.bfloat16:
+        raise ValueError("slide_decompose_split expects a contiguous bf16 weight")
+    out = alloc_compressed(rows, K, N, M, w.device, with_mask)
+    _check("slide_decompose_split", lib().slide_decompose_split(
+        _p(w), rows, K, N, M, _p(out.mask), _p(out.vals), _p(out.meta), _stream(w)))
+    return out
+
+
+def lift_odd(x_wide: torch.Tensor, K: int, M: int) -> torch.Tensor:
+    """In place: x_wide bf16 [rows, >= K'] holds X in its first K columns;
+    columns [K, K') receive X's odd windows (the split order).  Returns
+    x_wide[:, :K'], the dense operand for a slide_decompose_split() weight."""
+    _need_cuda(x_wide)
+    rows = x_wide.shape[0]
+    Kl = lifted_k(K, M)
+    _check("nm_lift_odd", lib().nm_lift_odd(_p(x_wide), rows, K, x_wide.stride(0), M, _stream(x_wide)))
+    return x_wide[:, :Kl]
 
 
 def lift(src: torch.Tensor, M: int, out: torch.Tensor | None = None) -> torch.Tensor:

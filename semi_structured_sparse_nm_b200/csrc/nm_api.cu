@@ -598,7 +598,7 @@ int run_gemm(const GemmPlan& p, cudaStream_t st) {
 // --------------------------------------------------------------- prune
 // early = false launches without programmatic serialisation (the prune then
 // waits for copies and event waits queued before it, not only for kernels).
-template <typename T, bool Q8 = false, bool XF = false>
+template <typename T, bool Q8 = false, bool XF = false, bool SPLIT = false>
 int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M, uint32_t* mask,
                  void* vals, void* meta, cudaStream_t st, const float* row_scale = nullptr,
                  const float* row_shift = nullptr, double* stats = nullptr, bool early = true) {
@@ -622,12 +622,21 @@ int launch_prune(const T* src, int64_t rows, int64_t K, int64_t ld, int N, int M
                                 row_shift, stats);
   };
   cudaError_t err;
-  switch (M) {
-    case 4: err = go(nm::k_prune_compress<4, T, Q8, XF>); break;
-    case 8: err = go(nm::k_prune_compress<8, T, Q8, XF>); break;
-    case 16: err = go(nm::k_prune_compress<16, T, Q8, XF>); break;
-    case 32: err = go(nm::k_prune_compress<32, T, Q8, XF>); break;
-    default: return NM_ERR_UNSUPPORTED;
+  if constexpr (SPLIT) {
+    switch (M) {
+      case 8: err = go(nm::k_prune_compress<8, T, false, false, true>); break;
+      case 16: err = go(nm::k_prune_compress<16, T, false, false, true>); break;
+      case 32: err = go(nm::k_prune_compress<32, T, false, false, true>); break;
+      default: return NM_ERR_UNSUPPORTED;
+    }
+  } else {
+    switch (M) {
+      case 4: err = go(nm::k_prune_compress<4, T, Q8, XF>); break;
+      case 8: err = go(nm::k_prune_compress<8, T, Q8, XF>); break;
+      case 16: err = go(nm::k_prune_compress<16, T, Q8, XF>); break;
+      case 32: err = go(nm::k_prune_compress<32, T, Q8, XF>); break;
+      default: return NM_ERR_UNSUPPORTED;
+    }
   }
   NM_CUDA_TRY(err);
   NM_CUDA_TRY(cudaGetLastError());
@@ -649,6 +658,22 @@ int launch_lift(const T* src, int64_t rows, int64_t K, int64_t ld, int M, void* 
     case 8: err = launch_pdl(nm::k_lift<8, T>, grid, block, 0, st, src, rows, K, ld, d, Kl); break;
     case 16: err = launch_pdl(nm::k_lift<16, T>, grid, block, 0, st, src, rows, K, ld, d, Kl); break;
     case 32: err = launch_pdl(nm::k_lift<32, T>, grid, block, 0, st, src, rows, K, ld, d, Kl); break;
+    default: return NM_ERR_UNSUPPORTED;
+  }
+  NM_CUDA_TRY(err);
+  NM_CUDA_TRY(cudaGetLastError());
+  return NM_OK;
+}
+
+int launch_lift_odd(uint16_t* x, int64_t rows, int64_t K, int64_t ld, int M, cudaStream_t st) {
+  const int64_t total = rows * (K / M / 2);
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(total, int64_t(256)), int64_t(num_sms()) * 8));
+  const dim3 grid(static_cast<unsigned>(blocks)), block(256);
+  cudaError_t err;
+  switch (M) {
+    case 8: err = launch_pdl(nm::k_lift_odd<8>, grid, block, 0, st, x, rows, K, ld); break;
+    case 16: err = launch_pdl(nm::k_lift_odd<16>, grid, block, 0, st, x, rows, K, ld); break;
+    case 32: err = launch_pdl(nm::k_lift_odd<32>, grid, block, 0, st, x, rows, K, ld); break;
     default: return NM_ERR_UNSUPPORTED;
   }
   NM_CUDA_TRY(err);
@@ -701,6 +726,27 @@ int slide_decompose(const void* w, nm_dtype dt, int64_t rows, int64_t K, int N, 
                     void* vals_out, void* meta_out, void* stream) {
   if (!(N == M - 2 || (M == 4 && N == 2))) return NM_ERR_UNSUPPORTED;
   return nm_prune_compress(w, dt, rows, K, K, N, M, mask_out, vals_out, meta_out, stream);
+}
+
+int slide_decompose_split(const void* w, int64_t rows, int64_t K, int N, int M, uint32_t* mask_out, void* vals_out,
+                          void* meta_out, void* stream) {
+  int rc = check_prune_args(w, NM_BF16, rows, K, K, N, M, vals_out, meta_out);
+  if (rc != NM_OK) return rc;
+  if (N != M - 2 || M < 8 || M % 4 != 0 || K % 128 != 0) return NM_ERR_UNSUPPORTED;
+  if (mask_out != nullptr && !aligned16(mask_out)) return NM_ERR_ALIGNMENT;
+  if (rows == 0) return NM_OK;
+  return launch_prune<uint16_t, false, false, true>(static_cast<const uint16_t*>(w), rows, K, K, N, M, mask_out,
+                                                     vals_out, meta_out, static_cast<cudaStream_t>(stream));
+}
+
+int nm_lift_odd(void* x, int64_t rows, int64_t K, int64_t ld, int M, void* stream) {
+  if (rows < 0 || K <= 0 || M <= 0 || K % M != 0) return NM_ERR_INVALID_ARG;
+  if (M < 8 || M % 4 != 0 || !m_supported(M) || K % 128 != 0) return NM_ERR_UNSUPPORTED;
+  if (ld < nm_lifted_k(K, M)) return NM_ERR_INVALID_ARG;
+  if (rows == 0) return NM_OK;
+  if (x == nullptr) return NM_ERR_INVALID_ARG;
+  if (!aligned16(x) || (ld * 2) % 16 != 0) return NM_ERR_ALIGNMENT;
+  return launch_lift_odd(static_cast<uint16_t*>(x), rows, K, ld, M, static_cast<cudaStream_t>(stream));
 }
 
 int nm_lift(const void* src, nm_dtype dt, int64_t rows, int64_t K, int64_t ld, int M, void* dst, void* stream) {

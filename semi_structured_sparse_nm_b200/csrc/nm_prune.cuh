@@ -412,7 +412,12 @@ struct PruneGrid {
 // stats, each (row, chunk of 32 G groups) leaves the fp64 sum and sum of
 // squares of its kept entries at stats[(r * chunks + chunk) * 2] for the VAR
 // factor.
-template <int M, typename T, bool Q8 = false, bool XF = false>
+// SPLIT = true (bf16 weights, M = 8, 16, 32) writes the windows of each row
+// in the split order: every group's even windows (which tile it, so that the
+// matching lifted activations are the raw ones), then every group's odd
+// windows.  A task row stages its even windows first; its metadata blocks go
+// to the even region (blocks below K/128) and the odd region after it.
+template <int M, typename T, bool Q8 = false, bool XF = false, bool SPLIT = false>
 __global__ void __launch_bounds__(kPruneWarps * 32, prune_min_blocks(M, sizeof(T)))
 k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld, int N,
                  uint32_t* __restrict__ mask_out, void* __restrict__ vals_out,
@@ -421,11 +426,15 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
                  double* __restrict__ stats) {
   static_assert(!Q8 || sizeof(T) == 2, "8-bit output from bf16 input");
   static_assert(!XF || (sizeof(T) == 2 && !Q8), "transform mode: bf16 input, bf16 output");
+  static_assert(!SPLIT || (sizeof(T) == 2 && !Q8 && !XF && M % 4 == 0 && M >= 8), "split order: bf16 weights");
   constexpr int G = prune_groups_per_lane(M, static_cast<int>(sizeof(T)));
   constexpr int NW = M / 2 - 1;                   // windows per group
   constexpr int NWL = G * NW;                     // windows per lane
   constexpr int WIN = 32 * NWL;                   // windows per task row = NWL blocks
   constexpr int LM = G * M;                       // elements (keep bits) per lane
+  constexpr int NE = M / 4, NO = M / 4 - 1;       // split order: even and odd windows per group
+  constexpr int WIN_E = 32 * G * NE;              // split order: even windows per task row
+  constexpr int NWLE = G * NE;                    // split order: even metadata blocks per task row
   // staged rows of 768 bytes and more leave as bulk copies; shorter ones (2:4)
   // were measured faster as 16-byte stores by the lanes
   constexpr bool kBulkRow = WIN * (Q8 ? 2 : 4) >= 768;
@@ -545,14 +554,20 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
           }
 #pragma unroll
           for (int w = 0; w < NWL; ++w) {
+            // staging slot of lane window w (group w / NW of the lane, window w % NW)
+            int pos = lane * NWL + w;
+            if constexpr (SPLIT) {
+              const int j = w / NW, wi = w % NW;
+              pos = (wi % 2 == 0) ? lane * G * NE + j * NE + wi / 2 : WIN_E + lane * G * NO + j * NO + wi / 2;
+            }
             if constexpr (Q8) {
-              reinterpret_cast<uint16_t*>(&s_val[warp][kBulkRow ? k : 0][0])[lane * NWL + w] = static_cast<uint16_t>(
+              reinterpret_cast<uint16_t*>(&s_val[warp][kBulkRow ? k : 0][0])[pos] = static_cast<uint16_t>(
                   e4m3x2(__fmul_rn(elem_f32(static_cast<uint16_t>(vals[w] & 0xFFFFu)), inv),
                          __fmul_rn(elem_f32(static_cast<uint16_t>(vals[w] >> 16)), inv)));
             } else {
-              s_val[warp][kBulkRow ? k : 0][lane * NWL + w] = vals[w];
+              s_val[warp][kBulkRow ? k : 0][pos] = vals[w];
             }
-            s_nib[it][lane * NWL + w] = nibs[w];
+            s_nib[it][pos] = nibs[w];
           }
           if (mask_out != nullptr)
             atomicOr(&s_mask[warp][(lane * LM) / 32],
@@ -577,6 +592,21 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
             for (int i = lane; i < WIN / 8; i += 32) dv[i] = sv[i];
           } else {
             for (int i = lane; i < ng * NW; i += 32) vrow[i] = sv16[i];
+          }
+        } else if constexpr (SPLIT) {
+          // the even run and the odd run of the task row, each to its region
+          uint32_t* vrow = static_cast<uint32_t*>(vals_out) + r * (Kl / 4);
+          uint32_t* ve = vrow + g0 * NE;
+          uint32_t* vo = vrow + K / 4 + g0 * NO;
+          const uint32_t* sv = &s_val[warp][kBulkRow ? k : 0][0];
+          if (bulk) {
+            if (lane == 0) {
+              bulk_store(ve, sv, WIN_E * 4);
+              bulk_store(vo, sv + WIN_E, (WIN - WIN_E) * 4);
+            }
+          } else {
+            for (int i = lane; i < ng * NE; i += 32) ve[i] = sv[i];
+            for (int i = lane; i < ng * NO; i += 32) vo[i] = sv[WIN_E + i];
           }
         } else {
           uint32_t* vrow = static_cast<uint32_t*>(vals_out) + r * (Kl / 4) + g0 * NW;
@@ -638,7 +668,17 @@ k_prune_compress(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
     } else {
       for (int i = threadIdx.x; i < NWL * 16; i += blockDim.x) {
         const int b = i / 16, L = i % 16;
-        const int64_t kb = static_cast<int64_t>(ch) * NWL + b;
+        int64_t kb = static_cast<int64_t>(ch) * NWL + b;
+        if constexpr (SPLIT) {
+          // even blocks below K/128 (padding blocks of a short last chunk are
+          // dropped there), odd blocks from K/128 on
+          if (b < NWLE) {
+            kb = static_cast<int64_t>(ch) * NWLE + b;
+            if (kb >= K / 128) continue;
+          } else {
+            kb = K / 128 + static_cast<int64_t>(ch) * (NWL - NWLE) + (b - NWLE);
+          }
+        }
         if (kb >= KB) continue;
         const int i8 = L % 8, h = L / 8;
         uint32_t wds[4];
@@ -745,6 +785,42 @@ k_lift(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
 }
 
 // ------------------------------------------------------------- hybrid prep
+
+// Odd-window lift in place (the split window order): x [rows][ld] holds X in
+// columns [0, K); columns [K, K') receive, group by group, the odd windows of
+// X.  Odd window o of a group covers its elements 4o + 2 .. 4o + 5, i.e. its
+// 32-bit words 2o + 1, 2o + 2, so a group's odd windows are its words 1 ..
+// 2(M/4 - 1): the group without its first and last two elements.  A thread
+// takes two groups of one row (K % 128 == 0 keeps the group count even):
+// 16-byte loads of both, 16-byte stores of their odd windows.
+template <int M>
+__global__ void __launch_bounds__(256) k_lift_odd(uint16_t* x, int64_t rows, int64_t K, int64_t ld) {
+  static_assert(M % 8 == 0 && M >= 8, "two groups make whole 16-byte loads and stores");
+  constexpr int NO = M / 4 - 1;                   // odd windows per group
+  griddep_launch_dependents();
+  griddep_wait();                                      // X may come from the preceding kernel
+  const int64_t pairs = K / M / 2;                     // group pairs per row
+  const int64_t total = rows * pairs;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = idx / pairs, t = idx - r * pairs;
+    const uint4* src = reinterpret_cast<const uint4*>(x + r * ld + t * 2 * M);
+    uint32_t w[M];                                     // the two groups, M / 2 words each
+#pragma unroll
+    for (int i = 0; i < M / 4; ++i) {
+      const uint4 q = src[i];
+      w[4 * i] = q.x; w[4 * i + 1] = q.y; w[4 * i + 2] = q.z; w[4 * i + 3] = q.w;
+    }
+    uint32_t o[4 * NO];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int k = 0; k < 2 * NO; ++k) o[h * 2 * NO + k] = w[h * (M / 2) + 1 + k];
+    uint4* dst = reinterpret_cast<uint4*>(x + r * ld + K + t * 8 * NO);
+#pragma unroll
+    for (int i = 0; i < NO; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+  }
+}
 
 // colnorm[c] = sum over rows r ascending of w[r][c]^2, fp64 (each square of a
 // bf16 value is exact in fp64, so fused and unfused updates agree).

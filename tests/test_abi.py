@@ -70,6 +70,18 @@ def test_validation_before_launch(L):
     # empty operands are a no-op
     assert L.nm_prune_compress(null, 0, 0, 256, 256, 2, 4, null, null, null, s) == nm.NM_OK
     assert L.nm_lift(null, 0, 0, 256, 256, 8, null, s) == nm.NM_OK
+    # the split window order: 6:8, 14:16, 30:32 with K % 128 == 0 only
+    assert L.slide_decompose_split(fake, 4, 192, 6, 8, null, fake, fake, s) == nm.NM_ERR_UNSUPPORTED
+    assert L.slide_decompose_split(fake, 4, 256, 2, 4, null, fake, fake, s) == nm.NM_ERR_UNSUPPORTED
+    assert L.slide_decompose_split(fake, 4, 256, 4, 8, null, fake, fake, s) == nm.NM_ERR_UNSUPPORTED
+    assert L.slide_decompose_split(null, 4, 256, 6, 8, null, fake, fake, s) == nm.NM_ERR_INVALID_ARG
+    assert L.slide_decompose_split(null, 0, 256, 6, 8, null, null, null, s) == nm.NM_OK
+    assert L.nm_lift_odd(fake, 4, 192, 288, 8, s) == nm.NM_ERR_UNSUPPORTED      # K % 128
+    assert L.nm_lift_odd(fake, 4, 256, 256, 8, s) == nm.NM_ERR_INVALID_ARG      # ld < K' = 384
+    assert L.nm_lift_odd(fake, 4, 256, 384, 4, s) == nm.NM_ERR_UNSUPPORTED      # 2:4 has no odd windows
+    assert L.nm_lift_odd(odd, 4, 256, 384, 8, s) == nm.NM_ERR_ALIGNMENT
+    assert L.nm_lift_odd(fake, 4, 256, 388, 8, s) == nm.NM_ERR_ALIGNMENT        # 776-byte rows
+    assert L.nm_lift_odd(null, 0, 256, 384, 8, s) == nm.NM_OK
     # GEMM
     S = nm.SparseOperand(0x10000, 0x10000, 128, 256, 2, 4, 256)
     assert L.nm_sparse_gemm(ctypes.byref(S), null, 64, 0, fake, 0, null, 0, s) == nm.NM_ERR_INVALID_ARG
