@@ -667,7 +667,7 @@ int launch_lift(const T* src, int64_t rows, int64_t K, int64_t ld, int M, void* 
 
 int launch_lift_odd(uint16_t* x, int64_t rows, int64_t K, int64_t ld, int M, cudaStream_t st) {
   const int64_t total = rows * (K / M / 2);
-  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(total, int64_t(256)), int64_t(num_sms()) * 8));
+  const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(ceil_div(total, int64_t(256)), int64_t(num_sms()) * 16));
   const dim3 grid(static_cast<unsigned>(blocks)), block(256);
   cudaError_t err;
   switch (M) {

@@ -791,34 +791,49 @@ k_lift(const T* __restrict__ src, int64_t rows, int64_t K, int64_t ld,
 // X.  Odd window o of a group covers its elements 4o + 2 .. 4o + 5, i.e. its
 // 32-bit words 2o + 1, 2o + 2, so a group's odd windows are its words 1 ..
 // 2(M/4 - 1): the group without its first and last two elements.  A thread
-// takes two groups of one row (K % 128 == 0 keeps the group count even):
-// 16-byte loads of both, 16-byte stores of their odd windows.
+// takes pairs of groups of one row (K % 128 == 0 keeps the group count even),
+// several pairs' 16-byte loads in flight before their 16-byte stores.
 template <int M>
 __global__ void __launch_bounds__(256) k_lift_odd(uint16_t* x, int64_t rows, int64_t K, int64_t ld) {
   static_assert(M % 8 == 0 && M >= 8, "two groups make whole 16-byte loads and stores");
   constexpr int NO = M / 4 - 1;                   // odd windows per group
+  constexpr int U = M == 8 ? 4 : (M == 16 ? 2 : 1);   // group pairs per thread and step, loads in flight together
   griddep_launch_dependents();
   griddep_wait();                                      // X may come from the preceding kernel
   const int64_t pairs = K / M / 2;                     // group pairs per row
   const int64_t total = rows * pairs;
-  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
-       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = idx / pairs, t = idx - r * pairs;
-    const uint4* src = reinterpret_cast<const uint4*>(x + r * ld + t * 2 * M);
-    uint32_t w[M];                                     // the two groups, M / 2 words each
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t base = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; base < total;
+       base += U * stride) {
+    uint32_t w[U][M];                                  // U pairs of groups, M / 2 words per group
 #pragma unroll
-    for (int i = 0; i < M / 4; ++i) {
-      const uint4 q = src[i];
-      w[4 * i] = q.x; w[4 * i + 1] = q.y; w[4 * i + 2] = q.z; w[4 * i + 3] = q.w;
+    for (int u = 0; u < U; ++u) {
+      const int64_t idx = base + u * stride;
+      if (idx < total) {
+        const int64_t r = idx / pairs, t = idx - r * pairs;
+        const uint4* src = reinterpret_cast<const uint4*>(x + r * ld + t * 2 * M);
+#pragma unroll
+        for (int i = 0; i < M / 4; ++i) {
+          const uint4 q = src[i];
+          w[u][4 * i] = q.x; w[u][4 * i + 1] = q.y; w[u][4 * i + 2] = q.z; w[u][4 * i + 3] = q.w;
+        }
+      }
     }
-    uint32_t o[4 * NO];
 #pragma unroll
-    for (int h = 0; h < 2; ++h)
+    for (int u = 0; u < U; ++u) {
+      const int64_t idx = base + u * stride;
+      if (idx < total) {
+        const int64_t r = idx / pairs, t = idx - r * pairs;
+        uint32_t o[4 * NO];
 #pragma unroll
-      for (int k = 0; k < 2 * NO; ++k) o[h * 2 * NO + k] = w[h * (M / 2) + 1 + k];
-    uint4* dst = reinterpret_cast<uint4*>(x + r * ld + K + t * 8 * NO);
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
-    for (int i = 0; i < NO; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+          for (int k = 0; k < 2 * NO; ++k) o[h * 2 * NO + k] = w[u][h * (M / 2) + 1 + k];
+        uint4* dst = reinterpret_cast<uint4*>(x + r * ld + K + t * 8 * NO);
+#pragma unroll
+        for (int i = 0; i < NO; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+      }
+    }
   }
 }
 
