@@ -51,7 +51,7 @@ TRAFFIC = {
     ("hybrid_decode_b8", "k_nm_gemm<16>"): 79020544 + 1609728,
     ("hybrid_decode_b128", "k_nm_gemm_2cta<128,2,1>"): 80018432 + 1831936,
     ("slide_6of8_wt_decode", "k_nm_gemm<16>"): 28556800 + 0,
-    ("slide_6of8_wt_prefill", "k_nm_gemm_2cta<224,2,1>"): 82914304 + 17293312,
+    ("slide_6of8_wt_prefill", "k_nm_gemm_2cta<224,2,1>"): 81972736 + 17421056,
 }
 OTHERS = ["up_proj_8of16_act", "up_proj_2of4_act", "up_proj_8of16_act_fp8", "up_proj_8of16_act_xf",
           "slide_6of8_wt_prefill", "slide_6of8_wt_prefill_fp8",
